@@ -1,0 +1,518 @@
+"""Benchmark of the KDA hot path on B200 through libkda's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libkda|reference]
+                    [--workload prefill|long|varlen|decode] [--no-cpu-baseline]
+
+A step is one pass of the path over one batch of synthetic inputs already
+resident in HBM: the gate (g = -5 sigmoid(e^A z)) then the chunkwise forward
+for the prefill workloads; gate + decode step for the decode workload.  The
+default workload is the dense prefill B=8, H=32, T=4096, dk=dv=128 (bf16
+q/k/v, fp32 g/beta/state); its line also carries the decode workload
+(256 sequences x 32 heads, 1024 consecutive steps) as a secondary figure.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and torch.cuda.synchronize(), with CUDA events on the launching stream; the
+per-kernel durations that feed the roofline come from events around each
+launch on the same stream.  Inputs are larger than L2 (126 MB), so no flush
+is needed.  Under torchrun every rank runs its own batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (the slow baseline), printing the same JSON keys.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gated_delta_rule_158_b200 as kda  # noqa: E402
+from gated_delta_rule_158_b200 import workloads as W  # noqa: E402
+
+METRIC = "KDA prefill Mtokens/s & decode steps/s on 1 B200; % of TC / HBM roofline"
+
+WORKLOADS = {
+    "prefill": dict(name="prefill B8 H32 T4096 d128", B=8, T=4096, H=32, dk=128, dv=128,
+                    seed=1, init=False, varlen=False),
+    "long": dict(name="long prefill B1 H32 T1048576 d128", B=1, T=1048576, H=32, dk=128,
+                 dv=128, seed=2, init=False, varlen=False),
+    "varlen": dict(name="varlen 64 seqs log-uniform[128,32768] H16 d128", B=1, T=None, H=16,
+                   dk=128, dv=128, seed=3, init=True, varlen=True, num_seqs=64),
+    "decode": dict(name="decode N256 H32 d128 x1024 steps", N=256, H=32, dk=128, dv=128,
+                   steps=1024, seed=4),
+}
+
+# bytes per (token, head) of the chunkwise forward, bf16 q/k/v/o, fp32 g/beta:
+# q, k, v 3*256 + g 512 + beta 4 + o 256
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 4 + 256
+# FLOPs per (token, head) of the chunk form (C = 32 on the tensor-core path)
+# counted once: C(3dk + 2dv) + C^2/3 + 6 dk dv
+def prefill_flops_per_token_head(C=32, dk=128, dv=128):
+    return C * (3 * dk + 2 * dv) + C * C / 3 + 6 * dk * dv
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], tc=d["bf16_tflops"], tc_sustained=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- prefill
+def make_prefill(wl, device):
+    if wl["varlen"]:
+        lens = W.varlen_lengths(wl["num_seqs"], wl["seed"])
+        cu_list = W.cu_seqlens_from_lengths(lens)
+        T = cu_list[-1]
+        inp = W.make_prefill_inputs(1, T, wl["H"], wl["dk"], wl["dv"], torch.bfloat16,
+                                    seed=wl["seed"], device=device, init_state=True,
+                                    num_states=wl["num_seqs"])
+        cu = torch.tensor(cu_list, dtype=torch.int32, device=device)
+        return inp, cu, T, wl["num_seqs"]
+    inp = W.make_prefill_inputs(wl["B"], wl["T"], wl["H"], wl["dk"], wl["dv"], torch.bfloat16,
+                                seed=wl["seed"], device=device, init_state=wl["init"])
+    return inp, None, wl["T"], wl["B"]
+
+
+class PrefillStep:
+    """gate + chunk_fwd on resident inputs, events around each launch."""
+
+    def __init__(self, inp, cu, N):
+        self.inp, self.cu = inp, cu
+        q = inp["q"]
+        B, T, H, dk = q.shape
+        dv = inp["v"].shape[-1]
+        self.g = torch.empty_like(inp["z"])
+        self.out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+        self.final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        nbytes = kda.kda_chunk_fwd_workspace_size(B, T, H, dk, dv,
+                                                  0 if cu is None else N, 0, kda.KDA_BF16)
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device)
+
+    def __call__(self, ev=None):
+        i = self.inp
+        if ev:
+            ev[0].record()
+        kda.kda_gate_fwd(i["z"], i["A_log"], self.g)
+        if ev:
+            ev[1].record()
+        kda.kda_chunk_fwd(i["q"], i["k"], i["v"], self.g, i["beta"], self.out, self.ws,
+                          init_state=i["init_state"], cu_seqlens=self.cu,
+                          final_state=self.final)
+        if ev:
+            ev[2].record()
+
+
+def time_steps(step, K, Wm, world):
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for k in range(K):
+        step(evs[k])
+    stop.record()
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(stop)
+    gate_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    chunk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    barrier(world)
+    return max_over_ranks(total_ms, world), gate_ms, chunk_ms
+
+
+def e2e_prefill(wl, inp, cu, N, K):
+    """Same step through the public API with host buffers: H2D of the step's
+    inputs from pinned memory, gate + chunk_fwd, D2H of o and final state."""
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    dev = {k: (torch.empty_like(v) if v is not None else None) for k, v in inp.items()}
+    step = PrefillStep(dev, cu, N)
+    out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    fin_h = torch.empty(step.final.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * 4
+
+    def one():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        step()
+        out_h.copy_(step.out, non_blocking=True)
+        fin_h.copy_(step.final, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / K, h2d, d2h
+
+
+# ----------------------------------------------------------------- decode
+def run_decode(wl, device, warmup=3):
+    N, H, dk, dv, steps = wl["N"], wl["H"], wl["dk"], wl["dv"], wl["steps"]
+    state = W.make_decode_state(N, H, dk, dv, wl["seed"], device)
+    A_log = W.make_decode_gate_params(H, wl["seed"] + 1000, device)
+    # all steps' inputs resident before timing (fresh inputs per step)
+    xs = [W.make_decode_step_inputs(N, H, dk, dv, torch.bfloat16, wl["seed"] + s, device)
+          for s in range(steps)]
+    g = torch.empty((N, H, dk), dtype=torch.float32, device=device)
+    o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=device)
+
+    def step(x, ev=None):
+        kda.kda_gate_fwd(x["z"], A_log, g)
+        if ev:
+            ev[0].record()
+        kda.kda_decode_step(x["q"], x["k"], x["v"], g, x["beta"], state, o)
+        if ev:
+            ev[1].record()
+
+    for s in range(warmup):
+        step(xs[s])
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(steps):
+        step(xs[s], evs[s])
+    b.record()
+    torch.cuda.synchronize()
+    total_ms = a.elapsed_time(b)
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    bytes_per_launch = N * H * (2 * dk * dv * 4 + (2 * dk + dv) * 2 + dk * 4 + 4 + dv * 2)
+    return total_ms, dec_ms, bytes_per_launch
+
+
+# ------------------------------------------------------- oracle baseline
+def oracle_prefill_parallel_sample(wl, inp, cu, budget_s=15.0):
+    """Same as above but runs the oracle's own thread pool over a batch of
+    units at once (what `cores` reports)."""
+    import numpy as np
+
+    import oracle
+    H = wl["H"]
+    nthreads = oracle.default_threads()
+    q = inp["q"]
+    if cu is None:
+        B, T = q.shape[0], q.shape[1]
+        n_b = 1
+        sl = (slice(0, n_b),)
+        per_unit = T
+        units_per_b = H
+        # one batch element at a time: H units of T tokens each
+        t_used, done = 0.0, 0
+        b = 0
+        while t_used < budget_s and b < B:
+            part = {k: inp[k][b:b + 1].detach().to("cpu", torch.float64).numpy()
+                    for k in ("q", "k", "v", "z", "beta")}
+            A_log = inp["A_log"].detach().cpu().double().numpy()
+            t0 = time.perf_counter()
+            g = oracle.gate(part["z"], A_log, -5.0)
+            oracle.forward(part["q"], part["k"], part["v"], g, part["beta"], nthreads=nthreads)
+            t_used += time.perf_counter() - t0
+            done += per_unit * units_per_b
+            b += 1
+            if t_used * (b + 1) / b > budget_s * 1.5:
+                break
+        sample = f"{b} of {B} batch rows ({b * H} (sequence, head) units x {T} tokens)"
+        return done / t_used / H, nthreads, sample, t_used
+    cu_l = cu.cpu().tolist()
+    Ns = len(cu_l) - 1
+    t_used, done, n = 0.0, 0, 0
+    A_log = inp["A_log"].detach().cpu().double().numpy()
+    while t_used < budget_s and n < Ns:
+        a, b = cu_l[n], cu_l[n + 1]
+        part = {k: inp[k][:, a:b].detach().to("cpu", torch.float64).numpy()
+                for k in ("q", "k", "v", "z", "beta")}
+        S0 = inp["init_state"][n:n + 1].detach().cpu().double().numpy()
+        t0 = time.perf_counter()
+        g = oracle.gate(part["z"], A_log, -5.0)
+        oracle.forward(part["q"], part["k"], part["v"], g, part["beta"], init_state=S0,
+                       nthreads=nthreads)
+        t_used += time.perf_counter() - t0
+        done += (b - a) * H
+        n += 1
+    sample = f"{n} of {Ns} sequences (all {H} heads each)"
+    return done / t_used / H, nthreads, sample, t_used
+
+
+def oracle_decode_sample(wl, budget_s=10.0):
+    import numpy as np
+
+    import oracle
+    N, H, dk, dv = wl["N"], wl["H"], wl["dk"], wl["dv"]
+    nthreads = oracle.default_threads()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    S = W.make_decode_state(N, H, dk, dv, wl["seed"], dev).cpu().double().numpy()
+    A_log = W.make_decode_gate_params(H, wl["seed"] + 1000, dev).cpu().double().numpy()
+    t_used, steps = 0.0, 0
+    while t_used < budget_s and steps < wl["steps"]:
+        x = W.make_decode_step_inputs(N, H, dk, dv, torch.bfloat16, wl["seed"] + steps, dev)
+        part = {k: x[k].detach().to("cpu", torch.float64).numpy()[:, None]
+                for k in ("q", "k", "v", "z", "beta")}
+        t0 = time.perf_counter()
+        g = oracle.gate(part["z"], A_log, -5.0)
+        _, S = oracle.forward(part["q"], part["k"], part["v"], g, part["beta"], init_state=S,
+                              nthreads=nthreads)
+        t_used += time.perf_counter() - t0
+        steps += 1
+    return steps / t_used, nthreads, f"{steps} of {wl['steps']} steps (all {N * H} heads)", t_used
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=list(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world, rank, local = dist_setup()
+    wl = WORKLOADS[args.workload]
+    peaks = load_peaks()
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    if args.workload == "decode":
+        line = bench_decode_line(args, wl, world, rank, peaks)
+    else:
+        line = bench_prefill_line(args, wl, world, rank, peaks)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def bench_prefill_line(args, wl, world, rank, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp, cu, T, N = make_prefill(wl, dev)
+    H, dk, dv = wl["H"], wl["dk"], wl["dv"]
+    B = inp["q"].shape[0]
+    tokens = B * T  # per rank
+    step = PrefillStep(inp, cu, N)
+    clocks = ClockSampler(dev.index)
+    total_ms, gate_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
+    clk = clocks.stop()
+    st, _ = kda.kda_get_device_status(step.ws)
+    if st != kda.KDA_OK:
+        raise RuntimeError(f"device status {kda.kda_status_string(st)}")
+    ms_per_step = total_ms / args.steps
+    value = tokens * world / (ms_per_step * 1e-3) / 1e6
+    tok_heads = tokens * H
+    alg_bytes = tok_heads * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * dk * dv * 4 * (
+        2 if inp["init_state"] is not None else 1)
+    achieved = alg_bytes / (chunk_ms * 1e-3) / 1e9
+    flops = tok_heads * prefill_flops_per_token_head(32, dk, dv)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "Mtokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T,
+                   "heads": H, "dk": dk, "dv": dv, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "step": "kda_gate_fwd + kda_chunk_fwd"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
+                     "traffic": None, "kernel": "kda_chunk_fwd",
+                     "kernel_ms": round(chunk_ms, 4), "algorithmic_bytes": alg_bytes,
+                     "peak_source": peaks["src"],
+                     "tensor_frac": round(flops / (chunk_ms * 1e-3) / (peaks["tc"] * 1e12), 4)},
+        "gate_ms": round(gate_ms, 4),
+        "gpu_launches": args.steps * 2,
+        "clocks": clk,
+    }
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_prefill(wl, inp, cu, N, max(2, min(args.steps, 5)))
+        line["e2e"] = {"value": round(tokens * world / (e2e_ms * 1e-3) / 1e6, 3),
+                       "unit": "Mtokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, secs = oracle_prefill_parallel_sample(wl, inp, cu, budget_s=15.0)
+        line["cpu_baseline"] = {"value": round(v / 1e6, 6), "unit": "Mtokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample + f", {secs:.1f} s"}
+    if not args.no_decode and args.workload == "prefill":
+        dwl = WORKLOADS["decode"]
+        del step, inp
+        torch.cuda.empty_cache()
+        total, dec_ms, bpl = run_decode(dwl, dev)
+        dach = bpl / (dec_ms * 1e-3) / 1e9
+        line["decode"] = {"workload": dwl["name"], "value": round(dwl["steps"] / (total * 1e-3), 2),
+                          "unit": "steps/s", "ms_per_step": round(total / dwl["steps"], 4),
+                          "roofline": {"bound": "hbm", "achieved": round(dach, 1),
+                                       "peak": peaks["hbm"], "unit": "GB/s",
+                                       "frac": round(dach / peaks["hbm"], 4),
+                                       "kernel": "kda_decode_step",
+                                       "kernel_ms": round(dec_ms, 4),
+                                       "algorithmic_bytes": bpl}}
+    return line
+
+
+def bench_decode_line(args, wl, world, rank, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    clocks = ClockSampler(dev.index)
+    barrier(world)
+    total, dec_ms, bpl = run_decode(wl, dev)
+    clk = clocks.stop()
+    total = max_over_ranks(total, world)
+    dach = bpl / (dec_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(wl["steps"] / (total * 1e-3) * world, 2),
+        "unit": "steps/s", "n_gpus": world, "steps": wl["steps"], "warmup": 3,
+        "ms_per_step": round(total / wl["steps"], 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["name"], "parallelism": f"dp{world} (independent batches)",
+                   "l2": "state (1 GiB) larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": round(dach, 1), "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": round(dach / peaks["hbm"], 4), "traffic": None,
+                     "kernel": "kda_decode_step", "kernel_ms": round(dec_ms, 4)},
+        "gpu_launches": wl["steps"] * 2, "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, secs = oracle_decode_sample(wl)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": "steps/s", "cores": cores,
+                                "kind": "oracle", "sample": sample + f", {secs:.1f} s"}
+    return line
+
+
+def run_reference(args, wl, world):
+    """The fp64 oracle as the reference arm, on this arm's config/metric."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if args.workload == "decode":
+        t_per = []
+        for _ in range(args.steps):
+            v, cores, sample, secs = oracle_decode_sample(wl, budget_s=5.0)
+            t_per.append(1.0 / v)
+        value = 1.0 / statistics.mean(t_per)
+        unit = "steps/s"
+        cfg = {"workload": wl["name"]}
+    else:
+        inp, cu, T, N = make_prefill(wl, dev)
+        vals = []
+        for _ in range(args.steps):
+            v, cores, sample, secs = oracle_prefill_parallel_sample(wl, inp, cu, budget_s=8.0)
+            vals.append(v / 1e6)
+        value = statistics.mean(vals)
+        unit = "Mtokens/s"
+        cfg = {"workload": wl["name"], "global_batch": inp["q"].shape[0], "seq_len": T}
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,151 @@
+"""ctypes binding of libkda's C ABI (include/kda.h): argument marshalling only.
+
+Every function below has the name of the C entry point it calls, takes torch
+tensors (device memory) and plain numbers, and passes their pointers, sizes
+and the current CUDA stream through unchanged.  No computation happens here;
+if libkda.so is missing or fails to load, every call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_MISALIGNED = 3
+KDA_ERR_WORKSPACE = 4
+KDA_ERR_CUDA = 5
+KDA_ERR_TIMEOUT = 6
+KDA_ERR_BAD_SEQLENS = 7
+
+KDA_F32 = 0
+KDA_BF16 = 1
+
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "kda_status_string": (ctypes.c_char_p, [_I]),
+    "kda_gate_fwd": (_I, [_VP, _VP, _F, _VP, _I64, _I, _I, _VP]),
+    "kda_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "kda_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
+                           _F, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "kda_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _I, _I, _I, _I, _F, _VP, _VP]),
+    "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
+    "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
+}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {kda_status_string(status)} ({status})")
+
+
+def lib():
+    """The loaded libkda.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libkda.so not found at {LIB_PATH}; build it with "
+                "`python -m gated_delta_rule_158_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("libkda takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype(t):
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported input dtype {t.dtype}")
+
+
+def _check(status, where):
+    if status != KDA_OK:
+        raise KdaError(status, where)
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def kda_gate_fwd(z, A_log, g, g_min=-5.0, stream=None):
+    """g = g_min * sigmoid(exp(A_log[h]) * z); z, g fp32 [..., H, dk]."""
+    H, dk = z.shape[-2], z.shape[-1]
+    rows = z.numel() // (H * dk) if z.numel() else 0
+    _check(lib().kda_gate_fwd(_ptr(z), _ptr(A_log), float(g_min), _ptr(g), rows, H, dk,
+                              _stream(stream)), "kda_gate_fwd")
+
+
+def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs=0, chunk_size=0,
+                                 in_dtype=KDA_BF16) -> int:
+    return int(lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size,
+                                                  in_dtype))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, out, workspace, init_state=None, cu_seqlens=None,
+                  final_state=None, scale=1.0, chunk_size=0, stream=None):
+    """Chunkwise forward; q, k, g [B,T,H,dk], v/out [B,T,H,dv], beta [B,T,H]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib().kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q), _ptr(init_state),
+        _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale), int(chunk_size), _ptr(out),
+        _ptr(final_state), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "kda_chunk_fwd")
+
+
+def kda_decode_step(q, k, v, g, beta, state, out, scale=1.0, stream=None):
+    """One decode step; q, k, g [N,H,dk], v/out [N,H,dv], beta [N,H], state in place."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q),
+                                 _ptr(state), N, H, dk, dv, float(scale), _ptr(out),
+                                 _stream(stream)), "kda_decode_step")
+
+
+def kda_get_device_status(workspace, stream=None):
+    """(status, detail) recorded on the device in this workspace; syncs the stream."""
+    detail = ctypes.c_int32(0)
+    st = lib().kda_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+def kda_selftest_bounded_wait(workspace, spin_limit_ns, stream=None):
+    _check(lib().kda_selftest_bounded_wait(_ptr(workspace), int(spin_limit_ns),
+                                           _stream(stream)), "kda_selftest_bounded_wait")

@@ -1,0 +1,248 @@
+// kda_api.cu -- the C ABI of libkda: host-side argument checks, workspace
+// layout, path selection and launches.  The contract of every entry point is
+// in include/kda.h.
+#include <math.h>
+#include <string.h>
+
+#include "kda_internal.cuh"
+#include "kda_sync.cuh"
+
+namespace kda {
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+namespace {
+
+// ---------------------------------------------------------------- varlen plan
+// Validates cu_seqlens on the device and orders sequences longest first, so
+// the longest (sequence, head) units start in the first wave.  One CTA; the
+// order is a rank count, O(N^2), done only for N <= kMaxSortSeqs (larger
+// batches keep their given order).
+constexpr int kMaxSortSeqs = 8192;
+
+__global__ void varlen_plan_kernel(const int32_t* __restrict__ cu, int N, int T,
+                                   int32_t* __restrict__ order, StatusBlock* sb) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
+  __syncthreads();
+  for (int n = threadIdx.x; n < N; n += blockDim.x)
+    if (cu[n + 1] < cu[n]) atomicOr(&bad, 1);
+  __syncthreads();
+  if (bad) {
+    if (threadIdx.x == 0) {
+      sb->seqlens_ok = 0;
+      record_status(sb, KDA_ERR_BAD_SEQLENS, 0);
+    }
+    return;
+  }
+  for (int n = threadIdx.x; n < N; n += blockDim.x) {
+    if (N > kMaxSortSeqs) {
+      order[n] = n;
+      continue;
+    }
+    const int Ln = cu[n + 1] - cu[n];
+    int rank = 0;
+    for (int m = 0; m < N; ++m) {
+      const int Lm = cu[m + 1] - cu[m];
+      rank += (Lm > Ln) || (Lm == Ln && m < n);
+    }
+    order[rank] = n;
+  }
+  if (threadIdx.x == 0) sb->seqlens_ok = 1;
+}
+
+// ------------------------------------------------------ bounded-wait selftest
+__global__ void selftest_wait_kernel(StatusBlock* sb, long long limit_ns) {
+  if (threadIdx.x != 0) return;
+  bounded_flag_wait(&sb->never_set, limit_ns, sb, (int32_t)blockIdx.x);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool use_tc_path(kda_dtype dt, int dk, int dv, int chunk) {
+  return dt == KDA_BF16 && dk == 128 && dv == 128 && (chunk == 0 || chunk == 32);
+}
+
+}  // namespace
+
+cudaError_t launch_varlen_plan(const int32_t* cu_seqlens, int num_seqs, int T, int32_t* order,
+                               StatusBlock* sb, cudaStream_t stream) {
+  varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, order, sb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(sb, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+kda_status kda_gate_fwd(const float* z, const float* A_log, float g_min, float* g, int64_t rows,
+                        int H, int dk, void* stream) {
+  if (!z || !A_log || !g) return KDA_ERR_INVALID_ARG;
+  if (rows < 0 || H <= 0 || dk <= 0 || dk % 4 != 0) return KDA_ERR_INVALID_ARG;
+  if (!(g_min < 0.f) || !isfinite(g_min)) return KDA_ERR_INVALID_ARG;
+  if (z == g) return KDA_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(g) || !aligned16(A_log)) return KDA_ERR_MISALIGNED;
+  if (rows == 0) return KDA_OK;
+  cudaError_t e = launch_gate(z, A_log, g_min, g, rows, H, dk, (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                    int chunk_size, kda_dtype in_dtype) {
+  size_t bytes = kStatusBytes;
+  if (num_seqs > 0) bytes += round_up(sizeof(int32_t) * (size_t)num_seqs, 256);
+  if (use_tc_path(in_dtype, dk, dv, chunk_size) && B > 0 && T > 0 && H > 0)
+    bytes += tc_workspace_bytes(B, T, H, num_seqs, device_sm_count());
+  return bytes;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, kda_dtype in_dtype, const float* init_state,
+                         const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                         int dv, float scale, int chunk_size, void* out, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !g || !beta || !out || !workspace) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (chunk_size != 0 && chunk_size != 16 && chunk_size != 32 && chunk_size != 64)
+    return KDA_ERR_UNSUPPORTED;
+  if (cu_seqlens) {
+    if (B != 1 || num_seqs <= 0) return KDA_ERR_INVALID_ARG;
+  } else if (num_seqs != 0 && num_seqs != B) {
+    return KDA_ERR_INVALID_ARG;
+  }
+  const void* ptrs[] = {q, k, v, g, beta, out, workspace, init_state, final_state, cu_seqlens};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* outs[] = {out};
+  const void* ins[] = {q, k, v, g, beta, init_state, cu_seqlens};
+  for (const void* o : outs)
+    for (const void* i : ins)
+      if (i && o == i) return KDA_ERR_INVALID_ARG;
+  const int nseq = cu_seqlens ? num_seqs : B;
+  const size_t need =
+      kda_chunk_fwd_workspace_size(B, T, H, dk, dv, cu_seqlens ? num_seqs : 0, chunk_size, in_dtype);
+  if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+  if ((int64_t)nseq * H > (int64_t)1 << 30) return KDA_ERR_UNSUPPORTED;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  StatusBlock* sb = static_cast<StatusBlock*>(workspace);
+  char* tail = static_cast<char*>(workspace) + kStatusBytes;
+  if (cudaMemsetAsync(sb, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+
+  ChunkArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.dt = in_dtype;
+  a.init_state = init_state;
+  a.final_state = final_state;
+  a.out = out;
+  a.map.cu_seqlens = cu_seqlens;
+  a.map.order = nullptr;
+  a.map.status = sb;
+  a.map.B = B;
+  a.map.T = T;
+  a.map.H = H;
+  a.num_units = nseq * H;
+  a.dk = dk;
+  a.dv = dv;
+  a.scale = scale;
+  a.chunk = chunk_size;
+  a.sb = sb;
+  if (cu_seqlens) {
+    int32_t* order = reinterpret_cast<int32_t*>(tail);
+    tail += round_up(sizeof(int32_t) * (size_t)num_seqs, 256);
+    if (launch_varlen_plan(cu_seqlens, num_seqs, T, order, sb, st) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    a.map.order = order;
+  }
+  cudaError_t e;
+  if (use_tc_path(in_dtype, dk, dv, chunk_size)) {
+    a.chunk = 32;
+    const size_t tail_bytes = workspace_bytes - (size_t)(tail - static_cast<char*>(workspace));
+    e = launch_chunk_tc(a, tail, tail_bytes, st);
+  } else {
+    if (a.chunk == 0) a.chunk = 32;
+    e = launch_chunk_simt(a, st);
+  }
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, kda_dtype in_dtype, float* state, int N, int H,
+                           int dk, int dv, float scale, void* out, void* stream) {
+  if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (N <= 0 || H <= 0 || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, g, beta, state, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {q, k, v, g, beta, state};
+  for (const void* i : ins)
+    if (i == out) return KDA_ERR_INVALID_ARG;
+  cudaError_t e =
+      launch_decode(q, k, v, g, beta, in_dtype, state, N, H, dk, dv, scale, out, (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_get_device_status(const void* workspace, void* stream, int32_t* detail) {
+  if (!workspace) return KDA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+  int32_t host[2] = {0, 0};
+  if (cudaMemcpy(host, workspace, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (detail) *detail = host[1];
+  return (kda_status)host[0];
+}
+
+kda_status kda_selftest_bounded_wait(void* workspace, int64_t spin_limit_ns, void* stream) {
+  if (!workspace) return KDA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return KDA_ERR_MISALIGNED;
+  long long lim = spin_limit_ns;
+  if (lim < 1000) lim = 1000;
+  if (lim > 5000000000LL) lim = 5000000000LL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+  cudaError_t e = launch_selftest_wait(static_cast<StatusBlock*>(workspace), lim, st);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// kda_internal.cuh -- shared declarations of libkda's kernels and launchers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// ---------------------------------------------------------------- workspace
+// The first 256 bytes of every workspace: the device status block.
+struct StatusBlock {
+  int32_t status;     // first kda_status recorded on the device (0 = OK)
+  int32_t detail;     // block index (or other code-specific value)
+  int32_t never_set;  // a flag nothing writes (bounded-wait self test)
+  int32_t seqlens_ok; // varlen plan verdict: 1 valid, 0 invalid
+  int32_t pad[60];
+};
+static_assert(sizeof(StatusBlock) == 256, "status block is 256 bytes");
+
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void record_status(StatusBlock* sb, int32_t code,
+                                              int32_t detail) {
+  if (sb == nullptr) return;
+  if (atomicCAS(&sb->status, 0, code) == 0) atomicExch(&sb->detail, detail);
+}
+
+// --------------------------------------------------------------- element io
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float load(const float* p) { return *p; }
+  static __device__ __forceinline__ void store(float* p, float x) { *p = x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float x) {
+    *p = __float2bfloat16_rn(x);
+  }
+};
+
+// ---------------------------------------------------------- unit addressing
+// A "unit" is one (sequence, head) pair processed start to end by one CTA.
+// Dense batches: sequence b spans rows [b*T, b*T + T) of the [B*T, H, *]
+// view.  Varlen: sequence n spans [cu[n], cu[n+1]).
+struct UnitMap {
+  const int32_t* cu_seqlens;  // nullptr = dense
+  const int32_t* order;       // varlen processing order (longest first) or nullptr
+  const StatusBlock* status;  // varlen validity verdict lives here
+  int B, T, H;
+};
+
+// Launchers (host side).  All return cudaSuccess or the launch error.
+cudaError_t launch_gate(const float* z, const float* A_log, float g_min,
+                        float* g, int64_t rows, int H, int dk,
+                        cudaStream_t stream);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v,
+                          const float* g, const float* beta, kda_dtype dt,
+                          float* state, int N, int H, int dk, int dv,
+                          float scale, void* out, cudaStream_t stream);
+
+cudaError_t launch_varlen_plan(const int32_t* cu_seqlens, int num_seqs, int T,
+                               int32_t* order, StatusBlock* sb,
+                               cudaStream_t stream);
+
+struct ChunkArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  kda_dtype dt;
+  const float* init_state;
+  float* final_state;
+  void* out;
+  UnitMap map;
+  int num_units;  // sequences * H
+  int dk, dv;
+  float scale;
+  int chunk;
+  StatusBlock* sb;
+};
+
+cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
+
+// tcgen05 tensor-core path (bf16, dk = dv = 128, chunk 32).
+size_t tc_workspace_bytes(int B, int T, int H, int num_seqs, int num_sms);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail,
+                            size_t ws_tail_bytes, cudaStream_t stream);
+
+cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns,
+                                 cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace kda

@@ -1,0 +1,93 @@
+// kda_sync.cuh -- bounded waits used by libkda's kernels.
+//
+// No kernel in libkda waits without a limit.  A wait polls its condition;
+// once it has polled kFastPolls times it starts reading the global
+// nanosecond timer and gives up after a time limit, recording
+// KDA_ERR_TIMEOUT in the workspace status word (read by
+// kda_get_device_status) instead of trapping, so the context stays usable.
+#pragma once
+
+#include <stdint.h>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+
+constexpr long long kWaitLimitNs = 2000000000LL;  // 2 s: far above any real wait
+constexpr int kFastPolls = 1 << 12;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits until *flag != 0.  Returns true on success, false on timeout (and
+// records the timeout with `detail`).
+__device__ __forceinline__ bool bounded_flag_wait(const volatile int32_t* flag,
+                                                  long long limit_ns, StatusBlock* sb,
+                                                  int32_t detail) {
+  for (int i = 0; i < kFastPolls; ++i)
+    if (*flag != 0) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (*flag != 0) return true;
+    if ((long long)(global_ns() - t0) > limit_ns) {
+      record_status(sb, KDA_ERR_TIMEOUT, detail);
+      return false;
+    }
+    __nanosleep(256);
+  }
+}
+
+// mbarrier helpers (shared::cta addresses as 32-bit integers)
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  On timeout sets
+// *abort (shared), records the status and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, StatusBlock* sb,
+                                                  int32_t detail) {
+  for (int i = 0; i < kFastPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if ((long long)(global_ns() - t0) > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_status(sb, KDA_ERR_TIMEOUT, detail);
+      return false;
+    }
+  }
+}
+
+}  // namespace kda

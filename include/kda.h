@@ -1,0 +1,168 @@
+/*
+ * kda.h -- C ABI of libkda, a CUDA (sm_100a / B200) implementation of the
+ * Kimi Delta Attention (KDA) recurrence.
+ *
+ * The operation (web page "NLP--技术报告解读-Kimi-K3", joezjh.github.io,
+ * section Model Architecture > Kimi Delta Attention (KDA)):
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *   o_t = scale * S_t^T q_t,          S_t in R^{dk x dv},  alpha_t = exp(g_t),
+ *
+ * with the lower-bounded log-decay gate of the same section
+ *   g_t^h = g_min * Sigmoid(exp(A_h) z_t^h),  g_min = -5,  so alpha > e^-5.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller; libkda
+ *    never allocates, frees or keeps device memory.  Scratch space comes from
+ *    a caller-provided workspace whose size a *_workspace_size query returns.
+ *  - Layouts are dense row-major ("C order"), innermost dimension last, with
+ *    no padding: q, k, g [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+ *    o [B, T, H, dv]; states [N, H, dk, dv] (row index = key channel).
+ *    Varlen batches pack N sequences along T with B == 1.
+ *  - q, k, v and o share one element type (kda_dtype); g, beta, z, A_log and
+ *    all states are fp32.  Arithmetic is fp32 (fp32 accumulation; bf16 or
+ *    tf32 tensor-core operands on the bf16 path).  o is rounded to nearest
+ *    even when it is bf16.
+ *  - Every pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls are asynchronous: they return after enqueueing work.
+ *  - Argument errors are detected on the host BEFORE anything is enqueued;
+ *    the call then returns the error and touches no buffer.  A failed launch
+ *    returns KDA_ERR_CUDA.  Problems found on the device (a bounded wait that
+ *    ran out, malformed cu_seqlens) are never trapped: they are written to a
+ *    status word in the workspace, read back with kda_get_device_status().
+ */
+#ifndef LIBKDA_KDA_H_
+#define LIBKDA_KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kda_status {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad scale */
+  KDA_ERR_UNSUPPORTED = 2,  /* dk/dv/chunk/dtype combination not built */
+  KDA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+  KDA_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+  KDA_ERR_CUDA = 5,         /* a CUDA launch or runtime call failed */
+  KDA_ERR_TIMEOUT = 6,      /* device: a bounded wait gave up */
+  KDA_ERR_BAD_SEQLENS = 7   /* device: cu_seqlens not monotone / not ending at T */
+} kda_status;
+
+typedef enum kda_dtype { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KDA_API const char *kda_status_string(kda_status s);
+
+/*
+ * Gate (same page, Model Architecture > KDA > Lower-bounded decay):
+ *   g[r, h, i] = g_min * Sigmoid(exp(A_log[h]) * z[r, h, i])
+ * z, g : fp32 [rows, H, dk] (rows = B*T);  A_log : fp32 [H].
+ * g may not alias z.  g_min must be finite and negative (KDA uses -5).
+ */
+KDA_API kda_status kda_gate_fwd(const float *z, const float *A_log, float g_min,
+                        float *g, int64_t rows, int H, int dk, void *stream);
+
+/*
+ * Bytes of workspace kda_chunk_fwd needs for these arguments (always > 0:
+ * it holds at least the device status word).  num_seqs is the number of
+ * varlen sequences, or 0 for a dense batch.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
+                                    int num_seqs, int chunk_size,
+                                    kda_dtype in_dtype);
+
+/*
+ * Chunkwise prefill / training forward of the recurrence above.
+ *
+ * Within chunks of chunk_size tokens the recurrence is evaluated in its
+ * WY/UT form as dense contractions; the state is carried across chunks
+ * (FlashKDA: same page, Infrastructure > KDA kernels, "training and
+ * prefill"), and a long sequence with too few (sequence, head) pairs to
+ * fill the GPU is split into segments whose transitions are computed
+ * independently and combined exactly (same bullet list, "intra-device CP";
+ * Infrastructure > KDA Context Parallelism, S = S~ + M S_prev).
+ *
+ *  q, k, v      : in_dtype, [B, T, H, dk|dv]
+ *  g            : fp32 [B, T, H, dk]  log-decay (typically kda_gate_fwd's output)
+ *  beta         : fp32 [B, T, H]
+ *  init_state   : fp32 [N, H, dk, dv] or NULL for zeros (N = num_seqs if
+ *                 cu_seqlens is given, else B).  May equal final_state.
+ *  cu_seqlens   : NULL for a dense batch, or device int32 [num_seqs + 1],
+ *                 non-decreasing from 0 to T, with B == 1.  Zero-length
+ *                 sequences are allowed (final = init, no output rows).
+ *                 Malformed offsets are reported on the device
+ *                 (KDA_ERR_BAD_SEQLENS) and no unit runs.
+ *  scale        : finite factor on o (1.0 for o = S^T q).
+ *  chunk_size   : 0 = library choice, or 16, 32, 64.  The result does not
+ *                 depend on it beyond rounding.  bf16 with dk = dv = 128 and
+ *                 chunk 0 or 32 runs the tcgen05 tensor-core kernel; every
+ *                 other supported combination runs an fp32 CUDA-core kernel.
+ *  out          : in_dtype [B, T, H, dv]; must not alias any input.
+ *  final_state  : fp32 [N, H, dk, dv] or NULL.
+ *  workspace    : device buffer of >= kda_chunk_fwd_workspace_size() bytes;
+ *                 its first 256 bytes hold the device status word, cleared
+ *                 by this call.
+ * Supported: dk, dv in {32, 64, 128}; in_dtype KDA_F32 or KDA_BF16.
+ */
+KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, kda_dtype in_dtype,
+                         const float *init_state, const int32_t *cu_seqlens,
+                         int num_seqs, int B, int T, int H, int dk, int dv,
+                         float scale, int chunk_size, void *out,
+                         float *final_state, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * One single-token decode step for N sequences, updating the state in place
+ * (KDA decoding: same page, Online serving > high-performance kernels; the
+ * state is rewritten in place every token).  Per (n, h):
+ *   S' = Diag(exp(g)) S;  e = beta (v - S'^T k);  S = S' + k e^T;
+ *   o  = scale * S^T q.
+ *  q, k : in_dtype [N, H, dk];  v, out : in_dtype [N, H, dv]
+ *  g    : fp32 [N, H, dk];      beta : fp32 [N, H]
+ *  state: fp32 [N, H, dk, dv], read and written once.
+ * Supported: dk, dv in {32, 64, 128}.  No workspace is needed.
+ */
+KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const float *g, const float *beta,
+                           kda_dtype in_dtype, float *state, int N, int H,
+                           int dk, int dv, float scale, void *out,
+                           void *stream);
+
+/*
+ * Synchronises `stream`, then returns the device status word that kernels
+ * of an earlier kda_chunk_fwd call on this workspace recorded (KDA_OK if
+ * none).  If detail is not NULL it receives a code-specific value (the
+ * block that recorded the error).  Returns KDA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+KDA_API kda_status kda_get_device_status(const void *workspace, void *stream,
+                                 int32_t *detail);
+
+/*
+ * Diagnostic for the device-side failure path: launches one block that
+ * waits on a flag in the workspace that nothing sets, giving up after
+ * `spin_limit_ns` nanoseconds (clamped to [1e3, 5e9]), and records
+ * KDA_ERR_TIMEOUT in the status word exactly as the chunk kernels do when
+ * one of their waits runs out.  Needs 256 bytes of workspace.
+ */
+KDA_API kda_status kda_selftest_bounded_wait(void *workspace, int64_t spin_limit_ns,
+                                     void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBKDA_KDA_H_ */

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+libkda.so must load, export every entry point include/kda.h declares, and
+reject bad arguments on the host before touching the device: the pointers
+passed here are fake, so a call that got past validation would fail loudly.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_158_b200 as kda
+from gated_delta_rule_158_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_158_b200 import build
+    build.build()
+    return _lib.lib()
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"KDA_API[^;(]*?\b(kda_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol(L):
+    declared = _declared_symbols()
+    assert {"kda_chunk_fwd", "kda_decode_step", "kda_gate_fwd"} <= declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(_lib._SIGNATURES) == declared
+
+
+def test_status_strings(L):
+    for code, name in [(0, "KDA_OK"), (1, "KDA_ERR_INVALID_ARG"), (2, "KDA_ERR_UNSUPPORTED"),
+                       (3, "KDA_ERR_MISALIGNED"), (4, "KDA_ERR_WORKSPACE"), (5, "KDA_ERR_CUDA"),
+                       (6, "KDA_ERR_TIMEOUT"), (7, "KDA_ERR_BAD_SEQLENS")]:
+        assert kda.kda_status_string(code) == name
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+
+
+def _chunk(L, **over):
+    a = dict(q=FAKE, k=FAKE + 0x1000, v=FAKE + 0x2000, g=FAKE + 0x3000, beta=FAKE + 0x4000,
+             dt=_lib.KDA_BF16, init=None, cu=None, nseq=0, B=2, T=64, H=4, dk=128, dv=128,
+             scale=1.0, chunk=0, out=FAKE + 0x5000, final=None, ws=FAKE + 0x6000,
+             ws_bytes=1 << 40, stream=None)
+    a.update(over)
+    return L.kda_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["dt"], a["init"],
+                           a["cu"], a["nseq"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                           a["scale"], a["chunk"], a["out"], a["final"], a["ws"], a["ws_bytes"],
+                           a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), _lib.KDA_ERR_INVALID_ARG),
+    (dict(out=None), _lib.KDA_ERR_INVALID_ARG),
+    (dict(ws=None), _lib.KDA_ERR_INVALID_ARG),
+    (dict(B=0), _lib.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), _lib.KDA_ERR_INVALID_ARG),
+    (dict(dt=7), _lib.KDA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(dv=256), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=48), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(q=FAKE + 8), _lib.KDA_ERR_MISALIGNED),
+    (dict(final=FAKE + 0x7004), _lib.KDA_ERR_MISALIGNED),
+    (dict(out=FAKE), _lib.KDA_ERR_INVALID_ARG),           # out aliases q
+    (dict(cu=FAKE + 0x8000, nseq=3), _lib.KDA_ERR_INVALID_ARG),  # varlen needs B == 1
+    (dict(cu=FAKE + 0x8000, nseq=0, B=1), _lib.KDA_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), _lib.KDA_ERR_WORKSPACE),
+])
+def test_chunk_fwd_rejects_on_host(L, over, code):
+    assert _chunk(L, **over) == code
+
+
+def test_workspace_size_positive(L):
+    n = kda.kda_chunk_fwd_workspace_size(8, 4096, 32, 128, 128, 0, 0, _lib.KDA_BF16)
+    assert n >= 256
+    n2 = kda.kda_chunk_fwd_workspace_size(1, 1000, 16, 128, 128, 64, 0, _lib.KDA_BF16)
+    assert n2 >= 256 + 64 * 4
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, FAKE, FAKE, FAKE, FAKE, 1, FAKE, 4, 2, 128, 128, 1.0, FAKE + 64, None), 1),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE, 4, 2, 100, 128, 1.0, FAKE + 64, None), 2),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE + 4, 4, 2, 128, 128, 1.0, FAKE + 64, None), 3),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE, 0, 2, 128, 128, 1.0, FAKE + 64, None), 1),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE + 64, 4, 2, 128, 128, 1.0, FAKE + 64, None), 1),
+])
+def test_decode_rejects_on_host(L, args, code):
+    assert L.kda_decode_step(*args) == code
+
+
+def test_gate_rejects_on_host(L):
+    assert L.kda_gate_fwd(None, FAKE, -5.0, FAKE + 64, 10, 2, 32, None) == 1
+    assert L.kda_gate_fwd(FAKE, FAKE + 16, 5.0, FAKE + 64, 10, 2, 32, None) == 1
+    assert L.kda_gate_fwd(FAKE, FAKE + 16, -5.0, FAKE, 10, 2, 32, None) == 1
+    assert L.kda_gate_fwd(FAKE + 4, FAKE + 16, -5.0, FAKE + 64, 10, 2, 32, None) == 3
+    assert L.kda_gate_fwd(FAKE, FAKE + 16, -5.0, FAKE + 64, 0, 2, 32, None) == 0  # no-op
+
+
+def test_device_status_rejects_null(L):
+    assert L.kda_get_device_status(None, None, None) == 1
+    assert L.kda_selftest_bounded_wait(None, 1000, None) == 1
+    assert L.kda_selftest_bounded_wait(FAKE + 4, 1000, None) == 3

@@ -1,0 +1,189 @@
+"""GPU parity: libkda (through its C ABI) against the fp64 oracle.
+
+Small cases compare every element; they span several chunks and a ragged
+tail.  Tolerances (relative L2, written in kda_testutil): 1e-5 for fp32
+inputs; 2e-2 on outputs and 1e-2 on final states for bf16 inputs with fp32
+state.  Every output buffer is filled with NaN first, so an element the
+kernels fail to write fails the comparison.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_158_b200 as kda
+from gated_delta_rule_158_b200 import workloads as W
+
+from kda_testutil import (TOL_BF16_O, TOL_BF16_S, TOL_F32, TOL_GATE, gpu_gate, gpu_prefill,
+                          oracle_prefill, rel_l2, to64, unit_slices)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+# ------------------------------------------------------------------- gate
+
+def test_gate_parity(oracle_mod):
+    inp = W.make_prefill_inputs(2, 77, 5, 64, 64, torch.float32, seed=11, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    ref = oracle_mod.gate(to64(inp["z"]), to64(inp["A_log"]), -5.0)
+    got = to64(g)
+    rel = np.max(np.abs(got - ref) / np.abs(ref))
+    assert rel <= TOL_GATE, rel
+    assert (got >= -5.0).all() and (got < 0).all()
+
+
+# ----------------------------------------------------------------- decode
+
+def _decode_run(oracle_mod, N, H, dk, dv, dtype, steps, seed0):
+    S0 = W.make_decode_state(N, H, dk, dv, seed0, DEV)
+    A_log = W.make_decode_gate_params(H, seed0 + 1000, DEV)
+    state = S0.clone()
+    outs, steps_in = [], []
+    for s in range(steps):
+        x = W.make_decode_step_inputs(N, H, dk, dv, dtype, seed0 + s, DEV)
+        g = gpu_gate(x["z"], A_log)
+        o = torch.full((N, H, dv), float("nan"), device=DEV, dtype=dtype)
+        kda.kda_decode_step(x["q"], x["k"], x["v"], g, x["beta"], state, o)
+        outs.append(o)
+        steps_in.append(x)
+    torch.cuda.synchronize()
+    # oracle: the decode steps form a length-`steps` sequence per (n, h)
+    st = lambda name: torch.stack([x[name] for x in steps_in], dim=1)  # [N, steps, H, ...]
+    g_ref = oracle_mod.gate(to64(st("z")), to64(A_log), -5.0)
+    o_ref, S_ref = oracle_mod.forward(to64(st("q")), to64(st("k")), to64(st("v")), g_ref,
+                                      to64(st("beta")), init_state=to64(S0))
+    o_gpu = to64(torch.stack(outs, dim=1))
+    return o_gpu, to64(state), o_ref, S_ref
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 128), (128, 64), (128, 128), (32, 128)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_parity(oracle_mod, dk, dv, dtype):
+    o, S, o_ref, S_ref = _decode_run(oracle_mod, 3, 5, dk, dv, dtype, steps=6, seed0=40)
+    tol_o, tol_s = (TOL_F32, TOL_F32) if dtype == torch.float32 else (TOL_BF16_O, TOL_BF16_S)
+    assert rel_l2(o, o_ref) <= tol_o
+    assert rel_l2(S, S_ref) <= tol_s
+
+
+# --------------------------------------------------------------- prefill
+
+def test_prefill_tiny_fp32_config(oracle_mod):
+    """B=1, H=2, T=64, dk=dv=32, chunk 16, fp32 throughout, seed 0, zero state."""
+    inp = W.make_prefill_inputs(1, 64, 2, 32, 32, torch.float32, seed=0, device=DEV)
+    o, S, _, _ = gpu_prefill(inp, chunk=16, with_init=False)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, with_init=False)
+    assert rel_l2(to64(o), o_ref) <= TOL_F32
+    assert rel_l2(to64(S), S_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("dk,dv", [(32, 64), (64, 32), (128, 128)])
+def test_prefill_fp32_shapes(oracle_mod, chunk, dk, dv):
+    inp = W.make_prefill_inputs(2, 150, 3, dk, dv, torch.float32, seed=5, device=DEV,
+                                init_state=True)
+    o, S, _, _ = gpu_prefill(inp, chunk=chunk, scale=0.75)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, scale=0.75)
+    assert rel_l2(to64(o), o_ref) <= TOL_F32
+    assert rel_l2(to64(S), S_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("chunk", [0, 16, 64])
+@pytest.mark.parametrize("T", [1, 31, 300])
+def test_prefill_bf16_dense(oracle_mod, chunk, T):
+    """bf16 dk = dv = 128: chunk 0 is the tensor-core path; 16/64 the fp32 one."""
+    inp = W.make_prefill_inputs(2, T, 3, 128, 128, torch.bfloat16, seed=6 + T, device=DEV,
+                                init_state=True)
+    o, S, _, _ = gpu_prefill(inp, chunk=chunk)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+
+
+@pytest.mark.parametrize("chunk", [0, 32])
+def test_prefill_bf16_varlen(oracle_mod, chunk):
+    lens = [1, 33, 0, 100, 64, 5, 257]
+    cu_list = W.cu_seqlens_from_lengths(lens)
+    T = cu_list[-1]
+    inp = W.make_prefill_inputs(1, T, 2, 128, 128, torch.bfloat16, seed=21, device=DEV,
+                                init_state=True, num_states=len(lens))
+    cu = torch.tensor(cu_list, dtype=torch.int32, device=DEV)
+    o, S, _, ws = gpu_prefill(inp, cu=cu, chunk=chunk)
+    assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, cu=cu)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+    # zero-length sequence: final state equals its initial state
+    assert torch.equal(S[2], inp["init_state"][2])
+
+
+def test_chunk_size_invariance():
+    inp = W.make_prefill_inputs(1, 200, 2, 64, 64, torch.float32, seed=3, device=DEV,
+                                init_state=True)
+    res = [gpu_prefill(inp, chunk=c)[:2] for c in (16, 32, 64)]
+    for o, S in res[1:]:
+        assert rel_l2(to64(o), to64(res[0][0])) <= 1e-5
+        assert rel_l2(to64(S), to64(res[0][1])) <= 1e-5
+
+
+def test_state_handoff_equals_full_run():
+    """Running T1 then T2 with final_state -> init_state equals one run over T."""
+    inp = W.make_prefill_inputs(1, 160, 2, 128, 128, torch.bfloat16, seed=9, device=DEV,
+                                init_state=True)
+    o_full, S_full, _, _ = gpu_prefill(inp)
+    for t1 in (64, 77):
+        a = {k: (v[:, :t1].contiguous() if k in ("q", "k", "v", "z", "beta") else v)
+             for k, v in inp.items()}
+        b = {k: (v[:, t1:].contiguous() if k in ("q", "k", "v", "z", "beta") else v)
+             for k, v in inp.items()}
+        o1, S1, _, _ = gpu_prefill(a)
+        b["init_state"] = S1
+        o2, S2, _, _ = gpu_prefill(b)
+        assert rel_l2(to64(torch.cat([o1, o2], 1)), to64(o_full)) <= 1e-2
+        assert rel_l2(to64(S2), to64(S_full)) <= 1e-2
+
+
+def test_guard_bands_untouched():
+    """Outputs are written only inside their extents (canary slack around them)."""
+    B, T, H, d = 1, 70, 2, 128
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=4, device=DEV,
+                                init_state=True)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    pad = 4096
+    o_buf = torch.full((pad + B * T * H * d + pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+    s_buf = torch.full((pad + B * H * d * d + pad,), 7.0, dtype=torch.float32, device=DEV)
+    out = o_buf[pad:pad + B * T * H * d].view(B, T, H, d)
+    fin = s_buf[pad:pad + B * H * d * d].view(B, H, d, d)
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(B, T, H, d, d), dtype=torch.uint8,
+                     device=DEV)
+    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], out, ws,
+                      init_state=inp["init_state"], final_state=fin)
+    torch.cuda.synchronize()
+    for buf in (o_buf, s_buf):
+        assert (buf[:pad] == 7.0).all() and (buf[-pad:] == 7.0).all()
+    assert torch.isfinite(out).all() and torch.isfinite(fin).all()
+
+
+def test_bad_seqlens_reported_on_device():
+    T, H, d = 96, 2, 128
+    inp = W.make_prefill_inputs(1, T, H, d, d, torch.bfloat16, seed=8, device=DEV)
+    cu = torch.tensor([0, 50, 40, 96], dtype=torch.int32, device=DEV)  # not monotone
+    out, _, _, ws = gpu_prefill(inp, cu=cu, with_init=False)
+    st, _ = kda.kda_get_device_status(ws)
+    assert st == kda.KDA_ERR_BAD_SEQLENS
+    assert torch.isnan(out.float()).all()  # no unit ran
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    kda.kda_selftest_bounded_wait(ws, 2_000_000)  # 2 ms on a flag nothing sets
+    st, _ = kda.kda_get_device_status(ws)
+    assert st == kda.KDA_ERR_TIMEOUT
+    x = torch.ones(4, device=DEV)
+    assert float((x * 2).sum()) == 8.0  # the context is still usable
