@@ -1,15 +1,691 @@
-// kda_chunk_tc.cu -- placeholder until the tcgen05 kernel lands: routes the
-// tensor-core configuration to the CUDA-core kernel.
+// kda_chunk_tc.cu -- chunkwise KDA forward on the sm_100a tensor cores
+// (tcgen05 + TMEM + TMA), bf16 q/k/v, fp32 g/beta/state, dk = dv = 128.
+//
+// What it computes: the KDA recurrence of "NLP--技术报告解读-Kimi-K3"
+// (joezjh.github.io), Model Architecture > Kimi Delta Attention (KDA),
+//   S_t = (I - b_t k_t k_t^T) Diag(e^{g_t}) S_{t-1} + b_t k_t v_t^T,  o_t = S_t^T q_t,
+// evaluated chunk by chunk (FlashKDA: Infrastructure > KDA kernels, "training
+// and prefill") in the WY/UT form.  For a chunk of C = 32 tokens starting
+// from state S, with Gamma_r the in-chunk cumulative sum of g:
+//   L[r,s] = sum_i k_ri k_si e^{Gamma_ri - Gamma_si}          (Gram, s <= r)
+//   T      = (I + Diag(b) strict_lower(L))^-1 Diag(b)
+//   W      = T (k e^Gamma),   U = T V - W S,
+//   O      = (q e^Gamma) S + lower(Lq) U,
+//   S     <- Diag(e^{Gamma_C}) S + (k e^{Gamma_C - Gamma})^T U.
+//
+// Why C = 32 and one rebasing point.  The lower bound g >= -5 of the gate
+// (same section, Lower-bounded decay) is what lets every Gram tile,
+// diagonal included, be a plain tensor-core GEMM: with the rebasing point at
+// row 15, the left factors x_r e^{Gamma_r - Gamma_15} and the right factor
+// k_s e^{Gamma_15 - Gamma_s} both stay inside [e^-80, e^80] (16 steps of at
+// most -5 on either side), far from fp32's e^88.7 limit; a longer chunk
+// would need more than one rebasing point per tile.
+//
+// B200 mapping.  One CTA (256 threads) owns one (sequence, head) for its
+// whole length; two CTAs share an SM (112 KB shared memory, 256 TMEM columns
+// each).  The fp32 state never leaves the SM: it lives in TMEM as S^T (lane =
+// value channel, column = key channel) and is read directly as the tf32 A
+// operand of the state-side GEMMs (U -= S^T W^T, O = S^T Q^T, S^T += U^T Kc),
+// with U^T also consumed straight from TMEM.  The key-side GEMMs (Gram,
+// W = T Ka, U~ = T V) are bf16.  TMA brings q/k/g (and separately v) for the
+// next chunk while the current one computes.  All MMAs are issued by one
+// thread and tracked by mbarriers; every wait is bounded (kda_sync.cuh).
+//
+// TMEM columns: S^T [0,128) | U^T [128,160) | W^T [160,192) | O^T [192,224)
+//               | Gram (M = 64 layout, lanes 0-15 of each quarter) [224,256)
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kda_internal.cuh"
+#include "kda_sync.cuh"
+#include "kda_tc_ptx.cuh"
 
 namespace kda {
+namespace {
 
-size_t tc_workspace_bytes(int, int, int, int, int) { return 0; }
+using namespace tc;
 
-cudaError_t launch_chunk_tc(const ChunkArgs& a, void*, size_t, cudaStream_t stream) {
-  ChunkArgs b = a;
-  b.chunk = 32;
-  return launch_chunk_simt(b, stream);
+constexpr int C = 32;     // tokens per chunk
+constexpr int D = 128;    // dk = dv
+constexpr int NT = 256;   // threads per CTA
+
+constexpr uint32_t S_COL = 0, U_COL = 128, W_COL = 160, O_COL = 192, G_COL = 224;
+constexpr uint32_t TMEM_COLS = 256;
+
+// shared memory map (byte offsets from a 1024-aligned base)
+constexpr uint32_t SM_Q = 0;         // q tile  bf16 [32][128] row-major (TMA, no swizzle)
+constexpr uint32_t SM_K = 8192;      // k tile  bf16 [32][128]
+constexpr uint32_t SM_V = 16384;     // v tile  bf16, 2 x [32 rows x 128 B] swizzled (TMA)
+constexpr uint32_t SM_G = 24576;     // g tile  fp32 [32][128]
+constexpr uint32_t SM_R1 = 40960;    // 24 KB, two lives:
+constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128 (Gram A)
+constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
+constexpr uint32_t SM_WF = SM_R1;             //  W                fp32 32 x 128 (tf32 B)
+constexpr uint32_t SM_AKK = SM_R1 + 16384;    //  A_kk fp32 32 x 32 (row-xor swizzled)
+constexpr uint32_t SM_AQK = SM_R1 + 20480;    //  A_qk fp32 32 x 32 (tf32 B)
+constexpr uint32_t SM_KA = 65536;    // k e^G        bf16 [s][i] (MN-major A of W)
+constexpr uint32_t SM_TT = 73728;    // T            bf16 [r][s] (B of W and U~); cumsum partials during prep
+constexpr uint32_t SM_QG = 77824;    // q e^G        fp32 [r][i] (tf32 B of O)
+constexpr uint32_t SM_KC = 94208;    // k e^{GC-G}   fp32 [s][i] (MN-major tf32 B of S)
+constexpr uint32_t SM_MISC = 110592;
+constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
+constexpr uint32_t SM_BETA = SM_MISC + 512;    // beta         fp32 [32]
+constexpr uint32_t SM_BAR = SM_MISC + 640;     // 3 mbarriers
+constexpr uint32_t SM_TMEM = SM_MISC + 672;    // TMEM base address
+constexpr uint32_t SM_ABORT = SM_MISC + 676;   // abort flag
+constexpr uint32_t SMEM_BYTES = SM_MISC + 1024;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024 + 2048;  // align the base; slack
+
+constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
+constexpr uint32_t TX_V = 8192;
+
+struct TcParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_g;
+  const float* beta;
+  __nv_bfloat16* out;
+  const float* init_state;
+  float* final_state;
+  const int32_t* cu_seqlens;
+  const int32_t* order;
+  StatusBlock* sb;
+  float* seg_ws;  // segment states (split modes)
+  int B, T, H;
+  int mode;       // 0 whole units, 1 segment transitions, 2 segment outputs
+  int G;          // segments per unit (modes 1, 2)
+  int seg_len;    // tokens per segment (multiple of C)
+  float scale;
+};
+
+struct Unit {
+  int64_t row0, len;
+  int h;
+  const float* init;
+  bool init_identity, vzero, out_on;
+  float* final_state;
+};
+
+__device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
+  const int H = P.H;
+  const size_t DD = (size_t)D * D;
+  u.init_identity = false;
+  u.vzero = false;
+  u.out_on = true;
+  if (P.mode == 0) {
+    const int idx = blockIdx.x;
+    int64_t sidx;
+    u.h = idx % H;
+    if (P.cu_seqlens == nullptr) {
+      const int b = idx / H;
+      u.row0 = (int64_t)b * P.T;
+      u.len = P.T;
+      sidx = idx;
+    } else {
+      if (P.sb->seqlens_ok != 1) return false;
+      const int n = P.order ? P.order[idx / H] : idx / H;
+      u.row0 = P.cu_seqlens[n];
+      u.len = (int64_t)P.cu_seqlens[n + 1] - u.row0;
+      sidx = (int64_t)n * H + u.h;
+    }
+    u.init = P.init_state ? P.init_state + sidx * DD : nullptr;
+    u.final_state = P.final_state ? P.final_state + sidx * DD : nullptr;
+    return true;
+  }
+  const int U = P.B * H;
+  if (P.mode == 1) {  // pairs (S~ from zero with v, M from I with v = 0)
+    const int pair = blockIdx.x >> 1, kind = blockIdx.x & 1;
+    const int un = pair / (P.G - 1), g = pair % (P.G - 1);
+    u.h = un % H;
+    u.row0 = (int64_t)(un / H) * P.T + (int64_t)g * P.seg_len;
+    u.len = P.seg_len;
+    u.init = nullptr;
+    u.init_identity = kind == 1;
+    u.vzero = kind == 1;
+    u.out_on = false;
+    u.final_state = P.seg_ws + ((size_t)(un * (P.G - 1) + g) * 2 + kind) * DD;
+    return true;
+  }
+  // mode 2: outputs of every segment from its true incoming state
+  const int un = blockIdx.x / P.G, g = blockIdx.x % P.G;
+  u.h = un % H;
+  u.row0 = (int64_t)(un / H) * P.T + (int64_t)g * P.seg_len;
+  const int64_t rem = (int64_t)P.T - (int64_t)g * P.seg_len;
+  u.len = rem < P.seg_len ? rem : P.seg_len;
+  if (g == 0)
+    u.init = P.init_state ? P.init_state + (size_t)un * DD : nullptr;
+  else
+    u.init = P.seg_ws + ((size_t)U * (P.G - 1) * 2 + (size_t)un * (P.G - 1) + (g - 1)) * DD;
+  u.final_state = (g == P.G - 1 && P.final_state) ? P.final_state + (size_t)un * DD : nullptr;
+  return true;
+}
+
+__global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+
+  Unit U;
+  if (!resolve_unit(P, U)) return;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + SM_BAR);
+  uint64_t* bar_v = bar_in + 1;
+  uint64_t* bar_mma = bar_in + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_ABORT);
+  float* gamc = reinterpret_cast<float*>(sm + SM_GAMC);
+  float* betas = reinterpret_cast<float*>(sm + SM_BETA);
+  const int H = P.H, h = U.h;
+
+  if (tid == 0) {
+    mbar_init(bar_in, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lanes
+  const int half = warp >> 2;                                   // column half (8-warp passes)
+
+  const int nchunks = (int)((U.len + C - 1) / C);
+  bool pend_in = false, pend_v = false;  // thread 0: TMA loads issued, not yet waited
+  auto issue_qkg = [&](int c) {
+    const int row = (int)(U.row0 + (int64_t)c * C);
+    mbar_arrive_expect_tx(bar_in, TX_QKG);
+    tma_load_3d(sm + SM_Q, &P.tm_q, bar_in, 0, h, row);
+    tma_load_3d(sm + SM_K, &P.tm_k, bar_in, 0, h, row);
+    tma_load_3d(sm + SM_G, &P.tm_g, bar_in, 0, h, row);
+    pend_in = true;
+  };
+  auto issue_v = [&](int c) {
+    const int row = (int)(U.row0 + (int64_t)c * C);
+    mbar_arrive_expect_tx(bar_v, TX_V);
+    tma_load_3d(sm + SM_V, &P.tm_v, bar_v, 0, h, row);
+    tma_load_3d(sm + SM_V + 4096, &P.tm_v, bar_v, 64, h, row);
+    pend_v = true;
+  };
+  if (tid == 0 && nchunks > 0) {
+    issue_qkg(0);
+    if (!U.vzero) issue_v(0);
+  }
+
+  // ---- initial state -> TMEM (S^T: lane j, column i)
+  {
+    const int j = 32 * (warp & 3) + lane;
+    float v[32];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int i0 = 64 * half + 32 * cc;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int i = i0 + k;
+        v[k] = U.init ? U.init[(size_t)i * D + j] : ((U.init_identity && i == j) ? 1.f : 0.f);
+      }
+      tmem_st32(tbase + lane_base + S_COL + i0, v);
+    }
+    wait_st();
+  }
+  fence_before_sync();
+  __syncthreads();
+
+  uint32_t ph_in = 0, ph_v = 0, ph_mma = 0;
+  const uint32_t id_gram = idesc(kFmtBF16, 64, C, false, false, false);
+  const uint32_t id_w = idesc(kFmtBF16, 128, C, true, false, false);
+  const uint32_t id_o = idesc(kFmtTF32, 128, C, false, false, false);
+  const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
+  const uint32_t id_s = idesc(kFmtTF32, 128, D, false, true, false);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int64_t t0 = (int64_t)c * C;
+    const int n = (int)((U.len - t0) < C ? (U.len - t0) : C);
+    if (tid < C) betas[tid] = tid < n ? P.beta[(size_t)(U.row0 + t0 + tid) * H + h] : 0.f;
+
+    // ================================================= prep (all 256 threads)
+    mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
+    ph_in ^= 1;
+    if (tid == 0) pend_in = false;
+    const int p = tid & 63;        // channel pair 2p, 2p+1
+    const int rq = tid >> 6;       // rows 8rq .. 8rq+7
+    const int c0 = 2 * p;
+    float2 G[8];
+    {
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * rq + rr;
+        float2 gv = *reinterpret_cast<const float2*>(sm + SM_G + (r * D + c0) * 4);
+        if (r >= n) gv = make_float2(0.f, 0.f);
+        acc.x += gv.x;
+        acc.y += gv.y;
+        G[rr] = acc;
+      }
+      reinterpret_cast<float2*>(sm + SM_TT)[rq * 64 + p] = acc;  // quarter totals
+    }
+    __syncthreads();
+    if (*abort_flag) break;
+    {
+      const float2* tot = reinterpret_cast<const float2*>(sm + SM_TT);
+      float2 off = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float2 t = tot[q4 * 64 + p];
+        if (q4 < rq) { off.x += t.x; off.y += t.y; }
+      }
+      const float2 t0v = tot[p], t1v = tot[64 + p], t2v = tot[128 + p], t3v = tot[192 + p];
+      const float2 g15 = make_float2(t0v.x + t1v.x, t0v.y + t1v.y);  // Gamma at row 15
+      const float2 g31 = make_float2(g15.x + t2v.x + t3v.x, g15.y + t2v.y + t3v.y);
+      const float2 e15 = make_float2(__expf(g15.x), __expf(g15.y));
+      const float2 e3115 = make_float2(__expf(g31.x - g15.x), __expf(g31.y - g15.y));
+      if (rq == 3) {
+        gamc[c0] = __expf(g31.x);
+        gamc[c0 + 1] = __expf(g31.y);
+      }
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = 8 * rq + rr;
+        const float gx = G[rr].x + off.x, gy = G[rr].y + off.y;
+        const float ex = __expf(gx - g15.x), ey = __expf(gy - g15.y);
+        const float ix = __expf(g15.x - gx), iy = __expf(g15.y - gy);
+        const __nv_bfloat162 kk =
+            *reinterpret_cast<const __nv_bfloat162*>(sm + SM_K + (r * D + c0) * 2);
+        const __nv_bfloat162 qq =
+            *reinterpret_cast<const __nv_bfloat162*>(sm + SM_Q + (r * D + c0) * 2);
+        float kx = __low2float(kk), ky = __high2float(kk);
+        float qx = __low2float(qq), qy = __high2float(qq);
+        if (r >= n) { kx = ky = qx = qy = 0.f; }
+        const float gamx = ex * e15.x, gamy = ey * e15.y;
+        const float kcx = e3115.x * ix, kcy = e3115.y * iy;
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + sw128_off(64, r, c0, 2)) =
+            __floats2bfloat162_rn(kx * ex, ky * ey);
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + sw128_off(64, 32 + r, c0, 2)) =
+            __floats2bfloat162_rn(qx * ex, qy * ey);
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + sw128_off(32, r, c0, 2)) =
+            __floats2bfloat162_rn(kx * ix, ky * iy);
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KA + sw128_off(32, r, c0, 2)) =
+            __floats2bfloat162_rn(kx * gamx, ky * gamy);
+        *reinterpret_cast<float2*>(sm + SM_QG + sw128_off(32, r, c0, 4)) =
+            make_float2(qx * gamx, qy * gamy);
+        *reinterpret_cast<float2*>(sm + SM_KC + sw128_off(32, r, c0, 4)) =
+            make_float2(kx * kcx, ky * kcy);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ============================================== Gram GEMM (M64 N32 K128)
+    if (tid == 0) {
+      if (c + 1 < nchunks) {
+        fence_proxy_async();
+        issue_qkg(c + 1);
+      }
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kb = ks >> 2, kk = ks & 3;
+        const uint64_t a = sw128_desc(sb + SM_KQL + kb * (64 * 128) + kk * 32, 16, 1024);
+        const uint64_t b = sw128_desc(sb + SM_KB + kb * (32 * 128) + kk * 32, 16, 1024);
+        mma_ss(tbase + G_COL, a, b, id_gram, 0, ks > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 2);
+    ph_mma ^= 1;
+    fence_after_sync();
+    if (warp < 4) {
+      float v[32];
+      tmem_ld32(tbase + lane_base + G_COL, v);
+      wait_ld();
+      if (lane < 16) {
+        const int r = 16 * (warp & 1) + lane;
+        if (warp < 2) {  // A_kk row r = beta_r * strict_lower(L)[r, :]
+          const float br = betas[r];
+          float* akk = reinterpret_cast<float*>(sm + SM_AKK);
+#pragma unroll
+          for (int s = 0; s < 32; ++s) akk[r * 32 + (s ^ r)] = s < r ? br * v[s] : 0.f;
+        } else {         // A_qk row r = lower_incl(Lq)[r, :]
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            float4 w4;
+            w4.x = (4 * s4 + 0 <= r) ? v[4 * s4 + 0] : 0.f;
+            w4.y = (4 * s4 + 1 <= r) ? v[4 * s4 + 1] : 0.f;
+            w4.z = (4 * s4 + 2 <= r) ? v[4 * s4 + 2] : 0.f;
+            w4.w = (4 * s4 + 3 <= r) ? v[4 * s4 + 3] : 0.f;
+            *reinterpret_cast<float4*>(sm + SM_AQK + sw128_off(32, r, 4 * s4, 4)) = w4;
+          }
+        }
+      }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ============================ T = (I + A_kk)^-1 Diag(beta), one column per lane
+    if (warp == 0) {
+      const int cidx = lane;
+      const float* akk = reinterpret_cast<const float*>(sm + SM_AKK);
+      float x[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        float arow[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 t4 = reinterpret_cast<const float4*>(akk + r * 32)[q4];
+          arow[4 * q4 + 0] = t4.x;
+          arow[4 * q4 + 1] = t4.y;
+          arow[4 * q4 + 2] = t4.z;
+          arow[4 * q4 + 3] = t4.w;
+        }
+        float acc = (r == cidx) ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < r; ++s) acc = fmaf(-arow[s ^ r], x[s], acc);
+        x[r] = acc;
+      }
+      const float bc = betas[cidx];
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        *reinterpret_cast<__nv_bfloat16*>(sm + SM_TT + sw128_off(32, r, cidx, 2)) =
+            __float2bfloat16_rn(x[r] * bc);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ============== W^T = Ka^T T^T, U~^T = V^T T^T (bf16); O^T = S^T Qg^T (tf32)
+    if (tid == 0) {
+      if (!U.vzero) {
+        mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
+        ph_v ^= 1;
+        pend_v = false;
+      }
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        const uint64_t b = sw128_desc(sb + SM_TT + ks * 32, 16, 1024);
+        mma_ss(tbase + W_COL, sw128_desc(sb + SM_KA + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
+        if (!U.vzero)
+          mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
+      }
+      if (U.out_on) {
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+          const uint64_t b = sw128_desc(sb + SM_QG + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks, b, id_o, ks > 0);
+        }
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 4);
+    ph_mma ^= 1;
+    fence_after_sync();
+    if (warp < 4) {  // W^T (lane i, column r) -> W[r][i] fp32, tf32 B operand
+      const int i = 32 * warp + lane;
+      float v[32];
+      tmem_ld32(tbase + lane_base + W_COL, v);
+      wait_ld();
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        *reinterpret_cast<float*>(sm + SM_WF + sw128_off(32, r, i, 4)) = v[r];
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ======================================== U^T -= S^T W^T (tf32, A in TMEM)
+    if (tid == 0) {
+      if (c + 1 < nchunks && !U.vzero) {
+        fence_proxy_async();
+        issue_v(c + 1);
+      }
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint64_t b = sw128_desc(sb + SM_WF + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+        mma_ts_tf32(tbase + U_COL, tbase + S_COL + 8 * ks, b, id_u, (ks > 0) || !U.vzero);
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 5);
+    ph_mma ^= 1;
+    fence_after_sync();
+    {  // decay the state: S^T[j][i] *= e^{Gamma_C, i}
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t col = S_COL + 64 * half + 32 * cc;
+        float v[32];
+        tmem_ld32(tbase + lane_base + col, v);
+        wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] *= gamc[64 * half + 32 * cc + k];
+        tmem_st32(tbase + lane_base + col, v);
+      }
+      wait_st();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ============ S^T += U^T Kc;  O^T += U^T A_qk^T   (tf32, U^T read from TMEM)
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t b = sw128_desc(sb + SM_KC + ks * 1024, 4096, 1024);
+        mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks, b, id_s, 1);
+      }
+      if (U.out_on) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t b = sw128_desc(sb + SM_AQK + ks * 32, 16, 1024);
+          mma_ts_tf32(tbase + O_COL, tbase + U_COL + 8 * ks, b, id_o, 1);
+        }
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
+    ph_mma ^= 1;
+    fence_after_sync();
+    if (U.out_on && warp < 4) {  // O^T (lane j, column r) -> o[row0 + t0 + r, h, j]
+      const int j = 32 * warp + lane;
+      float v[32];
+      tmem_ld32(tbase + lane_base + O_COL, v);
+      wait_ld();
+      __nv_bfloat16* orow = P.out + ((size_t)(U.row0 + t0) * H + h) * D + j;
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        if (r < n) orow[(size_t)r * H * D] = __float2bfloat16_rn(P.scale * v[r]);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+  }
+
+  // ---- final state (S^T lane j, column i -> final[i][j])
+  if (U.final_state && !*abort_flag) {
+    const int j = 32 * (warp & 3) + lane;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int i0 = 64 * half + 32 * cc;
+      float v[32];
+      tmem_ld32(tbase + lane_base + S_COL + i0, v);
+      wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) U.final_state[(size_t)(i0 + k) * D + j] = v[k];
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    // let any TMA load still in flight land before the CTA's memory is released
+    if (pend_in) mbar_wait_bounded(bar_in, ph_in, abort_flag, nullptr, 7);
+    if (pend_v) mbar_wait_bounded(bar_v, ph_v, abort_flag, nullptr, 8);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tbase, TMEM_COLS);
+}
+
+// S_in[g+1] = S~_g + M_g S_in[g] for every unit, one 32-column slice per CTA.
+__global__ void __launch_bounds__(256) segment_combine_kernel(const float* __restrict__ init,
+                                                              float* __restrict__ ws, int U,
+                                                              int G) {
+  __shared__ float X[D][33];
+  const size_t DD = (size_t)D * D;
+  const int un = blockIdx.x >> 2, j0 = (blockIdx.x & 3) * 32;
+  const int tid = threadIdx.x, jj = tid & 31, i0 = tid >> 5;
+  for (int k = 0; k < 16; ++k) {
+    const int i = i0 + 8 * k;
+    X[i][jj] = init ? init[un * DD + (size_t)i * D + j0 + jj] : 0.f;
+  }
+  __syncthreads();
+  const float* pairs = ws + (size_t)un * (G - 1) * 2 * DD;
+  float* s_in = ws + ((size_t)U * (G - 1) * 2 + (size_t)un * (G - 1)) * DD;
+  for (int g = 0; g < G - 1; ++g) {
+    const float* St = pairs + (size_t)(2 * g) * DD;
+    const float* M = pairs + (size_t)(2 * g + 1) * DD;
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = St[(size_t)(i0 + 8 * k) * D + j0 + jj];
+    for (int ip = 0; ip < D; ++ip) {
+      const float x = X[ip][jj];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = fmaf(__ldg(M + (size_t)(i0 + 8 * k) * D + ip), x, acc[k]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      X[i0 + 8 * k][jj] = acc[k];
+      s_in[(size_t)g * DD + (size_t)(i0 + 8 * k) * D + j0 + jj] = acc[k];
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base, int H,
+               int64_t R, uint32_t box0, CUtensorMapSwizzle sw) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)R};
+  cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz};
+  cuuint32_t box[3] = {box0, 1, (cuuint32_t)C};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Segment split for long dense sequences with too few (sequence, head)
+// units to occupy the GPU: returns G >= 2 and the segment length, or G = 1.
+void plan_split(int B, int T, int H, int num_sms, int* G_out, int* seg_out) {
+  const int U = B * H;
+  *G_out = 1;
+  *seg_out = T;
+  if (2 * U >= num_sms || T < 4 * 1024) return;
+  int G = (2 * num_sms + U - 1) / U;
+  const int max_g = T / 1024;
+  if (G > max_g) G = max_g;
+  if (G < 2) return;
+  int seg = (T + G - 1) / G;
+  seg = (seg + C - 1) / C * C;
+  G = (T + seg - 1) / seg;
+  if (G < 2) return;
+  *G_out = G;
+  *seg_out = seg;
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(int B, int T, int H, int num_seqs, int num_sms) {
+  if (num_seqs > 0) return 0;
+  int G, seg;
+  plan_split(B, T, H, num_sms, &G, &seg);
+  if (G < 2) return 0;
+  return (size_t)B * H * (G - 1) * 3 * D * D * sizeof(float);
+}
+
+cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_bytes,
+                            cudaStream_t stream) {
+  if (a.num_units == 0) return cudaSuccess;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  const int64_t R = (int64_t)a.map.B * a.map.T;
+  const int H = a.map.H;
+  if (!encode_3d(&P.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&P.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.k, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&P.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.v, H, R, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_3d(&P.tm_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.g, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  P.beta = a.beta;
+  P.out = static_cast<__nv_bfloat16*>(a.out);
+  P.init_state = a.init_state;
+  P.final_state = a.final_state;
+  P.cu_seqlens = a.map.cu_seqlens;
+  P.order = a.map.order;
+  P.sb = a.sb;
+  P.B = a.map.B;
+  P.T = a.map.T;
+  P.H = H;
+  P.scale = a.scale;
+  P.mode = 0;
+  P.G = 1;
+  P.seg_len = a.map.T;
+
+  int G = 1, seg = a.map.T;
+  if (a.map.cu_seqlens == nullptr) plan_split(a.map.B, a.map.T, H, device_sm_count(), &G, &seg);
+  if (G < 2) {
+    chunk_tc_kernel<<<a.num_units, NT, SMEM_ALLOC, stream>>>(P);
+    return cudaGetLastError();
+  }
+  const int U = a.map.B * H;
+  const size_t need = (size_t)U * (G - 1) * 3 * D * D * sizeof(float);
+  if (ws_tail_bytes < need) return cudaErrorInvalidValue;
+  P.seg_ws = static_cast<float*>(ws_tail);
+  P.G = G;
+  P.seg_len = seg;
+  P.mode = 1;
+  chunk_tc_kernel<<<U * (G - 1) * 2, NT, SMEM_ALLOC, stream>>>(P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  segment_combine_kernel<<<U * 4, 256, 0, stream>>>(a.init_state, P.seg_ws, U, G);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  P.mode = 2;
+  chunk_tc_kernel<<<U * G, NT, SMEM_ALLOC, stream>>>(P);
+  return cudaGetLastError();
 }
 
 }  // namespace kda

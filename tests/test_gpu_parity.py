@@ -196,3 +196,63 @@ def test_bounded_wait_times_out_and_context_survives():
     assert st == kda.KDA_ERR_TIMEOUT
     x = torch.ones(4, device=DEV)
     assert float((x * 2).sum()) == 8.0  # the context is still usable
+
+
+# ------------------------------------------------- tensor-core path specifics
+
+def _slow_decay(inp, shift=4.0):
+    """Same draws with z shifted down: g close to 0, so memory spans many
+    chunks and segment transitions M stay far from zero."""
+    out = dict(inp)
+    out["z"] = (inp["z"] - shift).contiguous()
+    return out
+
+
+@pytest.mark.parametrize("slow", [False, True])
+def test_prefill_tc_segment_split(oracle_mod, slow):
+    """B*H = 2 units over T = 5000 tokens: the tensor-core path splits each
+    sequence into segments, computes their transitions, combines them and
+    reruns the segments from the true incoming states."""
+    inp = W.make_prefill_inputs(1, 5000, 2, 128, 128, torch.bfloat16, seed=31, device=DEV,
+                                init_state=True)
+    if slow:
+        inp = _slow_decay(inp)
+    o, S, _, ws = gpu_prefill(inp)
+    assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+
+
+@pytest.mark.parametrize("T", [32, 33, 700])
+def test_prefill_tc_slow_decay(oracle_mod, T):
+    inp = _slow_decay(W.make_prefill_inputs(3, T, 2, 128, 128, torch.bfloat16, seed=40 + T,
+                                            device=DEV, init_state=True))
+    o, S, _, _ = gpu_prefill(inp, scale=0.5)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, scale=0.5)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+
+
+def test_tc_matches_fp32_kernel():
+    """Chunk-size / kernel consistency: tensor-core C = 32 against the fp32
+    CUDA-core kernel at C = 64 on the same bf16 inputs."""
+    inp = W.make_prefill_inputs(2, 257, 4, 128, 128, torch.bfloat16, seed=12, device=DEV,
+                                init_state=True)
+    o_tc, S_tc, _, _ = gpu_prefill(inp, chunk=0)
+    o_64, S_64, _, _ = gpu_prefill(inp, chunk=64)
+    assert rel_l2(to64(o_tc), to64(o_64)) <= TOL_BF16_O
+    assert rel_l2(to64(S_tc), to64(S_64)) <= TOL_BF16_S
+
+
+def test_tc_rerun_is_deterministic_and_input_sensitive():
+    """Same inputs twice give bit-identical outputs; changing one value of v
+    changes the output (no caching of results between calls)."""
+    inp = W.make_prefill_inputs(1, 96, 2, 128, 128, torch.bfloat16, seed=13, device=DEV)
+    o1, S1, _, _ = gpu_prefill(inp)
+    o2, S2, _, _ = gpu_prefill(inp)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    inp["v"][0, 50, 1, 7] += 1.0
+    o3, _, _, _ = gpu_prefill(inp)
+    assert not torch.equal(o1[0, 50:, 1], o3[0, 50:, 1])
+    assert torch.equal(o1[0, :50], o3[0, :50])
