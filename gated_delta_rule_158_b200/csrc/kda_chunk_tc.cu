@@ -66,7 +66,7 @@ constexpr uint32_t SM_AQK = SM_R1 + 20480;    //  A_qk fp32 32 x 32 (tf32 B)
 constexpr uint32_t SM_KA = 65536;    // k e^G        bf16 [s][i] (MN-major A of W)
 constexpr uint32_t SM_TT = 73728;    // T            bf16 [r][s] (B of W and U~); cumsum partials during prep
 constexpr uint32_t SM_QG = 77824;    // q e^G        fp32 [r][i] (tf32 B of O)
-constexpr uint32_t SM_KC = 94208;    // k e^{GC-G}   fp32 [s][i] (MN-major tf32 B of S)
+constexpr uint32_t SM_KC = 94208;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
 constexpr uint32_t SM_MISC = 110592;
 constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
 constexpr uint32_t SM_BETA = SM_MISC + 512;    // beta         fp32 [32]
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const uint32_t id_w = idesc(kFmtBF16, 128, C, true, false, false);
   const uint32_t id_o = idesc(kFmtTF32, 128, C, false, false, false);
   const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
-  const uint32_t id_s = idesc(kFmtTF32, 128, D, false, true, false);
+  const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
 
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = (int64_t)c * C;
@@ -313,8 +313,10 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
             __floats2bfloat162_rn(kx * gamx, ky * gamy);
         *reinterpret_cast<float2*>(sm + SM_QG + sw128_off(32, r, c0, 4)) =
             make_float2(qx * gamx, qy * gamy);
-        *reinterpret_cast<float2*>(sm + SM_KC + sw128_off(32, r, c0, 4)) =
-            make_float2(kx * kcx, ky * kcy);
+        // Kc^T [i][s]: K-major tf32 B of the state update (tf32 MMAs take
+        // no MN-major B operand, so the transpose is written here)
+        *reinterpret_cast<float*>(sm + SM_KC + sw128_off(128, c0, r, 4)) = kx * kcx;
+        *reinterpret_cast<float*>(sm + SM_KC + sw128_off(128, c0 + 1, r, 4)) = ky * kcy;
       }
     }
     fence_proxy_async();
@@ -480,7 +482,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t b = sw128_desc(sb + SM_KC + ks * 1024, 4096, 1024);
+        const uint64_t b = sw128_desc(sb + SM_KC + ks * 32, 16, 1024);
         mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks, b, id_s, 1);
       }
       if (U.out_on) {
