@@ -364,11 +364,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B of a dense prefill workload (smaller profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
     world, rank, local = dist_setup()
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    if args.batch is not None and not wl.get("varlen", True):
+        wl["B"] = args.batch
+        wl["name"] = wl["name"].replace(f"B{WORKLOADS[args.workload]['B']} ", f"B{args.batch} ")
     peaks = load_peaks()
 
     if args.impl == "reference":
