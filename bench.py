@@ -58,6 +58,18 @@ def prefill_flops_per_token_head(C=32, dk=128, dv=128):
     return C * (3 * dk + 2 * dv) + C * C / 3 + 6 * dk * dv
 
 
+def kernels_per_step(wl, B, T):
+    """libkda kernels one prefill step launches: one chunk kernel; the varlen
+    plan kernel in front for varlen; three (transitions, combine, outputs)
+    when the long-sequence split applies (B*H*2 < SMs and T >= 4096)."""
+    if wl.get("varlen"):
+        return 2
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if 2 * B * wl["H"] < sms and T >= 4096:
+        return 3
+    return 1
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -161,14 +173,14 @@ def make_prefill(wl, device):
 
 
 class PrefillStep:
-    """gate + chunk_fwd on resident inputs, events around each launch."""
+    """One step: kda_chunk_fwd_gated (gate fused into the chunk kernel) on
+    resident inputs, with events around the launch."""
 
     def __init__(self, inp, cu, N):
         self.inp, self.cu = inp, cu
         q = inp["q"]
         B, T, H, dk = q.shape
         dv = inp["v"].shape[-1]
-        self.g = torch.empty_like(inp["z"])
         self.out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
         self.final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
         nbytes = kda.kda_chunk_fwd_workspace_size(B, T, H, dk, dv,
@@ -179,14 +191,11 @@ class PrefillStep:
         i = self.inp
         if ev:
             ev[0].record()
-        kda.kda_gate_fwd(i["z"], i["A_log"], self.g)
+        kda.kda_chunk_fwd_gated(i["q"], i["k"], i["v"], i["z"], i["A_log"], i["beta"], self.out,
+                                self.ws, init_state=i["init_state"], cu_seqlens=self.cu,
+                                final_state=self.final)
         if ev:
             ev[1].record()
-        kda.kda_chunk_fwd(i["q"], i["k"], i["v"], self.g, i["beta"], self.out, self.ws,
-                          init_state=i["init_state"], cu_seqlens=self.cu,
-                          final_state=self.final)
-        if ev:
-            ev[2].record()
 
 
 def time_steps(step, K, Wm, world):
@@ -194,7 +203,7 @@ def time_steps(step, K, Wm, world):
         step()
     torch.cuda.synchronize()
     barrier(world)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -204,10 +213,9 @@ def time_steps(step, K, Wm, world):
     stop.record()
     torch.cuda.synchronize()
     total_ms = start.elapsed_time(stop)
-    gate_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    chunk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    chunk_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     barrier(world)
-    return max_over_ranks(total_ms, world), gate_ms, chunk_ms
+    return max_over_ranks(total_ms, world), chunk_ms
 
 
 def e2e_prefill(wl, inp, cu, N, K):
@@ -249,14 +257,12 @@ def run_decode(wl, device, warmup=3):
     # all steps' inputs resident before timing (fresh inputs per step)
     xs = [W.make_decode_step_inputs(N, H, dk, dv, torch.bfloat16, wl["seed"] + s, device)
           for s in range(steps)]
-    g = torch.empty((N, H, dk), dtype=torch.float32, device=device)
     o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=device)
 
     def step(x, ev=None):
-        kda.kda_gate_fwd(x["z"], A_log, g)
         if ev:
             ev[0].record()
-        kda.kda_decode_step(x["q"], x["k"], x["v"], g, x["beta"], state, o)
+        kda.kda_decode_step_gated(x["q"], x["k"], x["v"], x["z"], A_log, x["beta"], state, o)
         if ev:
             ev[1].record()
 
@@ -404,7 +410,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
     tokens = B * T  # per rank
     step = PrefillStep(inp, cu, N)
     clocks = ClockSampler(dev.index)
-    total_ms, gate_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
+    total_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
     clk = clocks.stop()
     st, _ = kda.kda_get_device_status(step.ws)
     if st != kda.KDA_OK:
@@ -424,15 +430,14 @@ def bench_prefill_line(args, wl, world, rank, peaks):
         "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T,
                    "heads": H, "dk": dk, "dv": dv, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (no flush needed)",
-                   "step": "kda_gate_fwd + kda_chunk_fwd"},
+                   "step": "kda_chunk_fwd_gated (gate fused)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                     "traffic": None, "kernel": "kda_chunk_fwd",
+                     "traffic": None, "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
                      "kernel_ms": round(chunk_ms, 4), "algorithmic_bytes": alg_bytes,
                      "peak_source": peaks["src"],
                      "tensor_frac": round(flops / (chunk_ms * 1e-3) / (peaks["tc"] * 1e12), 4)},
-        "gate_ms": round(gate_ms, 4),
-        "gpu_launches": args.steps * 2,
+        "gpu_launches": args.steps * kernels_per_step(wl, B, T),
         "clocks": clk,
     }
     if not args.no_e2e:
@@ -455,7 +460,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
                           "roofline": {"bound": "hbm", "achieved": round(dach, 1),
                                        "peak": peaks["hbm"], "unit": "GB/s",
                                        "frac": round(dach / peaks["hbm"], 4),
-                                       "kernel": "kda_decode_step",
+                                       "kernel": "decode_kernel (kda_decode_step_gated)",
                                        "kernel_ms": round(dec_ms, 4),
                                        "algorithmic_bytes": bpl}}
     return line
@@ -478,8 +483,9 @@ def bench_decode_line(args, wl, world, rank, peaks):
                    "l2": "state (1 GiB) larger than L2"},
         "roofline": {"bound": "hbm", "achieved": round(dach, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(dach / peaks["hbm"], 4), "traffic": None,
-                     "kernel": "kda_decode_step", "kernel_ms": round(dec_ms, 4)},
-        "gpu_launches": wl["steps"] * 2, "clocks": clk,
+                     "kernel": "decode_kernel (kda_decode_step_gated)",
+                     "kernel_ms": round(dec_ms, 4)},
+        "gpu_launches": wl["steps"], "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, secs = oracle_decode_sample(wl)

@@ -37,7 +37,11 @@ _SIGNATURES = {
     "kda_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "kda_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
                            _F, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "kda_chunk_fwd_gated": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _VP, _I, _I, _I, _I,
+                                 _I, _I, _F, _I, _VP, _VP, _VP, _SZ, _VP]),
     "kda_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _I, _I, _I, _I, _F, _VP, _VP]),
+    "kda_decode_step_gated": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _I, _I, _I, _I, _F,
+                                   _VP, _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
@@ -128,6 +132,30 @@ def kda_chunk_fwd(q, k, v, g, beta, out, workspace, init_state=None, cu_seqlens=
         _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale), int(chunk_size), _ptr(out),
         _ptr(final_state), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)), "kda_chunk_fwd")
+
+
+def kda_chunk_fwd_gated(q, k, v, z, A_log, beta, out, workspace, g_min=-5.0, init_state=None,
+                        cu_seqlens=None, final_state=None, scale=1.0, chunk_size=0, stream=None):
+    """kda_chunk_fwd with the gate fused in: z [B,T,H,dk] and A_log [H] replace g."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib().kda_chunk_fwd_gated(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta), _dtype(q),
+        _ptr(init_state), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale),
+        int(chunk_size), _ptr(out), _ptr(final_state), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "kda_chunk_fwd_gated")
+
+
+def kda_decode_step_gated(q, k, v, z, A_log, beta, state, out, g_min=-5.0, scale=1.0,
+                          stream=None):
+    """kda_decode_step with the gate fused in: z [N,H,dk] and A_log [H] replace g."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(lib().kda_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log),
+                                       float(g_min), _ptr(beta), _dtype(q), _ptr(state), N, H,
+                                       dk, dv, float(scale), _ptr(out), _stream(stream)),
+           "kda_decode_step_gated")
 
 
 def kda_decode_step(q, k, v, g, beta, state, out, scale=1.0, stream=None):

@@ -126,12 +126,20 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   return bytes;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
-                         const float* beta, kda_dtype in_dtype, const float* init_state,
-                         const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
-                         int dv, float scale, int chunk_size, void* out, float* final_state,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of kda_chunk_fwd and kda_chunk_fwd_gated: g is the log-decay,
+// or z when A_log is not null.
+kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
+                          const float* A_log, float g_min, const float* beta,
+                          kda_dtype in_dtype, const float* init_state,
+                          const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                          int dv, float scale, int chunk_size, void* out, float* final_state,
+                          void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !g || !beta || !out || !workspace) return KDA_ERR_INVALID_ARG;
+  if (A_log && (!(g_min < 0.f) || !isfinite(g_min))) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (B <= 0 || T <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
   if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
@@ -143,11 +151,11 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
   } else if (num_seqs != 0 && num_seqs != B) {
     return KDA_ERR_INVALID_ARG;
   }
-  const void* ptrs[] = {q, k, v, g, beta, out, workspace, init_state, final_state, cu_seqlens};
+  const void* ptrs[] = {q, k, v, g, beta, out, workspace, init_state, final_state, cu_seqlens, A_log};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
   const void* outs[] = {out};
-  const void* ins[] = {q, k, v, g, beta, init_state, cu_seqlens};
+  const void* ins[] = {q, k, v, g, beta, init_state, cu_seqlens, A_log};
   for (const void* o : outs)
     for (const void* i : ins)
       if (i && o == i) return KDA_ERR_INVALID_ARG;
@@ -167,6 +175,9 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
   a.k = k;
   a.v = v;
   a.g = g;
+  a.A_log = A_log;
+  a.g_min = g_min;
+  a.gated = A_log != nullptr;
   a.beta = beta;
   a.dt = in_dtype;
   a.init_state = init_state;
@@ -203,23 +214,76 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* g,
-                           const float* beta, kda_dtype in_dtype, float* state, int N, int H,
-                           int dk, int dv, float scale, void* out, void* stream) {
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, kda_dtype in_dtype, const float* init_state,
+                         const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                         int dv, float scale, int chunk_size, void* out, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return chunk_fwd_impl(q, k, v, g, nullptr, 0.f, beta, in_dtype, init_state, cu_seqlens,
+                        num_seqs, B, T, H, dk, dv, scale, chunk_size, out, final_state,
+                        workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* z,
+                               const float* A_log, float g_min, const float* beta,
+                               kda_dtype in_dtype, const float* init_state,
+                               const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                               int dk, int dv, float scale, int chunk_size, void* out,
+                               float* final_state, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!A_log) return KDA_ERR_INVALID_ARG;
+  return chunk_fwd_impl(q, k, v, z, A_log, g_min, beta, in_dtype, init_state, cu_seqlens,
+                        num_seqs, B, T, H, dk, dv, scale, chunk_size, out, final_state,
+                        workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+kda_status decode_impl(const void* q, const void* k, const void* v, const float* g,
+                       const float* A_log, float g_min, const float* beta, kda_dtype in_dtype,
+                       float* state, int N, int H, int dk, int dv, float scale, void* out,
+                       void* stream) {
   if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (N <= 0 || H <= 0 || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (A_log && (!(g_min < 0.f) || !isfinite(g_min))) return KDA_ERR_INVALID_ARG;
   if ((int64_t)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
   if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q, k, v, g, beta, state, out};
+  const void* ptrs[] = {q, k, v, g, beta, state, out, A_log};
   for (const void* p : ptrs)
-    if (!aligned16(p)) return KDA_ERR_MISALIGNED;
-  const void* ins[] = {q, k, v, g, beta, state};
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {q, k, v, g, beta, state, A_log};
   for (const void* i : ins)
     if (i == out) return KDA_ERR_INVALID_ARG;
-  cudaError_t e =
-      launch_decode(q, k, v, g, beta, in_dtype, state, N, H, dk, dv, scale, out, (cudaStream_t)stream);
+  cudaError_t e = launch_decode(q, k, v, g, A_log, g_min, beta, in_dtype, state, N, H, dk, dv,
+                                scale, out, (cudaStream_t)stream);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, kda_dtype in_dtype, float* state, int N, int H,
+                           int dk, int dv, float scale, void* out, void* stream) {
+  return decode_impl(q, k, v, g, nullptr, 0.f, beta, in_dtype, state, N, H, dk, dv, scale, out,
+                     stream);
+}
+
+kda_status kda_decode_step_gated(const void* q, const void* k, const void* v, const float* z,
+                                 const float* A_log, float g_min, const float* beta,
+                                 kda_dtype in_dtype, float* state, int N, int H, int dk, int dv,
+                                 float scale, void* out, void* stream) {
+  if (!A_log) return KDA_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, z, A_log, g_min, beta, in_dtype, state, N, H, dk, dv, scale, out,
+                     stream);
 }
 
 kda_status kda_get_device_status(const void* workspace, void* stream, int32_t* detail) {

@@ -40,6 +40,7 @@ template <typename Tin, int DK, int C>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                       const Tin* __restrict__ v, const float* __restrict__ g,
+                      const float* __restrict__ A_log, float g_min,
                       const float* __restrict__ beta, const float* __restrict__ init_state,
                       float* __restrict__ final_state, Tin* __restrict__ out, UnitMap map,
                       int dv, float scale) {
@@ -79,6 +80,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sidx = (int64_t)n * H + h;
   }
 
+  // g is the log-decay, or z when A_log is given (gate fused in)
+  const float a_h = A_log ? expf(A_log[h]) : 0.f;
+
   // state slice
   for (int idx = tid; idx < DK * kDVS; idx += kThreads) {
     const int i = idx / kDVS, j = idx % kDVS;
@@ -96,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         kv = Elem<Tin>::load(k + off);
         qv = Elem<Tin>::load(q + off);
         gv = g[off];
+        if (A_log) gv = gate_value(gv, a_h, g_min);
       }
       kS[r * LDK + i] = kv;
       qS[r * LDK + i] = qv;
@@ -225,7 +230,8 @@ cudaError_t launch_one(const ChunkArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(a.num_units * (a.dv / kDVS));
   kern<<<grid, kThreads, smem, st>>>(static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k),
-                                     static_cast<const Tin*>(a.v), a.g, a.beta, a.init_state,
+                                     static_cast<const Tin*>(a.v), a.g,
+                                     a.gated ? a.A_log : nullptr, a.g_min, a.beta, a.init_state,
                                      a.final_state, static_cast<Tin*>(a.out), a.map, a.dv,
                                      a.scale);
   return cudaGetLastError();

@@ -80,7 +80,9 @@ constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
 constexpr uint32_t TX_V = 8192;
 
 struct TcParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_g;
+  CUtensorMap tm_q, tm_k, tm_v, tm_g;  // tm_g maps g, or z when A_log is set
+  const float* A_log;                  // gate fused in when not null
+  float g_min;
   const float* beta;
   __nv_bfloat16* out;
   const float* init_state;
@@ -196,6 +198,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const int half = warp >> 2;                                   // column half (8-warp passes)
 
   const int nchunks = (int)((U.len + C - 1) / C);
+  const float a_h = P.A_log ? expf(P.A_log[h]) : 0.f;
   bool pend_in = false, pend_v = false;  // thread 0: TMA loads issued, not yet waited
   auto issue_qkg = [&](int c) {
     const int row = (int)(U.row0 + (int64_t)c * C);
@@ -262,6 +265,10 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       for (int rr = 0; rr < 8; ++rr) {
         const int r = 8 * rq + rr;
         float2 gv = *reinterpret_cast<const float2*>(sm + SM_G + (r * D + c0) * 4);
+        if (P.A_log) {  // fused gate: the tile holds z; g = g_min sigmoid(e^A z)
+          gv.x = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.x));
+          gv.y = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.y));
+        }
         if (r >= n) gv = make_float2(0.f, 0.f);
         acc.x += gv.x;
         acc.y += gv.y;
@@ -651,6 +658,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_by
       !encode_3d(&P.tm_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.g, H, R, 128,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  P.A_log = a.gated ? a.A_log : nullptr;
+  P.g_min = a.g_min;
   P.beta = a.beta;
   P.out = static_cast<__nv_bfloat16*>(a.out);
   P.init_state = a.init_state;

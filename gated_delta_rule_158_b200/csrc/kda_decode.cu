@@ -35,6 +35,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const float* __restrict__ g,
+                  const float* __restrict__ A_log, float g_min, int H,
                   const float* __restrict__ beta, float* __restrict__ state, float scale,
                   Tin* __restrict__ out) {
   constexpr int CG = DV / 4;         // threads per state row (float4 each)
@@ -56,10 +57,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
   for (int r = 0; r < RPT; ++r) s[r] = __ldcs(S4 + (rg + r * RG) * CG + cg);
 
+  // g is the log-decay, or z when A_log is given (gate fused in)
+  const float a_h = A_log ? expf(A_log[unit % H]) : 0.f;
   for (int i = tid; i < DK; i += kThreads) {
     sk[i] = Elem<Tin>::load(k + (size_t)unit * DK + i);
     sq[i] = Elem<Tin>::load(q + (size_t)unit * DK + i);
-    sa[i] = expf(g[(size_t)unit * DK + i]);
+    const float gi = g[(size_t)unit * DK + i];
+    sa[i] = expf(A_log ? gate_value(gi, a_h, g_min) : gi);
   }
   __syncthreads();
 
@@ -119,9 +123,9 @@ cudaError_t dispatch_dv(const ChunkArgs& a, int N, int H, int dv, cudaStream_t s
   Tin* o = static_cast<Tin*>(a.out);
   float* S = const_cast<float*>(a.init_state);
   switch (dv) {
-    case 32: decode_kernel<Tin, DK, 32><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.beta, S, a.scale, o); break;
-    case 64: decode_kernel<Tin, DK, 64><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.beta, S, a.scale, o); break;
-    case 128: decode_kernel<Tin, DK, 128><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.beta, S, a.scale, o); break;
+    case 32: decode_kernel<Tin, DK, 32><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.A_log, a.g_min, H, a.beta, S, a.scale, o); break;
+    case 64: decode_kernel<Tin, DK, 64><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.A_log, a.g_min, H, a.beta, S, a.scale, o); break;
+    case 128: decode_kernel<Tin, DK, 128><<<grid, kThreads, 0, st>>>(q, k, v, a.g, a.A_log, a.g_min, H, a.beta, S, a.scale, o); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -139,14 +143,17 @@ cudaError_t dispatch_dk(const ChunkArgs& a, int N, int H, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
-                          const float* beta, kda_dtype dt, float* state, int N, int H,
-                          int dk, int dv, float scale, void* out, cudaStream_t stream) {
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g_or_z,
+                          const float* A_log, float g_min, const float* beta, kda_dtype dt,
+                          float* state, int N, int H, int dk, int dv, float scale, void* out,
+                          cudaStream_t stream) {
   ChunkArgs a{};
   a.q = q;
   a.k = k;
   a.v = v;
-  a.g = g;
+  a.g = g_or_z;
+  a.A_log = A_log;
+  a.g_min = g_min;
   a.beta = beta;
   a.dt = dt;
   a.init_state = state;

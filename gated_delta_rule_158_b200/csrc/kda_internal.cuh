@@ -59,10 +59,16 @@ cudaError_t launch_gate(const float* z, const float* A_log, float g_min,
                         float* g, int64_t rows, int H, int dk,
                         cudaStream_t stream);
 
+// g_or_z is g, or z when A_log != nullptr (gate fused into the kernel)
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
-                          const float* g, const float* beta, kda_dtype dt,
-                          float* state, int N, int H, int dk, int dv,
-                          float scale, void* out, cudaStream_t stream);
+                          const float* g_or_z, const float* A_log, float g_min,
+                          const float* beta, kda_dtype dt, float* state, int N,
+                          int H, int dk, int dv, float scale, void* out,
+                          cudaStream_t stream);
+
+__device__ __forceinline__ float gate_value(float z, float a, float g_min) {
+  return g_min / (1.0f + expf(-a * z));
+}
 
 cudaError_t launch_varlen_plan(const int32_t* cu_seqlens, int num_seqs, int T,
                                int32_t* order, StatusBlock* sb,
@@ -72,7 +78,10 @@ struct ChunkArgs {
   const void* q;
   const void* k;
   const void* v;
-  const float* g;
+  const float* g;       // log-decay g, or z when `gated`
+  const float* A_log;   // gated only: per-head gate parameter
+  float g_min;          // gated only
+  bool gated;           // g = g_min * sigmoid(exp(A_log[h]) * z) formed in-kernel
   const float* beta;
   kda_dtype dt;
   const float* init_state;

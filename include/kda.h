@@ -125,6 +125,25 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
                          size_t workspace_bytes, void *stream);
 
 /*
+ * kda_chunk_fwd with the gate fused in (the chunk kernels read z instead of
+ * g and form g = g_min * Sigmoid(exp(A_log[h]) * z) on the fly, saving the
+ * write and re-read of g):
+ *  z      : fp32 [B, T, H, dk]   (replaces g)
+ *  A_log  : fp32 [H]
+ *  g_min  : finite and negative (KDA uses -5)
+ * Every other argument, the workspace size and the errors are as for
+ * kda_chunk_fwd.
+ */
+KDA_API kda_status kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
+                               const float *z, const float *A_log, float g_min,
+                               const float *beta, kda_dtype in_dtype,
+                               const float *init_state, const int32_t *cu_seqlens,
+                               int num_seqs, int B, int T, int H, int dk, int dv,
+                               float scale, int chunk_size, void *out,
+                               float *final_state, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
  * One single-token decode step for N sequences, updating the state in place
  * (KDA decoding: same page, Online serving > high-performance kernels; the
  * state is rewritten in place every token).  Per (n, h):
@@ -140,6 +159,18 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            kda_dtype in_dtype, float *state, int N, int H,
                            int dk, int dv, float scale, void *out,
                            void *stream);
+
+/*
+ * kda_decode_step with the gate fused in: z (fp32 [N, H, dk]) and A_log
+ * (fp32 [H]) replace g, and the kernel forms
+ * alpha = exp(g_min * Sigmoid(exp(A_log[h]) * z)).  Other arguments as for
+ * kda_decode_step.
+ */
+KDA_API kda_status kda_decode_step_gated(const void *q, const void *k, const void *v,
+                                 const float *z, const float *A_log, float g_min,
+                                 const float *beta, kda_dtype in_dtype,
+                                 float *state, int N, int H, int dk, int dv,
+                                 float scale, void *out, void *stream);
 
 /*
  * Synchronises `stream`, then returns the device status word that kernels

@@ -115,3 +115,20 @@ def test_device_status_rejects_null(L):
     assert L.kda_get_device_status(None, None, None) == 1
     assert L.kda_selftest_bounded_wait(None, 1000, None) == 1
     assert L.kda_selftest_bounded_wait(FAKE + 4, 1000, None) == 3
+
+
+def test_gated_entries_reject_on_host(L):
+    args = [FAKE, FAKE + 0x1000, FAKE + 0x2000, FAKE + 0x3000, FAKE + 0x9000, -5.0,
+            FAKE + 0x4000, _lib.KDA_BF16, None, None, 0, 2, 64, 4, 128, 128, 1.0, 0,
+            FAKE + 0x5000, None, FAKE + 0x6000, 1 << 40, None]
+    bad = list(args); bad[4] = None           # A_log missing
+    assert L.kda_chunk_fwd_gated(*bad) == _lib.KDA_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 5.0            # g_min must be negative
+    assert L.kda_chunk_fwd_gated(*bad) == _lib.KDA_ERR_INVALID_ARG
+    bad = list(args); bad[4] = FAKE + 0x9004  # misaligned A_log
+    assert L.kda_chunk_fwd_gated(*bad) == _lib.KDA_ERR_MISALIGNED
+    d = [FAKE, FAKE, FAKE, FAKE, None, -5.0, FAKE, 1, FAKE, 4, 2, 128, 128, 1.0, FAKE + 64, None]
+    assert L.kda_decode_step_gated(*d) == _lib.KDA_ERR_INVALID_ARG
+    d[4] = FAKE + 16
+    d[5] = float("inf")
+    assert L.kda_decode_step_gated(*d) == _lib.KDA_ERR_INVALID_ARG

@@ -256,3 +256,80 @@ def test_tc_rerun_is_deterministic_and_input_sensitive():
     o3, _, _, _ = gpu_prefill(inp)
     assert not torch.equal(o1[0, 50:, 1], o3[0, 50:, 1])
     assert torch.equal(o1[0, :50], o3[0, :50])
+
+
+# ------------------------------------------------------------ fused gate
+
+def _gated_prefill(inp, cu=None, chunk=0, scale=1.0):
+    q, k, v, z, A_log, beta = (inp[n] for n in ("q", "k", "v", "z", "A_log", "beta"))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu is None else cu.numel() - 1
+    out = torch.full((B, T, H, dv), float("nan"), device=q.device, dtype=q.dtype)
+    fin = torch.full((N, H, dk, dv), float("nan"), device=q.device)
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(
+        B, T, H, dk, dv, 0 if cu is None else N, chunk,
+        kda.KDA_BF16 if q.dtype == torch.bfloat16 else kda.KDA_F32), dtype=torch.uint8,
+        device=q.device)
+    kda.kda_chunk_fwd_gated(q, k, v, z, A_log, beta, out, ws, init_state=inp["init_state"],
+                            cu_seqlens=cu, final_state=fin, scale=scale, chunk_size=chunk)
+    assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
+    return out, fin
+
+
+def test_gated_prefill_fp32_tiny(oracle_mod):
+    inp = W.make_prefill_inputs(1, 64, 2, 32, 32, torch.float32, seed=0, device=DEV)
+    o, S = _gated_prefill(inp, chunk=16)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, with_init=False)
+    assert rel_l2(to64(o), o_ref) <= TOL_F32
+    assert rel_l2(to64(S), S_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 300, 3), (1, 5000, 2)])
+def test_gated_prefill_bf16(oracle_mod, B, T, H):
+    """Tensor-core path with the gate fused (the second case takes the
+    segment-split route)."""
+    inp = W.make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, seed=50 + T, device=DEV,
+                                init_state=True)
+    o, S = _gated_prefill(inp)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+    o2, S2, _, _ = gpu_prefill(inp)  # unfused: gate kernel + chunk kernel
+    assert rel_l2(to64(o), to64(o2)) <= 1e-2
+    assert rel_l2(to64(S), to64(S2)) <= 1e-3
+
+
+def test_gated_prefill_varlen(oracle_mod):
+    lens = [5, 0, 130, 64, 33]
+    cu_list = W.cu_seqlens_from_lengths(lens)
+    inp = W.make_prefill_inputs(1, cu_list[-1], 2, 128, 128, torch.bfloat16, seed=61,
+                                device=DEV, init_state=True, num_states=len(lens))
+    cu = torch.tensor(cu_list, dtype=torch.int32, device=DEV)
+    o, S = _gated_prefill(inp, cu=cu)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, cu=cu)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_BF16_S
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gated_decode(oracle_mod, dtype):
+    N, H, d, steps = 3, 4, 128, 5
+    S0 = W.make_decode_state(N, H, d, d, 70, DEV)
+    A_log = W.make_decode_gate_params(H, 71, DEV)
+    state = S0.clone()
+    xs, outs = [], []
+    for s in range(steps):
+        x = W.make_decode_step_inputs(N, H, d, d, dtype, 72 + s, DEV)
+        o = torch.full((N, H, d), float("nan"), device=DEV, dtype=dtype)
+        kda.kda_decode_step_gated(x["q"], x["k"], x["v"], x["z"], A_log, x["beta"], state, o)
+        xs.append(x)
+        outs.append(o)
+    torch.cuda.synchronize()
+    st = lambda n: torch.stack([x[n] for x in xs], dim=1)
+    g_ref = oracle_mod.gate(to64(st("z")), to64(A_log), -5.0)
+    o_ref, S_ref = oracle_mod.forward(to64(st("q")), to64(st("k")), to64(st("v")), g_ref,
+                                      to64(st("beta")), init_state=to64(S0))
+    tol_o, tol_s = (TOL_F32, TOL_F32) if dtype == torch.float32 else (TOL_BF16_O, TOL_BF16_S)
+    assert rel_l2(to64(torch.stack(outs, 1)), o_ref) <= tol_o
+    assert rel_l2(to64(state), S_ref) <= tol_s
