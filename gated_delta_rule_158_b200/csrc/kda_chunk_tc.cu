@@ -56,25 +56,26 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t SM_Q = 0;         // q tile  bf16 [32][128] row-major (TMA, no swizzle)
 constexpr uint32_t SM_K = 8192;      // k tile  bf16 [32][128]
 constexpr uint32_t SM_V = 16384;     // v tile  bf16, 2 x [32 rows x 128 B] swizzled (TMA)
-constexpr uint32_t SM_G = 24576;     // g tile  fp32 [32][128]
+constexpr uint32_t SM_G = 24576;     // g (or z) tile fp32 [32][128]
 constexpr uint32_t SM_R1 = 40960;    // 24 KB, two lives:
-constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128 (Gram A)
+constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128: Gram A, and
+                                              //  (rows 0-31) the MN-major A of W' = T K_L
 constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
 constexpr uint32_t SM_WF = SM_R1;             //  W                fp32 32 x 128 (tf32 B)
-constexpr uint32_t SM_AKK = SM_R1 + 16384;    //  A_kk fp32 32 x 32 (row-xor swizzled)
+constexpr uint32_t SM_AKKT = SM_R1 + 16384;   //  A_kk^T fp32 [s][r] 32 x 32 (inverse input)
 constexpr uint32_t SM_AQK = SM_R1 + 20480;    //  A_qk fp32 32 x 32 (tf32 B)
-constexpr uint32_t SM_KA = 65536;    // k e^G        bf16 [s][i] (MN-major A of W)
-constexpr uint32_t SM_TT = 73728;    // T            bf16 [r][s] (B of W and U~); cumsum partials during prep
-constexpr uint32_t SM_QG = 77824;    // q e^G        fp32 [r][i] (tf32 B of O)
-constexpr uint32_t SM_KC = 94208;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
-constexpr uint32_t SM_MISC = 110592;
+constexpr uint32_t SM_TT = 65536;    // T            bf16 [r][s] (B of W' and U~); cumsum partials during prep
+constexpr uint32_t SM_QG = 69632;    // q e^G        fp32 [r][i] (tf32 B of O)
+constexpr uint32_t SM_KC = 86016;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
+constexpr uint32_t SM_MISC = 102400;
 constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
-constexpr uint32_t SM_BETA = SM_MISC + 512;    // beta         fp32 [32]
-constexpr uint32_t SM_BAR = SM_MISC + 640;     // 3 mbarriers
-constexpr uint32_t SM_TMEM = SM_MISC + 672;    // TMEM base address
-constexpr uint32_t SM_ABORT = SM_MISC + 676;   // abort flag
-constexpr uint32_t SMEM_BYTES = SM_MISC + 1024;
-constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024 + 2048;  // align the base; slack
+constexpr uint32_t SM_E15 = SM_MISC + 512;     // e^{Gamma_15} fp32 [128]
+constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta         fp32 [32]
+constexpr uint32_t SM_BAR = SM_MISC + 1152;    // 3 mbarriers
+constexpr uint32_t SM_TMEM = SM_MISC + 1184;   // TMEM base address
+constexpr uint32_t SM_ABORT = SM_MISC + 1188;  // abort flag
+constexpr uint32_t SMEM_BYTES = SM_MISC + 2048;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to 1024
 
 constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
 constexpr uint32_t TX_V = 8192;
@@ -246,18 +247,32 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
   const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
 
+  // prep thread mapping: channels c0, c0+1 and rows 8rq .. 8rq+7 (so row & 7 = rr)
+  const int p = tid & 63, rq = tid >> 6, c0 = 2 * p;
+  // per-thread byte offsets of (row 8rq, channel c0) in each swizzled operand;
+  // the row-dependent part is + rr*128 and the swizzle chunk ^ rr
+  const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;   // bf16 tiles
+  const uint32_t ck32 = ((c0 & 31) * 4) >> 4, lo32 = ((c0 & 31) * 4) & 15;   // fp32 tiles
+  const uint32_t o_kql = (c0 >> 6) * 8192 + rq * 1024 + lo16;
+  const uint32_t o_kb = (c0 >> 6) * 4096 + rq * 1024 + lo16;
+  const uint32_t o_qg = (c0 >> 5) * 4096 + rq * 1024 + lo32;
+
+  float beta_next = 0.f;  // beta of the next chunk, prefetched one chunk ahead
+  if (tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
+
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = (int64_t)c * C;
     const int n = (int)((U.len - t0) < C ? (U.len - t0) : C);
-    if (tid < C) betas[tid] = tid < n ? P.beta[(size_t)(U.row0 + t0 + tid) * H + h] : 0.f;
+    if (tid < C) {
+      betas[tid] = beta_next;
+      const int64_t t1 = t0 + C + tid;
+      beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
+    }
 
     // ================================================= prep (all 256 threads)
     mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
     ph_in ^= 1;
     if (tid == 0) pend_in = false;
-    const int p = tid & 63;        // channel pair 2p, 2p+1
-    const int rq = tid >> 6;       // rows 8rq .. 8rq+7
-    const int c0 = 2 * p;
     float2 G[8];
     {
       float2 acc = make_float2(0.f, 0.f);
@@ -280,21 +295,20 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     if (*abort_flag) break;
     {
       const float2* tot = reinterpret_cast<const float2*>(sm + SM_TT);
-      float2 off = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float2 t = tot[q4 * 64 + p];
-        if (q4 < rq) { off.x += t.x; off.y += t.y; }
-      }
       const float2 t0v = tot[p], t1v = tot[64 + p], t2v = tot[128 + p], t3v = tot[192 + p];
+      float2 off = make_float2(0.f, 0.f);
+      if (rq > 0) { off.x += t0v.x; off.y += t0v.y; }
+      if (rq > 1) { off.x += t1v.x; off.y += t1v.y; }
+      if (rq > 2) { off.x += t2v.x; off.y += t2v.y; }
       const float2 g15 = make_float2(t0v.x + t1v.x, t0v.y + t1v.y);  // Gamma at row 15
       const float2 g31 = make_float2(g15.x + t2v.x + t3v.x, g15.y + t2v.y + t3v.y);
       const float2 e15 = make_float2(__expf(g15.x), __expf(g15.y));
       const float2 e3115 = make_float2(__expf(g31.x - g15.x), __expf(g31.y - g15.y));
       if (rq == 3) {
-        gamc[c0] = __expf(g31.x);
-        gamc[c0 + 1] = __expf(g31.y);
+        *reinterpret_cast<float2*>(gamc + c0) = make_float2(__expf(g31.x), __expf(g31.y));
+        *reinterpret_cast<float2*>(sm + SM_E15 + c0 * 4) = e15;
       }
+      float kcx[8], kcy[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
         const int r = 8 * rq + rr;
@@ -308,25 +322,32 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
         float kx = __low2float(kk), ky = __high2float(kk);
         float qx = __low2float(qq), qy = __high2float(qq);
         if (r >= n) { kx = ky = qx = qy = 0.f; }
-        const float gamx = ex * e15.x, gamy = ey * e15.y;
-        const float kcx = e3115.x * ix, kcy = e3115.y * iy;
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + sw128_off(64, r, c0, 2)) =
+        const uint32_t rb = rr * 128;
+        const uint32_t s16 = ((ck16 ^ rr) << 4), s32 = ((ck32 ^ rr) << 4);
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + rb + s16) =
             __floats2bfloat162_rn(kx * ex, ky * ey);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + sw128_off(64, 32 + r, c0, 2)) =
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
             __floats2bfloat162_rn(qx * ex, qy * ey);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + sw128_off(32, r, c0, 2)) =
+        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + o_kb + rb + s16) =
             __floats2bfloat162_rn(kx * ix, ky * iy);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KA + sw128_off(32, r, c0, 2)) =
-            __floats2bfloat162_rn(kx * gamx, ky * gamy);
-        *reinterpret_cast<float2*>(sm + SM_QG + sw128_off(32, r, c0, 4)) =
-            make_float2(qx * gamx, qy * gamy);
-        // Kc^T [i][s]: K-major tf32 B of the state update (tf32 MMAs take
-        // no MN-major B operand, so the transpose is written here)
-        *reinterpret_cast<float*>(sm + SM_KC + sw128_off(128, c0, r, 4)) = kx * kcx;
-        *reinterpret_cast<float*>(sm + SM_KC + sw128_off(128, c0 + 1, r, 4)) = ky * kcy;
+        *reinterpret_cast<float2*>(sm + SM_QG + o_qg + rb + s32) =
+            make_float2(qx * (ex * e15.x), qy * (ey * e15.y));
+        kcx[rr] = kx * (e3115.x * ix);
+        kcy[rr] = ky * (e3115.y * iy);
+      }
+      // Kc^T rows c0, c0+1; this thread's 8 rows are two 16-byte chunks of each
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t chx = (uint32_t)(2 * rq + hh) ^ (uint32_t)(c0 & 7);
+        const uint32_t chy = (uint32_t)(2 * rq + hh) ^ (uint32_t)((c0 + 1) & 7);
+        *reinterpret_cast<float4*>(sm + SM_KC + c0 * 128 + (chx << 4)) =
+            make_float4(kcx[4 * hh], kcx[4 * hh + 1], kcx[4 * hh + 2], kcx[4 * hh + 3]);
+        *reinterpret_cast<float4*>(sm + SM_KC + (c0 + 1) * 128 + (chy << 4)) =
+            make_float4(kcy[4 * hh], kcy[4 * hh + 1], kcy[4 * hh + 2], kcy[4 * hh + 3]);
       }
     }
     fence_proxy_async();
+    fence_before_sync();
     __syncthreads();
     if (*abort_flag) break;
 
@@ -355,11 +376,11 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       wait_ld();
       if (lane < 16) {
         const int r = 16 * (warp & 1) + lane;
-        if (warp < 2) {  // A_kk row r = beta_r * strict_lower(L)[r, :]
+        if (warp < 2) {  // A_kk[r][s] = beta_r L[r][s] (s < r), stored transposed [s][r]
           const float br = betas[r];
-          float* akk = reinterpret_cast<float*>(sm + SM_AKK);
+          float* akkt = reinterpret_cast<float*>(sm + SM_AKKT);
 #pragma unroll
-          for (int s = 0; s < 32; ++s) akk[r * 32 + (s ^ r)] = s < r ? br * v[s] : 0.f;
+          for (int s2 = 0; s2 < 32; ++s2) akkt[s2 * 32 + r] = s2 < r ? br * v[s2] : 0.f;
         } else {         // A_qk row r = lower_incl(Lq)[r, :]
 #pragma unroll
           for (int s4 = 0; s4 < 8; ++s4) {
@@ -368,7 +389,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
             w4.y = (4 * s4 + 1 <= r) ? v[4 * s4 + 1] : 0.f;
             w4.z = (4 * s4 + 2 <= r) ? v[4 * s4 + 2] : 0.f;
             w4.w = (4 * s4 + 3 <= r) ? v[4 * s4 + 3] : 0.f;
-            *reinterpret_cast<float4*>(sm + SM_AQK + sw128_off(32, r, 4 * s4, 4)) = w4;
+            *reinterpret_cast<float4*>(sm + SM_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
           }
         }
       }
@@ -378,38 +399,36 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ============================ T = (I + A_kk)^-1 Diag(beta), one column per lane
+    // ===== T = (I + A_kk)^-1 Diag(beta): lane = column, right-looking elimination
     if (warp == 0) {
-      const int cidx = lane;
-      const float* akk = reinterpret_cast<const float*>(sm + SM_AKK);
+      const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
       float x[32];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        float arow[32];
+      for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 t4 = reinterpret_cast<const float4*>(akk + r * 32)[q4];
-          arow[4 * q4 + 0] = t4.x;
-          arow[4 * q4 + 1] = t4.y;
-          arow[4 * q4 + 2] = t4.z;
-          arow[4 * q4 + 3] = t4.w;
+      for (int s2 = 0; s2 < 31; ++s2) {
+        const float xs = x[s2];  // final
+#pragma unroll
+        for (int r4 = (s2 + 1) / 4; r4 < 8; ++r4) {
+          const float4 a4 = reinterpret_cast<const float4*>(akkt + s2 * 32)[r4];
+          if (4 * r4 + 0 > s2) x[4 * r4 + 0] = fmaf(-a4.x, xs, x[4 * r4 + 0]);
+          if (4 * r4 + 1 > s2) x[4 * r4 + 1] = fmaf(-a4.y, xs, x[4 * r4 + 1]);
+          if (4 * r4 + 2 > s2) x[4 * r4 + 2] = fmaf(-a4.z, xs, x[4 * r4 + 2]);
+          if (4 * r4 + 3 > s2) x[4 * r4 + 3] = fmaf(-a4.w, xs, x[4 * r4 + 3]);
         }
-        float acc = (r == cidx) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < r; ++s) acc = fmaf(-arow[s ^ r], x[s], acc);
-        x[r] = acc;
       }
-      const float bc = betas[cidx];
+      const float bc = betas[lane];
+      const uint32_t ckl = (uint32_t)(lane * 2) >> 4, lol = (uint32_t)(lane * 2) & 15;
 #pragma unroll
       for (int r = 0; r < 32; ++r)
-        *reinterpret_cast<__nv_bfloat16*>(sm + SM_TT + sw128_off(32, r, cidx, 2)) =
+        *reinterpret_cast<__nv_bfloat16*>(sm + SM_TT + r * 128 + (((ckl ^ (r & 7)) << 4) | lol)) =
             __float2bfloat16_rn(x[r] * bc);
     }
     fence_proxy_async();
     __syncthreads();
     if (*abort_flag) break;
 
-    // ============== W^T = Ka^T T^T, U~^T = V^T T^T (bf16); O^T = S^T Qg^T (tf32)
+    // ====== W'^T = K_L^T T^T, U~^T = V^T T^T (bf16); O^T = S^T Qg^T (tf32)
     if (tid == 0) {
       if (!U.vzero) {
         mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
@@ -420,7 +439,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         const uint64_t b = sw128_desc(sb + SM_TT + ks * 32, 16, 1024);
-        mma_ss(tbase + W_COL, sw128_desc(sb + SM_KA + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
+        mma_ss(tbase + W_COL, sw128_desc(sb + SM_KQL + ks * 2048, 8192, 1024), b, id_w, 0,
+               ks > 0);
         if (!U.vzero)
           mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
       }
@@ -436,14 +456,18 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 4);
     ph_mma ^= 1;
     fence_after_sync();
-    if (warp < 4) {  // W^T (lane i, column r) -> W[r][i] fp32, tf32 B operand
+    if (warp < 4) {  // W = W' Diag(e^{Gamma_15}): lane i, column r -> W[r][i] fp32
       const int i = 32 * warp + lane;
+      const float e15i = reinterpret_cast<const float*>(sm + SM_E15)[i];
       float v[32];
       tmem_ld32(tbase + lane_base + W_COL, v);
       wait_ld();
+      const uint32_t base = (uint32_t)(i >> 5) * 4096 + (uint32_t)((i & 31) * 4 & 15);
+      const uint32_t ck = (uint32_t)((i & 31) * 4) >> 4;
 #pragma unroll
       for (int r = 0; r < 32; ++r)
-        *reinterpret_cast<float*>(sm + SM_WF + sw128_off(32, r, i, 4)) = v[r];
+        *reinterpret_cast<float*>(sm + SM_WF + base + r * 128 + ((ck ^ (r & 7)) << 4)) =
+            v[r] * e15i;
     }
     fence_proxy_async();
     fence_before_sync();
@@ -471,11 +495,18 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const uint32_t col = S_COL + 64 * half + 32 * cc;
+        const float4* g4 = reinterpret_cast<const float4*>(gamc + 64 * half + 32 * cc);
         float v[32];
         tmem_ld32(tbase + lane_base + col, v);
         wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] *= gamc[64 * half + 32 * cc + k];
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 gg = g4[k4];
+          v[4 * k4 + 0] *= gg.x;
+          v[4 * k4 + 1] *= gg.y;
+          v[4 * k4 + 2] *= gg.z;
+          v[4 * k4 + 3] *= gg.w;
+        }
         tmem_st32(tbase + lane_base + col, v);
       }
       wait_st();
@@ -504,20 +535,32 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
     ph_mma ^= 1;
     fence_after_sync();
-    if (U.out_on && warp < 4) {  // O^T (lane j, column r) -> o[row0 + t0 + r, h, j]
+    if (U.out_on && warp < 4) {
+      // O^T (lane j, column r) -> o[row0 + t0 + r, h, j]; lanes j, j^1 swap
+      // values so each writes a bf16 pair: even lane rows 2m, odd lane 2m+1
       const int j = 32 * warp + lane;
+      const bool odd = lane & 1;
       float v[32];
       tmem_ld32(tbase + lane_base + O_COL, v);
       wait_ld();
-      __nv_bfloat16* orow = P.out + ((size_t)(U.row0 + t0) * H + h) * D + j;
+      const int jp = j & ~1;
+      __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + t0) * H + h) * D + jp;
 #pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (r < n) orow[(size_t)r * H * D] = __float2bfloat16_rn(P.scale * v[r]);
+      for (int m = 0; m < 16; ++m) {
+        const float send = odd ? v[2 * m] : v[2 * m + 1];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+        const int r = 2 * m + (odd ? 1 : 0);
+        const float lo = odd ? recv : v[2 * m];        // column jp
+        const float hi = odd ? v[2 * m + 1] : recv;    // column jp + 1
+        if (r < n)
+          *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
+              __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
+      }
     }
+    // the O^T reads complete before the next chunk's O MMA (after its barriers)
     fence_before_sync();
-    __syncthreads();
-    if (*abort_flag) break;
   }
+  __syncthreads();
 
   // ---- final state (S^T lane j, column i -> final[i][j])
   if (U.final_state && !*abort_flag) {
