@@ -42,6 +42,8 @@ _SIGNATURES = {
     "kda_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _I, _I, _I, _I, _F, _VP, _VP]),
     "kda_decode_step_gated": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _I, _I, _I, _I, _F,
                                    _VP, _VP]),
+    "kda_chunk_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
+                                   _F, _I, _VP, _VP, _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
@@ -132,6 +134,19 @@ def kda_chunk_fwd(q, k, v, g, beta, out, workspace, init_state=None, cu_seqlens=
         _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale), int(chunk_size), _ptr(out),
         _ptr(final_state), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)), "kda_chunk_fwd")
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, out, init_state=None, cu_seqlens=None,
+                          final_state=None, scale=1.0, chunk_size=0, stream=None):
+    """kda_chunk_fwd using the library's built-in scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/kda.h)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib().kda_chunk_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q), _ptr(init_state),
+        _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale), int(chunk_size), _ptr(out),
+        _ptr(final_state), _stream(stream)), "kda_chunk_fwd_noalloc")
 
 
 def kda_chunk_fwd_gated(q, k, v, z, A_log, beta, out, workspace, g_min=-5.0, init_state=None,

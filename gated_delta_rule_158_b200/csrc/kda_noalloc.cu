@@ -1,0 +1,70 @@
+// kda_noalloc.cu -- kda_chunk_fwd for callers that cannot allocate device memory.
+//
+// Some callers of libkda have no way to hand it a workspace: an inference
+// engine plugin that may only use the memory its host engine planned before
+// serving starts, a service whose allocator is locked after warm-up so that
+// latency never depends on cudaMalloc or on fragmentation, or a caller with a
+// fixed device-memory budget fixed at start-up.  kda_chunk_fwd_noalloc gives
+// them the chunkwise forward without any allocation: its scratch (device
+// status word, varlen processing order, long-sequence segment states) is a
+// file-scope __device__ array compiled into the library, and it otherwise
+// runs exactly the kda_chunk_fwd path.
+//
+// Costs and rules of that choice:
+//  - every GPU on which the library's module is loaded holds the array
+//    (KDA_NOALLOC_SCRATCH_BYTES) until the process exits;
+//  - all calls share the one array: calls whose GPU work overlaps (other
+//    streams, other host threads) race on it and must be serialised by the
+//    caller; each call clears the status word it needs to start at zero;
+//  - problems whose scratch would exceed the array are rejected on the host
+//    with KDA_ERR_WORKSPACE before anything is enqueued;
+//  - the device address of the array is looked up (cudaGetSymbolAddress) on
+//    the first call made on each device, with that device current; make that
+//    first call before any stream capture begins.
+#include <mutex>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device
+// memory; the device address is looked up once per device and cached.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                            const float* g, const float* beta,
+                                            kda_dtype in_dtype, const float* init_state,
+                                            const int32_t* cu_seqlens, int num_seqs, int B,
+                                            int T, int H, int dk, int dv, float scale,
+                                            int chunk_size, void* out, float* final_state,
+                                            void* stream) {
+  void* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  // kda_chunk_fwd checks every argument and returns KDA_ERR_WORKSPACE, with
+  // nothing enqueued, when the problem needs more scratch than the array holds.
+  return kda_chunk_fwd(q, k, v, g, beta, in_dtype, init_state, cu_seqlens, num_seqs, B, T, H,
+                       dk, dv, scale, chunk_size, out, final_state, scratch,
+                       (size_t)KDA_NOALLOC_SCRATCH_BYTES, stream);
+}

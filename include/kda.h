@@ -192,6 +192,37 @@ KDA_API kda_status kda_get_device_status(const void *workspace, void *stream,
 KDA_API kda_status kda_selftest_bounded_wait(void *workspace, int64_t spin_limit_ns,
                                      void *stream);
 
+/*
+ * kda_chunk_fwd without a workspace, for callers that cannot allocate device
+ * memory (an engine plugin limited to memory its host planned up front, a
+ * service whose allocator is frozen after warm-up, a fixed device-memory
+ * budget).  The pages have no counterpart: this is a library convenience.
+ *
+ * Arguments, results and host-side errors are those of kda_chunk_fwd minus
+ * the workspace.  Its scratch is a __device__ array of
+ * KDA_NOALLOC_SCRATCH_BYTES compiled into the library, held on every GPU
+ * that loads the library until the process exits; a problem whose scratch
+ * would not fit (for instance a very long sequence with few heads, which
+ * the segment split needs room for) returns KDA_ERR_WORKSPACE with nothing
+ * enqueued.  All calls share that array, so calls whose GPU work overlaps
+ * race and must be serialised by the caller.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current: make it before any stream capture.  Device-side status
+ * (KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT) is recorded in the built-in array
+ * and is not reachable through kda_get_device_status; validate cu_seqlens on
+ * the host when using this entry point.  Returns KDA_ERR_CUDA if no device
+ * is current.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 kda_dtype in_dtype, const float *init_state,
+                                 const int32_t *cu_seqlens, int num_seqs, int B,
+                                 int T, int H, int dk, int dv, float scale,
+                                 int chunk_size, void *out, float *final_state,
+                                 void *stream);
+
 #ifdef __cplusplus
 }
 #endif
