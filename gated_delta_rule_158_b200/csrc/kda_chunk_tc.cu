@@ -63,11 +63,12 @@ constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128
 constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
 constexpr uint32_t SM_WF = SM_R1;             //  W                fp32 32 x 128 (tf32 B)
 constexpr uint32_t SM_AKKT = SM_R1 + 16384;   //  A_kk^T fp32 [s][r] 32 x 32 (inverse input)
-constexpr uint32_t SM_AQK = SM_R1 + 20480;    //  A_qk fp32 32 x 32 (tf32 B)
+constexpr uint32_t SM_XS = SM_R1 + 20480;     //  inverse blocks X00, X11 and A10 X00, fp32 32 x 32
 constexpr uint32_t SM_TT = 65536;    // T            bf16 [r][s] (B of W' and U~); cumsum partials during prep
 constexpr uint32_t SM_QG = 69632;    // q e^G        fp32 [r][i] (tf32 B of O)
 constexpr uint32_t SM_KC = 86016;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
-constexpr uint32_t SM_MISC = 102400;
+constexpr uint32_t SM_AQK = 102400;  // A_qk         fp32 [r][s] 32 x 32 (tf32 B of O)
+constexpr uint32_t SM_MISC = 106496;
 constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
 constexpr uint32_t SM_E15 = SM_MISC + 512;     // e^{Gamma_15} fp32 [128]
 constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta         fp32 [32]
@@ -256,107 +257,53 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const uint32_t o_kql = (c0 >> 6) * 8192 + rq * 1024 + lo16;
   const uint32_t o_kb = (c0 >> 6) * 4096 + rq * 1024 + lo16;
   const uint32_t o_qg = (c0 >> 5) * 4096 + rq * 1024 + lo32;
+  auto chunk_rows = [&](int cc) -> int {
+    const int64_t rem = U.len - (int64_t)cc * C;
+    return (int)(rem < C ? rem : C);
+  };
 
-  float beta_next = 0.f;  // beta of the next chunk, prefetched one chunk ahead
-  if (tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
+  float beta_next = 0.f;  // beta of the chunk after the one being prepared
+  float2 G[8];            // in-chunk cumulative log-decay of the chunk being prepared
+  float kcx[8], kcy[8];   // its Kc values, stored once the previous state update is done
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int64_t t0 = (int64_t)c * C;
-    const int n = (int)((U.len - t0) < C ? (U.len - t0) : C);
-    if (tid < C) {
-      betas[tid] = beta_next;
-      const int64_t t1 = t0 + C + tid;
-      beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
-    }
+  // ---- prep, part 1: wait for the chunk's tiles, beta, cumulative sums of g
 
-    // ================================================= prep (all 256 threads)
-    mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
-    ph_in ^= 1;
-    if (tid == 0) pend_in = false;
-    float2 G[8];
-    {
-      float2 acc = make_float2(0.f, 0.f);
+  // ---- prep, part 2 (after a barrier): rescaled operands of the chunk
+
+  // ---- Kc^T rows c0, c0+1: this thread's 8 rows are two 16-byte chunks of each
+
+  // ---- O^T of chunk cc (lane j, column r) -> o rows; lanes j, j^1 swap values so
+  //      each writes a bf16 pair (even lane rows 2m, odd lane rows 2m+1).  Warps 4-7.
+  auto export_o = [&](int cc) {
+    const int n = chunk_rows(cc);
+    const int j = 32 * (warp & 3) + lane;
+    const bool odd = lane & 1;
+    float v[32];
+    tmem_ld32(tbase + lane_base + O_COL, v);
+    wait_ld();
+    const int jp = j & ~1;
+    __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + (int64_t)cc * C) * H + h) * D + jp;
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * rq + rr;
-        float2 gv = *reinterpret_cast<const float2*>(sm + SM_G + (r * D + c0) * 4);
-        if (P.A_log) {  // fused gate: the tile holds z; g = g_min sigmoid(e^A z)
-          gv.x = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.x));
-          gv.y = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.y));
-        }
-        if (r >= n) gv = make_float2(0.f, 0.f);
-        acc.x += gv.x;
-        acc.y += gv.y;
-        G[rr] = acc;
-      }
-      reinterpret_cast<float2*>(sm + SM_TT)[rq * 64 + p] = acc;  // quarter totals
+    for (int m = 0; m < 16; ++m) {
+      const float send = odd ? v[2 * m] : v[2 * m + 1];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      const int r = 2 * m + (odd ? 1 : 0);
+      const float lo = odd ? recv : v[2 * m];      // column jp
+      const float hi = odd ? v[2 * m + 1] : recv;  // column jp + 1
+      if (r < n)
+        *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
+            __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
     }
-    __syncthreads();
-    if (*abort_flag) break;
-    {
-      const float2* tot = reinterpret_cast<const float2*>(sm + SM_TT);
-      const float2 t0v = tot[p], t1v = tot[64 + p], t2v = tot[128 + p], t3v = tot[192 + p];
-      float2 off = make_float2(0.f, 0.f);
-      if (rq > 0) { off.x += t0v.x; off.y += t0v.y; }
-      if (rq > 1) { off.x += t1v.x; off.y += t1v.y; }
-      if (rq > 2) { off.x += t2v.x; off.y += t2v.y; }
-      const float2 g15 = make_float2(t0v.x + t1v.x, t0v.y + t1v.y);  // Gamma at row 15
-      const float2 g31 = make_float2(g15.x + t2v.x + t3v.x, g15.y + t2v.y + t3v.y);
-      const float2 e15 = make_float2(__expf(g15.x), __expf(g15.y));
-      const float2 e3115 = make_float2(__expf(g31.x - g15.x), __expf(g31.y - g15.y));
-      if (rq == 3) {
-        *reinterpret_cast<float2*>(gamc + c0) = make_float2(__expf(g31.x), __expf(g31.y));
-        *reinterpret_cast<float2*>(sm + SM_E15 + c0 * 4) = e15;
-      }
-      float kcx[8], kcy[8];
-#pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * rq + rr;
-        const float gx = G[rr].x + off.x, gy = G[rr].y + off.y;
-        const float ex = __expf(gx - g15.x), ey = __expf(gy - g15.y);
-        const float ix = __expf(g15.x - gx), iy = __expf(g15.y - gy);
-        const __nv_bfloat162 kk =
-            *reinterpret_cast<const __nv_bfloat162*>(sm + SM_K + (r * D + c0) * 2);
-        const __nv_bfloat162 qq =
-            *reinterpret_cast<const __nv_bfloat162*>(sm + SM_Q + (r * D + c0) * 2);
-        float kx = __low2float(kk), ky = __high2float(kk);
-        float qx = __low2float(qq), qy = __high2float(qq);
-        if (r >= n) { kx = ky = qx = qy = 0.f; }
-        const uint32_t rb = rr * 128;
-        const uint32_t s16 = ((ck16 ^ rr) << 4), s32 = ((ck32 ^ rr) << 4);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + rb + s16) =
-            __floats2bfloat162_rn(kx * ex, ky * ey);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
-            __floats2bfloat162_rn(qx * ex, qy * ey);
-        *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + o_kb + rb + s16) =
-            __floats2bfloat162_rn(kx * ix, ky * iy);
-        *reinterpret_cast<float2*>(sm + SM_QG + o_qg + rb + s32) =
-            make_float2(qx * (ex * e15.x), qy * (ey * e15.y));
-        kcx[rr] = kx * (e3115.x * ix);
-        kcy[rr] = ky * (e3115.y * iy);
-      }
-      // Kc^T rows c0, c0+1; this thread's 8 rows are two 16-byte chunks of each
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t chx = (uint32_t)(2 * rq + hh) ^ (uint32_t)(c0 & 7);
-        const uint32_t chy = (uint32_t)(2 * rq + hh) ^ (uint32_t)((c0 + 1) & 7);
-        *reinterpret_cast<float4*>(sm + SM_KC + c0 * 128 + (chx << 4)) =
-            make_float4(kcx[4 * hh], kcx[4 * hh + 1], kcx[4 * hh + 2], kcx[4 * hh + 3]);
-        *reinterpret_cast<float4*>(sm + SM_KC + (c0 + 1) * 128 + (chy << 4)) =
-            make_float4(kcy[4 * hh], kcy[4 * hh + 1], kcy[4 * hh + 2], kcy[4 * hh + 3]);
-      }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (*abort_flag) break;
+  };
 
-    // ============================================== Gram GEMM (M64 N32 K128)
+  // the loop starts at c = -1: that pass only prepares chunk 0's operands
+  if (nchunks > 0 && tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
+  for (int c = -1; c < nchunks && !*abort_flag; ++c) {
+    const bool has_next = c + 1 < nchunks;
+    if (c >= 0) {
+
+    // ===== A: Gram GEMM (M64 N32 K128) of chunk c; warps 4-7 export O of chunk c-1
     if (tid == 0) {
-      if (c + 1 < nchunks) {
-        fence_proxy_async();
-        issue_qkg(c + 1);
-      }
       fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
@@ -367,21 +314,24 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       }
       mma_commit(bar_mma);
     }
+    if (c > 0 && U.out_on && warp >= 4) export_o(c - 1);
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 2);
     ph_mma ^= 1;
     fence_after_sync();
+
+    // ===== B: A_kk (transposed, x beta) and A_qk from the Gram accumulator
     if (warp < 4) {
       float v[32];
       tmem_ld32(tbase + lane_base + G_COL, v);
       wait_ld();
       if (lane < 16) {
         const int r = 16 * (warp & 1) + lane;
-        if (warp < 2) {  // A_kk[r][s] = beta_r L[r][s] (s < r), stored transposed [s][r]
+        if (warp < 2) {
           const float br = betas[r];
           float* akkt = reinterpret_cast<float*>(sm + SM_AKKT);
 #pragma unroll
           for (int s2 = 0; s2 < 32; ++s2) akkt[s2 * 32 + r] = s2 < r ? br * v[s2] : 0.f;
-        } else {         // A_qk row r = lower_incl(Lq)[r, :]
+        } else {
 #pragma unroll
           for (int s4 = 0; s4 < 8; ++s4) {
             float4 w4;
@@ -399,36 +349,70 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ===== T = (I + A_kk)^-1 Diag(beta): lane = column, right-looking elimination
-    if (warp == 0) {
+    // ===== C: T = (I + A_kk)^-1 Diag(beta), blocked 2 x 2 over 16-row blocks
+    if (warp < 4) {
       const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
-      float x[32];
+      float* xs = reinterpret_cast<float*>(sm + SM_XS);
+      auto tt_store = [&](int r, int col, float val) {
+        *reinterpret_cast<__nv_bfloat16*>(
+            sm + SM_TT + r * 128 + ((((uint32_t)(col * 2) >> 4) ^ (uint32_t)(r & 7)) << 4) +
+            ((col * 2) & 15)) = __float2bfloat16_rn(val);
+      };
+      if (warp == 0) {  // diagonal blocks: lane = (block b, column cb)
+        const int b = lane >> 4, cb = lane & 15, o = 16 * b;
+        float x[16];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == cb) ? 1.f : 0.f;
 #pragma unroll
-      for (int s2 = 0; s2 < 31; ++s2) {
-        const float xs = x[s2];  // final
+        for (int s2 = 0; s2 < 15; ++s2) {
+          const float xv = x[s2];
+          const float* col = akkt + (o + s2) * 32 + o;  // A[o + r][o + s2], r = 0..15
 #pragma unroll
-        for (int r4 = (s2 + 1) / 4; r4 < 8; ++r4) {
-          const float4 a4 = reinterpret_cast<const float4*>(akkt + s2 * 32)[r4];
-          if (4 * r4 + 0 > s2) x[4 * r4 + 0] = fmaf(-a4.x, xs, x[4 * r4 + 0]);
-          if (4 * r4 + 1 > s2) x[4 * r4 + 1] = fmaf(-a4.y, xs, x[4 * r4 + 1]);
-          if (4 * r4 + 2 > s2) x[4 * r4 + 2] = fmaf(-a4.z, xs, x[4 * r4 + 2]);
-          if (4 * r4 + 3 > s2) x[4 * r4 + 3] = fmaf(-a4.w, xs, x[4 * r4 + 3]);
+          for (int r4 = (s2 + 1) / 4; r4 < 4; ++r4) {
+            const float4 a4 = reinterpret_cast<const float4*>(col)[r4];
+            if (4 * r4 + 0 > s2) x[4 * r4 + 0] = fmaf(-a4.x, xv, x[4 * r4 + 0]);
+            if (4 * r4 + 1 > s2) x[4 * r4 + 1] = fmaf(-a4.y, xv, x[4 * r4 + 1]);
+            if (4 * r4 + 2 > s2) x[4 * r4 + 2] = fmaf(-a4.z, xv, x[4 * r4 + 2]);
+            if (4 * r4 + 3 > s2) x[4 * r4 + 3] = fmaf(-a4.w, xv, x[4 * r4 + 3]);
+          }
+        }
+        const float bc = betas[o + cb];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          xs[(o + r) * 32 + o + cb] = x[r];
+          tt_store(o + r, o + cb, x[r] * bc);
+          if (b == 0) tt_store(r, 16 + cb, 0.f);  // upper-right block of T is zero
         }
       }
-      const float bc = betas[lane];
-      const uint32_t ckl = (uint32_t)(lane * 2) >> 4, lol = (uint32_t)(lane * 2) & 15;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // Y = A10 X00 (rows 16..31 x columns 0..15), into the lower-left block of xs
+      const int cl = tid & 15, rp = tid >> 4;  // tid < 128 here
 #pragma unroll
-      for (int r = 0; r < 32; ++r)
-        *reinterpret_cast<__nv_bfloat16*>(sm + SM_TT + r * 128 + (((ckl ^ (r & 7)) << 4) | lol)) =
-            __float2bfloat16_rn(x[r] * bc);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = 2 * rp + h2;
+        float y = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) y = fmaf(akkt[s2 * 32 + 16 + r], xs[s2 * 32 + cl], y);
+        xs[(16 + r) * 32 + cl] = y;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // X10 = -X11 Y;  T[16 + r][c] = X10[r][c] beta_c
+      const float bcl = betas[cl];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = 2 * rp + h2;
+        float x10 = 0.f;
+#pragma unroll
+        for (int t2 = 0; t2 < 16; ++t2)
+          x10 = fmaf(xs[(16 + r) * 32 + 16 + t2], xs[(16 + t2) * 32 + cl], x10);
+        tt_store(16 + r, cl, -x10 * bcl);
+      }
     }
     fence_proxy_async();
     __syncthreads();
     if (*abort_flag) break;
 
-    // ====== W'^T = K_L^T T^T, U~^T = V^T T^T (bf16); O^T = S^T Qg^T (tf32)
+    // ===== D: W'^T = K_L^T T^T and U~^T = V^T T^T (bf16)
     if (tid == 0) {
       if (!U.vzero) {
         mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
@@ -444,19 +428,14 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
         if (!U.vzero)
           mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
       }
-      if (U.out_on) {
-#pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {
-          const uint64_t b = sw128_desc(sb + SM_QG + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks, b, id_o, ks > 0);
-        }
-      }
       mma_commit(bar_mma);
     }
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 4);
     ph_mma ^= 1;
     fence_after_sync();
-    if (warp < 4) {  // W = W' Diag(e^{Gamma_15}): lane i, column r -> W[r][i] fp32
+
+    // ===== E: W = W' Diag(e^{Gamma_15}) -> smem (lane i, column r -> W[r][i] fp32)
+    if (warp < 4) {
       const int i = 32 * warp + lane;
       const float e15i = reinterpret_cast<const float*>(sm + SM_E15)[i];
       float v[32];
@@ -474,24 +453,62 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ======================================== U^T -= S^T W^T (tf32, A in TMEM)
-    if (tid == 0) {
-      if (c + 1 < nchunks && !U.vzero) {
+    }  // c >= 0
+
+    // ===== F: U^T -= S^T W^T and O^T = S^T Qg^T, interleaved (tf32, A = S^T in TMEM);
+    //          meanwhile part 1 of the next chunk's prep
+    if (tid == 0 && c >= 0) {
+      if (has_next && !U.vzero) {
         fence_proxy_async();
         issue_v(c + 1);
       }
       fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks) {
-        const uint64_t b = sw128_desc(sb + SM_WF + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-        mma_ts_tf32(tbase + U_COL, tbase + S_COL + 8 * ks, b, id_u, (ks > 0) || !U.vzero);
+        const uint32_t boff = (ks >> 2) * 4096 + (ks & 3) * 32;
+        mma_ts_tf32(tbase + U_COL, tbase + S_COL + 8 * ks, sw128_desc(sb + SM_WF + boff, 16, 1024),
+                    id_u, (ks > 0) || !U.vzero);
+        if (U.out_on)
+          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
+                      sw128_desc(sb + SM_QG + boff, 16, 1024), id_o, ks > 0);
       }
       mma_commit(bar_mma);
     }
+    if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g
+      const int cc = c + 1;
+    const int n = chunk_rows(cc);
+    if (tid < C) {
+      betas[tid] = beta_next;
+      const int64_t t1 = (int64_t)(cc + 1) * C + tid;
+      beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
+    }
+    mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
+    ph_in ^= 1;
+    if (tid == 0) pend_in = false;
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const int r = 8 * rq + rr;
+      float2 gv = *reinterpret_cast<const float2*>(sm + SM_G + (r * D + c0) * 4);
+      if (P.A_log) {  // fused gate: the tile holds z; g = g_min sigmoid(e^A z)
+        gv.x = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.x));
+        gv.y = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.y));
+      }
+      if (r >= n) gv = make_float2(0.f, 0.f);
+      acc.x += gv.x;
+      acc.y += gv.y;
+      G[rr] = acc;
+    }
+    reinterpret_cast<float2*>(sm + SM_TT)[rq * 64 + p] = acc;  // quarter totals
+    }
+    __syncthreads();
+    if (c >= 0) {
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 5);
     ph_mma ^= 1;
     fence_after_sync();
-    {  // decay the state: S^T[j][i] *= e^{Gamma_C, i}
+
+    // ===== G: decay the state, S^T[j][i] *= e^{Gamma_C, i}
+    {
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const uint32_t col = S_COL + 64 * half + 32 * cc;
@@ -515,51 +532,92 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ============ S^T += U^T Kc;  O^T += U^T A_qk^T   (tf32, U^T read from TMEM)
+    // ===== H: S^T += U^T Kc and O^T += U^T A_qk^T (tf32, U^T from TMEM);
+    //          meanwhile part 2 of the next chunk's prep
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t b = sw128_desc(sb + SM_KC + ks * 32, 16, 1024);
-        mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks, b, id_s, 1);
-      }
-      if (U.out_on) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t b = sw128_desc(sb + SM_AQK + ks * 32, 16, 1024);
-          mma_ts_tf32(tbase + O_COL, tbase + U_COL + 8 * ks, b, id_o, 1);
-        }
+        mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
+                    sw128_desc(sb + SM_KC + ks * 32, 16, 1024), id_s, 1);
+        if (U.out_on)
+          mma_ts_tf32(tbase + O_COL, tbase + U_COL + 8 * ks,
+                      sw128_desc(sb + SM_AQK + ks * 32, 16, 1024), id_o, 1);
       }
       mma_commit(bar_mma);
     }
-    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
-    ph_mma ^= 1;
-    fence_after_sync();
-    if (U.out_on && warp < 4) {
-      // O^T (lane j, column r) -> o[row0 + t0 + r, h, j]; lanes j, j^1 swap
-      // values so each writes a bf16 pair: even lane rows 2m, odd lane 2m+1
-      const int j = 32 * warp + lane;
-      const bool odd = lane & 1;
-      float v[32];
-      tmem_ld32(tbase + lane_base + O_COL, v);
-      wait_ld();
-      const int jp = j & ~1;
-      __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + t0) * H + h) * D + jp;
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const float send = odd ? v[2 * m] : v[2 * m + 1];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-        const int r = 2 * m + (odd ? 1 : 0);
-        const float lo = odd ? recv : v[2 * m];        // column jp
-        const float hi = odd ? v[2 * m + 1] : recv;    // column jp + 1
-        if (r < n)
-          *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
-              __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
-      }
+    }  // c >= 0
+    if (has_next) {  // prep, part 2: rescaled operands (Kc kept in registers)
+      const int cc = c + 1;
+    const int n = chunk_rows(cc);
+    const float2* tot = reinterpret_cast<const float2*>(sm + SM_TT);
+    const float2 t0v = tot[p], t1v = tot[64 + p], t2v = tot[128 + p], t3v = tot[192 + p];
+    float2 off = make_float2(0.f, 0.f);
+    if (rq > 0) { off.x += t0v.x; off.y += t0v.y; }
+    if (rq > 1) { off.x += t1v.x; off.y += t1v.y; }
+    if (rq > 2) { off.x += t2v.x; off.y += t2v.y; }
+    const float2 g15 = make_float2(t0v.x + t1v.x, t0v.y + t1v.y);  // Gamma at row 15
+    const float2 g31 = make_float2(g15.x + t2v.x + t3v.x, g15.y + t2v.y + t3v.y);
+    const float2 e15 = make_float2(__expf(g15.x), __expf(g15.y));
+    const float2 e3115 = make_float2(__expf(g31.x - g15.x), __expf(g31.y - g15.y));
+    if (rq == 3) {
+      *reinterpret_cast<float2*>(gamc + c0) = make_float2(__expf(g31.x), __expf(g31.y));
+      *reinterpret_cast<float2*>(sm + SM_E15 + c0 * 4) = e15;
     }
-    // the O^T reads complete before the next chunk's O MMA (after its barriers)
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      const int r = 8 * rq + rr;
+      const float gx = G[rr].x + off.x, gy = G[rr].y + off.y;
+      const float ex = __expf(gx - g15.x), ey = __expf(gy - g15.y);
+      const float ix = __expf(g15.x - gx), iy = __expf(g15.y - gy);
+      const __nv_bfloat162 kk =
+          *reinterpret_cast<const __nv_bfloat162*>(sm + SM_K + (r * D + c0) * 2);
+      const __nv_bfloat162 qq =
+          *reinterpret_cast<const __nv_bfloat162*>(sm + SM_Q + (r * D + c0) * 2);
+      float kx = __low2float(kk), ky = __high2float(kk);
+      float qx = __low2float(qq), qy = __high2float(qq);
+      if (r >= n) { kx = ky = qx = qy = 0.f; }
+      const uint32_t rb = rr * 128;
+      const uint32_t s16 = ((ck16 ^ rr) << 4), s32 = ((ck32 ^ rr) << 4);
+      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + rb + s16) =
+          __floats2bfloat162_rn(kx * ex, ky * ey);
+      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
+          __floats2bfloat162_rn(qx * ex, qy * ey);
+      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + o_kb + rb + s16) =
+          __floats2bfloat162_rn(kx * ix, ky * iy);
+      *reinterpret_cast<float2*>(sm + SM_QG + o_qg + rb + s32) =
+          make_float2(qx * (ex * e15.x), qy * (ey * e15.y));
+      kcx[rr] = kx * (e3115.x * ix);
+      kcy[rr] = ky * (e3115.y * iy);
+    }
+    }
+    if (c >= 0) {
+      mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
+      ph_mma ^= 1;
+      fence_after_sync();
+    }
+    if (has_next) {  // Kc^T rows c0, c0+1: this thread's 8 rows are two 16-byte chunks
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t chx = (uint32_t)(2 * rq + hh) ^ (uint32_t)(c0 & 7);
+      const uint32_t chy = (uint32_t)(2 * rq + hh) ^ (uint32_t)((c0 + 1) & 7);
+      *reinterpret_cast<float4*>(sm + SM_KC + c0 * 128 + (chx << 4)) =
+          make_float4(kcx[4 * hh], kcx[4 * hh + 1], kcx[4 * hh + 2], kcx[4 * hh + 3]);
+      *reinterpret_cast<float4*>(sm + SM_KC + (c0 + 1) * 128 + (chy << 4)) =
+          make_float4(kcy[4 * hh], kcy[4 * hh + 1], kcy[4 * hh + 2], kcy[4 * hh + 3]);
+    }
+    }
+    fence_proxy_async();
     fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && c + 2 < nchunks) {
+      fence_proxy_async();
+      issue_qkg(c + 2);
+    }
   }
+  __syncthreads();
+  if (nchunks > 0 && U.out_on && warp >= 4 && !*abort_flag) export_o(nchunks - 1);
+  fence_before_sync();
   __syncthreads();
 
   // ---- final state (S^T lane j, column i -> final[i][j])
