@@ -96,6 +96,23 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def extend_window(self, step, min_s=1.5):
+        """The timed region can be shorter than nvidia-smi's start-up and its
+        50 ms period: keep running the same (untimed) step until the sampling
+        window spans min_s seconds, then stop and summarise."""
+        t0 = time.time()
+        n = 0
+        while time.time() - t0 < min_s:
+            step()
+            n += 1
+            if n % 8 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        out = self.stop()
+        if out is not None:
+            out["window"] = f"timed region + {n} further untimed steps ({min_s:.1f} s)"
+        return out
+
     def stop(self):
         if self.proc is None:
             return None
@@ -411,7 +428,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
     step = PrefillStep(inp, cu, N)
     clocks = ClockSampler(dev.index)
     total_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
-    clk = clocks.stop()
+    clk = clocks.extend_window(step)
     st, _ = kda.kda_get_device_status(step.ws)
     if st != kda.KDA_OK:
         raise RuntimeError(f"device status {kda.kda_status_string(st)}")

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const int half = warp >> 2;                                   // column half (8-warp passes)
 
   const int nchunks = (int)((U.len + C - 1) / C);
-  const float a_h = P.A_log ? expf(P.A_log[h]) : 0.f;
+  const float a2 = P.A_log ? expf(P.A_log[h]) * 1.4426950408889634f : 0.f;
   bool pend_in = false, pend_v = false;  // thread 0: TMA loads issued, not yet waited
   auto issue_qkg = [&](int c) {
     const int row = (int)(U.row0 + (int64_t)c * C);
@@ -248,23 +248,25 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
   const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
 
-  // prep thread mapping: channels c0, c0+1 and rows 8rq .. 8rq+7 (so row & 7 = rr)
-  const int p = tid & 63, rq = tid >> 6, c0 = 2 * p;
-  // per-thread byte offsets of (row 8rq, channel c0) in each swizzled operand;
-  // the row-dependent part is + rr*128 and the swizzle chunk ^ rr
+  // prep thread mapping: channels c0 .. c0+3 and rows 4ro .. 4ro+3 (warp ro)
+  const int cq = tid & 31, ro = tid >> 5, c0 = 4 * cq;
+  // byte offsets of (row 4ro, channel c0) in each swizzled operand; a row
+  // 4ro + rr adds rr*128 and xors the 16-byte chunk index with (4ro + rr) & 7
   const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;   // bf16 tiles
-  const uint32_t ck32 = ((c0 & 31) * 4) >> 4, lo32 = ((c0 & 31) * 4) & 15;   // fp32 tiles
-  const uint32_t o_kql = (c0 >> 6) * 8192 + rq * 1024 + lo16;
-  const uint32_t o_kb = (c0 >> 6) * 4096 + rq * 1024 + lo16;
-  const uint32_t o_qg = (c0 >> 5) * 4096 + rq * 1024 + lo32;
+  const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                                 // fp32 tiles
+  const uint32_t o_kql = (c0 >> 6) * 8192 + ro * 512 + lo16;
+  const uint32_t o_kb = (c0 >> 6) * 4096 + ro * 512 + lo16;
+  const uint32_t o_qg = (c0 >> 5) * 4096 + ro * 512;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float gmin2 = P.g_min * kLog2e;
   auto chunk_rows = [&](int cc) -> int {
     const int64_t rem = U.len - (int64_t)cc * C;
     return (int)(rem < C ? rem : C);
   };
 
   float beta_next = 0.f;  // beta of the chunk after the one being prepared
-  float2 G[8];            // in-chunk cumulative log-decay of the chunk being prepared
-  float kcx[8], kcy[8];   // its Kc values, stored once the previous state update is done
+  float4 G4[4];           // in-chunk cumulative log2-decay of the chunk being prepared
+  float kc[4][4];         // its Kc values [channel][row], stored after the state update
 
   // ---- prep, part 1: wait for the chunk's tiles, beta, cumulative sums of g
 
@@ -474,32 +476,45 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       }
       mma_commit(bar_mma);
     }
-    if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g
+    if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g (log2 units)
       const int cc = c + 1;
-    const int n = chunk_rows(cc);
-    if (tid < C) {
-      betas[tid] = beta_next;
-      const int64_t t1 = (int64_t)(cc + 1) * C + tid;
-      beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
-    }
-    mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
-    ph_in ^= 1;
-    if (tid == 0) pend_in = false;
-    float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      const int r = 8 * rq + rr;
-      float2 gv = *reinterpret_cast<const float2*>(sm + SM_G + (r * D + c0) * 4);
-      if (P.A_log) {  // fused gate: the tile holds z; g = g_min sigmoid(e^A z)
-        gv.x = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.x));
-        gv.y = __fdividef(P.g_min, 1.f + __expf(-a_h * gv.y));
+      const int n = chunk_rows(cc);
+      if (tid < C) {
+        betas[tid] = beta_next;
+        const int64_t t1 = (int64_t)(cc + 1) * C + tid;
+        beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
       }
-      if (r >= n) gv = make_float2(0.f, 0.f);
-      acc.x += gv.x;
-      acc.y += gv.y;
-      G[rr] = acc;
-    }
-    reinterpret_cast<float2*>(sm + SM_TT)[rq * 64 + p] = acc;  // quarter totals
+      mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
+      ph_in ^= 1;
+      if (tid == 0) pend_in = false;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = 4 * ro + rr;
+        float4 gv = *reinterpret_cast<const float4*>(sm + SM_G + (r * D + c0) * 4);
+        if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
+          gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
+          gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
+          gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
+          gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
+        } else {
+          gv.x *= kLog2e;
+          gv.y *= kLog2e;
+          gv.z *= kLog2e;
+          gv.w *= kLog2e;
+        }
+        if (r >= n) {  // tail rows act as g = 0, k = q = 0
+          gv = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<uint2*>(sm + SM_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(sm + SM_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
+        }
+        acc.x += gv.x;
+        acc.y += gv.y;
+        acc.z += gv.z;
+        acc.w += gv.w;
+        G4[rr] = acc;
+      }
+      reinterpret_cast<float4*>(sm + SM_TT)[ro * 32 + cq] = acc;  // 4-row group totals
     }
     __syncthreads();
     if (c >= 0) {
@@ -548,64 +563,82 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     }
     }  // c >= 0
     if (has_next) {  // prep, part 2: rescaled operands (Kc kept in registers)
-      const int cc = c + 1;
-    const int n = chunk_rows(cc);
-    const float2* tot = reinterpret_cast<const float2*>(sm + SM_TT);
-    const float2 t0v = tot[p], t1v = tot[64 + p], t2v = tot[128 + p], t3v = tot[192 + p];
-    float2 off = make_float2(0.f, 0.f);
-    if (rq > 0) { off.x += t0v.x; off.y += t0v.y; }
-    if (rq > 1) { off.x += t1v.x; off.y += t1v.y; }
-    if (rq > 2) { off.x += t2v.x; off.y += t2v.y; }
-    const float2 g15 = make_float2(t0v.x + t1v.x, t0v.y + t1v.y);  // Gamma at row 15
-    const float2 g31 = make_float2(g15.x + t2v.x + t3v.x, g15.y + t2v.y + t3v.y);
-    const float2 e15 = make_float2(__expf(g15.x), __expf(g15.y));
-    const float2 e3115 = make_float2(__expf(g31.x - g15.x), __expf(g31.y - g15.y));
-    if (rq == 3) {
-      *reinterpret_cast<float2*>(gamc + c0) = make_float2(__expf(g31.x), __expf(g31.y));
-      *reinterpret_cast<float2*>(sm + SM_E15 + c0 * 4) = e15;
-    }
+      const float4* tot = reinterpret_cast<const float4*>(sm + SM_TT);
+      float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
 #pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      const int r = 8 * rq + rr;
-      const float gx = G[rr].x + off.x, gy = G[rr].y + off.y;
-      const float ex = __expf(gx - g15.x), ey = __expf(gy - g15.y);
-      const float ix = __expf(g15.x - gx), iy = __expf(g15.y - gy);
-      const __nv_bfloat162 kk =
-          *reinterpret_cast<const __nv_bfloat162*>(sm + SM_K + (r * D + c0) * 2);
-      const __nv_bfloat162 qq =
-          *reinterpret_cast<const __nv_bfloat162*>(sm + SM_Q + (r * D + c0) * 2);
-      float kx = __low2float(kk), ky = __high2float(kk);
-      float qx = __low2float(qq), qy = __high2float(qq);
-      if (r >= n) { kx = ky = qx = qy = 0.f; }
-      const uint32_t rb = rr * 128;
-      const uint32_t s16 = ((ck16 ^ rr) << 4), s32 = ((ck32 ^ rr) << 4);
-      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + rb + s16) =
-          __floats2bfloat162_rn(kx * ex, ky * ey);
-      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
-          __floats2bfloat162_rn(qx * ex, qy * ey);
-      *reinterpret_cast<__nv_bfloat162*>(sm + SM_KB + o_kb + rb + s16) =
-          __floats2bfloat162_rn(kx * ix, ky * iy);
-      *reinterpret_cast<float2*>(sm + SM_QG + o_qg + rb + s32) =
-          make_float2(qx * (ex * e15.x), qy * (ey * e15.y));
-      kcx[rr] = kx * (e3115.x * ix);
-      kcy[rr] = ky * (e3115.y * iy);
-    }
+      for (int o8 = 0; o8 < 8; ++o8) {
+        const float4 t = tot[o8 * 32 + cq];
+        if (o8 < ro) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
+        if (o8 < 4) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
+        g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
+      }
+      const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
+                                     ex2_approx(g15.w));
+      const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
+                                       ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
+      if (ro == 7) {
+        *reinterpret_cast<float4*>(gamc + c0) = make_float4(
+            ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
+        *reinterpret_cast<float4*>(sm + SM_E15 + c0 * 4) = e15;
+      }
+      // G4[rr] - g15 + off: exponent of e^{Gamma_r - Gamma_15} in log2 units
+      const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = 4 * ro + rr;
+        float ex[4], ix[4];
+        ex[0] = ex2_approx(G4[rr].x + sh.x);
+        ex[1] = ex2_approx(G4[rr].y + sh.y);
+        ex[2] = ex2_approx(G4[rr].z + sh.z);
+        ex[3] = ex2_approx(G4[rr].w + sh.w);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
+        const uint2 kw = *reinterpret_cast<const uint2*>(sm + SM_K + (r * D + c0) * 2);
+        const uint2 qw = *reinterpret_cast<const uint2*>(sm + SM_Q + (r * D + c0) * 2);
+        const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
+                             __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
+        const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
+                             __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
+        float kl[4], ql[4], kb[4];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          kl[k4] = kv[k4] * ex[k4];
+          ql[k4] = qv[k4] * ex[k4];
+          kb[k4] = kv[k4] * ix[k4];
+        }
+        const uint32_t rb = rr * 128;
+        const uint32_t sw = (uint32_t)((4 * ro + rr) & 7);
+        const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
+        auto pack = [](float lo, float hi) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+          return *reinterpret_cast<const uint32_t*>(&b2);
+        };
+        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + rb + s16) =
+            make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
+        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
+            make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
+        *reinterpret_cast<uint2*>(sm + SM_KB + o_kb + rb + s16) =
+            make_uint2(pack(kb[0], kb[1]), pack(kb[2], kb[3]));
+        *reinterpret_cast<float4*>(sm + SM_QG + o_qg + rb + s32) =
+            make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
+        kc[0][rr] = kb[0] * e3115.x;
+        kc[1][rr] = kb[1] * e3115.y;
+        kc[2][rr] = kb[2] * e3115.z;
+        kc[3][rr] = kb[3] * e3115.w;
+      }
     }
     if (c >= 0) {
       mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
       ph_mma ^= 1;
       fence_after_sync();
     }
-    if (has_next) {  // Kc^T rows c0, c0+1: this thread's 8 rows are two 16-byte chunks
+    if (has_next) {  // Kc^T rows c0..c0+3: this thread's 4 rows are one 16-byte chunk of each
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t chx = (uint32_t)(2 * rq + hh) ^ (uint32_t)(c0 & 7);
-      const uint32_t chy = (uint32_t)(2 * rq + hh) ^ (uint32_t)((c0 + 1) & 7);
-      *reinterpret_cast<float4*>(sm + SM_KC + c0 * 128 + (chx << 4)) =
-          make_float4(kcx[4 * hh], kcx[4 * hh + 1], kcx[4 * hh + 2], kcx[4 * hh + 3]);
-      *reinterpret_cast<float4*>(sm + SM_KC + (c0 + 1) * 128 + (chy << 4)) =
-          make_float4(kcy[4 * hh], kcy[4 * hh + 1], kcy[4 * hh + 2], kcy[4 * hh + 3]);
-    }
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int row = c0 + k4;
+        *reinterpret_cast<float4*>(sm + SM_KC + row * 128 + ((ro ^ (row & 7)) << 4)) =
+            make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
+      }
     }
     fence_proxy_async();
     fence_before_sync();

@@ -148,6 +148,19 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, ui
       : "memory");
 }
 
+// 2^x and 1/x on the special-function unit (approximate: relative error a few
+// ulp), used where the result only feeds bf16/tf32 operands or fp32 decays.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
