@@ -44,6 +44,10 @@ _SIGNATURES = {
                                    _VP, _VP]),
     "kda_chunk_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
                                    _F, _I, _VP, _VP, _VP]),
+    "kda_decode_verify": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _I, _I, _I, _I, _I, _F,
+                               _VP, _VP]),
+    "kda_decode_replay": (_I, [_VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I,
+                               _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
@@ -180,6 +184,27 @@ def kda_decode_step(q, k, v, g, beta, state, out, scale=1.0, stream=None):
     _check(lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q),
                                  _ptr(state), N, H, dk, dv, float(scale), _ptr(out),
                                  _stream(stream)), "kda_decode_step")
+
+
+def kda_decode_verify(q, k, v, g, beta, state, out, A_log=None, g_min=-5.0, scale=1.0,
+                      stream=None):
+    """Outputs of K draft tokens per sequence, state read only.  q, k, g
+    [N,K,H,dk], v/out [N,K,H,dv], beta [N,K,H]; g is z when A_log is given."""
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(lib().kda_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(A_log),
+                                   float(g_min), _ptr(beta), _dtype(q), _ptr(state), N, H, K, dk,
+                                   dv, float(scale), _ptr(out), _stream(stream)),
+           "kda_decode_verify")
+
+
+def kda_decode_replay(k, v, g, beta, state, accept_len, A_log=None, g_min=-5.0, stream=None):
+    """Apply each sequence's first accept_len[n] tokens to the state in place."""
+    N, K, H, dk = k.shape
+    dv = v.shape[-1]
+    _check(lib().kda_decode_replay(_ptr(k), _ptr(v), _ptr(g), _ptr(A_log), float(g_min),
+                                   _ptr(beta), _dtype(k), _ptr(state), _ptr(accept_len), N, H, K,
+                                   dk, dv, _stream(stream)), "kda_decode_replay")
 
 
 def kda_get_device_status(workspace, stream=None):

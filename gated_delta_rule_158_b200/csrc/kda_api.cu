@@ -286,6 +286,52 @@ kda_status kda_decode_step_gated(const void* q, const void* k, const void* v, co
                      stream);
 }
 
+kda_status kda_decode_verify(const void* q, const void* k, const void* v, const float* g,
+                             const float* A_log, float g_min, const float* beta,
+                             kda_dtype in_dtype, const float* state, int N, int H, int K, int dk,
+                             int dv, float scale, void* out, void* stream) {
+  if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (N <= 0 || H <= 0 || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (K < 1 || K > decode_multi_max_tokens()) return KDA_ERR_UNSUPPORTED;
+  if (A_log && (!(g_min < 0.f) || !isfinite(g_min))) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, g, beta, state, out, A_log};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {q, k, v, g, beta, state, A_log};
+  for (const void* i : ins)
+    if (i == out) return KDA_ERR_INVALID_ARG;
+  DecodeMultiArgs a{q, k, v, g, A_log, g_min, beta, in_dtype, const_cast<float*>(state), nullptr,
+                    out, N, H, K, dk, dv, scale};
+  return launch_decode_multi(a, true, (cudaStream_t)stream) == cudaSuccess ? KDA_OK
+                                                                            : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_replay(const void* k, const void* v, const float* g, const float* A_log,
+                             float g_min, const float* beta, kda_dtype in_dtype, float* state,
+                             const int32_t* accept_len, int N, int H, int K, int dk, int dv,
+                             void* stream) {
+  if (!k || !v || !g || !beta || !state || !accept_len) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (N <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+  if (K < 1 || K > decode_multi_max_tokens()) return KDA_ERR_UNSUPPORTED;
+  if (A_log && (!(g_min < 0.f) || !isfinite(g_min))) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)N * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {k, v, g, beta, state, accept_len, A_log};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {k, v, g, beta, accept_len, A_log};
+  for (const void* i : ins)
+    if (i == state) return KDA_ERR_INVALID_ARG;
+  DecodeMultiArgs a{nullptr, k, v, g, A_log, g_min, beta, in_dtype, state, accept_len, nullptr,
+                    N, H, K, dk, dv, 1.f};
+  return launch_decode_multi(a, false, (cudaStream_t)stream) == cudaSuccess ? KDA_OK
+                                                                             : KDA_ERR_CUDA;
+}
+
 kda_status kda_get_device_status(const void* workspace, void* stream, int32_t* detail) {
   if (!workspace) return KDA_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;

@@ -66,6 +66,25 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v,
                           int H, int dk, int dv, float scale, void* out,
                           cudaStream_t stream);
 
+struct DecodeMultiArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;      // log-decay g, or z when A_log is set
+  const float* A_log;  // nullable
+  float g_min;
+  const float* beta;
+  kda_dtype dt;
+  float* state;
+  const int32_t* accept_len;  // replay only
+  void* out;                  // verify only
+  int N, H, K, dk, dv;
+  float scale;
+};
+
+int decode_multi_max_tokens();
+cudaError_t launch_decode_multi(const DecodeMultiArgs& a, bool verify, cudaStream_t stream);
+
 __device__ __forceinline__ float gate_value(float z, float a, float g_min) {
   return g_min / (1.0f + expf(-a * z));
 }

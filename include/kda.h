@@ -173,6 +173,37 @@ KDA_API kda_status kda_decode_step_gated(const void *q, const void *k, const voi
                                  float scale, void *out, void *stream);
 
 /*
+ * Speculative decoding: verify K draft tokens per sequence without touching
+ * the state (KDA Decoding: same page, Online serving > high-performance
+ * kernels -- keep the draft tokens' projected inputs instead of state
+ * snapshots, and rebuild the state by replaying the accepted ones).  For each
+ * (n, h) the recurrence runs over tokens t = 0 .. K-1 from the committed state
+ * and writes o for every token; `state` is only read.
+ *  q, k, g : [N, K, H, dk]   v, out : [N, K, H, dv]   beta : fp32 [N, K, H]
+ *  g is the log-decay g, or z when A_log (fp32 [H]) is not NULL, in which
+ *  case g = g_min * Sigmoid(exp(A_log[h]) * z) is formed in the kernel.
+ *  state : fp32 [N, H, dk, dv]  (read only)
+ * Supported: 1 <= K <= 16, dk, dv in {32, 64, 128}.
+ */
+KDA_API kda_status kda_decode_verify(const void *q, const void *k, const void *v,
+                             const float *g, const float *A_log, float g_min,
+                             const float *beta, kda_dtype in_dtype,
+                             const float *state, int N, int H, int K, int dk,
+                             int dv, float scale, void *out, void *stream);
+
+/*
+ * Commit the accepted prefix of the draft tokens: for each (n, h) apply the
+ * first m_n = accept_len[n] tokens (k, v, g or z, beta laid out as for
+ * kda_decode_verify) to the state in place; m_n = 0 leaves it untouched.
+ * accept_len is a device int32 [N]; values are clamped to [0, K].
+ */
+KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *g,
+                             const float *A_log, float g_min, const float *beta,
+                             kda_dtype in_dtype, float *state,
+                             const int32_t *accept_len, int N, int H, int K,
+                             int dk, int dv, void *stream);
+
+/*
  * Synchronises `stream`, then returns the device status word that kernels
  * of an earlier kda_chunk_fwd call on this workspace recorded (KDA_OK if
  * none).  If detail is not NULL it receives a code-specific value (the

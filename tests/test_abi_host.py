@@ -132,3 +132,19 @@ def test_gated_entries_reject_on_host(L):
     d[4] = FAKE + 16
     d[5] = float("inf")
     assert L.kda_decode_step_gated(*d) == _lib.KDA_ERR_INVALID_ARG
+
+
+def test_verify_replay_reject_on_host(L):
+    v = [FAKE, FAKE, FAKE, FAKE, None, -5.0, FAKE, 1, FAKE + 64, 4, 2, 4, 128, 128, 1.0,
+         FAKE + 128, None]
+    bad = list(v); bad[11] = 0            # K = 0
+    assert L.kda_decode_verify(*bad) == _lib.KDA_ERR_UNSUPPORTED
+    bad = list(v); bad[11] = 17           # K above 16
+    assert L.kda_decode_verify(*bad) == _lib.KDA_ERR_UNSUPPORTED
+    bad = list(v); bad[15] = FAKE         # out aliases q
+    assert L.kda_decode_verify(*bad) == _lib.KDA_ERR_INVALID_ARG
+    r = [FAKE, FAKE, FAKE, None, -5.0, FAKE, 1, FAKE + 64, FAKE + 128, 4, 2, 4, 128, 128, None]
+    bad = list(r); bad[8] = None          # accept_len missing
+    assert L.kda_decode_replay(*bad) == _lib.KDA_ERR_INVALID_ARG
+    bad = list(r); bad[8] = FAKE + 132    # misaligned accept_len
+    assert L.kda_decode_replay(*bad) == _lib.KDA_ERR_MISALIGNED

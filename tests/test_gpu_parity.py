@@ -333,3 +333,77 @@ def test_gated_decode(oracle_mod, dtype):
     tol_o, tol_s = (TOL_F32, TOL_F32) if dtype == torch.float32 else (TOL_BF16_O, TOL_BF16_S)
     assert rel_l2(to64(torch.stack(outs, 1)), o_ref) <= tol_o
     assert rel_l2(to64(state), S_ref) <= tol_s
+
+
+# ------------------------------------------ speculative decoding: verify / replay
+
+def _draft_inputs(N, K, H, dk, dv, dtype, seed):
+    """K draft tokens per sequence ([N, K, H, *] layouts) and a committed state."""
+    inp = W.make_prefill_inputs(N, K, H, dk, dv, dtype, seed=seed, device=DEV)
+    S0 = W.make_decode_state(N, H, dk, dv, seed + 500, DEV)
+    return inp, S0
+
+
+@pytest.mark.parametrize("K", [1, 4, 16])
+@pytest.mark.parametrize("dk,dv,dtype", [(128, 128, torch.bfloat16), (64, 32, torch.float32),
+                                         (32, 128, torch.bfloat16)])
+def test_decode_verify(oracle_mod, K, dk, dv, dtype):
+    N, H = 3, 4
+    inp, S0 = _draft_inputs(N, K, H, dk, dv, dtype, seed=90 + K)
+    state = S0.clone()
+    out = torch.full((N, K, H, dv), float("nan"), dtype=dtype, device=DEV)
+    kda.kda_decode_verify(inp["q"], inp["k"], inp["v"], inp["z"], inp["beta"], state, out,
+                          A_log=inp["A_log"], scale=0.8)
+    torch.cuda.synchronize()
+    assert torch.equal(state, S0)  # the committed state is only read
+    g_ref = oracle_mod.gate(to64(inp["z"]), to64(inp["A_log"]), -5.0)
+    o_ref, _ = oracle_mod.forward(to64(inp["q"]), to64(inp["k"]), to64(inp["v"]), g_ref,
+                                  to64(inp["beta"]), init_state=to64(S0), scale=0.8)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16_O
+    assert rel_l2(to64(out), o_ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_replay_accepted_prefix(oracle_mod, dtype):
+    N, K, H, d = 5, 8, 3, 128
+    inp, S0 = _draft_inputs(N, K, H, d, d, dtype, seed=120)
+    accept = [0, 8, 3, 1, 5]
+    acc = torch.tensor(accept, dtype=torch.int32, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    state = S0.clone()
+    kda.kda_decode_replay(inp["k"], inp["v"], g, inp["beta"], state, acc)
+    torch.cuda.synchronize()
+    g_ref = oracle_mod.gate(to64(inp["z"]), to64(inp["A_log"]), -5.0)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16_S
+    for n, m in enumerate(accept):
+        if m == 0:
+            assert torch.equal(state[n], S0[n])
+            continue
+        sl = lambda t: t[n:n + 1, :m]
+        _, S_ref = oracle_mod.forward(to64(sl(inp["q"])), to64(sl(inp["k"])), to64(sl(inp["v"])),
+                                      g_ref[n:n + 1, :m], to64(sl(inp["beta"])),
+                                      init_state=to64(S0[n:n + 1]))
+        assert rel_l2(to64(state[n]), S_ref[0]) <= tol
+
+
+def test_verify_then_replay_equals_step_by_step():
+    """verify(K) outputs and replay(K) state equal K single decode steps."""
+    N, K, H, d = 4, 6, 2, 128
+    inp, S0 = _draft_inputs(N, K, H, d, d, torch.bfloat16, seed=130)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    out = torch.empty((N, K, H, d), dtype=torch.bfloat16, device=DEV)
+    kda.kda_decode_verify(inp["q"], inp["k"], inp["v"], g, inp["beta"], S0, out)
+    state = S0.clone()
+    kda.kda_decode_replay(inp["k"], inp["v"], g, inp["beta"], state,
+                          torch.full((N,), K, dtype=torch.int32, device=DEV))
+    ref_state = S0.clone()
+    ref_out = []
+    for t in range(K):
+        o = torch.empty((N, H, d), dtype=torch.bfloat16, device=DEV)
+        kda.kda_decode_step(inp["q"][:, t].contiguous(), inp["k"][:, t].contiguous(),
+                            inp["v"][:, t].contiguous(), g[:, t].contiguous(),
+                            inp["beta"][:, t].contiguous(), ref_state, o)
+        ref_out.append(o)
+    torch.cuda.synchronize()
+    assert rel_l2(to64(out), to64(torch.stack(ref_out, 1))) <= 1e-2
+    assert rel_l2(to64(state), to64(ref_state)) <= 1e-5
