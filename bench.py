@@ -300,6 +300,42 @@ def run_decode(wl, device, warmup=3):
     return total_ms, dec_ms, bytes_per_launch
 
 
+def run_spec_decode(device, N=256, H=32, d=128, K=4, reps=50, seed=7):
+    """Speculative decoding: verify K draft tokens per sequence (state read
+    once, outputs for every token), then replay all K accepted tokens into the
+    state.  Returns per-launch times and algorithmic bytes."""
+    inp = W.make_prefill_inputs(N, K, H, d, d, torch.bfloat16, seed=seed, device=device)
+    state = W.make_decode_state(N, H, d, d, seed + 1, device)
+    out = torch.empty((N, K, H, d), dtype=torch.bfloat16, device=device)
+    acc = torch.full((N,), K, dtype=torch.int32, device=device)
+
+    def verify():
+        kda.kda_decode_verify(inp["q"], inp["k"], inp["v"], inp["z"], inp["beta"], state, out,
+                              A_log=inp["A_log"])
+
+    def replay():
+        kda.kda_decode_replay(inp["k"], inp["v"], inp["z"], inp["beta"], state, acc,
+                              A_log=inp["A_log"])
+
+    res = {}
+    for name, fn in (("verify", verify), ("replay", replay)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        res[name] = a.elapsed_time(b) / reps
+    per_head_in = K * (3 * d * 2 + d * 4 + 4)        # q, k, v bf16; z fp32; beta
+    bytes_verify = N * H * (d * d * 4 + per_head_in + K * d * 2)   # state read, o written
+    bytes_replay = N * H * (2 * d * d * 4 + per_head_in - K * d * 2)  # no q, state r+w
+    return res, bytes_verify, bytes_replay, K
+
+
 # ------------------------------------------------------- oracle baseline
 def oracle_prefill_parallel_sample(wl, inp, cu, budget_s=15.0):
     """Same as above but runs the oracle's own thread pool over a batch of
@@ -387,6 +423,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="skip nvidia-smi clock sampling (profiling runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of a dense prefill workload (smaller profiling captures)")
     args = ap.parse_args()
@@ -394,7 +432,10 @@ def main():
 
     world, rank, local = dist_setup()
     wl = dict(WORKLOADS[args.workload])
-    if args.batch is not None and not wl.get("varlen", True):
+    if args.batch is not None and args.workload == "decode":
+        wl["N"] = args.batch
+        wl["name"] = wl["name"].replace("N256 ", f"N{args.batch} ")
+    elif args.batch is not None and not wl.get("varlen", True):
         wl["B"] = args.batch
         wl["name"] = wl["name"].replace(f"B{WORKLOADS[args.workload]['B']} ", f"B{args.batch} ")
     peaks = load_peaks()
@@ -426,9 +467,9 @@ def bench_prefill_line(args, wl, world, rank, peaks):
     B = inp["q"].shape[0]
     tokens = B * T  # per rank
     step = PrefillStep(inp, cu, N)
-    clocks = ClockSampler(dev.index)
+    clocks = None if args.no_clocks else ClockSampler(dev.index)
     total_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
-    clk = clocks.extend_window(step)
+    clk = clocks.extend_window(step) if clocks else None
     st, _ = kda.kda_get_device_status(step.ws)
     if st != kda.KDA_OK:
         raise RuntimeError(f"device status {kda.kda_status_string(st)}")
@@ -480,15 +521,27 @@ def bench_prefill_line(args, wl, world, rank, peaks):
                                        "kernel": "decode_kernel (kda_decode_step_gated)",
                                        "kernel_ms": round(dec_ms, 4),
                                        "algorithmic_bytes": bpl}}
+        res, bv, br, K = run_spec_decode(dev)
+        line["spec_decode"] = {
+            "workload": f"verify/replay N256 H32 d128, K={K} draft tokens",
+            "verify_ms": round(res["verify"], 4),
+            "verify_tokens_per_s": round(256 * K / (res["verify"] * 1e-3), 1),
+            "verify_roofline": {"bound": "hbm", "achieved": round(bv / (res["verify"] * 1e-3) / 1e9, 1),
+                                "peak": peaks["hbm"], "unit": "GB/s",
+                                "frac": round(bv / (res["verify"] * 1e-3) / 1e9 / peaks["hbm"], 4)},
+            "replay_ms": round(res["replay"], 4),
+            "replay_roofline": {"bound": "hbm", "achieved": round(br / (res["replay"] * 1e-3) / 1e9, 1),
+                                "peak": peaks["hbm"], "unit": "GB/s",
+                                "frac": round(br / (res["replay"] * 1e-3) / 1e9 / peaks["hbm"], 4)}}
     return line
 
 
 def bench_decode_line(args, wl, world, rank, peaks):
     dev = torch.device("cuda", torch.cuda.current_device())
-    clocks = ClockSampler(dev.index)
+    clocks = None if args.no_clocks else ClockSampler(dev.index)
     barrier(world)
     total, dec_ms, bpl = run_decode(wl, dev)
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     total = max_over_ranks(total, world)
     dach = bpl / (dec_ms * 1e-3) / 1e9
     line = {
