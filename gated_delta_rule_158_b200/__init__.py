@@ -9,4 +9,5 @@ from ._lib import (  # noqa: F401
     KDA_ERR_TIMEOUT, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_F32, KDA_OK, KdaError,
     kda_chunk_fwd, kda_chunk_fwd_gated, kda_chunk_fwd_noalloc, kda_chunk_fwd_workspace_size, kda_decode_step,
     kda_decode_replay, kda_decode_step_gated, kda_decode_verify, kda_gate_fwd,
-    kda_get_device_status, kda_selftest_bounded_wait, kda_status_string, lib)
+    kda_get_device_status, kda_last_cuda_error_string, kda_selftest_bounded_wait, kda_status_string,
+    lib)

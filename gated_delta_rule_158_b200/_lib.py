@@ -33,6 +33,7 @@ _SZ = ctypes.c_size_t
 
 _SIGNATURES = {
     "kda_status_string": (ctypes.c_char_p, [_I]),
+    "kda_last_cuda_error_string": (ctypes.c_char_p, []),
     "kda_gate_fwd": (_I, [_VP, _VP, _F, _VP, _I64, _I, _I, _VP]),
     "kda_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "kda_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
@@ -58,7 +59,10 @@ _lib = None
 class KdaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where} failed: {kda_status_string(status)} ({status})")
+        msg = f"{where} failed: {kda_status_string(status)} ({status})"
+        if status == KDA_ERR_CUDA:
+            msg += f" [{kda_last_cuda_error_string()}]"
+        super().__init__(msg)
 
 
 def lib():
@@ -111,6 +115,10 @@ def _check(status, where):
 
 def kda_status_string(status: int) -> str:
     return lib().kda_status_string(int(status)).decode()
+
+
+def kda_last_cuda_error_string() -> str:
+    return lib().kda_last_cuda_error_string().decode()
 
 
 def kda_gate_fwd(z, A_log, g, g_min=-5.0, stream=None):

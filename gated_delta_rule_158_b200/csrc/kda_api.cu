@@ -2,12 +2,29 @@
 // layout, path selection and launches.  The contract of every entry point is
 // in include/kda.h.
 #include <math.h>
+#include <stdio.h>
 #include <string.h>
 
 #include "kda_internal.cuh"
 #include "kda_sync.cuh"
 
 namespace kda {
+
+namespace {
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+}
+
+kda_status cuda_failure(cudaError_t e) {
+  t_last_cuda_error = e;
+  return KDA_ERR_CUDA;
+}
+
+const char* last_cuda_error_text() {
+  thread_local char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", cudaGetErrorName(t_last_cuda_error),
+           cudaGetErrorString(t_last_cuda_error));
+  return buf;
+}
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -114,7 +131,7 @@ kda_status kda_gate_fwd(const float* z, const float* A_log, float g_min, float* 
   if (!aligned16(z) || !aligned16(g) || !aligned16(A_log)) return KDA_ERR_MISALIGNED;
   if (rows == 0) return KDA_OK;
   cudaError_t e = launch_gate(z, A_log, g_min, g, rows, H, dk, (cudaStream_t)stream);
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
@@ -168,7 +185,7 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   cudaStream_t st = (cudaStream_t)stream;
   StatusBlock* sb = static_cast<StatusBlock*>(workspace);
   char* tail = static_cast<char*>(workspace) + kStatusBytes;
-  if (cudaMemsetAsync(sb, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaError_t em = cudaMemsetAsync(sb, 0, kStatusBytes, st)) return cuda_failure(em);
 
   ChunkArgs a{};
   a.q = q;
@@ -198,8 +215,8 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   if (cu_seqlens) {
     int32_t* order = reinterpret_cast<int32_t*>(tail);
     tail += round_up(sizeof(int32_t) * (size_t)num_seqs, 256);
-    if (launch_varlen_plan(cu_seqlens, num_seqs, T, order, sb, st) != cudaSuccess)
-      return KDA_ERR_CUDA;
+    if (cudaError_t ep = launch_varlen_plan(cu_seqlens, num_seqs, T, order, sb, st))
+      return cuda_failure(ep);
     a.map.order = order;
   }
   cudaError_t e;
@@ -211,7 +228,7 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
     if (a.chunk == 0) a.chunk = 32;
     e = launch_chunk_simt(a, st);
   }
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 }  // namespace
@@ -263,7 +280,7 @@ kda_status decode_impl(const void* q, const void* k, const void* v, const float*
     if (i == out) return KDA_ERR_INVALID_ARG;
   cudaError_t e = launch_decode(q, k, v, g, A_log, g_min, beta, in_dtype, state, N, H, dk, dv,
                                 scale, out, (cudaStream_t)stream);
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 }  // namespace
@@ -305,8 +322,8 @@ kda_status kda_decode_verify(const void* q, const void* k, const void* v, const 
     if (i == out) return KDA_ERR_INVALID_ARG;
   DecodeMultiArgs a{q, k, v, g, A_log, g_min, beta, in_dtype, const_cast<float*>(state), nullptr,
                     out, N, H, K, dk, dv, scale};
-  return launch_decode_multi(a, true, (cudaStream_t)stream) == cudaSuccess ? KDA_OK
-                                                                            : KDA_ERR_CUDA;
+  const cudaError_t e = launch_decode_multi(a, true, (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 kda_status kda_decode_replay(const void* k, const void* v, const float* g, const float* A_log,
@@ -328,17 +345,19 @@ kda_status kda_decode_replay(const void* k, const void* v, const float* g, const
     if (i == state) return KDA_ERR_INVALID_ARG;
   DecodeMultiArgs a{nullptr, k, v, g, A_log, g_min, beta, in_dtype, state, accept_len, nullptr,
                     N, H, K, dk, dv, 1.f};
-  return launch_decode_multi(a, false, (cudaStream_t)stream) == cudaSuccess ? KDA_OK
-                                                                             : KDA_ERR_CUDA;
+  const cudaError_t e = launch_decode_multi(a, false, (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
+
+const char* kda_last_cuda_error_string(void) { return last_cuda_error_text(); }
 
 kda_status kda_get_device_status(const void* workspace, void* stream, int32_t* detail) {
   if (!workspace) return KDA_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaError_t es = cudaStreamSynchronize(st)) return cuda_failure(es);
   int32_t host[2] = {0, 0};
-  if (cudaMemcpy(host, workspace, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return KDA_ERR_CUDA;
+  if (cudaError_t ec = cudaMemcpy(host, workspace, sizeof(host), cudaMemcpyDeviceToHost))
+    return cuda_failure(ec);
   if (detail) *detail = host[1];
   return (kda_status)host[0];
 }
@@ -350,9 +369,9 @@ kda_status kda_selftest_bounded_wait(void* workspace, int64_t spin_limit_ns, voi
   if (lim < 1000) lim = 1000;
   if (lim > 5000000000LL) lim = 5000000000LL;
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaError_t em = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) return cuda_failure(em);
   cudaError_t e = launch_selftest_wait(static_cast<StatusBlock*>(workspace), lim, st);
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 }  // extern "C"

@@ -190,7 +190,10 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
   return true;
 }
 
-__global__ void __maxnreg__(152)
+// The register file is split across the SM's four sub-partitions and a CTA's
+// warps are dealt to them in turn, so with 13 warps one quarter holds four of
+// them: 16384 / (4 * 32) = 128 registers per thread is the most that launches.
+__global__ void __maxnreg__(128)
     chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);

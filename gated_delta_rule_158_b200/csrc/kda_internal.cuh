@@ -126,4 +126,8 @@ cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns,
 
 int device_sm_count();
 
+// Remembers the CUDA error behind a KDA_ERR_CUDA return (per host thread).
+kda_status cuda_failure(cudaError_t e);
+const char* last_cuda_error_text();
+
 }  // namespace kda

@@ -61,7 +61,7 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const 
                                             int chunk_size, void* out, float* final_state,
                                             void* stream) {
   void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaError_t e = scratch_address(&scratch)) return kda::cuda_failure(e);
   // kda_chunk_fwd checks every argument and returns KDA_ERR_WORKSPACE, with
   // nothing enqueued, when the problem needs more scratch than the array holds.
   return kda_chunk_fwd(q, k, v, g, beta, in_dtype, init_state, cu_seqlens, num_seqs, B, T, H,

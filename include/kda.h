@@ -204,6 +204,12 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
                              int dk, int dv, void *stream);
 
 /*
+ * Name and description of the last CUDA error a libkda call on this host
+ * thread turned into KDA_ERR_CUDA ("no error" if none).  Static storage.
+ */
+KDA_API const char *kda_last_cuda_error_string(void);
+
+/*
  * Synchronises `stream`, then returns the device status word that kernels
  * of an earlier kda_chunk_fwd call on this workspace recorded (KDA_OK if
  * none).  If detail is not NULL it receives a code-specific value (the

@@ -48,6 +48,11 @@ def test_status_strings(L):
     assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
 
 
+def test_last_cuda_error_string_starts_clean(L):
+    # host-only calls that fail validation never record a CUDA error
+    assert kda.kda_last_cuda_error_string().startswith("cudaSuccess")
+
+
 FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
 
 
