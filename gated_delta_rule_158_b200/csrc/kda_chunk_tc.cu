@@ -45,66 +45,38 @@ namespace {
 
 using namespace tc;
 
-constexpr int C = 32;        // tokens per chunk
-constexpr int D = 128;       // dk = dv
-constexpr int NKEY_WARPS = 8;    // warps 0-7: key side (operands, Gram, inverse, W)
-constexpr int STATE_WARP0 = 8;   // warps 8-11: state side (decay, outputs)
-constexpr int ISSUE_WARP = 12;   // warp 12: MMA and TMA issue
-constexpr int NT = 32 * 13;
+constexpr int C = 32;     // tokens per chunk
+constexpr int D = 128;    // dk = dv
+constexpr int NT = 256;   // threads per CTA
 
-// TMEM columns (512 allocated: one CTA per SM)
-constexpr uint32_t S_COL = 0;     // S^T            [0, 128)
-constexpr uint32_t U_COL = 128;   // U^T buffer b   [128 + 32b, 160 + 32b)
-constexpr uint32_t W_COL = 192;   // W'^T
-constexpr uint32_t O_COL = 224;   // O^T
-constexpr uint32_t G_COL = 256;   // Gram (M = 64 layout: lanes 0-15 of each quarter)
-constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0, U_COL = 128, W_COL = 160, O_COL = 192, G_COL = 224;
+constexpr uint32_t TMEM_COLS = 256;
 
 // shared memory map (byte offsets from a 1024-aligned base)
-constexpr uint32_t STAGE = 40960;               // one input stage; two stages at 0
-constexpr uint32_t OFF_Q = 0;                   //   q bf16 [32][128] (TMA, no swizzle)
-constexpr uint32_t OFF_K = 8192;                //   k bf16 [32][128]
-constexpr uint32_t OFF_V = 16384;               //   v bf16 2 x [32 x 128 B] (TMA, 128-B swizzle)
-constexpr uint32_t OFF_G = 24576;               //   g or z fp32 [32][128]
-constexpr uint32_t SM_KQL = 81920;              // [k;q] e^{G-G15} bf16 64 x 128 (Gram A; rows 0-31: A of W')
-constexpr uint32_t SM_KB = SM_KQL + 16384;      // k e^{G15-G} bf16 32 x 128 (Gram B)
-constexpr uint32_t SM_AKKT = SM_KB;             // A_kk^T fp32 [s][r] (after the Gram GEMM)
-constexpr uint32_t SM_XS = SM_KB + 4096;        // inverse blocks fp32 32 x 32
-constexpr uint32_t SM_TT = 106496;              // T bf16 [r][s]; 4-row cumsum totals during prep
-constexpr uint32_t SM_HO = 110592;              // two key -> state hand-off buffers
-constexpr uint32_t HO = 53248;
-constexpr uint32_t HO_WF = 0;                   //   W fp32 [r][i]  (tf32 B of U)
-constexpr uint32_t HO_QG = 16384;               //   q e^G fp32 [r][i] (tf32 B of O)
-constexpr uint32_t HO_KC = 32768;               //   Kc^T fp32 [i][s] (tf32 B of S)
-constexpr uint32_t HO_AQK = 49152;              //   A_qk fp32 [r][s] (tf32 B of O)
-constexpr uint32_t SM_MISC = SM_HO + 2 * HO;    // 217088
-constexpr uint32_t SM_GAMC = SM_MISC;           // e^{Gamma_C} fp32 [2][128]
-constexpr uint32_t SM_E15 = SM_MISC + 1024;     // e^{Gamma_15} fp32 [128]
-constexpr uint32_t SM_BETA = SM_MISC + 1536;    // beta fp32 [32]
-constexpr uint32_t SM_BAR = SM_MISC + 1664;     // mbarriers
-constexpr uint32_t SM_TMEM = SM_MISC + 1920;    // TMEM base address
-constexpr uint32_t SM_ABORT = SM_MISC + 1924;   // abort flag
+constexpr uint32_t SM_Q = 0;         // q tile  bf16 [32][128] row-major (TMA, no swizzle)
+constexpr uint32_t SM_K = 8192;      // k tile  bf16 [32][128]
+constexpr uint32_t SM_V = 16384;     // v tile  bf16, 2 x [32 rows x 128 B] swizzled (TMA)
+constexpr uint32_t SM_G = 24576;     // g (or z) tile fp32 [32][128]
+constexpr uint32_t SM_R1 = 40960;    // 24 KB, two lives:
+constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128: Gram A, and
+                                              //  (rows 0-31) the MN-major A of W' = T K_L
+constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
+constexpr uint32_t SM_WF = SM_R1;             //  W                fp32 32 x 128 (tf32 B)
+constexpr uint32_t SM_AKKT = SM_R1 + 16384;   //  A_kk^T fp32 [s][r] 32 x 32 (inverse input)
+constexpr uint32_t SM_XS = SM_R1 + 20480;     //  inverse blocks X00, X11 and A10 X00, fp32 32 x 32
+constexpr uint32_t SM_TT = 65536;    // T            bf16 [r][s] (B of W' and U~); cumsum partials during prep
+constexpr uint32_t SM_QG = 69632;    // q e^G        fp32 [r][i] (tf32 B of O)
+constexpr uint32_t SM_KC = 86016;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
+constexpr uint32_t SM_AQK = 102400;  // A_qk         fp32 [r][s] 32 x 32 (tf32 B of O)
+constexpr uint32_t SM_MISC = 106496;
+constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
+constexpr uint32_t SM_E15 = SM_MISC + 512;     // e^{Gamma_15} fp32 [128]
+constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta         fp32 [32]
+constexpr uint32_t SM_BAR = SM_MISC + 1152;    // 3 mbarriers
+constexpr uint32_t SM_TMEM = SM_MISC + 1184;   // TMEM base address
+constexpr uint32_t SM_ABORT = SM_MISC + 1188;  // abort flag
 constexpr uint32_t SMEM_BYTES = SM_MISC + 2048;
-constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
-
-// mbarrier indices
-enum : int {
-  B_IN_FULL = 0,      // [2] TMA q, k, g landed                 (tx)
-  B_IN_EMPTY = 2,     // [2] key warps done with q, k, g        (8 warps)
-  B_V_FULL = 4,       // [2] TMA v landed                       (tx)
-  B_V_EMPTY = 6,      // [2] U~ GEMM done with v                (commit)
-  B_OPER = 8,         // operands of the chunk written          (8 warps)
-  B_GRAM = 9,         // Gram GEMM done                         (commit)
-  B_T = 10,           // T written                              (4 warps)
-  B_WU = 11,          // W', U~ GEMMs done                      (commit)
-  B_KEY = 12,         // [2] hand-off buffer b complete         (8 warps)
-  B_UO = 14,          // U and O1 GEMMs done                    (commit)
-  B_DECAY = 15,       // state decayed                          (4 warps)
-  B_SO = 16,          // [2] S and O2 GEMMs done, buffer b free (commit)
-  B_OFREE = 18,       // O exported                             (4 warps)
-  B_DRAIN = 19,       // all GEMMs done (abort path)            (commit)
-  NBARS = 20
-};
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to 1024
 
 constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
 constexpr uint32_t TX_V = 8192;
@@ -190,11 +162,7 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
   return true;
 }
 
-// The register file is split across the SM's four sub-partitions and a CTA's
-// warps are dealt to them in turn, so with 13 warps one quarter holds four of
-// them: 16384 / (4 * 32) = 128 registers per thread is the most that launches.
-__global__ void __maxnreg__(128)
-    chunk_tc_kernel(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -204,25 +172,19 @@ __global__ void __maxnreg__(128)
   if (!resolve_unit(P, U)) return;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
+  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + SM_BAR);
+  uint64_t* bar_v = bar_in + 1;
+  uint64_t* bar_mma = bar_in + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_ABORT);
+  float* gamc = reinterpret_cast<float*>(sm + SM_GAMC);
   float* betas = reinterpret_cast<float*>(sm + SM_BETA);
   const int H = P.H, h = U.h;
-  const int nchunks = (int)((U.len + C - 1) / C);
-  auto chunk_rows = [&](int cc) -> int {
-    const int64_t rem = U.len - (int64_t)cc * C;
-    return (int)(rem < C ? rem : C);
-  };
 
   if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < NBARS; ++i) {
-      const bool per_key_warp = i == B_IN_EMPTY || i == B_IN_EMPTY + 1 || i == B_OPER ||
-                                i == B_KEY || i == B_KEY + 1;
-      const bool per_4_warps = i == B_T || i == B_DECAY || i == B_OFREE;
-      mbar_init(&bars[i], per_key_warp ? NKEY_WARPS : (per_4_warps ? 4u : 1u));
-    }
+    mbar_init(bar_in, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_mma, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -235,488 +197,482 @@ __global__ void __maxnreg__(128)
   fence_after_sync();
   const uint32_t tbase = *tmem_slot;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lanes
+  const int half = warp >> 2;                                   // column half (8-warp passes)
 
-  // ---- initial state -> TMEM (S^T: lane j, column i), by the state warps
-  if (warp >= STATE_WARP0 && warp < ISSUE_WARP) {
+  const int nchunks = (int)((U.len + C - 1) / C);
+  const float a2 = P.A_log ? expf(P.A_log[h]) * 1.4426950408889634f : 0.f;
+  bool pend_in = false, pend_v = false;  // thread 0: TMA loads issued, not yet waited
+  auto issue_qkg = [&](int c) {
+    const int row = (int)(U.row0 + (int64_t)c * C);
+    mbar_arrive_expect_tx(bar_in, TX_QKG);
+    tma_load_3d(sm + SM_Q, &P.tm_q, bar_in, 0, h, row);
+    tma_load_3d(sm + SM_K, &P.tm_k, bar_in, 0, h, row);
+    tma_load_3d(sm + SM_G, &P.tm_g, bar_in, 0, h, row);
+    pend_in = true;
+  };
+  auto issue_v = [&](int c) {
+    const int row = (int)(U.row0 + (int64_t)c * C);
+    mbar_arrive_expect_tx(bar_v, TX_V);
+    tma_load_3d(sm + SM_V, &P.tm_v, bar_v, 0, h, row);
+    tma_load_3d(sm + SM_V + 4096, &P.tm_v, bar_v, 64, h, row);
+    pend_v = true;
+  };
+  if (tid == 0 && nchunks > 0) {
+    issue_qkg(0);
+    if (!U.vzero) issue_v(0);
+  }
+
+  // ---- initial state -> TMEM (S^T: lane j, column i)
+  {
     const int j = 32 * (warp & 3) + lane;
     float v[32];
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
+      const int i0 = 64 * half + 32 * cc;
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const int i = 32 * cc + k;
+        const int i = i0 + k;
         v[k] = U.init ? U.init[(size_t)i * D + j] : ((U.init_identity && i == j) ? 1.f : 0.f);
       }
-      tmem_st32(tbase + lane_base + S_COL + 32 * cc, v);
+      tmem_st32(tbase + lane_base + S_COL + i0, v);
     }
     wait_st();
   }
   fence_before_sync();
   __syncthreads();
-  fence_after_sync();
 
-  if (warp < NKEY_WARPS) {
-    // ======================================================== key-side warps
-    const int cq = tid & 31, ro = warp, c0 = 4 * cq;  // channels c0..c0+3, rows 4ro..4ro+3
-    const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;
-    const uint32_t ck32 = ((c0 & 31) * 4) >> 4;
-    const uint32_t o_kql = (c0 >> 6) * 8192 + ro * 512 + lo16;
-    const uint32_t o_kb = (c0 >> 6) * 4096 + ro * 512 + lo16;
-    const uint32_t o_qg = (c0 >> 5) * 4096 + ro * 512;
-    constexpr float kLog2e = 1.4426950408889634f;
-    const float gmin2 = P.g_min * kLog2e;
-    const float a2 = P.A_log ? expf(P.A_log[h]) * kLog2e : 0.f;
-    float beta_next = 0.f;
-    if (tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
+  uint32_t ph_in = 0, ph_v = 0, ph_mma = 0;
+  const uint32_t id_gram = idesc(kFmtBF16, 64, C, false, false, false);
+  const uint32_t id_w = idesc(kFmtBF16, 128, C, true, false, false);
+  const uint32_t id_o = idesc(kFmtTF32, 128, C, false, false, false);
+  const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
+  const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
 
-    for (int c = 0; c < nchunks; ++c) {
-      if (bar_red_or(1, 256, *abort_flag != 0)) break;
-      const int st = c & 1, b = c & 1;
-      const int n = chunk_rows(c);
-      uint8_t* in = sm + st * STAGE;
-      uint8_t* ho = sm + SM_HO + b * HO;
+  // prep thread mapping: channels c0 .. c0+3 and rows 4ro .. 4ro+3 (warp ro)
+  const int cq = tid & 31, ro = tid >> 5, c0 = 4 * cq;
+  // byte offsets of (row 4ro, channel c0) in each swizzled operand; a row
+  // 4ro + rr adds rr*128 and xors the 16-byte chunk index with (4ro + rr) & 7
+  const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;   // bf16 tiles
+  const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                                 // fp32 tiles
+  const uint32_t o_kql = (c0 >> 6) * 8192 + ro * 512 + lo16;
+  const uint32_t o_kb = (c0 >> 6) * 4096 + ro * 512 + lo16;
+  const uint32_t o_qg = (c0 >> 5) * 4096 + ro * 512;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float gmin2 = P.g_min * kLog2e;
+  auto chunk_rows = [&](int cc) -> int {
+    const int64_t rem = U.len - (int64_t)cc * C;
+    return (int)(rem < C ? rem : C);
+  };
+
+  float beta_next = 0.f;  // beta of the chunk after the one being prepared
+  float4 G4[4];           // in-chunk cumulative log2-decay of the chunk being prepared
+  float kc[4][4];         // its Kc values [channel][row], stored after the state update
+
+  // ---- prep, part 1: wait for the chunk's tiles, beta, cumulative sums of g
+
+  // ---- prep, part 2 (after a barrier): rescaled operands of the chunk
+
+  // ---- Kc^T rows c0, c0+1: this thread's 8 rows are two 16-byte chunks of each
+
+  // ---- O^T of chunk cc (lane j, column r) -> o rows; lanes j, j^1 swap values so
+  //      each writes a bf16 pair (even lane rows 2m, odd lane rows 2m+1).  Warps 4-7.
+  auto export_o = [&](int cc) {
+    const int n = chunk_rows(cc);
+    const int j = 32 * (warp & 3) + lane;
+    const bool odd = lane & 1;
+    float v[32];
+    tmem_ld32(tbase + lane_base + O_COL, v);
+    wait_ld();
+    const int jp = j & ~1;
+    __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + (int64_t)cc * C) * H + h) * D + jp;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float send = odd ? v[2 * m] : v[2 * m + 1];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      const int r = 2 * m + (odd ? 1 : 0);
+      const float lo = odd ? recv : v[2 * m];      // column jp
+      const float hi = odd ? v[2 * m + 1] : recv;  // column jp + 1
+      if (r < n)
+        *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
+            __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
+    }
+  };
+
+  // the loop starts at c = -1: that pass only prepares chunk 0's operands
+  if (nchunks > 0 && tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
+  for (int c = -1; c < nchunks && !*abort_flag; ++c) {
+    const bool has_next = c + 1 < nchunks;
+    if (c >= 0) {
+
+    // ===== A: Gram GEMM (M64 N32 K128) of chunk c; warps 4-7 export O of chunk c-1
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kb = ks >> 2, kk = ks & 3;
+        const uint64_t a = sw128_desc(sb + SM_KQL + kb * (64 * 128) + kk * 32, 16, 1024);
+        const uint64_t b = sw128_desc(sb + SM_KB + kb * (32 * 128) + kk * 32, 16, 1024);
+        mma_ss(tbase + G_COL, a, b, id_gram, 0, ks > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    if (c > 0 && U.out_on && warp >= 4) export_o(c - 1);
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 2);
+    ph_mma ^= 1;
+    fence_after_sync();
+
+    // ===== B: A_kk (transposed, x beta) and A_qk from the Gram accumulator
+    if (warp < 4) {
+      float v[32];
+      tmem_ld32(tbase + lane_base + G_COL, v);
+      wait_ld();
+      if (lane < 16) {
+        const int r = 16 * (warp & 1) + lane;
+        if (warp < 2) {
+          const float br = betas[r];
+          float* akkt = reinterpret_cast<float*>(sm + SM_AKKT);
+#pragma unroll
+          for (int s2 = 0; s2 < 32; ++s2) akkt[s2 * 32 + r] = s2 < r ? br * v[s2] : 0.f;
+        } else {
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            float4 w4;
+            w4.x = (4 * s4 + 0 <= r) ? v[4 * s4 + 0] : 0.f;
+            w4.y = (4 * s4 + 1 <= r) ? v[4 * s4 + 1] : 0.f;
+            w4.z = (4 * s4 + 2 <= r) ? v[4 * s4 + 2] : 0.f;
+            w4.w = (4 * s4 + 3 <= r) ? v[4 * s4 + 3] : 0.f;
+            *reinterpret_cast<float4*>(sm + SM_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
+          }
+        }
+      }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ===== C: T = (I + A_kk)^-1 Diag(beta), blocked 2 x 2 over 16-row blocks
+    if (warp < 4) {
+      const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
+      float* xs = reinterpret_cast<float*>(sm + SM_XS);
+      auto tt_store = [&](int r, int col, float val) {
+        *reinterpret_cast<__nv_bfloat16*>(
+            sm + SM_TT + r * 128 + ((((uint32_t)(col * 2) >> 4) ^ (uint32_t)(r & 7)) << 4) +
+            ((col * 2) & 15)) = __float2bfloat16_rn(val);
+      };
+      if (warp == 0) {  // diagonal blocks: lane = (block b, column cb)
+        const int b = lane >> 4, cb = lane & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == cb) ? 1.f : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 15; ++s2) {
+          const float xv = x[s2];
+          const float* col = akkt + (o + s2) * 32 + o;  // A[o + r][o + s2], r = 0..15
+#pragma unroll
+          for (int r4 = (s2 + 1) / 4; r4 < 4; ++r4) {
+            const float4 a4 = reinterpret_cast<const float4*>(col)[r4];
+            if (4 * r4 + 0 > s2) x[4 * r4 + 0] = fmaf(-a4.x, xv, x[4 * r4 + 0]);
+            if (4 * r4 + 1 > s2) x[4 * r4 + 1] = fmaf(-a4.y, xv, x[4 * r4 + 1]);
+            if (4 * r4 + 2 > s2) x[4 * r4 + 2] = fmaf(-a4.z, xv, x[4 * r4 + 2]);
+            if (4 * r4 + 3 > s2) x[4 * r4 + 3] = fmaf(-a4.w, xv, x[4 * r4 + 3]);
+          }
+        }
+        const float bc = betas[o + cb];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          xs[(o + r) * 32 + o + cb] = x[r];
+          tt_store(o + r, o + cb, x[r] * bc);
+          if (b == 0) tt_store(r, 16 + cb, 0.f);  // upper-right block of T is zero
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // Y = A10 X00 (rows 16..31 x columns 0..15), into the lower-left block of xs
+      const int cl = tid & 15, rp = tid >> 4;  // tid < 128 here
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = 2 * rp + h2;
+        float y = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) y = fmaf(akkt[s2 * 32 + 16 + r], xs[s2 * 32 + cl], y);
+        xs[(16 + r) * 32 + cl] = y;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // X10 = -X11 Y;  T[16 + r][c] = X10[r][c] beta_c
+      const float bcl = betas[cl];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = 2 * rp + h2;
+        float x10 = 0.f;
+#pragma unroll
+        for (int t2 = 0; t2 < 16; ++t2)
+          x10 = fmaf(xs[(16 + r) * 32 + 16 + t2], xs[(16 + t2) * 32 + cl], x10);
+        tt_store(16 + r, cl, -x10 * bcl);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ===== D: W'^T = K_L^T T^T and U~^T = V^T T^T (bf16)
+    if (tid == 0) {
+      if (!U.vzero) {
+        mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
+        ph_v ^= 1;
+        pend_v = false;
+      }
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        const uint64_t b = sw128_desc(sb + SM_TT + ks * 32, 16, 1024);
+        mma_ss(tbase + W_COL, sw128_desc(sb + SM_KQL + ks * 2048, 8192, 1024), b, id_w, 0,
+               ks > 0);
+        if (!U.vzero)
+          mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 4);
+    ph_mma ^= 1;
+    fence_after_sync();
+
+    // ===== E: W = W' Diag(e^{Gamma_15}) -> smem (lane i, column r -> W[r][i] fp32)
+    if (warp < 4) {
+      const int i = 32 * warp + lane;
+      const float e15i = reinterpret_cast<const float*>(sm + SM_E15)[i];
+      float v[32];
+      tmem_ld32(tbase + lane_base + W_COL, v);
+      wait_ld();
+      const uint32_t base = (uint32_t)(i >> 5) * 4096 + (uint32_t)((i & 31) * 4 & 15);
+      const uint32_t ck = (uint32_t)((i & 31) * 4) >> 4;
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        *reinterpret_cast<float*>(sm + SM_WF + base + r * 128 + ((ck ^ (r & 7)) << 4)) =
+            v[r] * e15i;
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    }  // c >= 0
+
+    // ===== F: U^T -= S^T W^T and O^T = S^T Qg^T, interleaved (tf32, A = S^T in TMEM);
+    //          meanwhile part 1 of the next chunk's prep
+    if (tid == 0 && c >= 0) {
+      if (has_next && !U.vzero) {
+        fence_proxy_async();
+        issue_v(c + 1);
+      }
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint32_t boff = (ks >> 2) * 4096 + (ks & 3) * 32;
+        mma_ts_tf32(tbase + U_COL, tbase + S_COL + 8 * ks, sw128_desc(sb + SM_WF + boff, 16, 1024),
+                    id_u, (ks > 0) || !U.vzero);
+        if (U.out_on)
+          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
+                      sw128_desc(sb + SM_QG + boff, 16, 1024), id_o, ks > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g (log2 units)
+      const int cc = c + 1;
+      const int n = chunk_rows(cc);
       if (tid < C) {
         betas[tid] = beta_next;
-        const int64_t t1 = (int64_t)(c + 1) * C + tid;
+        const int64_t t1 = (int64_t)(cc + 1) * C + tid;
         beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
       }
-      mbar_wait_bounded(&bars[B_IN_FULL + st], (c >> 1) & 1, abort_flag, P.sb, 1);
-      __syncwarp();
-
-      // ---- prep 1: cumulative log2-decay over the chunk (rows 4ro .. 4ro+3)
-      float4 G4[4];
-      {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
+      ph_in ^= 1;
+      if (tid == 0) pend_in = false;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = 4 * ro + rr;
-          float4 gv = *reinterpret_cast<const float4*>(in + OFF_G + (r * D + c0) * 4);
-          if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
-            gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
-            gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
-            gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
-            gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
-          } else {
-            gv.x *= kLog2e;
-            gv.y *= kLog2e;
-            gv.z *= kLog2e;
-            gv.w *= kLog2e;
-          }
-          if (r >= n) {  // tail rows act as g = 0, k = q = 0
-            gv = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<uint2*>(in + OFF_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
-            *reinterpret_cast<uint2*>(in + OFF_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
-          }
-          acc.x += gv.x;
-          acc.y += gv.y;
-          acc.z += gv.z;
-          acc.w += gv.w;
-          G4[rr] = acc;
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = 4 * ro + rr;
+        float4 gv = *reinterpret_cast<const float4*>(sm + SM_G + (r * D + c0) * 4);
+        if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
+          gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
+          gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
+          gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
+          gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
+        } else {
+          gv.x *= kLog2e;
+          gv.y *= kLog2e;
+          gv.z *= kLog2e;
+          gv.w *= kLog2e;
         }
-        reinterpret_cast<float4*>(sm + SM_TT)[ro * 32 + cq] = acc;  // 4-row group totals
+        if (r >= n) {  // tail rows act as g = 0, k = q = 0
+          gv = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<uint2*>(sm + SM_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(sm + SM_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
+        }
+        acc.x += gv.x;
+        acc.y += gv.y;
+        acc.z += gv.z;
+        acc.w += gv.w;
+        G4[rr] = acc;
       }
-      named_bar(1, 256);
+      reinterpret_cast<float4*>(sm + SM_TT)[ro * 32 + cq] = acc;  // 4-row group totals
+    }
+    __syncthreads();
+    if (c >= 0) {
+    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 5);
+    ph_mma ^= 1;
+    fence_after_sync();
 
-      // ---- prep 2: rescaled operands; hand-off buffer b is free once the state
-      //      side finished chunk c - 2
-      if (c >= 2) mbar_wait_bounded(&bars[B_SO + b], ((c - 2) >> 1) & 1, abort_flag, P.sb, 2);
-      __syncwarp();
-      {
-        const float4* tot = reinterpret_cast<const float4*>(sm + SM_TT);
-        float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
+    // ===== G: decay the state, S^T[j][i] *= e^{Gamma_C, i}
+    {
 #pragma unroll
-        for (int o8 = 0; o8 < 8; ++o8) {
-          const float4 t = tot[o8 * 32 + cq];
-          if (o8 < ro) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
-          if (o8 < 4) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
-          g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t col = S_COL + 64 * half + 32 * cc;
+        const float4* g4 = reinterpret_cast<const float4*>(gamc + 64 * half + 32 * cc);
+        float v[32];
+        tmem_ld32(tbase + lane_base + col, v);
+        wait_ld();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 gg = g4[k4];
+          v[4 * k4 + 0] *= gg.x;
+          v[4 * k4 + 1] *= gg.y;
+          v[4 * k4 + 2] *= gg.z;
+          v[4 * k4 + 3] *= gg.w;
         }
-        const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
-                                       ex2_approx(g15.w));
-        const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
-                                         ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
-        if (ro == 7) {
-          *reinterpret_cast<float4*>(sm + SM_GAMC + b * 512 + c0 * 4) = make_float4(
-              ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
-          *reinterpret_cast<float4*>(sm + SM_E15 + c0 * 4) = e15;
-        }
-        const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
-        float kc[4][4];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const int r = 4 * ro + rr;
-          float ex[4], ix[4];
-          ex[0] = ex2_approx(G4[rr].x + sh.x);
-          ex[1] = ex2_approx(G4[rr].y + sh.y);
-          ex[2] = ex2_approx(G4[rr].z + sh.z);
-          ex[3] = ex2_approx(G4[rr].w + sh.w);
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
-          const uint2 kw = *reinterpret_cast<const uint2*>(in + OFF_K + (r * D + c0) * 2);
-          const uint2 qw = *reinterpret_cast<const uint2*>(in + OFF_Q + (r * D + c0) * 2);
-          const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
-                               __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
-          const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
-                               __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
-          float kl[4], ql[4], kb[4];
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            kl[k4] = kv[k4] * ex[k4];
-            ql[k4] = qv[k4] * ex[k4];
-            kb[k4] = kv[k4] * ix[k4];
-          }
-          const uint32_t rb = rr * 128;
-          const uint32_t sw = (uint32_t)((4 * ro + rr) & 7);
-          const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
-          auto pack = [](float lo_, float hi_) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo_, hi_);
-            return *reinterpret_cast<const uint32_t*>(&b2);
-          };
-          *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + rb + s16) =
-              make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
-          *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
-              make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
-          *reinterpret_cast<uint2*>(sm + SM_KB + o_kb + rb + s16) =
-              make_uint2(pack(kb[0], kb[1]), pack(kb[2], kb[3]));
-          *reinterpret_cast<float4*>(ho + HO_QG + o_qg + rb + s32) =
-              make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
-          kc[0][rr] = kb[0] * e3115.x;
-          kc[1][rr] = kb[1] * e3115.y;
-          kc[2][rr] = kb[2] * e3115.z;
-          kc[3][rr] = kb[3] * e3115.w;
-        }
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {  // Kc^T rows c0..c0+3: one 16-byte chunk each
-          const int row = c0 + k4;
-          *reinterpret_cast<float4*>(ho + HO_KC + row * 128 + ((ro ^ (row & 7)) << 4)) =
-              make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
-        }
+        tmem_st32(tbase + lane_base + col, v);
       }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars[B_IN_EMPTY + st]);
-        mbar_arrive(&bars[B_OPER]);
-        if (warp >= 4) mbar_arrive(&bars[B_KEY + b]);  // warps 4-7 wrote their share
+      wait_st();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (*abort_flag) break;
+
+    // ===== H: S^T += U^T Kc and O^T += U^T A_qk^T (tf32, U^T from TMEM);
+    //          meanwhile part 2 of the next chunk's prep
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
+                    sw128_desc(sb + SM_KC + ks * 32, 16, 1024), id_s, 1);
+        if (U.out_on)
+          mma_ts_tf32(tbase + O_COL, tbase + U_COL + 8 * ks,
+                      sw128_desc(sb + SM_AQK + ks * 32, 16, 1024), id_o, 1);
       }
-
-      if (warp < 4) {
-        // ---- Gram accumulator -> A_kk^T (x beta) and A_qk (into buffer b)
-        mbar_wait_bounded(&bars[B_GRAM], c & 1, abort_flag, P.sb, 3);
-        __syncwarp();
-        fence_after_sync();
-        {
-          float v[32];
-          tmem_ld32(tbase + lane_base + G_COL, v);
-          wait_ld();
-          if (lane < 16) {
-            const int r = 16 * (warp & 1) + lane;
-            if (warp < 2) {
-              const float br = betas[r];
-              float* akkt = reinterpret_cast<float*>(sm + SM_AKKT);
+      mma_commit(bar_mma);
+    }
+    }  // c >= 0
+    if (has_next) {  // prep, part 2: rescaled operands (Kc kept in registers)
+      const float4* tot = reinterpret_cast<const float4*>(sm + SM_TT);
+      float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
 #pragma unroll
-              for (int s2 = 0; s2 < 32; ++s2) akkt[s2 * 32 + r] = s2 < r ? br * v[s2] : 0.f;
-            } else {
+      for (int o8 = 0; o8 < 8; ++o8) {
+        const float4 t = tot[o8 * 32 + cq];
+        if (o8 < ro) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
+        if (o8 < 4) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
+        g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
+      }
+      const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
+                                     ex2_approx(g15.w));
+      const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
+                                       ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
+      if (ro == 7) {
+        *reinterpret_cast<float4*>(gamc + c0) = make_float4(
+            ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
+        *reinterpret_cast<float4*>(sm + SM_E15 + c0 * 4) = e15;
+      }
+      // G4[rr] - g15 + off: exponent of e^{Gamma_r - Gamma_15} in log2 units
+      const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
 #pragma unroll
-              for (int s4 = 0; s4 < 8; ++s4) {
-                float4 w4;
-                w4.x = (4 * s4 + 0 <= r) ? v[4 * s4 + 0] : 0.f;
-                w4.y = (4 * s4 + 1 <= r) ? v[4 * s4 + 1] : 0.f;
-                w4.z = (4 * s4 + 2 <= r) ? v[4 * s4 + 2] : 0.f;
-                w4.w = (4 * s4 + 3 <= r) ? v[4 * s4 + 3] : 0.f;
-                *reinterpret_cast<float4*>(ho + HO_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
-              }
-            }
-          }
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = 4 * ro + rr;
+        float ex[4], ix[4];
+        ex[0] = ex2_approx(G4[rr].x + sh.x);
+        ex[1] = ex2_approx(G4[rr].y + sh.y);
+        ex[2] = ex2_approx(G4[rr].z + sh.z);
+        ex[3] = ex2_approx(G4[rr].w + sh.w);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
+        const uint2 kw = *reinterpret_cast<const uint2*>(sm + SM_K + (r * D + c0) * 2);
+        const uint2 qw = *reinterpret_cast<const uint2*>(sm + SM_Q + (r * D + c0) * 2);
+        const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
+                             __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
+        const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
+                             __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
+        float kl[4], ql[4], kb[4];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          kl[k4] = kv[k4] * ex[k4];
+          ql[k4] = qv[k4] * ex[k4];
+          kb[k4] = kv[k4] * ix[k4];
         }
-        fence_proxy_async();
-        __syncwarp();
-        named_bar(2, 128);
-
-        // ---- T = (I + A_kk)^-1 Diag(beta), blocked 2 x 2 over 16-row blocks
-        const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
-        float* xs = reinterpret_cast<float*>(sm + SM_XS);
-        auto tt_store = [&](int r, int col, float val) {
-          *reinterpret_cast<__nv_bfloat16*>(
-              sm + SM_TT + r * 128 + ((((uint32_t)(col * 2) >> 4) ^ (uint32_t)(r & 7)) << 4) +
-              ((col * 2) & 15)) = __float2bfloat16_rn(val);
+        const uint32_t rb = rr * 128;
+        const uint32_t sw = (uint32_t)((4 * ro + rr) & 7);
+        const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
+        auto pack = [](float lo, float hi) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
+          return *reinterpret_cast<const uint32_t*>(&b2);
         };
-        if (warp == 0) {  // diagonal blocks: lane = (block bb, column cb)
-          const int bb = lane >> 4, cb = lane & 15, o = 16 * bb;
-          float x[16];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) x[r] = (r == cb) ? 1.f : 0.f;
-#pragma unroll
-          for (int s2 = 0; s2 < 15; ++s2) {
-            const float xv = x[s2];
-            const float* col = akkt + (o + s2) * 32 + o;  // A[o + r][o + s2], r = 0..15
-#pragma unroll
-            for (int r4 = (s2 + 1) / 4; r4 < 4; ++r4) {
-              const float4 a4 = reinterpret_cast<const float4*>(col)[r4];
-              if (4 * r4 + 0 > s2) x[4 * r4 + 0] = fmaf(-a4.x, xv, x[4 * r4 + 0]);
-              if (4 * r4 + 1 > s2) x[4 * r4 + 1] = fmaf(-a4.y, xv, x[4 * r4 + 1]);
-              if (4 * r4 + 2 > s2) x[4 * r4 + 2] = fmaf(-a4.z, xv, x[4 * r4 + 2]);
-              if (4 * r4 + 3 > s2) x[4 * r4 + 3] = fmaf(-a4.w, xv, x[4 * r4 + 3]);
-            }
-          }
-          const float bc = betas[o + cb];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            xs[(o + r) * 32 + o + cb] = x[r];
-            tt_store(o + r, o + cb, x[r] * bc);
-            if (bb == 0) tt_store(r, 16 + cb, 0.f);  // upper-right block of T is zero
-          }
-        }
-        __syncwarp();
-        named_bar(2, 128);
-        const int cl = tid & 15, rp = tid >> 4;  // tid < 128
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {  // Y = A10 X00 into the lower-left block of xs
-          const int r = 2 * rp + h2;
-          float y = 0.f;
-#pragma unroll
-          for (int s2 = 0; s2 < 16; ++s2) y = fmaf(akkt[s2 * 32 + 16 + r], xs[s2 * 32 + cl], y);
-          xs[(16 + r) * 32 + cl] = y;
-        }
-        named_bar(2, 128);
-        const float bcl = betas[cl];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {  // X10 = -X11 Y
-          const int r = 2 * rp + h2;
-          float x10 = 0.f;
-#pragma unroll
-          for (int t2 = 0; t2 < 16; ++t2)
-            x10 = fmaf(xs[(16 + r) * 32 + 16 + t2], xs[(16 + t2) * 32 + cl], x10);
-          tt_store(16 + r, cl, -x10 * bcl);
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_T]);
+        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + rb + s16) =
+            make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
+        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
+            make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
+        *reinterpret_cast<uint2*>(sm + SM_KB + o_kb + rb + s16) =
+            make_uint2(pack(kb[0], kb[1]), pack(kb[2], kb[3]));
+        *reinterpret_cast<float4*>(sm + SM_QG + o_qg + rb + s32) =
+            make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
+        kc[0][rr] = kb[0] * e3115.x;
+        kc[1][rr] = kb[1] * e3115.y;
+        kc[2][rr] = kb[2] * e3115.z;
+        kc[3][rr] = kb[3] * e3115.w;
       }
+    }
+    if (c >= 0) {
+      mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
+      ph_mma ^= 1;
+      fence_after_sync();
+    }
+    if (has_next) {  // Kc^T rows c0..c0+3: this thread's 4 rows are one 16-byte chunk of each
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int row = c0 + k4;
+        *reinterpret_cast<float4*>(sm + SM_KC + row * 128 + ((ro ^ (row & 7)) << 4)) =
+            make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
+      }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && c + 2 < nchunks) {
+      fence_proxy_async();
+      issue_qkg(c + 2);
+    }
+  }
+  __syncthreads();
+  if (nchunks > 0 && U.out_on && warp >= 4 && !*abort_flag) export_o(nchunks - 1);
+  fence_before_sync();
+  __syncthreads();
 
-      // ---- W = W' Diag(e^{Gamma_15}) into buffer b (lane i, column r -> W[r][i])
-      mbar_wait_bounded(&bars[B_WU], c & 1, abort_flag, P.sb, 4);
-      __syncwarp();
-      fence_after_sync();
-      if (warp < 4) {
-        const int i = 32 * warp + lane;
-        const float e15i = reinterpret_cast<const float*>(sm + SM_E15)[i];
-        float v[32];
-        tmem_ld32(tbase + lane_base + W_COL, v);
-        wait_ld();
-        const uint32_t base = (uint32_t)(i >> 5) * 4096 + (uint32_t)((i & 31) * 4 & 15);
-        const uint32_t ck = (uint32_t)((i & 31) * 4) >> 4;
+  // ---- final state (S^T lane j, column i -> final[i][j])
+  if (U.final_state && !*abort_flag) {
+    const int j = 32 * (warp & 3) + lane;
 #pragma unroll
-        for (int r = 0; r < 32; ++r)
-          *reinterpret_cast<float*>(ho + HO_WF + base + r * 128 + ((ck ^ (r & 7)) << 4)) =
-              v[r] * e15i;
-        fence_proxy_async();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_KEY + b]);
-      }
+    for (int cc = 0; cc < 2; ++cc) {
+      const int i0 = 64 * half + 32 * cc;
+      float v[32];
+      tmem_ld32(tbase + lane_base + S_COL + i0, v);
+      wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) U.final_state[(size_t)(i0 + k) * D + j] = v[k];
     }
-  } else if (warp < ISSUE_WARP) {
-    // ====================================================== state-side warps
-    for (int c = 0; c < nchunks; ++c) {
-      if (bar_red_or(3, 128, *abort_flag != 0)) break;
-      const int b = c & 1;
-      mbar_wait_bounded(&bars[B_UO], c & 1, abort_flag, P.sb, 5);
-      __syncwarp();
-      fence_after_sync();
-      {  // S^T[j][i] *= e^{Gamma_C, i}
-        const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + b * 512);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          tmem_ld32(tbase + lane_base + S_COL + 32 * cc, v);
-          wait_ld();
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 gg = g4[8 * cc + k4];
-            v[4 * k4 + 0] *= gg.x;
-            v[4 * k4 + 1] *= gg.y;
-            v[4 * k4 + 2] *= gg.z;
-            v[4 * k4 + 3] *= gg.w;
-          }
-          tmem_st32(tbase + lane_base + S_COL + 32 * cc, v);
-        }
-        wait_st();
-      }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_DECAY]);
-
-      mbar_wait_bounded(&bars[B_SO + b], (c >> 1) & 1, abort_flag, P.sb, 6);
-      __syncwarp();
-      fence_after_sync();
-      if (U.out_on) {  // O^T (lane j, column r) -> o; lanes j, j^1 write bf16 pairs
-        const int n = chunk_rows(c);
-        const int j = 32 * (warp & 3) + lane;
-        const bool odd = lane & 1;
-        float v[32];
-        tmem_ld32(tbase + lane_base + O_COL, v);
-        wait_ld();
-        const int jp = j & ~1;
-        __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + (int64_t)c * C) * H + h) * D + jp;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float send = odd ? v[2 * m] : v[2 * m + 1];
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-          const int r = 2 * m + (odd ? 1 : 0);
-          const float lo = odd ? recv : v[2 * m];
-          const float hi = odd ? v[2 * m + 1] : recv;
-          if (r < n)
-            *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
-                __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
-        }
-      }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_OFREE]);
-    }
-    // final state (S^T lane j, column i -> final[i][j]); all S GEMMs are done
-    if (U.final_state && !*abort_flag) {
-      const int j = 32 * (warp & 3) + lane;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(tbase + lane_base + S_COL + 32 * cc, v);
-        wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) U.final_state[(size_t)(32 * cc + k) * D + j] = v[k];
-      }
-    }
-  } else {
-    // =============================================== MMA and TMA issue (lane 0)
-    if (lane == 0) {
-    const uint32_t id_gram = idesc(kFmtBF16, 64, C, false, false, false);
-    const uint32_t id_w = idesc(kFmtBF16, 128, C, true, false, false);
-    const uint32_t id_o = idesc(kFmtTF32, 128, C, false, false, false);
-    const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
-    const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
-    int nq = 0, nv = U.vzero ? nchunks : 0, ng = 0, nw = 0, nu = 0, ns = 0;
-    unsigned long long t_last = global_ns();
-    while (ns < nchunks) {
-      bool progress = false;
-      if (*abort_flag) break;
-      // TMA: q, k, g of chunk nq into stage nq & 1 (free once chunk nq - 2 is prepared)
-      if (nq < nchunks &&
-          (nq < 2 || mbar_test(&bars[B_IN_EMPTY + (nq & 1)], ((nq - 2) >> 1) & 1))) {
-        const int row = (int)(U.row0 + (int64_t)nq * C);
-        uint8_t* in = sm + (nq & 1) * STAGE;
-        uint64_t* bf = &bars[B_IN_FULL + (nq & 1)];
-        fence_proxy_async();
-        mbar_arrive_expect_tx(bf, TX_QKG);
-        tma_load_3d(in + OFF_Q, &P.tm_q, bf, 0, h, row);
-        tma_load_3d(in + OFF_K, &P.tm_k, bf, 0, h, row);
-        tma_load_3d(in + OFF_G, &P.tm_g, bf, 0, h, row);
-        ++nq;
-        progress = true;
-      }
-      // TMA: v of chunk nv (stage free once the U~ GEMM of chunk nv - 2 is done)
-      if (nv < nchunks &&
-          (nv < 2 || mbar_test(&bars[B_V_EMPTY + (nv & 1)], ((nv - 2) >> 1) & 1))) {
-        const int row = (int)(U.row0 + (int64_t)nv * C);
-        uint8_t* in = sm + (nv & 1) * STAGE;
-        uint64_t* bf = &bars[B_V_FULL + (nv & 1)];
-        mbar_arrive_expect_tx(bf, TX_V);
-        tma_load_3d(in + OFF_V, &P.tm_v, bf, 0, h, row);
-        tma_load_3d(in + OFF_V + 4096, &P.tm_v, bf, 64, h, row);
-        ++nv;
-        progress = true;
-      }
-      // Gram GEMM of chunk ng: [K_L; Q_L] K_B^T (bf16, M64 N32 K128)
-      if (ng < nchunks && mbar_test(&bars[B_OPER], ng & 1)) {
-        fence_after_sync();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t kb = ks >> 2, kk = ks & 3;
-          mma_ss(tbase + G_COL, sw128_desc(sb + SM_KQL + kb * 8192 + kk * 32, 16, 1024),
-                 sw128_desc(sb + SM_KB + kb * 4096 + kk * 32, 16, 1024), id_gram, 0, ks > 0);
-        }
-        mma_commit(&bars[B_GRAM]);
-        ++ng;
-        progress = true;
-      }
-      // W'^T = K_L^T T^T and U~^T = V^T T^T of chunk nw (bf16)
-      if (nw < ng && mbar_test(&bars[B_T], nw & 1) &&
-          (U.vzero || mbar_test(&bars[B_V_FULL + (nw & 1)], (nw >> 1) & 1))) {
-        fence_after_sync();
-        const uint32_t vs = sb + (nw & 1) * STAGE + OFF_V;
-        const uint32_t ucol = U_COL + 32 * (nw & 1);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const uint64_t bd = sw128_desc(sb + SM_TT + ks * 32, 16, 1024);
-          mma_ss(tbase + W_COL, sw128_desc(sb + SM_KQL + ks * 2048, 8192, 1024), bd, id_w, 0,
-                 ks > 0);
-          if (!U.vzero)
-            mma_ss(tbase + ucol, sw128_desc(vs + ks * 2048, 4096, 1024), bd, id_w, 0, ks > 0);
-        }
-        mma_commit(&bars[B_WU]);
-        if (!U.vzero) mma_commit(&bars[B_V_EMPTY + (nw & 1)]);
-        ++nw;
-        progress = true;
-      }
-      // U^T -= S^T W^T and O^T = S^T Qg^T of chunk nu (tf32, A = S^T in TMEM),
-      // after the previous chunk's state update and output export
-      if (nu < nw && nu == ns && mbar_test(&bars[B_KEY + (nu & 1)], (nu >> 1) & 1) &&
-          (nu == 0 || mbar_test(&bars[B_OFREE], (nu - 1) & 1))) {
-        fence_after_sync();
-        const uint32_t hob = sb + SM_HO + (nu & 1) * HO;
-        const uint32_t ucol = U_COL + 32 * (nu & 1);
-#pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {
-          const uint32_t boff = (ks >> 2) * 4096 + (ks & 3) * 32;
-          mma_ts_tf32(tbase + ucol, tbase + S_COL + 8 * ks,
-                      sw128_desc(hob + HO_WF + boff, 16, 1024), id_u, (ks > 0) || !U.vzero);
-          if (U.out_on)
-            mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
-                        sw128_desc(hob + HO_QG + boff, 16, 1024), id_o, ks > 0);
-        }
-        mma_commit(&bars[B_UO]);
-        ++nu;
-        progress = true;
-      }
-      // S^T += U^T Kc and O^T += U^T A_qk^T of chunk ns, after the decay
-      if (ns < nu && mbar_test(&bars[B_DECAY], ns & 1)) {
-        fence_after_sync();
-        const uint32_t hob = sb + SM_HO + (ns & 1) * HO;
-        const uint32_t ucol = U_COL + 32 * (ns & 1);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_ts_tf32(tbase + S_COL, tbase + ucol + 8 * ks,
-                      sw128_desc(hob + HO_KC + ks * 32, 16, 1024), id_s, 1);
-          if (U.out_on)
-            mma_ts_tf32(tbase + O_COL, tbase + ucol + 8 * ks,
-                        sw128_desc(hob + HO_AQK + ks * 32, 16, 1024), id_o, 1);
-        }
-        mma_commit(&bars[B_SO + (ns & 1)]);
-        ++ns;
-        progress = true;
-      }
-      if (progress) {
-        t_last = global_ns();
-      } else if ((long long)(global_ns() - t_last) > kWaitLimitNs) {
-        *abort_flag = 1;
-        record_status(P.sb, KDA_ERR_TIMEOUT, 7);
-        break;
-      }
-    }
-    if (*abort_flag) {
-      // let every GEMM and TMA load issued so far finish before memory is released
-      mma_commit(&bars[B_DRAIN]);
-      mbar_wait_bounded(&bars[B_DRAIN], 0, abort_flag, nullptr, 8);
-      for (int k = (nq > 2 ? nq - 2 : 0); k < nq; ++k)
-        mbar_wait_bounded(&bars[B_IN_FULL + (k & 1)], (k >> 1) & 1, abort_flag, nullptr, 9);
-      if (!U.vzero)
-        for (int k = (nv > 2 ? nv - 2 : 0); k < nv; ++k)
-          mbar_wait_bounded(&bars[B_V_FULL + (k & 1)], (k >> 1) & 1, abort_flag, nullptr, 10);
-    }
-    }
-    __syncwarp();
   }
   fence_before_sync();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    // let any TMA load still in flight land before the CTA's memory is released
+    if (pend_in) mbar_wait_bounded(bar_in, ph_in, abort_flag, nullptr, 7);
+    if (pend_v) mbar_wait_bounded(bar_v, ph_v, abort_flag, nullptr, 8);
+  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tbase, TMEM_COLS);
 }
@@ -787,13 +743,11 @@ bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base
 // Segment split for long dense sequences with too few (sequence, head)
 // units to occupy the GPU: returns G >= 2 and the segment length, or G = 1.
 void plan_split(int B, int T, int H, int num_sms, int* G_out, int* seg_out) {
-  // one CTA per SM: split when the units fill less than half the SMs, into
-  // as many segments as keep one unit-segment per SM
   const int U = B * H;
   *G_out = 1;
   *seg_out = T;
   if (2 * U >= num_sms || T < 4 * 1024) return;
-  int G = num_sms / U;
+  int G = (2 * num_sms + U - 1) / U;
   const int max_g = T / 1024;
   if (G > max_g) G = max_g;
   if (G < 2) return;
