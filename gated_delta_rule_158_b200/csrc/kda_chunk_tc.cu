@@ -9,9 +9,11 @@
 // from state S, with Gamma_r the in-chunk cumulative sum of g:
 //   L[r,s] = sum_i k_ri k_si e^{Gamma_ri - Gamma_si}          (Gram, s <= r)
 //   T      = (I + Diag(b) strict_lower(L))^-1 Diag(b)
-//   W      = T (k e^Gamma),   U = T V - W S,
+//   P      = (k e^Gamma) S,   U = T V - T P,
 //   O      = (q e^Gamma) S + lower(Lq) U,
 //   S     <- Diag(e^{Gamma_C}) S + (k e^{Gamma_C - Gamma})^T U.
+// (T P is the W S of the WY form with W = T (k e^Gamma), associated the other
+// way so that no W has to be formed.)
 //
 // Why C = 32 and one rebasing point.  The lower bound g >= -5 of the gate
 // (same section, Lower-bounded decay) is what lets every Gram tile,
@@ -22,16 +24,22 @@
 // would need more than one rebasing point per tile.
 //
 // B200 mapping.  One CTA (256 threads) owns one (sequence, head) for its
-// whole length; two CTAs share an SM (112 KB shared memory, 256 TMEM columns
-// each).  The fp32 state never leaves the SM: it lives in TMEM as S^T (lane =
-// value channel, column = key channel) and is read directly as the tf32 A
-// operand of the state-side GEMMs (U -= S^T W^T, O = S^T Q^T, S^T += U^T Kc),
-// with U^T also consumed straight from TMEM.  The key-side GEMMs (Gram,
-// W = T Ka, U~ = T V) are bf16.  TMA brings q/k/g (and separately v) for the
-// next chunk while the current one computes.  All MMAs are issued by one
-// thread and tracked by mbarriers; every wait is bounded (kda_sync.cuh).
+// whole length; two CTAs share an SM (110 KB shared memory, 256 TMEM columns
+// each), so one CTA's SIMT phases overlap the other's GEMMs.  The fp32 state
+// never leaves the SM: it lives in TMEM as S^T (lane = value channel, column =
+// key channel) and is read directly as the tf32 A operand of the state-side
+// GEMMs.  tcgen05.mma costs a roughly fixed number of cycles per instruction
+// up to N = 128-256 (measured: ~90 with A in TMEM, ~190 with A in shared
+// memory), so products that share an A operand are fused into one wide MMA:
+//   [O^T | P^T]  = S^T [q e^G ; k e^G]^T            (N = 64, 16 k-steps)
+//   U^T         -= P^T T^T   onto  U^T = V^T T^T     (N = 32)
+//   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay (N = 160, 4 k-steps)
+// The Gram and U~ = T V are bf16 (A in shared memory).  TMA brings q/k/g for
+// the next chunk while the current one computes, and v into the Gram operand
+// region once the Gram is done.  All MMAs are issued by one thread and
+// tracked by mbarriers; every wait is bounded (kda_sync.cuh).
 //
-// TMEM columns: S^T [0,128) | U^T [128,160) | W^T [160,192) | O^T [192,224)
+// TMEM columns: S^T [0,128) | O^T [128,160) | P^T [160,192) | U^T [192,224)
 //               | Gram (M = 64 layout, lanes 0-15 of each quarter) [224,256)
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -49,34 +57,36 @@ constexpr int C = 32;     // tokens per chunk
 constexpr int D = 128;    // dk = dv
 constexpr int NT = 256;   // threads per CTA
 
-constexpr uint32_t S_COL = 0, U_COL = 128, W_COL = 160, O_COL = 192, G_COL = 224;
+constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192, G_COL = 224;
 constexpr uint32_t TMEM_COLS = 256;
 
 // shared memory map (byte offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q = 0;         // q tile  bf16 [32][128] row-major (TMA, no swizzle)
 constexpr uint32_t SM_K = 8192;      // k tile  bf16 [32][128]
-constexpr uint32_t SM_V = 16384;     // v tile  bf16, 2 x [32 rows x 128 B] swizzled (TMA)
-constexpr uint32_t SM_G = 24576;     // g (or z) tile fp32 [32][128]
-constexpr uint32_t SM_R1 = 40960;    // 24 KB, two lives:
-constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128: Gram A, and
-                                              //  (rows 0-31) the MN-major A of W' = T K_L
+constexpr uint32_t SM_G = 16384;     // g (or z) tile fp32 [32][128]; 4-row cumsum totals in prep
+constexpr uint32_t SM_R1 = 32768;    // 24 KB, two lives:
+constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128 (Gram A)
 constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
-constexpr uint32_t SM_WF = SM_R1;             //  W                fp32 32 x 128 (tf32 B)
+                                              // and once the Gram GEMM is done:
+constexpr uint32_t SM_TT = SM_R1;             //  T      bf16 [r][s] (B of U~)
+constexpr uint32_t SM_TF = SM_R1 + 4096;      //  T      fp32 [r][s] (tf32 B of U -= P^T T^T)
+constexpr uint32_t SM_V = SM_R1 + 8192;       //  v tile bf16, 2 x [32 rows x 128 B] swizzled (TMA)
 constexpr uint32_t SM_AKKT = SM_R1 + 16384;   //  A_kk^T fp32 [s][r] 32 x 32 (inverse input)
 constexpr uint32_t SM_XS = SM_R1 + 20480;     //  inverse blocks X00, X11 and A10 X00, fp32 32 x 32
-constexpr uint32_t SM_TT = 65536;    // T            bf16 [r][s] (B of W' and U~); cumsum partials during prep
-constexpr uint32_t SM_QG = 69632;    // q e^G        fp32 [r][i] (tf32 B of O)
-constexpr uint32_t SM_KC = 86016;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S)
-constexpr uint32_t SM_AQK = 102400;  // A_qk         fp32 [r][s] 32 x 32 (tf32 B of O)
-constexpr uint32_t SM_MISC = 106496;
+constexpr uint32_t SM_QK = 57344;    // [q e^G ; k e^G] fp32, per 32-channel block 64 rows x 128 B
+                                     // (tf32 B of [O | P])
+constexpr uint32_t SM_KC = 90112;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S), rows 0-127,
+constexpr uint32_t SM_AQK = 106496;  // A_qk         fp32 [r][s], rows 128-159 of the same B tile
+constexpr uint32_t SM_MISC = 110592;
 constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
-constexpr uint32_t SM_E15 = SM_MISC + 512;     // e^{Gamma_15} fp32 [128]
-constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta         fp32 [32]
-constexpr uint32_t SM_BAR = SM_MISC + 1152;    // 3 mbarriers
-constexpr uint32_t SM_TMEM = SM_MISC + 1184;   // TMEM base address
-constexpr uint32_t SM_ABORT = SM_MISC + 1188;  // abort flag
-constexpr uint32_t SMEM_BYTES = SM_MISC + 2048;
+constexpr uint32_t SM_BETA = SM_MISC + 512;    // beta         fp32 [32]
+constexpr uint32_t SM_BAR = SM_MISC + 640;     // 5 mbarriers
+constexpr uint32_t SM_TMEM = SM_MISC + 680;    // TMEM base address
+constexpr uint32_t SM_ABORT = SM_MISC + 684;   // abort flag
+constexpr uint32_t SMEM_BYTES = SM_MISC + 1024;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to 1024
+static_assert(SM_AQK == SM_KC + 16384, "A_qk rows must follow the Kc^T rows");
+static_assert(2 * (SMEM_ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 
 constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
 constexpr uint32_t TX_V = 8192;
@@ -175,6 +185,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + SM_BAR);
   uint64_t* bar_v = bar_in + 1;
   uint64_t* bar_mma = bar_in + 2;
+  uint64_t* bar_u = bar_in + 3;      // U -= P^T T^T done
+  uint64_t* bar_drain = bar_in + 4;  // abort path: every MMA issued so far done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_ABORT);
   float* gamc = reinterpret_cast<float*>(sm + SM_GAMC);
@@ -185,6 +197,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     mbar_init(bar_in, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_u, 1);
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -210,16 +224,21 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     tma_load_3d(sm + SM_G, &P.tm_g, bar_in, 0, h, row);
     pend_in = true;
   };
-  auto issue_v = [&](int c) {
+  auto issue_v = [&](int c) {  // into the Gram operand region: only once the Gram is done
     const int row = (int)(U.row0 + (int64_t)c * C);
     mbar_arrive_expect_tx(bar_v, TX_V);
     tma_load_3d(sm + SM_V, &P.tm_v, bar_v, 0, h, row);
     tma_load_3d(sm + SM_V + 4096, &P.tm_v, bar_v, 64, h, row);
     pend_v = true;
   };
+  auto prefetch_v = [&](int c) {
+    const int row = (int)(U.row0 + (int64_t)c * C);
+    tma_prefetch_3d(&P.tm_v, 0, h, row);
+    tma_prefetch_3d(&P.tm_v, 64, h, row);
+  };
   if (tid == 0 && nchunks > 0) {
     issue_qkg(0);
-    if (!U.vzero) issue_v(0);
+    if (!U.vzero) prefetch_v(0);
   }
 
   // ---- initial state -> TMEM (S^T: lane j, column i)
@@ -241,12 +260,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   fence_before_sync();
   __syncthreads();
 
-  uint32_t ph_in = 0, ph_v = 0, ph_mma = 0;
+  uint32_t ph_in = 0, ph_v = 0, ph_mma = 0, ph_u = 0;
   const uint32_t id_gram = idesc(kFmtBF16, 64, C, false, false, false);
-  const uint32_t id_w = idesc(kFmtBF16, 128, C, true, false, false);
-  const uint32_t id_o = idesc(kFmtTF32, 128, C, false, false, false);
-  const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);
-  const uint32_t id_s = idesc(kFmtTF32, 128, D, false, false, false);
+  const uint32_t id_tv = idesc(kFmtBF16, 128, C, true, false, false);        // U~^T = V^T T^T
+  const uint32_t id_op = idesc(kFmtTF32, 128, 2 * C, false, false, false);   // [O^T | P^T]
+  const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);         // U^T -= P^T T^T
+  const uint32_t id_so = idesc(kFmtTF32, 128, D + C, false, false, false);   // [S^T | O^T]
 
   // prep thread mapping: channels c0 .. c0+3 and rows 4ro .. 4ro+3 (warp ro)
   const int cq = tid & 31, ro = tid >> 5, c0 = 4 * cq;
@@ -256,7 +275,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                                 // fp32 tiles
   const uint32_t o_kql = (c0 >> 6) * 8192 + ro * 512 + lo16;
   const uint32_t o_kb = (c0 >> 6) * 4096 + ro * 512 + lo16;
-  const uint32_t o_qg = (c0 >> 5) * 4096 + ro * 512;
+  const uint32_t o_qk = (c0 >> 5) * 8192 + ro * 512;
   constexpr float kLog2e = 1.4426950408889634f;
   const float gmin2 = P.g_min * kLog2e;
   auto chunk_rows = [&](int cc) -> int {
@@ -320,6 +339,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 2);
     ph_mma ^= 1;
     fence_after_sync();
+    if (tid == 0 && !U.vzero && !*abort_flag) issue_v(c);  // the Gram operands are dead now
 
     // ===== B: A_kk (transposed, x beta) and A_qk from the Gram accumulator
     if (warp < 4) {
@@ -355,10 +375,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     if (warp < 4) {
       const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
       float* xs = reinterpret_cast<float*>(sm + SM_XS);
-      auto tt_store = [&](int r, int col, float val) {
+      auto tt_store = [&](int r, int col, float val) {  // bf16 and fp32 copies of T[r][col]
         *reinterpret_cast<__nv_bfloat16*>(
             sm + SM_TT + r * 128 + ((((uint32_t)(col * 2) >> 4) ^ (uint32_t)(r & 7)) << 4) +
             ((col * 2) & 15)) = __float2bfloat16_rn(val);
+        *reinterpret_cast<float*>(
+            sm + SM_TF + r * 128 + ((((uint32_t)(col * 4) >> 4) ^ (uint32_t)(r & 7)) << 4) +
+            ((col * 4) & 15)) = val;
       };
       if (warp == 0) {  // diagonal blocks: lane = (block b, column cb)
         const int b = lane >> 4, cb = lane & 15, o = 16 * b;
@@ -414,7 +437,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ===== D: W'^T = K_L^T T^T and U~^T = V^T T^T (bf16)
+    // ===== D: U~^T = V^T T^T (bf16) and [O^T | P^T] = S^T [Qg ; Ka]^T (tf32, A = S^T
+    //          in TMEM); meanwhile part 1 of the next chunk's prep
     if (tid == 0) {
       if (!U.vzero) {
         mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
@@ -422,60 +446,21 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
         pend_v = false;
       }
       fence_after_sync();
+      if (!U.vzero) {
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const uint64_t b = sw128_desc(sb + SM_TT + ks * 32, 16, 1024);
-        mma_ss(tbase + W_COL, sw128_desc(sb + SM_KQL + ks * 2048, 8192, 1024), b, id_w, 0,
-               ks > 0);
-        if (!U.vzero)
-          mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024), b, id_w, 0, ks > 0);
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024),
+                 sw128_desc(sb + SM_TT + ks * 32, 16, 1024), id_tv, 0, ks > 0);
       }
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks)
+        mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
+                    sw128_desc(sb + SM_QK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_op,
+                    ks > 0);
       mma_commit(bar_mma);
     }
-    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 4);
-    ph_mma ^= 1;
-    fence_after_sync();
-
-    // ===== E: W = W' Diag(e^{Gamma_15}) -> smem (lane i, column r -> W[r][i] fp32)
-    if (warp < 4) {
-      const int i = 32 * warp + lane;
-      const float e15i = reinterpret_cast<const float*>(sm + SM_E15)[i];
-      float v[32];
-      tmem_ld32(tbase + lane_base + W_COL, v);
-      wait_ld();
-      const uint32_t base = (uint32_t)(i >> 5) * 4096 + (uint32_t)((i & 31) * 4 & 15);
-      const uint32_t ck = (uint32_t)((i & 31) * 4) >> 4;
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        *reinterpret_cast<float*>(sm + SM_WF + base + r * 128 + ((ck ^ (r & 7)) << 4)) =
-            v[r] * e15i;
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (*abort_flag) break;
-
     }  // c >= 0
 
-    // ===== F: U^T -= S^T W^T and O^T = S^T Qg^T, interleaved (tf32, A = S^T in TMEM);
-    //          meanwhile part 1 of the next chunk's prep
-    if (tid == 0 && c >= 0) {
-      if (has_next && !U.vzero) {
-        fence_proxy_async();
-        issue_v(c + 1);
-      }
-      fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-        const uint32_t boff = (ks >> 2) * 4096 + (ks & 3) * 32;
-        mma_ts_tf32(tbase + U_COL, tbase + S_COL + 8 * ks, sw128_desc(sb + SM_WF + boff, 16, 1024),
-                    id_u, (ks > 0) || !U.vzero);
-        if (U.out_on)
-          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
-                      sw128_desc(sb + SM_QG + boff, 16, 1024), id_o, ks > 0);
-      }
-      mma_commit(bar_mma);
-    }
     if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g (log2 units)
       const int cc = c + 1;
       const int n = chunk_rows(cc);
@@ -514,7 +499,9 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
         acc.w += gv.w;
         G4[rr] = acc;
       }
-      reinterpret_cast<float4*>(sm + SM_TT)[ro * 32 + cq] = acc;  // 4-row group totals
+      // 4-row group total, over the g values of (row 4ro, channels c0..c0+3) that
+      // only this thread reads
+      *reinterpret_cast<float4*>(sm + SM_G + (4 * ro * D + c0) * 4) = acc;
     }
     __syncthreads();
     if (c >= 0) {
@@ -522,7 +509,15 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     ph_mma ^= 1;
     fence_after_sync();
 
-    // ===== G: decay the state, S^T[j][i] *= e^{Gamma_C, i}
+    // ===== G: U^T -= P^T T^T (tf32, A = P^T in TMEM, onto U~^T), issued once P is
+    //          complete; meanwhile decay the state, S^T[j][i] *= e^{Gamma_C, i}
+    if (tid == 0) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_ts_tf32(tbase + U_COL, tbase + P_COL + 8 * ks,
+                    sw128_desc(sb + SM_TF + ks * 32, 16, 1024), id_u, (ks > 0) || !U.vzero);
+      mma_commit(bar_u);
+    }
     {
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -547,27 +542,26 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
     __syncthreads();
     if (*abort_flag) break;
 
-    // ===== H: S^T += U^T Kc and O^T += U^T A_qk^T (tf32, U^T from TMEM);
-    //          meanwhile part 2 of the next chunk's prep
+    // ===== H: [S^T | O^T] += U^T [Kc ; A_qk^T] (tf32, U^T from TMEM, one N = 160 MMA
+    //          per k-step); meanwhile part 2 of the next chunk's prep
+    // U is also the last reader of T in the Gram operand region, which part 2
+    // of the prep overwrites: everyone waits for it
+    mbar_wait_bounded(bar_u, ph_u, abort_flag, P.sb, 9);
+    ph_u ^= 1;
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
+      for (int ks = 0; ks < 4; ++ks)
         mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
-                    sw128_desc(sb + SM_KC + ks * 32, 16, 1024), id_s, 1);
-        if (U.out_on)
-          mma_ts_tf32(tbase + O_COL, tbase + U_COL + 8 * ks,
-                      sw128_desc(sb + SM_AQK + ks * 32, 16, 1024), id_o, 1);
-      }
+                    sw128_desc(sb + SM_KC + ks * 32, 16, 1024), id_so, 1);
       mma_commit(bar_mma);
     }
     }  // c >= 0
     if (has_next) {  // prep, part 2: rescaled operands (Kc kept in registers)
-      const float4* tot = reinterpret_cast<const float4*>(sm + SM_TT);
       float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
 #pragma unroll
       for (int o8 = 0; o8 < 8; ++o8) {
-        const float4 t = tot[o8 * 32 + cq];
+        const float4 t = *reinterpret_cast<const float4*>(sm + SM_G + (4 * o8 * D + c0) * 4);
         if (o8 < ro) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
         if (o8 < 4) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
         g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
@@ -579,7 +573,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       if (ro == 7) {
         *reinterpret_cast<float4*>(gamc + c0) = make_float4(
             ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
-        *reinterpret_cast<float4*>(sm + SM_E15 + c0 * 4) = e15;
       }
       // G4[rr] - g15 + off: exponent of e^{Gamma_r - Gamma_15} in log2 units
       const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
@@ -619,8 +612,10 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
             make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
         *reinterpret_cast<uint2*>(sm + SM_KB + o_kb + rb + s16) =
             make_uint2(pack(kb[0], kb[1]), pack(kb[2], kb[3]));
-        *reinterpret_cast<float4*>(sm + SM_QG + o_qg + rb + s32) =
+        *reinterpret_cast<float4*>(sm + SM_QK + o_qk + rb + s32) =
             make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
+        *reinterpret_cast<float4*>(sm + SM_QK + o_qk + 4096 + rb + s32) =
+            make_float4(kl[0] * e15.x, kl[1] * e15.y, kl[2] * e15.z, kl[3] * e15.w);
         kc[0][rr] = kb[0] * e3115.x;
         kc[1][rr] = kb[1] * e3115.y;
         kc[2][rr] = kb[2] * e3115.z;
@@ -647,6 +642,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
       fence_proxy_async();
       issue_qkg(c + 2);
     }
+    if (tid == 0 && c + 1 < nchunks && !U.vzero) prefetch_v(c + 1);
   }
   __syncthreads();
   if (nchunks > 0 && U.out_on && warp >= 4 && !*abort_flag) export_o(nchunks - 1);
@@ -669,9 +665,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   fence_before_sync();
   __syncthreads();
   if (tid == 0 && *abort_flag) {
-    // let any TMA load still in flight land before the CTA's memory is released
-    if (pend_in) mbar_wait_bounded(bar_in, ph_in, abort_flag, nullptr, 7);
-    if (pend_v) mbar_wait_bounded(bar_v, ph_v, abort_flag, nullptr, 8);
+    // let every MMA and TMA load still in flight land before the CTA's shared
+    // memory and TMEM are released
+    mma_commit(bar_drain);
+    mbar_wait_drain(bar_drain, 0);
+    if (pend_in) mbar_wait_drain(bar_in, ph_in);
+    if (pend_v) mbar_wait_drain(bar_v, ph_v);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tbase, TMEM_COLS);

@@ -122,4 +122,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Abort-path drain: waits (up to the time limit, whatever the abort flag says)
+// for asynchronous work this CTA already issued to land before its shared
+// memory or TMEM is released.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < kFastPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((long long)(global_ns() - t0) > kWaitLimitNs) return false;
+  }
+}
+
 }  // namespace kda

@@ -148,6 +148,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, ui
       : "memory");
 }
 
+// Pull a tensor tile into L2 ahead of its tma_load_3d (no shared memory written).
+__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 // 2^x and 1/x on the special-function unit (approximate: relative error a few
 // ulp), used where the result only feeds bf16/tf32 operands or fp32 decays.
 __device__ __forceinline__ float ex2_approx(float x) {
