@@ -23,24 +23,36 @@
 // most -5 on either side), far from fp32's e^88.7 limit; a longer chunk
 // would need more than one rebasing point per tile.
 //
-// B200 mapping.  One CTA (256 threads) owns one (sequence, head) for its
-// whole length; two CTAs share an SM (110 KB shared memory, 256 TMEM columns
-// each), so one CTA's SIMT phases overlap the other's GEMMs.  The fp32 state
-// never leaves the SM: it lives in TMEM as S^T (lane = value channel, column =
-// key channel) and is read directly as the tf32 A operand of the state-side
-// GEMMs.  tcgen05.mma costs a roughly fixed number of cycles per instruction
-// up to N = 128-256 (measured: ~90 with A in TMEM, ~190 with A in shared
-// memory), so products that share an A operand are fused into one wide MMA:
-//   [O^T | P^T]  = S^T [q e^G ; k e^G]^T            (N = 64, 16 k-steps)
-//   U^T         -= P^T T^T   onto  U^T = V^T T^T     (N = 32)
-//   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay (N = 160, 4 k-steps)
-// The Gram and U~ = T V are bf16 (A in shared memory).  TMA brings q/k/g for
-// the next chunk while the current one computes, and v into the Gram operand
-// region once the Gram is done.  All MMAs are issued by one thread and
-// tracked by mbarriers; every wait is bounded (kda_sync.cuh).
+// B200 mapping.  One CTA (13 warps) owns one (sequence, head) for its whole
+// length, one CTA per SM.  The fp32 state never leaves the SM: it lives in
+// TMEM as S^T (lane = value channel, column = key channel) and is read
+// directly as the tf32 A operand of the state-side GEMMs.  tcgen05.mma costs
+// a roughly fixed number of cycles per instruction up to N = 128-256
+// (measured: ~90 with A in TMEM, ~190 with A in shared memory), so products
+// that share an A operand are fused into one wide MMA:
+//   [O^T | P^T] += S^T [q e^G ; k e^G]^T  onto [0 | -V^T]  (N = 64, 16 k-steps)
+//   U^T          = -P^T T^T,  i.e. U = T (V - k e^G S)       (N = 32)
+//   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay        (N = 160, 4 k-steps)
+// The Gram is bf16 with A in shared memory, as M = 128, N = 64, K = 64: the
+// two 64-channel halves of [k;q] are stacked as rows against the two halves
+// of k, and the two diagonal blocks of the result are summed.
+//
+// The warps are specialised and hand work over through mbarriers, so the
+// key-side work of later chunks (which does not depend on the state)
+// overlaps the state-side chain of the current one:
+//   warps 0-3   prep: gate, in-chunk cumulative decay, rescaled operands
+//   warps 4-7   solve: Gram export, T = (I + A_kk)^-1 Diag(beta)
+//   warps 8-11  state: decay of S (a 32-column block as soon as the [O | P]
+//               k-steps reading it are done), export of O, seeding of [O | P]
+//   warp  12    one lane issues the state-side MMAs ([O | P], U, [S | O]) in
+//               chunk order, each after a blocking wait on what it needs
+//   warp  13    one lane issues the TMA loads and the Gram MMAs
+// Per-chunk operands are double-buffered by chunk parity; the Gram operand
+// region of a chunk is reused for T, v and the inverse's scratch once the
+// Gram is done.  Every wait is bounded (kda_sync.cuh).
 //
 // TMEM columns: S^T [0,128) | O^T [128,160) | P^T [160,192) | U^T [192,224)
-//               | Gram (M = 64 layout, lanes 0-15 of each quarter) [224,256)
+//               | Gram, 2 buffers [256,384)
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -53,40 +65,65 @@ namespace {
 
 using namespace tc;
 
-constexpr int C = 32;     // tokens per chunk
-constexpr int D = 128;    // dk = dv
-constexpr int NT = 256;   // threads per CTA
+constexpr int C = 32;    // tokens per chunk
+constexpr int D = 128;   // dk = dv
+constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12, KEYISSUE_W = 13;
+constexpr int NT = 32 * 14;
 
-constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192, G_COL = 224;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192, G_COL = 256;  // G: +64 b
+constexpr uint32_t TMEM_COLS = 512;
 
 // shared memory map (byte offsets from a 1024-aligned base)
-constexpr uint32_t SM_Q = 0;         // q tile  bf16 [32][128] row-major (TMA, no swizzle)
-constexpr uint32_t SM_K = 8192;      // k tile  bf16 [32][128]
-constexpr uint32_t SM_G = 16384;     // g (or z) tile fp32 [32][128]; 4-row cumsum totals in prep
-constexpr uint32_t SM_R1 = 32768;    // 24 KB, two lives:
-constexpr uint32_t SM_KQL = SM_R1;            //  [k;q] e^{G-G15}  bf16 64 x 128 (Gram A)
-constexpr uint32_t SM_KB = SM_R1 + 16384;     //  k e^{G15-G}      bf16 32 x 128 (Gram B)
-                                              // and once the Gram GEMM is done:
-constexpr uint32_t SM_TT = SM_R1;             //  T      bf16 [r][s] (B of U~)
-constexpr uint32_t SM_TF = SM_R1 + 4096;      //  T      fp32 [r][s] (tf32 B of U -= P^T T^T)
-constexpr uint32_t SM_V = SM_R1 + 8192;       //  v tile bf16, 2 x [32 rows x 128 B] swizzled (TMA)
-constexpr uint32_t SM_AKKT = SM_R1 + 16384;   //  A_kk^T fp32 [s][r] 32 x 32 (inverse input)
-constexpr uint32_t SM_XS = SM_R1 + 20480;     //  inverse blocks X00, X11 and A10 X00, fp32 32 x 32
-constexpr uint32_t SM_QK = 57344;    // [q e^G ; k e^G] fp32, per 32-channel block 64 rows x 128 B
-                                     // (tf32 B of [O | P])
-constexpr uint32_t SM_KC = 90112;    // k e^{GC-G}   fp32 [i][s] (K-major tf32 B of S), rows 0-127,
-constexpr uint32_t SM_AQK = 106496;  // A_qk         fp32 [r][s], rows 128-159 of the same B tile
-constexpr uint32_t SM_MISC = 110592;
-constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C}  fp32 [128]
-constexpr uint32_t SM_BETA = SM_MISC + 512;    // beta         fp32 [32]
-constexpr uint32_t SM_BAR = SM_MISC + 640;     // 5 mbarriers
-constexpr uint32_t SM_TMEM = SM_MISC + 680;    // TMEM base address
-constexpr uint32_t SM_ABORT = SM_MISC + 684;   // abort flag
-constexpr uint32_t SMEM_BYTES = SM_MISC + 1024;
+constexpr uint32_t STAGE = 32768;   // input stage s at s * STAGE, two stages
+constexpr uint32_t OFF_Q = 0;       //   q bf16 [32][128] (TMA, no swizzle)
+constexpr uint32_t OFF_K = 8192;    //   k bf16 [32][128]
+constexpr uint32_t OFF_G = 16384;   //   g or z fp32 [32][128]; in-chunk cumsum (log2) in prep
+constexpr uint32_t SM_KEY = 65536;  // key buffer b at SM_KEY + b * KEYB
+constexpr uint32_t KEYB = 24576;
+constexpr uint32_t K_KQL = 0;       //   Gram A: 128 rows x 64 channels bf16: rows 0-31 k e^{G-G15}
+                                    //   and 32-63 q e^{G-G15} of channels 0-63, rows 64-127
+                                    //   the same of channels 64-127
+constexpr uint32_t K_KB = 16384;    //   Gram B: 64 rows x 64 channels bf16: k e^{G15-G} of
+                                    //   channels 0-63 (rows 0-31) and 64-127 (rows 32-63)
+                                    //   and once the Gram GEMM is done:
+constexpr uint32_t K_PART = 0;      //   second-half Gram partials fp32 [2][32][32] (export),
+constexpr uint32_t K_TF = 4096;     //   then T fp32 [r][s] (tf32 B of U = -P^T T^T)
+constexpr uint32_t K_V = 8192;      //   v tile bf16, 2 x [32 rows x 128 B] swizzled (TMA)
+constexpr uint32_t K_AKKT = 16384;  //   A_kk^T fp32 [s][r] (inverse input)
+constexpr uint32_t K_XS = 20480;    //   inverse blocks, fp32 32 x 32
+constexpr uint32_t SM_HB = SM_KEY + 2 * KEYB;  // hand-off buffer b at SM_HB + b * HBB
+constexpr uint32_t HBB = 53248;
+constexpr uint32_t H_QK = 0;        //   [q e^G ; k e^G] fp32, per 32-channel block 64 rows x 128 B
+constexpr uint32_t H_KC = 32768;    //   k e^{GC-G} fp32 [i][s] (rows 0-127 of the B of [S | O])
+constexpr uint32_t H_AQK = 49152;   //   A_qk fp32 [r][s]       (rows 128-159 of the same tile)
+constexpr uint32_t SM_MISC = SM_HB + 2 * HBB;
+constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C} fp32 [2][128]
+constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta        fp32 [2][32]
+constexpr uint32_t SM_BAR = SM_MISC + 1280;    // mbarriers
+constexpr uint32_t SM_TMEM = SM_MISC + 1536;   // TMEM base address
+constexpr uint32_t SM_ABORT = SM_MISC + 1540;  // abort flag
+constexpr uint32_t SMEM_BYTES = SM_MISC + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to 1024
-static_assert(SM_AQK == SM_KC + 16384, "A_qk rows must follow the Kc^T rows");
-static_assert(2 * (SMEM_ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(H_AQK == H_KC + 16384, "A_qk rows must follow the Kc^T rows");
+static_assert(SMEM_ALLOC <= 227 * 1024, "one CTA per SM");
+
+// mbarriers ([2] = one per chunk parity)
+enum : int {
+  B_IN_FULL = 0,    // [2] TMA q, k, g landed                      (tx)
+  B_IN_EMPTY = 2,   // [2] prep done with the input stage          (4 prep warps)
+  B_OPER = 4,       // [2] chunk operands written                  (4 prep warps)
+  B_GRAM = 6,       // [2] Gram GEMM done                          (commit)
+  B_T = 8,          // [2] T and A_qk written                      (4 solve warps)
+  B_UOQ = 10,       // [4] [O | P] k-steps 4q .. 4q+3 done           (commit)
+  B_U = 14,         //     U GEMM done                             (commit)
+  B_DECAY = 15,     //     state decayed                           (4 state warps)
+  B_SO = 16,        // [2] [S | O] GEMM done                       (commit)
+  B_OREADY = 18,    //     O read out, [O | P] seeded with [0 | -V^T] (4 state warps)
+  B_DRAIN = 19,     // [2] abort path: every MMA an issuing thread issued done (commit)
+  B_V = 21,         // [2] TMA v landed                            (tx)
+  NBARS = 23
+};
+static_assert(NBARS * 8 <= SM_TMEM - SM_BAR, "mbarrier space");
 
 constexpr uint32_t TX_QKG = 8192 + 8192 + 16384;
 constexpr uint32_t TX_V = 8192;
@@ -172,7 +209,10 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
   return true;
 }
 
-__global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__ TcParams P) {
+// The register file is split across the SM's four sub-partitions and a CTA's
+// warps are dealt to them in turn, so with 14 warps two quarters hold four of
+// them: 16384 / (4 * 32) = 128 registers per thread is the most that launches.
+__global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -182,23 +222,24 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   if (!resolve_unit(P, U)) return;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + SM_BAR);
-  uint64_t* bar_v = bar_in + 1;
-  uint64_t* bar_mma = bar_in + 2;
-  uint64_t* bar_u = bar_in + 3;      // U -= P^T T^T done
-  uint64_t* bar_drain = bar_in + 4;  // abort path: every MMA issued so far done
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_ABORT);
-  float* gamc = reinterpret_cast<float*>(sm + SM_GAMC);
-  float* betas = reinterpret_cast<float*>(sm + SM_BETA);
   const int H = P.H, h = U.h;
+  const int nchunks = (int)((U.len + C - 1) / C);
+  auto chunk_rows = [&](int cc) -> int {
+    const int64_t rem = U.len - (int64_t)cc * C;
+    return (int)(rem < C ? rem : C);
+  };
 
   if (tid == 0) {
-    mbar_init(bar_in, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar_mma, 1);
-    mbar_init(bar_u, 1);
-    mbar_init(bar_drain, 1);
+#pragma unroll
+    for (int i = 0; i < NBARS; ++i) {
+      const bool four = i == B_IN_EMPTY || i == B_IN_EMPTY + 1 || i == B_OPER ||
+                        i == B_OPER + 1 || i == B_T || i == B_T + 1 || i == B_DECAY ||
+                        i == B_OREADY;
+      mbar_init(&bars[i], four ? 4u : 1u);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -211,180 +252,264 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
   fence_after_sync();
   const uint32_t tbase = *tmem_slot;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lanes
-  const int half = warp >> 2;                                   // column half (8-warp passes)
 
-  const int nchunks = (int)((U.len + C - 1) / C);
-  const float a2 = P.A_log ? expf(P.A_log[h]) * 1.4426950408889634f : 0.f;
-  bool pend_in = false, pend_v = false;  // thread 0: TMA loads issued, not yet waited
-  auto issue_qkg = [&](int c) {
-    const int row = (int)(U.row0 + (int64_t)c * C);
-    mbar_arrive_expect_tx(bar_in, TX_QKG);
-    tma_load_3d(sm + SM_Q, &P.tm_q, bar_in, 0, h, row);
-    tma_load_3d(sm + SM_K, &P.tm_k, bar_in, 0, h, row);
-    tma_load_3d(sm + SM_G, &P.tm_g, bar_in, 0, h, row);
-    pend_in = true;
-  };
-  auto issue_v = [&](int c) {  // into the Gram operand region: only once the Gram is done
-    const int row = (int)(U.row0 + (int64_t)c * C);
-    mbar_arrive_expect_tx(bar_v, TX_V);
-    tma_load_3d(sm + SM_V, &P.tm_v, bar_v, 0, h, row);
-    tma_load_3d(sm + SM_V + 4096, &P.tm_v, bar_v, 64, h, row);
-    pend_v = true;
-  };
-  auto prefetch_v = [&](int c) {
-    const int row = (int)(U.row0 + (int64_t)c * C);
-    tma_prefetch_3d(&P.tm_v, 0, h, row);
-    tma_prefetch_3d(&P.tm_v, 64, h, row);
-  };
-  if (tid == 0 && nchunks > 0) {
-    issue_qkg(0);
-    if (!U.vzero) prefetch_v(0);
-  }
-
-  // ---- initial state -> TMEM (S^T: lane j, column i)
-  {
+  // ---- initial state -> TMEM (S^T: lane j, column i), by the state warps
+  if (warp >= STATE_W0 && warp < ISSUE_W) {
     const int j = 32 * (warp & 3) + lane;
     float v[32];
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int i0 = 64 * half + 32 * cc;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const int i = i0 + k;
+        const int i = 32 * cc + k;
         v[k] = U.init ? U.init[(size_t)i * D + j] : ((U.init_identity && i == j) ? 1.f : 0.f);
       }
-      tmem_st32(tbase + lane_base + S_COL + i0, v);
+      tmem_st32(tbase + lane_base + S_COL + 32 * cc, v);
     }
     wait_st();
   }
   fence_before_sync();
   __syncthreads();
+  fence_after_sync();
 
-  uint32_t ph_in = 0, ph_v = 0, ph_mma = 0, ph_u = 0;
-  const uint32_t id_gram = idesc(kFmtBF16, 64, C, false, false, false);
-  const uint32_t id_tv = idesc(kFmtBF16, 128, C, true, false, false);        // U~^T = V^T T^T
-  const uint32_t id_op = idesc(kFmtTF32, 128, 2 * C, false, false, false);   // [O^T | P^T]
-  const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);         // U^T -= P^T T^T
-  const uint32_t id_so = idesc(kFmtTF32, 128, D + C, false, false, false);   // [S^T | O^T]
+  if (warp < SOLVE_W0) {
+    // =============================================================== prep warps
+    // thread: channels c0 .. c0+3, rows 8pw .. 8pw+7
+    const int pw = warp - PREP_W0, c0 = 4 * lane;
+    const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;  // bf16 tiles
+    const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                              // fp32 tiles
+    const uint32_t o_kql = (c0 >> 6) * 8192 + lo16;
+    const uint32_t o_kb = (c0 >> 6) * 4096 + lo16;
+    const uint32_t o_qk = (c0 >> 5) * 8192;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float gmin2 = P.g_min * kLog2e;
+    const float a2 = P.A_log ? expf(P.A_log[h]) * kLog2e : 0.f;
+    float beta_next = 0.f;
+    if (pw == 0 && lane < U.len) beta_next = P.beta[(size_t)(U.row0 + lane) * H + h];
 
-  // prep thread mapping: channels c0 .. c0+3 and rows 4ro .. 4ro+3 (warp ro)
-  const int cq = tid & 31, ro = tid >> 5, c0 = 4 * cq;
-  // byte offsets of (row 4ro, channel c0) in each swizzled operand; a row
-  // 4ro + rr adds rr*128 and xors the 16-byte chunk index with (4ro + rr) & 7
-  const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;   // bf16 tiles
-  const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                                 // fp32 tiles
-  const uint32_t o_kql = (c0 >> 6) * 8192 + ro * 512 + lo16;
-  const uint32_t o_kb = (c0 >> 6) * 4096 + ro * 512 + lo16;
-  const uint32_t o_qk = (c0 >> 5) * 8192 + ro * 512;
-  constexpr float kLog2e = 1.4426950408889634f;
-  const float gmin2 = P.g_min * kLog2e;
-  auto chunk_rows = [&](int cc) -> int {
-    const int64_t rem = U.len - (int64_t)cc * C;
-    return (int)(rem < C ? rem : C);
-  };
-
-  float beta_next = 0.f;  // beta of the chunk after the one being prepared
-  float4 G4[4];           // in-chunk cumulative log2-decay of the chunk being prepared
-  float kc[4][4];         // its Kc values [channel][row], stored after the state update
-
-  // ---- prep, part 1: wait for the chunk's tiles, beta, cumulative sums of g
-
-  // ---- prep, part 2 (after a barrier): rescaled operands of the chunk
-
-  // ---- Kc^T rows c0, c0+1: this thread's 8 rows are two 16-byte chunks of each
-
-  // ---- O^T of chunk cc (lane j, column r) -> o rows; lanes j, j^1 swap values so
-  //      each writes a bf16 pair (even lane rows 2m, odd lane rows 2m+1).  Warps 4-7.
-  auto export_o = [&](int cc) {
-    const int n = chunk_rows(cc);
-    const int j = 32 * (warp & 3) + lane;
-    const bool odd = lane & 1;
-    float v[32];
-    tmem_ld32(tbase + lane_base + O_COL, v);
-    wait_ld();
-    const int jp = j & ~1;
-    __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + (int64_t)cc * C) * H + h) * D + jp;
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float send = odd ? v[2 * m] : v[2 * m + 1];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-      const int r = 2 * m + (odd ? 1 : 0);
-      const float lo = odd ? recv : v[2 * m];      // column jp
-      const float hi = odd ? v[2 * m + 1] : recv;  // column jp + 1
-      if (r < n)
-        *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
-            __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
-    }
-  };
-
-  // the loop starts at c = -1: that pass only prepares chunk 0's operands
-  if (nchunks > 0 && tid < C && tid < U.len) beta_next = P.beta[(size_t)(U.row0 + tid) * H + h];
-  for (int c = -1; c < nchunks && !*abort_flag; ++c) {
-    const bool has_next = c + 1 < nchunks;
-    if (c >= 0) {
-
-    // ===== A: Gram GEMM (M64 N32 K128) of chunk c; warps 4-7 export O of chunk c-1
-    if (tid == 0) {
-      fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t kb = ks >> 2, kk = ks & 3;
-        const uint64_t a = sw128_desc(sb + SM_KQL + kb * (64 * 128) + kk * 32, 16, 1024);
-        const uint64_t b = sw128_desc(sb + SM_KB + kb * (32 * 128) + kk * 32, 16, 1024);
-        mma_ss(tbase + G_COL, a, b, id_gram, 0, ks > 0);
+    for (int c = 0; c < nchunks; ++c) {
+      if (bar_red_or(1, 128, *abort_flag != 0)) break;
+      const int st = c & 1, b = c & 1;
+      const int n = chunk_rows(c);
+      uint8_t* in = sm + st * STAGE;
+      uint8_t* kb_buf = sm + SM_KEY + b * KEYB;
+      uint8_t* hb = sm + SM_HB + b * HBB;
+      const float beta_cur = beta_next;
+      if (pw == 0) {
+        const int64_t t1 = (int64_t)(c + 1) * C + lane;
+        beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
       }
-      mma_commit(bar_mma);
-    }
-    if (c > 0 && U.out_on && warp >= 4) export_o(c - 1);
-    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 2);
-    ph_mma ^= 1;
-    fence_after_sync();
-    if (tid == 0 && !U.vzero && !*abort_flag) issue_v(c);  // the Gram operands are dead now
+      mbar_wait_bounded(&bars[B_IN_FULL + st], (c >> 1) & 1, abort_flag, P.sb, 1);
+      __syncwarp();
 
-    // ===== B: A_kk (transposed, x beta) and A_qk from the Gram accumulator
-    if (warp < 4) {
-      float v[32];
-      tmem_ld32(tbase + lane_base + G_COL, v);
-      wait_ld();
-      if (lane < 16) {
-        const int r = 16 * (warp & 1) + lane;
-        if (warp < 2) {
-          const float br = betas[r];
-          float* akkt = reinterpret_cast<float*>(sm + SM_AKKT);
+      // ---- part 1: gate and cumulative log2-decay over rows 8pw .. 8pw+7, written
+      //      back in place (only this thread touches these elements)
+      {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int s2 = 0; s2 < 32; ++s2) akkt[s2 * 32 + r] = s2 < r ? br * v[s2] : 0.f;
-        } else {
+        for (int rr = 0; rr < 8; ++rr) {
+          const int r = 8 * pw + rr;
+          float4* gp = reinterpret_cast<float4*>(in + OFF_G + (r * D + c0) * 4);
+          float4 gv = *gp;
+          if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
+            gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
+            gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
+            gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
+            gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
+          } else {
+            gv.x *= kLog2e;
+            gv.y *= kLog2e;
+            gv.z *= kLog2e;
+            gv.w *= kLog2e;
+          }
+          if (r >= n) {  // tail rows act as g = 0, k = q = 0
+            gv = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<uint2*>(in + OFF_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2*>(in + OFF_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
+          }
+          acc.x += gv.x;
+          acc.y += gv.y;
+          acc.z += gv.z;
+          acc.w += gv.w;
+          *gp = acc;
+        }
+      }
+      named_bar(1, 128);
+
+      // ---- part 2: rescaled operands; buffer b is free once chunk c - 2 is
+      //      completely done (its [S | O] GEMM is the last reader)
+      if (c >= 2) mbar_wait_bounded(&bars[B_SO + b], ((c - 2) >> 1) & 1, abort_flag, P.sb, 2);
+      __syncwarp();
+      {
+        float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
 #pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            float4 w4;
-            w4.x = (4 * s4 + 0 <= r) ? v[4 * s4 + 0] : 0.f;
-            w4.y = (4 * s4 + 1 <= r) ? v[4 * s4 + 1] : 0.f;
-            w4.z = (4 * s4 + 2 <= r) ? v[4 * s4 + 2] : 0.f;
-            w4.w = (4 * s4 + 3 <= r) ? v[4 * s4 + 3] : 0.f;
-            *reinterpret_cast<float4*>(sm + SM_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
+        for (int o4 = 0; o4 < 4; ++o4) {  // group totals: the partial sums at rows 8 o4 + 7
+          const float4 t =
+              *reinterpret_cast<const float4*>(in + OFF_G + ((8 * o4 + 7) * D + c0) * 4);
+          if (o4 < pw) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
+          if (o4 < 2) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
+          g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
+        }
+        const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
+                                       ex2_approx(g15.w));
+        const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
+                                         ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
+        if (pw == 0) {
+          *reinterpret_cast<float4*>(sm + SM_GAMC + b * 512 + c0 * 4) = make_float4(
+              ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
+          reinterpret_cast<float*>(sm + SM_BETA + b * 128)[lane] = beta_cur;
+        }
+        const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
+        auto pack = [](float lo_, float hi_) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo_, hi_);
+          return *reinterpret_cast<const uint32_t*>(&b2);
+        };
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          float kc[4][4];  // [channel][row] of rows 8pw + 4hf .. +3
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4) {
+            const int r = 8 * pw + 4 * hf + r4;
+            const float4 G = *reinterpret_cast<const float4*>(in + OFF_G + (r * D + c0) * 4);
+            float ex[4], ix[4];
+            ex[0] = ex2_approx(G.x + sh.x);
+            ex[1] = ex2_approx(G.y + sh.y);
+            ex[2] = ex2_approx(G.z + sh.z);
+            ex[3] = ex2_approx(G.w + sh.w);
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
+            const uint2 kw = *reinterpret_cast<const uint2*>(in + OFF_K + (r * D + c0) * 2);
+            const uint2 qw = *reinterpret_cast<const uint2*>(in + OFF_Q + (r * D + c0) * 2);
+            const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
+                                 __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
+            const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
+                                 __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
+            float kl[4], ql[4], kbv[4];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              kl[k4] = kv[k4] * ex[k4];
+              ql[k4] = qv[k4] * ex[k4];
+              kbv[k4] = kv[k4] * ix[k4];
+            }
+            const uint32_t sw = (uint32_t)(r & 7);
+            const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
+            // Gram operands (rows 64 hh + r, 64 hh + 32 + r of A and 32 hh + r of B
+            // for channel half hh = c0 / 64)
+            *reinterpret_cast<uint2*>(kb_buf + K_KQL + o_kql + r * 128 + s16) =
+                make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
+            *reinterpret_cast<uint2*>(kb_buf + K_KQL + o_kql + (32 + r) * 128 + s16) =
+                make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
+            *reinterpret_cast<uint2*>(kb_buf + K_KB + o_kb + r * 128 + s16) =
+                make_uint2(pack(kbv[0], kbv[1]), pack(kbv[2], kbv[3]));
+            // B of [O | P]: q e^G rows 0-31, k e^G rows 32-63
+            *reinterpret_cast<float4*>(hb + H_QK + o_qk + r * 128 + s32) =
+                make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
+            *reinterpret_cast<float4*>(hb + H_QK + o_qk + (32 + r) * 128 + s32) =
+                make_float4(kl[0] * e15.x, kl[1] * e15.y, kl[2] * e15.z, kl[3] * e15.w);
+            kc[0][r4] = kbv[0] * e3115.x;
+            kc[1][r4] = kbv[1] * e3115.y;
+            kc[2][r4] = kbv[2] * e3115.z;
+            kc[3][r4] = kbv[3] * e3115.w;
+          }
+          // Kc^T rows c0..c0+3, one 16-byte chunk each; in step k lane l writes row
+          // c0 + (k + l/2) % 4, so the 8 lanes of a quarter warp hit 8 different
+          // swizzled chunks (no bank conflicts)
+          const uint32_t chunk = (uint32_t)(2 * pw + hf);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int k4 = (k + (lane >> 1)) & 3;
+            float4 w;
+            w.x = k4 == 0 ? kc[0][0] : k4 == 1 ? kc[1][0] : k4 == 2 ? kc[2][0] : kc[3][0];
+            w.y = k4 == 0 ? kc[0][1] : k4 == 1 ? kc[1][1] : k4 == 2 ? kc[2][1] : kc[3][1];
+            w.z = k4 == 0 ? kc[0][2] : k4 == 1 ? kc[1][2] : k4 == 2 ? kc[2][2] : kc[3][2];
+            w.w = k4 == 0 ? kc[0][3] : k4 == 1 ? kc[1][3] : k4 == 2 ? kc[2][3] : kc[3][3];
+            const int row = c0 + k4;
+            *reinterpret_cast<float4*>(hb + H_KC + row * 128 +
+                                       ((chunk ^ (uint32_t)(row & 7)) << 4)) = w;
           }
         }
       }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars[B_OPER + b]);
+        mbar_arrive(&bars[B_IN_EMPTY + st]);
+      }
     }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (*abort_flag) break;
+  } else if (warp < STATE_W0) {
+    // ============================================================== solve warps
+    const int sw = warp - SOLVE_W0;  // TMEM lane quarter
+    const int stid = tid - 32 * SOLVE_W0;
+    for (int c = 0; c < nchunks; ++c) {
+      if (bar_red_or(2, 128, *abort_flag != 0)) break;
+      const int b = c & 1;
+      uint8_t* kb_buf = sm + SM_KEY + b * KEYB;
+      uint8_t* hb = sm + SM_HB + b * HBB;
+      const float* betas = reinterpret_cast<const float*>(sm + SM_BETA + b * 128);
+      mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 3);
+      mbar_wait_bounded(&bars[B_GRAM + b], (c >> 1) & 1, abort_flag, P.sb, 4);
+      __syncwarp();
+      fence_after_sync();
+      {  // Gram accumulator (lane quarter sw: k rows / q rows of channel half sw / 2,
+         // columns of the matching half of k) -> A_kk^T (x beta) and A_qk, in
+         // groups of 8 columns
+        const uint32_t gcol = tbase + lane_base + G_COL + 64 * b + (sw >= 2 ? 32 : 0);
+        float* part = reinterpret_cast<float*>(kb_buf + K_PART + (sw & 1) * 4096);
+        const int r = lane;
+        if (sw >= 2) {
+#pragma unroll 1
+          for (int g8 = 0; g8 < 4; ++g8) {
+            float v[8];
+            tmem_ld8(gcol + 8 * g8, v);
+            wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) part[r * 32 + ((8 * g8 + e) ^ r)] = v[e];
+          }
+        }
+        named_bar(2, 128);
+        if (sw < 2) {
+          const float br = betas[r];
+          float* akkt = reinterpret_cast<float*>(kb_buf + K_AKKT);
+#pragma unroll 1
+          for (int g8 = 0; g8 < 4; ++g8) {
+            float v[8];
+            tmem_ld8(gcol + 8 * g8, v);
+            wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] += part[r * 32 + ((8 * g8 + e) ^ r)];
+            if (sw == 0) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int s2 = 8 * g8 + e;
+                akkt[s2 * 32 + r] = s2 < r ? br * v[e] : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int h4 = 0; h4 < 2; ++h4) {
+                const int s4 = 2 * g8 + h4;
+                float4 w4;
+                w4.x = (4 * s4 + 0 <= r) ? v[4 * h4 + 0] : 0.f;
+                w4.y = (4 * s4 + 1 <= r) ? v[4 * h4 + 1] : 0.f;
+                w4.z = (4 * s4 + 2 <= r) ? v[4 * h4 + 2] : 0.f;
+                w4.w = (4 * s4 + 3 <= r) ? v[4 * h4 + 3] : 0.f;
+                *reinterpret_cast<float4*>(hb + H_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
+              }
+            }
+          }
+        }
+      }
+      named_bar(2, 128);
 
-    // ===== C: T = (I + A_kk)^-1 Diag(beta), blocked 2 x 2 over 16-row blocks
-    if (warp < 4) {
-      const float* akkt = reinterpret_cast<const float*>(sm + SM_AKKT);
-      float* xs = reinterpret_cast<float*>(sm + SM_XS);
-      auto tt_store = [&](int r, int col, float val) {  // bf16 and fp32 copies of T[r][col]
-        *reinterpret_cast<__nv_bfloat16*>(
-            sm + SM_TT + r * 128 + ((((uint32_t)(col * 2) >> 4) ^ (uint32_t)(r & 7)) << 4) +
-            ((col * 2) & 15)) = __float2bfloat16_rn(val);
+      // ---- T = (I + A_kk)^-1 Diag(beta), blocked 2 x 2 over 16-row blocks
+      const float* akkt = reinterpret_cast<const float*>(kb_buf + K_AKKT);
+      float* xs = reinterpret_cast<float*>(kb_buf + K_XS);
+      auto tt_store = [&](int r, int col, float val) {  // T[r][col], tf32 B operand layout
         *reinterpret_cast<float*>(
-            sm + SM_TF + r * 128 + ((((uint32_t)(col * 4) >> 4) ^ (uint32_t)(r & 7)) << 4) +
+            kb_buf + K_TF + r * 128 + ((((uint32_t)(col * 4) >> 4) ^ (uint32_t)(r & 7)) << 4) +
             ((col * 4) & 15)) = val;
       };
-      if (warp == 0) {  // diagonal blocks: lane = (block b, column cb)
-        const int b = lane >> 4, cb = lane & 15, o = 16 * b;
+      if (sw == 0) {  // diagonal blocks: lane = (block bb, column cb)
+        const int bb = lane >> 4, cb = lane & 15, o = 16 * bb;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == cb) ? 1.f : 0.f;
@@ -406,25 +531,23 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
         for (int r = 0; r < 16; ++r) {
           xs[(o + r) * 32 + o + cb] = x[r];
           tt_store(o + r, o + cb, x[r] * bc);
-          if (b == 0) tt_store(r, 16 + cb, 0.f);  // upper-right block of T is zero
+          if (bb == 0) tt_store(r, 16 + cb, 0.f);  // upper-right block of T is zero
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // Y = A10 X00 (rows 16..31 x columns 0..15), into the lower-left block of xs
-      const int cl = tid & 15, rp = tid >> 4;  // tid < 128 here
+      named_bar(2, 128);
+      const int cl = stid & 15, rp = stid >> 4;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < 2; ++h2) {  // Y = A10 X00 into the lower-left block of xs
         const int r = 2 * rp + h2;
         float y = 0.f;
 #pragma unroll
         for (int s2 = 0; s2 < 16; ++s2) y = fmaf(akkt[s2 * 32 + 16 + r], xs[s2 * 32 + cl], y);
         xs[(16 + r) * 32 + cl] = y;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // X10 = -X11 Y;  T[16 + r][c] = X10[r][c] beta_c
+      named_bar(2, 128);
       const float bcl = betas[cl];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < 2; ++h2) {  // X10 = -X11 Y
         const int r = 2 * rp + h2;
         float x10 = 0.f;
 #pragma unroll
@@ -432,246 +555,237 @@ __global__ void __launch_bounds__(NT, 2) chunk_tc_kernel(const __grid_constant__
           x10 = fmaf(xs[(16 + r) * 32 + 16 + t2], xs[(16 + t2) * 32 + cl], x10);
         tt_store(16 + r, cl, -x10 * bcl);
       }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_T + b]);
     }
-    fence_proxy_async();
-    __syncthreads();
-    if (*abort_flag) break;
-
-    // ===== D: U~^T = V^T T^T (bf16) and [O^T | P^T] = S^T [Qg ; Ka]^T (tf32, A = S^T
-    //          in TMEM); meanwhile part 1 of the next chunk's prep
-    if (tid == 0) {
-      if (!U.vzero) {
-        mbar_wait_bounded(bar_v, ph_v, abort_flag, P.sb, 3);
-        ph_v ^= 1;
-        pend_v = false;
-      }
-      fence_after_sync();
-      if (!U.vzero) {
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-          mma_ss(tbase + U_COL, sw128_desc(sb + SM_V + ks * 2048, 4096, 1024),
-                 sw128_desc(sb + SM_TT + ks * 32, 16, 1024), id_tv, 0, ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks)
-        mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
-                    sw128_desc(sb + SM_QK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_op,
-                    ks > 0);
-      mma_commit(bar_mma);
-    }
-    }  // c >= 0
-
-    if (has_next) {  // prep, part 1: tiles, beta, cumulative sums of g (log2 units)
-      const int cc = c + 1;
+  } else if (warp < ISSUE_W) {
+    // ============================================================== state warps
+    const int j = 32 * (warp & 3) + lane;
+    float vn[32];  // -v of the next chunk, column j
+    // -V^T (lane j, column r) of chunk cc from its v tile; rows past the end
+    // read as 0 (T has zero columns there, so any finite value would do)
+    const uint32_t v_off = (uint32_t)(j >> 6) * 4096 + (uint32_t)(((j & 63) * 2) & 15);
+    const uint32_t v_ck = (uint32_t)((j & 63) * 2) >> 4;
+    auto load_v = [&](int cc) {
       const int n = chunk_rows(cc);
-      if (tid < C) {
-        betas[tid] = beta_next;
-        const int64_t t1 = (int64_t)(cc + 1) * C + tid;
-        beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
+      if (!U.vzero) {
+        mbar_wait_bounded(&bars[B_V + (cc & 1)], (cc >> 1) & 1, abort_flag, P.sb, 9);
+        __syncwarp();
       }
-      mbar_wait_bounded(bar_in, ph_in, abort_flag, P.sb, 1);
-      ph_in ^= 1;
-      if (tid == 0) pend_in = false;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const uint8_t* vt = sm + SM_KEY + (cc & 1) * KEYB + K_V + v_off;
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int r = 4 * ro + rr;
-        float4 gv = *reinterpret_cast<const float4*>(sm + SM_G + (r * D + c0) * 4);
-        if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
-          gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
-          gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
-          gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
-          gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
-        } else {
-          gv.x *= kLog2e;
-          gv.y *= kLog2e;
-          gv.z *= kLog2e;
-          gv.w *= kLog2e;
-        }
-        if (r >= n) {  // tail rows act as g = 0, k = q = 0
-          gv = make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<uint2*>(sm + SM_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
-          *reinterpret_cast<uint2*>(sm + SM_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
-        }
-        acc.x += gv.x;
-        acc.y += gv.y;
-        acc.z += gv.z;
-        acc.w += gv.w;
-        G4[rr] = acc;
+      for (int r = 0; r < C; ++r) {
+        const uint32_t bits =
+            *reinterpret_cast<const unsigned short*>(vt + r * 128 + ((v_ck ^ (uint32_t)(r & 7)) << 4));
+        vn[r] = (!U.vzero && r < n) ? -__uint_as_float(bits << 16) : 0.f;
       }
-      // 4-row group total, over the g values of (row 4ro, channels c0..c0+3) that
-      // only this thread reads
-      *reinterpret_cast<float4*>(sm + SM_G + (4 * ro * D + c0) * 4) = acc;
+    };
+    // [O^T | P^T] of the next chunk start as [0 | -V^T]
+    auto seed_op = [&]() {
+      float z[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) z[k] = 0.f;
+      tmem_st32(tbase + lane_base + O_COL, z);
+      tmem_st32(tbase + lane_base + P_COL, vn);
+      wait_st();
+    };
+    if (nchunks > 0) {
+      load_v(0);
+      seed_op();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_OREADY]);
     }
-    __syncthreads();
-    if (c >= 0) {
-    mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 5);
-    ph_mma ^= 1;
-    fence_after_sync();
+    for (int c = 0; c < nchunks; ++c) {
+      if (bar_red_or(3, 128, *abort_flag != 0)) break;
+      const int b = c & 1;
+      const bool more = c + 1 < nchunks;
+      mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 5);
+      {  // S^T[j][i] *= e^{Gamma_C, i}, a 32-column block once the [O | P] k-steps
+         // that read it are done
+        const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + b * 512);
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          mbar_wait_bounded(&bars[B_UOQ + q], c & 1, abort_flag, P.sb, 6);
+          __syncwarp();
+          fence_after_sync();
+          float v[32];
+          tmem_ld32(tbase + lane_base + S_COL + 32 * q, v);
+          wait_ld();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 gg = g4[8 * q + k4];
+            v[4 * k4 + 0] *= gg.x;
+            v[4 * k4 + 1] *= gg.y;
+            v[4 * k4 + 2] *= gg.z;
+            v[4 * k4 + 3] *= gg.w;
+          }
+          tmem_st32(tbase + lane_base + S_COL + 32 * q, v);
+        }
+        wait_st();
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_DECAY]);
+      if (more) load_v(c + 1);
 
-    // ===== G: U^T -= P^T T^T (tf32, A = P^T in TMEM, onto U~^T), issued once P is
-    //          complete; meanwhile decay the state, S^T[j][i] *= e^{Gamma_C, i}
-    if (tid == 0) {
+      mbar_wait_bounded(&bars[B_SO + b], (c >> 1) & 1, abort_flag, P.sb, 7);
+      __syncwarp();
+      fence_after_sync();
+      float vo[32];  // O^T (lane j, column r)
+      tmem_ld32(tbase + lane_base + O_COL, vo);
+      wait_ld();
+      if (more) seed_op();  // U of this chunk, the last reader of P, is done
+      fence_before_sync();
+      __syncwarp();
+      if (more && lane == 0) mbar_arrive(&bars[B_OREADY]);
+      if (U.out_on) {  // lanes j, j^1 swap values so each writes a bf16 pair
+        const int n = chunk_rows(c);
+        const bool odd = lane & 1;
+        const int jp = j & ~1;
+        __nv_bfloat16* obase = P.out + ((size_t)(U.row0 + (int64_t)c * C) * H + h) * D + jp;
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_ts_tf32(tbase + U_COL, tbase + P_COL + 8 * ks,
-                    sw128_desc(sb + SM_TF + ks * 32, 16, 1024), id_u, (ks > 0) || !U.vzero);
-      mma_commit(bar_u);
+        for (int m = 0; m < 16; ++m) {
+          const float send = odd ? vo[2 * m] : vo[2 * m + 1];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+          const int r = 2 * m + (odd ? 1 : 0);
+          const float lo = odd ? recv : vo[2 * m];      // column jp
+          const float hi = odd ? vo[2 * m + 1] : recv;  // column jp + 1
+          if (r < n)
+            *reinterpret_cast<__nv_bfloat162*>(obase + (size_t)r * H * D) =
+                __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
+        }
+      }
     }
-    {
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const uint32_t col = S_COL + 64 * half + 32 * cc;
-        const float4* g4 = reinterpret_cast<const float4*>(gamc + 64 * half + 32 * cc);
+    // final state (S^T lane j, column i -> final[i][j]); every S GEMM is done
+    if (U.final_state && !*abort_flag) {
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
         float v[32];
-        tmem_ld32(tbase + lane_base + col, v);
+        tmem_ld32(tbase + lane_base + S_COL + 32 * cc, v);
         wait_ld();
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 gg = g4[k4];
-          v[4 * k4 + 0] *= gg.x;
-          v[4 * k4 + 1] *= gg.y;
-          v[4 * k4 + 2] *= gg.z;
-          v[4 * k4 + 3] *= gg.w;
+        for (int k = 0; k < 32; ++k) U.final_state[(size_t)(32 * cc + k) * D + j] = v[k];
+      }
+    }
+  } else if (warp == ISSUE_W) {
+    // ============================================ state-side MMA issue (lane 0)
+    if (lane == 0) {
+      const uint32_t id_op = idesc(kFmtTF32, 128, 2 * C, false, false, false);    // [O^T | P^T]
+      const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);          // U^T = -P^T T^T
+      const uint32_t id_so = idesc(kFmtTF32, 128, D + C, false, false, false);    // [S^T | O^T]
+      for (int c = 0; c < nchunks; ++c) {
+        if (*abort_flag) break;
+        const int b = c & 1;
+        // [O^T | P^T] += S^T [Qg ; Ka]^T once the operands are written and O / P are
+        // seeded (which the state warps do after the previous [S | O] completed)
+        mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 10);
+        mbar_wait_bounded(&bars[B_OREADY], c & 1, abort_flag, P.sb, 11);
+        if (*abort_flag) break;
+        fence_after_sync();
+        const uint32_t hb = sb + SM_HB + b * HBB;
+#pragma unroll 1
+        for (int ks = 0; ks < 16; ++ks) {
+          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
+                      sw128_desc(hb + H_QK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_op,
+                      1);
+          if ((ks & 3) == 3) mma_commit(&bars[B_UOQ + (ks >> 2)]);
         }
-        tmem_st32(tbase + lane_base + col, v);
+        // U^T = -P^T T^T once P is complete and T is in
+        mbar_wait_bounded(&bars[B_T + b], (c >> 1) & 1, abort_flag, P.sb, 12);
+        mbar_wait_bounded(&bars[B_UOQ + 3], c & 1, abort_flag, P.sb, 13);
+        if (*abort_flag) break;
+        fence_after_sync();
+        const uint32_t kbb = sb + SM_KEY + b * KEYB;
+#pragma unroll 1
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts_tf32(tbase + U_COL, tbase + P_COL + 8 * ks,
+                      sw128_desc(kbb + K_TF + ks * 32, 16, 1024), id_u, ks > 0);
+        mma_commit(&bars[B_U]);
+        // [S^T | O^T] += U^T [Kc ; A_qk]^T once U is done and the state is decayed
+        mbar_wait_bounded(&bars[B_U], c & 1, abort_flag, P.sb, 14);
+        mbar_wait_bounded(&bars[B_DECAY], c & 1, abort_flag, P.sb, 15);
+        if (*abort_flag) break;
+        fence_after_sync();
+#pragma unroll 1
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
+                      sw128_desc(hb + H_KC + ks * 32, 16, 1024), id_so, 1);
+        mma_commit(&bars[B_SO + b]);
       }
-      wait_st();
+      if (*abort_flag) {  // every MMA this thread issued lands before TMEM is released
+        mma_commit(&bars[B_DRAIN]);
+        mbar_wait_drain(&bars[B_DRAIN], 0);
+      }
     }
-    fence_before_sync();
-    __syncthreads();
-    if (*abort_flag) break;
-
-    // ===== H: [S^T | O^T] += U^T [Kc ; A_qk^T] (tf32, U^T from TMEM, one N = 160 MMA
-    //          per k-step); meanwhile part 2 of the next chunk's prep
-    // U is also the last reader of T in the Gram operand region, which part 2
-    // of the prep overwrites: everyone waits for it
-    mbar_wait_bounded(bar_u, ph_u, abort_flag, P.sb, 9);
-    ph_u ^= 1;
-    if (tid == 0) {
-      fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
-                    sw128_desc(sb + SM_KC + ks * 32, 16, 1024), id_so, 1);
-      mma_commit(bar_mma);
-    }
-    }  // c >= 0
-    if (has_next) {  // prep, part 2: rescaled operands (Kc kept in registers)
-      float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
-#pragma unroll
-      for (int o8 = 0; o8 < 8; ++o8) {
-        const float4 t = *reinterpret_cast<const float4*>(sm + SM_G + (4 * o8 * D + c0) * 4);
-        if (o8 < ro) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
-        if (o8 < 4) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
-        g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
-      }
-      const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
-                                     ex2_approx(g15.w));
-      const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
-                                       ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
-      if (ro == 7) {
-        *reinterpret_cast<float4*>(gamc + c0) = make_float4(
-            ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
-      }
-      // G4[rr] - g15 + off: exponent of e^{Gamma_r - Gamma_15} in log2 units
-      const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
-#pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int r = 4 * ro + rr;
-        float ex[4], ix[4];
-        ex[0] = ex2_approx(G4[rr].x + sh.x);
-        ex[1] = ex2_approx(G4[rr].y + sh.y);
-        ex[2] = ex2_approx(G4[rr].z + sh.z);
-        ex[3] = ex2_approx(G4[rr].w + sh.w);
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
-        const uint2 kw = *reinterpret_cast<const uint2*>(sm + SM_K + (r * D + c0) * 2);
-        const uint2 qw = *reinterpret_cast<const uint2*>(sm + SM_Q + (r * D + c0) * 2);
-        const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
-                             __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
-        const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
-                             __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
-        float kl[4], ql[4], kb[4];
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          kl[k4] = kv[k4] * ex[k4];
-          ql[k4] = qv[k4] * ex[k4];
-          kb[k4] = kv[k4] * ix[k4];
+    __syncwarp();
+  } else {
+    // ==================================== TMA and Gram issue (lane 0 of the last warp)
+    if (lane == 0) {
+      const uint32_t id_gram = idesc(kFmtBF16, 128, 2 * C, false, false, false);  // 2 halves
+      auto issue_qkg = [&](int cc) {  // into stage cc & 1
+        const int row = (int)(U.row0 + (int64_t)cc * C);
+        uint8_t* in = sm + (cc & 1) * STAGE;
+        uint64_t* bf = &bars[B_IN_FULL + (cc & 1)];
+        fence_proxy_async();
+        mbar_arrive_expect_tx(bf, TX_QKG);
+        tma_load_3d(in + OFF_Q, &P.tm_q, bf, 0, h, row);
+        tma_load_3d(in + OFF_K, &P.tm_k, bf, 0, h, row);
+        tma_load_3d(in + OFF_G, &P.tm_g, bf, 0, h, row);
+        if (!U.vzero) {  // v follows once this chunk's Gram is done: warm L2 now
+          tma_prefetch_3d(&P.tm_v, 0, h, row);
+          tma_prefetch_3d(&P.tm_v, 64, h, row);
         }
-        const uint32_t rb = rr * 128;
-        const uint32_t sw = (uint32_t)((4 * ro + rr) & 7);
-        const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
-        auto pack = [](float lo, float hi) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
-          return *reinterpret_cast<const uint32_t*>(&b2);
-        };
-        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + rb + s16) =
-            make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
-        *reinterpret_cast<uint2*>(sm + SM_KQL + o_kql + 4096 + rb + s16) =
-            make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
-        *reinterpret_cast<uint2*>(sm + SM_KB + o_kb + rb + s16) =
-            make_uint2(pack(kb[0], kb[1]), pack(kb[2], kb[3]));
-        *reinterpret_cast<float4*>(sm + SM_QK + o_qk + rb + s32) =
-            make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
-        *reinterpret_cast<float4*>(sm + SM_QK + o_qk + 4096 + rb + s32) =
-            make_float4(kl[0] * e15.x, kl[1] * e15.y, kl[2] * e15.z, kl[3] * e15.w);
-        kc[0][rr] = kb[0] * e3115.x;
-        kc[1][rr] = kb[1] * e3115.y;
-        kc[2][rr] = kb[2] * e3115.z;
-        kc[3][rr] = kb[3] * e3115.w;
+      };
+      int nq = 0, nv = 0;  // TMA loads issued
+      for (; nq < 2 && nq < nchunks; ++nq) issue_qkg(nq);
+      for (int c = 0; c < nchunks; ++c) {
+        if (*abort_flag) break;
+        const int b = c & 1;
+        // Gram GEMM of chunk c (bf16, M128 N64 K64) once its operands are written
+        mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 16);
+        if (*abort_flag) break;
+        fence_after_sync();
+        const uint32_t kbb = sb + SM_KEY + b * KEYB;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tbase + G_COL + 64 * b, sw128_desc(kbb + K_KQL + kk * 32, 16, 1024),
+                 sw128_desc(kbb + K_KB + kk * 32, 16, 1024), id_gram, 0, kk > 0);
+        mma_commit(&bars[B_GRAM + b]);
+        // q, k, g of chunk c + 2 into the stage chunk c's prep has released
+        if (nq < nchunks) {
+          mbar_wait_bounded(&bars[B_IN_EMPTY + b], (c >> 1) & 1, abort_flag, P.sb, 17);
+          if (*abort_flag) break;
+          issue_qkg(nq++);
+        }
+        // v of chunk c into its Gram operand region once that Gram is done
+        if (!U.vzero) {
+          mbar_wait_bounded(&bars[B_GRAM + b], (c >> 1) & 1, abort_flag, P.sb, 18);
+          if (*abort_flag) break;
+          const int row = (int)(U.row0 + (int64_t)c * C);
+          uint8_t* dst = sm + SM_KEY + b * KEYB + K_V;
+          uint64_t* bf = &bars[B_V + b];
+          mbar_arrive_expect_tx(bf, TX_V);
+          tma_load_3d(dst, &P.tm_v, bf, 0, h, row);
+          tma_load_3d(dst + 4096, &P.tm_v, bf, 64, h, row);
+          ++nv;
+        }
+      }
+      if (*abort_flag) {
+        // every MMA and TMA load this thread issued lands before shared memory
+        // and TMEM are released
+        mma_commit(&bars[B_DRAIN + 1]);
+        mbar_wait_drain(&bars[B_DRAIN + 1], 0);
+        for (int k = (nq > 2 ? nq - 2 : 0); k < nq; ++k)
+          mbar_wait_drain(&bars[B_IN_FULL + (k & 1)], (k >> 1) & 1);
+        for (int k = (nv > 2 ? nv - 2 : 0); k < nv; ++k)
+          mbar_wait_drain(&bars[B_V + (k & 1)], (k >> 1) & 1);
       }
     }
-    if (c >= 0) {
-      mbar_wait_bounded(bar_mma, ph_mma, abort_flag, P.sb, 6);
-      ph_mma ^= 1;
-      fence_after_sync();
-    }
-    if (has_next) {  // Kc^T rows c0..c0+3: this thread's 4 rows are one 16-byte chunk of each
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int row = c0 + k4;
-        *reinterpret_cast<float4*>(sm + SM_KC + row * 128 + ((ro ^ (row & 7)) << 4)) =
-            make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
-      }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && c + 2 < nchunks) {
-      fence_proxy_async();
-      issue_qkg(c + 2);
-    }
-    if (tid == 0 && c + 1 < nchunks && !U.vzero) prefetch_v(c + 1);
-  }
-  __syncthreads();
-  if (nchunks > 0 && U.out_on && warp >= 4 && !*abort_flag) export_o(nchunks - 1);
-  fence_before_sync();
-  __syncthreads();
-
-  // ---- final state (S^T lane j, column i -> final[i][j])
-  if (U.final_state && !*abort_flag) {
-    const int j = 32 * (warp & 3) + lane;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int i0 = 64 * half + 32 * cc;
-      float v[32];
-      tmem_ld32(tbase + lane_base + S_COL + i0, v);
-      wait_ld();
-#pragma unroll
-      for (int k = 0; k < 32; ++k) U.final_state[(size_t)(i0 + k) * D + j] = v[k];
-    }
+    __syncwarp();
   }
   fence_before_sync();
-  __syncthreads();
-  if (tid == 0 && *abort_flag) {
-    // let every MMA and TMA load still in flight land before the CTA's shared
-    // memory and TMEM are released
-    mma_commit(bar_drain);
-    mbar_wait_drain(bar_drain, 0);
-    if (pend_in) mbar_wait_drain(bar_in, ph_in);
-    if (pend_v) mbar_wait_drain(bar_v, ph_v);
-  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tbase, TMEM_COLS);
 }
@@ -742,11 +856,13 @@ bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base
 // Segment split for long dense sequences with too few (sequence, head)
 // units to occupy the GPU: returns G >= 2 and the segment length, or G = 1.
 void plan_split(int B, int T, int H, int num_sms, int* G_out, int* seg_out) {
+  // one CTA per SM: split when the units fill less than half the SMs, into
+  // as many segments as keep one unit-segment per SM
   const int U = B * H;
   *G_out = 1;
   *seg_out = T;
   if (2 * U >= num_sms || T < 4 * 1024) return;
-  int G = (2 * num_sms + U - 1) / U;
+  int G = num_sms / U;
   const int max_g = T / 1024;
   if (G > max_g) G = max_g;
   if (G < 2) return;

@@ -104,10 +104,13 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 }
 
 // Waits for the phase with the given parity to complete.  On timeout sets
-// *abort (shared), records the status and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, StatusBlock* sb,
-                                                  int32_t detail) {
+// *abort (shared), records the status and returns false.  The first
+// try_wait (which may itself suspend the thread for a while) is inline; the
+// polling loop is an out-of-line call, so the many call sites of a kernel
+// stay small in the instruction cache.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                            volatile int* abort_flag, StatusBlock* sb,
+                                            int32_t detail) {
   for (int i = 0; i < kFastPolls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
@@ -120,6 +123,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, StatusBlock* sb,
+                                                  int32_t detail) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, sb, detail);
 }
 
 // Abort-path drain: waits (up to the time limit, whatever the abort flag says)
