@@ -23,16 +23,18 @@
 // most -5 on either side), far from fp32's e^88.7 limit; a longer chunk
 // would need more than one rebasing point per tile.
 //
-// B200 mapping.  One CTA (13 warps) owns one (sequence, head) for its whole
+// B200 mapping.  One CTA (14 warps) owns one (sequence, head) for its whole
 // length, one CTA per SM.  The fp32 state never leaves the SM: it lives in
-// TMEM as S^T (lane = value channel, column = key channel) and is read
-// directly as the tf32 A operand of the state-side GEMMs.  tcgen05.mma costs
+// TMEM as S^T (lane = value channel, column = key channel), next to a bf16
+// copy of it that is the A operand of the [O | P] GEMM (the state is cast to
+// bf16 for that product, as is usual for chunked delta-rule kernels; it is
+// accumulated in fp32 throughout).  tcgen05.mma costs
 // a roughly fixed number of cycles per instruction up to N = 128-256
 // (measured: ~90 with A in TMEM, ~190 with A in shared memory), so products
 // that share an A operand are fused into one wide MMA:
-//   [O^T | P^T] += S^T [q e^G ; k e^G]^T  onto [0 | -V^T]  (N = 64, 16 k-steps)
-//   U^T          = -P^T T^T,  i.e. U = T (V - k e^G S)       (N = 32)
-//   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay        (N = 160, 4 k-steps)
+//   [O^T | P^T] += S^T [q e^G ; k e^G]^T  onto [0 | -V^T]  (bf16, N = 64, 8 k-steps)
+//   U^T          = -P^T T^T,  i.e. U = T (V - k e^G S)       (tf32, N = 32)
+//   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay        (tf32, N = 160, 4 k-steps)
 // The Gram is bf16 with A in shared memory, as M = 128, N = 64, K = 64: the
 // two 64-channel halves of [k;q] are stacked as rows against the two halves
 // of k, and the two diagonal blocks of the result are summed.
@@ -42,17 +44,18 @@
 // overlaps the state-side chain of the current one:
 //   warps 0-3   prep: gate, in-chunk cumulative decay, rescaled operands
 //   warps 4-7   solve: Gram export, T = (I + A_kk)^-1 Diag(beta)
-//   warps 8-11  state: decay of S (a 32-column block as soon as the [O | P]
-//               k-steps reading it are done), export of O, seeding of [O | P]
+//   warps 8-11  state: once [S | O] of a chunk is done, the bf16 copy of S and
+//               the seed [0 | -V^T] of the next chunk's [O | P] (the critical
+//               path), then export of O and the next chunk's decay of S
 //   warp  12    one lane issues the state-side MMAs ([O | P], U, [S | O]) in
 //               chunk order, each after a blocking wait on what it needs
 //   warp  13    one lane issues the TMA loads and the Gram MMAs
-// Per-chunk operands are double-buffered by chunk parity; the Gram operand
-// region of a chunk is reused for T, v and the inverse's scratch once the
-// Gram is done.  Every wait is bounded (kda_sync.cuh).
+// Per-chunk operands are double-buffered by chunk parity (v four-deep); the
+// Gram operand region of a chunk is reused for T and the inverse's scratch
+// once the Gram is done.  Every wait is bounded (kda_sync.cuh).
 //
 // TMEM columns: S^T [0,128) | O^T [128,160) | P^T [160,192) | U^T [192,224)
-//               | Gram, 2 buffers [256,384)
+//               | Gram, 2 buffers [256,384) | bf16 S^T [384,448)
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -71,6 +74,7 @@ constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12, KEYISSUE_W 
 constexpr int NT = 32 * 14;
 
 constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192, G_COL = 256;  // G: +64 b
+constexpr uint32_t SB_COL = 384;  // bf16 S^T: column c holds key channels 2c, 2c + 1
 constexpr uint32_t TMEM_COLS = 512;
 
 // shared memory map (byte offsets from a 1024-aligned base)
@@ -88,15 +92,16 @@ constexpr uint32_t K_KB = 16384;    //   Gram B: 64 rows x 64 channels bf16: k e
                                     //   and once the Gram GEMM is done:
 constexpr uint32_t K_PART = 0;      //   second-half Gram partials fp32 [2][32][32] (export),
 constexpr uint32_t K_TF = 4096;     //   then T fp32 [r][s] (tf32 B of U = -P^T T^T)
-constexpr uint32_t K_V = 8192;      //   v tile bf16, 2 x [32 rows x 128 B] swizzled (TMA)
 constexpr uint32_t K_AKKT = 16384;  //   A_kk^T fp32 [s][r] (inverse input)
 constexpr uint32_t K_XS = 20480;    //   inverse blocks, fp32 32 x 32
 constexpr uint32_t SM_HB = SM_KEY + 2 * KEYB;  // hand-off buffer b at SM_HB + b * HBB
-constexpr uint32_t HBB = 53248;
-constexpr uint32_t H_QK = 0;        //   [q e^G ; k e^G] fp32, per 32-channel block 64 rows x 128 B
-constexpr uint32_t H_KC = 32768;    //   k e^{GC-G} fp32 [i][s] (rows 0-127 of the B of [S | O])
-constexpr uint32_t H_AQK = 49152;   //   A_qk fp32 [r][s]       (rows 128-159 of the same tile)
-constexpr uint32_t SM_MISC = SM_HB + 2 * HBB;
+constexpr uint32_t HBB = 36864;
+constexpr uint32_t H_QK = 0;        //   [q e^G ; k e^G] bf16, per 64-channel block 64 rows x 128 B
+constexpr uint32_t H_KC = 16384;    //   k e^{GC-G} fp32 [i][s] (rows 0-127 of the B of [S | O])
+constexpr uint32_t H_AQK = 32768;   //   A_qk fp32 [r][s]       (rows 128-159 of the same tile)
+constexpr uint32_t SM_V = SM_HB + 2 * HBB;  // v tile of chunk c at SM_V + (c % 4) * 8192:
+constexpr int NVBUF = 4;                    //   bf16, 2 x [32 rows x 128 B] swizzled (TMA)
+constexpr uint32_t SM_MISC = SM_V + NVBUF * 8192;
 constexpr uint32_t SM_GAMC = SM_MISC;          // e^{Gamma_C} fp32 [2][128]
 constexpr uint32_t SM_BETA = SM_MISC + 1024;   // beta        fp32 [2][32]
 constexpr uint32_t SM_BAR = SM_MISC + 1280;    // mbarriers
@@ -107,21 +112,22 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to
 static_assert(H_AQK == H_KC + 16384, "A_qk rows must follow the Kc^T rows");
 static_assert(SMEM_ALLOC <= 227 * 1024, "one CTA per SM");
 
-// mbarriers ([2] = one per chunk parity)
+// mbarriers ([2] = one per chunk parity, [4] = one per v buffer)
 enum : int {
   B_IN_FULL = 0,    // [2] TMA q, k, g landed                      (tx)
   B_IN_EMPTY = 2,   // [2] prep done with the input stage          (4 prep warps)
   B_OPER = 4,       // [2] chunk operands written                  (4 prep warps)
   B_GRAM = 6,       // [2] Gram GEMM done                          (commit)
   B_T = 8,          // [2] T and A_qk written                      (4 solve warps)
-  B_UOQ = 10,       // [4] [O | P] k-steps 4q .. 4q+3 done           (commit)
-  B_U = 14,         //     U GEMM done                             (commit)
-  B_DECAY = 15,     //     state decayed                           (4 state warps)
-  B_SO = 16,        // [2] [S | O] GEMM done                       (commit)
-  B_OREADY = 18,    //     O read out, [O | P] seeded with [0 | -V^T] (4 state warps)
-  B_DRAIN = 19,     // [2] abort path: every MMA an issuing thread issued done (commit)
-  B_V = 21,         // [2] TMA v landed                            (tx)
-  NBARS = 23
+  B_UO = 10,        //     [O | P] GEMM done                       (commit)
+  B_U = 11,         //     U GEMM done                             (commit)
+  B_DECAY = 12,     //     state decayed for the chunk             (4 state warps)
+  B_SO = 13,        // [2] [S | O] GEMM done                       (commit)
+  B_OREADY = 15,    //     bf16 S written, O read out, [O | P] seeded (4 state warps)
+  B_DRAIN = 16,     // [2] abort path: every MMA an issuing thread issued done (commit)
+  B_V = 18,         // [4] TMA v landed                            (tx)
+  B_VEMPTY = 22,    // [4] v buffer read                           (4 state warps)
+  NBARS = 26
 };
 static_assert(NBARS * 8 <= SM_TMEM - SM_BAR, "mbarrier space");
 
@@ -237,7 +243,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     for (int i = 0; i < NBARS; ++i) {
       const bool four = i == B_IN_EMPTY || i == B_IN_EMPTY + 1 || i == B_OPER ||
                         i == B_OPER + 1 || i == B_T || i == B_T + 1 || i == B_DECAY ||
-                        i == B_OREADY;
+                        i == B_OREADY || (i >= B_VEMPTY && i < B_VEMPTY + NVBUF);
       mbar_init(&bars[i], four ? 4u : 1u);
     }
     *abort_flag = 0;
@@ -277,10 +283,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     // thread: channels c0 .. c0+3, rows 8pw .. 8pw+7
     const int pw = warp - PREP_W0, c0 = 4 * lane;
     const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;  // bf16 tiles
-    const uint32_t ck32 = ((c0 & 31) * 4) >> 4;                              // fp32 tiles
     const uint32_t o_kql = (c0 >> 6) * 8192 + lo16;
     const uint32_t o_kb = (c0 >> 6) * 4096 + lo16;
-    const uint32_t o_qk = (c0 >> 5) * 8192;
     constexpr float kLog2e = 1.4426950408889634f;
     const float gmin2 = P.g_min * kLog2e;
     const float a2 = P.A_log ? expf(P.A_log[h]) * kLog2e : 0.f;
@@ -392,7 +396,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
               kbv[k4] = kv[k4] * ix[k4];
             }
             const uint32_t sw = (uint32_t)(r & 7);
-            const uint32_t s16 = (ck16 ^ sw) << 4, s32 = (ck32 ^ sw) << 4;
+            const uint32_t s16 = (ck16 ^ sw) << 4;
             // Gram operands (rows 64 hh + r, 64 hh + 32 + r of A and 32 hh + r of B
             // for channel half hh = c0 / 64)
             *reinterpret_cast<uint2*>(kb_buf + K_KQL + o_kql + r * 128 + s16) =
@@ -401,11 +405,12 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
                 make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
             *reinterpret_cast<uint2*>(kb_buf + K_KB + o_kb + r * 128 + s16) =
                 make_uint2(pack(kbv[0], kbv[1]), pack(kbv[2], kbv[3]));
-            // B of [O | P]: q e^G rows 0-31, k e^G rows 32-63
-            *reinterpret_cast<float4*>(hb + H_QK + o_qk + r * 128 + s32) =
-                make_float4(ql[0] * e15.x, ql[1] * e15.y, ql[2] * e15.z, ql[3] * e15.w);
-            *reinterpret_cast<float4*>(hb + H_QK + o_qk + (32 + r) * 128 + s32) =
-                make_float4(kl[0] * e15.x, kl[1] * e15.y, kl[2] * e15.z, kl[3] * e15.w);
+            // B of [O | P] (bf16, same layout as the Gram A): q e^G rows 0-31,
+            // k e^G rows 32-63 of each 64-channel block
+            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + r * 128 + s16) =
+                make_uint2(pack(ql[0] * e15.x, ql[1] * e15.y), pack(ql[2] * e15.z, ql[3] * e15.w));
+            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (32 + r) * 128 + s16) =
+                make_uint2(pack(kl[0] * e15.x, kl[1] * e15.y), pack(kl[2] * e15.z, kl[3] * e15.w));
             kc[0][r4] = kbv[0] * e3115.x;
             kc[1][r4] = kbv[1] * e3115.y;
             kc[2][r4] = kbv[2] * e3115.z;
@@ -569,16 +574,35 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     const uint32_t v_ck = (uint32_t)((j & 63) * 2) >> 4;
     auto load_v = [&](int cc) {
       const int n = chunk_rows(cc);
+      const int vb = cc % NVBUF;
       if (!U.vzero) {
-        mbar_wait_bounded(&bars[B_V + (cc & 1)], (cc >> 1) & 1, abort_flag, P.sb, 9);
+        mbar_wait_bounded(&bars[B_V + vb], (cc / NVBUF) & 1, abort_flag, P.sb, 9);
         __syncwarp();
       }
-      const uint8_t* vt = sm + SM_KEY + (cc & 1) * KEYB + K_V + v_off;
+      const uint8_t* vt = sm + SM_V + vb * 8192 + v_off;
 #pragma unroll
       for (int r = 0; r < C; ++r) {
-        const uint32_t bits =
-            *reinterpret_cast<const unsigned short*>(vt + r * 128 + ((v_ck ^ (uint32_t)(r & 7)) << 4));
+        const uint32_t bits = *reinterpret_cast<const unsigned short*>(
+            vt + r * 128 + ((v_ck ^ (uint32_t)(r & 7)) << 4));
         vn[r] = (!U.vzero && r < n) ? -__uint_as_float(bits << 16) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_VEMPTY + vb]);
+    };
+    // the A operand of the next [O | P] GEMM: bf16 copy of the current S^T
+    auto write_sb = [&]() {
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        tmem_ld32(tbase + lane_base + S_COL + 32 * q, v);
+        wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          pk[k] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        tmem_st16(tbase + lane_base + SB_COL + 16 * q, pk);
       }
     };
     // [O^T | P^T] of the next chunk start as [0 | -V^T]
@@ -588,58 +612,61 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       for (int k = 0; k < 32; ++k) z[k] = 0.f;
       tmem_st32(tbase + lane_base + O_COL, z);
       tmem_st32(tbase + lane_base + P_COL, vn);
-      wait_st();
     };
-    if (nchunks > 0) {
+    // S^T[j][i] *= e^{Gamma_C, i} of chunk cc, ahead of that chunk's [S | O] GEMM
+    auto decay = [&](int cc) {
+      mbar_wait_bounded(&bars[B_OPER + (cc & 1)], (cc >> 1) & 1, abort_flag, P.sb, 5);
+      __syncwarp();
+      const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + (cc & 1) * 512);
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        tmem_ld32(tbase + lane_base + S_COL + 32 * q, v);
+        wait_ld();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 gg = g4[8 * q + k4];
+          v[4 * k4 + 0] *= gg.x;
+          v[4 * k4 + 1] *= gg.y;
+          v[4 * k4 + 2] *= gg.z;
+          v[4 * k4 + 3] *= gg.w;
+        }
+        tmem_st32(tbase + lane_base + S_COL + 32 * q, v);
+      }
+      wait_st();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_DECAY]);
+    };
+    if (nchunks > 0) {  // chunk 0: bf16 S, seed, then the decay
+      write_sb();
       load_v(0);
       seed_op();
+      wait_st();
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_OREADY]);
+      decay(0);
     }
     for (int c = 0; c < nchunks; ++c) {
       if (bar_red_or(3, 128, *abort_flag != 0)) break;
       const int b = c & 1;
       const bool more = c + 1 < nchunks;
-      mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 5);
-      {  // S^T[j][i] *= e^{Gamma_C, i}, a 32-column block once the [O | P] k-steps
-         // that read it are done
-        const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + b * 512);
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          mbar_wait_bounded(&bars[B_UOQ + q], c & 1, abort_flag, P.sb, 6);
-          __syncwarp();
-          fence_after_sync();
-          float v[32];
-          tmem_ld32(tbase + lane_base + S_COL + 32 * q, v);
-          wait_ld();
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 gg = g4[8 * q + k4];
-            v[4 * k4 + 0] *= gg.x;
-            v[4 * k4 + 1] *= gg.y;
-            v[4 * k4 + 2] *= gg.z;
-            v[4 * k4 + 3] *= gg.w;
-          }
-          tmem_st32(tbase + lane_base + S_COL + 32 * q, v);
-        }
-        wait_st();
-      }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_DECAY]);
-      if (more) load_v(c + 1);
-
+      if (more) load_v(c + 1);  // while this chunk's GEMMs run
       mbar_wait_bounded(&bars[B_SO + b], (c >> 1) & 1, abort_flag, P.sb, 7);
       __syncwarp();
       fence_after_sync();
+      // critical path: bf16 S for the next [O | P], O read out, seed
+      if (more) write_sb();
       float vo[32];  // O^T (lane j, column r)
       tmem_ld32(tbase + lane_base + O_COL, vo);
       wait_ld();
-      if (more) seed_op();  // U of this chunk, the last reader of P, is done
+      if (more) seed_op();
+      wait_st();
       fence_before_sync();
       __syncwarp();
       if (more && lane == 0) mbar_arrive(&bars[B_OREADY]);
+      if (more) decay(c + 1);  // overlaps the next [O | P] and U GEMMs
       if (U.out_on) {  // lanes j, j^1 swap values so each writes a bf16 pair
         const int n = chunk_rows(c);
         const bool odd = lane & 1;
@@ -672,29 +699,29 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
   } else if (warp == ISSUE_W) {
     // ============================================ state-side MMA issue (lane 0)
     if (lane == 0) {
-      const uint32_t id_op = idesc(kFmtTF32, 128, 2 * C, false, false, false);    // [O^T | P^T]
+      const uint32_t id_op = idesc(kFmtBF16, 128, 2 * C, false, false, false);    // [O^T | P^T]
       const uint32_t id_u = idesc(kFmtTF32, 128, C, false, false, true);          // U^T = -P^T T^T
       const uint32_t id_so = idesc(kFmtTF32, 128, D + C, false, false, false);    // [S^T | O^T]
       for (int c = 0; c < nchunks; ++c) {
         if (*abort_flag) break;
         const int b = c & 1;
-        // [O^T | P^T] += S^T [Qg ; Ka]^T once the operands are written and O / P are
-        // seeded (which the state warps do after the previous [S | O] completed)
+        // [O^T | P^T] += S^T [Qg ; Ka]^T (bf16, A = the bf16 copy of S^T) once the
+        // operands are written and O / P are seeded (which the state warps do
+        // after the previous [S | O] completed)
         mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 10);
         mbar_wait_bounded(&bars[B_OREADY], c & 1, abort_flag, P.sb, 11);
         if (*abort_flag) break;
         fence_after_sync();
         const uint32_t hb = sb + SM_HB + b * HBB;
 #pragma unroll 1
-        for (int ks = 0; ks < 16; ++ks) {
-          mma_ts_tf32(tbase + O_COL, tbase + S_COL + 8 * ks,
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts_bf16(tbase + O_COL, tbase + SB_COL + 8 * ks,
                       sw128_desc(hb + H_QK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_op,
                       1);
-          if ((ks & 3) == 3) mma_commit(&bars[B_UOQ + (ks >> 2)]);
-        }
+        mma_commit(&bars[B_UO]);
         // U^T = -P^T T^T once P is complete and T is in
         mbar_wait_bounded(&bars[B_T + b], (c >> 1) & 1, abort_flag, P.sb, 12);
-        mbar_wait_bounded(&bars[B_UOQ + 3], c & 1, abort_flag, P.sb, 13);
+        mbar_wait_bounded(&bars[B_UO], c & 1, abort_flag, P.sb, 13);
         if (*abort_flag) break;
         fence_after_sync();
         const uint32_t kbb = sb + SM_KEY + b * KEYB;
@@ -724,6 +751,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     // ==================================== TMA and Gram issue (lane 0 of the last warp)
     if (lane == 0) {
       const uint32_t id_gram = idesc(kFmtBF16, 128, 2 * C, false, false, false);  // 2 halves
+      int nv = 0;  // v loads issued
       auto issue_qkg = [&](int cc) {  // into stage cc & 1
         const int row = (int)(U.row0 + (int64_t)cc * C);
         uint8_t* in = sm + (cc & 1) * STAGE;
@@ -733,12 +761,21 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         tma_load_3d(in + OFF_Q, &P.tm_q, bf, 0, h, row);
         tma_load_3d(in + OFF_K, &P.tm_k, bf, 0, h, row);
         tma_load_3d(in + OFF_G, &P.tm_g, bf, 0, h, row);
-        if (!U.vzero) {  // v follows once this chunk's Gram is done: warm L2 now
-          tma_prefetch_3d(&P.tm_v, 0, h, row);
-          tma_prefetch_3d(&P.tm_v, 64, h, row);
+        if (!U.vzero) {  // v into its ring slot, once the chunk 4 back has been read
+          const int vb = cc % NVBUF;
+          if (cc >= NVBUF &&
+              !mbar_wait_bounded(&bars[B_VEMPTY + vb], ((cc - NVBUF) / NVBUF) & 1, abort_flag,
+                                 P.sb, 18))
+            return;
+          uint8_t* dst = sm + SM_V + vb * 8192;
+          uint64_t* bv = &bars[B_V + vb];
+          mbar_arrive_expect_tx(bv, TX_V);
+          tma_load_3d(dst, &P.tm_v, bv, 0, h, row);
+          tma_load_3d(dst + 4096, &P.tm_v, bv, 64, h, row);
+          nv = cc + 1;
         }
       };
-      int nq = 0, nv = 0;  // TMA loads issued
+      int nq = 0;
       for (; nq < 2 && nq < nchunks; ++nq) issue_qkg(nq);
       for (int c = 0; c < nchunks; ++c) {
         if (*abort_flag) break;
@@ -759,18 +796,6 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
           if (*abort_flag) break;
           issue_qkg(nq++);
         }
-        // v of chunk c into its Gram operand region once that Gram is done
-        if (!U.vzero) {
-          mbar_wait_bounded(&bars[B_GRAM + b], (c >> 1) & 1, abort_flag, P.sb, 18);
-          if (*abort_flag) break;
-          const int row = (int)(U.row0 + (int64_t)c * C);
-          uint8_t* dst = sm + SM_KEY + b * KEYB + K_V;
-          uint64_t* bf = &bars[B_V + b];
-          mbar_arrive_expect_tx(bf, TX_V);
-          tma_load_3d(dst, &P.tm_v, bf, 0, h, row);
-          tma_load_3d(dst + 4096, &P.tm_v, bf, 64, h, row);
-          ++nv;
-        }
       }
       if (*abort_flag) {
         // every MMA and TMA load this thread issued lands before shared memory
@@ -779,8 +804,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         mbar_wait_drain(&bars[B_DRAIN + 1], 0);
         for (int k = (nq > 2 ? nq - 2 : 0); k < nq; ++k)
           mbar_wait_drain(&bars[B_IN_FULL + (k & 1)], (k >> 1) & 1);
-        for (int k = (nv > 2 ? nv - 2 : 0); k < nv; ++k)
-          mbar_wait_drain(&bars[B_V + (k & 1)], (k >> 1) & 1);
+        for (int k = (nv > NVBUF ? nv - NVBUF : 0); k < nv; ++k)
+          mbar_wait_drain(&bars[B_V + k % NVBUF], (k / NVBUF) & 1);
       }
     }
     __syncwarp();

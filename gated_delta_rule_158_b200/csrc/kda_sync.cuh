@@ -15,6 +15,7 @@ namespace kda {
 
 constexpr long long kWaitLimitNs = 2000000000LL;  // 2 s: far above any real wait
 constexpr int kFastPolls = 1 << 12;
+constexpr uint32_t kSuspendNs = 1000;  // longest single suspension in a bounded wait
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
@@ -71,6 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended for up to hint_ns until the
+// phase completes (it is woken as soon as it does), instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking: has the phase with the given parity completed?
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -109,13 +125,12 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 // polling loop is an out-of-line call, so the many call sites of a kernel
 // stay small in the instruction cache.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
-                                            volatile int* abort_flag, StatusBlock* sb,
-                                            int32_t detail) {
-  for (int i = 0; i < kFastPolls; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+                                                   volatile int* abort_flag, StatusBlock* sb,
+                                                   int32_t detail) {
+  // suspended waits of up to kSuspendNs each: no issue slots spent while waiting
   const unsigned long long t0 = global_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity, kSuspendNs)) return true;
     if (*abort_flag) return false;
     if ((long long)(global_ns() - t0) > kWaitLimitNs) {
       *abort_flag = 1;
