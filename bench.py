@@ -21,6 +21,7 @@ collective on the data path); the step time is the max over ranks.
 workload (the slow baseline), printing the same JSON keys.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -56,6 +57,35 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 4 + 256
 # counted once: C(3dk + 2dv) + C^2/3 + 6 dk dv
 def prefill_flops_per_token_head(C=32, dk=128, dv=128):
     return C * (3 * dk + 2 * dv) + C * C / 3 + 6 * dk * dv
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# chunk_tc_kernel launch, from the ncu capture summarised in
+# profiles/chunk_tc_kernel_prefill_B4_H32_T4096.md (128 (sequence, head) units
+# of 4096 tokens): 673.3 MB read + 121.9 MB written.  Traffic grows with the
+# units a launch processes, so a launch over U such units moves U times the
+# per-unit figure.  The figure belongs to the kernel sources it was taken on:
+# once they change it is reported as null until a new capture replaces it.
+CHUNK_TRAFFIC = {
+    "sources": ["gated_delta_rule_158_b200/csrc/kda_chunk_tc.cu",
+                "gated_delta_rule_158_b200/csrc/kda_sync.cuh",
+                "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
+                "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
+    "sha256": "07d77167d808c45bf1b7c6f7f105374f0be582b096684cf11aa65ba3f15409cb",
+    "bytes_per_unit_T4096": (673.334528e6 + 121.89952e6) / 128,
+}
+
+
+def chunk_traffic(B, H, T):
+    if T != 4096:
+        return None
+    h = hashlib.sha256()
+    for f in CHUNK_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != CHUNK_TRAFFIC["sha256"]:
+        return None
+    return round(B * H * CHUNK_TRAFFIC["bytes_per_unit_T4096"])
 
 
 def kernels_per_step(wl, B, T):
@@ -491,7 +521,8 @@ def bench_prefill_line(args, wl, world, rank, peaks):
                    "step": "kda_chunk_fwd_gated (gate fused)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                     "traffic": None, "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
+                     "traffic": chunk_traffic(B, H, T) if not wl.get("varlen") else None,
+                     "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
                      "kernel_ms": round(chunk_ms, 4), "algorithmic_bytes": alg_bytes,
                      "peak_source": peaks["src"],
                      "tensor_frac": round(flops / (chunk_ms * 1e-3) / (peaks["tc"] * 1e12), 4)},

@@ -881,19 +881,31 @@ bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base
 // Segment split for long dense sequences with too few (sequence, head)
 // units to occupy the GPU: returns G >= 2 and the segment length, or G = 1.
 void plan_split(int B, int T, int H, int num_sms, int* G_out, int* seg_out) {
-  // one CTA per SM: split when the units fill less than half the SMs, into
-  // as many segments as keep one unit-segment per SM
+  // one CTA per SM: split when the units fill less than half the SMs.  A split
+  // into G segments runs 2 (G - 1) U transition CTAs, then G U output CTAs,
+  // each over T / G tokens; take the G with the fewest waves per token, and
+  // a larger G only when it saves more than 5 % (each segment adds
+  // 3 x 64 KB of workspace per unit and a step of the serial combine).
   const int U = B * H;
   *G_out = 1;
   *seg_out = T;
   if (2 * U >= num_sms || T < 4 * 1024) return;
-  int G = num_sms / U;
   const int max_g = T / 1024;
-  if (G > max_g) G = max_g;
-  if (G < 2) return;
-  int seg = (T + G - 1) / G;
+  int best_g = 1;
+  double best_cost = 1.0;  // no split: one wave over T tokens
+  for (int G = 2; G <= max_g && G <= 64; ++G) {
+    const int w1 = (2 * (G - 1) * U + num_sms - 1) / num_sms;
+    const int w2 = (G * U + num_sms - 1) / num_sms;
+    const double cost = (double)(w1 + w2) / G;
+    if (cost < 0.95 * best_cost) {
+      best_cost = cost;
+      best_g = G;
+    }
+  }
+  if (best_g < 2) return;
+  int seg = (T + best_g - 1) / best_g;
   seg = (seg + C - 1) / C * C;
-  G = (T + seg - 1) / seg;
+  const int G = (T + seg - 1) / seg;
   if (G < 2) return;
   *G_out = G;
   *seg_out = seg;

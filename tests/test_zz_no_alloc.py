@@ -77,7 +77,7 @@ def test_noalloc_matches_workspace_entry_two_calls(case):
 
 
 def test_noalloc_rejects_oversized_problem():
-    """A million-token sequence over 32 heads needs ~56 MB of segment states,
+    """A million-token sequence over 32 heads needs ~12 MB of segment states,
     more than the built-in scratch: rejected before anything is enqueued."""
     need = kda.kda_chunk_fwd_workspace_size(1, 1 << 20, 32, 128, 128)
     assert need > (8 << 20)
