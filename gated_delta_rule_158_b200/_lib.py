@@ -38,6 +38,9 @@ _SIGNATURES = {
     "kda_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "kda_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
                            _F, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "kda_chunk_segment_transition": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _I, _I, _I, _I,
+                                          _I, _VP, _VP, _SZ, _VP]),
+    "kda_chunk_state_prefix": (_I, [_VP, _I, _I, _VP, _I, _I, _I, _I, _VP, _VP]),
     "kda_chunk_fwd_gated": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _VP, _I, _I, _I, _I,
                                  _I, _I, _F, _I, _VP, _VP, _VP, _SZ, _VP]),
     "kda_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _I, _I, _I, _I, _F, _VP, _VP]),
@@ -172,6 +175,29 @@ def kda_chunk_fwd_gated(q, k, v, z, A_log, beta, out, workspace, g_min=-5.0, ini
         _ptr(init_state), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, float(scale),
         int(chunk_size), _ptr(out), _ptr(final_state), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)), "kda_chunk_fwd_gated")
+
+
+def kda_chunk_segment_transition(q, k, v, z, A_log, beta, pairs, workspace, g_min=-5.0,
+                                 stream=None):
+    """Per (b, h) of the segment given: pairs[b, h, 0] = S~ (from a zero state),
+    pairs[b, h, 1] = M (the segment's transition); pairs fp32 [B, H, 2, 128, 128]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(lib().kda_chunk_segment_transition(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta), _dtype(q),
+        B, T, H, dk, dv, _ptr(pairs), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "kda_chunk_segment_transition")
+
+
+def kda_chunk_state_prefix(pairs, index, state_out, init_state=None, stream=None):
+    """Incoming state of segment `index` from the pairs [count, B, H, 2, dk, dv] of the
+    segments in order: S_in[0] = init (or 0), S_in[r + 1] = S~_r + M_r S_in[r]."""
+    count, B, H = pairs.shape[0], pairs.shape[1], pairs.shape[2]
+    dk, dv = pairs.shape[-2], pairs.shape[-1]
+    _check(lib().kda_chunk_state_prefix(_ptr(pairs), count, int(index), _ptr(init_state), B, H,
+                                        dk, dv, _ptr(state_out), _stream(stream)),
+           "kda_chunk_state_prefix")
 
 
 def kda_decode_step_gated(q, k, v, z, A_log, beta, state, out, g_min=-5.0, scale=1.0,

@@ -245,6 +245,70 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                         workspace, workspace_bytes, stream);
 }
 
+kda_status kda_chunk_segment_transition(const void* q, const void* k, const void* v,
+                                        const float* z, const float* A_log, float g_min,
+                                        const float* beta, kda_dtype in_dtype, int B, int T,
+                                        int H, int dk, int dv, float* pairs, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !z || !A_log || !beta || !pairs || !workspace)
+    return KDA_ERR_INVALID_ARG;
+  if (!(g_min < 0.f) || !isfinite(g_min)) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (!use_tc_path(in_dtype, dk, dv, 0)) return KDA_ERR_UNSUPPORTED;  // bf16, 128 x 128 only
+  if ((int64_t)B * H > (int64_t)1 << 30) return KDA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, z, A_log, beta, pairs, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {q, k, v, z, A_log, beta};
+  for (const void* i : ins)
+    if (i == pairs) return KDA_ERR_INVALID_ARG;
+  if (workspace_bytes < kStatusBytes) return KDA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  StatusBlock* sb = static_cast<StatusBlock*>(workspace);
+  if (cudaError_t em = cudaMemsetAsync(sb, 0, kStatusBytes, st)) return cuda_failure(em);
+  ChunkArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = z;
+  a.A_log = A_log;
+  a.g_min = g_min;
+  a.gated = true;
+  a.beta = beta;
+  a.dt = in_dtype;
+  a.map.status = sb;
+  a.map.B = B;
+  a.map.T = T;
+  a.map.H = H;
+  a.num_units = B * H;
+  a.dk = dk;
+  a.dv = dv;
+  a.scale = 1.f;
+  a.chunk = 32;
+  a.sb = sb;
+  const cudaError_t e = launch_chunk_tc_transition(a, pairs, st);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
+}
+
+kda_status kda_chunk_state_prefix(const float* pairs, int count, int index,
+                                  const float* init_state, int B, int H, int dk, int dv,
+                                  float* state_out, void* stream) {
+  if (!pairs || !state_out) return KDA_ERR_INVALID_ARG;
+  if (count <= 0 || index < 0 || index >= count || B <= 0 || H <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > (int64_t)1 << 30) return KDA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {pairs, init_state, state_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  if (state_out == pairs || (init_state && state_out == init_state)) return KDA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_state_prefix(pairs, count, index, init_state, B * H, state_out,
+                                            (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
+}
+
 kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* z,
                                const float* A_log, float g_min, const float* beta,
                                kda_dtype in_dtype, const float* init_state,

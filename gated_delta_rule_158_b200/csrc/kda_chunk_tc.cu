@@ -851,6 +851,43 @@ __global__ void __launch_bounds__(256) segment_combine_kernel(const float* __res
   }
 }
 
+// S_in of segment `index`: fold S_in <- S~_r + M_r S_in over r < index, from
+// pairs laid out [count][units]{S~, M}; one 32-column slice per CTA.
+__global__ void __launch_bounds__(256) state_prefix_kernel(const float* __restrict__ pairs,
+                                                           int count, int index,
+                                                           const float* __restrict__ init,
+                                                           int units, float* __restrict__ out) {
+  __shared__ float X[D][33];
+  const size_t DD = (size_t)D * D;
+  const int un = blockIdx.x >> 2, j0 = (blockIdx.x & 3) * 32;
+  const int tid = threadIdx.x, jj = tid & 31, i0 = tid >> 5;
+  for (int k = 0; k < 16; ++k) {
+    const int i = i0 + 8 * k;
+    X[i][jj] = init ? init[un * DD + (size_t)i * D + j0 + jj] : 0.f;
+  }
+  __syncthreads();
+  for (int r = 0; r < index && r < count; ++r) {
+    const float* St = pairs + ((size_t)r * units + un) * 2 * DD;
+    const float* M = St + DD;
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = St[(size_t)(i0 + 8 * k) * D + j0 + jj];
+    for (int ip = 0; ip < D; ++ip) {
+      const float x = X[ip][jj];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = fmaf(__ldg(M + (size_t)(i0 + 8 * k) * D + ip), x, acc[k]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) X[i0 + 8 * k][jj] = acc[k];
+    __syncthreads();
+  }
+  for (int k = 0; k < 16; ++k) {
+    const int i = i0 + 8 * k;
+    out[un * DD + (size_t)i * D + j0 + jj] = X[i][jj];
+  }
+}
+
 // ------------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -982,6 +1019,54 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_by
   if (e != cudaSuccess) return e;
   P.mode = 2;
   chunk_tc_kernel<<<U * G, NT, SMEM_ALLOC, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStream_t stream) {
+  if (a.num_units == 0) return cudaSuccess;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  TcParams P;
+  memset(&P, 0, sizeof(P));
+  const int64_t R = (int64_t)a.map.B * a.map.T;
+  const int H = a.map.H;
+  if (!encode_3d(&P.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&P.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.k, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_3d(&P.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.v, H, R, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_3d(&P.tm_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.g, H, R, 128,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  P.A_log = a.gated ? a.A_log : nullptr;
+  P.g_min = a.g_min;
+  P.beta = a.beta;
+  P.sb = a.sb;
+  P.B = a.map.B;
+  P.T = a.map.T;
+  P.H = H;
+  P.scale = 1.f;
+  // transition mode over the whole range as the one segment before a second:
+  // CTA pair u = (S~ from zero with v, M from the identity with v = 0)
+  P.mode = 1;
+  P.G = 2;
+  P.seg_len = a.map.T;
+  P.seg_ws = pairs;
+  chunk_tc_kernel<<<a.num_units * 2, NT, SMEM_ALLOC, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_prefix(const float* pairs, int count, int index, const float* init,
+                                int units, float* state_out, cudaStream_t stream) {
+  if (units == 0) return cudaSuccess;
+  state_prefix_kernel<<<units * 4, 256, 0, stream>>>(pairs, count, index, init, units,
+                                                     state_out);
   return cudaGetLastError();
 }
 

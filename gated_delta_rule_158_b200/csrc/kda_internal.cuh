@@ -121,6 +121,13 @@ size_t tc_workspace_bytes(int B, int T, int H, int num_seqs, int num_sms);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail,
                             size_t ws_tail_bytes, cudaStream_t stream);
 
+// Cross-device context parallelism: per (sequence, head) unit of the whole
+// [B, T] range, S~ (from a zero state) and M (the segment's transition) into
+// pairs[unit] = {S~, M}; and the incoming state of segment `index` of `count`.
+cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStream_t stream);
+cudaError_t launch_state_prefix(const float* pairs, int count, int index, const float* init,
+                                int units, float* state_out, cudaStream_t stream);
+
 cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns,
                                  cudaStream_t stream);
 

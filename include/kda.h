@@ -125,6 +125,47 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
                          size_t workspace_bytes, void *stream);
 
 /*
+ * Cross-device context parallelism, "NLP--技术报告解读-Kimi-K3"
+ * (joezjh.github.io), Infrastructure > KDA kernels (KCP): with a sequence
+ * cut into consecutive segments, the state a segment leaves is
+ * S_end = S~ + M S_in, where S~ is the state the segment leaves from a zero
+ * state and M (dk x dk) the product of its per-token transitions
+ * (I - beta_t k_t k_t^T) Diag(exp(g_t)).  Each device computes the pair of
+ * its own segment, the pairs are exchanged, and each device folds the pairs
+ * of the segments before its own into its incoming state.
+ *
+ * kda_chunk_segment_transition: the pair of every (b, h) over the T tokens
+ * of q, k, v, z, beta (layouts as kda_chunk_fwd_gated, gate fused):
+ *  pairs  : fp32 [B, H, 2, 128, 128]; pairs[b][h][0] = S~, pairs[b][h][1] = M
+ *           (row-major, M acts on the left of the state).  Must not alias an
+ *           input.
+ *  workspace : device buffer of >= 256 bytes (device status word, cleared
+ *           by this call).
+ * Supported: in_dtype KDA_BF16, dk = dv = 128 (KDA_ERR_UNSUPPORTED
+ * otherwise).  Errors as kda_chunk_fwd.
+ */
+KDA_API kda_status kda_chunk_segment_transition(const void *q, const void *k, const void *v,
+                                                const float *z, const float *A_log,
+                                                float g_min, const float *beta,
+                                                kda_dtype in_dtype, int B, int T, int H,
+                                                int dk, int dv, float *pairs, void *workspace,
+                                                size_t workspace_bytes, void *stream);
+
+/*
+ * kda_chunk_state_prefix: the incoming state of segment `index` of `count`
+ * consecutive segments: S_in[0] = init_state (or zeros if NULL),
+ * S_in[r + 1] = S~_r + M_r S_in[r].
+ *  pairs      : fp32 [count, B, H, 2, 128, 128], the segments' pairs in order
+ *               (as gathered from the devices); only the first `index` are read.
+ *  init_state : fp32 [B, H, 128, 128] or NULL.
+ *  state_out  : fp32 [B, H, 128, 128]; must not alias pairs or init_state.
+ * 0 <= index < count.  Supported: dk = dv = 128.
+ */
+KDA_API kda_status kda_chunk_state_prefix(const float *pairs, int count, int index,
+                                          const float *init_state, int B, int H, int dk,
+                                          int dv, float *state_out, void *stream);
+
+/*
  * kda_chunk_fwd with the gate fused in (the chunk kernels read z instead of
  * g and form g = g_min * Sigmoid(exp(A_log[h]) * z) on the fly, saving the
  * write and re-read of g):

@@ -153,3 +153,36 @@ def test_verify_replay_reject_on_host(L):
     assert L.kda_decode_replay(*bad) == _lib.KDA_ERR_INVALID_ARG
     bad = list(r); bad[8] = FAKE + 132    # misaligned accept_len
     assert L.kda_decode_replay(*bad) == _lib.KDA_ERR_MISALIGNED
+
+
+def test_kcp_entries_reject_on_host(L):
+    fake = 0x7F0000000000
+    ptr = lambda i: fake + 0x1000 * i
+    # fp32 inputs: only the bf16 tensor-core kernel has the transition mode
+    assert L.kda_chunk_segment_transition(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), -5.0, ptr(5),
+                                          kda.KDA_F32, 1, 64, 2, 128, 128, ptr(6), ptr(7),
+                                          256, None) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_segment_transition(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), -5.0, ptr(5),
+                                          kda.KDA_BF16, 1, 64, 2, 64, 64, ptr(6), ptr(7),
+                                          256, None) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_segment_transition(ptr(0), ptr(1), ptr(2), ptr(3), None, -5.0, ptr(5),
+                                          kda.KDA_BF16, 1, 64, 2, 128, 128, ptr(6), ptr(7),
+                                          256, None) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_segment_transition(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), -5.0, ptr(5),
+                                          kda.KDA_BF16, 1, 64, 2, 128, 128, ptr(6), ptr(7),
+                                          16, None) == kda.KDA_ERR_WORKSPACE
+    assert L.kda_chunk_segment_transition(ptr(0), ptr(1), ptr(2), ptr(3), ptr(4), -5.0, ptr(5),
+                                          kda.KDA_BF16, 1, 64, 2, 128, 128, ptr(0), ptr(7),
+                                          256, None) == kda.KDA_ERR_INVALID_ARG
+    # prefix: index must be in [0, count); 128 x 128 only; no aliasing
+    assert L.kda_chunk_state_prefix(ptr(0), 3, 3, None, 1, 2, 128, 128, ptr(1), None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_state_prefix(ptr(0), 3, -1, None, 1, 2, 128, 128, ptr(1), None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_state_prefix(ptr(0), 3, 1, None, 1, 2, 64, 64, ptr(1), None) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_state_prefix(ptr(0), 3, 1, ptr(1), 1, 2, 128, 128, ptr(1), None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_state_prefix(ptr(0) + 4, 3, 1, None, 1, 2, 128, 128, ptr(1), None) == \
+        kda.KDA_ERR_MISALIGNED
+
