@@ -64,26 +64,36 @@ def prefill_flops_per_token_head(C=32, dk=128, dv=128):
 # profiles/chunk_tc_kernel_prefill_B4_H32_T4096.md (128 (sequence, head) units
 # of 4096 tokens): 673.3 MB read + 121.9 MB written.  Traffic grows with the
 # units a launch processes, so a launch over U such units moves U times the
-# per-unit figure.  The figure belongs to the kernel sources it was taken on:
-# once they change it is reported as null until a new capture replaces it.
+# per-unit figure.  The figure belongs to the kernel it was taken on: the
+# text of kda_chunk_tc.cu up to the end of chunk_tc_kernel (its constants,
+# structures and body) and the headers it includes.  Once those change it is
+# reported as null until a new capture replaces it.
 CHUNK_TRAFFIC = {
-    "sources": ["gated_delta_rule_158_b200/csrc/kda_chunk_tc.cu",
-                "gated_delta_rule_158_b200/csrc/kda_sync.cuh",
+    "kernel_file": "gated_delta_rule_158_b200/csrc/kda_chunk_tc.cu",
+    "kernel_end_marker": "\n// S_in[g+1] = S~_g + M_g S_in[g]",
+    "headers": ["gated_delta_rule_158_b200/csrc/kda_sync.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
-    "sha256": "07d77167d808c45bf1b7c6f7f105374f0be582b096684cf11aa65ba3f15409cb",
+    "sha256": "8b9be6bb522022b9a7ab0e4946fba5c52ef1949669f168df23416608c3f0e006",
     "bytes_per_unit_T4096": (673.334528e6 + 121.89952e6) / 128,
 }
 
 
-def chunk_traffic(B, H, T):
-    if T != 4096:
+def chunk_kernel_source_hash():
+    with open(os.path.join(ROOT, CHUNK_TRAFFIC["kernel_file"]), encoding="utf-8") as fh:
+        text = fh.read()
+    end = text.find(CHUNK_TRAFFIC["kernel_end_marker"])
+    if end < 0:
         return None
-    h = hashlib.sha256()
-    for f in CHUNK_TRAFFIC["sources"]:
+    h = hashlib.sha256(text[:end].encode("utf-8"))
+    for f in CHUNK_TRAFFIC["headers"]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    if h.hexdigest() != CHUNK_TRAFFIC["sha256"]:
+    return h.hexdigest()
+
+
+def chunk_traffic(B, H, T):
+    if T != 4096 or chunk_kernel_source_hash() != CHUNK_TRAFFIC["sha256"]:
         return None
     return round(B * H * CHUNK_TRAFFIC["bytes_per_unit_T4096"])
 
