@@ -35,27 +35,28 @@
 //   [O^T | P^T] += S^T [q e^G ; k e^G]^T  onto [0 | -V^T]  (bf16, N = 64, 8 k-steps)
 //   U^T          = -P^T T^T,  i.e. U = T (V - k e^G S)       (tf32, N = 32)
 //   [S^T | O^T] += U^T [Kc ; A_qk]^T  after the decay        (tf32, N = 160, 4 k-steps)
-// The Gram is bf16 with A in shared memory, as M = 128, N = 64, K = 64: the
-// two 64-channel halves of [k;q] are stacked as rows against the two halves
-// of k, and the two diagonal blocks of the result are summed.
+// The Gram ([k;q] e^{G-G15} against k e^{G15-G}, 64 x 32 x 128) is small and
+// off the state chain: the solve warps compute it with warp-level bf16 MMAs
+// (mma.sync, fp32 accumulation) straight from the swizzled operand tiles, so
+// it costs the tcgen05 pipe nothing and its result is already in registers.
 //
 // The warps are specialised and hand work over through mbarriers, so the
 // key-side work of later chunks (which does not depend on the state)
 // overlaps the state-side chain of the current one:
 //   warps 0-3   prep: gate, in-chunk cumulative decay, rescaled operands
-//   warps 4-7   solve: Gram export, T = (I + A_kk)^-1 Diag(beta)
+//   warps 4-7   solve: Gram (warp MMA), T = (I + A_kk)^-1 Diag(beta)
 //   warps 8-11  state: once [S | O] of a chunk is done, the bf16 copy of S and
 //               the seed [0 | -V^T] of the next chunk's [O | P] (the critical
 //               path), then export of O and the next chunk's decay of S
 //   warp  12    one lane issues the state-side MMAs ([O | P], U, [S | O]) in
 //               chunk order, each after a blocking wait on what it needs
-//   warp  13    one lane issues the TMA loads and the Gram MMAs
+//   warp  13    one lane issues the TMA loads
 // Per-chunk operands are double-buffered by chunk parity (v four-deep); the
 // Gram operand region of a chunk is reused for T and the inverse's scratch
 // once the Gram is done.  Every wait is bounded (kda_sync.cuh).
 //
 // TMEM columns: S^T [0,128) | O^T [128,160) | P^T [160,192) | U^T [192,224)
-//               | Gram, 2 buffers [256,384) | bf16 S^T [384,448)
+//               | bf16 S^T [384,448)
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -73,7 +74,7 @@ constexpr int D = 128;   // dk = dv
 constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12, KEYISSUE_W = 13;
 constexpr int NT = 32 * 14;
 
-constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192, G_COL = 256;  // G: +64 b
+constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192;
 constexpr uint32_t SB_COL = 384;  // bf16 S^T: column c holds key channels 2c, 2c + 1
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -84,14 +85,11 @@ constexpr uint32_t OFF_K = 8192;    //   k bf16 [32][128]
 constexpr uint32_t OFF_G = 16384;   //   g or z fp32 [32][128]; in-chunk cumsum (log2) in prep
 constexpr uint32_t SM_KEY = 65536;  // key buffer b at SM_KEY + b * KEYB
 constexpr uint32_t KEYB = 24576;
-constexpr uint32_t K_KQL = 0;       //   Gram A: 128 rows x 64 channels bf16: rows 0-31 k e^{G-G15}
-                                    //   and 32-63 q e^{G-G15} of channels 0-63, rows 64-127
-                                    //   the same of channels 64-127
-constexpr uint32_t K_KB = 16384;    //   Gram B: 64 rows x 64 channels bf16: k e^{G15-G} of
-                                    //   channels 0-63 (rows 0-31) and 64-127 (rows 32-63)
-                                    //   and once the Gram GEMM is done:
-constexpr uint32_t K_PART = 0;      //   second-half Gram partials fp32 [2][32][32] (export),
-constexpr uint32_t K_TF = 4096;     //   then T fp32 [r][s] (tf32 B of U = -P^T T^T)
+constexpr uint32_t K_KQL = 0;       //   Gram A [k;q] e^{G-G15} bf16 64 x 128, per 64-channel
+                                    //   block 64 rows x 128 B (rows 0-31 k, 32-63 q)
+constexpr uint32_t K_KB = 16384;    //   Gram B k e^{G15-G} bf16 32 x 128, per block 32 x 128 B
+                                    //   and once the Gram is done:
+constexpr uint32_t K_TF = 4096;     //   T fp32 [r][s] (tf32 B of U = -P^T T^T)
 constexpr uint32_t K_AKKT = 16384;  //   A_kk^T fp32 [s][r] (inverse input)
 constexpr uint32_t K_XS = 20480;    //   inverse blocks, fp32 32 x 32
 constexpr uint32_t SM_HB = SM_KEY + 2 * KEYB;  // hand-off buffer b at SM_HB + b * HBB
@@ -117,17 +115,16 @@ enum : int {
   B_IN_FULL = 0,    // [2] TMA q, k, g landed                      (tx)
   B_IN_EMPTY = 2,   // [2] prep done with the input stage          (4 prep warps)
   B_OPER = 4,       // [2] chunk operands written                  (4 prep warps)
-  B_GRAM = 6,       // [2] Gram GEMM done                          (commit)
-  B_T = 8,          // [2] T and A_qk written                      (4 solve warps)
-  B_UO = 10,        //     [O | P] GEMM done                       (commit)
-  B_U = 11,         //     U GEMM done                             (commit)
-  B_DECAY = 12,     //     state decayed for the chunk             (4 state warps)
-  B_SO = 13,        // [2] [S | O] GEMM done                       (commit)
-  B_OREADY = 15,    //     bf16 S written, O read out, [O | P] seeded (4 state warps)
-  B_DRAIN = 16,     // [2] abort path: every MMA an issuing thread issued done (commit)
-  B_V = 18,         // [4] TMA v landed                            (tx)
-  B_VEMPTY = 22,    // [4] v buffer read                           (4 state warps)
-  NBARS = 26
+  B_T = 6,          // [2] T and A_qk written                      (4 solve warps)
+  B_UO = 8,         //     [O | P] GEMM done                       (commit)
+  B_U = 9,          //     U GEMM done                             (commit)
+  B_DECAY = 10,     //     state decayed for the chunk             (4 state warps)
+  B_SO = 11,        // [2] [S | O] GEMM done                       (commit)
+  B_OREADY = 13,    //     bf16 S written, O read out, [O | P] seeded (4 state warps)
+  B_DRAIN = 14,     //     abort path: every MMA the state issuer issued done (commit)
+  B_V = 15,         // [4] TMA v landed                            (tx)
+  B_VEMPTY = 19,    // [4] v buffer read                           (4 state warps)
+  NBARS = 23
 };
 static_assert(NBARS * 8 <= SM_TMEM - SM_BAR, "mbarrier space");
 
@@ -452,53 +449,66 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       uint8_t* hb = sm + SM_HB + b * HBB;
       const float* betas = reinterpret_cast<const float*>(sm + SM_BETA + b * 128);
       mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 3);
-      mbar_wait_bounded(&bars[B_GRAM + b], (c >> 1) & 1, abort_flag, P.sb, 4);
       __syncwarp();
-      fence_after_sync();
-      {  // Gram accumulator (lane quarter sw: k rows / q rows of channel half sw / 2,
-         // columns of the matching half of k) -> A_kk^T (x beta) and A_qk, in
-         // groups of 8 columns
-        const uint32_t gcol = tbase + lane_base + G_COL + 64 * b + (sw >= 2 ? 32 : 0);
-        float* part = reinterpret_cast<float*>(kb_buf + K_PART + (sw & 1) * 4096);
-        const int r = lane;
-        if (sw >= 2) {
-#pragma unroll 1
-          for (int g8 = 0; g8 < 4; ++g8) {
-            float v[8];
-            tmem_ld8(gcol + 8 * g8, v);
-            wait_ld();
+      {  // Gram: warp sw computes rows 16 sw .. +15 of [K_L ; Q_L] K_B^T (64 x 32,
+         // K = 128 channels) with m16n8k16 MMAs from the swizzled tiles, then
+         // A_kk^T (x beta, strictly lower; sw 0, 1) or A_qk (lower; sw 2, 3)
+        const uint32_t kbase = sb + SM_KEY + b * KEYB;
+        const int jm = lane >> 3, rr = lane & 7;
+        float acc[4][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) part[r * 32 + ((8 * g8 + e) ^ r)] = v[e];
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll 2
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t kb = (uint32_t)(kk >> 2), c16 = (uint32_t)((kk & 3) * 2);
+          const int arow = 16 * sw + rr + 8 * (jm & 1);  // matrices: rows x channel halves
+          const uint32_t ac = c16 + (uint32_t)(jm >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kbase + K_KQL + kb * 8192 + arow * 128 + ((ac ^ (uint32_t)(arow & 7)) << 4), a0,
+                  a1, a2, a3);
+#pragma unroll
+          for (int np = 0; np < 2; ++np) {  // n-tiles 2np, 2np + 1
+            const int brow = 8 * (2 * np + (jm >> 1)) + rr;
+            const uint32_t bc = c16 + (uint32_t)(jm & 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kbase + K_KB + kb * 4096 + brow * 128 + ((bc ^ (uint32_t)(brow & 7)) << 4), b0,
+                    b1, b2, b3);
+            mma_m16n8k16_bf16(acc[2 * np], a0, a1, a2, a3, b0, b1);
+            mma_m16n8k16_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
           }
         }
+        // A_kk^T goes where K_B was: every warp's Gram must be done first
         named_bar(2, 128);
+        // fragment: rows lane / 4 (+ 8), columns 8 nt + 2 (lane % 4) + {0, 1}
+        const int rl = lane >> 2, cq = 2 * (lane & 3);
         if (sw < 2) {
-          const float br = betas[r];
           float* akkt = reinterpret_cast<float*>(kb_buf + K_AKKT);
-#pragma unroll 1
-          for (int g8 = 0; g8 < 4; ++g8) {
-            float v[8];
-            tmem_ld8(gcol + 8 * g8, v);
-            wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] += part[r * 32 + ((8 * g8 + e) ^ r)];
-            if (sw == 0) {
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = 16 * sw + rl + 8 * hh;
+            const float br = betas[r];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int s2 = 8 * g8 + e;
-                akkt[s2 * 32 + r] = s2 < r ? br * v[e] : 0.f;
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int s2 = 8 * nt + cq + e;
+                akkt[s2 * 32 + r] = s2 < r ? br * acc[nt][2 * hh + e] : 0.f;
               }
-            } else {
+          }
+        } else {
 #pragma unroll
-              for (int h4 = 0; h4 < 2; ++h4) {
-                const int s4 = 2 * g8 + h4;
-                float4 w4;
-                w4.x = (4 * s4 + 0 <= r) ? v[4 * h4 + 0] : 0.f;
-                w4.y = (4 * s4 + 1 <= r) ? v[4 * h4 + 1] : 0.f;
-                w4.z = (4 * s4 + 2 <= r) ? v[4 * h4 + 2] : 0.f;
-                w4.w = (4 * s4 + 3 <= r) ? v[4 * h4 + 3] : 0.f;
-                *reinterpret_cast<float4*>(hb + H_AQK + r * 128 + ((s4 ^ (r & 7)) << 4)) = w4;
-              }
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = 16 * (sw - 2) + rl + 8 * hh;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+              const int s2 = 8 * nt + cq;
+              const float2 w2 = make_float2(s2 <= r ? acc[nt][2 * hh] : 0.f,
+                                            s2 + 1 <= r ? acc[nt][2 * hh + 1] : 0.f);
+              *reinterpret_cast<float2*>(hb + H_AQK + r * 128 +
+                                         ((((uint32_t)s2 >> 2) ^ (uint32_t)(r & 7)) << 4) +
+                                         (s2 & 3) * 4) = w2;
             }
           }
         }
@@ -748,9 +758,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     }
     __syncwarp();
   } else {
-    // ==================================== TMA and Gram issue (lane 0 of the last warp)
+    // ========================================= TMA issue (lane 0 of the last warp)
     if (lane == 0) {
-      const uint32_t id_gram = idesc(kFmtBF16, 128, 2 * C, false, false, false);  // 2 halves
       int nv = 0;  // v loads issued
       auto issue_qkg = [&](int cc) {  // into stage cc & 1
         const int row = (int)(U.row0 + (int64_t)cc * C);
@@ -777,31 +786,15 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       };
       int nq = 0;
       for (; nq < 2 && nq < nchunks; ++nq) issue_qkg(nq);
-      for (int c = 0; c < nchunks; ++c) {
+      for (int c = 0; c + 2 < nchunks; ++c) {
         if (*abort_flag) break;
-        const int b = c & 1;
-        // Gram GEMM of chunk c (bf16, M128 N64 K64) once its operands are written
-        mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 16);
-        if (*abort_flag) break;
-        fence_after_sync();
-        const uint32_t kbb = sb + SM_KEY + b * KEYB;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tbase + G_COL + 64 * b, sw128_desc(kbb + K_KQL + kk * 32, 16, 1024),
-                 sw128_desc(kbb + K_KB + kk * 32, 16, 1024), id_gram, 0, kk > 0);
-        mma_commit(&bars[B_GRAM + b]);
         // q, k, g of chunk c + 2 into the stage chunk c's prep has released
-        if (nq < nchunks) {
-          mbar_wait_bounded(&bars[B_IN_EMPTY + b], (c >> 1) & 1, abort_flag, P.sb, 17);
-          if (*abort_flag) break;
-          issue_qkg(nq++);
-        }
+        mbar_wait_bounded(&bars[B_IN_EMPTY + (c & 1)], (c >> 1) & 1, abort_flag, P.sb, 17);
+        if (*abort_flag) break;
+        issue_qkg(nq++);
       }
       if (*abort_flag) {
-        // every MMA and TMA load this thread issued lands before shared memory
-        // and TMEM are released
-        mma_commit(&bars[B_DRAIN + 1]);
-        mbar_wait_drain(&bars[B_DRAIN + 1], 0);
+        // every TMA load this thread issued lands before shared memory is released
         for (int k = (nq > 2 ? nq - 2 : 0); k < nq; ++k)
           mbar_wait_drain(&bars[B_IN_FULL + (k & 1)], (k >> 1) & 1);
         for (int k = (nv > NVBUF ? nv - NVBUF : 0); k < nv; ++k)

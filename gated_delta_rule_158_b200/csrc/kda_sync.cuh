@@ -126,11 +126,11 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 // stay small in the instruction cache.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                                    volatile int* abort_flag, StatusBlock* sb,
-                                                   int32_t detail) {
+                                                   int32_t detail, uint32_t hint_ns) {
   // suspended waits of up to kSuspendNs each: no issue slots spent while waiting
   const unsigned long long t0 = global_ns();
   for (;;) {
-    if (mbar_try_wait_hint(bar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
     if (*abort_flag) return false;
     if ((long long)(global_ns() - t0) > kWaitLimitNs) {
       *abort_flag = 1;
@@ -142,9 +142,10 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag, StatusBlock* sb,
-                                                  int32_t detail) {
+                                                  int32_t detail,
+                                                  uint32_t hint_ns = kSuspendNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag, sb, detail);
+  return mbar_wait_slow(bar, parity, abort_flag, sb, detail, hint_ns);
 }
 
 // Abort-path drain: waits (up to the time limit, whatever the abort flag says)

@@ -212,6 +212,28 @@ __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// ------------------------------------------- warp-level MMA (small GEMMs)
+// ldmatrix: lanes 8j .. 8j+7 give the row addresses (16 bytes each) of 8x8
+// b16 matrix j; lane t receives elements (t / 4, 2 (t % 4) .. +1) of matrix j
+// in register j.
+__device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(saddr));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col); fragments as in
+// the PTX ISA's m16n8k16 layout (lane groups of 4 share a row).
+__device__ __forceinline__ void mma_m16n8k16_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ------------------------------------------------------- swizzled smem writes
 // Byte offset of element `col` of row `row` inside a tile stored as 128-byte
 // swizzled column blocks of `rows` rows each; esz = element size in bytes.
