@@ -19,7 +19,10 @@
 //
 // Both keep one (sequence, head) state in registers for all K tokens, so the
 // fp32 state (dk*dv*4 bytes) crosses HBM once per launch instead of once per
-// token.  Thread layout and reductions follow kda_decode.cu.
+// token.  The value columns of the recurrence are independent given k, q, g
+// and beta, so for dv >= 64 each state is split over two CTAs by column halves:
+// half the registers per thread, four CTAs per SM, twice the loads in flight.
+// Thread layout and reductions follow kda_decode.cu.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -28,25 +31,31 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxK = 16;  // draft tokens per launch
 
+template <int DV>
+constexpr int cols_per_cta() { return DV >= 64 ? DV / 2 : DV; }
+
 template <typename Tin, int DK, int DV, bool VERIFY>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, (cols_per_cta<DV>() * DK <= 64 * 128) ? 4 : 2)
     decode_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         const Tin* __restrict__ v, const float* __restrict__ g,
                         const float* __restrict__ A_log, float g_min,
                         const float* __restrict__ beta, float* __restrict__ state,
                         const int32_t* __restrict__ accept_len, int H, int K, float scale,
                         Tin* __restrict__ out) {
-  constexpr int CG = DV / 4;
+  constexpr int DVC = cols_per_cta<DV>();  // value columns of this CTA
+  constexpr int NSPLIT = DV / DVC;
+  constexpr int CG = DVC / 4;
   constexpr int RG = kThreads / CG;
   constexpr int RPT = DK / RG;
   static_assert(RPT >= 1 && DK % RG == 0, "tile shape");
 
   __shared__ float sk[kMaxK][DK], sq[kMaxK][DK], sa[kMaxK][DK];
-  __shared__ float sv[kMaxK][DV], sb[kMaxK], skq[kMaxK];
+  __shared__ float sv[kMaxK][DVC], sb[kMaxK], skq[kMaxK];
   __shared__ float4 red_p[RG][CG], red_r[RG][CG];
-  __shared__ float se[DV];
+  __shared__ float se[DVC];
 
-  const int unit = blockIdx.x;  // n * H + h
+  const int unit = blockIdx.x / NSPLIT;  // n * H + h
+  const int j0 = (blockIdx.x % NSPLIT) * DVC;
   const int n = unit / H, h = unit % H;
   const int tid = threadIdx.x;
   const int cg = tid % CG, rg = tid / CG;
@@ -58,10 +67,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (steps == 0) return;  // nothing accepted: the committed state stands
   }
 
-  float4* S4 = reinterpret_cast<float4*>(state + (size_t)unit * DK * DV);
+  float4* S4 = reinterpret_cast<float4*>(state + (size_t)unit * DK * DV + j0);
   float4 s[RPT];
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) s[r] = S4[(rg + r * RG) * CG + cg];
+  for (int r = 0; r < RPT; ++r) s[r] = S4[(rg + r * RG) * (DV / 4) + cg];
 
   // inputs of the tokens, [N, K, H, *] layouts; g is the log-decay, or z
   // when A_log is given (gate fused in)
@@ -74,9 +83,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float gi = g[off];
     sa[t][i] = expf(A_log ? gate_value(gi, a_h, g_min) : gi);
   }
-  for (int idx = tid; idx < steps * DV; idx += kThreads) {
-    const int t = idx / DV, j = idx % DV;
-    sv[t][j] = Elem<Tin>::load(v + (((size_t)n * K + t) * H + h) * DV + j);
+  for (int idx = tid; idx < steps * DVC; idx += kThreads) {
+    const int t = idx / DVC, j = idx % DVC;
+    sv[t][j] = Elem<Tin>::load(v + (((size_t)n * K + t) * H + h) * DV + j0 + j);
   }
   for (int t = tid; t < steps; t += kThreads) sb[t] = beta[((size_t)n * K + t) * H + h];
   __syncthreads();
@@ -108,19 +117,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     red_p[rg][cg] = p;
     if (VERIFY) red_r[rg][cg] = rr;
     __syncthreads();
-    if (tid < DV) {
+    if (tid < DVC) {
       const float* rp = reinterpret_cast<const float*>(red_p);
       float pj = 0.f;
 #pragma unroll 8
-      for (int w = 0; w < RG; ++w) pj += rp[w * DV + tid];
+      for (int w = 0; w < RG; ++w) pj += rp[w * DVC + tid];
       const float e = sb[t] * (sv[t][tid] - pj);
       se[tid] = e;
       if (VERIFY) {
         const float* rq = reinterpret_cast<const float*>(red_r);
         float rj = 0.f;
 #pragma unroll 8
-        for (int w = 0; w < RG; ++w) rj += rq[w * DV + tid];
-        Elem<Tin>::store(out + (((size_t)n * K + t) * H + h) * DV + tid,
+        for (int w = 0; w < RG; ++w) rj += rq[w * DVC + tid];
+        Elem<Tin>::store(out + (((size_t)n * K + t) * H + h) * DV + j0 + tid,
                          scale * fmaf(skq[t], e, rj));
       }
     }
@@ -136,13 +145,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   if (!VERIFY) {
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) S4[(rg + r * RG) * CG + cg] = s[r];
+    for (int r = 0; r < RPT; ++r) S4[(rg + r * RG) * (DV / 4) + cg] = s[r];
   }
 }
 
 template <typename Tin, int DK, int DV, bool VERIFY>
 cudaError_t launch3(const DecodeMultiArgs& a, cudaStream_t st) {
-  decode_multi_kernel<Tin, DK, DV, VERIFY><<<(unsigned)(a.N * a.H), kThreads, 0, st>>>(
+  decode_multi_kernel<Tin, DK, DV, VERIFY>
+      <<<(unsigned)(a.N * a.H * (DV / cols_per_cta<DV>())), kThreads, 0, st>>>(
       static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
       a.g, a.A_log, a.g_min, a.beta, a.state, a.accept_len, a.H, a.K, a.scale,
       static_cast<Tin*>(a.out));
