@@ -62,7 +62,7 @@ def prefill_flops_per_token_head(C=32, dk=128, dv=128):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # chunk_tc_kernel launch, from the ncu capture summarised in
 # profiles/chunk_tc_kernel_prefill_B4_H32_T4096.md (128 (sequence, head) units
-# of 4096 tokens): 673.3 MB read + 121.9 MB written.  Traffic grows with the
+# of 4096 tokens): 673.3 MB read + 122.5 MB written.  Traffic grows with the
 # units a launch processes, so a launch over U such units moves U times the
 # per-unit figure.  The figure belongs to the kernel it was taken on: the
 # text of kda_chunk_tc.cu up to the end of chunk_tc_kernel (its constants,
@@ -74,8 +74,8 @@ CHUNK_TRAFFIC = {
     "headers": ["gated_delta_rule_158_b200/csrc/kda_sync.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
-    "sha256": "8b9be6bb522022b9a7ab0e4946fba5c52ef1949669f168df23416608c3f0e006",
-    "bytes_per_unit_T4096": (673.334528e6 + 121.89952e6) / 128,
+    "sha256": "bff3ac3e66af8c336fa3acabecf21b9cad274c66fb68fcbbee39f648d607464c",
+    "bytes_per_unit_T4096": (673.284096e6 + 122.502912e6) / 128,
 }
 
 
