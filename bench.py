@@ -74,7 +74,7 @@ CHUNK_TRAFFIC = {
     "headers": ["gated_delta_rule_158_b200/csrc/kda_sync.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
-    "sha256": "bff3ac3e66af8c336fa3acabecf21b9cad274c66fb68fcbbee39f648d607464c",
+    "sha256": "f4dca814e6685695ebfeead2206537af91e085ccaf75095b04b82703ee0cd5bd",
     "bytes_per_unit_T4096": (673.284096e6 + 122.502912e6) / 128,
 }
 

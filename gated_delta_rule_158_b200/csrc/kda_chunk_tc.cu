@@ -30,7 +30,7 @@
 // bf16 for that product, as is usual for chunked delta-rule kernels; it is
 // accumulated in fp32 throughout).  tcgen05.mma costs
 // a roughly fixed number of cycles per instruction up to N = 128-256
-// (measured: ~90 with A in TMEM, ~190 with A in shared memory), so products
+// (measured: ~90-125 with A in TMEM, ~190-210 with A in shared memory), so products
 // that share an A operand are fused into one wide MMA:
 //   [O^T | P^T] += S^T [q e^G ; k e^G]^T  onto [0 | -V^T]  (bf16, N = 64, 8 k-steps)
 //   U^T          = -P^T T^T,  i.e. U = T (V - k e^G S)       (tf32, N = 32)
@@ -71,7 +71,7 @@ using namespace tc;
 
 constexpr int C = 32;    // tokens per chunk
 constexpr int D = 128;   // dk = dv
-constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12, KEYISSUE_W = 13;
+constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12;  // warp 13: TMA issue
 constexpr int NT = 32 * 14;
 
 constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192;
