@@ -14,6 +14,9 @@ forward(q, k, v, g, beta, ...)
     Same page and section, state-update equation: the sequential recurrence
     S_t = (I - b_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + b_t k_t v_t^T and
     o_t = scale * S_t^T q_t, token by token in fp64.
+backward(q, k, v, g, beta, dout, ...)
+    Gradients of a loss through that recurrence (reverse-mode chain rule on
+    the same steps; the pages give the forward only), dense layout, fp64.
 
 Every function is pinned by tests/test_oracle_pins.py (closed forms,
 invariants, brute-force product form, special cases).
@@ -44,6 +47,13 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
+        lib.kda_oracle_backward.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [
+            ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         _lib = lib
     return _lib
 
@@ -114,3 +124,30 @@ def forward(q, k, v, g, beta, init_state=None, cu_seqlens=None,
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return o, S_out
+
+
+def backward(q, k, v, g, beta, dout, init_state=None, d_final=None, scale: float = 1.0):
+    """Gradients of L = sum(o * dout) + sum(S_T * d_final) with respect to
+    q, k, v, g, beta and the initial state, dense layout [B, T, H, *],
+    in fp64.  Returns a dict with keys dq, dk, dv, dg, dbeta, dS0."""
+    q, k, v, g, beta, dout = (_f64(a) for a in (q, k, v, g, beta, dout))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and g.shape == q.shape
+    assert v.shape == (B, T, H, dv) and dout.shape == v.shape and beta.shape == (B, T, H)
+    S0 = None if init_state is None else _f64(init_state)
+    dF = None if d_final is None else _f64(d_final)
+    for s_ in (S0, dF):
+        if s_ is not None:
+            assert s_.shape == (B, H, dk, dv)
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dg=np.zeros_like(g), dbeta=np.zeros_like(beta),
+               dS0=np.zeros((B, H, dk, dv)))
+    rc = _load().kda_oracle_backward(
+        B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+        _ptr(dout), _ptr(dF), float(scale), _ptr(out["dq"]), _ptr(out["dk"]),
+        _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]))
+    if rc != 0:
+        raise MemoryError("oracle backward: out of memory")
+    return out
+

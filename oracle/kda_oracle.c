@@ -180,3 +180,145 @@ int kda_oracle_forward(int num_seqs, const int64_t *seq_off, int H, int dk,
   pthread_mutex_destroy(&J.lock);
   return 0;
 }
+
+/* ------------------------------------------------------------- backward */
+
+/* Gradients of a loss through the same recurrence, by reverse-mode
+ * differentiation of the steps written above (the pages give the forward
+ * only; this is the chain rule applied to it, step by step).  Dense layout,
+ * one (b, h) unit at a time, all states of the forward kept:
+ *
+ *   forward   S'_t = Diag(a_t) S_{t-1},  a_t = exp(g_t)
+ *             p_t = S'_t^T k_t,  e_t = beta_t (v_t - p_t)
+ *             S_t = S'_t + k_t e_t^T,  o_t = scale S_t^T q_t
+ *
+ *   backward  with G = dL/dS_t (starting from dL/dS_T = d_final, or 0):
+ *             G    += scale q_t do_t^T          dq_t  = scale S_t do_t
+ *             de    = G^T k_t                   dk_t  = G e_t + S'_t dp
+ *             dv_t  = beta_t de                 dbeta = de . (v_t - p_t)
+ *             dp    = -beta_t de                G'    = G + k_t dp^T
+ *             da_i  = sum_j G'_ij S_{t-1,ij}    dg_t  = da * a_t
+ *             G     = Diag(a_t) G'   (= dL/dS_{t-1});   dS_0 = final G.
+ *
+ * Inputs q, k, g [B, T, H, dk]; v, dout [B, T, H, dv]; beta [B, T, H];
+ * S0, dfinal [B, H, dk, dv] or NULL (zeros).  Outputs of the same shapes:
+ * dq, dk, dg, dv, dbeta, dS0 (dS0 may be NULL).  Returns 0, or -1 when out of
+ * memory. */
+int kda_oracle_backward(int B, int64_t T, int H, int dk, int dv, const double *q,
+                        const double *k, const double *v, const double *g,
+                        const double *beta, const double *S0, const double *dout,
+                        const double *dfinal, double scale, double *dq, double *dk_out,
+                        double *dv_out, double *dg, double *dbeta, double *dS0) {
+  const int64_t SZ = (int64_t)dk * dv;
+  double *St = (double *)malloc(sizeof(double) * (size_t)((T + 1) * SZ));
+  double *G = (double *)malloc(sizeof(double) * (size_t)SZ);
+  double *Sp = (double *)malloc(sizeof(double) * (size_t)SZ);
+  double *p = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *e = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *de = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *dp = (double *)malloc(sizeof(double) * (size_t)dv);
+  if (!St || !G || !Sp || !p || !e || !de || !dp) {
+    free(St); free(G); free(Sp); free(p); free(e); free(de); free(dp);
+    return -1;
+  }
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < H; ++h) {
+      const int64_t unit = (int64_t)b * H + h;
+      /* forward, keeping S_0 .. S_T */
+      for (int64_t x = 0; x < SZ; ++x) St[x] = S0 ? S0[unit * SZ + x] : 0.0;
+      for (int64_t t = 0; t < T; ++t) {
+        const int64_t r = (int64_t)b * T + t;
+        const double *kt = k + (r * H + h) * (int64_t)dk;
+        const double *vt = v + (r * H + h) * (int64_t)dv;
+        const double *gt = g + (r * H + h) * (int64_t)dk;
+        const double bt = beta[r * H + h];
+        const double *prev = St + t * SZ;
+        double *cur = St + (t + 1) * SZ;
+        for (int i = 0; i < dk; ++i) {
+          const double a = exp(gt[i]);
+          for (int j = 0; j < dv; ++j) cur[i * dv + j] = a * prev[i * dv + j];
+        }
+        for (int j = 0; j < dv; ++j) p[j] = 0.0;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) p[j] += cur[i * dv + j] * kt[i];
+        for (int j = 0; j < dv; ++j) e[j] = bt * (vt[j] - p[j]);
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) cur[i * dv + j] += kt[i] * e[j];
+      }
+      /* backward */
+      for (int64_t x = 0; x < SZ; ++x) G[x] = dfinal ? dfinal[unit * SZ + x] : 0.0;
+      for (int64_t t = T - 1; t >= 0; --t) {
+        const int64_t r = (int64_t)b * T + t;
+        const double *qt = q + (r * H + h) * (int64_t)dk;
+        const double *kt = k + (r * H + h) * (int64_t)dk;
+        const double *vt = v + (r * H + h) * (int64_t)dv;
+        const double *gt = g + (r * H + h) * (int64_t)dk;
+        const double *dot = dout + (r * H + h) * (int64_t)dv;
+        const double bt = beta[r * H + h];
+        const double *pre = St + t * SZ, *post = St + (t + 1) * SZ;
+        double *dqt = dq + (r * H + h) * (int64_t)dk;
+        double *dkt = dk_out + (r * H + h) * (int64_t)dk;
+        double *dvt = dv_out + (r * H + h) * (int64_t)dv;
+        double *dgt = dg + (r * H + h) * (int64_t)dk;
+        /* output: o_t = scale S_t^T q_t */
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) G[i * dv + j] += scale * qt[i] * dot[j];
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) acc += post[i * dv + j] * dot[j];
+          dqt[i] = scale * acc;
+        }
+        /* recompute S'_t, p_t, e_t */
+        for (int i = 0; i < dk; ++i) {
+          const double a = exp(gt[i]);
+          for (int j = 0; j < dv; ++j) Sp[i * dv + j] = a * pre[i * dv + j];
+        }
+        for (int j = 0; j < dv; ++j) p[j] = 0.0;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) p[j] += Sp[i * dv + j] * kt[i];
+        for (int j = 0; j < dv; ++j) e[j] = bt * (vt[j] - p[j]);
+        /* S_t = S' + k e^T */
+        for (int j = 0; j < dv; ++j) de[j] = 0.0;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) de[j] += G[i * dv + j] * kt[i];
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) acc += G[i * dv + j] * e[j];
+          dkt[i] = acc;
+        }
+        /* e = beta (v - p) */
+        double db = 0.0;
+        for (int j = 0; j < dv; ++j) {
+          dvt[j] = bt * de[j];
+          db += de[j] * (vt[j] - p[j]);
+          dp[j] = -bt * de[j];
+        }
+        dbeta[r * H + h] = db;
+        /* p = S'^T k: G' = G + k dp^T, dk += S' dp */
+        for (int i = 0; i < dk; ++i) {
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            G[i * dv + j] += kt[i] * dp[j];
+            acc += Sp[i * dv + j] * dp[j];
+          }
+          dkt[i] += acc;
+        }
+        /* S' = Diag(a) S_{t-1} */
+        for (int i = 0; i < dk; ++i) {
+          const double a = exp(gt[i]);
+          double acc = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            acc += G[i * dv + j] * pre[i * dv + j];
+            G[i * dv + j] *= a;
+          }
+          dgt[i] = acc * a;
+        }
+      }
+      if (dS0)
+        for (int64_t x = 0; x < SZ; ++x) dS0[unit * SZ + x] = G[x];
+    }
+  }
+  free(St); free(G); free(Sp); free(p); free(e); free(de); free(dp);
+  return 0;
+}
+
