@@ -376,6 +376,47 @@ def run_spec_decode(device, N=256, H=32, d=128, K=4, reps=50, seed=7):
     return res, bytes_verify, bytes_replay, K
 
 
+# --------------------------------------------------------------- backward
+# Algorithmic bytes of the backward per token-head at d = 128 with bf16 q, k,
+# v, dout: those four read (4 x 256 B), g fp32 read (512 B), beta (4 B), and
+# dq, dk, dg, dv fp32 written (4 x 512 B), dbeta (4 B).
+BWD_BYTES_PER_TOKEN_HEAD = 4 * 256 + 512 + 4 + 4 * 512 + 4
+
+
+def run_backward(device, B=8, H=32, T=4096, d=128, reps=3, seed=3):
+    """kda_recurrent_bwd on the prefill workload's shape (bf16 inputs, with an
+    initial state and a final-state gradient).  Returns the per-launch time
+    and the algorithmic bytes of one launch (states read and written once)."""
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=seed, device=device,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, d, dk=d, seed=seed + 1, device=device)
+    g = torch.empty_like(inp["z"])
+    kda.kda_gate_fwd(inp["z"], inp["A_log"], g)
+    f32 = lambda *s: torch.empty(s, dtype=torch.float32, device=device)
+    grads = dict(dq=f32(B, T, H, d), dk=f32(B, T, H, d), dv=f32(B, T, H, d),
+                 dg=f32(B, T, H, d), dbeta=f32(B, T, H), d_init=f32(B, H, d, d))
+    ws = torch.empty(kda.kda_recurrent_bwd_workspace_size(B, T, H, d, d), dtype=torch.uint8,
+                     device=device)
+
+    def run():
+        kda.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], cot["dout"], grads,
+                              ws, init_state=inp["init_state"], d_final=cot["d_final"])
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    alg = B * T * H * BWD_BYTES_PER_TOKEN_HEAD + B * H * d * d * 4 * 3
+    return ms, alg, B * T
+
+
 # ------------------------------------------------------- oracle baseline
 def oracle_prefill_parallel_sample(wl, inp, cu, budget_s=15.0):
     """Same as above but runs the oracle's own thread pool over a batch of
@@ -463,6 +504,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",
                     help="skip nvidia-smi clock sampling (profiling runs)")
     ap.add_argument("--batch", type=int, default=None,
@@ -574,6 +616,17 @@ def bench_prefill_line(args, wl, world, rank, peaks):
             "replay_roofline": {"bound": "hbm", "achieved": round(br / (res["replay"] * 1e-3) / 1e9, 1),
                                 "peak": peaks["hbm"], "unit": "GB/s",
                                 "frac": round(br / (res["replay"] * 1e-3) / 1e9 / peaks["hbm"], 4)}}
+    if not args.no_backward and args.workload == "prefill":
+        torch.cuda.empty_cache()
+        ms, alg, ntok = run_backward(dev)
+        ach = alg / (ms * 1e-3) / 1e9
+        line["backward"] = {
+            "workload": "backward B8 H32 T4096 d128, bf16 q/k/v/dout, fp32 gradients",
+            "value": round(ntok / (ms * 1e-3) / 1e6, 4), "unit": "Mtokens/s",
+            "ms_per_launch": round(ms, 3),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
+                         "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
+                         "kernel": "bwd_kernel (kda_recurrent_bwd)", "algorithmic_bytes": alg}}
     return line
 
 

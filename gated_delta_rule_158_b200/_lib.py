@@ -52,6 +52,9 @@ _SIGNATURES = {
                                _VP, _VP]),
     "kda_decode_replay": (_I, [_VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I,
                                _VP]),
+    "kda_recurrent_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "kda_recurrent_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F,
+                               _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
@@ -239,6 +242,26 @@ def kda_decode_replay(k, v, g, beta, state, accept_len, A_log=None, g_min=-5.0, 
     _check(lib().kda_decode_replay(_ptr(k), _ptr(v), _ptr(g), _ptr(A_log), float(g_min),
                                    _ptr(beta), _dtype(k), _ptr(state), _ptr(accept_len), N, H, K,
                                    dk, dv, _stream(stream)), "kda_decode_replay")
+
+
+def kda_recurrent_bwd_workspace_size(B, T, H, dk, dv) -> int:
+    return int(lib().kda_recurrent_bwd_workspace_size(B, T, H, dk, dv))
+
+
+def kda_recurrent_bwd(q, k, v, g, beta, dout, grads, workspace, init_state=None, d_final=None,
+                      scale=1.0, stream=None):
+    """Gradients through the recurrence.  q, k, g [B,T,H,dk]; v, dout
+    [B,T,H,dv]; beta [B,T,H].  `grads` is a dict of fp32 output tensors
+    dq, dk, dg [B,T,H,dk], dv [B,T,H,dv], dbeta [B,T,H] and optionally
+    d_init [B,H,dk,dv]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(lib().kda_recurrent_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q), _ptr(init_state), _ptr(dout),
+        _ptr(d_final), B, T, H, dk, dv, float(scale), _ptr(grads["dq"]), _ptr(grads["dk"]),
+        _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["dbeta"]), _ptr(grads.get("d_init")),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "kda_recurrent_bwd")
 
 
 def kda_get_device_status(workspace, stream=None):

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "kda_internal.cuh"
+#include "kda_bwd.cuh"
 #include "kda_sync.cuh"
 
 namespace kda {
@@ -410,6 +411,46 @@ kda_status kda_decode_replay(const void* k, const void* v, const float* g, const
   DecodeMultiArgs a{nullptr, k, v, g, A_log, g_min, beta, in_dtype, state, accept_len, nullptr,
                     N, H, K, dk, dv, 1.f};
   const cudaError_t e = launch_decode_multi(a, false, (cudaStream_t)stream);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
+}
+
+size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+  if (B <= 0 || T < 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+  return bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
+kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, kda_dtype in_dtype, const float* init_state,
+                             const void* dout, const float* d_final, int B, int T, int H, int dk,
+                             int dv, float scale, float* dq, float* dk_out, float* dv_out,
+                             float* dg, float* dbeta, float* d_init, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (B <= 0 || T < 0 || H <= 0 || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !dout || !dq || !dk_out || !dv_out || !dg ||
+                !dbeta))
+    return KDA_ERR_INVALID_ARG;
+  if ((int64_t)B * H > 0x7fffffffLL || (int64_t)B * T * H > 0x7fffffffLL)
+    return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < bwd_workspace_bytes(B, T, H, dk, dv))
+    return KDA_ERR_WORKSPACE;
+  const void* ptrs[] = {q, k, v, g, beta, init_state, dout, d_final, dq, dk_out, dv_out, dg,
+                        dbeta, d_init, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* ins[] = {q, k, v, g, beta, init_state, dout, d_final, workspace};
+  const void* outs[] = {dq, dk_out, dv_out, dg, dbeta, d_init};
+  for (const void* o : outs) {
+    if (!o) continue;
+    for (const void* i : ins)
+      if (i == o) return KDA_ERR_INVALID_ARG;
+  }
+  if (T == 0 && !d_init) return KDA_OK;
+  BwdArgs a{q,  k,  v,     g,     beta,   init_state, dout,   d_final, in_dtype, B,
+            T,  H,  dk,    dv,    scale,  dq,         dk_out, dv_out,  dg,       dbeta,
+            d_init, static_cast<float*>(workspace)};
+  const cudaError_t e = launch_bwd(a, (cudaStream_t)stream);
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 

@@ -1,0 +1,34 @@
+// kda_bwd.cuh -- declarations of the backward kernel's launcher.
+#pragma once
+
+#include "kda_internal.cuh"
+
+namespace kda {
+
+// Backward through the recurrence (token by token, fp32): per (sequence,
+// head) the gradients of q, k, v, g, beta and the initial state.
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  const float* init;    // nullable: zero initial state
+  const void* dout;     // same element type as q
+  const float* dfinal;  // nullable: no gradient on the final state
+  kda_dtype dt;
+  int B, T, H, dk_dim, dv_dim;
+  float scale;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dg;
+  float* dbeta;
+  float* dinit;  // nullable
+  float* ws;     // bwd_workspace_bytes(B, T, H, dk, dv), 16-byte aligned
+};
+
+size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+
+}  // namespace kda

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   __shared__ float sk[DK], sq[DK], sa[DK];
   __shared__ float4 red_p[RG][CG], red_r[RG][CG];
-  __shared__ float se[DV];
+  __shared__ __align__(16) float se[DV];  // read back as float4
   __shared__ float s_kq;
 
   const int unit = blockIdx.x;  // n * H + h

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kThreads, (cols_per_cta<DV>() * DK <= 64 * 128
   __shared__ float sk[kMaxK][DK], sq[kMaxK][DK], sa[kMaxK][DK];
   __shared__ float sv[kMaxK][DVC], sb[kMaxK], skq[kMaxK];
   __shared__ float4 red_p[RG][CG], red_r[RG][CG];
-  __shared__ float se[DVC];
+  __shared__ __align__(16) float se[DVC];  // read back as float4
 
   const int unit = blockIdx.x / NSPLIT;  // n * H + h
   const int j0 = (blockIdx.x % NSPLIT) * DVC;

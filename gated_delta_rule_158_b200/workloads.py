@@ -88,6 +88,20 @@ def make_prefill_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, seed=0,
     return dict(q=q, k=k, v=v, z=z, A_log=A_log, beta=beta, init_state=S0)
 
 
+def make_backward_cotangents(B, T, H, dv, dk=None, dtype=torch.bfloat16, seed=0,
+                             device="cpu"):
+    """Seeded upstream gradients for the backward: dout [B, T, H, dv]
+    (dtype, unit-variance Gaussian) and, when dk is given, d_final
+    [B, H, dk, dv] fp32 (Gaussian, std 0.1); otherwise d_final is None."""
+    gen = _gen(seed, device)
+    dout = _normal((B, T, H, dv), gen, device, dtype, slab_dim=1)
+    d_final = None
+    if dk is not None:
+        d_final = 0.1 * torch.randn((B, H, dk, dv), generator=gen, device=device,
+                                    dtype=torch.float32)
+    return dict(dout=dout, d_final=d_final)
+
+
 def make_decode_state(N, H, dk, dv, seed, device):
     gen = _gen(seed, device)
     return 0.02 * torch.randn((N, H, dk, dv), generator=gen, device=device,

@@ -245,6 +245,36 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
                              int dk, int dv, void *stream);
 
 /*
+ * Training backward: gradients of a loss L through the recurrence, given
+ * dL/do (dout) and, optionally, dL/dS_T of the final state (d_final).  The
+ * pages define the forward only (Model Architecture > Kimi Delta Attention
+ * (KDA); FlashKDA serves training too: Infrastructure > KDA kernels); this
+ * is the chain rule applied to each step
+ *   S'_t = Diag(exp(g_t)) S_{t-1},  p_t = S'_t^T k_t,  e_t = beta_t (v_t - p_t),
+ *   S_t = S'_t + k_t e_t^T,  o_t = scale S_t^T q_t,
+ * in reverse token order, with the states recomputed from saved checkpoints.
+ *  q, k, g : [B, T, H, dk]   v, dout : [B, T, H, dv]   beta : fp32 [B, T, H]
+ *  init_state, d_final : fp32 [B, H, dk, dv] or NULL (zeros)
+ * Outputs (fp32, written whole; d_init may be NULL to skip it):
+ *  dq, dk_out, dg : [B, T, H, dk]   dv_out : [B, T, H, dv]   dbeta : [B, T, H]
+ *  d_init : [B, H, dk, dv]  (dL/dS_0)
+ * dout has the element type of q, k, v.  g is the log-decay (a gated caller
+ * chains dg through its gate).  Dense batches only.  The workspace (size from
+ * kda_recurrent_bwd_workspace_size, 0 for unsupported shapes) is scratch;
+ * outputs must not alias inputs.
+ * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
+ */
+KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+
+KDA_API kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta, kda_dtype in_dtype,
+                             const float *init_state, const void *dout,
+                             const float *d_final, int B, int T, int H, int dk,
+                             int dv, float scale, float *dq, float *dk_out,
+                             float *dv_out, float *dg, float *dbeta, float *d_init,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Name and description of the last CUDA error a libkda call on this host
  * thread turned into KDA_ERR_CUDA ("no error" if none).  Static storage.
  */

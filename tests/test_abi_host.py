@@ -186,3 +186,35 @@ def test_kcp_entries_reject_on_host(L):
     assert L.kda_chunk_state_prefix(ptr(0) + 4, 3, 1, None, 1, 2, 128, 128, ptr(1), None) == \
         kda.KDA_ERR_MISALIGNED
 
+
+
+def test_backward_entries_reject_on_host(L):
+    ptr = lambda i: FAKE + 0x1000 * i
+    ws = L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128)
+    # (64 + 2 checkpoint blocks of 64 tokens) x B*H states of 64 KB
+    assert ws == (64 + 2) * 2 * 128 * 128 * 4
+    assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 96, 128) == 0
+
+    def args(**over):
+        a = dict(q=ptr(0), k=ptr(1), v=ptr(2), g=ptr(3), beta=ptr(4), dt=kda.KDA_BF16,
+                 init=None, dout=ptr(5), dfinal=None, B=1, T=100, H=2, dk=128, dv=128,
+                 scale=1.0, dq=ptr(6), dko=ptr(7), dvo=ptr(8), dg=ptr(9), dbeta=ptr(10),
+                 dinit=None, ws=ptr(11), wsb=ws, stream=None)
+        a.update(over)
+        return list(a.values())
+
+    assert L.kda_recurrent_bwd(*args(dk=96)) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_recurrent_bwd(*args(dt=7)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(dout=None)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(B=0)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(scale=float("nan"))) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(wsb=ws - 16)) == kda.KDA_ERR_WORKSPACE
+    assert L.kda_recurrent_bwd(*args(ws=None)) == kda.KDA_ERR_WORKSPACE
+    assert L.kda_recurrent_bwd(*args(dg=ptr(9) + 4)) == kda.KDA_ERR_MISALIGNED
+    assert L.kda_recurrent_bwd(*args(dq=ptr(0))) == kda.KDA_ERR_INVALID_ARG  # dq aliases q
+    assert L.kda_recurrent_bwd(*args(dinit=ptr(11))) == kda.KDA_ERR_INVALID_ARG  # aliases ws
+    # empty sequence with no d_init requested: nothing to do, nothing launched
+    ws0 = L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128)
+    assert L.kda_recurrent_bwd(*args(T=0, q=None, k=None, v=None, g=None, beta=None, dout=None,
+                                     dq=None, dko=None, dvo=None, dg=None, dbeta=None,
+                                     wsb=ws0)) == kda.KDA_OK

@@ -1,0 +1,146 @@
+"""GPU parity of the training backward (kda_recurrent_bwd, through the C ABI)
+against the fp64 oracle backward.
+
+The kernel reads q, k, v, dout in their element type and computes in fp32
+from there on, so bf16 inputs change nothing in the arithmetic: the oracle
+takes the same bf16 values, widened exactly.  Every gradient is held to the
+fp32 bound (relative L2 <= 1e-5).  An fp32 re-run of the same token-by-token
+chain rule on the CPU lands near 2e-7 on these shapes, so the bound leaves a
+factor of ~50 for the different summation order and expf.  Every output is
+filled with NaN first, so an element the kernel fails to write fails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_158_b200 as kda
+from gated_delta_rule_158_b200 import workloads as W
+
+from kda_testutil import TOL_F32, gpu_gate, rel_l2, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+NAMES = ("dq", "dk", "dv", "dg", "dbeta")
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def gpu_backward(inp, cot, g, scale, with_init, with_dfinal, want_dinit=True):
+    q, v = inp["q"], inp["v"]
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    nan = lambda *s: torch.full(s, float("nan"), device=DEV)
+    grads = dict(dq=nan(B, T, H, dk), dk=nan(B, T, H, dk), dv=nan(B, T, H, dv),
+                 dg=nan(B, T, H, dk), dbeta=nan(B, T, H))
+    if want_dinit:
+        grads["d_init"] = nan(B, H, dk, dv)
+    ws = torch.empty(kda.kda_recurrent_bwd_workspace_size(B, T, H, dk, dv), dtype=torch.uint8,
+                     device=DEV)
+    kda.kda_recurrent_bwd(q, inp["k"], v, g, inp["beta"], cot["dout"], grads, ws,
+                          init_state=inp["init_state"] if with_init else None,
+                          d_final=cot["d_final"] if with_dfinal else None, scale=scale)
+    torch.cuda.synchronize()
+    return {n: to64(t) for n, t in grads.items()}
+
+
+def oracle_backward(oracle, inp, cot, scale, with_init, with_dfinal):
+    """The oracle's own gate, then its backward, on the same inputs."""
+    g = oracle.gate(to64(inp["z"]), to64(inp["A_log"]), -5.0)
+    return oracle.backward(to64(inp["q"]), to64(inp["k"]), to64(inp["v"]), g,
+                           to64(inp["beta"]), to64(cot["dout"]),
+                           init_state=to64(inp["init_state"]) if with_init else None,
+                           d_final=to64(cot["d_final"]) if with_dfinal else None, scale=scale)
+
+
+def unit_inputs(inp, cot, b, h):
+    """The inputs of one (b, h) unit as a B = 1, H = 1 problem (units are
+    independent)."""
+    tok = lambda t: t[b:b + 1, :, h:h + 1].contiguous()
+    st = lambda t: t[b:b + 1, h:h + 1].contiguous()
+    u = {n: tok(inp[n]) for n in ("q", "k", "v", "z", "beta")}
+    u["A_log"] = inp["A_log"][h:h + 1].contiguous()
+    u["init_state"] = st(inp["init_state"])
+    return u, dict(dout=tok(cot["dout"]), d_final=st(cot["d_final"]))
+
+
+CASES = [
+    # B, T, H, dk, dv, dtype, init, d_final, scale
+    (2, 150, 3, 128, 128, torch.float32, True, True, 0.7),   # 3 blocks of 64, ragged 22
+    (1, 64, 2, 128, 128, torch.bfloat16, False, False, 1.0),  # exactly one block
+    (2, 97, 2, 64, 32, torch.bfloat16, True, True, 0.5),
+    (1, 200, 2, 32, 128, torch.float32, False, True, 1.0),
+    (1, 130, 2, 128, 64, torch.bfloat16, True, False, 0.125),
+    (3, 1, 2, 32, 32, torch.float32, True, True, 1.0),       # one token
+    (1, 129, 1, 64, 64, torch.float32, True, True, 1.0),     # one token past two blocks
+]
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,dtype,init,dfin,scale", CASES)
+def test_backward_parity(oracle_mod, B, T, H, dk, dv, dtype, init, dfin, scale):
+    inp = W.make_prefill_inputs(B, T, H, dk, dv, dtype, seed=T + dk, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, dv, dk=dk, dtype=dtype, seed=T + 1, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    got = gpu_backward(inp, cot, g, scale, init, dfin)
+    ref = oracle_backward(oracle_mod, inp, cot, scale, init, dfin)
+    for n in NAMES:
+        assert np.isfinite(got[n]).all(), n
+        assert rel_l2(got[n], ref[n]) <= TOL_F32, (n, rel_l2(got[n], ref[n]))
+    assert rel_l2(got["d_init"], ref["dS0"]) <= TOL_F32
+
+
+def test_backward_empty_sequence_passes_d_final_through():
+    B, H, dk, dv = 2, 3, 64, 128
+    inp = W.make_prefill_inputs(B, 0, H, dk, dv, torch.bfloat16, seed=3, device=DEV)
+    cot = W.make_backward_cotangents(B, 0, H, dv, dk=dk, seed=4, device=DEV)
+    g = torch.empty((B, 0, H, dk), device=DEV)
+    got = gpu_backward(inp, cot, g, 1.0, False, True)
+    assert np.array_equal(got["d_init"], to64(cot["d_final"]))
+    got = gpu_backward(inp, cot, g, 1.0, False, False)
+    assert (got["d_init"] == 0).all()
+
+
+def test_backward_without_d_init_leaves_other_grads_unchanged(oracle_mod):
+    B, T, H, dk, dv = 1, 70, 2, 64, 64
+    inp = W.make_prefill_inputs(B, T, H, dk, dv, torch.float32, seed=21, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, dv, dk=dk, dtype=torch.float32, seed=22,
+                                     device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    a = gpu_backward(inp, cot, g, 1.0, True, True, want_dinit=False)
+    b = gpu_backward(inp, cot, g, 1.0, True, True, want_dinit=True)
+    for n in NAMES:
+        assert np.array_equal(a[n], b[n]), n
+
+
+def test_backward_fullsize_sampled(oracle_mod):
+    """The prefill workload's shape (B 8, H 32, T 4096, d 128, bf16 inputs):
+    every gradient finite (so written: the buffers start as NaN), and three
+    (b, h) units against the oracle element by element."""
+    B, T, H, d = 8, 4096, 32, 128
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=1, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, d, dk=d, seed=2, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    nan = lambda *s: torch.full(s, float("nan"), device=DEV)
+    grads = dict(dq=nan(B, T, H, d), dk=nan(B, T, H, d), dv=nan(B, T, H, d),
+                 dg=nan(B, T, H, d), dbeta=nan(B, T, H), d_init=nan(B, H, d, d))
+    ws = torch.empty(kda.kda_recurrent_bwd_workspace_size(B, T, H, d, d), dtype=torch.uint8,
+                     device=DEV)
+    kda.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], cot["dout"], grads, ws,
+                          init_state=inp["init_state"], d_final=cot["d_final"])
+    torch.cuda.synchronize()
+    for n, t in grads.items():
+        assert bool(torch.isfinite(t).all()), n
+    for b, h in [(0, 0), (B - 1, H - 1), (3, 17)]:
+        ui, uc = unit_inputs(inp, cot, b, h)
+        ref = oracle_backward(oracle_mod, ui, uc, 1.0, True, True)
+        for n in NAMES:
+            got = to64(grads[n][b, :, h])
+            assert rel_l2(got, ref[n][0, :, 0]) <= TOL_F32, (b, h, n)
+        assert rel_l2(to64(grads["d_init"][b, h]), ref["dS0"][0, 0]) <= TOL_F32
