@@ -48,6 +48,8 @@ WORKLOADS = {
                    dk=128, dv=128, seed=3, init=True, varlen=True, num_seqs=64),
     "decode": dict(name="decode N256 H32 d128 x1024 steps", N=256, H=32, dk=128, dv=128,
                    steps=1024, seed=4),
+    "backward": dict(name="backward B8 H32 T4096 d128", B=8, T=4096, H=32, dk=128, dv=128,
+                     seed=3, varlen=False),
 }
 
 # bytes per (token, head) of the chunkwise forward, bf16 q/k/v/o, fp32 g/beta:
@@ -275,9 +277,50 @@ def time_steps(step, K, Wm, world):
     return max_over_ranks(total_ms, world), chunk_ms
 
 
+def e2e_prefill_host_entry(inp, K):
+    """Dense batches: one kda_chunk_fwd_gated_host call per step on page-locked
+    host buffers (the library streams the batch through the device in time
+    slices, copies in both directions overlapping the kernels).  The timed
+    region holds every step's host-to-device copies of q, k, v, z, beta (and
+    A_log, init_state) and the device-to-host copies of o and the final state."""
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    q = host["q"]
+    B, T, H, dk = q.shape
+    dv = host["v"].shape[-1]
+    out_h = torch.empty((B, T, H, dv), dtype=q.dtype).pin_memory()
+    fin_h = torch.empty((B, H, dk, dv), dtype=torch.float32).pin_memory()
+    dt = kda.KDA_BF16 if q.dtype == torch.bfloat16 else kda.KDA_F32
+    ws = torch.empty(kda.kda_chunk_fwd_gated_host_workspace_size(B, T, H, dk, dv, dt),
+                     dtype=torch.uint8, device=inp["q"].device)
+    cs, xs = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * 4
+
+    def one():
+        kda.kda_chunk_fwd_gated_host(host["q"], host["k"], host["v"], host["z"], host["A_log"],
+                                     host["beta"], out_h, ws, init_state=host["init_state"],
+                                     final_state=fin_h, stream=cs, copy_stream=xs)
+
+    one()
+    cs.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(cs)
+    for _ in range(K):
+        one()
+    b.record(cs)
+    b.synchronize()
+    st, _ = kda.kda_get_device_status(ws, stream=cs)
+    if st != kda.KDA_OK:
+        raise RuntimeError(f"device status {kda.kda_status_string(st)}")
+    return a.elapsed_time(b) / K, h2d, d2h
+
+
 def e2e_prefill(wl, inp, cu, N, K):
     """Same step through the public API with host buffers: H2D of the step's
     inputs from pinned memory, gate + chunk_fwd, D2H of o and final state."""
+    if cu is None:
+        return e2e_prefill_host_entry(inp, K)
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
     dev = {k: (torch.empty_like(v) if v is not None else None) for k, v in inp.items()}
     step = PrefillStep(dev, cu, N)
@@ -381,6 +424,30 @@ def run_spec_decode(device, N=256, H=32, d=128, K=4, reps=50, seed=7):
 # v, dout: those four read (4 x 256 B), g fp32 read (512 B), beta (4 B), and
 # dq, dk, dg, dv fp32 written (4 x 512 B), dbeta (4 B).
 BWD_BYTES_PER_TOKEN_HEAD = 4 * 256 + 512 + 4 + 4 * 512 + 4
+
+
+def oracle_backward_sample(T=4096, d=128, budget_s=8.0, seed=3):
+    """The oracle's backward on whole (sequence, head) units of the backward
+    workload's shape, one after another until the budget is spent; returns
+    Mtokens/s counted like the GPU line (a position with all 32 heads is one
+    token), the cores used and a description of the sample."""
+    import oracle
+    inp = W.make_prefill_inputs(1, T, 1, d, d, torch.bfloat16, seed=seed, init_state=True)
+    cot = W.make_backward_cotangents(1, T, 1, d, dk=d, seed=seed + 1)
+    f = lambda t: t.to(torch.float64).numpy()
+    g = oracle.gate(f(inp["z"]), f(inp["A_log"]), -5.0)
+    t0 = time.perf_counter()
+    units = 0
+    while True:
+        oracle.backward(f(inp["q"]), f(inp["k"]), f(inp["v"]), g, f(inp["beta"]),
+                        f(cot["dout"]), init_state=f(inp["init_state"]),
+                        d_final=f(cot["d_final"]))
+        units += 1
+        secs = time.perf_counter() - t0
+        if secs >= budget_s:
+            break
+    value = units * T / 32 / secs / 1e6
+    return value, 1, f"{units} (sequence, head) units x {T} tokens, one thread", secs
 
 
 def run_backward(device, B=8, H=32, T=4096, d=128, reps=3, seed=3):
@@ -532,6 +599,8 @@ def main():
 
     if args.workload == "decode":
         line = bench_decode_line(args, wl, world, rank, peaks)
+    elif args.workload == "backward":
+        line = bench_backward_line(args, wl, world, rank, peaks)
     else:
         line = bench_prefill_line(args, wl, world, rank, peaks)
     if rank == 0:
@@ -658,10 +727,49 @@ def bench_decode_line(args, wl, world, rank, peaks):
     return line
 
 
+def bench_backward_line(args, wl, world, rank, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, T, H, d = wl["B"], wl["T"], wl["H"], wl["dk"]
+    clocks = None if args.no_clocks else ClockSampler(dev.index)
+    barrier(world)
+    ms, alg, ntok = run_backward(dev, B=B, H=H, T=T, d=d, reps=args.steps)
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(ms, world)
+    ach = alg / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(ntok * world / (ms * 1e-3) / 1e6, 4),
+        "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps, "warmup": 3,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T,
+                   "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs and workspace larger than L2",
+                   "step": "kda_recurrent_bwd (bf16 q/k/v/dout, fp32 gradients)"},
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4), "traffic": None,
+                     "kernel": "bwd_kernel (kda_recurrent_bwd)", "kernel_ms": round(ms, 3),
+                     "algorithmic_bytes": alg},
+        "gpu_launches": args.steps, "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, secs = oracle_backward_sample(T=T, d=d)
+        line["cpu_baseline"] = {"value": round(v, 6), "unit": "Mtokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample + f", {secs:.1f} s"}
+    return line
+
+
 def run_reference(args, wl, world):
     """The fp64 oracle as the reference arm, on this arm's config/metric."""
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    if args.workload == "decode":
+    if args.workload == "backward":
+        vals = []
+        for _ in range(args.steps):
+            v, cores, sample, secs = oracle_backward_sample(T=wl["T"], d=wl["dk"], budget_s=5.0)
+            vals.append(v)
+        value = statistics.mean(vals)
+        unit = "Mtokens/s"
+        cfg = {"workload": wl["name"], "global_batch": wl["B"], "seq_len": wl["T"]}
+    elif args.workload == "decode":
         t_per = []
         for _ in range(args.steps):
             v, cores, sample, secs = oracle_decode_sample(wl, budget_s=5.0)

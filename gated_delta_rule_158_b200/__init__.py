@@ -7,7 +7,8 @@ Build the library with ``python -m gated_delta_rule_158_b200.build``.
 from ._lib import (  # noqa: F401
     KDA_BF16, KDA_ERR_BAD_SEQLENS, KDA_ERR_CUDA, KDA_ERR_INVALID_ARG, KDA_ERR_MISALIGNED,
     KDA_ERR_TIMEOUT, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_F32, KDA_OK, KdaError,
-    kda_chunk_fwd, kda_chunk_fwd_gated, kda_chunk_fwd_noalloc, kda_chunk_fwd_workspace_size,
+    kda_chunk_fwd, kda_chunk_fwd_gated, kda_chunk_fwd_gated_host,
+    kda_chunk_fwd_gated_host_workspace_size, kda_chunk_fwd_noalloc, kda_chunk_fwd_workspace_size,
     kda_chunk_segment_transition, kda_chunk_state_prefix, kda_decode_step,
     kda_decode_replay, kda_decode_step_gated, kda_decode_verify, kda_gate_fwd,
     kda_get_device_status, kda_last_cuda_error_string, kda_recurrent_bwd,

@@ -52,6 +52,9 @@ _SIGNATURES = {
                                _VP, _VP]),
     "kda_decode_replay": (_I, [_VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I,
                                _VP]),
+    "kda_chunk_fwd_gated_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "kda_chunk_fwd_gated_host": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _I, _I, _I, _I,
+                                      _I, _F, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "kda_recurrent_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "kda_recurrent_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F,
                                _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -242,6 +245,30 @@ def kda_decode_replay(k, v, g, beta, state, accept_len, A_log=None, g_min=-5.0, 
     _check(lib().kda_decode_replay(_ptr(k), _ptr(v), _ptr(g), _ptr(A_log), float(g_min),
                                    _ptr(beta), _dtype(k), _ptr(state), _ptr(accept_len), N, H, K,
                                    dk, dv, _stream(stream)), "kda_decode_replay")
+
+
+def kda_chunk_fwd_gated_host_workspace_size(B, T, H, dk, dv, in_dtype=KDA_BF16) -> int:
+    return int(lib().kda_chunk_fwd_gated_host_workspace_size(B, T, H, dk, dv, in_dtype))
+
+
+def kda_chunk_fwd_gated_host(q, k, v, z, A_log, beta, out, workspace, g_min=-5.0,
+                             init_state=None, final_state=None, scale=1.0, stream=None,
+                             copy_stream=None):
+    """Gated chunked prefill of a dense batch in host memory (CPU tensors,
+    page-locked for overlap): q, k [B,T,H,dk], v [B,T,H,dv], z [B,T,H,dk]
+    fp32, A_log [H], beta [B,T,H]; out [B,T,H,dv] and final_state
+    [B,H,dk,dv] are host tensors written by the time `stream` reaches the end
+    of the call's work.  workspace is a device uint8 tensor."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t in (q, k, v, z, A_log, beta, out, init_state, final_state):
+        if t is not None and t.is_cuda:
+            raise ValueError("kda_chunk_fwd_gated_host takes host tensors")
+    _check(lib().kda_chunk_fwd_gated_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta), _dtype(q),
+        _ptr(init_state), B, T, H, dk, dv, float(scale), _ptr(out), _ptr(final_state),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+        None if copy_stream is None else _stream(copy_stream)), "kda_chunk_fwd_gated_host")
 
 
 def kda_recurrent_bwd_workspace_size(B, T, H, dk, dv) -> int:

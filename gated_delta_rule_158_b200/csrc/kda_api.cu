@@ -7,6 +7,7 @@
 
 #include "kda_internal.cuh"
 #include "kda_bwd.cuh"
+#include "kda_host.cuh"
 #include "kda_sync.cuh"
 
 namespace kda {
@@ -146,16 +147,18 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
 
 }  // extern "C"
 
-namespace {
+namespace kda {
 
 // Shared body of kda_chunk_fwd and kda_chunk_fwd_gated: g is the log-decay,
-// or z when A_log is not null.
+// or z when A_log is not null.  reset_status = false keeps the device status
+// word as it is (a caller running several slices on one workspace).
 kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
                           const float* A_log, float g_min, const float* beta,
                           kda_dtype in_dtype, const float* init_state,
                           const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
                           int dv, float scale, int chunk_size, void* out, float* final_state,
-                          void* workspace, size_t workspace_bytes, void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          bool reset_status) {
   if (!q || !k || !v || !g || !beta || !out || !workspace) return KDA_ERR_INVALID_ARG;
   if (A_log && (!(g_min < 0.f) || !isfinite(g_min))) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -186,7 +189,8 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   cudaStream_t st = (cudaStream_t)stream;
   StatusBlock* sb = static_cast<StatusBlock*>(workspace);
   char* tail = static_cast<char*>(workspace) + kStatusBytes;
-  if (cudaError_t em = cudaMemsetAsync(sb, 0, kStatusBytes, st)) return cuda_failure(em);
+  if (reset_status)
+    if (cudaError_t em = cudaMemsetAsync(sb, 0, kStatusBytes, st)) return cuda_failure(em);
 
   ChunkArgs a{};
   a.q = q;
@@ -232,7 +236,7 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
-}  // namespace
+}  // namespace kda
 
 extern "C" {
 

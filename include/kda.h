@@ -185,6 +185,44 @@ KDA_API kda_status kda_chunk_fwd_gated(const void *q, const void *k, const void 
                                size_t workspace_bytes, void *stream);
 
 /*
+ * kda_chunk_fwd_gated (the chunkwise prefill of Infrastructure > KDA kernels,
+ * same page) for a dense batch held in HOST memory: the same
+ * result as copying q, k, v, z, beta (and init_state) to the device, calling
+ * kda_chunk_fwd_gated and copying o and the final state back, but the batch
+ * goes through the device in time slices of about T/8 tokens (>= 512), so
+ * the host-to-device copies of one slice, the kernels of the previous one
+ * and the device-to-host copy of the one before overlap.  The state passes
+ * from slice to slice on the device.
+ *  q, k, v, z, beta, A_log, init_state : HOST pointers, layouts and dtypes as
+ *      kda_chunk_fwd_gated (init_state may be NULL: zeros).  Page-locked
+ *      memory lets the copies run asynchronously; pageable memory works but
+ *      serialises them.
+ *  out : HOST [B, T, H, dv] in_dtype;  final_state : HOST fp32 [B, H, dk, dv]
+ *      or NULL.  Written when `stream` reaches the end of this call's work;
+ *      host buffers must stay valid until then.
+ *  workspace : DEVICE, 256-byte aligned, at least
+ *      kda_chunk_fwd_gated_host_workspace_size(...) bytes (two slices of
+ *      inputs and outputs, two states, the chunk workspace; its first 256
+ *      bytes are the device status word of every slice, for
+ *      kda_get_device_status).
+ *  stream : kernels and device-to-host copies; copy_stream : host-to-device
+ *      copies (NULL = `stream`, no overlap).  The copies into the workspace
+ *      wait for work already queued on `stream`.
+ * Dense batches only (no cu_seqlens).  Supported shapes as
+ * kda_chunk_fwd_gated.
+ */
+KDA_API size_t kda_chunk_fwd_gated_host_workspace_size(int B, int T, int H, int dk, int dv,
+                                                       kda_dtype in_dtype);
+
+KDA_API kda_status kda_chunk_fwd_gated_host(const void *q, const void *k, const void *v,
+                                    const float *z, const float *A_log, float g_min,
+                                    const float *beta, kda_dtype in_dtype,
+                                    const float *init_state, int B, int T, int H, int dk,
+                                    int dv, float scale, void *out, float *final_state,
+                                    void *workspace, size_t workspace_bytes, void *stream,
+                                    void *copy_stream);
+
+/*
  * One single-token decode step for N sequences, updating the state in place
  * (KDA decoding: same page, Online serving > high-performance kernels; the
  * state is rewritten in place every token).  Per (n, h):

@@ -218,3 +218,29 @@ def test_backward_entries_reject_on_host(L):
     assert L.kda_recurrent_bwd(*args(T=0, q=None, k=None, v=None, g=None, beta=None, dout=None,
                                      dq=None, dko=None, dvo=None, dg=None, dbeta=None,
                                      wsb=ws0)) == kda.KDA_OK
+
+
+def test_host_stream_entry_rejects_on_host(L):
+    ptr = lambda i: FAKE + 0x1000 * i
+    n = L.kda_chunk_fwd_gated_host_workspace_size(2, 4096, 4, 128, 128, kda.KDA_BF16)
+    assert n > 0
+    assert L.kda_chunk_fwd_gated_host_workspace_size(4, 4096, 4, 128, 128, kda.KDA_BF16) > n
+    assert L.kda_chunk_fwd_gated_host_workspace_size(2, 4096, 4, 96, 128, kda.KDA_BF16) == 0
+    assert L.kda_chunk_fwd_gated_host_workspace_size(2, 0, 4, 128, 128, kda.KDA_BF16) == 0
+
+    def args(**over):
+        a = dict(q=ptr(0), k=ptr(1), v=ptr(2), z=ptr(3), A_log=ptr(4), g_min=-5.0, beta=ptr(5),
+                 dt=kda.KDA_BF16, init=None, B=2, T=4096, H=4, dk=128, dv=128, scale=1.0,
+                 out=ptr(6), final=None, ws=ptr(16), wsb=n, stream=None, copy=None)
+        a.update(over)
+        return list(a.values())
+
+    assert L.kda_chunk_fwd_gated_host(*args(out=None)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_fwd_gated_host(*args(A_log=None)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_fwd_gated_host(*args(g_min=0.5)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_fwd_gated_host(*args(dt=9)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_fwd_gated_host(*args(T=0)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_chunk_fwd_gated_host(*args(dv=48)) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_fwd_gated_host(*args(ws=ptr(16) + 16)) == kda.KDA_ERR_MISALIGNED
+    assert L.kda_chunk_fwd_gated_host(*args(wsb=n - 1)) == kda.KDA_ERR_WORKSPACE
+    assert L.kda_chunk_fwd_gated_host(*args(out=ptr(2))) == kda.KDA_ERR_INVALID_ARG  # aliases v
