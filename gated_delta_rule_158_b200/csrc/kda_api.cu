@@ -420,7 +420,7 @@ kda_status kda_decode_replay(const void* k, const void* v, const float* g, const
 
 size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
   if (B <= 0 || T < 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
-  return bwd_workspace_bytes(B, T, H, dk, dv);
+  return bwd_chunk_workspace_bytes(B, T, H, dk, dv);
 }
 
 kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
@@ -437,8 +437,8 @@ kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const 
   if ((int64_t)B * H > 0x7fffffffLL || (int64_t)B * T * H > 0x7fffffffLL)
     return KDA_ERR_UNSUPPORTED;
   if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-  if (!workspace || workspace_bytes < bwd_workspace_bytes(B, T, H, dk, dv))
-    return KDA_ERR_WORKSPACE;
+  const size_t need = bwd_chunk_workspace_bytes(B, T, H, dk, dv);  // 0 when T = 0
+  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
   const void* ptrs[] = {q, k, v, g, beta, init_state, dout, d_final, dq, dk_out, dv_out, dg,
                         dbeta, d_init, workspace};
   for (const void* p : ptrs)
@@ -454,7 +454,7 @@ kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const 
   BwdArgs a{q,  k,  v,     g,     beta,   init_state, dout,   d_final, in_dtype, B,
             T,  H,  dk,    dv,    scale,  dq,         dk_out, dv_out,  dg,       dbeta,
             d_init, static_cast<float*>(workspace)};
-  const cudaError_t e = launch_bwd(a, (cudaStream_t)stream);
+  const cudaError_t e = launch_bwd_chunk(a, (cudaStream_t)stream);
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 

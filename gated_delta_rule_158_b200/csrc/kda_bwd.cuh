@@ -5,8 +5,8 @@
 
 namespace kda {
 
-// Backward through the recurrence (token by token, fp32): per (sequence,
-// head) the gradients of q, k, v, g, beta and the initial state.
+// Backward through the recurrence (fp32): per (sequence, head) the gradients
+// of q, k, v, g, beta and the initial state.
 struct BwdArgs {
   const void* q;
   const void* k;
@@ -25,10 +25,13 @@ struct BwdArgs {
   float* dg;
   float* dbeta;
   float* dinit;  // nullable
-  float* ws;     // bwd_workspace_bytes(B, T, H, dk, dv), 16-byte aligned
+  float* ws;     // bwd_chunk_workspace_bytes(B, T, H, dk, dv), 16-byte aligned
 };
 
-size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+// In chunk form (kda_bwd_chunk.cu): a forward pass saving chunk-start states,
+// a reverse pass of the state gradient, then every chunk's token gradients in
+// parallel.
+size_t bwd_chunk_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace kda

@@ -1,0 +1,724 @@
+// kda_bwd_chunk.cu -- gradients through the KDA recurrence in chunk form.
+//
+// The recurrence ("NLP--技术报告解读-Kimi-K3", joezjh.github.io, Model
+// Architecture > Kimi Delta Attention (KDA)) evaluated chunk by chunk as in
+// the forward kernels (Infrastructure > KDA kernels: FlashKDA serves training
+// and prefill), differentiated.  Per (sequence, head), chunks of C = 32
+// tokens, Gamma the in-chunk cumulative log-decay, E_rsi = e^{Gamma_ri -
+// Gamma_si} (s <= r, never above 1 for g <= 0):
+//   L = strict_lower(sum_i k_ri k_si E_rsi),  A_qk = lower(sum_i q_ri k_si E_rsi)
+//   X = (I + Diag(beta) L)^-1,  T = X Diag(beta)
+//   Qg = q e^Gamma,  Ka = k e^Gamma,  Kc = k e^{Gamma_C - Gamma}
+//   U = T (V - Ka S),  S_next = Diag(e^{Gamma_C}) S + Kc^T U,  O = scale (Qg S + A_qk U)
+// Three passes, fp32 throughout:
+//   F  chunk order, one CTA per (unit, 32 dv columns): the key-side matrices
+//      (saved once per chunk: X, A_qk, L) and the chunk-start states.
+//   A  reverse chunk order, same grid: the state gradient dS = dL/dS_next,
+//        dU = A_qk^T dO' + Kc dS,  dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T T^T dU
+//      (dO' = scale dO); needs no state.  Saves dS of every chunk.
+//   B  one CTA per (unit, chunk), all chunks at once: with U, R = V - Ka S,
+//      dU and W = T^T dU (= dv) recomputed per 32 dv columns,
+//        dQg = dO' S^T, dKa = -W S^T, dKc = U dS^T,
+//        dA_qk = lower(dO' U^T), dT = dU R^T,
+//      then through T, X, L and A_qk (their entries' gradients back onto q, k
+//      and Gamma through E) and the decays, and a reverse cumulative sum of
+//      dGamma gives dg.
+// Tail chunks are padded with g = 0, beta = 0, k = q = v = dO = 0.
+#include "kda_bwd.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int C = 32;
+constexpr int NTH = 256;
+constexpr int VB = 32;         // dv columns per block
+constexpr int LDC = C + 1;     // C x C tiles
+constexpr int LDB = VB + 1;    // x 32-column tiles
+static_assert(NTH == 8 * 32, "forward substitution: 8 warps x 4 columns");
+
+// acc[i][j] += sum_k a(m_i, k) b(k, n_j) over a 256-thread tile of an M x N
+// product: thread (tm, tn) owns rows tm + i M/TM and columns tn + j N/TN.
+template <int M, int N, int TM, int TN, int K, typename FA, typename FB>
+__device__ __forceinline__ void mm(float (&acc)[TM][TN], FA a, FB b) {
+  static_assert((M / TM) * (N / TN) == NTH, "one output tile per thread");
+  constexpr int NTN = N / TN, MS = M / TM;
+  const int tn = threadIdx.x % NTN, tm = threadIdx.x / NTN;
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float av[TM], bv[TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i) av[i] = a(tm + i * MS, k);
+#pragma unroll
+    for (int j = 0; j < TN; ++j) bv[j] = b(k, tn + j * NTN);
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
+template <int M, int N, int TM, int TN, typename F>
+__device__ __forceinline__ void for_tile(F f) {  // f(m, n, i, j) over this thread's tile
+  constexpr int NTN = N / TN, MS = M / TM;
+  const int tn = threadIdx.x % NTN, tm = threadIdx.x / NTN;
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) f(tm + i * MS, tn + j * NTN, i, j);
+}
+
+template <int TM, int TN>
+__device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+}
+
+// per-unit workspace: S_c [nc][DK][DV], dS_c [nc][DK][DV], X, A_qk, L [nc][C][C]
+struct UnitWs {
+  float* S;
+  float* dS;
+  float* X;
+  float* Aqk;
+  float* L;
+};
+
+__host__ __device__ inline size_t unit_ws_floats(int nc, int DK, int DV) {
+  return (size_t)nc * (2 * (size_t)DK * DV + 3 * C * C);
+}
+
+__device__ inline UnitWs unit_ws(float* ws, int unit, int nc, int DK, int DV) {
+  UnitWs w;
+  float* base = ws + (size_t)unit * unit_ws_floats(nc, DK, DV);
+  w.S = base;
+  w.dS = w.S + (size_t)nc * DK * DV;
+  w.X = w.dS + (size_t)nc * DK * DV;
+  w.Aqk = w.X + (size_t)nc * C * C;
+  w.L = w.Aqk + (size_t)nc * C * C;
+  return w;
+}
+
+// chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to C
+template <typename Tin, int DK>
+__device__ void load_keys(const Tin* q, const Tin* k, const float* g, const float* beta,
+                          size_t rowbase, int H, int n, float* qS, float* kS, float* GS,
+                          float* bS) {
+  constexpr int LDK = DK + 1;
+  for (int idx = threadIdx.x; idx < C * DK; idx += NTH) {
+    const int r = idx / DK, i = idx % DK;
+    float qv = 0.f, kv = 0.f, gv = 0.f;
+    if (r < n) {
+      const size_t off = (rowbase + (size_t)r * H) * DK + i;
+      qv = Elem<Tin>::load(q + off);
+      kv = Elem<Tin>::load(k + off);
+      gv = g[off];
+    }
+    qS[r * LDK + i] = qv;
+    kS[r * LDK + i] = kv;
+    GS[r * LDK + i] = gv;
+  }
+  for (int r = threadIdx.x; r < C; r += NTH) bS[r] = r < n ? beta[rowbase + (size_t)r * H] : 0.f;
+  __syncthreads();
+  for (int i = threadIdx.x; i < DK; i += NTH) {  // Gamma = inclusive cumsum over the chunk
+    float acc = 0.f;
+    for (int r = 0; r < C; ++r) {
+      acc += GS[r * LDK + i];
+      GS[r * LDK + i] = acc;
+    }
+  }
+  __syncthreads();
+}
+
+// [C x 32] block of a [*, DV] token tensor (columns j0 .. j0+31), times mul
+template <typename Tin>
+__device__ void load_vblock(const Tin* x, size_t rowbase, int H, int DV, int j0, int n,
+                            float mul, float* dst) {
+  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
+    const int r = idx / VB, j = idx % VB;
+    dst[r * LDB + j] =
+        r < n ? mul * Elem<Tin>::load(x + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+  }
+}
+
+// ===================================================================== pass F
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(NTH, 2)
+    bwd_fwd_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                 const Tin* __restrict__ v, const float* __restrict__ g,
+                 const float* __restrict__ beta, const float* __restrict__ init, int T, int H,
+                 int DV, float* __restrict__ ws) {
+  constexpr int LDK = DK + 1;
+  extern __shared__ float sm[];
+  float* qS = sm;                 // [C][LDK]
+  float* kS = qS + C * LDK;       // [C][LDK]  k, later Kc
+  float* GS = kS + C * LDK;       // [C][LDK]  Gamma, later Ka
+  float* SS = GS + C * LDK;       // [DK][LDB] state block
+  float* VS = SS + DK * LDB;      // [C][LDB]  V, then V - P
+  float* US = VS + C * LDB;       // [C][LDB]
+  float* LS = US + C * LDB;       // [C][LDC]
+  float* AqS = LS + C * LDC;      // [C][LDC]
+  float* XS = AqS + C * LDC;      // [C][LDC]  X, then T
+  float* bS = XS + C * LDC;       // [C]
+  float* gC = bS + C;             // [DK]
+
+  const int nblk = DV / VB;
+  const int unit = blockIdx.x / nblk, j0 = (blockIdx.x % nblk) * VB;
+  const int b = unit / H, h = unit % H;
+  const int nc = (T + C - 1) / C;
+  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  const int tid = threadIdx.x;
+
+  for (int idx = tid; idx < DK * VB; idx += NTH) {
+    const int i = idx / VB, j = idx % VB;
+    SS[i * LDB + j] = init ? init[((size_t)unit * DK + i) * DV + j0 + j] : 0.f;
+  }
+  for (int c = 0; c < nc; ++c) {
+    const int t0 = c * C, n = min(C, T - t0);
+    const size_t rowbase = ((size_t)b * T + t0) * H + h;
+    __syncthreads();
+    load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+    load_vblock<Tin>(v, rowbase, H, DV, j0, n, 1.f, VS);
+    // chunk-start state block
+    for (int idx = tid; idx < DK * VB; idx += NTH) {
+      const int i = idx / VB, j = idx % VB;
+      w.S[((size_t)c * DK + i) * DV + j0 + j] = SS[i * LDB + j];
+    }
+    // Gram matrices, exponents as differences (s <= r)
+    for (int p = tid; p < C * (C + 1) / 2; p += NTH) {
+      int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+      while ((r + 1) * (r + 2) / 2 <= p) ++r;
+      while (r * (r + 1) / 2 > p) --r;
+      const int s = p - r * (r + 1) / 2;
+      float lk = 0.f, lq = 0.f;
+#pragma unroll 4
+      for (int i = 0; i < DK; ++i) {
+        const float e = expf(GS[r * LDK + i] - GS[s * LDK + i]);
+        const float ks = kS[s * LDK + i] * e;
+        lk = fmaf(kS[r * LDK + i], ks, lk);
+        lq = fmaf(qS[r * LDK + i], ks, lq);
+      }
+      LS[r * LDC + s] = s < r ? lk : 0.f;
+      AqS[r * LDC + s] = lq;
+    }
+    for (int idx = tid; idx < C * C; idx += NTH) {
+      const int r = idx / C, s = idx % C;
+      if (s > r) {
+        LS[r * LDC + s] = 0.f;
+        AqS[r * LDC + s] = 0.f;
+      }
+    }
+    __syncthreads();
+    // X = (I + Diag(beta) L)^-1 by forward substitution; the columns are
+    // independent, so warp w takes columns 4w .. 4w+3 with 8 lanes per column
+    {
+      const int lane = tid & 31, cc = 4 * (tid >> 5) + (lane >> 3), sub = lane & 7;
+      for (int r = sub; r < C; r += 8) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
+      __syncwarp();
+      for (int r = 1; r < C; ++r) {
+        float acc = 0.f;
+        for (int s = cc + sub; s < r; s += 8) acc = fmaf(LS[r * LDC + s], XS[s * LDC + cc], acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if (sub == 0 && r > cc) XS[r * LDC + cc] = -bS[r] * acc;
+        __syncwarp();
+      }
+    }
+    for (int i = tid; i < DK; i += NTH) gC[i] = GS[(C - 1) * LDK + i];
+    __syncthreads();
+    if (j0 == 0) {  // the key-side matrices, once per chunk
+      for (int idx = tid; idx < C * C; idx += NTH) {
+        const int r = idx / C, s = idx % C;
+        const size_t o = ((size_t)c * C + r) * C + s;
+        w.X[o] = XS[r * LDC + s];
+        w.Aqk[o] = AqS[r * LDC + s];
+        w.L[o] = LS[r * LDC + s];
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * C; idx += NTH) {  // T = X Diag(beta)
+      const int r = idx / C, s = idx % C;
+      XS[r * LDC + s] *= bS[s];
+    }
+    for (int idx = tid; idx < C * DK; idx += NTH) {  // Ka, Kc
+      const int r = idx / DK, i = idx % DK;
+      const float G = GS[r * LDK + i], kv = kS[r * LDK + i];
+      GS[r * LDK + i] = kv * expf(G);
+      kS[r * LDK + i] = kv * expf(gC[i] - G);
+    }
+    __syncthreads();
+    {  // V <- V - Ka S
+      float acc[2][2];
+      zero(acc);
+      mm<C, VB, 2, 2, DK>(acc, [&](int m, int kk) { return GS[m * LDK + kk]; },
+                          [&](int kk, int nn) { return SS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { VS[m * LDB + nn] -= acc[i][j]; });
+    }
+    __syncthreads();
+    {  // U = T (V - Ka S)
+      float acc[2][2];
+      zero(acc);
+      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return XS[m * LDC + kk]; },
+                         [&](int kk, int nn) { return VS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { US[m * LDB + nn] = acc[i][j]; });
+    }
+    __syncthreads();
+    {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
+      constexpr int TM = DK / 32;
+      float acc[TM][4];
+      zero(acc);
+      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
+                           [&](int kk, int nn) { return US[kk * LDB + nn]; });
+      for_tile<DK, VB, TM, 4>([&](int m, int nn, int i, int j) {
+        SS[m * LDB + nn] = fmaf(expf(gC[m]), SS[m * LDB + nn], acc[i][j]);
+      });
+    }
+  }
+}
+
+// ===================================================================== pass A
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(NTH, 2)
+    bwd_state_grad_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                        const float* __restrict__ g, const float* __restrict__ beta,
+                        const Tin* __restrict__ dout, const float* __restrict__ dfinal, int T,
+                        int H, int DV, float scale, float* __restrict__ dinit,
+                        float* __restrict__ ws) {
+  constexpr int LDK = DK + 1;
+  extern __shared__ float sm[];
+  float* qS = sm;                 // [C][LDK]  q, later Qg
+  float* kS = qS + C * LDK;       // [C][LDK]  k, later Kc
+  float* GS = kS + C * LDK;       // [C][LDK]  Gamma, later Ka
+  float* dSS = GS + C * LDK;      // [DK][LDB] state-gradient block
+  float* dOS = dSS + DK * LDB;    // [C][LDB]  scale dO
+  float* dUS = dOS + C * LDB;     // [C][LDB]
+  float* WS = dUS + C * LDB;      // [C][LDB]
+  float* AqS = WS + C * LDB;      // [C][LDC]
+  float* TS = AqS + C * LDC;      // [C][LDC]
+  float* bS = TS + C * LDC;       // [C]
+  float* gC = bS + C;             // [DK]
+
+  const int nblk = DV / VB;
+  const int unit = blockIdx.x / nblk, j0 = (blockIdx.x % nblk) * VB;
+  const int b = unit / H, h = unit % H;
+  const int nc = (T + C - 1) / C;
+  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  const int tid = threadIdx.x;
+
+  for (int idx = tid; idx < DK * VB; idx += NTH) {
+    const int i = idx / VB, j = idx % VB;
+    dSS[i * LDB + j] = dfinal ? dfinal[((size_t)unit * DK + i) * DV + j0 + j] : 0.f;
+  }
+  for (int c = nc - 1; c >= 0; --c) {
+    const int t0 = c * C, n = min(C, T - t0);
+    const size_t rowbase = ((size_t)b * T + t0) * H + h;
+    __syncthreads();
+    load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+    load_vblock<Tin>(dout, rowbase, H, DV, j0, n, scale, dOS);
+    for (int idx = tid; idx < C * C; idx += NTH) {
+      const int r = idx / C, s = idx % C;
+      const size_t o = ((size_t)c * C + r) * C + s;
+      AqS[r * LDC + s] = w.Aqk[o];
+      TS[r * LDC + s] = w.X[o] * bS[s];
+    }
+    for (int idx = tid; idx < DK * VB; idx += NTH) {  // dL/dS_next of this chunk
+      const int i = idx / VB, j = idx % VB;
+      w.dS[((size_t)c * DK + i) * DV + j0 + j] = dSS[i * LDB + j];
+    }
+    for (int i = tid; i < DK; i += NTH) gC[i] = GS[(C - 1) * LDK + i];
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += NTH) {  // Qg, Ka, Kc
+      const int r = idx / DK, i = idx % DK;
+      const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LDK + i];
+      qS[r * LDK + i] *= e;
+      GS[r * LDK + i] = kv * e;
+      kS[r * LDK + i] = kv * expf(gC[i] - G);
+    }
+    __syncthreads();
+    {  // dU = A_qk^T dO' + Kc dS
+      float acc[2][2];
+      zero(acc);
+      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
+                         [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
+      mm<C, VB, 2, 2, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
+                          [&](int kk, int nn) { return dSS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { dUS[m * LDB + nn] = acc[i][j]; });
+    }
+    __syncthreads();
+    {  // W = T^T dU
+      float acc[2][2];
+      zero(acc);
+      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
+                         [&](int kk, int nn) { return dUS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { WS[m * LDB + nn] = acc[i][j]; });
+    }
+    __syncthreads();
+    {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
+      constexpr int TM = DK / 32;
+      float acc[TM][4];
+      zero(acc);
+      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
+                           [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
+      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
+                           [&](int kk, int nn) { return WS[kk * LDB + nn]; });
+      for_tile<DK, VB, TM, 4>([&](int m, int nn, int i, int j) {
+        dSS[m * LDB + nn] = fmaf(expf(gC[m]), dSS[m * LDB + nn], acc[i][j]);
+      });
+    }
+  }
+  __syncthreads();
+  if (dinit) {
+    for (int idx = tid; idx < DK * VB; idx += NTH) {
+      const int i = idx / VB, j = idx % VB;
+      dinit[((size_t)unit * DK + i) * DV + j0 + j] = dSS[i * LDB + j];
+    }
+  }
+}
+
+// ===================================================================== pass B
+template <int DK>
+struct BSmem {
+  static constexpr int LDK = DK + 1;
+  // the dv-block loop's tiles (S and dS blocks; dO', R, U, dU, W blocks) are
+  // dead once the loop ends, and the dq, dk, dGamma accumulators take their place
+  static constexpr int loop = 2 * DK * LDB + 5 * C * LDB;
+  static constexpr int accs = 3 * C * LDK;
+  static_assert(accs <= loop, "accumulators fit the loop tiles");
+  static constexpr int floats = 6 * C * LDK      // q, k, Gamma, Qg, Ka, Kc
+                                + loop
+                                + 7 * C * LDC    // X, T, A_qk, L, dA_qk, dT (then dM), scratch
+                                + C + 3 * DK;    // beta, Gamma_C, two dGamma_C terms
+  static constexpr size_t bytes = sizeof(float) * floats;
+};
+
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(NTH, 1)
+    bwd_chunk_grads(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                    const Tin* __restrict__ v, const float* __restrict__ g,
+                    const float* __restrict__ beta, const Tin* __restrict__ dout, int T, int H,
+                    int DV, float scale, float* __restrict__ dq, float* __restrict__ dk,
+                    float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
+                    float* __restrict__ ws) {
+  constexpr int LDK = DK + 1;
+  extern __shared__ float sm[];
+  float* qS = sm;
+  float* kS = qS + C * LDK;
+  float* GS = kS + C * LDK;       // Gamma
+  float* QgS = GS + C * LDK;
+  float* KaS = QgS + C * LDK;
+  float* KcS = KaS + C * LDK;
+  float* SS = KcS + C * LDK;      // [DK][LDB]   (dv-block loop)
+  float* dSS = SS + DK * LDB;     // [DK][LDB]
+  float* dOS = dSS + DK * LDB;    // [C][LDB]
+  float* RS = dOS + C * LDB;
+  float* US = RS + C * LDB;
+  float* dUS = US + C * LDB;
+  float* WS = dUS + C * LDB;
+  float* aq = SS;                 // after the loop: dq accumulator [C][LDK]
+  float* ak = aq + C * LDK;       //                 dk accumulator
+  float* aG = ak + C * LDK;       //                 dGamma accumulator
+  float* XS = WS + C * LDB;       // [C][LDC]
+  float* TS = XS + C * LDC;
+  float* AqS = TS + C * LDC;
+  float* LS = AqS + C * LDC;
+  float* dAqS = LS + C * LDC;
+  float* dTS = dAqS + C * LDC;    // dT, then dM
+  float* YS = dTS + C * LDC;      // scratch
+  float* bS = YS + C * LDC;       // [C]
+  float* gC = bS + C;             // [DK] Gamma_C
+  float* rsum = gC + DK;          // [DK] sum_j dS_ij S_ij
+  float* kcsum = rsum + DK;       // [DK] sum_r dKc_ri Kc_ri
+
+  const int nc = (T + C - 1) / C;
+  const int unit = blockIdx.x / nc, c = blockIdx.x % nc;
+  const int b = unit / H, h = unit % H;
+  const int t0 = c * C, n = min(C, T - t0);
+  const size_t rowbase = ((size_t)b * T + t0) * H + h;
+  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  const int tid = threadIdx.x;
+  constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
+
+  load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  for (int idx = tid; idx < C * C; idx += NTH) {
+    const int r = idx / C, s = idx % C;
+    const size_t o = ((size_t)c * C + r) * C + s;
+    const float x = w.X[o];
+    XS[r * LDC + s] = x;
+    TS[r * LDC + s] = x * bS[s];
+    AqS[r * LDC + s] = w.Aqk[o];
+    LS[r * LDC + s] = w.L[o];
+  }
+  for (int i = tid; i < DK; i += NTH) {
+    gC[i] = GS[(C - 1) * LDK + i];
+    rsum[i] = 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * DK; idx += NTH) {
+    const int r = idx / DK, i = idx % DK;
+    const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LDK + i];
+    QgS[r * LDK + i] = qS[r * LDK + i] * e;
+    KaS[r * LDK + i] = kv * e;
+    KcS[r * LDK + i] = kv * expf(gC[i] - G);
+  }
+
+  // products summed over the dv columns, accumulated block by block:
+  // dQg^T = S dO'^T, -dKa^T = S W^T, dKc^T = dS U^T  (DK x C); dA_qk, dT (C x C)
+  float aQ[TMK][4], aKa[TMK][4], aKc[TMK][4], aA[2][2], aT[2][2];
+  zero(aQ);
+  zero(aKa);
+  zero(aKc);
+  zero(aA);
+  zero(aT);
+  for (int j0 = 0; j0 < DV; j0 += VB) {
+    __syncthreads();
+    for (int idx = tid; idx < DK * VB; idx += NTH) {
+      const int i = idx / VB, j = idx % VB;
+      const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
+      SS[i * LDB + j] = w.S[o];
+      dSS[i * LDB + j] = w.dS[o];
+    }
+    load_vblock<Tin>(v, rowbase, H, DV, j0, n, 1.f, RS);
+    load_vblock<Tin>(dout, rowbase, H, DV, j0, n, scale, dOS);
+    __syncthreads();
+    {  // R = V - Ka S;  dU = A_qk^T dO' + Kc dS
+      float p[2][2], u[2][2];
+      zero(p);
+      zero(u);
+      mm<C, VB, 2, 2, DK>(p, [&](int m, int kk) { return KaS[m * LDK + kk]; },
+                          [&](int kk, int nn) { return SS[kk * LDB + nn]; });
+      mm<C, VB, 2, 2, C>(u, [&](int m, int kk) { return AqS[kk * LDC + m]; },
+                         [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
+      mm<C, VB, 2, 2, DK>(u, [&](int m, int kk) { return KcS[m * LDK + kk]; },
+                          [&](int kk, int nn) { return dSS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
+        RS[m * LDB + nn] -= p[i][j];
+        dUS[m * LDB + nn] = u[i][j];
+      });
+    }
+    for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
+      float acc = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < VB; ++j) acc = fmaf(dSS[i * LDB + j], SS[i * LDB + j], acc);
+      rsum[i] += acc;
+    }
+    __syncthreads();
+    {  // U = T R;  W = T^T dU  (W is dv)
+      float u[2][2], wv[2][2];
+      zero(u);
+      zero(wv);
+      mm<C, VB, 2, 2, C>(u, [&](int m, int kk) { return TS[m * LDC + kk]; },
+                         [&](int kk, int nn) { return RS[kk * LDB + nn]; });
+      mm<C, VB, 2, 2, C>(wv, [&](int m, int kk) { return TS[kk * LDC + m]; },
+                         [&](int kk, int nn) { return dUS[kk * LDB + nn]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
+        US[m * LDB + nn] = u[i][j];
+        WS[m * LDB + nn] = wv[i][j];
+        if (m < n) dv[(rowbase + (size_t)m * H) * DV + j0 + nn] = wv[i][j];
+      });
+    }
+    __syncthreads();
+    // block contributions, contracted over this block's 32 columns
+    mm<DK, C, TMK, 4, VB>(aQ, [&](int m, int kk) { return SS[m * LDB + kk]; },
+                          [&](int kk, int nn) { return dOS[nn * LDB + kk]; });
+    mm<DK, C, TMK, 4, VB>(aKa, [&](int m, int kk) { return SS[m * LDB + kk]; },
+                          [&](int kk, int nn) { return WS[nn * LDB + kk]; });
+    mm<DK, C, TMK, 4, VB>(aKc, [&](int m, int kk) { return dSS[m * LDB + kk]; },
+                          [&](int kk, int nn) { return US[nn * LDB + kk]; });
+    mm<C, C, 2, 2, VB>(aA, [&](int m, int kk) { return dOS[m * LDB + kk]; },
+                       [&](int kk, int nn) { return US[nn * LDB + kk]; });
+    mm<C, C, 2, 2, VB>(aT, [&](int m, int kk) { return dUS[m * LDB + kk]; },
+                       [&](int kk, int nn) { return RS[nn * LDB + kk]; });
+  }
+  __syncthreads();  // the loop tiles become the accumulators
+  // dq, dk, dGamma from the state-side products and the decays
+  for_tile<DK, C, TMK, 4>([&](int i, int r, int a, int bb) {
+    const float e = expf(GS[r * LDK + i]);
+    const float ec = expf(gC[i] - GS[r * LDK + i]);
+    const float dQg = aQ[a][bb], dKa = -aKa[a][bb], dKc = aKc[a][bb];
+    aq[r * LDK + i] = dQg * e;
+    ak[r * LDK + i] = fmaf(dKa, e, dKc * ec);
+    const float kck = dKc * KcS[r * LDK + i];
+    aG[r * LDK + i] = dQg * QgS[r * LDK + i] + dKa * KaS[r * LDK + i] - kck;
+  });
+  {  // sum_r dKc_ri Kc_ri: this thread's 4 columns, then the 8 lanes of its row block
+    constexpr int NTN = C / 4;
+    const int tn = tid % NTN, tm = tid / NTN;
+#pragma unroll
+    for (int a = 0; a < TMK; ++a) {
+      const int i = tm + a * (DK / TMK);
+      float sacc = 0.f;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int r = tn + bb * NTN;
+        sacc = fmaf(aKc[a][bb], KcS[r * LDK + i], sacc);
+      }
+#pragma unroll
+      for (int o = NTN / 2; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+      if (tn == 0) kcsum[i] = sacc;
+    }
+  }
+  for_tile<C, C, 2, 2>([&](int r, int s, int i, int j) {
+    dAqS[r * LDC + s] = s <= r ? aA[i][j] : 0.f;
+    dTS[r * LDC + s] = aT[i][j];
+  });
+  __syncthreads();
+  // dbeta_s = sum_r dT_rs X_rs (from T = X Diag(beta)); dX = dT Diag(beta)
+  float db = 0.f;
+  if (tid < C) {
+    for (int r = 0; r < C; ++r) db = fmaf(dTS[r * LDC + tid], XS[r * LDC + tid], db);
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += NTH) {
+    const int r = idx / C, s = idx % C;
+    dTS[r * LDC + s] *= bS[s];
+  }
+  __syncthreads();
+  {  // dM = -X^T dX X^T, two C x C x C products; Y = dX X^T
+    float y[2][2];
+    zero(y);
+    mm<C, C, 2, 2, C>(y, [&](int m, int kk) { return dTS[m * LDC + kk]; },
+                      [&](int kk, int nn) { return XS[nn * LDC + kk]; });
+    for_tile<C, C, 2, 2>([&](int m, int nn, int i, int j) { YS[m * LDC + nn] = y[i][j]; });
+    __syncthreads();
+    float dm[2][2];
+    zero(dm);
+    mm<C, C, 2, 2, C>(dm, [&](int m, int kk) { return XS[kk * LDC + m]; },
+                      [&](int kk, int nn) { return YS[kk * LDC + nn]; });
+    for_tile<C, C, 2, 2>([&](int m, int nn, int i, int j) {
+      dTS[m * LDC + nn] = nn < m ? -dm[i][j] : 0.f;  // strict lower part of dM
+    });
+  }
+  __syncthreads();
+  // dbeta_r += sum_{s<r} dM_rs L_rs;  dL = Diag(beta) strict_lower(dM) (in place)
+  if (tid < C) {
+    float acc = 0.f;
+    for (int s = 0; s < tid; ++s) acc = fmaf(dTS[tid * LDC + s], LS[tid * LDC + s], acc);
+    db += acc;
+    if (tid < n) dbeta[rowbase + (size_t)tid * H] = db;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += NTH) {
+    const int r = idx / C, s = idx % C;
+    dTS[r * LDC + s] *= bS[r];
+  }
+  __syncthreads();
+  // through E: L_rs = sum_i k_ri k_si E_rsi, A_qk,rs = sum_i q_ri k_si E_rsi.
+  // Row side (thread of channel i owns rows r = part, part + P, ...):
+  //   a_k = sum_{s<=r} dL_rs k_si E_rsi, a_q = sum_s dA_qk,rs k_si E_rsi;
+  //   dk_ri += a_k, dq_ri += a_q, dGamma_ri += k_ri a_k + q_ri a_q.
+  // Column side (owns columns s): c_k = sum_{r>=s} (dL_rs k_ri + dA_qk,rs q_ri) E_rsi;
+  //   dk_si += c_k, dGamma_si -= k_si c_k.  Each element has one writer, in a
+  //   fixed order, so the result does not depend on scheduling.
+  {
+    constexpr int P = NTH / DK;
+    const int i = tid % DK, part = tid / DK;
+    for (int r = part; r < C; r += P) {
+      const float Gr = GS[r * LDK + i];
+      float ak_ = 0.f, aq_ = 0.f;
+      for (int s2 = 0; s2 <= r; ++s2) {
+        const float ke = kS[s2 * LDK + i] * expf(Gr - GS[s2 * LDK + i]);
+        ak_ = fmaf(dTS[r * LDC + s2], ke, ak_);
+        aq_ = fmaf(dAqS[r * LDC + s2], ke, aq_);
+      }
+      const float kr = kS[r * LDK + i], qr = qS[r * LDK + i];
+      ak[r * LDK + i] += ak_;
+      aq[r * LDK + i] += aq_;
+      aG[r * LDK + i] += fmaf(kr, ak_, qr * aq_);
+    }
+    __syncthreads();
+    for (int s2 = part; s2 < C; s2 += P) {
+      const float Gs = GS[s2 * LDK + i];
+      float ck = 0.f;
+      for (int r = s2; r < C; ++r) {
+        const float f = fmaf(dTS[r * LDC + s2], kS[r * LDK + i], dAqS[r * LDC + s2] * qS[r * LDK + i]);
+        ck = fmaf(f, expf(GS[r * LDK + i] - Gs), ck);
+      }
+      ak[s2 * LDK + i] += ck;
+      aG[s2 * LDK + i] -= kS[s2 * LDK + i] * ck;
+    }
+  }
+  __syncthreads();
+  // dg = reverse cumulative sum of dGamma, with dGamma_C (Kc and the state
+  // decay e^{Gamma_C} S depend on it) entering at the last row
+  for (int i = tid; i < DK; i += NTH) {
+    float acc = fmaf(expf(gC[i]), rsum[i], kcsum[i]);
+    for (int r = C - 1; r >= 0; --r) {
+      acc += aG[r * LDK + i];
+      aG[r * LDK + i] = acc;
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * DK; idx += NTH) {
+    const int r = idx / DK, i = idx % DK;
+    if (r < n) {
+      const size_t o = (rowbase + (size_t)r * H) * DK + i;
+      dq[o] = aq[r * LDK + i];
+      dk[o] = ak[r * LDK + i];
+      dg[o] = aG[r * LDK + i];
+    }
+  }
+}
+
+template <typename Tin, int DK>
+cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
+  constexpr int LDK = DK + 1;
+  const int nc = (a.T + C - 1) / C;
+  const int units = a.B * a.H, nblk = a.dv_dim / VB;
+  const size_t smF = sizeof(float) * (3 * C * LDK + DK * LDB + 2 * C * LDB + 3 * C * LDC + C + DK);
+  const size_t smA = sizeof(float) * (3 * C * LDK + DK * LDB + 3 * C * LDB + 2 * C * LDC + C + DK);
+  const size_t smB = BSmem<DK>::bytes;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smF)))
+    return e;
+  if ((e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA)))
+    return e;
+  if ((e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB)))
+    return e;
+  const Tin* q = static_cast<const Tin*>(a.q);
+  const Tin* k = static_cast<const Tin*>(a.k);
+  const Tin* v = static_cast<const Tin*>(a.v);
+  const Tin* dout = static_cast<const Tin*>(a.dout);
+  if (nc > 0) {
+    bwd_fwd_scan<Tin, DK><<<units * nblk, NTH, smF, st>>>(q, k, v, a.g, a.beta, a.init, a.T,
+                                                          a.H, a.dv_dim, a.ws);
+    if ((e = cudaGetLastError())) return e;
+  }
+  bwd_state_grad_scan<Tin, DK><<<units * nblk, NTH, smA, st>>>(
+      q, k, a.g, a.beta, dout, a.dfinal, a.T, a.H, a.dv_dim, a.scale, a.dinit, a.ws);
+  if ((e = cudaGetLastError())) return e;
+  if (nc > 0) {
+    bwd_chunk_grads<Tin, DK><<<units * nc, NTH, smB, st>>>(q, k, v, a.g, a.beta, dout, a.T, a.H,
+                                                           a.dv_dim, a.scale, a.dq, a.dk, a.dv,
+                                                           a.dg, a.dbeta, a.ws);
+    if ((e = cudaGetLastError())) return e;
+  }
+  return cudaSuccess;
+}
+
+template <typename Tin>
+cudaError_t by_dk(const BwdArgs& a, cudaStream_t st) {
+  switch (a.dk_dim) {
+    case 32: return launch_dk<Tin, 32>(a, st);
+    case 64: return launch_dk<Tin, 64>(a, st);
+    case 128: return launch_dk<Tin, 128>(a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+size_t bwd_chunk_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  const int nc = (T + C - 1) / C;
+  return (size_t)B * H * unit_ws_floats(nc, dk, dv) * sizeof(float);
+}
+
+cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t stream) {
+  if (a.B * a.H == 0) return cudaSuccess;
+  return a.dt == KDA_BF16 ? by_dk<__nv_bfloat16>(a, stream) : by_dk<float>(a, stream);
+}
+
+}  // namespace kda

@@ -287,10 +287,12 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * dL/do (dout) and, optionally, dL/dS_T of the final state (d_final).  The
  * pages define the forward only (Model Architecture > Kimi Delta Attention
  * (KDA); FlashKDA serves training too: Infrastructure > KDA kernels); this
- * is the chain rule applied to each step
- *   S'_t = Diag(exp(g_t)) S_{t-1},  p_t = S'_t^T k_t,  e_t = beta_t (v_t - p_t),
- *   S_t = S'_t + k_t e_t^T,  o_t = scale S_t^T q_t,
- * in reverse token order, with the states recomputed from saved checkpoints.
+ * is the chain rule of that recurrence, evaluated in the chunk form of the
+ * forward (32-token chunks): a forward pass saves every chunk's start state
+ * and key-side matrices, a reverse pass carries dL/dS from chunk to chunk,
+ * and every chunk's token gradients are then formed in parallel.  fp32
+ * arithmetic throughout (exponents of the decay taken as differences <= 0,
+ * so g must be <= 0, as the gate makes it).
  *  q, k, g : [B, T, H, dk]   v, dout : [B, T, H, dv]   beta : fp32 [B, T, H]
  *  init_state, d_final : fp32 [B, H, dk, dv] or NULL (zeros)
  * Outputs (fp32, written whole; d_init may be NULL to skip it):
@@ -298,8 +300,10 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  *  d_init : [B, H, dk, dv]  (dL/dS_0)
  * dout has the element type of q, k, v.  g is the log-decay (a gated caller
  * chains dg through its gate).  Dense batches only.  The workspace (size from
- * kda_recurrent_bwd_workspace_size, 0 for unsupported shapes) is scratch;
- * outputs must not alias inputs.
+ * kda_recurrent_bwd_workspace_size: per (sequence, head) and chunk two
+ * dk x dv states and three 32 x 32 matrices; 0 for unsupported shapes and for
+ * T = 0, when the workspace may be NULL) is scratch; outputs must not alias
+ * inputs.
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
  */
 KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv);

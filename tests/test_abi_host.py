@@ -191,8 +191,10 @@ def test_kcp_entries_reject_on_host(L):
 def test_backward_entries_reject_on_host(L):
     ptr = lambda i: FAKE + 0x1000 * i
     ws = L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128)
-    # (64 + 2 checkpoint blocks of 64 tokens) x B*H states of 64 KB
-    assert ws == (64 + 2) * 2 * 128 * 128 * 4
+    # per (sequence, head) and 32-token chunk: its start state, the gradient of
+    # its end state (64 KB each) and three 32 x 32 key-side matrices
+    assert ws == 2 * 4 * (2 * 128 * 128 + 3 * 32 * 32) * 4
+    assert L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128) == 0
     assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 96, 128) == 0
 
     def args(**over):
