@@ -51,7 +51,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
             subprocess.run(cmd, check=True)
-    if force or _stale(LIB, objs):
+    if force or _stale(LIB, objs + [CSRC]):  # the directory's mtime: a source removed
         cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs,
                "-Xcompiler", "-fvisibility=hidden"]
         subprocess.run(cmd, check=True)
