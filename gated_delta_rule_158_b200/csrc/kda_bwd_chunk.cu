@@ -12,12 +12,13 @@
 //   U = T (V - Ka S),  S_next = Diag(e^{Gamma_C}) S + Kc^T U,  O = scale (Qg S + A_qk U)
 // Three passes, fp32 throughout:
 //   F  chunk order, one CTA per (unit, 32 dv columns): the key-side matrices
-//      (saved once per chunk: X, A_qk, L) and the chunk-start states.
+//      (saved once per chunk: X, A_qk, L), the chunk-start states and
+//      R = V - Ka S, U = T R of every chunk.
 //   A  reverse chunk order, same grid: the state gradient dS = dL/dS_next,
 //        dU = A_qk^T dO' + Kc dS,  dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T T^T dU
-//      (dO' = scale dO); needs no state.  Saves dS of every chunk.
-//   B  one CTA per (unit, chunk), all chunks at once: with U, R = V - Ka S,
-//      dU and W = T^T dU (= dv) recomputed per 32 dv columns,
+//      (dO' = scale dO); needs no state.  Saves dS, dU and W = T^T dU of every
+//      chunk and writes dv = W.
+//   B  one CTA per (unit, chunk), all chunks at once, per 32 dv columns:
 //        dQg = dO' S^T, dKa = -W S^T, dKc = U dS^T,
 //        dA_qk = lower(dO' U^T), dT = dU R^T,
 //      then through T, X, L and A_qk (their entries' gradients back onto q, k
@@ -75,17 +76,22 @@ __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
     for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
 }
 
-// per-unit workspace: S_c [nc][DK][DV], dS_c [nc][DK][DV], X, A_qk, L [nc][C][C]
+// per-unit workspace: S_c, dS_c [nc][DK][DV]; X, A_qk, L [nc][C][C];
+// R, U, dU, W [nc][C][DV]
 struct UnitWs {
   float* S;
   float* dS;
   float* X;
   float* Aqk;
   float* L;
+  float* R;
+  float* U;
+  float* dU;
+  float* W;
 };
 
 __host__ __device__ inline size_t unit_ws_floats(int nc, int DK, int DV) {
-  return (size_t)nc * (2 * (size_t)DK * DV + 3 * C * C);
+  return (size_t)nc * (2 * (size_t)DK * DV + 3 * C * C + 4 * (size_t)C * DV);
 }
 
 __device__ inline UnitWs unit_ws(float* ws, int unit, int nc, int DK, int DV) {
@@ -96,6 +102,10 @@ __device__ inline UnitWs unit_ws(float* ws, int unit, int nc, int DK, int DV) {
   w.X = w.dS + (size_t)nc * DK * DV;
   w.Aqk = w.X + (size_t)nc * C * C;
   w.L = w.Aqk + (size_t)nc * C * C;
+  w.R = w.L + (size_t)nc * C * C;
+  w.U = w.R + (size_t)nc * C * DV;
+  w.dU = w.U + (size_t)nc * C * DV;
+  w.W = w.dU + (size_t)nc * C * DV;
   return w;
 }
 
@@ -138,6 +148,20 @@ __device__ void load_vblock(const Tin* x, size_t rowbase, int H, int DV, int j0,
     const int r = idx / VB, j = idx % VB;
     dst[r * LDB + j] =
         r < n ? mul * Elem<Tin>::load(x + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+  }
+}
+
+// [C x 32] tile <-> the chunk's rows of a [nc][C][DV] workspace array
+__device__ inline void store_tile(float* dst, int c, int DV, int j0, const float* src) {
+  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
+    const int r = idx / VB, j = idx % VB;
+    dst[((size_t)c * C + r) * DV + j0 + j] = src[r * LDB + j];
+  }
+}
+__device__ inline void load_tile(float* dst, const float* src, int c, int DV, int j0) {
+  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
+    const int r = idx / VB, j = idx % VB;
+    dst[r * LDB + j] = src[((size_t)c * C + r) * DV + j0 + j];
   }
 }
 
@@ -184,7 +208,7 @@ __global__ void __launch_bounds__(NTH, 2)
       const int i = idx / VB, j = idx % VB;
       w.S[((size_t)c * DK + i) * DV + j0 + j] = SS[i * LDB + j];
     }
-    // Gram matrices, exponents as differences (s <= r)
+    // Gram matrices, exponents as differences (s <= r), one pair per thread
     for (int p = tid; p < C * (C + 1) / 2; p += NTH) {
       int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
       while ((r + 1) * (r + 2) / 2 <= p) ++r;
@@ -193,8 +217,7 @@ __global__ void __launch_bounds__(NTH, 2)
       float lk = 0.f, lq = 0.f;
 #pragma unroll 4
       for (int i = 0; i < DK; ++i) {
-        const float e = expf(GS[r * LDK + i] - GS[s * LDK + i]);
-        const float ks = kS[s * LDK + i] * e;
+        const float ks = kS[s * LDK + i] * expf(GS[r * LDK + i] - GS[s * LDK + i]);
         lk = fmaf(kS[r * LDK + i], ks, lk);
         lq = fmaf(qS[r * LDK + i], ks, lq);
       }
@@ -264,6 +287,8 @@ __global__ void __launch_bounds__(NTH, 2)
       for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { US[m * LDB + nn] = acc[i][j]; });
     }
     __syncthreads();
+    store_tile(w.R, c, DV, j0, VS);
+    store_tile(w.U, c, DV, j0, US);
     {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
       constexpr int TM = DK / 32;
       float acc[TM][4];
@@ -283,8 +308,8 @@ __global__ void __launch_bounds__(NTH, 2)
     bwd_state_grad_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         const float* __restrict__ g, const float* __restrict__ beta,
                         const Tin* __restrict__ dout, const float* __restrict__ dfinal, int T,
-                        int H, int DV, float scale, float* __restrict__ dinit,
-                        float* __restrict__ ws) {
+                        int H, int DV, float scale, float* __restrict__ dv,
+                        float* __restrict__ dinit, float* __restrict__ ws) {
   constexpr int LDK = DK + 1;
   extern __shared__ float sm[];
   float* qS = sm;                 // [C][LDK]  q, later Qg
@@ -351,9 +376,14 @@ __global__ void __launch_bounds__(NTH, 2)
       zero(acc);
       mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
                          [&](int kk, int nn) { return dUS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { WS[m * LDB + nn] = acc[i][j]; });
+      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
+        WS[m * LDB + nn] = acc[i][j];
+        if (m < n) dv[(rowbase + (size_t)m * H) * DV + j0 + nn] = acc[i][j];
+      });
     }
     __syncthreads();
+    store_tile(w.dU, c, DV, j0, dUS);
+    store_tile(w.W, c, DV, j0, WS);
     {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
       constexpr int TM = DK / 32;
       float acc[TM][4];
@@ -377,55 +407,52 @@ __global__ void __launch_bounds__(NTH, 2)
 }
 
 // ===================================================================== pass B
+// B takes the dv columns 16 at a time, which keeps it at two CTAs per SM
+constexpr int VBB = 16;
+constexpr int LDBB = VBB + 1;
+
 template <int DK>
 struct BSmem {
   static constexpr int LDK = DK + 1;
   // the dv-block loop's tiles (S and dS blocks; dO', R, U, dU, W blocks) are
-  // dead once the loop ends, and the dq, dk, dGamma accumulators take their place
-  static constexpr int loop = 2 * DK * LDB + 5 * C * LDB;
-  static constexpr int accs = 3 * C * LDK;
-  static_assert(accs <= loop, "accumulators fit the loop tiles");
-  static constexpr int floats = 6 * C * LDK      // q, k, Gamma, Qg, Ka, Kc
+  // dead once the loop ends; the dGamma accumulator and a C x C scratch tile
+  // take their place (dq and dk accumulate in their outputs)
+  static constexpr int loop = 2 * DK * LDBB + 5 * C * LDBB;
+  static constexpr int after = C * LDK + C * LDC;
+  static_assert(after <= loop, "post-loop tiles fit the loop tiles");
+  static constexpr int floats = 3 * C * LDK      // q, k, Gamma
                                 + loop
-                                + 7 * C * LDC    // X, T, A_qk, L, dA_qk, dT (then dM), scratch
+                                + 4 * C * LDC    // X, L, dA_qk, dT (then dM)
                                 + C + 3 * DK;    // beta, Gamma_C, two dGamma_C terms
   static constexpr size_t bytes = sizeof(float) * floats;
 };
 
 template <typename Tin, int DK>
-__global__ void __launch_bounds__(NTH, 1)
+__global__ void __launch_bounds__(NTH, 2)
     bwd_chunk_grads(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                    const Tin* __restrict__ v, const float* __restrict__ g,
-                    const float* __restrict__ beta, const Tin* __restrict__ dout, int T, int H,
-                    int DV, float scale, float* __restrict__ dq, float* __restrict__ dk,
-                    float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
-                    float* __restrict__ ws) {
+                    const float* __restrict__ g, const float* __restrict__ beta,
+                    const Tin* __restrict__ dout, int T, int H, int DV, float scale,
+                    float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dg,
+                    float* __restrict__ dbeta, float* __restrict__ ws) {
   constexpr int LDK = DK + 1;
   extern __shared__ float sm[];
   float* qS = sm;
   float* kS = qS + C * LDK;
   float* GS = kS + C * LDK;       // Gamma
-  float* QgS = GS + C * LDK;
-  float* KaS = QgS + C * LDK;
-  float* KcS = KaS + C * LDK;
-  float* SS = KcS + C * LDK;      // [DK][LDB]   (dv-block loop)
-  float* dSS = SS + DK * LDB;     // [DK][LDB]
-  float* dOS = dSS + DK * LDB;    // [C][LDB]
-  float* RS = dOS + C * LDB;
-  float* US = RS + C * LDB;
-  float* dUS = US + C * LDB;
-  float* WS = dUS + C * LDB;
-  float* aq = SS;                 // after the loop: dq accumulator [C][LDK]
-  float* ak = aq + C * LDK;       //                 dk accumulator
-  float* aG = ak + C * LDK;       //                 dGamma accumulator
-  float* XS = WS + C * LDB;       // [C][LDC]
-  float* TS = XS + C * LDC;
-  float* AqS = TS + C * LDC;
-  float* LS = AqS + C * LDC;
+  float* SS = GS + C * LDK;       // [DK][LDBB]   (dv-block loop)
+  float* dSS = SS + DK * LDBB;    // [DK][LDBB]
+  float* dOS = dSS + DK * LDBB;   // [C][LDBB]
+  float* RS = dOS + C * LDBB;
+  float* US = RS + C * LDBB;
+  float* dUS = US + C * LDBB;
+  float* WS = dUS + C * LDBB;
+  float* aG = SS;                 // after the loop: dGamma accumulator [C][LDK]
+  float* YS = aG + C * LDK;       //                 scratch [C][LDC]
+  float* XS = WS + C * LDBB;      // [C][LDC]
+  float* LS = XS + C * LDC;
   float* dAqS = LS + C * LDC;
   float* dTS = dAqS + C * LDC;    // dT, then dM
-  float* YS = dTS + C * LDC;      // scratch
-  float* bS = YS + C * LDC;       // [C]
+  float* bS = dTS + C * LDC;      // [C]
   float* gC = bS + C;             // [DK] Gamma_C
   float* rsum = gC + DK;          // [DK] sum_j dS_ij S_ij
   float* kcsum = rsum + DK;       // [DK] sum_r dKc_ri Kc_ri
@@ -443,26 +470,16 @@ __global__ void __launch_bounds__(NTH, 1)
   for (int idx = tid; idx < C * C; idx += NTH) {
     const int r = idx / C, s = idx % C;
     const size_t o = ((size_t)c * C + r) * C + s;
-    const float x = w.X[o];
-    XS[r * LDC + s] = x;
-    TS[r * LDC + s] = x * bS[s];
-    AqS[r * LDC + s] = w.Aqk[o];
+    XS[r * LDC + s] = w.X[o];
     LS[r * LDC + s] = w.L[o];
   }
   for (int i = tid; i < DK; i += NTH) {
     gC[i] = GS[(C - 1) * LDK + i];
     rsum[i] = 0.f;
   }
-  __syncthreads();
-  for (int idx = tid; idx < C * DK; idx += NTH) {
-    const int r = idx / DK, i = idx % DK;
-    const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LDK + i];
-    QgS[r * LDK + i] = qS[r * LDK + i] * e;
-    KaS[r * LDK + i] = kv * e;
-    KcS[r * LDK + i] = kv * expf(gC[i] - G);
-  }
 
-  // products summed over the dv columns, accumulated block by block:
+  // products summed over the dv columns, accumulated block by block from
+  // the saved R, U, dU, W:
   // dQg^T = S dO'^T, -dKa^T = S W^T, dKc^T = dS U^T  (DK x C); dA_qk, dT (C x C)
   float aQ[TMK][4], aKa[TMK][4], aKc[TMK][4], aA[2][2], aT[2][2];
   zero(aQ);
@@ -470,76 +487,58 @@ __global__ void __launch_bounds__(NTH, 1)
   zero(aKc);
   zero(aA);
   zero(aT);
-  for (int j0 = 0; j0 < DV; j0 += VB) {
+  for (int j0 = 0; j0 < DV; j0 += VBB) {
     __syncthreads();
-    for (int idx = tid; idx < DK * VB; idx += NTH) {
-      const int i = idx / VB, j = idx % VB;
+    for (int idx = tid; idx < DK * VBB; idx += NTH) {
+      const int i = idx / VBB, j = idx % VBB;
       const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
-      SS[i * LDB + j] = w.S[o];
-      dSS[i * LDB + j] = w.dS[o];
+      SS[i * LDBB + j] = w.S[o];
+      dSS[i * LDBB + j] = w.dS[o];
     }
-    load_vblock<Tin>(v, rowbase, H, DV, j0, n, 1.f, RS);
-    load_vblock<Tin>(dout, rowbase, H, DV, j0, n, scale, dOS);
+    for (int idx = tid; idx < C * VBB; idx += NTH) {
+      const int r = idx / VBB, j = idx % VBB;
+      const size_t o = ((size_t)c * C + r) * DV + j0 + j;
+      dOS[r * LDBB + j] =
+          r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+      RS[r * LDBB + j] = w.R[o];
+      US[r * LDBB + j] = w.U[o];
+      dUS[r * LDBB + j] = w.dU[o];
+      WS[r * LDBB + j] = w.W[o];
+    }
     __syncthreads();
-    {  // R = V - Ka S;  dU = A_qk^T dO' + Kc dS
-      float p[2][2], u[2][2];
-      zero(p);
-      zero(u);
-      mm<C, VB, 2, 2, DK>(p, [&](int m, int kk) { return KaS[m * LDK + kk]; },
-                          [&](int kk, int nn) { return SS[kk * LDB + nn]; });
-      mm<C, VB, 2, 2, C>(u, [&](int m, int kk) { return AqS[kk * LDC + m]; },
-                         [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
-      mm<C, VB, 2, 2, DK>(u, [&](int m, int kk) { return KcS[m * LDK + kk]; },
-                          [&](int kk, int nn) { return dSS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
-        RS[m * LDB + nn] -= p[i][j];
-        dUS[m * LDB + nn] = u[i][j];
-      });
-    }
     for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
       float acc = 0.f;
 #pragma unroll 8
-      for (int j = 0; j < VB; ++j) acc = fmaf(dSS[i * LDB + j], SS[i * LDB + j], acc);
+      for (int j = 0; j < VBB; ++j) acc = fmaf(dSS[i * LDBB + j], SS[i * LDBB + j], acc);
       rsum[i] += acc;
     }
-    __syncthreads();
-    {  // U = T R;  W = T^T dU  (W is dv)
-      float u[2][2], wv[2][2];
-      zero(u);
-      zero(wv);
-      mm<C, VB, 2, 2, C>(u, [&](int m, int kk) { return TS[m * LDC + kk]; },
-                         [&](int kk, int nn) { return RS[kk * LDB + nn]; });
-      mm<C, VB, 2, 2, C>(wv, [&](int m, int kk) { return TS[kk * LDC + m]; },
-                         [&](int kk, int nn) { return dUS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
-        US[m * LDB + nn] = u[i][j];
-        WS[m * LDB + nn] = wv[i][j];
-        if (m < n) dv[(rowbase + (size_t)m * H) * DV + j0 + nn] = wv[i][j];
-      });
-    }
-    __syncthreads();
-    // block contributions, contracted over this block's 32 columns
-    mm<DK, C, TMK, 4, VB>(aQ, [&](int m, int kk) { return SS[m * LDB + kk]; },
-                          [&](int kk, int nn) { return dOS[nn * LDB + kk]; });
-    mm<DK, C, TMK, 4, VB>(aKa, [&](int m, int kk) { return SS[m * LDB + kk]; },
-                          [&](int kk, int nn) { return WS[nn * LDB + kk]; });
-    mm<DK, C, TMK, 4, VB>(aKc, [&](int m, int kk) { return dSS[m * LDB + kk]; },
-                          [&](int kk, int nn) { return US[nn * LDB + kk]; });
-    mm<C, C, 2, 2, VB>(aA, [&](int m, int kk) { return dOS[m * LDB + kk]; },
-                       [&](int kk, int nn) { return US[nn * LDB + kk]; });
-    mm<C, C, 2, 2, VB>(aT, [&](int m, int kk) { return dUS[m * LDB + kk]; },
-                       [&](int kk, int nn) { return RS[nn * LDB + kk]; });
+    // block contributions, contracted over this block's 16 columns
+    mm<DK, C, TMK, 4, VBB>(aQ, [&](int m, int kk) { return SS[m * LDBB + kk]; },
+                           [&](int kk, int nn) { return dOS[nn * LDBB + kk]; });
+    mm<DK, C, TMK, 4, VBB>(aKa, [&](int m, int kk) { return SS[m * LDBB + kk]; },
+                           [&](int kk, int nn) { return WS[nn * LDBB + kk]; });
+    mm<DK, C, TMK, 4, VBB>(aKc, [&](int m, int kk) { return dSS[m * LDBB + kk]; },
+                           [&](int kk, int nn) { return US[nn * LDBB + kk]; });
+    mm<C, C, 2, 2, VBB>(aA, [&](int m, int kk) { return dOS[m * LDBB + kk]; },
+                        [&](int kk, int nn) { return US[nn * LDBB + kk]; });
+    mm<C, C, 2, 2, VBB>(aT, [&](int m, int kk) { return dUS[m * LDBB + kk]; },
+                        [&](int kk, int nn) { return RS[nn * LDBB + kk]; });
   }
-  __syncthreads();  // the loop tiles become the accumulators
-  // dq, dk, dGamma from the state-side products and the decays
+  __syncthreads();  // the loop tiles become the dGamma accumulator
+  // dq, dk (into the outputs, rows < n) and dGamma from the state-side
+  // products and the decays
   for_tile<DK, C, TMK, 4>([&](int i, int r, int a, int bb) {
     const float e = expf(GS[r * LDK + i]);
     const float ec = expf(gC[i] - GS[r * LDK + i]);
     const float dQg = aQ[a][bb], dKa = -aKa[a][bb], dKc = aKc[a][bb];
-    aq[r * LDK + i] = dQg * e;
-    ak[r * LDK + i] = fmaf(dKa, e, dKc * ec);
-    const float kck = dKc * KcS[r * LDK + i];
-    aG[r * LDK + i] = dQg * QgS[r * LDK + i] + dKa * KaS[r * LDK + i] - kck;
+    const float qv = qS[r * LDK + i], kv = kS[r * LDK + i];
+    if (r < n) {
+      const size_t o = (rowbase + (size_t)r * H) * DK + i;
+      dq[o] = dQg * e;
+      dk[o] = fmaf(dKa, e, dKc * ec);
+    }
+    // dGamma: dQg Qg + dKa Ka - dKc Kc  (Qg = q e, Ka = k e, Kc = k ec)
+    aG[r * LDK + i] = fmaf(fmaf(dQg, qv, dKa * kv), e, -dKc * kv * ec);
   });
   {  // sum_r dKc_ri Kc_ri: this thread's 4 columns, then the 8 lanes of its row block
     constexpr int NTN = C / 4;
@@ -551,7 +550,7 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
       for (int bb = 0; bb < 4; ++bb) {
         const int r = tn + bb * NTN;
-        sacc = fmaf(aKc[a][bb], KcS[r * LDK + i], sacc);
+        sacc = fmaf(aKc[a][bb], kS[r * LDK + i] * expf(gC[i] - GS[r * LDK + i]), sacc);
       }
 #pragma unroll
       for (int o = NTN / 2; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
@@ -622,8 +621,11 @@ __global__ void __launch_bounds__(NTH, 1)
         aq_ = fmaf(dAqS[r * LDC + s2], ke, aq_);
       }
       const float kr = kS[r * LDK + i], qr = qS[r * LDK + i];
-      ak[r * LDK + i] += ak_;
-      aq[r * LDK + i] += aq_;
+      if (r < n) {
+        const size_t o = (rowbase + (size_t)r * H) * DK + i;
+        dk[o] += ak_;
+        dq[o] += aq_;
+      }
       aG[r * LDK + i] += fmaf(kr, ak_, qr * aq_);
     }
     __syncthreads();
@@ -634,7 +636,7 @@ __global__ void __launch_bounds__(NTH, 1)
         const float f = fmaf(dTS[r * LDC + s2], kS[r * LDK + i], dAqS[r * LDC + s2] * qS[r * LDK + i]);
         ck = fmaf(f, expf(GS[r * LDK + i] - Gs), ck);
       }
-      ak[s2 * LDK + i] += ck;
+      if (s2 < n) dk[(rowbase + (size_t)s2 * H) * DK + i] += ck;
       aG[s2 * LDK + i] -= kS[s2 * LDK + i] * ck;
     }
   }
@@ -651,12 +653,7 @@ __global__ void __launch_bounds__(NTH, 1)
   __syncthreads();
   for (int idx = tid; idx < C * DK; idx += NTH) {
     const int r = idx / DK, i = idx % DK;
-    if (r < n) {
-      const size_t o = (rowbase + (size_t)r * H) * DK + i;
-      dq[o] = aq[r * LDK + i];
-      dk[o] = ak[r * LDK + i];
-      dg[o] = aG[r * LDK + i];
-    }
+    if (r < n) dg[(rowbase + (size_t)r * H) * DK + i] = aG[r * LDK + i];
   }
 }
 
@@ -688,12 +685,12 @@ cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError())) return e;
   }
   bwd_state_grad_scan<Tin, DK><<<units * nblk, NTH, smA, st>>>(
-      q, k, a.g, a.beta, dout, a.dfinal, a.T, a.H, a.dv_dim, a.scale, a.dinit, a.ws);
+      q, k, a.g, a.beta, dout, a.dfinal, a.T, a.H, a.dv_dim, a.scale, a.dv, a.dinit, a.ws);
   if ((e = cudaGetLastError())) return e;
   if (nc > 0) {
-    bwd_chunk_grads<Tin, DK><<<units * nc, NTH, smB, st>>>(q, k, v, a.g, a.beta, dout, a.T, a.H,
-                                                           a.dv_dim, a.scale, a.dq, a.dk, a.dv,
-                                                           a.dg, a.dbeta, a.ws);
+    bwd_chunk_grads<Tin, DK><<<units * nc, NTH, smB, st>>>(q, k, a.g, a.beta, dout, a.T, a.H,
+                                                           a.dv_dim, a.scale, a.dq, a.dk, a.dg,
+                                                           a.dbeta, a.ws);
     if ((e = cudaGetLastError())) return e;
   }
   return cudaSuccess;

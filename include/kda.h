@@ -301,7 +301,8 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * dout has the element type of q, k, v.  g is the log-decay (a gated caller
  * chains dg through its gate).  Dense batches only.  The workspace (size from
  * kda_recurrent_bwd_workspace_size: per (sequence, head) and chunk two
- * dk x dv states and three 32 x 32 matrices; 0 for unsupported shapes and for
+ * dk x dv states, three 32 x 32 matrices and four 32 x dv tiles; 0 for
+ * unsupported shapes and for
  * T = 0, when the workspace may be NULL) is scratch; outputs must not alias
  * inputs.
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.

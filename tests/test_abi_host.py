@@ -192,8 +192,9 @@ def test_backward_entries_reject_on_host(L):
     ptr = lambda i: FAKE + 0x1000 * i
     ws = L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128)
     # per (sequence, head) and 32-token chunk: its start state, the gradient of
-    # its end state (64 KB each) and three 32 x 32 key-side matrices
-    assert ws == 2 * 4 * (2 * 128 * 128 + 3 * 32 * 32) * 4
+    # its end state (64 KB each), three 32 x 32 key-side matrices and four
+    # 32 x dv intermediates (R, U, dU, W)
+    assert ws == 2 * 4 * (2 * 128 * 128 + 3 * 32 * 32 + 4 * 32 * 128) * 4
     assert L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128) == 0
     assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 96, 128) == 0
 
