@@ -11,9 +11,9 @@
 //   Qg = q e^Gamma,  Ka = k e^Gamma,  Kc = k e^{Gamma_C - Gamma}
 //   U = T (V - Ka S),  S_next = Diag(e^{Gamma_C}) S + Kc^T U,  O = scale (Qg S + A_qk U)
 // Three passes, fp32 throughout:
-//   F  chunk order, one CTA per (unit, 32 dv columns): the key-side matrices
-//      (saved once per chunk: X, A_qk, L), the chunk-start states and
-//      R = V - Ka S, U = T R of every chunk.
+//   F  chunk order, one CTA per unit: the key-side matrices (saved once per
+//      chunk: X, A_qk, L), the chunk-start states and R = V - Ka S, U = T R
+//      of every chunk.
 //   A  reverse chunk order, same grid: the state gradient dS = dL/dS_next,
 //        dU = A_qk^T dO' + Kc dS,  dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T T^T dU
 //      (dO' = scale dO); needs no state.  Saves dS, dU and W = T^T dU of every
@@ -31,17 +31,21 @@ namespace kda {
 namespace {
 
 constexpr int C = 32;
-constexpr int NTH = 256;
+constexpr int NTH = 256;       // threads of the A and B kernels
+constexpr int NTF = 512;       // threads of the F kernel (one CTA per unit)
+constexpr int MREB = 15;       // rebasing row of the factorised Gram
 constexpr int VB = 32;         // dv columns per block
 constexpr int LDC = C + 1;     // C x C tiles
 constexpr int LDB = VB + 1;    // x 32-column tiles
 static_assert(NTH == 8 * 32, "forward substitution: 8 warps x 4 columns");
 
-// acc[i][j] += sum_k a(m_i, k) b(k, n_j) over a 256-thread tile of an M x N
-// product: thread (tm, tn) owns rows tm + i M/TM and columns tn + j N/TN.
+// acc[i][j] += sum_k a(m_i, k) b(k, n_j) over an M x N product split into
+// one TM x TN tile per thread of the block (256 or 512 threads): thread
+// (tm, tn) owns rows tm + i M/TM and columns tn + j N/TN.
 template <int M, int N, int TM, int TN, int K, typename FA, typename FB>
 __device__ __forceinline__ void mm(float (&acc)[TM][TN], FA a, FB b) {
-  static_assert((M / TM) * (N / TN) == NTH, "one output tile per thread");
+  static_assert((M / TM) * (N / TN) == NTH || (M / TM) * (N / TN) == NTF,
+                "one output tile per thread");
   constexpr int NTN = N / TN, MS = M / TM;
   const int tn = threadIdx.x % NTN, tm = threadIdx.x / NTN;
 #pragma unroll 4
@@ -151,152 +155,203 @@ __device__ void load_vblock(const Tin* x, size_t rowbase, int H, int DV, int j0,
   }
 }
 
-// [C x 32] tile <-> the chunk's rows of a [nc][C][DV] workspace array
+// [C x 32] tile -> the chunk's rows of a [nc][C][DV] workspace array
 __device__ inline void store_tile(float* dst, int c, int DV, int j0, const float* src) {
   for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
     const int r = idx / VB, j = idx % VB;
     dst[((size_t)c * C + r) * DV + j0 + j] = src[r * LDB + j];
   }
 }
-__device__ inline void load_tile(float* dst, const float* src, int c, int DV, int j0) {
-  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
-    const int r = idx / VB, j = idx % VB;
-    dst[r * LDB + j] = src[((size_t)c * C + r) * DV + j0 + j];
-  }
-}
 
 // ===================================================================== pass F
-template <typename Tin, int DK>
-__global__ void __launch_bounds__(NTH, 2)
+// One CTA of 512 threads per unit, all dv columns, so the key-side matrices
+// are formed once per chunk.  The Gram matrices are one product each when
+// the chunk's decays let every factor e^{+-(Gamma_r - Gamma_15)} stay below
+// e^80 (always, for the gate's g >= -5): L = (k e^{Gamma - Gamma_15})
+// (k e^{Gamma_15 - Gamma})^T; otherwise each entry takes exponentials of
+// differences Gamma_r - Gamma_s <= 0.
+template <int DK, int DV>
+struct FSmem {
+  static constexpr int LDK = DK + 1, LDV = DV + 1;
+  static constexpr int floats = 5 * C * LDK       // q (then q factor), k (then Kc), Gamma, two factors
+                                + DK * LDV        // state
+                                + 2 * C * LDV     // V (then R), U
+                                + 3 * C * LDC     // L, A_qk, X (then T)
+                                + C + 2 * DK;     // beta, Gamma_C, e^{Gamma_C}
+  static constexpr size_t bytes = sizeof(float) * floats;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(NTF, 1)
     bwd_fwd_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                  const Tin* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const float* __restrict__ init, int T, int H,
-                 int DV, float* __restrict__ ws) {
-  constexpr int LDK = DK + 1;
+                 float* __restrict__ ws) {
+  constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
-  float* qS = sm;                 // [C][LDK]
-  float* kS = qS + C * LDK;       // [C][LDK]  k, later Kc
-  float* GS = kS + C * LDK;       // [C][LDK]  Gamma, later Ka
-  float* SS = GS + C * LDK;       // [DK][LDB] state block
-  float* VS = SS + DK * LDB;      // [C][LDB]  V, then V - P
-  float* US = VS + C * LDB;       // [C][LDB]
-  float* LS = US + C * LDB;       // [C][LDC]
+  float* qS = sm;                 // [C][LDK]  q, then q e^{Gamma - Gamma_15}
+  float* kS = qS + C * LDK;       // [C][LDK]  k, then Kc
+  float* GS = kS + C * LDK;       // [C][LDK]  Gamma
+  float* FaS = GS + C * LDK;      // [C][LDK]  k e^{Gamma - Gamma_15}, then Ka
+  float* FbS = FaS + C * LDK;     // [C][LDK]  k e^{Gamma_15 - Gamma}
+  float* SS = FbS + C * LDK;      // [DK][LDV] state
+  float* VS = SS + DK * LDV;      // [C][LDV]  V, then R = V - Ka S
+  float* US = VS + C * LDV;       // [C][LDV]
+  float* LS = US + C * LDV;       // [C][LDC]
   float* AqS = LS + C * LDC;      // [C][LDC]
   float* XS = AqS + C * LDC;      // [C][LDC]  X, then T
   float* bS = XS + C * LDC;       // [C]
-  float* gC = bS + C;             // [DK]
+  float* gC = bS + C;             // [DK] Gamma_C
+  float* eC = gC + DK;            // [DK] e^{Gamma_C}
 
-  const int nblk = DV / VB;
-  const int unit = blockIdx.x / nblk, j0 = (blockIdx.x % nblk) * VB;
+  const int unit = blockIdx.x;
   const int b = unit / H, h = unit % H;
   const int nc = (T + C - 1) / C;
   const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
   const int tid = threadIdx.x;
 
-  for (int idx = tid; idx < DK * VB; idx += NTH) {
-    const int i = idx / VB, j = idx % VB;
-    SS[i * LDB + j] = init ? init[((size_t)unit * DK + i) * DV + j0 + j] : 0.f;
+  for (int idx = tid; idx < DK * DV; idx += NTF) {
+    const int i = idx / DV, j = idx % DV;
+    SS[i * LDV + j] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
   }
   for (int c = 0; c < nc; ++c) {
     const int t0 = c * C, n = min(C, T - t0);
     const size_t rowbase = ((size_t)b * T + t0) * H + h;
     __syncthreads();
-    load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
-    load_vblock<Tin>(v, rowbase, H, DV, j0, n, 1.f, VS);
-    // chunk-start state block
-    for (int idx = tid; idx < DK * VB; idx += NTH) {
-      const int i = idx / VB, j = idx % VB;
-      w.S[((size_t)c * DK + i) * DV + j0 + j] = SS[i * LDB + j];
-    }
-    // Gram matrices, exponents as differences (s <= r), one pair per thread
-    for (int p = tid; p < C * (C + 1) / 2; p += NTH) {
-      int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
-      while ((r + 1) * (r + 2) / 2 <= p) ++r;
-      while (r * (r + 1) / 2 > p) --r;
-      const int s = p - r * (r + 1) / 2;
-      float lk = 0.f, lq = 0.f;
-#pragma unroll 4
-      for (int i = 0; i < DK; ++i) {
-        const float ks = kS[s * LDK + i] * expf(GS[r * LDK + i] - GS[s * LDK + i]);
-        lk = fmaf(kS[r * LDK + i], ks, lk);
-        lq = fmaf(qS[r * LDK + i], ks, lq);
+    for (int idx = tid; idx < C * DK; idx += NTF) {
+      const int r = idx / DK, i = idx % DK;
+      float qv = 0.f, kv = 0.f, gv = 0.f;
+      if (r < n) {
+        const size_t off = (rowbase + (size_t)r * H) * DK + i;
+        qv = Elem<Tin>::load(q + off);
+        kv = Elem<Tin>::load(k + off);
+        gv = g[off];
       }
-      LS[r * LDC + s] = s < r ? lk : 0.f;
-      AqS[r * LDC + s] = lq;
+      qS[r * LDK + i] = qv;
+      kS[r * LDK + i] = kv;
+      GS[r * LDK + i] = gv;
     }
-    for (int idx = tid; idx < C * C; idx += NTH) {
-      const int r = idx / C, s = idx % C;
-      if (s > r) {
-        LS[r * LDC + s] = 0.f;
-        AqS[r * LDC + s] = 0.f;
+    for (int idx = tid; idx < C * DV; idx += NTF) {
+      const int r = idx / DV, j = idx % DV;
+      VS[r * LDV + j] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+    }
+    if (tid < C) bS[tid] = tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+    for (int idx = tid; idx < DK * DV; idx += NTF) {  // chunk-start state
+      const int i = idx / DV, j = idx % DV;
+      w.S[(size_t)c * DK * DV + idx] = SS[i * LDV + j];
+    }
+    __syncthreads();
+    bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LDK + i];
+        GS[r * LDK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+      const float g15 = GS[MREB * LDK + i];
+      for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - g15) > 80.f;
+    }
+    wide = __syncthreads_or(wide);
+    if (!wide) {
+      for (int idx = tid; idx < C * DK; idx += NTF) {
+        const int r = idx / DK, i = idx % DK;
+        const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+        const float ea = expf(d), eb = expf(-d), kv = kS[r * LDK + i];
+        FaS[r * LDK + i] = kv * ea;
+        FbS[r * LDK + i] = kv * eb;
+        qS[r * LDK + i] *= ea;
+      }
+      __syncthreads();
+      float lk[1][2], lq[1][2];
+      zero(lk);
+      zero(lq);
+      mm<C, C, 1, 2, DK>(lk, [&](int m, int kk) { return FaS[m * LDK + kk]; },
+                         [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
+      mm<C, C, 1, 2, DK>(lq, [&](int m, int kk) { return qS[m * LDK + kk]; },
+                         [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
+      for_tile<C, C, 1, 2>([&](int r, int s2, int i, int j) {
+        LS[r * LDC + s2] = s2 < r ? lk[i][j] : 0.f;
+        AqS[r * LDC + s2] = s2 <= r ? lq[i][j] : 0.f;
+      });
+    } else {
+      for (int p = tid; p < C * C; p += NTF) {
+        const int r = p / C, s2 = p % C;
+        float lk = 0.f, lq = 0.f;
+        if (s2 <= r) {
+#pragma unroll 4
+          for (int i = 0; i < DK; ++i) {
+            const float ks = kS[s2 * LDK + i] * expf(GS[r * LDK + i] - GS[s2 * LDK + i]);
+            lk = fmaf(kS[r * LDK + i], ks, lk);
+            lq = fmaf(qS[r * LDK + i], ks, lq);
+          }
+        }
+        LS[r * LDC + s2] = s2 < r ? lk : 0.f;
+        AqS[r * LDC + s2] = lq;
       }
     }
     __syncthreads();
     // X = (I + Diag(beta) L)^-1 by forward substitution; the columns are
-    // independent, so warp w takes columns 4w .. 4w+3 with 8 lanes per column
+    // independent, so warp w takes columns 2w, 2w + 1 with 16 lanes per column
     {
-      const int lane = tid & 31, cc = 4 * (tid >> 5) + (lane >> 3), sub = lane & 7;
-      for (int r = sub; r < C; r += 8) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
+      const int lane = tid & 31, cc = 2 * (tid >> 5) + (lane >> 4), sub = lane & 15;
+      for (int r = sub; r < C; r += 16) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
       __syncwarp();
       for (int r = 1; r < C; ++r) {
         float acc = 0.f;
-        for (int s = cc + sub; s < r; s += 8) acc = fmaf(LS[r * LDC + s], XS[s * LDC + cc], acc);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        for (int s2 = cc + sub; s2 < r; s2 += 16) acc = fmaf(LS[r * LDC + s2], XS[s2 * LDC + cc], acc);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (sub == 0 && r > cc) XS[r * LDC + cc] = -bS[r] * acc;
         __syncwarp();
       }
     }
-    for (int i = tid; i < DK; i += NTH) gC[i] = GS[(C - 1) * LDK + i];
     __syncthreads();
-    if (j0 == 0) {  // the key-side matrices, once per chunk
-      for (int idx = tid; idx < C * C; idx += NTH) {
-        const int r = idx / C, s = idx % C;
-        const size_t o = ((size_t)c * C + r) * C + s;
-        w.X[o] = XS[r * LDC + s];
-        w.Aqk[o] = AqS[r * LDC + s];
-        w.L[o] = LS[r * LDC + s];
-      }
+    for (int idx = tid; idx < C * C; idx += NTF) {  // the key-side matrices, then T
+      const int r = idx / C, s2 = idx % C;
+      const size_t o = ((size_t)c * C + r) * C + s2;
+      const float x = XS[r * LDC + s2];
+      w.X[o] = x;
+      w.Aqk[o] = AqS[r * LDC + s2];
+      w.L[o] = LS[r * LDC + s2];
+      XS[r * LDC + s2] = x * bS[s2];
     }
-    __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NTH) {  // T = X Diag(beta)
-      const int r = idx / C, s = idx % C;
-      XS[r * LDC + s] *= bS[s];
-    }
-    for (int idx = tid; idx < C * DK; idx += NTH) {  // Ka, Kc
+    for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka (into FaS), Kc (into kS)
       const int r = idx / DK, i = idx % DK;
       const float G = GS[r * LDK + i], kv = kS[r * LDK + i];
-      GS[r * LDK + i] = kv * expf(G);
+      FaS[r * LDK + i] = kv * expf(G);
       kS[r * LDK + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
-    {  // V <- V - Ka S
-      float acc[2][2];
+    {  // R = V - Ka S
+      float acc[1][DV / 16];
       zero(acc);
-      mm<C, VB, 2, 2, DK>(acc, [&](int m, int kk) { return GS[m * LDK + kk]; },
-                          [&](int kk, int nn) { return SS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { VS[m * LDB + nn] -= acc[i][j]; });
+      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return FaS[m * LDK + kk]; },
+                                [&](int kk, int nn) { return SS[kk * LDV + nn]; });
+      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { VS[m * LDV + nn] -= acc[i][j]; });
     }
     __syncthreads();
-    {  // U = T (V - Ka S)
-      float acc[2][2];
+    {  // U = T R
+      float acc[1][DV / 16];
       zero(acc);
-      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return XS[m * LDC + kk]; },
-                         [&](int kk, int nn) { return VS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { US[m * LDB + nn] = acc[i][j]; });
+      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return XS[m * LDC + kk]; },
+                               [&](int kk, int nn) { return VS[kk * LDV + nn]; });
+      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
     }
     __syncthreads();
-    store_tile(w.R, c, DV, j0, VS);
-    store_tile(w.U, c, DV, j0, US);
+    for (int idx = tid; idx < C * DV; idx += NTF) {
+      const int r = idx / DV, j = idx % DV;
+      w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
+      w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
+    }
     {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
-      constexpr int TM = DK / 32;
-      float acc[TM][4];
+      float acc[DK / 32][DV / 16];
       zero(acc);
-      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
-                           [&](int kk, int nn) { return US[kk * LDB + nn]; });
-      for_tile<DK, VB, TM, 4>([&](int m, int nn, int i, int j) {
-        SS[m * LDB + nn] = fmaf(expf(gC[m]), SS[m * LDB + nn], acc[i][j]);
+      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
+                                      [&](int kk, int nn) { return US[kk * LDV + nn]; });
+      for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
+        SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
       });
     }
   }
@@ -657,18 +712,26 @@ __global__ void __launch_bounds__(NTH, 2)
   }
 }
 
+template <typename Tin, int DK, int DV>
+cudaError_t launch_fwd_scan(const BwdArgs& a, cudaStream_t st) {
+  const size_t smF = FSmem<DK, DV>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
+  if (e != cudaSuccess) return e;
+  bwd_fwd_scan<Tin, DK, DV><<<a.B * a.H, NTF, smF, st>>>(
+      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+      a.g, a.beta, a.init, a.T, a.H, a.ws);
+  return cudaGetLastError();
+}
+
 template <typename Tin, int DK>
 cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
   constexpr int LDK = DK + 1;
   const int nc = (a.T + C - 1) / C;
   const int units = a.B * a.H, nblk = a.dv_dim / VB;
-  const size_t smF = sizeof(float) * (3 * C * LDK + DK * LDB + 2 * C * LDB + 3 * C * LDC + C + DK);
   const size_t smA = sizeof(float) * (3 * C * LDK + DK * LDB + 3 * C * LDB + 2 * C * LDC + C + DK);
   const size_t smB = BSmem<DK>::bytes;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smF)))
-    return e;
   if ((e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA)))
     return e;
@@ -677,12 +740,15 @@ cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
     return e;
   const Tin* q = static_cast<const Tin*>(a.q);
   const Tin* k = static_cast<const Tin*>(a.k);
-  const Tin* v = static_cast<const Tin*>(a.v);
   const Tin* dout = static_cast<const Tin*>(a.dout);
   if (nc > 0) {
-    bwd_fwd_scan<Tin, DK><<<units * nblk, NTH, smF, st>>>(q, k, v, a.g, a.beta, a.init, a.T,
-                                                          a.H, a.dv_dim, a.ws);
-    if ((e = cudaGetLastError())) return e;
+    switch (a.dv_dim) {
+      case 32: e = launch_fwd_scan<Tin, DK, 32>(a, st); break;
+      case 64: e = launch_fwd_scan<Tin, DK, 64>(a, st); break;
+      case 128: e = launch_fwd_scan<Tin, DK, 128>(a, st); break;
+      default: e = cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
   }
   bwd_state_grad_scan<Tin, DK><<<units * nblk, NTH, smA, st>>>(
       q, k, a.g, a.beta, dout, a.dfinal, a.T, a.H, a.dv_dim, a.scale, a.dv, a.dinit, a.ws);

@@ -144,3 +144,26 @@ def test_backward_fullsize_sampled(oracle_mod):
             got = to64(grads[n][b, :, h])
             assert rel_l2(got, ref[n][0, :, 0]) <= TOL_F32, (b, h, n)
         assert rel_l2(to64(grads["d_init"][b, h]), ref["dS0"][0, 0]) <= TOL_F32
+
+
+def test_backward_strong_decay_takes_exact_exponents(oracle_mod):
+    """A gate floor of -40 lets a 16-token half chunk decay by far more than
+    e^80, which sends the key-side Gram to its exponent-difference form; the
+    gradients still meet the fp32 bar."""
+    B, T, H, dk, dv = 1, 150, 2, 64, 64
+    inp = W.make_prefill_inputs(B, T, H, dk, dv, torch.float32, seed=31, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, dv, dk=dk, dtype=torch.float32, seed=32,
+                                     device=DEV)
+    g = torch.empty_like(inp["z"])
+    kda.kda_gate_fwd(inp["z"], inp["A_log"], g, g_min=-40.0)
+    assert float(g.min()) < -10.0
+    got = gpu_backward(inp, cot, g, 1.0, True, True)
+    g_ref = oracle_mod.gate(to64(inp["z"]), to64(inp["A_log"]), -40.0)
+    ref = oracle_mod.backward(to64(inp["q"]), to64(inp["k"]), to64(inp["v"]), g_ref,
+                              to64(inp["beta"]), to64(cot["dout"]),
+                              init_state=to64(inp["init_state"]),
+                              d_final=to64(cot["d_final"]))
+    for n in NAMES:
+        assert rel_l2(got[n], ref[n]) <= TOL_F32, (n, rel_l2(got[n], ref[n]))
+    assert rel_l2(got["d_init"], ref["dS0"]) <= TOL_F32
