@@ -34,10 +34,7 @@ constexpr int C = 32;
 constexpr int NTH = 256;       // threads of the A and B kernels
 constexpr int NTF = 512;       // threads of the F kernel (one CTA per unit)
 constexpr int MREB = 15;       // rebasing row of the factorised Gram
-constexpr int VB = 32;         // dv columns per block
 constexpr int LDC = C + 1;     // C x C tiles
-constexpr int LDB = VB + 1;    // x 32-column tiles
-static_assert(NTH == 8 * 32, "forward substitution: 8 warps x 4 columns");
 
 // acc[i][j] += sum_k a(m_i, k) b(k, n_j) over an M x N product split into
 // one TM x TN tile per thread of the block (256 or 512 threads): thread
@@ -142,25 +139,6 @@ __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const floa
     }
   }
   __syncthreads();
-}
-
-// [C x 32] block of a [*, DV] token tensor (columns j0 .. j0+31), times mul
-template <typename Tin>
-__device__ void load_vblock(const Tin* x, size_t rowbase, int H, int DV, int j0, int n,
-                            float mul, float* dst) {
-  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
-    const int r = idx / VB, j = idx % VB;
-    dst[r * LDB + j] =
-        r < n ? mul * Elem<Tin>::load(x + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
-  }
-}
-
-// [C x 32] tile -> the chunk's rows of a [nc][C][DV] workspace array
-__device__ inline void store_tile(float* dst, int c, int DV, int j0, const float* src) {
-  for (int idx = threadIdx.x; idx < C * VB; idx += NTH) {
-    const int r = idx / VB, j = idx % VB;
-    dst[((size_t)c * C + r) * DV + j0 + j] = src[r * LDB + j];
-  }
 }
 
 // ===================================================================== pass F
@@ -358,57 +336,96 @@ __global__ void __launch_bounds__(NTF, 1)
 }
 
 // ===================================================================== pass A
-template <typename Tin, int DK>
-__global__ void __launch_bounds__(NTH, 2)
+// One CTA of 512 threads per unit, all dv columns (the key-side loads and
+// decays once per chunk).
+template <int DK, int DV>
+struct ASmem {
+  static constexpr int LDK = DK + 1, LDV = DV + 1;
+  static constexpr int floats = 3 * C * LDK       // q (then Qg), k (then Kc), Gamma (then Ka)
+                                + DK * LDV        // state gradient
+                                + 3 * C * LDV     // dO', dU, W
+                                + 2 * C * LDC     // A_qk, T
+                                + C + 2 * DK;     // beta, Gamma_C, e^{Gamma_C}
+  static constexpr size_t bytes = sizeof(float) * floats;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(NTF, 1)
     bwd_state_grad_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         const float* __restrict__ g, const float* __restrict__ beta,
                         const Tin* __restrict__ dout, const float* __restrict__ dfinal, int T,
-                        int H, int DV, float scale, float* __restrict__ dv,
-                        float* __restrict__ dinit, float* __restrict__ ws) {
-  constexpr int LDK = DK + 1;
+                        int H, float scale, float* __restrict__ dv, float* __restrict__ dinit,
+                        float* __restrict__ ws) {
+  constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
   float* qS = sm;                 // [C][LDK]  q, later Qg
   float* kS = qS + C * LDK;       // [C][LDK]  k, later Kc
   float* GS = kS + C * LDK;       // [C][LDK]  Gamma, later Ka
-  float* dSS = GS + C * LDK;      // [DK][LDB] state-gradient block
-  float* dOS = dSS + DK * LDB;    // [C][LDB]  scale dO
-  float* dUS = dOS + C * LDB;     // [C][LDB]
-  float* WS = dUS + C * LDB;      // [C][LDB]
-  float* AqS = WS + C * LDB;      // [C][LDC]
+  float* dSS = GS + C * LDK;      // [DK][LDV] state gradient
+  float* dOS = dSS + DK * LDV;    // [C][LDV]  scale dO
+  float* dUS = dOS + C * LDV;     // [C][LDV]
+  float* WS = dUS + C * LDV;      // [C][LDV]
+  float* AqS = WS + C * LDV;      // [C][LDC]
   float* TS = AqS + C * LDC;      // [C][LDC]
   float* bS = TS + C * LDC;       // [C]
   float* gC = bS + C;             // [DK]
+  float* eC = gC + DK;            // [DK]
 
-  const int nblk = DV / VB;
-  const int unit = blockIdx.x / nblk, j0 = (blockIdx.x % nblk) * VB;
+  const int unit = blockIdx.x;
   const int b = unit / H, h = unit % H;
   const int nc = (T + C - 1) / C;
   const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
   const int tid = threadIdx.x;
 
-  for (int idx = tid; idx < DK * VB; idx += NTH) {
-    const int i = idx / VB, j = idx % VB;
-    dSS[i * LDB + j] = dfinal ? dfinal[((size_t)unit * DK + i) * DV + j0 + j] : 0.f;
+  for (int idx = tid; idx < DK * DV; idx += NTF) {
+    const int i = idx / DV, j = idx % DV;
+    dSS[i * LDV + j] = dfinal ? dfinal[(size_t)unit * DK * DV + idx] : 0.f;
   }
   for (int c = nc - 1; c >= 0; --c) {
     const int t0 = c * C, n = min(C, T - t0);
     const size_t rowbase = ((size_t)b * T + t0) * H + h;
     __syncthreads();
-    load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
-    load_vblock<Tin>(dout, rowbase, H, DV, j0, n, scale, dOS);
-    for (int idx = tid; idx < C * C; idx += NTH) {
-      const int r = idx / C, s = idx % C;
-      const size_t o = ((size_t)c * C + r) * C + s;
-      AqS[r * LDC + s] = w.Aqk[o];
-      TS[r * LDC + s] = w.X[o] * bS[s];
+    for (int idx = tid; idx < C * DK; idx += NTF) {
+      const int r = idx / DK, i = idx % DK;
+      float qv = 0.f, kv = 0.f, gv = 0.f;
+      if (r < n) {
+        const size_t off = (rowbase + (size_t)r * H) * DK + i;
+        qv = Elem<Tin>::load(q + off);
+        kv = Elem<Tin>::load(k + off);
+        gv = g[off];
+      }
+      qS[r * LDK + i] = qv;
+      kS[r * LDK + i] = kv;
+      GS[r * LDK + i] = gv;
     }
-    for (int idx = tid; idx < DK * VB; idx += NTH) {  // dL/dS_next of this chunk
-      const int i = idx / VB, j = idx % VB;
-      w.dS[((size_t)c * DK + i) * DV + j0 + j] = dSS[i * LDB + j];
+    for (int idx = tid; idx < C * DV; idx += NTF) {
+      const int r = idx / DV, j = idx % DV;
+      dOS[r * LDV + j] =
+          r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j) : 0.f;
     }
-    for (int i = tid; i < DK; i += NTH) gC[i] = GS[(C - 1) * LDK + i];
+    if (tid < C) bS[tid] = tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+    for (int idx = tid; idx < DK * DV; idx += NTF) {  // dL/dS_next of this chunk
+      const int i = idx / DV, j = idx % DV;
+      w.dS[(size_t)c * DK * DV + idx] = dSS[i * LDV + j];
+    }
     __syncthreads();
-    for (int idx = tid; idx < C * DK; idx += NTH) {  // Qg, Ka, Kc
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LDK + i];
+        GS[r * LDK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+    }
+    for (int idx = tid; idx < C * C; idx += NTF) {
+      const int r = idx / C, s2 = idx % C;
+      const size_t o = ((size_t)c * C + r) * C + s2;
+      AqS[r * LDC + s2] = w.Aqk[o];
+      TS[r * LDC + s2] = w.X[o] * bS[s2];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += NTF) {  // Qg, Ka, Kc
       const int r = idx / DK, i = idx % DK;
       const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LDK + i];
       qS[r * LDK + i] *= e;
@@ -417,46 +434,48 @@ __global__ void __launch_bounds__(NTH, 2)
     }
     __syncthreads();
     {  // dU = A_qk^T dO' + Kc dS
-      float acc[2][2];
+      float acc[1][DV / 16];
       zero(acc);
-      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
-                         [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
-      mm<C, VB, 2, 2, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
-                          [&](int kk, int nn) { return dSS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) { dUS[m * LDB + nn] = acc[i][j]; });
+      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
+                               [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
+      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
+                                [&](int kk, int nn) { return dSS[kk * LDV + nn]; });
+      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { dUS[m * LDV + nn] = acc[i][j]; });
     }
     __syncthreads();
-    {  // W = T^T dU
-      float acc[2][2];
+    {  // W = T^T dU  (= dv)
+      float acc[1][DV / 16];
       zero(acc);
-      mm<C, VB, 2, 2, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
-                         [&](int kk, int nn) { return dUS[kk * LDB + nn]; });
-      for_tile<C, VB, 2, 2>([&](int m, int nn, int i, int j) {
-        WS[m * LDB + nn] = acc[i][j];
-        if (m < n) dv[(rowbase + (size_t)m * H) * DV + j0 + nn] = acc[i][j];
+      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
+                               [&](int kk, int nn) { return dUS[kk * LDV + nn]; });
+      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) {
+        WS[m * LDV + nn] = acc[i][j];
+        if (m < n) dv[(rowbase + (size_t)m * H) * DV + nn] = acc[i][j];
       });
     }
     __syncthreads();
-    store_tile(w.dU, c, DV, j0, dUS);
-    store_tile(w.W, c, DV, j0, WS);
+    for (int idx = tid; idx < C * DV; idx += NTF) {
+      const int r = idx / DV, j = idx % DV;
+      w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
+      w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
+    }
     {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
-      constexpr int TM = DK / 32;
-      float acc[TM][4];
+      float acc[DK / 32][DV / 16];
       zero(acc);
-      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
-                           [&](int kk, int nn) { return dOS[kk * LDB + nn]; });
-      mm<DK, VB, TM, 4, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
-                           [&](int kk, int nn) { return WS[kk * LDB + nn]; });
-      for_tile<DK, VB, TM, 4>([&](int m, int nn, int i, int j) {
-        dSS[m * LDB + nn] = fmaf(expf(gC[m]), dSS[m * LDB + nn], acc[i][j]);
+      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
+                                      [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
+      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
+                                      [&](int kk, int nn) { return WS[kk * LDV + nn]; });
+      for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
+        dSS[m * LDV + nn] = fmaf(eC[m], dSS[m * LDV + nn], acc[i][j]);
       });
     }
   }
   __syncthreads();
   if (dinit) {
-    for (int idx = tid; idx < DK * VB; idx += NTH) {
-      const int i = idx / VB, j = idx % VB;
-      dinit[((size_t)unit * DK + i) * DV + j0 + j] = dSS[i * LDB + j];
+    for (int idx = tid; idx < DK * DV; idx += NTF) {
+      const int i = idx / DV, j = idx % DV;
+      dinit[(size_t)unit * DK * DV + idx] = dSS[i * LDV + j];
     }
   }
 }
@@ -544,21 +563,31 @@ __global__ void __launch_bounds__(NTH, 2)
   zero(aT);
   for (int j0 = 0; j0 < DV; j0 += VBB) {
     __syncthreads();
-    for (int idx = tid; idx < DK * VBB; idx += NTH) {
-      const int i = idx / VBB, j = idx % VBB;
+    // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
+    auto put4 = [](float* dst, float4 x) {
+      dst[0] = x.x;
+      dst[1] = x.y;
+      dst[2] = x.z;
+      dst[3] = x.w;
+    };
+    for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
+      const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
       const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
-      SS[i * LDBB + j] = w.S[o];
-      dSS[i * LDBB + j] = w.dS[o];
+      put4(SS + i * LDBB + j, *reinterpret_cast<const float4*>(w.S + o));
+      put4(dSS + i * LDBB + j, *reinterpret_cast<const float4*>(w.dS + o));
+    }
+    for (int idx = tid; idx < C * VBB / 4; idx += NTH) {
+      const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+      const size_t o = ((size_t)c * C + r) * DV + j0 + j;
+      put4(RS + r * LDBB + j, *reinterpret_cast<const float4*>(w.R + o));
+      put4(US + r * LDBB + j, *reinterpret_cast<const float4*>(w.U + o));
+      put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
+      put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
     }
     for (int idx = tid; idx < C * VBB; idx += NTH) {
       const int r = idx / VBB, j = idx % VBB;
-      const size_t o = ((size_t)c * C + r) * DV + j0 + j;
       dOS[r * LDBB + j] =
           r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
-      RS[r * LDBB + j] = w.R[o];
-      US[r * LDBB + j] = w.U[o];
-      dUS[r * LDBB + j] = w.dU[o];
-      WS[r * LDBB + j] = w.W[o];
     }
     __syncthreads();
     for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
@@ -712,54 +741,49 @@ __global__ void __launch_bounds__(NTH, 2)
   }
 }
 
+// F (when there are chunks) and A, one CTA per unit each
 template <typename Tin, int DK, int DV>
-cudaError_t launch_fwd_scan(const BwdArgs& a, cudaStream_t st) {
-  const size_t smF = FSmem<DK, DV>::bytes;
+cudaError_t launch_scans(const BwdArgs& a, cudaStream_t st) {
+  const size_t smF = FSmem<DK, DV>::bytes, smA = ASmem<DK, DV>::bytes;
   cudaError_t e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
   if (e != cudaSuccess) return e;
-  bwd_fwd_scan<Tin, DK, DV><<<a.B * a.H, NTF, smF, st>>>(
-      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-      a.g, a.beta, a.init, a.T, a.H, a.ws);
+  e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK, DV>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
+  if (e != cudaSuccess) return e;
+  const Tin* q = static_cast<const Tin*>(a.q);
+  const Tin* k = static_cast<const Tin*>(a.k);
+  if (a.T > 0) {
+    bwd_fwd_scan<Tin, DK, DV><<<a.B * a.H, NTF, smF, st>>>(
+        q, k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, a.T, a.H, a.ws);
+    if ((e = cudaGetLastError())) return e;
+  }
+  bwd_state_grad_scan<Tin, DK, DV><<<a.B * a.H, NTF, smA, st>>>(
+      q, k, a.g, a.beta, static_cast<const Tin*>(a.dout), a.dfinal, a.T, a.H, a.scale, a.dv,
+      a.dinit, a.ws);
   return cudaGetLastError();
 }
 
 template <typename Tin, int DK>
 cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
-  constexpr int LDK = DK + 1;
   const int nc = (a.T + C - 1) / C;
-  const int units = a.B * a.H, nblk = a.dv_dim / VB;
-  const size_t smA = sizeof(float) * (3 * C * LDK + DK * LDB + 3 * C * LDB + 2 * C * LDC + C + DK);
   const size_t smB = BSmem<DK>::bytes;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA)))
-    return e;
+  switch (a.dv_dim) {
+    case 32: e = launch_scans<Tin, DK, 32>(a, st); break;
+    case 64: e = launch_scans<Tin, DK, 64>(a, st); break;
+    case 128: e = launch_scans<Tin, DK, 128>(a, st); break;
+    default: e = cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess || nc == 0) return e;
   if ((e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB)))
     return e;
-  const Tin* q = static_cast<const Tin*>(a.q);
-  const Tin* k = static_cast<const Tin*>(a.k);
-  const Tin* dout = static_cast<const Tin*>(a.dout);
-  if (nc > 0) {
-    switch (a.dv_dim) {
-      case 32: e = launch_fwd_scan<Tin, DK, 32>(a, st); break;
-      case 64: e = launch_fwd_scan<Tin, DK, 64>(a, st); break;
-      case 128: e = launch_fwd_scan<Tin, DK, 128>(a, st); break;
-      default: e = cudaErrorInvalidValue;
-    }
-    if (e != cudaSuccess) return e;
-  }
-  bwd_state_grad_scan<Tin, DK><<<units * nblk, NTH, smA, st>>>(
-      q, k, a.g, a.beta, dout, a.dfinal, a.T, a.H, a.dv_dim, a.scale, a.dv, a.dinit, a.ws);
-  if ((e = cudaGetLastError())) return e;
-  if (nc > 0) {
-    bwd_chunk_grads<Tin, DK><<<units * nc, NTH, smB, st>>>(q, k, a.g, a.beta, dout, a.T, a.H,
-                                                           a.dv_dim, a.scale, a.dq, a.dk, a.dg,
-                                                           a.dbeta, a.ws);
-    if ((e = cudaGetLastError())) return e;
-  }
-  return cudaSuccess;
+  bwd_chunk_grads<Tin, DK><<<a.B * a.H * nc, NTH, smB, st>>>(
+      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
+      static_cast<const Tin*>(a.dout), a.T, a.H, a.dv_dim, a.scale, a.dq, a.dk, a.dg, a.dbeta,
+      a.ws);
+  return cudaGetLastError();
 }
 
 template <typename Tin>
