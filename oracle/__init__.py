@@ -17,6 +17,8 @@ forward(q, k, v, g, beta, ...)
 backward(q, k, v, g, beta, dout, ...)
     Gradients of a loss through that recurrence (reverse-mode chain rule on
     the same steps; the pages give the forward only), dense layout, fp64.
+gate_backward(z, A_log, dg, g_min=-5.0)
+    dz and dA_log from dg through the gate (chain rule of the gate formula).
 
 Every function is pinned by tests/test_oracle_pins.py (closed forms,
 invariants, brute-force product form, special cases).
@@ -40,6 +42,11 @@ def _load():
         lib.kda_oracle_gate.argtypes = [
             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p]
+        lib.kda_oracle_gate_backward.restype = None
+        lib.kda_oracle_gate_backward.argtypes = [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p]
         lib.kda_oracle_forward.restype = ctypes.c_int
         lib.kda_oracle_forward.argtypes = [
             ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
@@ -81,6 +88,22 @@ def gate(z, A_log, g_min: float = -5.0):
     _load().kda_oracle_gate(rows, H, dk, _ptr(z), _ptr(A_log), float(g_min),
                             _ptr(out))
     return out
+
+
+def gate_backward(z, A_log, dg, g_min: float = -5.0):
+    """(dz, dA_log) for the gate g = g_min * sigmoid(exp(A_log[h]) * z), given
+    dg of z's shape [..., H, dk]; fp64."""
+    z = _f64(z)
+    dg = _f64(dg)
+    A_log = _f64(A_log).reshape(-1)
+    H, dk = z.shape[-2], z.shape[-1]
+    assert A_log.shape[0] == H and dg.shape == z.shape
+    rows = int(np.prod(z.shape[:-2])) if z.ndim > 2 else 1
+    dz = np.empty_like(z)
+    dA = np.empty(H)
+    _load().kda_oracle_gate_backward(rows, H, dk, _ptr(z), _ptr(A_log), float(g_min),
+                                     _ptr(dg), _ptr(dz), _ptr(dA))
+    return dz, dA
 
 
 def forward(q, k, v, g, beta, init_state=None, cu_seqlens=None,

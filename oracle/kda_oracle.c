@@ -49,6 +49,29 @@ void kda_oracle_gate(int64_t rows, int H, int dk, const double *z,
   }
 }
 
+/* Gradients of the gate above (chain rule; the pages give the forward only):
+ * with x = e^{A_h} z and s = sigmoid(x), dg/dz = g_min s (1 - s) e^{A_h} and
+ * dg/dA_h = g_min s (1 - s) x, so
+ *   dz = dg g_min s (1 - s) e^{A_h},   dA_log[h] = sum over rows, i of dg g_min s (1 - s) x. */
+void kda_oracle_gate_backward(int64_t rows, int H, int dk, const double *z,
+                              const double *A_log, double g_min, const double *dg,
+                              double *dz, double *dA_log) {
+  for (int h = 0; h < H; ++h) dA_log[h] = 0.0;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int h = 0; h < H; ++h) {
+      const double a = exp(A_log[h]);
+      const int64_t base = (r * H + h) * (int64_t)dk;
+      for (int i = 0; i < dk; ++i) {
+        const double x = a * z[base + i];
+        const double s = 1.0 / (1.0 + exp(-x));
+        const double d = dg[base + i] * g_min * s * (1.0 - s);
+        dz[base + i] = d * a;
+        dA_log[h] += d * x;
+      }
+    }
+  }
+}
+
 /* ----------------------------------------------------------- recurrence */
 
 /* One (sequence, head): tokens t0 .. t0+L-1 of the packed [Ttot, H, *]

@@ -73,3 +73,39 @@ def test_backward_beta_zero_writes_nothing(oracle_mod):
                             init_state=x["S0"], d_final=V)
     np.testing.assert_array_equal(r["dv"], 0.0)
     assert np.abs(r["dbeta"]).max() > 0  # but the loss still depends on beta
+
+
+def test_gate_backward_matches_finite_differences(oracle_mod):
+    """dz and dA_log of L = sum(g * W) against central differences of the
+    (separately pinned) gate oracle, element by element."""
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((3, 2, 4, 5))
+    A_log = rng.uniform(-1.0, 2.0, 4)
+    W = rng.standard_normal(z.shape)
+    dz, dA = oracle_mod.gate_backward(z, A_log, W, g_min=-5.0)
+    loss = lambda zz, aa: float(np.sum(oracle_mod.gate(zz, aa, -5.0) * W))
+    eps = 1e-6
+    fz = np.zeros_like(z)
+    for idx in np.ndindex(*z.shape):
+        zp, zm = z.copy(), z.copy()
+        zp[idx] += eps
+        zm[idx] -= eps
+        fz[idx] = (loss(zp, A_log) - loss(zm, A_log)) / (2 * eps)
+    np.testing.assert_allclose(dz, fz, rtol=1e-6, atol=1e-8)
+    fa = np.zeros_like(A_log)
+    for h in range(A_log.shape[0]):
+        ap, am = A_log.copy(), A_log.copy()
+        ap[h] += eps
+        am[h] -= eps
+        fa[h] = (loss(z, ap) - loss(z, am)) / (2 * eps)
+    np.testing.assert_allclose(dA, fa, rtol=1e-6, atol=1e-8)
+
+
+def test_gate_backward_closed_form_at_zero(oracle_mod):
+    """At z = 0: sigmoid = 1/2, so dz = dg g_min e^{A} / 4 and dA_log = 0."""
+    A_log = np.array([0.3, -0.7])
+    z = np.zeros((2, 2, 3))
+    dg = np.arange(12, dtype=np.float64).reshape(z.shape) - 5.0
+    dz, dA = oracle_mod.gate_backward(z, A_log, dg, g_min=-5.0)
+    np.testing.assert_allclose(dz, dg * -5.0 * np.exp(A_log)[None, :, None] / 4.0, rtol=1e-15)
+    np.testing.assert_array_equal(dA, np.zeros(2))
