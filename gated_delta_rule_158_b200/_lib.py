@@ -35,6 +35,8 @@ _SIGNATURES = {
     "kda_status_string": (ctypes.c_char_p, [_I]),
     "kda_last_cuda_error_string": (ctypes.c_char_p, []),
     "kda_gate_fwd": (_I, [_VP, _VP, _F, _VP, _I64, _I, _I, _VP]),
+    "kda_gate_bwd_workspace_size": (_SZ, [_I]),
+    "kda_gate_bwd": (_I, [_VP, _VP, _F, _VP, _VP, _VP, _I64, _I, _I, _VP, _SZ, _VP]),
     "kda_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "kda_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _I, _I, _I, _I, _I, _I,
                            _F, _I, _VP, _VP, _VP, _SZ, _VP]),
@@ -136,6 +138,21 @@ def kda_gate_fwd(z, A_log, g, g_min=-5.0, stream=None):
     rows = z.numel() // (H * dk) if z.numel() else 0
     _check(lib().kda_gate_fwd(_ptr(z), _ptr(A_log), float(g_min), _ptr(g), rows, H, dk,
                               _stream(stream)), "kda_gate_fwd")
+
+
+def kda_gate_bwd_workspace_size(H) -> int:
+    return int(lib().kda_gate_bwd_workspace_size(H))
+
+
+def kda_gate_bwd(z, A_log, dg, dz, dA_log, workspace, g_min=-5.0, stream=None):
+    """dz [..., H, dk] and dA_log [H] from dg through the gate
+    g = g_min * sigmoid(exp(A_log[h]) * z); dz may be dg itself."""
+    H, dk = z.shape[-2], z.shape[-1]
+    rows = z.numel() // (H * dk) if z.numel() else 0
+    _check(lib().kda_gate_bwd(_ptr(z), _ptr(A_log), float(g_min), _ptr(dg), _ptr(dz),
+                              _ptr(dA_log), rows, H, dk, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "kda_gate_bwd")
 
 
 def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs=0, chunk_size=0,

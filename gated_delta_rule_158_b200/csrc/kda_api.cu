@@ -136,6 +136,37 @@ kda_status kda_gate_fwd(const float* z, const float* A_log, float g_min, float* 
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
+size_t kda_gate_bwd_workspace_size(int H) {
+  return H > 0 ? sizeof(float) * (size_t)H * kGateBwdMaxParts : 0;
+}
+
+kda_status kda_gate_bwd(const float* z, const float* A_log, float g_min, const float* dg,
+                        float* dz, float* dA_log, int64_t rows, int H, int dk, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!z || !A_log || !dg || !dz || !dA_log) return KDA_ERR_INVALID_ARG;
+  if (rows < 0 || H <= 0 || dk <= 0) return KDA_ERR_INVALID_ARG;
+  if (!(g_min < 0.f) || !isfinite(g_min)) return KDA_ERR_INVALID_ARG;
+  if (dk < 4 || dk > 1024 || (dk & (dk - 1)) != 0) return KDA_ERR_UNSUPPORTED;
+  if (rows * (int64_t)H > ((int64_t)1 << 40)) return KDA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < kda_gate_bwd_workspace_size(H)) return KDA_ERR_WORKSPACE;
+  const void* ptrs[] = {z, A_log, dg, dz, dA_log, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+  // dz may overwrite dg; nothing else may alias
+  if (dz == z || dz == A_log || (const void*)dA_log == z || (const void*)dA_log == dg ||
+      dA_log == dz || workspace == z || workspace == dg || workspace == dz ||
+      workspace == dA_log)
+    return KDA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 0) {
+    cudaError_t em = cudaMemsetAsync(dA_log, 0, sizeof(float) * (size_t)H, st);
+    return em == cudaSuccess ? KDA_OK : cuda_failure(em);
+  }
+  cudaError_t e = launch_gate_bwd(z, A_log, g_min, dg, dz, dA_log, rows, H, dk,
+                                  static_cast<float*>(workspace), st);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
+}
+
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
                                     int chunk_size, kda_dtype in_dtype) {
   size_t bytes = kStatusBytes;

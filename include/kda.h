@@ -84,6 +84,25 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
                                     kda_dtype in_dtype);
 
 /*
+ * Gate backward: the chain rule of kda_gate_fwd's formula (the pages give
+ * the forward only).  With x = exp(A_log[h]) z and s = Sigmoid(x):
+ *   dz[r, h, i]  = dg[r, h, i] g_min s (1 - s) exp(A_log[h])
+ *   dA_log[h]    = sum over r, i of dg[r, h, i] g_min s (1 - s) x
+ * so a caller of kda_recurrent_bwd with a gated g gets dz and dA_log from
+ * its dg.  z, dg, dz : fp32 [rows, H, dk];  A_log, dA_log : fp32 [H].
+ * dz may equal dg (in place); no other aliasing.  dA_log is summed in a fixed
+ * order (deterministic), through a workspace of
+ * kda_gate_bwd_workspace_size(H) bytes.  Supported: dk a power of two in
+ * [4, 1024].
+ */
+KDA_API size_t kda_gate_bwd_workspace_size(int H);
+
+KDA_API kda_status kda_gate_bwd(const float *z, const float *A_log, float g_min,
+                                const float *dg, float *dz, float *dA_log, int64_t rows,
+                                int H, int dk, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
  * Chunkwise prefill / training forward of the recurrence above.
  *
  * Within chunks of chunk_size tokens the recurrence is evaluated in its

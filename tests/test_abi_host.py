@@ -247,3 +247,24 @@ def test_host_stream_entry_rejects_on_host(L):
     assert L.kda_chunk_fwd_gated_host(*args(ws=ptr(16) + 16)) == kda.KDA_ERR_MISALIGNED
     assert L.kda_chunk_fwd_gated_host(*args(wsb=n - 1)) == kda.KDA_ERR_WORKSPACE
     assert L.kda_chunk_fwd_gated_host(*args(out=ptr(2))) == kda.KDA_ERR_INVALID_ARG  # aliases v
+
+
+def test_gate_backward_rejects_on_host(L):
+    ptr = lambda i: FAKE + 0x1000 * i
+    n = L.kda_gate_bwd_workspace_size(4)
+    assert n == 4 * 256 * 4 and L.kda_gate_bwd_workspace_size(0) == 0
+
+    def args(**over):
+        a = dict(z=ptr(0), A_log=ptr(1), g_min=-5.0, dg=ptr(2), dz=ptr(3), dA=ptr(4), rows=10,
+                 H=4, dk=64, ws=ptr(5), wsb=n, stream=None)
+        a.update(over)
+        return list(a.values())
+
+    assert L.kda_gate_bwd(*args(dg=None)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_gate_bwd(*args(g_min=1.0)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_gate_bwd(*args(dk=96)) == kda.KDA_ERR_UNSUPPORTED      # not a power of two
+    assert L.kda_gate_bwd(*args(dk=2048)) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_gate_bwd(*args(wsb=n - 4)) == kda.KDA_ERR_WORKSPACE
+    assert L.kda_gate_bwd(*args(dz=ptr(3) + 8)) == kda.KDA_ERR_MISALIGNED
+    assert L.kda_gate_bwd(*args(dz=ptr(0))) == kda.KDA_ERR_INVALID_ARG   # dz aliases z
+    assert L.kda_gate_bwd(*args(dA=ptr(3))) == kda.KDA_ERR_INVALID_ARG   # dA_log aliases dz

@@ -167,3 +167,57 @@ def test_backward_strong_decay_takes_exact_exponents(oracle_mod):
     for n in NAMES:
         assert rel_l2(got[n], ref[n]) <= TOL_F32, (n, rel_l2(got[n], ref[n]))
     assert rel_l2(got["d_init"], ref["dS0"]) <= TOL_F32
+
+
+def gpu_gate_bwd(z, A_log, dg, g_min=-5.0, in_place=False):
+    H = z.shape[-2]
+    dz = dg.clone() if in_place else torch.full_like(z, float("nan"))
+    src = dz if in_place else dg
+    dA = torch.full((H,), float("nan"), device=DEV)
+    ws = torch.empty(kda.kda_gate_bwd_workspace_size(H), dtype=torch.uint8, device=DEV)
+    kda.kda_gate_bwd(z, A_log, src, dz, dA, ws, g_min=g_min)
+    torch.cuda.synchronize()
+    return dz, dA
+
+
+@pytest.mark.parametrize("shape,g_min,in_place", [((2, 77, 5, 64), -5.0, False),
+                                                  ((1, 1, 3, 32), -5.0, False),
+                                                  ((3, 40, 2, 128), -40.0, True),
+                                                  ((8, 4096, 32, 128), -5.0, False)])
+def test_gate_backward_parity(oracle_mod, shape, g_min, in_place):
+    """dz elementwise and dA_log per head against the fp64 gate backward: the
+    fp32 bar (relative L2 1e-5)."""
+    inp = W.make_prefill_inputs(shape[0], shape[1], shape[2], shape[3], 32, torch.float32,
+                                seed=shape[1], device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(77)
+    dg = torch.randn(inp["z"].shape, generator=gen, device=DEV)
+    dz, dA = gpu_gate_bwd(inp["z"], inp["A_log"], dg, g_min, in_place)
+    rz, rA = oracle_mod.gate_backward(to64(inp["z"]), to64(inp["A_log"]), to64(dg), g_min)
+    assert rel_l2(to64(dz), rz) <= TOL_F32
+    # dA_log is a sum of rows * dk signed terms: bound its error by the fp32 bar
+    # times the sum of the terms' magnitudes (the scale summation error has)
+    x = np.exp(to64(inp["A_log"]))[None, None, :, None] * to64(inp["z"])
+    sg = 1.0 / (1.0 + np.exp(-x))
+    terms = np.abs(to64(dg) * g_min * sg * (1.0 - sg) * x)
+    scale = terms.sum(axis=(0, 1, 3))
+    assert (np.abs(to64(dA) - rA) <= TOL_F32 * scale).all()
+    dz2, dA2 = gpu_gate_bwd(inp["z"], inp["A_log"], dg, g_min, in_place)
+    assert torch.equal(dz, dz2) and torch.equal(dA, dA2)  # fixed summation order
+
+
+def test_gated_training_backward_chain(oracle_mod):
+    """The gated model's input gradients: kda_recurrent_bwd gives dg, the gate
+    backward turns it into dz and dA_log; the oracle does the same chain in
+    fp64 on its own gate.  All at the fp32 bar."""
+    B, T, H, dk, dv = 2, 90, 3, 64, 64
+    inp = W.make_prefill_inputs(B, T, H, dk, dv, torch.bfloat16, seed=41, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, dv, dk=dk, seed=42, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    got = gpu_backward(inp, cot, g, 1.0, True, True)
+    dz, dA = gpu_gate_bwd(inp["z"], inp["A_log"],
+                          torch.from_numpy(got["dg"]).float().to(DEV))
+    ref = oracle_backward(oracle_mod, inp, cot, 1.0, True, True)
+    rz, rA = oracle_mod.gate_backward(to64(inp["z"]), to64(inp["A_log"]), ref["dg"], -5.0)
+    assert rel_l2(to64(dz), rz) <= TOL_F32
+    assert rel_l2(to64(dA), rA) <= TOL_F32
