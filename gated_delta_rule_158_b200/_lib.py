@@ -57,9 +57,9 @@ _SIGNATURES = {
     "kda_chunk_fwd_gated_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "kda_chunk_fwd_gated_host": (_I, [_VP, _VP, _VP, _VP, _VP, _F, _VP, _I, _VP, _I, _I, _I, _I,
                                       _I, _F, _VP, _VP, _VP, _SZ, _VP, _VP]),
-    "kda_recurrent_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
-    "kda_recurrent_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F,
-                               _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "kda_recurrent_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "kda_recurrent_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _I,
+                               _I, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
@@ -288,24 +288,25 @@ def kda_chunk_fwd_gated_host(q, k, v, z, A_log, beta, out, workspace, g_min=-5.0
         None if copy_stream is None else _stream(copy_stream)), "kda_chunk_fwd_gated_host")
 
 
-def kda_recurrent_bwd_workspace_size(B, T, H, dk, dv) -> int:
-    return int(lib().kda_recurrent_bwd_workspace_size(B, T, H, dk, dv))
+def kda_recurrent_bwd_workspace_size(B, T, H, dk, dv, num_seqs=0) -> int:
+    return int(lib().kda_recurrent_bwd_workspace_size(B, T, H, dk, dv, num_seqs))
 
 
 def kda_recurrent_bwd(q, k, v, g, beta, dout, grads, workspace, init_state=None, d_final=None,
-                      scale=1.0, stream=None):
+                      cu_seqlens=None, scale=1.0, stream=None):
     """Gradients through the recurrence.  q, k, g [B,T,H,dk]; v, dout
-    [B,T,H,dv]; beta [B,T,H].  `grads` is a dict of fp32 output tensors
-    dq, dk, dg [B,T,H,dk], dv [B,T,H,dv], dbeta [B,T,H] and optionally
-    d_init [B,H,dk,dv]."""
+    [B,T,H,dv]; beta [B,T,H]; cu_seqlens (int32 [N+1], B == 1) for a packed
+    batch.  `grads` is a dict of fp32 output tensors dq, dk, dg [B,T,H,dk],
+    dv [B,T,H,dv], dbeta [B,T,H] and optionally d_init [N,H,dk,dv]."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    N = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     _check(lib().kda_recurrent_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _dtype(q), _ptr(init_state), _ptr(dout),
-        _ptr(d_final), B, T, H, dk, dv, float(scale), _ptr(grads["dq"]), _ptr(grads["dk"]),
-        _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["dbeta"]), _ptr(grads.get("d_init")),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
-        "kda_recurrent_bwd")
+        _ptr(d_final), _ptr(cu_seqlens), N, B, T, H, dk, dv, float(scale), _ptr(grads["dq"]),
+        _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["dbeta"]),
+        _ptr(grads.get("d_init")), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "kda_recurrent_bwd")
 
 
 def kda_get_device_status(workspace, stream=None):

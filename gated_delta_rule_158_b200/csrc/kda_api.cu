@@ -449,32 +449,39 @@ kda_status kda_decode_replay(const void* k, const void* v, const float* g, const
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
-size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
-  if (B <= 0 || T < 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
-  return bwd_chunk_workspace_bytes(B, T, H, dk, dv);
+size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {
+  if (B <= 0 || T < 0 || H <= 0 || num_seqs < 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+  if (num_seqs > 0 && B != 1) return 0;
+  return bwd_chunk_workspace_bytes(B, T, H, dk, dv, num_seqs);
 }
 
 kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
                              const float* beta, kda_dtype in_dtype, const float* init_state,
-                             const void* dout, const float* d_final, int B, int T, int H, int dk,
-                             int dv, float scale, float* dq, float* dk_out, float* dv_out,
-                             float* dg, float* dbeta, float* d_init, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+                             const void* dout, const float* d_final, const int32_t* cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk, int dv, float scale,
+                             float* dq, float* dk_out, float* dv_out, float* dg, float* dbeta,
+                             float* d_init, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   if (in_dtype != KDA_F32 && in_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (B <= 0 || T < 0 || H <= 0 || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens) {
+    if (B != 1 || num_seqs <= 0) return KDA_ERR_INVALID_ARG;
+  } else if (num_seqs != 0) {
+    return KDA_ERR_INVALID_ARG;
+  }
   if (T > 0 && (!q || !k || !v || !g || !beta || !dout || !dq || !dk_out || !dv_out || !dg ||
                 !dbeta))
     return KDA_ERR_INVALID_ARG;
-  if ((int64_t)B * H > 0x7fffffffLL || (int64_t)B * T * H > 0x7fffffffLL)
-    return KDA_ERR_UNSUPPORTED;
+  const int64_t nseq = cu_seqlens ? num_seqs : B;
+  if (nseq * H > 0x7fffffffLL || (int64_t)B * T * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
   if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-  const size_t need = bwd_chunk_workspace_bytes(B, T, H, dk, dv);  // 0 when T = 0
-  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-  const void* ptrs[] = {q, k, v, g, beta, init_state, dout, d_final, dq, dk_out, dv_out, dg,
-                        dbeta, d_init, workspace};
+  const size_t need = bwd_chunk_workspace_bytes(B, T, H, dk, dv, cu_seqlens ? num_seqs : 0);
+  if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+  const void* ptrs[] = {q, k, v, g, beta, init_state, dout, d_final, cu_seqlens, dq, dk_out,
+                        dv_out, dg, dbeta, d_init, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
-  const void* ins[] = {q, k, v, g, beta, init_state, dout, d_final, workspace};
+  const void* ins[] = {q, k, v, g, beta, init_state, dout, d_final, cu_seqlens, workspace};
   const void* outs[] = {dq, dk_out, dv_out, dg, dbeta, d_init};
   for (const void* o : outs) {
     if (!o) continue;
@@ -482,9 +489,31 @@ kda_status kda_recurrent_bwd(const void* q, const void* k, const void* v, const 
       if (i == o) return KDA_ERR_INVALID_ARG;
   }
   if (T == 0 && !d_init) return KDA_OK;
-  BwdArgs a{q,  k,  v,     g,     beta,   init_state, dout,   d_final, in_dtype, B,
-            T,  H,  dk,    dv,    scale,  dq,         dk_out, dv_out,  dg,       dbeta,
-            d_init, static_cast<float*>(workspace)};
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.init = init_state;
+  a.dout = dout;
+  a.dfinal = d_final;
+  a.cu_seqlens = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.dt = in_dtype;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.dk_dim = dk;
+  a.dv_dim = dv;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk_out;
+  a.dv = dv_out;
+  a.dg = dg;
+  a.dbeta = dbeta;
+  a.dinit = d_init;
+  a.ws = workspace;
   const cudaError_t e = launch_bwd_chunk(a, (cudaStream_t)stream);
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }

@@ -95,9 +95,46 @@ __host__ __device__ inline size_t unit_ws_floats(int nc, int DK, int DV) {
   return (size_t)nc * (2 * (size_t)DK * DV + 3 * C * C + 4 * (size_t)C * DV);
 }
 
-__device__ inline UnitWs unit_ws(float* ws, int unit, int nc, int DK, int DV) {
+// Where a (sequence, head) unit's tokens and workspace are.  Dense batches:
+// sequence n is rows [n T, n T + T).  Packed (varlen) batches: rows
+// [cu[n], cu[n+1]), and the chunks of sequence n start at chunk coff[n] of the
+// workspace (coff = prefix sums of the sequences' chunk counts, written by the
+// plan kernel), its H units' chunks one after another.
+struct SeqMap {
+  const int32_t* cu;     // nullptr = dense
+  const int32_t* coff;   // varlen: chunk offsets [N + 1]
+  const StatusBlock* sb; // varlen: validity verdict of the plan kernel
+  int T, H;
+};
+
+struct UnitPos {
+  int64_t row0;    // first row of the sequence
+  int len;         // its tokens
+  int nc;          // its chunks
+  int64_t chunk0;  // the unit's first chunk in the workspace
+};
+
+__device__ inline UnitPos unit_pos(const SeqMap& m, int n, int h) {
+  UnitPos p;
+  if (m.cu == nullptr) {
+    p.row0 = (int64_t)n * m.T;
+    p.len = m.T;
+    p.nc = (m.T + C - 1) / C;
+    p.chunk0 = ((int64_t)n * m.H + h) * p.nc;
+  } else {
+    p.row0 = m.cu[n];
+    p.len = m.cu[n + 1] - m.cu[n];
+    p.nc = (p.len + C - 1) / C;
+    p.chunk0 = (int64_t)m.coff[n] * m.H + (int64_t)h * p.nc;
+  }
+  return p;
+}
+
+__device__ inline bool seqs_ok(const SeqMap& m) { return m.cu == nullptr || m.sb->seqlens_ok == 1; }
+
+__device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int DV) {
   UnitWs w;
-  float* base = ws + (size_t)unit * unit_ws_floats(nc, DK, DV);
+  float* base = ws + (size_t)chunk0 * unit_ws_floats(1, DK, DV);
   w.S = base;
   w.dS = w.S + (size_t)nc * DK * DV;
   w.X = w.dS + (size_t)nc * DK * DV;
@@ -141,6 +178,53 @@ __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const floa
   __syncthreads();
 }
 
+// ================================================================ varlen plan
+// Validates cu_seqlens (0 at the start, T at the end, non-decreasing) and
+// writes the chunk offsets coff[n] = sum over m < n of ceil(len_m / C).  One
+// CTA; thread t sums a contiguous run of sequences, then a sequential scan of
+// the runs.
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads)
+    bwd_varlen_plan(const int32_t* __restrict__ cu, int N, int T, int32_t* __restrict__ coff,
+                    StatusBlock* sb) {
+  __shared__ int bad;
+  __shared__ int32_t run[kPlanThreads];
+  const int tid = threadIdx.x;
+  if (tid == 0) bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
+  __syncthreads();
+  const int per = (N + kPlanThreads - 1) / kPlanThreads;
+  const int n0 = tid * per, n1 = min(N, n0 + per);
+  int32_t local = 0;
+  for (int n = n0; n < n1; ++n) {
+    const int32_t len = cu[n + 1] - cu[n];
+    if (len < 0) atomicOr(&bad, 1);
+    local += len > 0 ? (len + C - 1) / C : 0;
+  }
+  run[tid] = local;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int t = 0; t < kPlanThreads; ++t) {
+      const int32_t x = run[t];
+      run[t] = acc;
+      acc += x;
+    }
+    coff[N] = acc;
+  }
+  __syncthreads();
+  int32_t acc = run[tid];
+  for (int n = n0; n < n1; ++n) {
+    coff[n] = acc;
+    const int32_t len = cu[n + 1] - cu[n];
+    acc += len > 0 ? (len + C - 1) / C : 0;
+  }
+  if (tid == 0) {
+    sb->seqlens_ok = bad ? 0 : 1;
+    if (bad) record_status(sb, KDA_ERR_BAD_SEQLENS, 0);
+  }
+}
+
 // ===================================================================== pass F
 // One CTA of 512 threads per unit, all dv columns, so the key-side matrices
 // are formed once per chunk.  The Gram matrices are one product each when
@@ -163,7 +247,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NTF, 1)
     bwd_fwd_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                  const Tin* __restrict__ v, const float* __restrict__ g,
-                 const float* __restrict__ beta, const float* __restrict__ init, int T, int H,
+                 const float* __restrict__ beta, const float* __restrict__ init, SeqMap map,
                  float* __restrict__ ws) {
   constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
@@ -182,10 +266,13 @@ __global__ void __launch_bounds__(NTF, 1)
   float* gC = bS + C;             // [DK] Gamma_C
   float* eC = gC + DK;            // [DK] e^{Gamma_C}
 
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
   const int unit = blockIdx.x;
-  const int b = unit / H, h = unit % H;
-  const int nc = (T + C - 1) / C;
-  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  const int nc = up.nc;
+  const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
   const int tid = threadIdx.x;
 
   for (int idx = tid; idx < DK * DV; idx += NTF) {
@@ -193,8 +280,8 @@ __global__ void __launch_bounds__(NTF, 1)
     SS[i * LDV + j] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
   }
   for (int c = 0; c < nc; ++c) {
-    const int t0 = c * C, n = min(C, T - t0);
-    const size_t rowbase = ((size_t)b * T + t0) * H + h;
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {
       const int r = idx / DK, i = idx % DK;
@@ -353,9 +440,9 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NTF, 1)
     bwd_state_grad_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         const float* __restrict__ g, const float* __restrict__ beta,
-                        const Tin* __restrict__ dout, const float* __restrict__ dfinal, int T,
-                        int H, float scale, float* __restrict__ dv, float* __restrict__ dinit,
-                        float* __restrict__ ws) {
+                        const Tin* __restrict__ dout, const float* __restrict__ dfinal,
+                        SeqMap map, float scale, float* __restrict__ dv,
+                        float* __restrict__ dinit, float* __restrict__ ws) {
   constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
   float* qS = sm;                 // [C][LDK]  q, later Qg
@@ -371,10 +458,13 @@ __global__ void __launch_bounds__(NTF, 1)
   float* gC = bS + C;             // [DK]
   float* eC = gC + DK;            // [DK]
 
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
   const int unit = blockIdx.x;
-  const int b = unit / H, h = unit % H;
-  const int nc = (T + C - 1) / C;
-  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  const int nc = up.nc;
+  const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
   const int tid = threadIdx.x;
 
   for (int idx = tid; idx < DK * DV; idx += NTF) {
@@ -382,8 +472,8 @@ __global__ void __launch_bounds__(NTF, 1)
     dSS[i * LDV + j] = dfinal ? dfinal[(size_t)unit * DK * DV + idx] : 0.f;
   }
   for (int c = nc - 1; c >= 0; --c) {
-    const int t0 = c * C, n = min(C, T - t0);
-    const size_t rowbase = ((size_t)b * T + t0) * H + h;
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {
       const int r = idx / DK, i = idx % DK;
@@ -505,7 +595,7 @@ template <typename Tin, int DK>
 __global__ void __launch_bounds__(NTH, 2)
     bwd_chunk_grads(const Tin* __restrict__ q, const Tin* __restrict__ k,
                     const float* __restrict__ g, const float* __restrict__ beta,
-                    const Tin* __restrict__ dout, int T, int H, int DV, float scale,
+                    const Tin* __restrict__ dout, SeqMap map, int N, int DV, float scale,
                     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dg,
                     float* __restrict__ dbeta, float* __restrict__ ws) {
   constexpr int LDK = DK + 1;
@@ -531,12 +621,29 @@ __global__ void __launch_bounds__(NTH, 2)
   float* rsum = gC + DK;          // [DK] sum_j dS_ij S_ij
   float* kcsum = rsum + DK;       // [DK] sum_r dKc_ri Kc_ri
 
-  const int nc = (T + C - 1) / C;
-  const int unit = blockIdx.x / nc, c = blockIdx.x % nc;
-  const int b = unit / H, h = unit % H;
-  const int t0 = c * C, n = min(C, T - t0);
-  const size_t rowbase = ((size_t)b * T + t0) * H + h;
-  const UnitWs w = unit_ws(ws, unit, nc, DK, DV);
+  // block = (global chunk, head): dense chunk cg is chunk cg % nc of sequence
+  // cg / nc; packed, the sequence whose chunk range holds cg (binary search)
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  const int64_t cg = blockIdx.x / H;
+  const int h = blockIdx.x % H;
+  int seq;
+  if (map.cu == nullptr) {
+    seq = (int)(cg / ((map.T + C - 1) / C));
+  } else {
+    if (cg >= map.coff[N]) return;
+    int lo = 0, hi = N;  // coff[lo] <= cg < coff[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (map.coff[mid] <= cg) lo = mid; else hi = mid;
+    }
+    seq = lo;
+  }
+  const UnitPos up = unit_pos(map, seq, h);
+  const int c = (int)(cg - (map.cu == nullptr ? (int64_t)seq * up.nc : (int64_t)map.coff[seq]));
+  const int t0 = c * C, n = min(C, up.len - t0);
+  const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+  const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
   const int tid = threadIdx.x;
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
@@ -741,9 +848,10 @@ __global__ void __launch_bounds__(NTH, 2)
   }
 }
 
-// F (when there are chunks) and A, one CTA per unit each
+// F and A, one CTA per unit each
 template <typename Tin, int DK, int DV>
-cudaError_t launch_scans(const BwdArgs& a, cudaStream_t st) {
+cudaError_t launch_scans(const BwdArgs& a, const SeqMap& map, int units, float* ws,
+                         cudaStream_t st) {
   const size_t smF = FSmem<DK, DV>::bytes, smA = ASmem<DK, DV>::bytes;
   cudaError_t e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
@@ -754,35 +862,61 @@ cudaError_t launch_scans(const BwdArgs& a, cudaStream_t st) {
   const Tin* q = static_cast<const Tin*>(a.q);
   const Tin* k = static_cast<const Tin*>(a.k);
   if (a.T > 0) {
-    bwd_fwd_scan<Tin, DK, DV><<<a.B * a.H, NTF, smF, st>>>(
-        q, k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, a.T, a.H, a.ws);
+    bwd_fwd_scan<Tin, DK, DV><<<units, NTF, smF, st>>>(
+        q, k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, map, ws);
     if ((e = cudaGetLastError())) return e;
   }
-  bwd_state_grad_scan<Tin, DK, DV><<<a.B * a.H, NTF, smA, st>>>(
-      q, k, a.g, a.beta, static_cast<const Tin*>(a.dout), a.dfinal, a.T, a.H, a.scale, a.dv,
-      a.dinit, a.ws);
+  bwd_state_grad_scan<Tin, DK, DV><<<units, NTF, smA, st>>>(
+      q, k, a.g, a.beta, static_cast<const Tin*>(a.dout), a.dfinal, map, a.scale, a.dv,
+      a.dinit, ws);
   return cudaGetLastError();
+}
+
+struct WsLayout {
+  size_t coff_off, data_off, total;
+  int64_t max_chunks;  // per head
+};
+
+WsLayout ws_layout(int B, int T, int H, int dk, int dv, int num_seqs) {
+  WsLayout L;
+  const int64_t nc = ((int64_t)T + C - 1) / C;
+  L.coff_off = kStatusBytes;
+  L.data_off = kStatusBytes + (num_seqs > 0 ? (sizeof(int32_t) * (size_t)(num_seqs + 1) + 255) / 256 * 256 : 0);
+  L.max_chunks = num_seqs > 0 ? nc + num_seqs : (int64_t)B * nc;
+  L.total = L.data_off + (size_t)H * L.max_chunks * unit_ws_floats(1, dk, dv) * sizeof(float);
+  return L;
 }
 
 template <typename Tin, int DK>
 cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
-  const int nc = (a.T + C - 1) / C;
-  const size_t smB = BSmem<DK>::bytes;
-  cudaError_t e;
+  const WsLayout lay = ws_layout(a.B, a.T, a.H, DK, a.dv_dim, a.cu_seqlens ? a.num_seqs : 0);
+  char* base = static_cast<char*>(a.ws);
+  StatusBlock* sb = reinterpret_cast<StatusBlock*>(base);
+  int32_t* coff = reinterpret_cast<int32_t*>(base + lay.coff_off);
+  float* ws = reinterpret_cast<float*>(base + lay.data_off);
+  cudaError_t e = cudaMemsetAsync(sb, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return e;
+  SeqMap map{a.cu_seqlens, a.cu_seqlens ? coff : nullptr, sb, a.T, a.H};
+  const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
+  if (a.cu_seqlens) {
+    bwd_varlen_plan<<<1, kPlanThreads, 0, st>>>(a.cu_seqlens, a.num_seqs, a.T, coff, sb);
+    if ((e = cudaGetLastError())) return e;
+  }
   switch (a.dv_dim) {
-    case 32: e = launch_scans<Tin, DK, 32>(a, st); break;
-    case 64: e = launch_scans<Tin, DK, 64>(a, st); break;
-    case 128: e = launch_scans<Tin, DK, 128>(a, st); break;
+    case 32: e = launch_scans<Tin, DK, 32>(a, map, nseq * a.H, ws, st); break;
+    case 64: e = launch_scans<Tin, DK, 64>(a, map, nseq * a.H, ws, st); break;
+    case 128: e = launch_scans<Tin, DK, 128>(a, map, nseq * a.H, ws, st); break;
     default: e = cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess || nc == 0) return e;
+  if (e != cudaSuccess || lay.max_chunks == 0) return e;
+  const size_t smB = BSmem<DK>::bytes;
   if ((e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB)))
     return e;
-  bwd_chunk_grads<Tin, DK><<<a.B * a.H * nc, NTH, smB, st>>>(
+  bwd_chunk_grads<Tin, DK><<<(unsigned)(lay.max_chunks * a.H), NTH, smB, st>>>(
       static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
-      static_cast<const Tin*>(a.dout), a.T, a.H, a.dv_dim, a.scale, a.dq, a.dk, a.dg, a.dbeta,
-      a.ws);
+      static_cast<const Tin*>(a.dout), map, nseq, a.dv_dim, a.scale, a.dq, a.dk, a.dg, a.dbeta,
+      ws);
   return cudaGetLastError();
 }
 
@@ -798,13 +932,12 @@ cudaError_t by_dk(const BwdArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-size_t bwd_chunk_workspace_bytes(int B, int T, int H, int dk, int dv) {
-  const int nc = (T + C - 1) / C;
-  return (size_t)B * H * unit_ws_floats(nc, dk, dv) * sizeof(float);
+size_t bwd_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int num_seqs) {
+  return ws_layout(B, T, H, dk, dv, num_seqs).total;
 }
 
 cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t stream) {
-  if (a.B * a.H == 0) return cudaSuccess;
+  if (a.H == 0 || (a.cu_seqlens ? a.num_seqs : a.B) == 0) return cudaSuccess;
   return a.dt == KDA_BF16 ? by_dk<__nv_bfloat16>(a, stream) : by_dk<float>(a, stream);
 }
 

@@ -313,25 +313,30 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * arithmetic throughout (exponents of the decay taken as differences <= 0,
  * so g must be <= 0, as the gate makes it).
  *  q, k, g : [B, T, H, dk]   v, dout : [B, T, H, dv]   beta : fp32 [B, T, H]
- *  init_state, d_final : fp32 [B, H, dk, dv] or NULL (zeros)
+ *  cu_seqlens, num_seqs : as kda_chunk_fwd (NULL and 0 for a dense batch; a
+ *      packed batch has B == 1; malformed offsets are reported on the device,
+ *      KDA_ERR_BAD_SEQLENS through kda_get_device_status, and nothing is
+ *      written)
+ *  init_state, d_final : fp32 [N, H, dk, dv] or NULL (zeros), N = num_seqs or B
  * Outputs (fp32, written whole; d_init may be NULL to skip it):
  *  dq, dk_out, dg : [B, T, H, dk]   dv_out : [B, T, H, dv]   dbeta : [B, T, H]
- *  d_init : [B, H, dk, dv]  (dL/dS_0)
+ *  d_init : [N, H, dk, dv]  (dL/dS_0)
  * dout has the element type of q, k, v.  g is the log-decay (a gated caller
- * chains dg through its gate).  Dense batches only.  The workspace (size from
- * kda_recurrent_bwd_workspace_size: per (sequence, head) and chunk two
- * dk x dv states, three 32 x 32 matrices and four 32 x dv tiles; 0 for
- * unsupported shapes and for
- * T = 0, when the workspace may be NULL) is scratch; outputs must not alias
- * inputs.
+ * chains dg through its gate: kda_gate_bwd).  The workspace (size from
+ * kda_recurrent_bwd_workspace_size: the 256-byte device status word, the
+ * packed batch's chunk offsets, and per (sequence, head) and 32-token chunk
+ * two dk x dv states, three 32 x 32 matrices and four 32 x dv tiles; 0 for
+ * unsupported shapes) is scratch; outputs must not alias inputs.
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
  */
-KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv,
+                                                int num_seqs);
 
 KDA_API kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v,
                              const float *g, const float *beta, kda_dtype in_dtype,
                              const float *init_state, const void *dout,
-                             const float *d_final, int B, int T, int H, int dk,
+                             const float *d_final, const int32_t *cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk,
                              int dv, float scale, float *dq, float *dk_out,
                              float *dv_out, float *dg, float *dbeta, float *d_init,
                              void *workspace, size_t workspace_bytes, void *stream);

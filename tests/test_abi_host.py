@@ -190,18 +190,22 @@ def test_kcp_entries_reject_on_host(L):
 
 def test_backward_entries_reject_on_host(L):
     ptr = lambda i: FAKE + 0x1000 * i
-    ws = L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128)
-    # per (sequence, head) and 32-token chunk: its start state, the gradient of
-    # its end state (64 KB each), three 32 x 32 key-side matrices and four
-    # 32 x dv intermediates (R, U, dU, W)
-    assert ws == 2 * 4 * (2 * 128 * 128 + 3 * 32 * 32 + 4 * 32 * 128) * 4
-    assert L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128) == 0
-    assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 96, 128) == 0
+    ws = L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128, 0)
+    # the device status word, then per (sequence, head) and 32-token chunk: its
+    # start state, the gradient of its end state (64 KB each), three 32 x 32
+    # key-side matrices and four 32 x dv intermediates (R, U, dU, W)
+    per_chunk = (2 * 128 * 128 + 3 * 32 * 32 + 4 * 32 * 128) * 4
+    assert ws == 256 + 2 * 4 * per_chunk
+    assert L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128, 0) == 256
+    assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 96, 128, 0) == 0
+    # packed: 3 sequences in 100 tokens take at most ceil(100/32) + 3 chunks
+    assert L.kda_recurrent_bwd_workspace_size(1, 100, 2, 128, 128, 3) == 256 + 256 + 2 * 7 * per_chunk
+    assert L.kda_recurrent_bwd_workspace_size(2, 100, 2, 128, 128, 3) == 0  # packed needs B == 1
 
     def args(**over):
         a = dict(q=ptr(0), k=ptr(1), v=ptr(2), g=ptr(3), beta=ptr(4), dt=kda.KDA_BF16,
-                 init=None, dout=ptr(5), dfinal=None, B=1, T=100, H=2, dk=128, dv=128,
-                 scale=1.0, dq=ptr(6), dko=ptr(7), dvo=ptr(8), dg=ptr(9), dbeta=ptr(10),
+                 init=None, dout=ptr(5), dfinal=None, cu=None, nseq=0, B=1, T=100, H=2, dk=128,
+                 dv=128, scale=1.0, dq=ptr(6), dko=ptr(7), dvo=ptr(8), dg=ptr(9), dbeta=ptr(10),
                  dinit=None, ws=ptr(11), wsb=ws, stream=None)
         a.update(over)
         return list(a.values())
@@ -216,8 +220,15 @@ def test_backward_entries_reject_on_host(L):
     assert L.kda_recurrent_bwd(*args(dg=ptr(9) + 4)) == kda.KDA_ERR_MISALIGNED
     assert L.kda_recurrent_bwd(*args(dq=ptr(0))) == kda.KDA_ERR_INVALID_ARG  # dq aliases q
     assert L.kda_recurrent_bwd(*args(dinit=ptr(11))) == kda.KDA_ERR_INVALID_ARG  # aliases ws
+    assert L.kda_recurrent_bwd(*args(cu=ptr(12), nseq=0)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(cu=ptr(12), nseq=3, B=2)) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_recurrent_bwd(*args(nseq=3)) == kda.KDA_ERR_INVALID_ARG  # counts without offsets
+    assert L.kda_recurrent_bwd(*args(cu=ptr(12) + 4, nseq=3, wsb=10 ** 9)) == \
+        kda.KDA_ERR_MISALIGNED
+    # packed workspace is larger than the dense one for the same T
+    assert L.kda_recurrent_bwd(*args(cu=ptr(12), nseq=3)) == kda.KDA_ERR_WORKSPACE
     # empty sequence with no d_init requested: nothing to do, nothing launched
-    ws0 = L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128)
+    ws0 = L.kda_recurrent_bwd_workspace_size(1, 0, 2, 128, 128, 0)
     assert L.kda_recurrent_bwd(*args(T=0, q=None, k=None, v=None, g=None, beta=None, dout=None,
                                      dq=None, dko=None, dvo=None, dg=None, dbeta=None,
                                      wsb=ws0)) == kda.KDA_OK

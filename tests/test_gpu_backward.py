@@ -221,3 +221,68 @@ def test_gated_training_backward_chain(oracle_mod):
     rz, rA = oracle_mod.gate_backward(to64(inp["z"]), to64(inp["A_log"]), ref["dg"], -5.0)
     assert rel_l2(to64(dz), rz) <= TOL_F32
     assert rel_l2(to64(dA), rA) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_varlen_parity(oracle_mod, dtype):
+    """A packed batch (cu_seqlens) with empty, one-token, ragged and
+    whole-chunk sequences: each sequence's gradients and dS0 against the
+    oracle run on that sequence alone; an empty sequence passes d_final
+    through to d_init."""
+    lengths = [0, 1, 31, 32, 33, 100, 64, 7, 0, 45]
+    N, H, dk, dv = len(lengths), 2, 64, 64
+    cu_list = W.cu_seqlens_from_lengths(lengths)
+    T = cu_list[-1]
+    cu = torch.tensor(cu_list, dtype=torch.int32, device=DEV)
+    inp = W.make_prefill_inputs(1, T, H, dk, dv, dtype, seed=51, device=DEV, init_state=True,
+                                num_states=N)
+    cot = W.make_backward_cotangents(1, T, H, dv, dk=None, dtype=dtype, seed=52, device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(53)
+    cot["d_final"] = 0.1 * torch.randn((N, H, dk, dv), generator=gen, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    nan = lambda *s: torch.full(s, float("nan"), device=DEV)
+    grads = dict(dq=nan(1, T, H, dk), dk=nan(1, T, H, dk), dv=nan(1, T, H, dv),
+                 dg=nan(1, T, H, dk), dbeta=nan(1, T, H), d_init=nan(N, H, dk, dv))
+    ws = torch.empty(kda.kda_recurrent_bwd_workspace_size(1, T, H, dk, dv, N), dtype=torch.uint8,
+                     device=DEV)
+    kda.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], cot["dout"], grads, ws,
+                          init_state=inp["init_state"], d_final=cot["d_final"], cu_seqlens=cu)
+    st, _ = kda.kda_get_device_status(ws)
+    assert st == kda.KDA_OK
+    got = {n_: to64(t) for n_, t in grads.items()}
+    g_ref = oracle_mod.gate(to64(inp["z"]), to64(inp["A_log"]), -5.0)
+    for n in range(N):
+        a, b = cu_list[n], cu_list[n + 1]
+        if a == b:
+            assert np.array_equal(got["d_init"][n], to64(cot["d_final"][n]))
+            continue
+        sl = lambda x: np.ascontiguousarray(x[:, a:b])
+        ref = oracle_mod.backward(sl(to64(inp["q"])), sl(to64(inp["k"])), sl(to64(inp["v"])),
+                                  sl(g_ref), sl(to64(inp["beta"])), sl(to64(cot["dout"])),
+                                  init_state=to64(inp["init_state"][n:n + 1]),
+                                  d_final=to64(cot["d_final"][n:n + 1]))
+        for name in NAMES:
+            assert rel_l2(got[name][:, a:b], ref[name]) <= TOL_F32, (n, name)
+        assert rel_l2(got["d_init"][n], ref["dS0"][0]) <= TOL_F32, n
+
+
+def test_backward_varlen_bad_offsets_are_reported():
+    """Offsets that decrease: the plan kernel records KDA_ERR_BAD_SEQLENS and
+    no gradient is written (the outputs keep their NaN fill)."""
+    T, H, d = 64, 2, 32
+    cu = torch.tensor([0, 40, 20, 64], dtype=torch.int32, device=DEV)
+    inp = W.make_prefill_inputs(1, T, H, d, d, torch.float32, seed=61, device=DEV)
+    cot = W.make_backward_cotangents(1, T, H, d, dk=None, dtype=torch.float32, seed=62,
+                                     device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    nan = lambda *s: torch.full(s, float("nan"), device=DEV)
+    grads = dict(dq=nan(1, T, H, d), dk=nan(1, T, H, d), dv=nan(1, T, H, d), dg=nan(1, T, H, d),
+                 dbeta=nan(1, T, H), d_init=nan(3, H, d, d))
+    ws = torch.empty(kda.kda_recurrent_bwd_workspace_size(1, T, H, d, d, 3), dtype=torch.uint8,
+                     device=DEV)
+    kda.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], cot["dout"], grads, ws,
+                          cu_seqlens=cu)
+    st, _ = kda.kda_get_device_status(ws)
+    assert st == kda.KDA_ERR_BAD_SEQLENS
+    for name, t in grads.items():
+        assert bool(torch.isnan(t).all()), name
