@@ -10,10 +10,10 @@
 //   X = (I + Diag(beta) L)^-1,  T = X Diag(beta)
 //   Qg = q e^Gamma,  Ka = k e^Gamma,  Kc = k e^{Gamma_C - Gamma}
 //   U = T (V - Ka S),  S_next = Diag(e^{Gamma_C}) S + Kc^T U,  O = scale (Qg S + A_qk U)
-// Three passes, fp32 throughout:
-//   F  chunk order, one CTA per unit: the key-side matrices (saved once per
-//      chunk: X, A_qk, L), the chunk-start states and R = V - Ka S, U = T R
-//      of every chunk.
+// Four passes, fp32 throughout:
+//   K  every chunk at once: the key-side matrices X, A_qk, L.
+//   F  chunk order, one CTA per unit: the chunk-start states and
+//      R = V - Ka S, U = T R of every chunk.
 //   A  reverse chunk order, same grid: the state gradient dS = dL/dS_next,
 //        dU = A_qk^T dO' + Kc dS,  dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T T^T dU
 //      (dO' = scale dO); needs no state.  Saves dS, dU and W = T^T dU of every
@@ -132,6 +132,30 @@ __device__ inline UnitPos unit_pos(const SeqMap& m, int n, int h) {
 
 __device__ inline bool seqs_ok(const SeqMap& m) { return m.cu == nullptr || m.sb->seqlens_ok == 1; }
 
+// The chunk a block of a per-chunk kernel takes: block = (global chunk cg,
+// head h); dense, chunk cg % nc of sequence cg / nc; packed, the sequence
+// whose chunk range holds cg (binary search over the offsets).  False for
+// the blocks past the last chunk of a packed batch.
+__device__ inline bool chunk_of_block(const SeqMap& m, int N, int& h, int& c, UnitPos& up) {
+  const int64_t cg = blockIdx.x / m.H;
+  h = blockIdx.x % m.H;
+  int seq;
+  if (m.cu == nullptr) {
+    seq = (int)(cg / ((m.T + C - 1) / C));
+  } else {
+    if (cg >= m.coff[N]) return false;
+    int lo = 0, hi = N;  // coff[lo] <= cg < coff[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (m.coff[mid] <= cg) lo = mid; else hi = mid;
+    }
+    seq = lo;
+  }
+  up = unit_pos(m, seq, h);
+  c = (int)(cg - (m.cu == nullptr ? (int64_t)seq * up.nc : (int64_t)m.coff[seq]));
+  return true;
+}
+
 __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int DV) {
   UnitWs w;
   float* base = ws + (size_t)chunk0 * unit_ws_floats(1, DK, DV);
@@ -225,44 +249,150 @@ __global__ void __launch_bounds__(kPlanThreads)
   }
 }
 
-// ===================================================================== pass F
-// One CTA of 512 threads per unit, all dv columns, so the key-side matrices
-// are formed once per chunk.  The Gram matrices are one product each when
+// ===================================================================== pass K
+// The key-side matrices of every chunk at once, one CTA per (chunk, head):
+// L = strict_lower(sum_i k_ri k_si E_rsi), A_qk = lower(sum_i q_ri k_si E_rsi)
+// and X = (I + Diag(beta) L)^-1.  The Gram matrices are one product each when
 // the chunk's decays let every factor e^{+-(Gamma_r - Gamma_15)} stay below
 // e^80 (always, for the gate's g >= -5): L = (k e^{Gamma - Gamma_15})
 // (k e^{Gamma_15 - Gamma})^T; otherwise each entry takes exponentials of
 // differences Gamma_r - Gamma_s <= 0.
+template <int DK>
+struct KSmem {
+  static constexpr int LDK = DK + 1;
+  static constexpr int floats = 5 * C * LDK       // q (then q factor), k, Gamma, two factors
+                                + 3 * C * LDC     // L, A_qk, X
+                                + C;              // beta
+  static constexpr size_t bytes = sizeof(float) * floats;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(NTH, 2)
+    bwd_keyside(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                const float* __restrict__ g, const float* __restrict__ beta, SeqMap map, int N,
+                float* __restrict__ ws) {
+  constexpr int LDK = DK + 1;
+  extern __shared__ float sm[];
+  float* qS = sm;                 // [C][LDK]  q, then q e^{Gamma - Gamma_15}
+  float* kS = qS + C * LDK;       // [C][LDK]
+  float* GS = kS + C * LDK;       // [C][LDK]  Gamma
+  float* FaS = GS + C * LDK;      // [C][LDK]  k e^{Gamma - Gamma_15}
+  float* FbS = FaS + C * LDK;     // [C][LDK]  k e^{Gamma_15 - Gamma}
+  float* LS = FbS + C * LDK;      // [C][LDC]
+  float* AqS = LS + C * LDC;      // [C][LDC]
+  float* XS = AqS + C * LDC;      // [C][LDC]
+  float* bS = XS + C * LDC;       // [C]
+
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  int h, c;
+  UnitPos up;
+  if (!chunk_of_block(map, N, h, c, up)) return;
+  const int t0 = c * C, n = min(C, up.len - t0);
+  const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+  const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
+  const int tid = threadIdx.x;
+
+  load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
+  for (int i = tid; i < DK; i += NTH) {
+    const float g15 = GS[MREB * LDK + i];
+    for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - g15) > 80.f;
+  }
+  wide = __syncthreads_or(wide);
+  if (!wide) {
+    for (int idx = tid; idx < C * DK; idx += NTH) {
+      const int r = idx / DK, i = idx % DK;
+      const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+      const float ea = expf(d), eb = expf(-d), kv = kS[r * LDK + i];
+      FaS[r * LDK + i] = kv * ea;
+      FbS[r * LDK + i] = kv * eb;
+      qS[r * LDK + i] *= ea;
+    }
+    __syncthreads();
+    float lk[2][2], lq[2][2];
+    zero(lk);
+    zero(lq);
+    mm<C, C, 2, 2, DK>(lk, [&](int m, int kk) { return FaS[m * LDK + kk]; },
+                       [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
+    mm<C, C, 2, 2, DK>(lq, [&](int m, int kk) { return qS[m * LDK + kk]; },
+                       [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
+    for_tile<C, C, 2, 2>([&](int r, int s2, int i, int j) {
+      LS[r * LDC + s2] = s2 < r ? lk[i][j] : 0.f;
+      AqS[r * LDC + s2] = s2 <= r ? lq[i][j] : 0.f;
+    });
+  } else {
+    for (int p = tid; p < C * C; p += NTH) {
+      const int r = p / C, s2 = p % C;
+      float lk = 0.f, lq = 0.f;
+      if (s2 <= r) {
+#pragma unroll 4
+        for (int i = 0; i < DK; ++i) {
+          const float ks = kS[s2 * LDK + i] * expf(GS[r * LDK + i] - GS[s2 * LDK + i]);
+          lk = fmaf(kS[r * LDK + i], ks, lk);
+          lq = fmaf(qS[r * LDK + i], ks, lq);
+        }
+      }
+      LS[r * LDC + s2] = s2 < r ? lk : 0.f;
+      AqS[r * LDC + s2] = lq;
+    }
+  }
+  __syncthreads();
+  // X = (I + Diag(beta) L)^-1 by forward substitution; the columns are
+  // independent, so warp w takes columns 4w .. 4w+3 with 8 lanes per column
+  {
+    const int lane = tid & 31, cc = 4 * (tid >> 5) + (lane >> 3), sub = lane & 7;
+    for (int r = sub; r < C; r += 8) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
+    __syncwarp();
+    for (int r = 1; r < C; ++r) {
+      float acc = 0.f;
+      for (int s2 = cc + sub; s2 < r; s2 += 8) acc = fmaf(LS[r * LDC + s2], XS[s2 * LDC + cc], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (sub == 0 && r > cc) XS[r * LDC + cc] = -bS[r] * acc;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += NTH) {
+    const int r = idx / C, s2 = idx % C;
+    const size_t o = ((size_t)c * C + r) * C + s2;
+    w.X[o] = XS[r * LDC + s2];
+    w.Aqk[o] = AqS[r * LDC + s2];
+    w.L[o] = LS[r * LDC + s2];
+  }
+}
+
+// ===================================================================== pass F
+// The state scan, one CTA of 512 threads per unit, all dv columns: per chunk
+// R = V - Ka S, U = T R (T = X Diag(beta) from pass K) and the state update.
 template <int DK, int DV>
 struct FSmem {
   static constexpr int LDK = DK + 1, LDV = DV + 1;
-  static constexpr int floats = 5 * C * LDK       // q (then q factor), k (then Kc), Gamma, two factors
+  static constexpr int floats = 3 * C * LDK       // k (then Kc), Gamma, Ka
                                 + DK * LDV        // state
                                 + 2 * C * LDV     // V (then R), U
-                                + 3 * C * LDC     // L, A_qk, X (then T)
+                                + C * LDC         // T
                                 + C + 2 * DK;     // beta, Gamma_C, e^{Gamma_C}
   static constexpr size_t bytes = sizeof(float) * floats;
 };
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NTF, 1)
-    bwd_fwd_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                 const Tin* __restrict__ v, const float* __restrict__ g,
-                 const float* __restrict__ beta, const float* __restrict__ init, SeqMap map,
-                 float* __restrict__ ws) {
+    bwd_fwd_scan(const Tin* __restrict__ k, const Tin* __restrict__ v,
+                 const float* __restrict__ g, const float* __restrict__ beta,
+                 const float* __restrict__ init, SeqMap map, float* __restrict__ ws) {
   constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
-  float* qS = sm;                 // [C][LDK]  q, then q e^{Gamma - Gamma_15}
-  float* kS = qS + C * LDK;       // [C][LDK]  k, then Kc
+  float* kS = sm;                 // [C][LDK]  k, then Kc
   float* GS = kS + C * LDK;       // [C][LDK]  Gamma
-  float* FaS = GS + C * LDK;      // [C][LDK]  k e^{Gamma - Gamma_15}, then Ka
-  float* FbS = FaS + C * LDK;     // [C][LDK]  k e^{Gamma_15 - Gamma}
-  float* SS = FbS + C * LDK;      // [DK][LDV] state
+  float* KaS = GS + C * LDK;      // [C][LDK]  Ka
+  float* SS = KaS + C * LDK;      // [DK][LDV] state
   float* VS = SS + DK * LDV;      // [C][LDV]  V, then R = V - Ka S
   float* US = VS + C * LDV;       // [C][LDV]
-  float* LS = US + C * LDV;       // [C][LDC]
-  float* AqS = LS + C * LDC;      // [C][LDC]
-  float* XS = AqS + C * LDC;      // [C][LDC]  X, then T
-  float* bS = XS + C * LDC;       // [C]
+  float* TS = US + C * LDV;       // [C][LDC]
+  float* bS = TS + C * LDC;       // [C]
   float* gC = bS + C;             // [DK] Gamma_C
   float* eC = gC + DK;            // [DK] e^{Gamma_C}
 
@@ -285,14 +415,12 @@ __global__ void __launch_bounds__(NTF, 1)
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {
       const int r = idx / DK, i = idx % DK;
-      float qv = 0.f, kv = 0.f, gv = 0.f;
+      float kv = 0.f, gv = 0.f;
       if (r < n) {
         const size_t off = (rowbase + (size_t)r * H) * DK + i;
-        qv = Elem<Tin>::load(q + off);
         kv = Elem<Tin>::load(k + off);
         gv = g[off];
       }
-      qS[r * LDK + i] = qv;
       kS[r * LDK + i] = kv;
       GS[r * LDK + i] = gv;
     }
@@ -306,7 +434,6 @@ __global__ void __launch_bounds__(NTF, 1)
       w.S[(size_t)c * DK * DV + idx] = SS[i * LDV + j];
     }
     __syncthreads();
-    bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
     for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
       float acc = 0.f;
       for (int r = 0; r < C; ++r) {
@@ -315,84 +442,23 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       gC[i] = acc;
       eC[i] = expf(acc);
-      const float g15 = GS[MREB * LDK + i];
-      for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - g15) > 80.f;
     }
-    wide = __syncthreads_or(wide);
-    if (!wide) {
-      for (int idx = tid; idx < C * DK; idx += NTF) {
-        const int r = idx / DK, i = idx % DK;
-        const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
-        const float ea = expf(d), eb = expf(-d), kv = kS[r * LDK + i];
-        FaS[r * LDK + i] = kv * ea;
-        FbS[r * LDK + i] = kv * eb;
-        qS[r * LDK + i] *= ea;
-      }
-      __syncthreads();
-      float lk[1][2], lq[1][2];
-      zero(lk);
-      zero(lq);
-      mm<C, C, 1, 2, DK>(lk, [&](int m, int kk) { return FaS[m * LDK + kk]; },
-                         [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
-      mm<C, C, 1, 2, DK>(lq, [&](int m, int kk) { return qS[m * LDK + kk]; },
-                         [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
-      for_tile<C, C, 1, 2>([&](int r, int s2, int i, int j) {
-        LS[r * LDC + s2] = s2 < r ? lk[i][j] : 0.f;
-        AqS[r * LDC + s2] = s2 <= r ? lq[i][j] : 0.f;
-      });
-    } else {
-      for (int p = tid; p < C * C; p += NTF) {
-        const int r = p / C, s2 = p % C;
-        float lk = 0.f, lq = 0.f;
-        if (s2 <= r) {
-#pragma unroll 4
-          for (int i = 0; i < DK; ++i) {
-            const float ks = kS[s2 * LDK + i] * expf(GS[r * LDK + i] - GS[s2 * LDK + i]);
-            lk = fmaf(kS[r * LDK + i], ks, lk);
-            lq = fmaf(qS[r * LDK + i], ks, lq);
-          }
-        }
-        LS[r * LDC + s2] = s2 < r ? lk : 0.f;
-        AqS[r * LDC + s2] = lq;
-      }
-    }
-    __syncthreads();
-    // X = (I + Diag(beta) L)^-1 by forward substitution; the columns are
-    // independent, so warp w takes columns 2w, 2w + 1 with 16 lanes per column
-    {
-      const int lane = tid & 31, cc = 2 * (tid >> 5) + (lane >> 4), sub = lane & 15;
-      for (int r = sub; r < C; r += 16) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
-      __syncwarp();
-      for (int r = 1; r < C; ++r) {
-        float acc = 0.f;
-        for (int s2 = cc + sub; s2 < r; s2 += 16) acc = fmaf(LS[r * LDC + s2], XS[s2 * LDC + cc], acc);
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (sub == 0 && r > cc) XS[r * LDC + cc] = -bS[r] * acc;
-        __syncwarp();
-      }
-    }
-    __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NTF) {  // the key-side matrices, then T
+    for (int idx = tid; idx < C * C; idx += NTF) {  // T = X Diag(beta)
       const int r = idx / C, s2 = idx % C;
-      const size_t o = ((size_t)c * C + r) * C + s2;
-      const float x = XS[r * LDC + s2];
-      w.X[o] = x;
-      w.Aqk[o] = AqS[r * LDC + s2];
-      w.L[o] = LS[r * LDC + s2];
-      XS[r * LDC + s2] = x * bS[s2];
+      TS[r * LDC + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
     }
-    for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka (into FaS), Kc (into kS)
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka, Kc (into kS)
       const int r = idx / DK, i = idx % DK;
       const float G = GS[r * LDK + i], kv = kS[r * LDK + i];
-      FaS[r * LDK + i] = kv * expf(G);
+      KaS[r * LDK + i] = kv * expf(G);
       kS[r * LDK + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
     {  // R = V - Ka S
       float acc[1][DV / 16];
       zero(acc);
-      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return FaS[m * LDK + kk]; },
+      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return KaS[m * LDK + kk]; },
                                 [&](int kk, int nn) { return SS[kk * LDV + nn]; });
       for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { VS[m * LDV + nn] -= acc[i][j]; });
     }
@@ -400,7 +466,7 @@ __global__ void __launch_bounds__(NTF, 1)
     {  // U = T R
       float acc[1][DV / 16];
       zero(acc);
-      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return XS[m * LDC + kk]; },
+      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDC + kk]; },
                                [&](int kk, int nn) { return VS[kk * LDV + nn]; });
       for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
     }
@@ -621,26 +687,11 @@ __global__ void __launch_bounds__(NTH, 2)
   float* rsum = gC + DK;          // [DK] sum_j dS_ij S_ij
   float* kcsum = rsum + DK;       // [DK] sum_r dKc_ri Kc_ri
 
-  // block = (global chunk, head): dense chunk cg is chunk cg % nc of sequence
-  // cg / nc; packed, the sequence whose chunk range holds cg (binary search)
   if (!seqs_ok(map)) return;
   const int H = map.H;
-  const int64_t cg = blockIdx.x / H;
-  const int h = blockIdx.x % H;
-  int seq;
-  if (map.cu == nullptr) {
-    seq = (int)(cg / ((map.T + C - 1) / C));
-  } else {
-    if (cg >= map.coff[N]) return;
-    int lo = 0, hi = N;  // coff[lo] <= cg < coff[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) / 2;
-      if (map.coff[mid] <= cg) lo = mid; else hi = mid;
-    }
-    seq = lo;
-  }
-  const UnitPos up = unit_pos(map, seq, h);
-  const int c = (int)(cg - (map.cu == nullptr ? (int64_t)seq * up.nc : (int64_t)map.coff[seq]));
+  int h, c;
+  UnitPos up;
+  if (!chunk_of_block(map, N, h, c, up)) return;
   const int t0 = c * C, n = min(C, up.len - t0);
   const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
   const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
@@ -850,20 +901,27 @@ __global__ void __launch_bounds__(NTH, 2)
 
 // F and A, one CTA per unit each
 template <typename Tin, int DK, int DV>
-cudaError_t launch_scans(const BwdArgs& a, const SeqMap& map, int units, float* ws,
-                         cudaStream_t st) {
-  const size_t smF = FSmem<DK, DV>::bytes, smA = ASmem<DK, DV>::bytes;
-  cudaError_t e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
+cudaError_t launch_scans(const BwdArgs& a, const SeqMap& map, int units, int64_t chunk_blocks,
+                         float* ws, cudaStream_t st) {
+  const size_t smK = KSmem<DK>::bytes, smF = FSmem<DK, DV>::bytes, smA = ASmem<DK, DV>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(bwd_keyside<Tin, DK, DV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smK);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK, DV>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
   if (e != cudaSuccess) return e;
   const Tin* q = static_cast<const Tin*>(a.q);
   const Tin* k = static_cast<const Tin*>(a.k);
+  const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
   if (a.T > 0) {
+    bwd_keyside<Tin, DK, DV><<<(unsigned)chunk_blocks, NTH, smK, st>>>(q, k, a.g, a.beta, map,
+                                                                       nseq, ws);
+    if ((e = cudaGetLastError())) return e;
     bwd_fwd_scan<Tin, DK, DV><<<units, NTF, smF, st>>>(
-        q, k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, map, ws);
+        k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, map, ws);
     if ((e = cudaGetLastError())) return e;
   }
   bwd_state_grad_scan<Tin, DK, DV><<<units, NTF, smA, st>>>(
@@ -903,9 +961,9 @@ cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError())) return e;
   }
   switch (a.dv_dim) {
-    case 32: e = launch_scans<Tin, DK, 32>(a, map, nseq * a.H, ws, st); break;
-    case 64: e = launch_scans<Tin, DK, 64>(a, map, nseq * a.H, ws, st); break;
-    case 128: e = launch_scans<Tin, DK, 128>(a, map, nseq * a.H, ws, st); break;
+    case 32: e = launch_scans<Tin, DK, 32>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
+    case 64: e = launch_scans<Tin, DK, 64>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
+    case 128: e = launch_scans<Tin, DK, 128>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
     default: e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess || lay.max_chunks == 0) return e;
