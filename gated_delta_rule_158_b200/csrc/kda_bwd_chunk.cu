@@ -77,6 +77,46 @@ __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
     for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
 }
 
+// Warp-level tensor-core products in tf32 with fp32 accuracy: each operand
+// x = hi + lo with hi = tf32(x), lo = tf32(x - hi), and a b = a_lo b_hi +
+// a_hi b_lo + a_hi b_hi (the dropped a_lo b_lo is below fp32 rounding).
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// m16n8k8 fragments from shared memory: A rows row0.. (row-major, leading
+// dimension ld), B given as [n][k] rows col0..; lane = 4 g + t
+struct Frag3 {
+  uint32_t ah[4], al[4];
+};
+__device__ __forceinline__ void load_a(Frag3& f, const float* X, int ld, int row0, int k0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  split_tf32(X[(row0 + g) * ld + k0 + t], f.ah[0], f.al[0]);
+  split_tf32(X[(row0 + g + 8) * ld + k0 + t], f.ah[1], f.al[1]);
+  split_tf32(X[(row0 + g) * ld + k0 + t + 4], f.ah[2], f.al[2]);
+  split_tf32(X[(row0 + g + 8) * ld + k0 + t + 4], f.ah[3], f.al[3]);
+}
+__device__ __forceinline__ void mma3(float (&d)[4], const Frag3& a, const float* Y, int ld,
+                                     int col0, int k0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  uint32_t bh[2], bl[2];
+  split_tf32(Y[(col0 + g) * ld + k0 + t], bh[0], bl[0]);
+  split_tf32(Y[(col0 + g) * ld + k0 + t + 4], bh[1], bl[1]);
+  mma_tf32(d, a.al, bh);
+  mma_tf32(d, a.ah, bl);
+  mma_tf32(d, a.ah, bh);
+}
+
 // per-unit workspace: S_c, dS_c [nc][DK][DV]; X, A_qk, L [nc][C][C];
 // R, U, dU, W [nc][C][DV]
 struct UnitWs {
@@ -637,9 +677,10 @@ __global__ void __launch_bounds__(NTF, 1)
 }
 
 // ===================================================================== pass B
-// B takes the dv columns 16 at a time, which keeps it at two CTAs per SM
+// B takes the dv columns 16 at a time, which keeps it at two CTAs per SM;
+// rows of 20 floats keep the tensor-core fragment loads free of bank conflicts
 constexpr int VBB = 16;
-constexpr int LDBB = VBB + 1;
+constexpr int LDBB = VBB + 4;
 
 template <int DK>
 struct BSmem {
@@ -713,66 +754,11 @@ __global__ void __launch_bounds__(NTH, 2)
   // products summed over the dv columns, accumulated block by block from
   // the saved R, U, dU, W:
   // dQg^T = S dO'^T, -dKa^T = S W^T, dKc^T = dS U^T  (DK x C); dA_qk, dT (C x C)
-  float aQ[TMK][4], aKa[TMK][4], aKc[TMK][4], aA[2][2], aT[2][2];
-  zero(aQ);
-  zero(aKa);
-  zero(aKc);
-  zero(aA);
-  zero(aT);
-  for (int j0 = 0; j0 < DV; j0 += VBB) {
-    __syncthreads();
-    // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
-    auto put4 = [](float* dst, float4 x) {
-      dst[0] = x.x;
-      dst[1] = x.y;
-      dst[2] = x.z;
-      dst[3] = x.w;
-    };
-    for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
-      const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
-      const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
-      put4(SS + i * LDBB + j, *reinterpret_cast<const float4*>(w.S + o));
-      put4(dSS + i * LDBB + j, *reinterpret_cast<const float4*>(w.dS + o));
-    }
-    for (int idx = tid; idx < C * VBB / 4; idx += NTH) {
-      const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
-      const size_t o = ((size_t)c * C + r) * DV + j0 + j;
-      put4(RS + r * LDBB + j, *reinterpret_cast<const float4*>(w.R + o));
-      put4(US + r * LDBB + j, *reinterpret_cast<const float4*>(w.U + o));
-      put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
-      put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
-    }
-    for (int idx = tid; idx < C * VBB; idx += NTH) {
-      const int r = idx / VBB, j = idx % VBB;
-      dOS[r * LDBB + j] =
-          r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
-    }
-    __syncthreads();
-    for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
-      float acc = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < VBB; ++j) acc = fmaf(dSS[i * LDBB + j], SS[i * LDBB + j], acc);
-      rsum[i] += acc;
-    }
-    // block contributions, contracted over this block's 16 columns
-    mm<DK, C, TMK, 4, VBB>(aQ, [&](int m, int kk) { return SS[m * LDBB + kk]; },
-                           [&](int kk, int nn) { return dOS[nn * LDBB + kk]; });
-    mm<DK, C, TMK, 4, VBB>(aKa, [&](int m, int kk) { return SS[m * LDBB + kk]; },
-                           [&](int kk, int nn) { return WS[nn * LDBB + kk]; });
-    mm<DK, C, TMK, 4, VBB>(aKc, [&](int m, int kk) { return dSS[m * LDBB + kk]; },
-                           [&](int kk, int nn) { return US[nn * LDBB + kk]; });
-    mm<C, C, 2, 2, VBB>(aA, [&](int m, int kk) { return dOS[m * LDBB + kk]; },
-                        [&](int kk, int nn) { return US[nn * LDBB + kk]; });
-    mm<C, C, 2, 2, VBB>(aT, [&](int m, int kk) { return dUS[m * LDBB + kk]; },
-                        [&](int kk, int nn) { return RS[nn * LDBB + kk]; });
-  }
-  __syncthreads();  // the loop tiles become the dGamma accumulator
-  // dq, dk (into the outputs, rows < n) and dGamma from the state-side
-  // products and the decays
-  for_tile<DK, C, TMK, 4>([&](int i, int r, int a, int bb) {
+  // dq, dk (into the outputs, rows < n) and dGamma of element (i, r) from the
+  // state-side products dQg_ri, dKa_ri, dKc_ri and the decays
+  auto elem = [&](int i, int r, float dQg, float dKa, float dKc) {
     const float e = expf(GS[r * LDK + i]);
     const float ec = expf(gC[i] - GS[r * LDK + i]);
-    const float dQg = aQ[a][bb], dKa = -aKa[a][bb], dKc = aKc[a][bb];
     const float qv = qS[r * LDK + i], kv = kS[r * LDK + i];
     if (r < n) {
       const size_t o = (rowbase + (size_t)r * H) * DK + i;
@@ -781,28 +767,174 @@ __global__ void __launch_bounds__(NTH, 2)
     }
     // dGamma: dQg Qg + dKa Ka - dKc Kc  (Qg = q e, Ka = k e, Kc = k ec)
     aG[r * LDK + i] = fmaf(fmaf(dQg, qv, dKa * kv), e, -dKc * kv * ec);
-  });
-  {  // sum_r dKc_ri Kc_ri: this thread's 4 columns, then the 8 lanes of its row block
-    constexpr int NTN = C / 4;
-    const int tn = tid % NTN, tm = tid / NTN;
-#pragma unroll
-    for (int a = 0; a < TMK; ++a) {
-      const int i = tm + a * (DK / TMK);
-      float sacc = 0.f;
-#pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
-        const int r = tn + bb * NTN;
-        sacc = fmaf(aKc[a][bb], kS[r * LDK + i] * expf(gC[i] - GS[r * LDK + i]), sacc);
+    return dKc * kv * ec;  // dKc Kc, summed over r into dGamma_C
+  };
+  if constexpr (DK == 128) {
+    // tensor cores: warp w owns rows 16w .. 16w+15 of dQg^T, -dKa^T, dKc^T
+    // (4 n-tiles of 8 chunk rows each) and one 16 x 16 corner of dA_qk
+    // (warps 0-3) or dT (warps 4-7)
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int mc = (warp & 3) >> 1, nc0 = (warp & 1) * 2;
+    float aQ[4][4], aKa[4][4], aKc[4][4], aC[2][4];
+    zero(aQ);
+    zero(aKa);
+    zero(aKc);
+    zero(aC);
+    for (int j0 = 0; j0 < DV; j0 += VBB) {
+      __syncthreads();
+      // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
+      auto put4 = [](float* dst, float4 x) {
+        dst[0] = x.x;
+        dst[1] = x.y;
+        dst[2] = x.z;
+        dst[3] = x.w;
+      };
+      for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
+        const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
+        put4(SS + i * LDBB + j, *reinterpret_cast<const float4*>(w.S + o));
+        put4(dSS + i * LDBB + j, *reinterpret_cast<const float4*>(w.dS + o));
       }
+      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {
+        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        const size_t o = ((size_t)c * C + r) * DV + j0 + j;
+        put4(RS + r * LDBB + j, *reinterpret_cast<const float4*>(w.R + o));
+        put4(US + r * LDBB + j, *reinterpret_cast<const float4*>(w.U + o));
+        put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
+        put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
+      }
+      for (int idx = tid; idx < C * VBB; idx += NTH) {
+        const int r = idx / VBB, j = idx % VBB;
+        dOS[r * LDBB + j] =
+            r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+      }
+      __syncthreads();
+      for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < VBB; ++j) acc = fmaf(dSS[i * LDBB + j], SS[i * LDBB + j], acc);
+        rsum[i] += acc;
+      }
+      for (int k0 = 0; k0 < VBB; k0 += 8) {
+        Frag3 fs, fd, fc;
+        load_a(fs, SS, LDBB, 16 * warp, k0);
+        load_a(fd, dSS, LDBB, 16 * warp, k0);
 #pragma unroll
-      for (int o = NTN / 2; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
-      if (tn == 0) kcsum[i] = sacc;
+        for (int nt = 0; nt < 4; ++nt) {
+          mma3(aQ[nt], fs, dOS, LDBB, 8 * nt, k0);
+          mma3(aKa[nt], fs, WS, LDBB, 8 * nt, k0);
+          mma3(aKc[nt], fd, US, LDBB, 8 * nt, k0);
+        }
+        load_a(fc, warp < 4 ? dOS : dUS, LDBB, 16 * mc, k0);
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+          mma3(aC[q2], fc, warp < 4 ? US : RS, LDBB, 8 * (nc0 + q2), k0);
+      }
     }
+    __syncthreads();  // the loop tiles become the dGamma accumulator
+    float kc0 = 0.f, kc1 = 0.f;  // sum_r dKc Kc of rows 16w + g and 16w + g + 8
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 16 * warp + g + 8 * (e >> 1), r = 8 * nt + 2 * t + (e & 1);
+        const float kk = elem(i, r, aQ[nt][e], -aKa[nt][e], aKc[nt][e]);
+        if (e < 2) kc0 += kk; else kc1 += kk;
+      }
+    kc0 += __shfl_xor_sync(0xffffffffu, kc0, 1);
+    kc1 += __shfl_xor_sync(0xffffffffu, kc1, 1);
+    kc0 += __shfl_xor_sync(0xffffffffu, kc0, 2);
+    kc1 += __shfl_xor_sync(0xffffffffu, kc1, 2);
+    if (t == 0) {
+      kcsum[16 * warp + g] = kc0;
+      kcsum[16 * warp + g + 8] = kc1;
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = 16 * mc + g + 8 * (e >> 1), s2 = 8 * (nc0 + q2) + 2 * t + (e & 1);
+        if (warp < 4)
+          dAqS[r * LDC + s2] = s2 <= r ? aC[q2][e] : 0.f;
+        else
+          dTS[r * LDC + s2] = aC[q2][e];
+      }
+  } else {
+    float aQ[TMK][4], aKa[TMK][4], aKc[TMK][4], aA[2][2], aT[2][2];
+    zero(aQ);
+    zero(aKa);
+    zero(aKc);
+    zero(aA);
+    zero(aT);
+    for (int j0 = 0; j0 < DV; j0 += VBB) {
+      __syncthreads();
+      // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
+      auto put4 = [](float* dst, float4 x) {
+        dst[0] = x.x;
+        dst[1] = x.y;
+        dst[2] = x.z;
+        dst[3] = x.w;
+      };
+      for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
+        const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
+        put4(SS + i * LDBB + j, *reinterpret_cast<const float4*>(w.S + o));
+        put4(dSS + i * LDBB + j, *reinterpret_cast<const float4*>(w.dS + o));
+      }
+      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {
+        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        const size_t o = ((size_t)c * C + r) * DV + j0 + j;
+        put4(RS + r * LDBB + j, *reinterpret_cast<const float4*>(w.R + o));
+        put4(US + r * LDBB + j, *reinterpret_cast<const float4*>(w.U + o));
+        put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
+        put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
+      }
+      for (int idx = tid; idx < C * VBB; idx += NTH) {
+        const int r = idx / VBB, j = idx % VBB;
+        dOS[r * LDBB + j] =
+            r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+      }
+      __syncthreads();
+      for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < VBB; ++j) acc = fmaf(dSS[i * LDBB + j], SS[i * LDBB + j], acc);
+        rsum[i] += acc;
+      }
+      mm<DK, C, TMK, 4, VBB>(aQ, [&](int m, int kk) { return SS[m * LDBB + kk]; },
+                             [&](int kk, int nn) { return dOS[nn * LDBB + kk]; });
+      mm<DK, C, TMK, 4, VBB>(aKa, [&](int m, int kk) { return SS[m * LDBB + kk]; },
+                             [&](int kk, int nn) { return WS[nn * LDBB + kk]; });
+      mm<DK, C, TMK, 4, VBB>(aKc, [&](int m, int kk) { return dSS[m * LDBB + kk]; },
+                             [&](int kk, int nn) { return US[nn * LDBB + kk]; });
+      mm<C, C, 2, 2, VBB>(aA, [&](int m, int kk) { return dOS[m * LDBB + kk]; },
+                          [&](int kk, int nn) { return US[nn * LDBB + kk]; });
+      mm<C, C, 2, 2, VBB>(aT, [&](int m, int kk) { return dUS[m * LDBB + kk]; },
+                          [&](int kk, int nn) { return RS[nn * LDBB + kk]; });
+    }
+    __syncthreads();  // the loop tiles become the dGamma accumulator
+    float kcp[TMK];
+#pragma unroll
+    for (int a = 0; a < TMK; ++a) kcp[a] = 0.f;
+    for_tile<DK, C, TMK, 4>([&](int i, int r, int a, int bb) {
+      kcp[a] += elem(i, r, aQ[a][bb], -aKa[a][bb], aKc[a][bb]);
+    });
+    {  // sum_r dKc_ri Kc_ri: this thread's 4 columns, then the 8 lanes of its row block
+      constexpr int NTN = C / 4;
+      const int tn = tid % NTN, tm = tid / NTN;
+#pragma unroll
+      for (int a = 0; a < TMK; ++a) {
+        float sacc = kcp[a];
+#pragma unroll
+        for (int o = NTN / 2; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+        if (tn == 0) kcsum[tm + a * (DK / TMK)] = sacc;
+      }
+    }
+    for_tile<C, C, 2, 2>([&](int r, int s2, int i, int j) {
+      dAqS[r * LDC + s2] = s2 <= r ? aA[i][j] : 0.f;
+      dTS[r * LDC + s2] = aT[i][j];
+    });
   }
-  for_tile<C, C, 2, 2>([&](int r, int s, int i, int j) {
-    dAqS[r * LDC + s] = s <= r ? aA[i][j] : 0.f;
-    dTS[r * LDC + s] = aT[i][j];
-  });
   __syncthreads();
   // dbeta_s = sum_r dT_rs X_rs (from T = X Diag(beta)); dX = dT Diag(beta)
   float db = 0.f;
