@@ -94,27 +94,42 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// m16n8k8 fragments from shared memory: A rows row0.. (row-major, leading
-// dimension ld), B given as [n][k] rows col0..; lane = 4 g + t
+// m16n8k8 fragments from shared memory (lane = 4 g + t).  A: rows row0 ..
+// row0+15 of an [M][K] tile (TA = false) or of the transpose of a [K][M] tile
+// (TA = true), times `sign`.  B: columns col0 .. col0+7 of a K x N operand
+// given as [N][K] (KN = false) or [K][N] (KN = true).
 struct Frag3 {
   uint32_t ah[4], al[4];
 };
-__device__ __forceinline__ void load_a(Frag3& f, const float* X, int ld, int row0, int k0) {
+template <bool TA = false>
+__device__ __forceinline__ void load_a(Frag3& f, const float* X, int ld, int row0, int k0,
+                                       float sign = 1.f) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  split_tf32(X[(row0 + g) * ld + k0 + t], f.ah[0], f.al[0]);
-  split_tf32(X[(row0 + g + 8) * ld + k0 + t], f.ah[1], f.al[1]);
-  split_tf32(X[(row0 + g) * ld + k0 + t + 4], f.ah[2], f.al[2]);
-  split_tf32(X[(row0 + g + 8) * ld + k0 + t + 4], f.ah[3], f.al[3]);
+  auto at = [&](int m, int k) { return TA ? X[k * ld + m] : X[m * ld + k]; };
+  split_tf32(sign * at(row0 + g, k0 + t), f.ah[0], f.al[0]);
+  split_tf32(sign * at(row0 + g + 8, k0 + t), f.ah[1], f.al[1]);
+  split_tf32(sign * at(row0 + g, k0 + t + 4), f.ah[2], f.al[2]);
+  split_tf32(sign * at(row0 + g + 8, k0 + t + 4), f.ah[3], f.al[3]);
 }
+template <bool KN = false>
 __device__ __forceinline__ void mma3(float (&d)[4], const Frag3& a, const float* Y, int ld,
                                      int col0, int k0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  auto at = [&](int k, int n) { return KN ? Y[k * ld + n] : Y[n * ld + k]; };
   uint32_t bh[2], bl[2];
-  split_tf32(Y[(col0 + g) * ld + k0 + t], bh[0], bl[0]);
-  split_tf32(Y[(col0 + g) * ld + k0 + t + 4], bh[1], bl[1]);
+  split_tf32(at(k0 + t, col0 + g), bh[0], bl[0]);
+  split_tf32(at(k0 + t + 4, col0 + g), bh[1], bl[1]);
   mma_tf32(d, a.al, bh);
   mma_tf32(d, a.ah, bl);
   mma_tf32(d, a.ah, bh);
+}
+
+// C / D fragment element e of the m16n8 tile at (row0, col0): its row and column
+__device__ __forceinline__ int frag_row(int row0, int e) {
+  return row0 + ((threadIdx.x & 31) >> 2) + 8 * (e >> 1);
+}
+__device__ __forceinline__ int frag_col(int col0, int e) {
+  return col0 + 2 * (threadIdx.x & 3) + (e & 1);
 }
 
 // per-unit workspace: S_c, dS_c [nc][DK][DV]; X, A_qk, L [nc][C][C];
@@ -495,35 +510,96 @@ __global__ void __launch_bounds__(NTF, 1)
       kS[r * LDK + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
-    {  // R = V - Ka S
-      float acc[1][DV / 16];
-      zero(acc);
-      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return KaS[m * LDK + kk]; },
-                                [&](int kk, int nn) { return SS[kk * LDV + nn]; });
-      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { VS[m * LDV + nn] -= acc[i][j]; });
-    }
-    __syncthreads();
-    {  // U = T R
-      float acc[1][DV / 16];
-      zero(acc);
-      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDC + kk]; },
-                               [&](int kk, int nn) { return VS[kk * LDV + nn]; });
-      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
-    }
-    __syncthreads();
-    for (int idx = tid; idx < C * DV; idx += NTF) {
-      const int r = idx / DV, j = idx % DV;
-      w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
-      w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
-    }
-    {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
-      float acc[DK / 32][DV / 16];
-      zero(acc);
-      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
-                                      [&](int kk, int nn) { return US[kk * LDV + nn]; });
-      for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
-        SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
-      });
+    if constexpr (DK == 128 && DV == 128) {
+      // tensor cores: warp w owns C x DV tiles (w >> 3, 2 (w & 7) + {0, 1}) and
+      // DK x DV tiles (w >> 1, 8 (w & 1) + 0..7)
+      const int wp = tid >> 5, mt = wp >> 3, nt0 = 2 * (wp & 7);
+      const int mt8 = wp >> 1, nt8 = 8 * (wp & 1);
+      {  // R = V - Ka S
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < DK; k0 += 8) {
+          Frag3 a;
+          load_a(a, KaS, LDK, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, SS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            VS[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] -= acc[q2][e];
+      }
+      __syncthreads();
+      {  // U = T R
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a(a, TS, LDC, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, VS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            US[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] = acc[q2][e];
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DV; idx += NTF) {
+        const int r = idx / DV, j = idx % DV;
+        w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
+        w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
+      }
+      {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
+        float acc[8][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a<true>(a, kS, LDK, 16 * mt8, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 8; ++q2) mma3<true>(acc[q2], a, US, LDV, 8 * (nt8 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 8; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = frag_row(16 * mt8, e), j = frag_col(8 * (nt8 + q2), e);
+            SS[i * LDV + j] = fmaf(eC[i], SS[i * LDV + j], acc[q2][e]);
+          }
+      }
+    } else {
+      {  // R = V - Ka S
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return KaS[m * LDK + kk]; },
+                                  [&](int kk, int nn) { return SS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { VS[m * LDV + nn] -= acc[i][j]; });
+      }
+      __syncthreads();
+      {  // U = T R
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDC + kk]; },
+                                 [&](int kk, int nn) { return VS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DV; idx += NTF) {
+        const int r = idx / DV, j = idx % DV;
+        w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
+        w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
+      }
+      {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
+        float acc[DK / 32][DV / 16];
+        zero(acc);
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
+                                        [&](int kk, int nn) { return US[kk * LDV + nn]; });
+        for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
+          SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
+        });
+      }
     }
   }
 }
@@ -629,42 +705,115 @@ __global__ void __launch_bounds__(NTF, 1)
       kS[r * LDK + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
-    {  // dU = A_qk^T dO' + Kc dS
-      float acc[1][DV / 16];
-      zero(acc);
-      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
-                               [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
-      mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
-                                [&](int kk, int nn) { return dSS[kk * LDV + nn]; });
-      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { dUS[m * LDV + nn] = acc[i][j]; });
-    }
-    __syncthreads();
-    {  // W = T^T dU  (= dv)
-      float acc[1][DV / 16];
-      zero(acc);
-      mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
-                               [&](int kk, int nn) { return dUS[kk * LDV + nn]; });
-      for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) {
-        WS[m * LDV + nn] = acc[i][j];
-        if (m < n) dv[(rowbase + (size_t)m * H) * DV + nn] = acc[i][j];
-      });
-    }
-    __syncthreads();
-    for (int idx = tid; idx < C * DV; idx += NTF) {
-      const int r = idx / DV, j = idx % DV;
-      w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
-      w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
-    }
-    {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
-      float acc[DK / 32][DV / 16];
-      zero(acc);
-      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
-                                      [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
-      mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
-                                      [&](int kk, int nn) { return WS[kk * LDV + nn]; });
-      for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
-        dSS[m * LDV + nn] = fmaf(eC[m], dSS[m * LDV + nn], acc[i][j]);
-      });
+    if constexpr (DK == 128 && DV == 128) {
+      // tensor cores, tiles owned as in pass F
+      const int wp = tid >> 5, mt = wp >> 3, nt0 = 2 * (wp & 7);
+      const int mt8 = wp >> 1, nt8 = 8 * (wp & 1);
+      {  // dU = A_qk^T dO' + Kc dS
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a<true>(a, AqS, LDC, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, dOS, LDV, 8 * (nt0 + q2), k0);
+        }
+        for (int k0 = 0; k0 < DK; k0 += 8) {
+          Frag3 a;
+          load_a(a, kS, LDK, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, dSS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dUS[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] = acc[q2][e];
+      }
+      __syncthreads();
+      {  // W = T^T dU  (= dv)
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a<true>(a, TS, LDC, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, dUS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int m = frag_row(16 * mt, e), nn = frag_col(8 * (nt0 + q2), e);
+            WS[m * LDV + nn] = acc[q2][e];
+            if (m < n) dv[(rowbase + (size_t)m * H) * DV + nn] = acc[q2][e];
+          }
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DV; idx += NTF) {
+        const int r = idx / DV, j = idx % DV;
+        w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
+        w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
+      }
+      {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
+        float acc[8][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a, b;
+          load_a<true>(a, qS, LDK, 16 * mt8, k0);
+          load_a<true>(b, GS, LDK, 16 * mt8, k0, -1.f);
+#pragma unroll
+          for (int q2 = 0; q2 < 8; ++q2) {
+            mma3<true>(acc[q2], a, dOS, LDV, 8 * (nt8 + q2), k0);
+            mma3<true>(acc[q2], b, WS, LDV, 8 * (nt8 + q2), k0);
+          }
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 8; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = frag_row(16 * mt8, e), j = frag_col(8 * (nt8 + q2), e);
+            dSS[i * LDV + j] = fmaf(eC[i], dSS[i * LDV + j], acc[q2][e]);
+          }
+      }
+    } else {
+      {  // dU = A_qk^T dO' + Kc dS
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
+                                 [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
+        mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
+                                  [&](int kk, int nn) { return dSS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { dUS[m * LDV + nn] = acc[i][j]; });
+      }
+      __syncthreads();
+      {  // W = T^T dU  (= dv)
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
+                                 [&](int kk, int nn) { return dUS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) {
+          WS[m * LDV + nn] = acc[i][j];
+          if (m < n) dv[(rowbase + (size_t)m * H) * DV + nn] = acc[i][j];
+        });
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DV; idx += NTF) {
+        const int r = idx / DV, j = idx % DV;
+        w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
+        w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
+      }
+      {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
+        float acc[DK / 32][DV / 16];
+        zero(acc);
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
+                                        [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
+                                        [&](int kk, int nn) { return WS[kk * LDV + nn]; });
+        for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
+          dSS[m * LDV + nn] = fmaf(eC[m], dSS[m * LDV + nn], acc[i][j]);
+        });
+      }
     }
   }
   __syncthreads();
