@@ -692,7 +692,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
         line["backward"] = {
             "workload": "backward B8 H32 T4096 d128, bf16 q/k/v/dout, fp32 gradients",
             "value": round(ntok / (ms * 1e-3) / 1e6, 4), "unit": "Mtokens/s",
-            "ms_per_launch": round(ms, 3),
+            "ms_per_call": round(ms, 3),
             "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
                          "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
                          "kernel": "bwd_keyside + bwd_fwd_scan + bwd_state_grad_scan + bwd_chunk_grads "
