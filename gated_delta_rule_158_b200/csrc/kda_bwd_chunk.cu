@@ -311,7 +311,8 @@ __global__ void __launch_bounds__(kPlanThreads)
 // the chunk's decays let every factor e^{+-(Gamma_r - Gamma_15)} stay below
 // e^80 (always, for the gate's g >= -5): L = (k e^{Gamma - Gamma_15})
 // (k e^{Gamma_15 - Gamma})^T; otherwise each entry takes exponentials of
-// differences Gamma_r - Gamma_s <= 0.
+// differences Gamma_r - Gamma_s <= 0.  The products run on the tensor cores
+// (tf32 with the hi/lo split, fp32 accuracy).
 template <int DK>
 struct KSmem {
   static constexpr int LDK = DK + 1;
@@ -365,17 +366,28 @@ __global__ void __launch_bounds__(NTH, 2)
       qS[r * LDK + i] *= ea;
     }
     __syncthreads();
-    float lk[2][2], lq[2][2];
-    zero(lk);
-    zero(lq);
-    mm<C, C, 2, 2, DK>(lk, [&](int m, int kk) { return FaS[m * LDK + kk]; },
-                       [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
-    mm<C, C, 2, 2, DK>(lq, [&](int m, int kk) { return qS[m * LDK + kk]; },
-                       [&](int kk, int nn) { return FbS[nn * LDK + kk]; });
-    for_tile<C, C, 2, 2>([&](int r, int s2, int i, int j) {
-      LS[r * LDC + s2] = s2 < r ? lk[i][j] : 0.f;
-      AqS[r * LDC + s2] = s2 <= r ? lq[i][j] : 0.f;
-    });
+    // on the tensor cores: warp w takes two 16 x 8 tiles of L (w < 4) or of
+    // A_qk (w >= 4): rows 16 ((w & 3) >> 1), columns 16 (w & 1) + {0, 8}
+    const int wp = tid >> 5, mt = (wp & 3) >> 1, nt0 = 2 * (wp & 1);
+    const float* Aop = wp < 4 ? FaS : qS;
+    float acc[2][4];
+    zero(acc);
+    for (int k0 = 0; k0 < DK; k0 += 8) {
+      Frag3 a;
+      load_a(a, Aop, LDK, 16 * mt, k0);
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) mma3(acc[q2], a, FbS, LDK, 8 * (nt0 + q2), k0);
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frag_row(16 * mt, e), s2 = frag_col(8 * (nt0 + q2), e);
+        if (wp < 4)
+          LS[r * LDC + s2] = s2 < r ? acc[q2][e] : 0.f;
+        else
+          AqS[r * LDC + s2] = s2 <= r ? acc[q2][e] : 0.f;
+      }
   } else {
     for (int p = tid; p < C * C; p += NTH) {
       const int r = p / C, s2 = p % C;
