@@ -195,7 +195,7 @@ def dist_setup():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    else:
+    elif torch.cuda.is_available():  # the reference arm also runs on a host without a GPU
         torch.cuda.set_device(0)
     return world, rank, local
 
