@@ -20,8 +20,10 @@ backward(q, k, v, g, beta, dout, ...)
 gate_backward(z, A_log, dg, g_min=-5.0)
     dz and dA_log from dg through the gate (chain rule of the gate formula).
 
-Every function is pinned by tests/test_oracle_pins.py (closed forms,
-invariants, brute-force product form, special cases).
+Every function is pinned: gate and forward by tests/test_oracle_pins.py
+(closed forms, invariants, brute-force product form, special cases), the two
+backward functions by tests/test_oracle_backward_pins.py (central finite
+differences of the forward functions, closed forms).
 """
 import ctypes
 import os
