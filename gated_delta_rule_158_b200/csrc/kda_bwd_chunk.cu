@@ -852,6 +852,7 @@ struct BSmem {
   static constexpr int loop = 2 * DK * LDBB + 5 * C * LDBB;
   static constexpr int after = C * LDK + C * LDC;
   static_assert(after <= loop, "post-loop tiles fit the loop tiles");
+  static_assert(2 * C * LDK <= loop, "dGamma and the k e^{Gamma_15 - Gamma} factor fit the loop tiles");
   static constexpr int floats = 3 * C * LDK      // q, k, Gamma
                                 + loop
                                 + 4 * C * LDC    // X, L, dA_qk, dT (then dM)
@@ -901,6 +902,15 @@ __global__ void __launch_bounds__(NTH, 2)
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
   load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  // the factorised backward through the Gram matrices scales sums of up to C
+  // terms of size e^{|Gamma_r - Gamma_15|} |dL| by the opposite factor, so it
+  // takes the chunk only while every |Gamma_r - Gamma_15| stays below 60
+  bool wide = false;
+  for (int i = tid; i < DK; i += NTH) {
+    const float g15 = GS[MREB * LDK + i];
+    for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - g15) > 60.f;
+  }
+  wide = __syncthreads_or(wide);
   for (int idx = tid; idx < C * C; idx += NTH) {
     const int r = idx / C, s = idx % C;
     const size_t o = ((size_t)c * C + r) * C + s;
@@ -1138,41 +1148,96 @@ __global__ void __launch_bounds__(NTH, 2)
   }
   __syncthreads();
   // through E: L_rs = sum_i k_ri k_si E_rsi, A_qk,rs = sum_i q_ri k_si E_rsi.
-  // Row side (thread of channel i owns rows r = part, part + P, ...):
-  //   a_k = sum_{s<=r} dL_rs k_si E_rsi, a_q = sum_s dA_qk,rs k_si E_rsi;
-  //   dk_ri += a_k, dq_ri += a_q, dGamma_ri += k_ri a_k + q_ri a_q.
-  // Column side (owns columns s): c_k = sum_{r>=s} (dL_rs k_ri + dA_qk,rs q_ri) E_rsi;
-  //   dk_si += c_k, dGamma_si -= k_si c_k.  Each element has one writer, in a
-  //   fixed order, so the result does not depend on scheduling.
-  {
-    constexpr int P = NTH / DK;
-    const int i = tid % DK, part = tid / DK;
-    for (int r = part; r < C; r += P) {
-      const float Gr = GS[r * LDK + i];
-      float ak_ = 0.f, aq_ = 0.f;
-      for (int s2 = 0; s2 <= r; ++s2) {
-        const float ke = kS[s2 * LDK + i] * expf(Gr - GS[s2 * LDK + i]);
-        ak_ = fmaf(dTS[r * LDC + s2], ke, ak_);
-        aq_ = fmaf(dAqS[r * LDC + s2], ke, aq_);
-      }
-      const float kr = kS[r * LDK + i], qr = qS[r * LDK + i];
-      if (r < n) {
-        const size_t o = (rowbase + (size_t)r * H) * DK + i;
-        dk[o] += ak_;
-        dq[o] += aq_;
-      }
-      aG[r * LDK + i] += fmaf(kr, ak_, qr * aq_);
+  // Row side of element (r, i): a_k = sum_{s<=r} dL_rs k_si E_rsi and
+  // a_q = sum_s dA_qk,rs k_si E_rsi (dk += a_k, dq += a_q, dGamma += k a_k +
+  // q a_q); column side: c_k = sum_{r>=s} (dL_rs k_ri + dA_qk,rs q_ri) E_rsi
+  // (dk += c_k, dGamma -= k c_k).
+  if (!wide) {
+    // E_rsi = a_ri b_si with a = e^{Gamma - Gamma_15}, b = 1 / a, so with
+    // Ka' = k a, Qa' = q a, Kb' = k b:  a_k = a (dL Kb'), a_q = a (dA_qk Kb'),
+    // c_k = b (dL^T Ka' + dA_qk^T Qa'), three C x DK products on the tensor
+    // cores; warp w owns rows 16 (w >> 2) and DK / 32 column tiles of all three,
+    // so each element has one writer.
+    float* KbS = aG + C * LDK;  // the scratch tile is dead: k e^{Gamma_15 - Gamma}
+    for (int idx = tid; idx < C * DK; idx += NTH) {
+      const int r = idx / DK, i = idx % DK;
+      const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+      const float ea = expf(d), eb = expf(-d), kv = kS[r * LDK + i];
+      KbS[r * LDK + i] = kv * eb;
+      kS[r * LDK + i] = kv * ea;   // Ka'
+      qS[r * LDK + i] *= ea;       // Qa'
     }
     __syncthreads();
-    for (int s2 = part; s2 < C; s2 += P) {
-      const float Gs = GS[s2 * LDK + i];
-      float ck = 0.f;
-      for (int r = s2; r < C; ++r) {
-        const float f = fmaf(dTS[r * LDC + s2], kS[r * LDK + i], dAqS[r * LDC + s2] * qS[r * LDK + i]);
-        ck = fmaf(f, expf(GS[r * LDK + i] - Gs), ck);
+    constexpr int NTW = DK / 32;  // column tiles per warp
+    const int wp = tid >> 5, mt = wp >> 2, nt0 = NTW * (wp & 3);
+    float p1[NTW][4], p2[NTW][4], p3[NTW][4];
+    zero(p1);
+    zero(p2);
+    zero(p3);
+    for (int k0 = 0; k0 < C; k0 += 8) {
+      Frag3 al, aa, alt, aat;
+      load_a(al, dTS, LDC, 16 * mt, k0);
+      load_a(aa, dAqS, LDC, 16 * mt, k0);
+      load_a<true>(alt, dTS, LDC, 16 * mt, k0);
+      load_a<true>(aat, dAqS, LDC, 16 * mt, k0);
+#pragma unroll
+      for (int q2 = 0; q2 < NTW; ++q2) {
+        const int col0 = 8 * (nt0 + q2);
+        mma3<true>(p1[q2], al, KbS, LDK, col0, k0);
+        mma3<true>(p2[q2], aa, KbS, LDK, col0, k0);
+        mma3<true>(p3[q2], alt, kS, LDK, col0, k0);
+        mma3<true>(p3[q2], aat, qS, LDK, col0, k0);
       }
-      if (s2 < n) dk[(rowbase + (size_t)s2 * H) * DK + i] += ck;
-      aG[s2 * LDK + i] -= kS[s2 * LDK + i] * ck;
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frag_row(16 * mt, e), i = frag_col(8 * (nt0 + q2), e);
+        const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+        const float ea = expf(d), eb = expf(-d);
+        if (r < n) {
+          const size_t o = (rowbase + (size_t)r * H) * DK + i;
+          dk[o] += fmaf(ea, p1[q2][e], eb * p3[q2][e]);
+          dq[o] += ea * p2[q2][e];
+        }
+        // k a_k + q a_q - k c_k = Ka' P1 + Qa' P2 - Kb' P3
+        aG[r * LDK + i] += fmaf(kS[r * LDK + i], p1[q2][e],
+                                fmaf(qS[r * LDK + i], p2[q2][e], -KbS[r * LDK + i] * p3[q2][e]));
+      }
+  } else {
+    // exponentials of differences, by element owner: thread of channel i owns
+    // rows r = part, part + P, ... (row side), then columns (column side)
+    {
+      constexpr int P = NTH / DK;
+      const int i = tid % DK, part = tid / DK;
+      for (int r = part; r < C; r += P) {
+        const float Gr = GS[r * LDK + i];
+        float ak_ = 0.f, aq_ = 0.f;
+        for (int s2 = 0; s2 <= r; ++s2) {
+          const float ke = kS[s2 * LDK + i] * expf(Gr - GS[s2 * LDK + i]);
+          ak_ = fmaf(dTS[r * LDC + s2], ke, ak_);
+          aq_ = fmaf(dAqS[r * LDC + s2], ke, aq_);
+        }
+        const float kr = kS[r * LDK + i], qr = qS[r * LDK + i];
+        if (r < n) {
+          const size_t o = (rowbase + (size_t)r * H) * DK + i;
+          dk[o] += ak_;
+          dq[o] += aq_;
+        }
+        aG[r * LDK + i] += fmaf(kr, ak_, qr * aq_);
+      }
+      __syncthreads();
+      for (int s2 = part; s2 < C; s2 += P) {
+        const float Gs = GS[s2 * LDK + i];
+        float ck = 0.f;
+        for (int r = s2; r < C; ++r) {
+          const float f = fmaf(dTS[r * LDC + s2], kS[r * LDK + i], dAqS[r * LDC + s2] * qS[r * LDK + i]);
+          ck = fmaf(f, expf(GS[r * LDK + i] - Gs), ck);
+        }
+        if (s2 < n) dk[(rowbase + (size_t)s2 * H) * DK + i] += ck;
+        aG[s2 * LDK + i] -= kS[s2 * LDK + i] * ck;
+      }
     }
   }
   __syncthreads();
