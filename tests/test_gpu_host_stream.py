@@ -1,6 +1,6 @@
 """GPU parity of the host-buffer prefill (kda_chunk_fwd_gated_host): inputs in
 page-locked host memory, streamed through the device in time slices with the
-state carried across slices.  Checked against the fp64 oracle (the benchmark spec's
+state carried across slices.  Checked against the fp64 oracle (the parity
 bars: rel-L2 1e-5 for fp32 inputs, 2e-2 on o and 1e-2 on the final state for
 bf16 inputs) and against the device-buffer entry on the same inputs.
 Outputs start as NaN, so an element never copied back fails."""
