@@ -279,3 +279,13 @@ def test_gate_backward_rejects_on_host(L):
     assert L.kda_gate_bwd(*args(dz=ptr(3) + 8)) == kda.KDA_ERR_MISALIGNED
     assert L.kda_gate_bwd(*args(dz=ptr(0))) == kda.KDA_ERR_INVALID_ARG   # dz aliases z
     assert L.kda_gate_bwd(*args(dA=ptr(3))) == kda.KDA_ERR_INVALID_ARG   # dA_log aliases dz
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without libkda.so every entry point raises."""
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libkda.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(RuntimeError, match="libkda.so not found"):
+        _lib.lib()
+    with pytest.raises(RuntimeError):
+        kda.kda_status_string(0)
