@@ -55,8 +55,10 @@ WORKLOADS = {
 # bytes per (token, head) of the chunkwise forward, bf16 q/k/v/o, fp32 g/beta:
 # q, k, v 3*256 + g 512 + beta 4 + o 256
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 4 + 256
-# FLOPs per (token, head) of the chunk form (C = 32 on the tensor-core path)
-# counted once: C(3dk + 2dv) + C^2/3 + 6 dk dv
+# FLOPs per (token, head) of the chunk form counted once:
+# C(3dk + 2dv) + C^2/3 + 6 dk dv.  The tensor-core kernel runs C = 32
+# (118,869 at d = 128); the reference count of the measurement plan is taken
+# at C = 64 (140,629).  Both are reported.
 def prefill_flops_per_token_head(C=32, dk=128, dv=128):
     return C * (3 * dk + 2 * dv) + C * C / 3 + 6 * dk * dv
 
@@ -572,6 +574,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-long", action="store_true",
+                    help="leave the 1M-token prefill out of the default line")
+    ap.add_argument("--no-varlen", action="store_true",
+                    help="leave the varlen prefill out of the default line")
     ap.add_argument("--no-clocks", action="store_true",
                     help="skip nvidia-smi clock sampling (profiling runs)")
     ap.add_argument("--batch", type=int, default=None,
@@ -611,44 +617,65 @@ def main():
         dist.destroy_process_group()
 
 
-def bench_prefill_line(args, wl, world, rank, peaks):
-    dev = torch.device("cuda", torch.cuda.current_device())
+def measure_prefill(wl, dev, steps, warmup, world, with_clocks):
+    """Times `steps` gated chunkwise-forward steps of workload `wl` on resident
+    inputs; returns the inputs, the step and the measured figures."""
     inp, cu, T, N = make_prefill(wl, dev)
     H, dk, dv = wl["H"], wl["dk"], wl["dv"]
     B = inp["q"].shape[0]
-    tokens = B * T  # per rank
     step = PrefillStep(inp, cu, N)
-    clocks = None if args.no_clocks else ClockSampler(dev.index)
-    total_ms, chunk_ms = time_steps(step, args.steps, args.warmup, world)
+    clocks = ClockSampler(dev.index) if with_clocks else None
+    total_ms, chunk_ms = time_steps(step, steps, warmup, world)
     clk = clocks.extend_window(step) if clocks else None
     st, _ = kda.kda_get_device_status(step.ws)
     if st != kda.KDA_OK:
         raise RuntimeError(f"device status {kda.kda_status_string(st)}")
-    ms_per_step = total_ms / args.steps
-    value = tokens * world / (ms_per_step * 1e-3) / 1e6
+    ms_per_step = total_ms / steps
+    tokens = B * T  # per rank
     tok_heads = tokens * H
     alg_bytes = tok_heads * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * dk * dv * 4 * (
         2 if inp["init_state"] is not None else 1)
     achieved = alg_bytes / (chunk_ms * 1e-3) / 1e9
-    flops = tok_heads * prefill_flops_per_token_head(32, dk, dv)
+    return dict(inp=inp, cu=cu, T=T, N=N, B=B, H=H, dk=dk, dv=dv, step=step, clk=clk,
+                ms_per_step=ms_per_step, chunk_ms=chunk_ms, tokens=tokens, tok_heads=tok_heads,
+                alg_bytes=alg_bytes, achieved=achieved,
+                value=tokens * world / (ms_per_step * 1e-3) / 1e6)
+
+
+def prefill_roofline(m, peaks, wl):
+    dk, dv = m["dk"], m["dv"]
+    f32 = m["tok_heads"] * prefill_flops_per_token_head(32, dk, dv)
+    f64 = m["tok_heads"] * prefill_flops_per_token_head(64, dk, dv)
+    secs = m["chunk_ms"] * 1e-3
+    return {"bound": "hbm", "achieved": round(m["achieved"], 1), "peak": peaks["hbm"],
+            "unit": "GB/s", "frac": round(m["achieved"] / peaks["hbm"], 4),
+            "traffic": chunk_traffic(m["B"], m["H"], m["T"]) if not wl.get("varlen") else None,
+            "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
+            "kernel_ms": round(m["chunk_ms"], 4), "algorithmic_bytes": m["alg_bytes"],
+            "peak_source": peaks["src"],
+            "tensor_frac": round(f32 / secs / (peaks["tc"] * 1e12), 4),
+            "tensor_flops_count": "C(3dk+2dv)+C^2/3+6dk dv per token-head at C=32 "
+                                  "(the chunk the kernel runs)",
+            "tensor_frac_c64_count": round(f64 / secs / (peaks["tc"] * 1e12), 4)}
+
+
+def bench_prefill_line(args, wl, world, rank, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    m = measure_prefill(wl, dev, args.steps, args.warmup, world, not args.no_clocks)
+    inp, cu, T, N, B, H = m["inp"], m["cu"], m["T"], m["N"], m["B"], m["H"]
+    dk, dv, step, tokens = m["dk"], m["dv"], m["step"], m["tokens"]
     line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "Mtokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "metric": METRIC, "value": round(m["value"], 3), "unit": "Mtokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(m["ms_per_step"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T,
                    "heads": H, "dk": dk, "dv": dv, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (no flush needed)",
                    "step": "kda_chunk_fwd_gated (gate fused)"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
-                     "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                     "traffic": chunk_traffic(B, H, T) if not wl.get("varlen") else None,
-                     "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
-                     "kernel_ms": round(chunk_ms, 4), "algorithmic_bytes": alg_bytes,
-                     "peak_source": peaks["src"],
-                     "tensor_frac": round(flops / (chunk_ms * 1e-3) / (peaks["tc"] * 1e12), 4)},
+        "roofline": prefill_roofline(m, peaks, wl),
         "gpu_launches": args.steps * kernels_per_step(wl, B, T),
-        "clocks": clk,
+        "clocks": m["clk"],
     }
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_prefill(wl, inp, cu, N, max(2, min(args.steps, 5)))
@@ -659,10 +686,31 @@ def bench_prefill_line(args, wl, world, rank, peaks):
         v, cores, sample, secs = oracle_prefill_parallel_sample(wl, inp, cu, budget_s=15.0)
         line["cpu_baseline"] = {"value": round(v / 1e6, 6), "unit": "Mtokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample + f", {secs:.1f} s"}
+    del step, inp, m
+    torch.cuda.empty_cache()
+    if args.workload == "prefill":
+        for name, skip, steps in (("long", args.no_long, 3), ("varlen", args.no_varlen, 10)):
+            if skip:
+                continue
+            swl = WORKLOADS[name]
+            sm = measure_prefill(swl, dev, steps, 3, world, not args.no_clocks)
+            nk = kernels_per_step(swl, sm["B"], sm["T"])
+            roof = prefill_roofline(sm, peaks, swl)
+            if nk == 3:
+                roof["kernel"] = ("chunk_tc_kernel (segment transitions) + segment_combine_kernel + "
+                                  "chunk_tc_kernel (segment outputs): one kda_chunk_fwd_gated call")
+            elif swl.get("varlen"):
+                roof["kernel"] = "varlen_plan_kernel + chunk_tc_kernel (kda_chunk_fwd_gated)"
+            line[name] = {
+                "workload": swl["name"], "value": round(sm["value"], 3), "unit": "Mtokens/s",
+                "steps": steps, "warmup": 3, "ms_per_step": round(sm["ms_per_step"], 4),
+                "tokens_per_step": sm["tokens"], "heads": sm["H"],
+                "roofline": roof, "gpu_launches": steps * nk,
+                "clocks": sm["clk"]}
+            del sm
+            torch.cuda.empty_cache()
     if not args.no_decode and args.workload == "prefill":
         dwl = WORKLOADS["decode"]
-        del step, inp
-        torch.cuda.empty_cache()
         total, dec_ms, bpl = run_decode(dwl, dev)
         dach = bpl / (dec_ms * 1e-3) / 1e9
         line["decode"] = {"workload": dwl["name"], "value": round(dwl["steps"] / (total * 1e-3), 2),

@@ -61,6 +61,7 @@ _SIGNATURES = {
     "kda_recurrent_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _I,
                                _I, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
+    "kda_noalloc_get_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _VP]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
 }
 
@@ -313,6 +314,14 @@ def kda_get_device_status(workspace, stream=None):
     """(status, detail) recorded on the device in this workspace; syncs the stream."""
     detail = ctypes.c_int32(0)
     st = lib().kda_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+def kda_noalloc_get_device_status(stream=None):
+    """(status, detail) that the last kda_chunk_fwd_noalloc call on the current
+    device recorded in the library's built-in scratch; syncs the stream."""
+    detail = ctypes.c_int32(0)
+    st = lib().kda_noalloc_get_device_status(ctypes.byref(detail), _stream(stream))
     return int(st), int(detail.value)
 
 

@@ -882,17 +882,27 @@ __global__ void __launch_bounds__(256) state_prefix_kernel(const float* __restri
 }
 
 // ------------------------------------------------------------------- host
+// The driver's entry point is the same for every device; the function-local
+// static is initialised once, thread-safely.
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
+}
+
+// The shared-memory limit is a per-device attribute of the kernel: set it on
+// every launch (a cheap host call) so that any device the caller makes
+// current gets it, from any host thread.
+cudaError_t allow_chunk_smem() {
+  return cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SMEM_ALLOC);
 }
 
 bool encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base, int H,
@@ -954,12 +964,9 @@ size_t tc_workspace_bytes(int B, int T, int H, int num_seqs, int num_sms) {
 cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_bytes,
                             cudaStream_t stream) {
   if (a.num_units == 0) return cudaSuccess;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  {
+    const cudaError_t e = allow_chunk_smem();
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   TcParams P;
   memset(&P, 0, sizeof(P));
@@ -1017,12 +1024,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_by
 
 cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStream_t stream) {
   if (a.num_units == 0) return cudaSuccess;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  {
+    const cudaError_t e = allow_chunk_smem();
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   TcParams P;
   memset(&P, 0, sizeof(P));

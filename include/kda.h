@@ -382,11 +382,13 @@ KDA_API kda_status kda_selftest_bounded_wait(void *workspace, int64_t spin_limit
  * enqueued.  All calls share that array, so calls whose GPU work overlaps
  * race and must be serialised by the caller.  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress) with that
- * device current: make it before any stream capture.  Device-side status
- * (KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT) is recorded in the built-in array
- * and is not reachable through kda_get_device_status; validate cu_seqlens on
- * the host when using this entry point.  Returns KDA_ERR_CUDA if no device
- * is current.
+ * device current: make it before any stream capture.  If the device is
+ * reset (cudaDeviceReset), the next call sees a new context and looks the
+ * address up again.  Device-side status (KDA_ERR_BAD_SEQLENS,
+ * KDA_ERR_TIMEOUT) is recorded in the built-in array, where
+ * kda_noalloc_get_device_status reads it; with malformed cu_seqlens no unit
+ * runs and out / final_state are left as they were.  Returns KDA_ERR_CUDA if
+ * no device is current.
  */
 #define KDA_NOALLOC_SCRATCH_BYTES (8u << 20)
 
@@ -397,6 +399,16 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
                                  int T, int H, int dk, int dv, float scale,
                                  int chunk_size, void *out, float *final_state,
                                  void *stream);
+
+/*
+ * The device status word of the last kda_chunk_fwd_noalloc call on the
+ * current device: synchronises `stream`, then reads the status the kernels
+ * recorded in the built-in scratch (KDA_OK if none), exactly as
+ * kda_get_device_status does for a workspace; `detail` (nullable) receives
+ * the code-specific value.  The pages have no counterpart.  Allocates
+ * nothing.  Returns KDA_ERR_CUDA if the synchronisation or the read failed.
+ */
+KDA_API kda_status kda_noalloc_get_device_status(int32_t *detail, void *stream);
 
 #ifdef __cplusplus
 }
