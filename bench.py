@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import gated_delta_rule_158_b200 as kda  # noqa: E402
+from gated_delta_rule_158_b200 import kcp  # noqa: E402
 from gated_delta_rule_158_b200 import workloads as W  # noqa: E402
 
 METRIC = "KDA prefill Mtokens/s & decode steps/s on 1 B200; % of TC / HBM roofline"
@@ -351,6 +352,83 @@ def e2e_prefill(wl, inp, cu, N, K):
     return a.elapsed_time(b) / K, h2d, d2h
 
 
+# --------------------------------------------- context parallelism (KCP)
+def kcp_segment_inputs(wl, rank, world, device, dtype=torch.bfloat16):
+    """This rank's segment of the long workload's sequence (whole 32-token
+    chunks in token order, kcp.segment_bounds).  Each rank draws only its own
+    segment (seed derived from the rank), with the workload's shapes and
+    distributions; the per-head gate parameter A_log is drawn from a seed
+    shared by all ranks, as one sequence has one A_log."""
+    s, e = kcp.segment_bounds(wl["T"], world)[rank]
+    seg = W.make_prefill_inputs(1, e - s, wl["H"], wl["dk"], wl["dv"], dtype,
+                                seed=wl["seed"] * 1000 + 1 + rank, device=device)
+    shared = W.make_prefill_inputs(1, 1, wl["H"], wl["dk"], wl["dv"], dtype,
+                                   seed=wl["seed"] * 1000, device=device)
+    seg["A_log"] = shared["A_log"]
+    return seg, (s, e)
+
+
+class KcpStep:
+    """One step of the long workload split across the ranks: kcp_prefill on
+    this rank's segment (segment transition, one all-gather of the pairs,
+    prefix fold, segment outputs)."""
+
+    def __init__(self, seg, backend=None, group=None):
+        self.seg, self.backend, self.group = seg, backend, group
+        self.o = self.S = None
+
+    def __call__(self, ev=None):
+        if ev:
+            ev[0].record()
+        self.o, self.S = kcp.kcp_prefill(self.seg, init_state=None, group=self.group,
+                                         backend=self.backend)
+        if ev:
+            ev[1].record()
+
+
+def bench_kcp_line(args, wl, world, rank, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if world == 1:  # kcp_prefill needs a process group, even of one rank
+        import datetime
+        import torch.distributed as dist
+        if not dist.is_initialized():
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29533")
+            dist.init_process_group("nccl", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=120),
+                                    device_id=dev)
+    seg, (s, e) = kcp_segment_inputs(wl, rank, world, dev)
+    step = KcpStep(seg)
+    clocks = None if args.no_clocks else ClockSampler(dev.index)
+    total_ms, step_ms = time_steps(step, args.steps, args.warmup, world)
+    clk = clocks.stop() if clocks else None
+    step_ms = max_over_ranks(step_ms, world)
+    ms = total_ms / args.steps
+    T, H, dk, dv = wl["T"], wl["H"], wl["dk"], wl["dv"]
+    alg = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * dk * dv * 4
+    ach = alg / (step_ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC, "value": round(T / (ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (each rank draws its own segment)",
+        "config": {"workload": wl["name"] + " (KCP)", "global_batch": 1, "seq_len": T,
+                   "heads": H, "dk": dk, "dv": dv,
+                   "parallelism": f"kcp{world} (one sequence split over the ranks; "
+                                  "one all-gather of 2 x 64 KB per head per rank)",
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "step": "kcp.kcp_prefill: kda_chunk_segment_transition, all_gather, "
+                           "kda_chunk_state_prefix, kda_chunk_fwd_gated"},
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"] * world,
+                     "unit": "GB/s", "frac": round(ach / (peaks["hbm"] * world), 4),
+                     "traffic": None, "kernel": "whole KCP step, all ranks",
+                     "kernel_ms": round(step_ms, 4), "algorithmic_bytes": alg,
+                     "peak_source": peaks["src"] + " (x ranks)"},
+        "gpu_launches": args.steps * ((2 if world > 1 else 0) + 1 + 3),
+        "clocks": clk,
+    }
+
+
 # ----------------------------------------------------------------- decode
 def run_decode(wl, device, warmup=3):
     N, H, dk, dv, steps = wl["N"], wl["H"], wl["dk"], wl["dv"], wl["steps"]
@@ -574,6 +652,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--kcp", action="store_true",
+                    help="with --workload long: split the one sequence across the torchrun "
+                         "ranks (context parallelism) instead of replicating it")
     ap.add_argument("--no-long", action="store_true",
                     help="leave the 1M-token prefill out of the default line")
     ap.add_argument("--no-varlen", action="store_true",
@@ -603,7 +684,11 @@ def main():
             dist.destroy_process_group()
         return
 
-    if args.workload == "decode":
+    if args.kcp and args.workload != "long":
+        ap.error("--kcp applies to --workload long")
+    if args.kcp:
+        line = bench_kcp_line(args, wl, world, rank, peaks)
+    elif args.workload == "decode":
         line = bench_decode_line(args, wl, world, rank, peaks)
     elif args.workload == "backward":
         line = bench_backward_line(args, wl, world, rank, peaks)
@@ -611,8 +696,8 @@ def main():
         line = bench_prefill_line(args, wl, world, rank, peaks)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
+    import torch.distributed as dist
+    if dist.is_initialized():
         dist.barrier()
         dist.destroy_process_group()
 

@@ -13,5 +13,6 @@ from ._lib import (  # noqa: F401
     kda_decode_replay, kda_decode_step_gated, kda_decode_verify, kda_gate_bwd,
     kda_gate_bwd_workspace_size, kda_gate_fwd,
     kda_get_device_status, kda_last_cuda_error_string, kda_noalloc_get_device_status, kda_recurrent_bwd,
-    kda_recurrent_bwd_workspace_size, kda_selftest_bounded_wait, kda_status_string,
+    kda_recurrent_bwd_workspace_size, kda_selftest_bounded_wait, kda_set_wait_limit_ns,
+    kda_status_string,
     lib)

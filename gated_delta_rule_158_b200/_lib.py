@@ -63,6 +63,7 @@ _SIGNATURES = {
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_noalloc_get_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _VP]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
+    "kda_set_wait_limit_ns": (_I, [_I64]),
 }
 
 _lib = None
@@ -323,6 +324,11 @@ def kda_noalloc_get_device_status(stream=None):
     detail = ctypes.c_int32(0)
     st = lib().kda_noalloc_get_device_status(ctypes.byref(detail), _stream(stream))
     return int(st), int(detail.value)
+
+
+def kda_set_wait_limit_ns(limit_ns):
+    """Diagnostic: bound of the chunk kernel's internal waits (default 2e9 ns)."""
+    _check(lib().kda_set_wait_limit_ns(int(limit_ns)), "kda_set_wait_limit_ns")
 
 
 def kda_selftest_bounded_wait(workspace, spin_limit_ns, stream=None):

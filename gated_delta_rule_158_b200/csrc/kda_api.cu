@@ -531,6 +531,14 @@ kda_status kda_get_device_status(const void* workspace, void* stream, int32_t* d
   return (kda_status)host[0];
 }
 
+kda_status kda_set_wait_limit_ns(int64_t limit_ns) {
+  long long lim = limit_ns;
+  if (lim < 0) lim = 0;
+  if (lim > 5000000000LL) lim = 5000000000LL;
+  set_wait_limit_ns(lim);
+  return KDA_OK;
+}
+
 kda_status kda_selftest_bounded_wait(void* workspace, int64_t spin_limit_ns, void* stream) {
   if (!workspace) return KDA_ERR_INVALID_ARG;
   if (!aligned16(workspace)) return KDA_ERR_MISALIGNED;

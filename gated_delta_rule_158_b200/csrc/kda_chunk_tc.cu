@@ -60,6 +60,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "kda_internal.cuh"
 #include "kda_sync.cuh"
 #include "kda_tc_ptx.cuh"
@@ -118,9 +120,9 @@ enum : int {
   B_T = 6,          // [2] T and A_qk written                      (4 solve warps)
   B_UO = 8,         //     [O | P] GEMM done                       (commit)
   B_U = 9,          //     U GEMM done                             (commit)
-  B_DECAY = 10,     //     state decayed for the chunk             (4 state warps)
+  B_DECAY = 10,     //     state decayed for the chunk (with B_OREADY) (4 state warps)
   B_SO = 11,        // [2] [S | O] GEMM done                       (commit)
-  B_OREADY = 13,    //     bf16 S written, O read out, [O | P] seeded (4 state warps)
+  B_OREADY = 13,    //     O read out, [O | P] seeded, bf16 S written (4 state warps)
   B_DRAIN = 14,     //     abort path: every MMA the state issuer issued done (commit)
   B_V = 15,         // [4] TMA v landed                            (tx)
   B_VEMPTY = 19,    // [4] v buffer read                           (4 state warps)
@@ -148,6 +150,7 @@ struct TcParams {
   int G;          // segments per unit (modes 1, 2)
   int seg_len;    // tokens per segment (multiple of C)
   float scale;
+  long long wait_limit_ns;  // bound of every mbarrier wait (lowered only by diagnostics)
 };
 
 struct Unit {
@@ -230,6 +233,10 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM_ABORT);
   const int H = P.H, h = U.h;
   const int nchunks = (int)((U.len + C - 1) / C);
+  // every mbarrier wait of the pipeline: bounded, abort-aware, `where` names it
+  auto wait = [&](uint64_t* bar, uint32_t parity, int32_t where) {
+    return mbar_wait_bounded(bar, parity, abort_flag, P.sb, where, P.wait_limit_ns);
+  };
   auto chunk_rows = [&](int cc) -> int {
     const int64_t rem = U.len - (int64_t)cc * C;
     return (int)(rem < C ? rem : C);
@@ -277,7 +284,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
 
   if (warp < SOLVE_W0) {
     // =============================================================== prep warps
-    // thread: channels c0 .. c0+3, rows 8pw .. 8pw+7
+    // thread: channels c0 .. c0+3, rows 8pw .. 8pw+7; fp32 pairs in packed
+    // f32x2 arithmetic (two lanes of work per instruction)
     const int pw = warp - PREP_W0, c0 = 4 * lane;
     const uint32_t ck16 = ((c0 & 63) * 2) >> 4, lo16 = ((c0 & 63) * 2) & 15;  // bf16 tiles
     const uint32_t o_kql = (c0 >> 6) * 8192 + lo16;
@@ -285,86 +293,104 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
     constexpr float kLog2e = 1.4426950408889634f;
     const float gmin2 = P.g_min * kLog2e;
     const float a2 = P.A_log ? expf(P.A_log[h]) * kLog2e : 0.f;
+    const float2 na2 = make_float2(-a2, -a2), one2 = make_float2(1.f, 1.f);
     float beta_next = 0.f;
     if (pw == 0 && lane < U.len) beta_next = P.beta[(size_t)(U.row0 + lane) * H + h];
+    auto pack = [](float lo_, float hi_) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo_, hi_);
+      return *reinterpret_cast<const uint32_t*>(&b2);
+    };
+    auto bf_lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+    auto bf_hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
 
     for (int c = 0; c < nchunks; ++c) {
-      if (bar_red_or(1, 128, *abort_flag != 0)) break;
       const int st = c & 1, b = c & 1;
       const int n = chunk_rows(c);
       uint8_t* in = sm + st * STAGE;
       uint8_t* kb_buf = sm + SM_KEY + b * KEYB;
       uint8_t* hb = sm + SM_HB + b * HBB;
       const float beta_cur = beta_next;
-      if (pw == 0) {
-        const int64_t t1 = (int64_t)(c + 1) * C + lane;
-        beta_next = (t1 < U.len) ? P.beta[(size_t)(U.row0 + t1) * H + h] : 0.f;
-      }
-      mbar_wait_bounded(&bars[B_IN_FULL + st], (c >> 1) & 1, abort_flag, P.sb, 1);
+      wait(&bars[B_IN_FULL + st], (c >> 1) & 1, 1);
       __syncwarp();
+      if (n < C) {  // tail rows act as k = q = 0 (and g = 0 below)
+#pragma unroll 1
+        for (int rr = 0; rr < 8; ++rr) {
+          const int r = 8 * pw + rr;
+          if (r >= n) {
+            *reinterpret_cast<uint2*>(in + OFF_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2*>(in + OFF_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
+          }
+        }
+      }
 
       // ---- part 1: gate and cumulative log2-decay over rows 8pw .. 8pw+7, written
       //      back in place (only this thread touches these elements)
       {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 acc01 = make_float2(0.f, 0.f), acc23 = acc01;
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
           const int r = 8 * pw + rr;
           float4* gp = reinterpret_cast<float4*>(in + OFF_G + (r * D + c0) * 4);
-          float4 gv = *gp;
+          const float4 gv = *gp;
+          const float2 g01 = make_float2(gv.x, gv.y), g23 = make_float2(gv.z, gv.w);
           if (P.A_log) {  // fused gate: tile holds z; g log2e = g_min log2e sigmoid(e^A z)
-            gv.x = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.x));
-            gv.y = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.y));
-            gv.z = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.z));
-            gv.w = gmin2 * rcp_approx(1.f + ex2_approx(-a2 * gv.w));
+            const float gm = r < n ? gmin2 : 0.f;
+            const float2 gm2 = make_float2(gm, gm);
+            const float2 x01 = __fmul2_rn(g01, na2), x23 = __fmul2_rn(g23, na2);
+            const float2 d01 = __fadd2_rn(make_float2(ex2_approx(x01.x), ex2_approx(x01.y)), one2);
+            const float2 d23 = __fadd2_rn(make_float2(ex2_approx(x23.x), ex2_approx(x23.y)), one2);
+            acc01 = __ffma2_rn(make_float2(rcp_approx(d01.x), rcp_approx(d01.y)), gm2, acc01);
+            acc23 = __ffma2_rn(make_float2(rcp_approx(d23.x), rcp_approx(d23.y)), gm2, acc23);
           } else {
-            gv.x *= kLog2e;
-            gv.y *= kLog2e;
-            gv.z *= kLog2e;
-            gv.w *= kLog2e;
+            const float lm = r < n ? kLog2e : 0.f;
+            const float2 lm2 = make_float2(lm, lm);
+            acc01 = __ffma2_rn(g01, lm2, acc01);
+            acc23 = __ffma2_rn(g23, lm2, acc23);
           }
-          if (r >= n) {  // tail rows act as g = 0, k = q = 0
-            gv = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<uint2*>(in + OFF_K + (r * D + c0) * 2) = make_uint2(0u, 0u);
-            *reinterpret_cast<uint2*>(in + OFF_Q + (r * D + c0) * 2) = make_uint2(0u, 0u);
-          }
-          acc.x += gv.x;
-          acc.y += gv.y;
-          acc.z += gv.z;
-          acc.w += gv.w;
-          *gp = acc;
+          *gp = make_float4(acc01.x, acc01.y, acc23.x, acc23.y);
         }
       }
-      named_bar(1, 128);
+      // every prep warp's partial sums are in; the same barrier agrees on an abort
+      if (bar_red_or(1, 128, *abort_flag != 0)) break;
 
       // ---- part 2: rescaled operands; buffer b is free once chunk c - 2 is
       //      completely done (its [S | O] GEMM is the last reader)
-      if (c >= 2) mbar_wait_bounded(&bars[B_SO + b], ((c - 2) >> 1) & 1, abort_flag, P.sb, 2);
+      if (c >= 2) wait(&bars[B_SO + b], ((c - 2) >> 1) & 1, 2);
       __syncwarp();
+      // beta of the next chunk: issued here, after this chunk's waits, so that no
+      // out-of-line wait call has to hold the pending load
+      if (pw == 0) {
+        const int64_t t1 = (int64_t)(c + 1) * C + lane;
+        beta_next = (t1 < U.len) ? __ldg(P.beta + (size_t)(U.row0 + t1) * H + h) : 0.f;
+      }
       {
-        float4 off = make_float4(0.f, 0.f, 0.f, 0.f), g15 = off, g31 = off;
+        float2 off01 = make_float2(0.f, 0.f), off23 = off01, g15_01 = off01, g15_23 = off01;
+        float2 g31_01 = off01, g31_23 = off01;
 #pragma unroll
         for (int o4 = 0; o4 < 4; ++o4) {  // group totals: the partial sums at rows 8 o4 + 7
           const float4 t =
               *reinterpret_cast<const float4*>(in + OFF_G + ((8 * o4 + 7) * D + c0) * 4);
-          if (o4 < pw) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
-          if (o4 < 2) { g15.x += t.x; g15.y += t.y; g15.z += t.z; g15.w += t.w; }
-          g31.x += t.x; g31.y += t.y; g31.z += t.z; g31.w += t.w;
+          const float2 t01 = make_float2(t.x, t.y), t23 = make_float2(t.z, t.w);
+          if (o4 < pw) { off01 = __fadd2_rn(off01, t01); off23 = __fadd2_rn(off23, t23); }
+          if (o4 < 2) { g15_01 = __fadd2_rn(g15_01, t01); g15_23 = __fadd2_rn(g15_23, t23); }
+          g31_01 = __fadd2_rn(g31_01, t01);
+          g31_23 = __fadd2_rn(g31_23, t23);
         }
-        const float4 e15 = make_float4(ex2_approx(g15.x), ex2_approx(g15.y), ex2_approx(g15.z),
-                                       ex2_approx(g15.w));
-        const float4 e3115 = make_float4(ex2_approx(g31.x - g15.x), ex2_approx(g31.y - g15.y),
-                                         ex2_approx(g31.z - g15.z), ex2_approx(g31.w - g15.w));
+        const float2 e15_01 = make_float2(ex2_approx(g15_01.x), ex2_approx(g15_01.y));
+        const float2 e15_23 = make_float2(ex2_approx(g15_23.x), ex2_approx(g15_23.y));
+        const float2 d31_01 = __fadd2_rn(g31_01, make_float2(-g15_01.x, -g15_01.y));
+        const float2 d31_23 = __fadd2_rn(g31_23, make_float2(-g15_23.x, -g15_23.y));
+        const float2 e3115_01 = make_float2(ex2_approx(d31_01.x), ex2_approx(d31_01.y));
+        const float2 e3115_23 = make_float2(ex2_approx(d31_23.x), ex2_approx(d31_23.y));
         if (pw == 0) {
           *reinterpret_cast<float4*>(sm + SM_GAMC + b * 512 + c0 * 4) = make_float4(
-              ex2_approx(g31.x), ex2_approx(g31.y), ex2_approx(g31.z), ex2_approx(g31.w));
+              ex2_approx(g31_01.x), ex2_approx(g31_01.y), ex2_approx(g31_23.x),
+              ex2_approx(g31_23.y));
           reinterpret_cast<float*>(sm + SM_BETA + b * 128)[lane] = beta_cur;
         }
-        const float4 sh = make_float4(off.x - g15.x, off.y - g15.y, off.z - g15.z, off.w - g15.w);
-        auto pack = [](float lo_, float hi_) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo_, hi_);
-          return *reinterpret_cast<const uint32_t*>(&b2);
-        };
+        // shift of this warp's rows: the earlier groups' totals, re-based at row 15
+        const float2 sh01 = __fadd2_rn(off01, make_float2(-g15_01.x, -g15_01.y));
+        const float2 sh23 = __fadd2_rn(off23, make_float2(-g15_23.x, -g15_23.y));
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
           float kc[4][4];  // [channel][row] of rows 8pw + 4hf .. +3
@@ -372,62 +398,55 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
           for (int r4 = 0; r4 < 4; ++r4) {
             const int r = 8 * pw + 4 * hf + r4;
             const float4 G = *reinterpret_cast<const float4*>(in + OFF_G + (r * D + c0) * 4);
-            float ex[4], ix[4];
-            ex[0] = ex2_approx(G.x + sh.x);
-            ex[1] = ex2_approx(G.y + sh.y);
-            ex[2] = ex2_approx(G.z + sh.z);
-            ex[3] = ex2_approx(G.w + sh.w);
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) ix[k4] = rcp_approx(ex[k4]);
+            const float2 t01 = __fadd2_rn(make_float2(G.x, G.y), sh01);
+            const float2 t23 = __fadd2_rn(make_float2(G.z, G.w), sh23);
+            // e^{G_r - G_15} and its inverse (two independent exponentials)
+            const float2 ex01 = make_float2(ex2_approx(t01.x), ex2_approx(t01.y));
+            const float2 ex23 = make_float2(ex2_approx(t23.x), ex2_approx(t23.y));
+            const float2 ix01 = make_float2(ex2_approx(-t01.x), ex2_approx(-t01.y));
+            const float2 ix23 = make_float2(ex2_approx(-t23.x), ex2_approx(-t23.y));
             const uint2 kw = *reinterpret_cast<const uint2*>(in + OFF_K + (r * D + c0) * 2);
             const uint2 qw = *reinterpret_cast<const uint2*>(in + OFF_Q + (r * D + c0) * 2);
-            const float kv[4] = {__uint_as_float(kw.x << 16), __uint_as_float(kw.x & 0xffff0000u),
-                                 __uint_as_float(kw.y << 16), __uint_as_float(kw.y & 0xffff0000u)};
-            const float qv[4] = {__uint_as_float(qw.x << 16), __uint_as_float(qw.x & 0xffff0000u),
-                                 __uint_as_float(qw.y << 16), __uint_as_float(qw.y & 0xffff0000u)};
-            float kl[4], ql[4], kbv[4];
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              kl[k4] = kv[k4] * ex[k4];
-              ql[k4] = qv[k4] * ex[k4];
-              kbv[k4] = kv[k4] * ix[k4];
-            }
+            const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x));
+            const float2 k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
+            const float2 q01 = make_float2(bf_lo(qw.x), bf_hi(qw.x));
+            const float2 q23 = make_float2(bf_lo(qw.y), bf_hi(qw.y));
+            const float2 kl01 = __fmul2_rn(k01, ex01), kl23 = __fmul2_rn(k23, ex23);
+            const float2 ql01 = __fmul2_rn(q01, ex01), ql23 = __fmul2_rn(q23, ex23);
+            const float2 kb01 = __fmul2_rn(k01, ix01), kb23 = __fmul2_rn(k23, ix23);
+            const float2 qg01 = __fmul2_rn(ql01, e15_01), qg23 = __fmul2_rn(ql23, e15_23);
+            const float2 kg01 = __fmul2_rn(kl01, e15_01), kg23 = __fmul2_rn(kl23, e15_23);
+            const float2 kc01 = __fmul2_rn(kb01, e3115_01), kc23 = __fmul2_rn(kb23, e3115_23);
+            kc[0][r4] = kc01.x;
+            kc[1][r4] = kc01.y;
+            kc[2][r4] = kc23.x;
+            kc[3][r4] = kc23.y;
             const uint32_t sw = (uint32_t)(r & 7);
             const uint32_t s16 = (ck16 ^ sw) << 4;
             // Gram operands (rows 64 hh + r, 64 hh + 32 + r of A and 32 hh + r of B
             // for channel half hh = c0 / 64)
             *reinterpret_cast<uint2*>(kb_buf + K_KQL + o_kql + r * 128 + s16) =
-                make_uint2(pack(kl[0], kl[1]), pack(kl[2], kl[3]));
+                make_uint2(pack(kl01.x, kl01.y), pack(kl23.x, kl23.y));
             *reinterpret_cast<uint2*>(kb_buf + K_KQL + o_kql + (32 + r) * 128 + s16) =
-                make_uint2(pack(ql[0], ql[1]), pack(ql[2], ql[3]));
+                make_uint2(pack(ql01.x, ql01.y), pack(ql23.x, ql23.y));
             *reinterpret_cast<uint2*>(kb_buf + K_KB + o_kb + r * 128 + s16) =
-                make_uint2(pack(kbv[0], kbv[1]), pack(kbv[2], kbv[3]));
+                make_uint2(pack(kb01.x, kb01.y), pack(kb23.x, kb23.y));
             // B of [O | P] (bf16, same layout as the Gram A): q e^G rows 0-31,
             // k e^G rows 32-63 of each 64-channel block
             *reinterpret_cast<uint2*>(hb + H_QK + o_kql + r * 128 + s16) =
-                make_uint2(pack(ql[0] * e15.x, ql[1] * e15.y), pack(ql[2] * e15.z, ql[3] * e15.w));
+                make_uint2(pack(qg01.x, qg01.y), pack(qg23.x, qg23.y));
             *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (32 + r) * 128 + s16) =
-                make_uint2(pack(kl[0] * e15.x, kl[1] * e15.y), pack(kl[2] * e15.z, kl[3] * e15.w));
-            kc[0][r4] = kbv[0] * e3115.x;
-            kc[1][r4] = kbv[1] * e3115.y;
-            kc[2][r4] = kbv[2] * e3115.z;
-            kc[3][r4] = kbv[3] * e3115.w;
+                make_uint2(pack(kg01.x, kg01.y), pack(kg23.x, kg23.y));
           }
-          // Kc^T rows c0..c0+3, one 16-byte chunk each; in step k lane l writes row
-          // c0 + (k + l/2) % 4, so the 8 lanes of a quarter warp hit 8 different
-          // swizzled chunks (no bank conflicts)
+          // Kc^T rows c0..c0+3 (K-major: row = channel, 32 tokens of fp32), the
+          // 16-byte chunk of tokens 8pw + 4hf .. +3 of each
           const uint32_t chunk = (uint32_t)(2 * pw + hf);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int k4 = (k + (lane >> 1)) & 3;
-            float4 w;
-            w.x = k4 == 0 ? kc[0][0] : k4 == 1 ? kc[1][0] : k4 == 2 ? kc[2][0] : kc[3][0];
-            w.y = k4 == 0 ? kc[0][1] : k4 == 1 ? kc[1][1] : k4 == 2 ? kc[2][1] : kc[3][1];
-            w.z = k4 == 0 ? kc[0][2] : k4 == 1 ? kc[1][2] : k4 == 2 ? kc[2][2] : kc[3][2];
-            w.w = k4 == 0 ? kc[0][3] : k4 == 1 ? kc[1][3] : k4 == 2 ? kc[2][3] : kc[3][3];
+          for (int k4 = 0; k4 < 4; ++k4) {
             const int row = c0 + k4;
             *reinterpret_cast<float4*>(hb + H_KC + row * 128 +
-                                       ((chunk ^ (uint32_t)(row & 7)) << 4)) = w;
+                                       ((chunk ^ (uint32_t)(row & 7)) << 4)) =
+                make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
           }
         }
       }
@@ -448,7 +467,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       uint8_t* kb_buf = sm + SM_KEY + b * KEYB;
       uint8_t* hb = sm + SM_HB + b * HBB;
       const float* betas = reinterpret_cast<const float*>(sm + SM_BETA + b * 128);
-      mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 3);
+      wait(&bars[B_OPER + b], (c >> 1) & 1, 3);
       __syncwarp();
       {  // Gram: warp sw computes rows 16 sw .. +15 of [K_L ; Q_L] K_B^T (64 x 32,
          // K = 128 channels) with m16n8k16 MMAs from the swizzled tiles, then
@@ -586,7 +605,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       const int n = chunk_rows(cc);
       const int vb = cc % NVBUF;
       if (!U.vzero) {
-        mbar_wait_bounded(&bars[B_V + vb], (cc / NVBUF) & 1, abort_flag, P.sb, 9);
+        wait(&bars[B_V + vb], (cc / NVBUF) & 1, 9);
         __syncwarp();
       }
       const uint8_t* vt = sm + SM_V + vb * 8192 + v_off;
@@ -599,8 +618,22 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_VEMPTY + vb]);
     };
-    // the A operand of the next [O | P] GEMM: bf16 copy of the current S^T
-    auto write_sb = [&]() {
+    // [O^T | P^T] of the next chunk start as [0 | -V^T]: P (free once the U
+    // GEMM that read it is done) and O (once this chunk's O is read out)
+    auto seed_p = [&]() { tmem_st32(tbase + lane_base + P_COL, vn); };
+    auto seed_o = [&]() {
+      const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      tmem_st16(tbase + lane_base + O_COL, z);
+      tmem_st16(tbase + lane_base + O_COL + 16, z);
+    };
+    // One pass over the state once the previous [S | O] GEMM is done: the bf16
+    // copy of S^T (the A operand of chunk cc's [O | P]) and, from the same load,
+    // S^T *= e^{Gamma_C, i} of chunk cc (what chunk cc's [S | O] accumulates onto).
+    // Doing both here keeps tensor-memory traffic off the time the GEMMs run.
+    auto copy_and_decay = [&](int cc) {
+      wait(&bars[B_OPER + (cc & 1)], (cc >> 1) & 1, 5);  // e^{Gamma_C} of chunk cc
+      __syncwarp();
+      const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + (cc & 1) * 512);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float v[32];
@@ -613,70 +646,55 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
           pk[k] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         tmem_st16(tbase + lane_base + SB_COL + 16 * q, pk);
-      }
-    };
-    // [O^T | P^T] of the next chunk start as [0 | -V^T]
-    auto seed_op = [&]() {
-      float z[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = 0.f;
-      tmem_st32(tbase + lane_base + O_COL, z);
-      tmem_st32(tbase + lane_base + P_COL, vn);
-    };
-    // S^T[j][i] *= e^{Gamma_C, i} of chunk cc, ahead of that chunk's [S | O] GEMM
-    auto decay = [&](int cc) {
-      mbar_wait_bounded(&bars[B_OPER + (cc & 1)], (cc >> 1) & 1, abort_flag, P.sb, 5);
-      __syncwarp();
-      const float4* g4 = reinterpret_cast<const float4*>(sm + SM_GAMC + (cc & 1) * 512);
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld32(tbase + lane_base + S_COL + 32 * q, v);
-        wait_ld();
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
           const float4 gg = g4[8 * q + k4];
-          v[4 * k4 + 0] *= gg.x;
-          v[4 * k4 + 1] *= gg.y;
-          v[4 * k4 + 2] *= gg.z;
-          v[4 * k4 + 3] *= gg.w;
+          const float2 a = __fmul2_rn(make_float2(v[4 * k4], v[4 * k4 + 1]), make_float2(gg.x, gg.y));
+          const float2 b2 =
+              __fmul2_rn(make_float2(v[4 * k4 + 2], v[4 * k4 + 3]), make_float2(gg.z, gg.w));
+          v[4 * k4 + 0] = a.x;
+          v[4 * k4 + 1] = a.y;
+          v[4 * k4 + 2] = b2.x;
+          v[4 * k4 + 3] = b2.y;
         }
         tmem_st32(tbase + lane_base + S_COL + 32 * q, v);
       }
-      wait_st();
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_DECAY]);
     };
-    if (nchunks > 0) {  // chunk 0: bf16 S, seed, then the decay
-      write_sb();
-      load_v(0);
-      seed_op();
+    // hand-off to the issuer: [O | P] seeded, the bf16 state written, the state decayed
+    auto publish = [&]() {
       wait_st();
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_OREADY]);
-      decay(0);
+      if (lane == 0) {
+        mbar_arrive(&bars[B_OREADY]);
+        mbar_arrive(&bars[B_DECAY]);
+      }
+    };
+    if (nchunks > 0) {  // chunk 0
+      load_v(0);
+      seed_p();
+      seed_o();
+      copy_and_decay(0);
+      publish();
     }
     for (int c = 0; c < nchunks; ++c) {
       if (bar_red_or(3, 128, *abort_flag != 0)) break;
       const int b = c & 1;
       const bool more = c + 1 < nchunks;
       if (more) load_v(c + 1);  // while this chunk's GEMMs run
-      mbar_wait_bounded(&bars[B_SO + b], (c >> 1) & 1, abort_flag, P.sb, 7);
+      wait(&bars[B_SO + b], (c >> 1) & 1, 7);
       __syncwarp();
       fence_after_sync();
-      // critical path: bf16 S for the next [O | P], O read out, seed
-      if (more) write_sb();
+      // critical path: seed, O read out, bf16 S and decay for the next chunk
+      if (more) seed_p();
       float vo[32];  // O^T (lane j, column r)
       tmem_ld32(tbase + lane_base + O_COL, vo);
       wait_ld();
-      if (more) seed_op();
-      wait_st();
-      fence_before_sync();
-      __syncwarp();
-      if (more && lane == 0) mbar_arrive(&bars[B_OREADY]);
-      if (more) decay(c + 1);  // overlaps the next [O | P] and U GEMMs
+      if (more) {
+        seed_o();
+        copy_and_decay(c + 1);
+        publish();
+      }
       if (U.out_on) {  // lanes j, j^1 swap values so each writes a bf16 pair
         const int n = chunk_rows(c);
         const bool odd = lane & 1;
@@ -718,8 +736,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         // [O^T | P^T] += S^T [Qg ; Ka]^T (bf16, A = the bf16 copy of S^T) once the
         // operands are written and O / P are seeded (which the state warps do
         // after the previous [S | O] completed)
-        mbar_wait_bounded(&bars[B_OPER + b], (c >> 1) & 1, abort_flag, P.sb, 10);
-        mbar_wait_bounded(&bars[B_OREADY], c & 1, abort_flag, P.sb, 11);
+        wait(&bars[B_OPER + b], (c >> 1) & 1, 10);
+        wait(&bars[B_OREADY], c & 1, 11);
         if (*abort_flag) break;
         fence_after_sync();
         const uint32_t hb = sb + SM_HB + b * HBB;
@@ -730,8 +748,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
                       1);
         mma_commit(&bars[B_UO]);
         // U^T = -P^T T^T once P is complete and T is in
-        mbar_wait_bounded(&bars[B_T + b], (c >> 1) & 1, abort_flag, P.sb, 12);
-        mbar_wait_bounded(&bars[B_UO], c & 1, abort_flag, P.sb, 13);
+        wait(&bars[B_T + b], (c >> 1) & 1, 12);
+        wait(&bars[B_UO], c & 1, 13);
         if (*abort_flag) break;
         fence_after_sync();
         const uint32_t kbb = sb + SM_KEY + b * KEYB;
@@ -741,8 +759,8 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
                       sw128_desc(kbb + K_TF + ks * 32, 16, 1024), id_u, ks > 0);
         mma_commit(&bars[B_U]);
         // [S^T | O^T] += U^T [Kc ; A_qk]^T once U is done and the state is decayed
-        mbar_wait_bounded(&bars[B_U], c & 1, abort_flag, P.sb, 14);
-        mbar_wait_bounded(&bars[B_DECAY], c & 1, abort_flag, P.sb, 15);
+        wait(&bars[B_U], c & 1, 14);
+        wait(&bars[B_DECAY], c & 1, 15);
         if (*abort_flag) break;
         fence_after_sync();
 #pragma unroll 1
@@ -772,9 +790,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         tma_load_3d(in + OFF_G, &P.tm_g, bf, 0, h, row);
         if (!U.vzero) {  // v into its ring slot, once the chunk 4 back has been read
           const int vb = cc % NVBUF;
-          if (cc >= NVBUF &&
-              !mbar_wait_bounded(&bars[B_VEMPTY + vb], ((cc - NVBUF) / NVBUF) & 1, abort_flag,
-                                 P.sb, 18))
+          if (cc >= NVBUF && !wait(&bars[B_VEMPTY + vb], ((cc - NVBUF) / NVBUF) & 1, 18))
             return;
           uint8_t* dst = sm + SM_V + vb * 8192;
           uint64_t* bv = &bars[B_V + vb];
@@ -789,7 +805,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       for (int c = 0; c + 2 < nchunks; ++c) {
         if (*abort_flag) break;
         // q, k, g of chunk c + 2 into the stage chunk c's prep has released
-        mbar_wait_bounded(&bars[B_IN_EMPTY + (c & 1)], (c >> 1) & 1, abort_flag, P.sb, 17);
+        wait(&bars[B_IN_EMPTY + (c & 1)], (c >> 1) & 1, 17);
         if (*abort_flag) break;
         issue_qkg(nq++);
       }
@@ -897,6 +913,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+// Bound of the kernel's mbarrier waits: kWaitLimitNs unless a diagnostic
+// lowered it (kda_set_wait_limit_ns), process-wide.
+std::atomic<long long> g_wait_limit_ns{kWaitLimitNs};
+long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 // The shared-memory limit is a per-device attribute of the kernel: set it on
 // every launch (a cheap host call) so that any device the caller makes
 // current gets it, from any host thread.
@@ -994,6 +1015,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail, size_t ws_tail_by
   P.T = a.map.T;
   P.H = H;
   P.scale = a.scale;
+  P.wait_limit_ns = wait_limit_ns();
   P.mode = 0;
   P.G = 1;
   P.seg_len = a.map.T;
@@ -1049,6 +1071,7 @@ cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStr
   P.T = a.map.T;
   P.H = H;
   P.scale = 1.f;
+  P.wait_limit_ns = wait_limit_ns();
   // transition mode over the whole range as the one segment before a second:
   // CTA pair u = (S~ from zero with v, M from the identity with v = 0)
   P.mode = 1;
@@ -1058,6 +1081,8 @@ cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStr
   chunk_tc_kernel<<<a.num_units * 2, NT, SMEM_ALLOC, stream>>>(P);
   return cudaGetLastError();
 }
+
+void set_wait_limit_ns(long long ns) { g_wait_limit_ns.store(ns, std::memory_order_relaxed); }
 
 cudaError_t launch_state_prefix(const float* pairs, int count, int index, const float* init,
                                 int units, float* state_out, cudaStream_t stream) {

@@ -128,6 +128,9 @@ cudaError_t launch_chunk_tc_transition(const ChunkArgs& a, float* pairs, cudaStr
 cudaError_t launch_state_prefix(const float* pairs, int count, int index, const float* init,
                                 int units, float* state_out, cudaStream_t stream);
 
+// Bound of every mbarrier wait in the tensor-core chunk kernel (diagnostics).
+void set_wait_limit_ns(long long ns);
+
 cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns,
                                  cudaStream_t stream);
 

@@ -126,13 +126,14 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 // stay small in the instruction cache.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                                    volatile int* abort_flag, StatusBlock* sb,
-                                                   int32_t detail, uint32_t hint_ns) {
+                                                   int32_t detail, uint32_t hint_ns,
+                                                   long long limit_ns) {
   // suspended waits of up to kSuspendNs each: no issue slots spent while waiting
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
     if (*abort_flag) return false;
-    if ((long long)(global_ns() - t0) > kWaitLimitNs) {
+    if ((long long)(global_ns() - t0) > limit_ns) {
       *abort_flag = 1;
       record_status(sb, KDA_ERR_TIMEOUT, detail);
       return false;
@@ -140,12 +141,15 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
   }
 }
 
+// limit_ns bounds the wait (kWaitLimitNs unless a caller lowers it to
+// exercise the timeout path).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag, StatusBlock* sb,
                                                   int32_t detail,
+                                                  long long limit_ns = kWaitLimitNs,
                                                   uint32_t hint_ns = kSuspendNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag, sb, detail, hint_ns);
+  return mbar_wait_slow(bar, parity, abort_flag, sb, detail, hint_ns, limit_ns);
 }
 
 // Abort-path drain: waits (up to the time limit, whatever the abort flag says)

@@ -368,6 +368,20 @@ KDA_API kda_status kda_selftest_bounded_wait(void *workspace, int64_t spin_limit
                                      void *stream);
 
 /*
+ * Diagnostic for the chunk kernels' own failure path: sets the limit of
+ * every bounded wait inside the tensor-core chunk kernel (the hand-offs
+ * between its warp roles), process-wide, for launches that follow.  The
+ * default is 2e9 ns (far above any real wait); `limit_ns` is clamped to
+ * [0, 5e9].  With a limit of 0 a wait that is not satisfied at its first
+ * poll runs out: the kernel records KDA_ERR_TIMEOUT in the workspace status
+ * word, lets the asynchronous copies and tensor-core operations it issued
+ * land, releases its tensor memory and returns, leaving its outputs
+ * partly written; the context stays usable.  Waits that drain in-flight work
+ * keep the default bound.  Returns KDA_OK.
+ */
+KDA_API kda_status kda_set_wait_limit_ns(int64_t limit_ns);
+
+/*
  * kda_chunk_fwd without a workspace, for callers that cannot allocate device
  * memory (an engine plugin limited to memory its host planned up front, a
  * service whose allocator is frozen after warm-up, a fixed device-memory

@@ -198,6 +198,38 @@ def test_bounded_wait_times_out_and_context_survives():
     assert float((x * 2).sum()) == 8.0  # the context is still usable
 
 
+def test_chunk_kernel_timeout_path_returns_and_context_survives():
+    """The tensor-core chunk kernel's own abort path: with its internal wait
+    limit lowered to 0, a hand-off between its warp roles runs out; the kernel
+    records KDA_ERR_TIMEOUT, drains what it issued, frees its tensor memory and
+    returns.  With the limit restored the same call on the same workspace
+    succeeds and matches a fresh run bit for bit."""
+    B, T, H, d = 2, 4096, 4, 128
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=12, device=DEV,
+                                init_state=True)
+    o_ref, S_ref, g, _ = gpu_prefill(inp)
+    out = torch.full_like(o_ref, float("nan"))
+    fin = torch.full_like(S_ref, float("nan"))
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(B, T, H, d, d), dtype=torch.uint8,
+                     device=DEV)
+    try:
+        kda.kda_set_wait_limit_ns(0)
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], out, ws,
+                          init_state=inp["init_state"], final_state=fin)
+        st, where = kda.kda_get_device_status(ws)
+    finally:
+        kda.kda_set_wait_limit_ns(2_000_000_000)
+    assert st == kda.KDA_ERR_TIMEOUT, kda.kda_status_string(st)
+    assert where > 0  # the wait that ran out names itself
+    x = torch.ones(4, device=DEV)
+    assert float((x * 2).sum()) == 8.0  # the context is still usable
+    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], out, ws,
+                      init_state=inp["init_state"], final_state=fin)
+    st, _ = kda.kda_get_device_status(ws)
+    assert st == kda.KDA_OK
+    assert torch.equal(out, o_ref) and torch.equal(fin, S_ref)
+
+
 # ------------------------------------------------- tensor-core path specifics
 
 def _slow_decay(inp, shift=4.0):
