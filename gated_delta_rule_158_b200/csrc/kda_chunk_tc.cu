@@ -95,10 +95,19 @@ constexpr uint32_t K_TF = 4096;     //   T fp32 [r][s] (tf32 B of U = -P^T T^T)
 constexpr uint32_t K_AKKT = 16384;  //   A_kk^T fp32 [s][r] (inverse input)
 constexpr uint32_t K_XS = 20480;    //   inverse blocks, fp32 32 x 32
 constexpr uint32_t SM_HB = SM_KEY + 2 * KEYB;  // hand-off buffer b at SM_HB + b * HBB
-constexpr uint32_t HBB = 36864;
+constexpr uint32_t HBB = 39936;
 constexpr uint32_t H_QK = 0;        //   [q e^G ; k e^G] bf16, per 64-channel block 64 rows x 128 B
-constexpr uint32_t H_KC = 16384;    //   k e^{GC-G} fp32 [i][s] (rows 0-127 of the B of [S | O])
-constexpr uint32_t H_AQK = 32768;   //   A_qk fp32 [r][s]       (rows 128-159 of the same tile)
+constexpr uint32_t H_KC = 16384;    //   B of [S | O], tf32 K-major without swizzle: rows n < 128
+                                    //   key channel i of k e^{GC-G}, n >= 128 row r = n - 128 of
+                                    //   A_qk; K = token s.  Core matrices of 8 rows x 16 bytes;
+                                    //   8-row groups KC_SBO apart (16 bytes of padding, so the
+                                    //   prep warps' 16-byte stores of 8 consecutive row groups
+                                    //   fall in distinct banks), 4-token groups KC_LBO apart.
+constexpr uint32_t KC_SBO = 144, KC_LBO = 20 * KC_SBO;
+static_assert(H_KC + 8 * KC_LBO <= HBB, "[S | O] operand tile fits the hand-off buffer");
+__device__ __forceinline__ uint32_t kc_off(uint32_t n, uint32_t s) {
+  return (s >> 2) * KC_LBO + (n >> 3) * KC_SBO + (n & 7) * 16 + (s & 3) * 4;
+}
 constexpr uint32_t SM_V = SM_HB + 2 * HBB;  // v tile of chunk c at SM_V + (c % 4) * 8192:
 constexpr int NVBUF = 4;                    //   bf16, 2 x [32 rows x 128 B] swizzled (TMA)
 constexpr uint32_t SM_MISC = SM_V + NVBUF * 8192;
@@ -109,7 +118,6 @@ constexpr uint32_t SM_TMEM = SM_MISC + 1536;   // TMEM base address
 constexpr uint32_t SM_ABORT = SM_MISC + 1540;  // abort flag
 constexpr uint32_t SMEM_BYTES = SM_MISC + 2048;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base to 1024
-static_assert(H_AQK == H_KC + 16384, "A_qk rows must follow the Kc^T rows");
 static_assert(SMEM_ALLOC <= 227 * 1024, "one CTA per SM");
 
 // mbarriers ([2] = one per chunk parity, [4] = one per v buffer)
@@ -438,16 +446,11 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
             *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (32 + r) * 128 + s16) =
                 make_uint2(pack(kg01.x, kg01.y), pack(kg23.x, kg23.y));
           }
-          // Kc^T rows c0..c0+3 (K-major: row = channel, 32 tokens of fp32), the
-          // 16-byte chunk of tokens 8pw + 4hf .. +3 of each
-          const uint32_t chunk = (uint32_t)(2 * pw + hf);
+          // Kc^T rows c0..c0+3 (K-major: row = channel), tokens 8pw + 4hf .. +3 of each
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const int row = c0 + k4;
-            *reinterpret_cast<float4*>(hb + H_KC + row * 128 +
-                                       ((chunk ^ (uint32_t)(row & 7)) << 4)) =
+          for (int k4 = 0; k4 < 4; ++k4)
+            *reinterpret_cast<float4*>(hb + H_KC + kc_off(c0 + k4, 8 * pw + 4 * hf)) =
                 make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
-          }
         }
       }
       fence_proxy_async();
@@ -525,9 +528,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
               const int s2 = 8 * nt + cq;
               const float2 w2 = make_float2(s2 <= r ? acc[nt][2 * hh] : 0.f,
                                             s2 + 1 <= r ? acc[nt][2 * hh + 1] : 0.f);
-              *reinterpret_cast<float2*>(hb + H_AQK + r * 128 +
-                                         ((((uint32_t)s2 >> 2) ^ (uint32_t)(r & 7)) << 4) +
-                                         (s2 & 3) * 4) = w2;
+              *reinterpret_cast<float2*>(hb + H_KC + kc_off(128u + r, (uint32_t)s2)) = w2;
             }
           }
         }
@@ -766,7 +767,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
 #pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
           mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
-                      sw128_desc(hb + H_KC + ks * 32, 16, 1024), id_so, 1);
+                      plain_desc(hb + H_KC + 2 * ks * KC_LBO, KC_LBO, KC_SBO), id_so, 1);
         mma_commit(&bars[B_SO + b]);
       }
       if (*abort_flag) {  // every MMA this thread issued lands before TMEM is released

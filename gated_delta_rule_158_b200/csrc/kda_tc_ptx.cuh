@@ -43,6 +43,19 @@ __device__ __forceinline__ uint64_t sw128b32_desc(uint32_t saddr, uint32_t lbo_b
   return d;
 }
 
+// Descriptor of a K-major operand without swizzle: core matrices of 8 rows x 16
+// bytes (rows contiguous), lbo = stride between cores along K, sbo = stride
+// between 8-row groups.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
 // ------------------------------------------------------ instruction descriptor
 // [4,6) D format (1 = f32)  [7,10) A format  [10,13) B format
 // (kind::f16: 1 = bf16; kind::tf32: 2 = tf32)  [13] negate A  [15] A MN-major
