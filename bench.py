@@ -744,9 +744,32 @@ def prefill_roofline(m, peaks, wl):
             "tensor_frac_c64_count": round(f64 / secs / (peaks["tc"] * 1e12), 4)}
 
 
+def check_input_sensitivity(step):
+    """Outside the timed region: the step's output must follow its inputs.
+    One value of v (token 0, head 0, channel 0) is changed, the step rerun, the
+    output compared with the previous one (it must differ at token 0 of head 0),
+    then the input is restored and the step rerun once more (it must give the
+    original output back bit for bit)."""
+    inp = step.inp
+    before = step.out.clone()
+    keep = inp["v"][0, 0, 0, 0].clone()
+    inp["v"][0, 0, 0, 0] = keep + 1.0
+    step()
+    changed = not torch.equal(step.out[0, 0, 0], before[0, 0, 0])
+    inp["v"][0, 0, 0, 0] = keep
+    step()
+    restored = torch.equal(step.out, before)
+    torch.cuda.synchronize()
+    if not (changed and restored):
+        raise RuntimeError(f"output does not follow the input (changed={changed}, "
+                           f"restored={restored})")
+    return True
+
+
 def bench_prefill_line(args, wl, world, rank, peaks):
     dev = torch.device("cuda", torch.cuda.current_device())
     m = measure_prefill(wl, dev, args.steps, args.warmup, world, not args.no_clocks)
+    sensitivity = check_input_sensitivity(m["step"])
     inp, cu, T, N, B, H = m["inp"], m["cu"], m["T"], m["N"], m["B"], m["H"]
     dk, dv, step, tokens = m["dk"], m["dv"], m["step"], m["tokens"]
     line = {
@@ -761,6 +784,8 @@ def bench_prefill_line(args, wl, world, rank, peaks):
         "roofline": prefill_roofline(m, peaks, wl),
         "gpu_launches": args.steps * kernels_per_step(wl, B, T),
         "clocks": m["clk"],
+        "input_sensitivity": "checked: one value of v changed changes the output; restored gives "
+                             "it back bit for bit" if sensitivity else None,
     }
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_prefill(wl, inp, cu, N, max(2, min(args.steps, 5)))

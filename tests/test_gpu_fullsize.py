@@ -48,6 +48,30 @@ def _oracle_units(oracle_mod, inp, units, cu=None):
     return res
 
 
+def _unit_gate(oracle_mod, inp, h, z64):
+    return oracle_mod.gate(z64, to64(inp["A_log"])[h:h + 1], -5.0)
+
+
+def _oracle_packed(oracle_mod, inp, units, cu):
+    """The oracle on many (sequence, head) units of a packed batch in one call:
+    each unit's rows of its head become one sequence of a packed batch with a
+    single head, run by the oracle's thread pool.  Returns per-unit (o, S)."""
+    rows = [(int(cu[n]), int(cu[n + 1])) for n, _ in units]
+    cat = lambda name: np.concatenate([to64(inp[name][0, a:b, h]) for (a, b), (_, h) in
+                                       zip(rows, units)], axis=0)
+    z = [to64(inp["z"][0, a:b, h:h + 1])[None] for (a, b), (_, h) in zip(rows, units)]
+    g = np.concatenate([_unit_gate(oracle_mod, inp, h, zz)[0, :, 0] for zz, (_, h) in
+                        zip(z, units)], axis=0)
+    sub_cu = np.concatenate([[0], np.cumsum([b - a for a, b in rows])]).astype(np.int64)
+    init = None
+    if inp["init_state"] is not None:
+        init = np.stack([to64(inp["init_state"][n, h]) for n, h in units])[:, None]
+    o, S = oracle_mod.forward(cat("q")[None, :, None], cat("k")[None, :, None],
+                              cat("v")[None, :, None], g[None, :, None],
+                              cat("beta")[None, :, None], init_state=init, cu_seqlens=sub_cu)
+    return [(o[0, sub_cu[u]:sub_cu[u + 1], 0], S[u, 0]) for u in range(len(units))]
+
+
 def _check_units(o, S, ref, units, cu=None):
     for (n, h), (o_ref, S_ref) in zip(units, ref):
         if cu is None:
@@ -78,8 +102,13 @@ def test_varlen_prefill_full_size(oracle_mod):
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
     longest = int(np.argmax(lens))
     shortest = int(np.argmin(lens))
-    units = [(longest, 3), (shortest, 0), (17, 15), (40, 8)]
-    _check_units(o, S, _oracle_units(oracle_mod, inp, units, cu=cu_list), units, cu=cu_list)
+    # 16 sequences: the longest and the shortest, the rest spread over the batch,
+    # each with its own head (every head appears)
+    others = [n for n in range(0, 64, 4) if n not in (longest, shortest)][:14]
+    seqs = [longest, shortest] + others
+    units = [(n, (3 * i) % 16) for i, n in enumerate(seqs)]
+    assert len(units) == 16
+    _check_units(o, S, _oracle_packed(oracle_mod, inp, units, cu_list), units, cu=cu_list)
 
 
 def test_decode_full_size(oracle_mod):
@@ -114,13 +143,64 @@ def test_decode_full_size(oracle_mod):
         assert rel_l2(to64(state[n, h]), S_ref[0, 0]) <= TOL_BF16_S
 
 
+def _unsplit_reference(inp, g, piece=4064):
+    """The long sequence without the segment split: consecutive calls of fewer
+    than 4096 tokens each (below the split's threshold), each starting from the
+    previous call's final state (the fp32 state is handed over exactly)."""
+    q = inp["q"]
+    B, T, H, d = q.shape
+    out = torch.empty_like(q)
+    state = None
+    for a in range(0, T, piece):
+        b = min(T, a + piece)
+        sl = lambda t: t[:, a:b].contiguous()
+        o_p = torch.empty((1, b - a, H, d), dtype=q.dtype, device=DEV)
+        fin = torch.empty((1, H, d, d), device=DEV)
+        ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(1, b - a, H, d, d), dtype=torch.uint8,
+                         device=DEV)
+        kda.kda_chunk_fwd(sl(q), sl(inp["k"]), sl(inp["v"]), sl(g), sl(inp["beta"]), o_p, ws,
+                          init_state=state, final_state=fin)
+        out[:, a:b] = o_p
+        state = fin
+    return out, state
+
+
 def test_long_prefill_full_size(oracle_mod):
-    """T = 1,048,576 with B*H = 32: the segment-split launch sequence."""
+    """T = 1,048,576 with B*H = 32: the segment-split launch sequence.  Every
+    unit (outputs and final state) against the same recurrence run without the
+    split, and 8 units spread over the heads against the oracle over the whole
+    sequence (run in pieces, its fp64 state carried from piece to piece, which
+    is exactly one sequential run)."""
     T, H = 1 << 20, 32
     inp = W.make_prefill_inputs(1, T, H, 128, 128, torch.bfloat16, seed=2, device=DEV)
-    o, S, _, ws = gpu_prefill(inp, with_init=False)
+    o, S, g, ws = gpu_prefill(inp, with_init=False)
     assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
-    assert torch.isfinite(S).all()
-    assert torch.isfinite(o[0, ::4096].float()).all()
-    units = [(0, 11)]
-    _check_units(o, S, _oracle_units(oracle_mod, inp, units), units)
+    assert torch.isfinite(S).all() and torch.isfinite(o.float()).all()
+
+    o_ref, S_ref = _unsplit_reference(inp, g)
+    torch.cuda.synchronize()
+    for h in range(H):
+        d_o = (o[0, :, h].double() - o_ref[0, :, h].double()).norm() / o_ref[0, :, h].double().norm()
+        d_s = (S[0, h] - S_ref[0, h]).double().norm() / S_ref[0, h].double().norm()
+        assert float(d_o) <= TOL_BF16_O, (h, float(d_o))
+        assert float(d_s) <= TOL_BF16_S, (h, float(d_s))
+    del o_ref, S_ref
+
+    heads = [0, 5, 9, 14, 18, 23, 27, 31]
+    piece = 1 << 16
+    num = np.zeros(len(heads))
+    den = np.zeros(len(heads))
+    state = None
+    for a in range(0, T, piece):
+        b = a + piece
+        stack = lambda name: np.stack([to64(inp[name][0, a:b, h]) for h in heads])[:, :, None]
+        gg = np.stack([_unit_gate(oracle_mod, inp, h, to64(inp["z"][0:1, a:b, h:h + 1]))[0, :, 0]
+                       for h in heads])[:, :, None]
+        o_u, state = oracle_mod.forward(stack("q"), stack("k"), stack("v"), gg, stack("beta"),
+                                        init_state=state)
+        got = np.stack([to64(o[0, a:b, h]) for h in heads])
+        num += ((got - o_u[:, :, 0]) ** 2).sum(axis=(1, 2))
+        den += (o_u[:, :, 0] ** 2).sum(axis=(1, 2))
+    for u, h in enumerate(heads):
+        assert np.sqrt(num[u] / den[u]) <= TOL_BF16_O, (h, np.sqrt(num[u] / den[u]))
+        assert rel_l2(to64(S[0, h]), state[u, 0]) <= TOL_BF16_S, h
