@@ -76,8 +76,21 @@ constexpr int D = 128;   // dk = dv
 constexpr int PREP_W0 = 0, SOLVE_W0 = 4, STATE_W0 = 8, ISSUE_W = 12;  // warp 13: TMA issue
 constexpr int NT = 32 * 14;
 
-constexpr uint32_t S_COL = 0, O_COL = 128, P_COL = 160, U_COL = 192;
-constexpr uint32_t SB_COL = 384;  // bf16 S^T: column c holds key channels 2c, 2c + 1
+// [O | P] and its O are double-buffered by chunk parity b, each buffer next to
+// S on the side the fused GEMMs need: b = 0 as [P | O] left of S and [O | S];
+// b = 1 as [S | O] and [O | P] right of S.  A chunk's O is then read out, and
+// the next-but-one chunk's [O | P] seeded, while the chain goes on.
+constexpr uint32_t S_COL = 64, U_COL = 256;
+constexpr uint32_t SB_COL = 288;  // bf16 S^T: column c holds key channels 2c, 2c + 1
+__device__ __forceinline__ uint32_t o_col(int b) { return b ? 192u : 32u; }
+__device__ __forceinline__ uint32_t p_col(int b) { return b ? 224u : 0u; }
+__device__ __forceinline__ uint32_t op_col(int b) { return b ? 192u : 0u; }   // [O|P] / [P|O]
+__device__ __forceinline__ uint32_t so_col(int b) { return b ? 64u : 32u; }   // [S|O] / [O|S]
+// operand rows of those GEMMs: q e^G / k e^G rows of [O | P], Kc^T / A_qk rows of [S | O]
+__device__ __forceinline__ uint32_t q_row(int b) { return b ? 0u : 32u; }
+__device__ __forceinline__ uint32_t k_row(int b) { return b ? 32u : 0u; }
+__device__ __forceinline__ uint32_t kc_row(int b) { return b ? 0u : 32u; }
+__device__ __forceinline__ uint32_t aqk_row(int b) { return b ? 128u : 0u; }
 constexpr uint32_t TMEM_COLS = 512;
 
 // shared memory map (byte offsets from a 1024-aligned base)
@@ -439,17 +452,17 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
                 make_uint2(pack(ql01.x, ql01.y), pack(ql23.x, ql23.y));
             *reinterpret_cast<uint2*>(kb_buf + K_KB + o_kb + r * 128 + s16) =
                 make_uint2(pack(kb01.x, kb01.y), pack(kb23.x, kb23.y));
-            // B of [O | P] (bf16, same layout as the Gram A): q e^G rows 0-31,
-            // k e^G rows 32-63 of each 64-channel block
-            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + r * 128 + s16) =
+            // B of [O | P] (bf16, same layout as the Gram A): q e^G and k e^G rows
+            // of each 64-channel block in the order of buffer b's columns
+            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (q_row(b) + r) * 128 + s16) =
                 make_uint2(pack(qg01.x, qg01.y), pack(qg23.x, qg23.y));
-            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (32 + r) * 128 + s16) =
+            *reinterpret_cast<uint2*>(hb + H_QK + o_kql + (k_row(b) + r) * 128 + s16) =
                 make_uint2(pack(kg01.x, kg01.y), pack(kg23.x, kg23.y));
           }
           // Kc^T rows c0..c0+3 (K-major: row = channel), tokens 8pw + 4hf .. +3 of each
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
-            *reinterpret_cast<float4*>(hb + H_KC + kc_off(c0 + k4, 8 * pw + 4 * hf)) =
+            *reinterpret_cast<float4*>(hb + H_KC + kc_off(kc_row(b) + c0 + k4, 8 * pw + 4 * hf)) =
                 make_float4(kc[k4][0], kc[k4][1], kc[k4][2], kc[k4][3]);
         }
       }
@@ -528,7 +541,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
               const int s2 = 8 * nt + cq;
               const float2 w2 = make_float2(s2 <= r ? acc[nt][2 * hh] : 0.f,
                                             s2 + 1 <= r ? acc[nt][2 * hh + 1] : 0.f);
-              *reinterpret_cast<float2*>(hb + H_KC + kc_off(128u + r, (uint32_t)s2)) = w2;
+              *reinterpret_cast<float2*>(hb + H_KC + kc_off(aqk_row(b) + r, (uint32_t)s2)) = w2;
             }
           }
         }
@@ -619,13 +632,14 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_VEMPTY + vb]);
     };
-    // [O^T | P^T] of the next chunk start as [0 | -V^T]: P (free once the U
-    // GEMM that read it is done) and O (once this chunk's O is read out)
-    auto seed_p = [&]() { tmem_st32(tbase + lane_base + P_COL, vn); };
-    auto seed_o = [&]() {
+    // chunk cc's [O^T | P^T] starts as [0 | -V^T], in buffer cc & 1 (free once
+    // chunk cc - 2's O is read out and its U GEMM has read its P)
+    auto seed = [&](int cc) {
+      load_v(cc);
+      tmem_st32(tbase + lane_base + p_col(cc & 1), vn);
       const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      tmem_st16(tbase + lane_base + O_COL, z);
-      tmem_st16(tbase + lane_base + O_COL + 16, z);
+      tmem_st16(tbase + lane_base + o_col(cc & 1), z);
+      tmem_st16(tbase + lane_base + o_col(cc & 1) + 16, z);
     };
     // One pass over the state once the previous [S | O] GEMM is done: the bf16
     // copy of S^T (the A operand of chunk cc's [O | P]) and, from the same load,
@@ -671,10 +685,9 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         mbar_arrive(&bars[B_DECAY]);
       }
     };
-    if (nchunks > 0) {  // chunk 0
-      load_v(0);
-      seed_p();
-      seed_o();
+    if (nchunks > 0) {  // chunks 0 and 1
+      seed(0);
+      if (nchunks > 1) seed(1);
       copy_and_decay(0);
       publish();
     }
@@ -682,20 +695,17 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       if (bar_red_or(3, 128, *abort_flag != 0)) break;
       const int b = c & 1;
       const bool more = c + 1 < nchunks;
-      if (more) load_v(c + 1);  // while this chunk's GEMMs run
       wait(&bars[B_SO + b], (c >> 1) & 1, 7);
       __syncwarp();
       fence_after_sync();
-      // critical path: seed, O read out, bf16 S and decay for the next chunk
-      if (more) seed_p();
-      float vo[32];  // O^T (lane j, column r)
-      tmem_ld32(tbase + lane_base + O_COL, vo);
-      wait_ld();
+      // critical path: bf16 S and decay for the next chunk
       if (more) {
-        seed_o();
         copy_and_decay(c + 1);
         publish();
       }
+      float vo[32];  // O^T (lane j, column r)
+      tmem_ld32(tbase + lane_base + o_col(b), vo);
+      wait_ld();
       if (U.out_on) {  // lanes j, j^1 swap values so each writes a bf16 pair
         const int n = chunk_rows(c);
         const bool odd = lane & 1;
@@ -713,6 +723,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
                 __floats2bfloat162_rn(P.scale * lo, P.scale * hi);
         }
       }
+      if (c + 2 < nchunks) seed(c + 2);  // buffer b is free again: O read, P used
     }
     // final state (S^T lane j, column i -> final[i][j]); every S GEMM is done
     if (U.final_state && !*abort_flag) {
@@ -744,7 +755,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         const uint32_t hb = sb + SM_HB + b * HBB;
 #pragma unroll 1
         for (int ks = 0; ks < 8; ++ks)
-          mma_ts_bf16(tbase + O_COL, tbase + SB_COL + 8 * ks,
+          mma_ts_bf16(tbase + op_col(b), tbase + SB_COL + 8 * ks,
                       sw128_desc(hb + H_QK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_op,
                       1);
         mma_commit(&bars[B_UO]);
@@ -756,7 +767,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         const uint32_t kbb = sb + SM_KEY + b * KEYB;
 #pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts_tf32(tbase + U_COL, tbase + P_COL + 8 * ks,
+          mma_ts_tf32(tbase + U_COL, tbase + p_col(b) + 8 * ks,
                       sw128_desc(kbb + K_TF + ks * 32, 16, 1024), id_u, ks > 0);
         mma_commit(&bars[B_U]);
         // [S^T | O^T] += U^T [Kc ; A_qk]^T once U is done and the state is decayed
@@ -766,7 +777,7 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
         fence_after_sync();
 #pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
-          mma_ts_tf32(tbase + S_COL, tbase + U_COL + 8 * ks,
+          mma_ts_tf32(tbase + so_col(b), tbase + U_COL + 8 * ks,
                       plain_desc(hb + H_KC + 2 * ks * KC_LBO, KC_LBO, KC_SBO), id_so, 1);
         mma_commit(&bars[B_SO + b]);
       }
