@@ -32,6 +32,8 @@
 // element has one writer and every sum a fixed order: results are
 // deterministic.
 // Tail chunks are padded with g = 0, beta = 0, k = q = v = dO = 0.
+#include <algorithm>
+
 #include "kda_bwd.cuh"
 
 namespace kda {
@@ -166,7 +168,9 @@ struct SeqMap {
   const int32_t* cu;     // nullptr = dense
   const int32_t* coff;   // varlen: chunk offsets [N + 1]
   const StatusBlock* sb; // varlen: validity verdict of the plan kernel
-  int T, H;
+  int T, H;              // dense: T = tokens processed per sequence (a window of it)
+  int64_t row_stride;    // dense: rows from one sequence to the next (0: T)
+  int64_t row_off;       // dense: first row of the processed window in each sequence
 };
 
 struct UnitPos {
@@ -179,7 +183,7 @@ struct UnitPos {
 __device__ inline UnitPos unit_pos(const SeqMap& m, int n, int h) {
   UnitPos p;
   if (m.cu == nullptr) {
-    p.row0 = (int64_t)n * m.T;
+    p.row0 = (int64_t)n * (m.row_stride ? m.row_stride : (int64_t)m.T) + m.row_off;
     p.len = m.T;
     p.nc = (m.T + C - 1) / C;
     p.chunk0 = ((int64_t)n * m.H + h) * p.nc;
@@ -456,7 +460,8 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NTF, 1)
     bwd_fwd_scan(const Tin* __restrict__ k, const Tin* __restrict__ v,
                  const float* __restrict__ g, const float* __restrict__ beta,
-                 const float* __restrict__ init, SeqMap map, float* __restrict__ ws) {
+                 const float* __restrict__ init, SeqMap map, float* __restrict__ ws,
+                 float* __restrict__ fin) {
   constexpr int LDK = DK + 1, LDV = DV + 1;
   extern __shared__ float sm[];
   float* kS = sm;                 // [C][LDK]  k, then Kc
@@ -619,6 +624,13 @@ __global__ void __launch_bounds__(NTF, 1)
           SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
         });
       }
+    }
+  }
+  if (fin) {  // the state after the last chunk (a window's end state)
+    __syncthreads();
+    for (int idx = tid; idx < DK * DV; idx += NTF) {
+      const int i = idx / DV, j = idx % DV;
+      fin[(size_t)unit * DK * DV + idx] = SS[i * LDV + j];
     }
   }
 }
@@ -1264,83 +1276,152 @@ __global__ void __launch_bounds__(NTH, 2)
   }
 }
 
-// F and A, one CTA per unit each
-template <typename Tin, int DK, int DV>
-cudaError_t launch_scans(const BwdArgs& a, const SeqMap& map, int units, int64_t chunk_blocks,
-                         float* ws, cudaStream_t st) {
-  const size_t smK = KSmem<DK>::bytes, smF = FSmem<DK, DV>::bytes, smA = ASmem<DK, DV>::bytes;
-  cudaError_t e = cudaFuncSetAttribute(bwd_keyside<Tin, DK, DV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smK);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK, DV>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
-  if (e != cudaSuccess) return e;
-  const Tin* q = static_cast<const Tin*>(a.q);
-  const Tin* k = static_cast<const Tin*>(a.k);
-  const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
-  if (a.T > 0) {
-    bwd_keyside<Tin, DK, DV><<<(unsigned)chunk_blocks, NTH, smK, st>>>(q, k, a.g, a.beta, map,
-                                                                       nseq, ws);
-    if ((e = cudaGetLastError())) return e;
-    bwd_fwd_scan<Tin, DK, DV><<<units, NTF, smF, st>>>(
-        k, static_cast<const Tin*>(a.v), a.g, a.beta, a.init, map, ws);
-    if ((e = cudaGetLastError())) return e;
-  }
-  bwd_state_grad_scan<Tin, DK, DV><<<units, NTF, smA, st>>>(
-      q, k, a.g, a.beta, static_cast<const Tin*>(a.dout), a.dfinal, map, a.scale, a.dv,
-      a.dinit, ws);
-  return cudaGetLastError();
-}
+// Dense batches longer than this run in windows of this many tokens (whole
+// chunks) so that the workspace holds one window's chunks, not the sequence's:
+// a first pass of K and F over the windows in order keeps only each window's
+// start state (checkpoints); then, window by window from the last, K and F
+// recompute the window's chunk states from its checkpoint, A runs from the
+// state gradient the later window handed over, and B takes the chunks.  The
+// forward scan runs twice; every chunk sees the same arithmetic as in one
+// pass, so results are identical to an unwindowed run.
+constexpr int kBwdWindow = 8192;
+
+bool bwd_windowed(int T, int num_seqs) { return num_seqs == 0 && T > kBwdWindow; }
 
 struct WsLayout {
-  size_t coff_off, data_off, total;
-  int64_t max_chunks;  // per head
+  size_t coff_off, data_off, ck_off, ds_off, total;
+  int64_t max_chunks;  // per head (of the window when windowed)
 };
 
 WsLayout ws_layout(int B, int T, int H, int dk, int dv, int num_seqs) {
   WsLayout L;
-  const int64_t nc = ((int64_t)T + C - 1) / C;
+  const bool win = bwd_windowed(T, num_seqs);
+  const int64_t nc = ((int64_t)(win ? kBwdWindow : T) + C - 1) / C;
   L.coff_off = kStatusBytes;
   L.data_off = kStatusBytes + (num_seqs > 0 ? (sizeof(int32_t) * (size_t)(num_seqs + 1) + 255) / 256 * 256 : 0);
   L.max_chunks = num_seqs > 0 ? nc + num_seqs : (int64_t)B * nc;
-  L.total = L.data_off + (size_t)H * L.max_chunks * unit_ws_floats(1, dk, dv) * sizeof(float);
+  L.ck_off = L.data_off + (size_t)H * L.max_chunks * unit_ws_floats(1, dk, dv) * sizeof(float);
+  const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
+  const int nw = win ? (T + kBwdWindow - 1) / kBwdWindow : 1;
+  L.ds_off = L.ck_off + (win ? (size_t)(nw - 1) * state_bytes : 0);
+  L.total = L.ds_off + (win ? 2 * state_bytes : 0);
   return L;
 }
 
+template <typename Tin, int DK, int DV>
+struct Passes {
+  static cudaError_t attrs() {
+    cudaError_t e = cudaFuncSetAttribute(bwd_keyside<Tin, DK, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)KSmem<DK>::bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)FSmem<DK, DV>::bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK, DV>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)ASmem<DK, DV>::bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BSmem<DK>::bytes);
+    return e;
+  }
+  // K: the key-side matrices of every chunk, one CTA per (chunk, head)
+  static cudaError_t K(const BwdArgs& a, const SeqMap& m, int nseq, int64_t blocks, float* ws,
+                       cudaStream_t st) {
+    bwd_keyside<Tin, DK, DV><<<(unsigned)blocks, NTH, KSmem<DK>::bytes, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta, m, nseq, ws);
+    return cudaGetLastError();
+  }
+  // F: chunk-start states, R and U, one CTA per unit; fin (nullable) gets the end state
+  static cudaError_t F(const BwdArgs& a, const SeqMap& m, int units, const float* init,
+                       float* ws, float* fin, cudaStream_t st) {
+    bwd_fwd_scan<Tin, DK, DV><<<units, NTF, FSmem<DK, DV>::bytes, st>>>(
+        static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.g, a.beta, init, m, ws,
+        fin);
+    return cudaGetLastError();
+  }
+  // A: the state gradient in reverse chunk order from dfinal, writing dv and dinit
+  static cudaError_t A(const BwdArgs& a, const SeqMap& m, int units, const float* dfinal,
+                       float* dinit, float* ws, cudaStream_t st) {
+    bwd_state_grad_scan<Tin, DK, DV><<<units, NTF, ASmem<DK, DV>::bytes, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
+        static_cast<const Tin*>(a.dout), dfinal, m, a.scale, a.dv, dinit, ws);
+    return cudaGetLastError();
+  }
+  // B: every chunk's token gradients, one CTA per (chunk, head)
+  static cudaError_t Bp(const BwdArgs& a, const SeqMap& m, int nseq, int64_t blocks, float* ws,
+                        cudaStream_t st) {
+    bwd_chunk_grads<Tin, DK><<<(unsigned)blocks, NTH, BSmem<DK>::bytes, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
+        static_cast<const Tin*>(a.dout), m, nseq, a.dv_dim, a.scale, a.dq, a.dk, a.dg, a.dbeta,
+        ws);
+    return cudaGetLastError();
+  }
+
+  static cudaError_t run(const BwdArgs& a, cudaStream_t st) {
+    const WsLayout lay = ws_layout(a.B, a.T, a.H, DK, DV, a.cu_seqlens ? a.num_seqs : 0);
+    char* base = static_cast<char*>(a.ws);
+    StatusBlock* sb = reinterpret_cast<StatusBlock*>(base);
+    int32_t* coff = reinterpret_cast<int32_t*>(base + lay.coff_off);
+    float* ws = reinterpret_cast<float*>(base + lay.data_off);
+    cudaError_t e = attrs();
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(sb, 0, kStatusBytes, st))) return e;
+    const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
+    const int units = nseq * a.H;
+    if (!bwd_windowed(a.T, a.cu_seqlens ? a.num_seqs : 0)) {
+      SeqMap map{a.cu_seqlens, a.cu_seqlens ? coff : nullptr, sb, a.T, a.H, 0, 0};
+      if (a.cu_seqlens) {
+        bwd_varlen_plan<<<1, kPlanThreads, 0, st>>>(a.cu_seqlens, a.num_seqs, a.T, coff, sb);
+        if ((e = cudaGetLastError())) return e;
+      }
+      const int64_t blocks = lay.max_chunks * a.H;
+      if (a.T > 0) {
+        if ((e = K(a, map, nseq, blocks, ws, st))) return e;
+        if ((e = F(a, map, units, a.init, ws, nullptr, st))) return e;
+      }
+      if ((e = A(a, map, units, a.dfinal, a.dinit, ws, st))) return e;
+      if (lay.max_chunks == 0) return cudaSuccess;
+      return Bp(a, map, nseq, blocks, ws, st);
+    }
+    const size_t state_floats = (size_t)units * DK * DV;
+    float* ck = reinterpret_cast<float*>(base + lay.ck_off);  // start of window w: ck[w - 1]
+    float* ds = reinterpret_cast<float*>(base + lay.ds_off);  // two state gradients
+    const int nw = (a.T + kBwdWindow - 1) / kBwdWindow;
+    auto window = [&](int w) {
+      const int tw = std::min(kBwdWindow, a.T - w * kBwdWindow);
+      return SeqMap{nullptr, nullptr, sb, tw, a.H, (int64_t)a.T, (int64_t)w * kBwdWindow};
+    };
+    auto blocks_of = [&](const SeqMap& m) { return (int64_t)a.B * ((m.T + C - 1) / C) * a.H; };
+    auto start_state = [&](int w) -> const float* { return w == 0 ? a.init : ck + (w - 1) * state_floats; };
+    for (int w = 0; w + 1 < nw; ++w) {  // checkpoints: the start state of every later window
+      const SeqMap m = window(w);
+      if ((e = K(a, m, nseq, blocks_of(m), ws, st))) return e;
+      if ((e = F(a, m, units, start_state(w), ws, ck + w * state_floats, st))) return e;
+    }
+    for (int w = nw - 1; w >= 0; --w) {
+      const SeqMap m = window(w);
+      if ((e = K(a, m, nseq, blocks_of(m), ws, st))) return e;
+      if ((e = F(a, m, units, start_state(w), ws, nullptr, st))) return e;
+      const float* dfin = w == nw - 1 ? a.dfinal : ds + ((w + 1) & 1) * state_floats;
+      float* dst = w == 0 ? a.dinit : ds + (w & 1) * state_floats;
+      if ((e = A(a, m, units, dfin, dst, ws, st))) return e;
+      if ((e = Bp(a, m, nseq, blocks_of(m), ws, st))) return e;
+    }
+    return cudaSuccess;
+  }
+};
+
 template <typename Tin, int DK>
 cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
-  const WsLayout lay = ws_layout(a.B, a.T, a.H, DK, a.dv_dim, a.cu_seqlens ? a.num_seqs : 0);
-  char* base = static_cast<char*>(a.ws);
-  StatusBlock* sb = reinterpret_cast<StatusBlock*>(base);
-  int32_t* coff = reinterpret_cast<int32_t*>(base + lay.coff_off);
-  float* ws = reinterpret_cast<float*>(base + lay.data_off);
-  cudaError_t e = cudaMemsetAsync(sb, 0, kStatusBytes, st);
-  if (e != cudaSuccess) return e;
-  SeqMap map{a.cu_seqlens, a.cu_seqlens ? coff : nullptr, sb, a.T, a.H};
-  const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
-  if (a.cu_seqlens) {
-    bwd_varlen_plan<<<1, kPlanThreads, 0, st>>>(a.cu_seqlens, a.num_seqs, a.T, coff, sb);
-    if ((e = cudaGetLastError())) return e;
-  }
   switch (a.dv_dim) {
-    case 32: e = launch_scans<Tin, DK, 32>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
-    case 64: e = launch_scans<Tin, DK, 64>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
-    case 128: e = launch_scans<Tin, DK, 128>(a, map, nseq * a.H, lay.max_chunks * a.H, ws, st); break;
-    default: e = cudaErrorInvalidValue;
+    case 32: return Passes<Tin, DK, 32>::run(a, st);
+    case 64: return Passes<Tin, DK, 64>::run(a, st);
+    case 128: return Passes<Tin, DK, 128>::run(a, st);
+    default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess || lay.max_chunks == 0) return e;
-  const size_t smB = BSmem<DK>::bytes;
-  if ((e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB)))
-    return e;
-  bwd_chunk_grads<Tin, DK><<<(unsigned)(lay.max_chunks * a.H), NTH, smB, st>>>(
-      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
-      static_cast<const Tin*>(a.dout), map, nseq, a.dv_dim, a.scale, a.dq, a.dk, a.dg, a.dbeta,
-      ws);
-  return cudaGetLastError();
 }
 
 template <typename Tin>

@@ -326,7 +326,12 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * kda_recurrent_bwd_workspace_size: the 256-byte device status word, the
  * packed batch's chunk offsets, and per (sequence, head) and 32-token chunk
  * two dk x dv states, three 32 x 32 matrices and four 32 x dv tiles; 0 for
- * unsupported shapes) is scratch; outputs must not alias inputs.
+ * unsupported shapes) is scratch; outputs must not alias inputs.  Dense
+ * batches longer than 8192 tokens run in windows of 8192 tokens: the
+ * workspace then holds one window's chunks, the start state of every later
+ * window and two state gradients, so it grows by one dk x dv state per 8192
+ * tokens instead of two per 32; the forward scan runs twice and the results
+ * are identical to an unwindowed run.
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
  */
 KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv,

@@ -286,3 +286,57 @@ def test_backward_varlen_bad_offsets_are_reported():
     assert st == kda.KDA_ERR_BAD_SEQLENS
     for name, t in grads.items():
         assert bool(torch.isnan(t).all()), name
+
+
+# ------------------------------------------------- long sequences (windowed)
+
+def test_backward_windowed_matches_oracle(oracle_mod):
+    """T = 20000 > 8192: the bounded-workspace schedule (windows of 8192
+    tokens, the last ragged, start states checkpointed, the state gradient
+    handed from window to window) against the oracle, with an initial state, a
+    final-state gradient and a scale; every gradient element at the fp32 bar."""
+    B, T, H, d = 1, 20000, 2, 64
+    assert kda.kda_recurrent_bwd_workspace_size(B, T, H, d, d) < \
+        kda.kda_recurrent_bwd_workspace_size(B, 8192, H, d, d) * 1.1
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=301, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, d, dk=d, dtype=torch.bfloat16, seed=302, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    got = gpu_backward(inp, cot, g, 0.9, True, True)
+    ref = oracle_backward(oracle_mod, inp, cot, 0.9, True, True)
+    for n in NAMES:
+        assert np.isfinite(got[n]).all(), n
+        assert rel_l2(got[n], ref[n]) <= TOL_F32, (n, rel_l2(got[n], ref[n]))
+    assert rel_l2(got["d_init"], ref["dS0"]) <= TOL_F32
+
+
+def test_backward_long_sequence_bounded_workspace(oracle_mod):
+    """B1 H32 T = 262,144: the workspace stays bounded (one window's chunks
+    plus a state per window, not two states per 32 tokens), and sampled units
+    match the oracle over the whole sequence at the fp32 bar."""
+    B, T, H, d = 1, 1 << 18, 32, 32
+    per_chunk = 2 * d * d + 3 * 32 * 32 + 4 * 32 * d  # floats per chunk of the full schedule
+    full = B * H * (T // 32) * per_chunk * 4
+    ws_bytes = kda.kda_recurrent_bwd_workspace_size(B, T, H, d, d)
+    assert ws_bytes < full / 20, (ws_bytes, full)
+    inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=311, device=DEV,
+                                init_state=True)
+    cot = W.make_backward_cotangents(B, T, H, d, dk=d, dtype=torch.bfloat16, seed=312, device=DEV)
+    g = gpu_gate(inp["z"], inp["A_log"])
+    nan = lambda *s: torch.full(s, float("nan"), device=DEV)
+    grads = dict(dq=nan(B, T, H, d), dk=nan(B, T, H, d), dv=nan(B, T, H, d),
+                 dg=nan(B, T, H, d), dbeta=nan(B, T, H), d_init=nan(B, H, d, d))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
+    kda.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], g, inp["beta"], cot["dout"], grads, ws,
+                          init_state=inp["init_state"], d_final=cot["d_final"])
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
+    for n, t in grads.items():
+        assert torch.isfinite(t).all(), n
+    for h in (0, 21):
+        ui, uc = unit_inputs(inp, cot, 0, h)
+        ref = oracle_backward(oracle_mod, ui, uc, 1.0, True, True)
+        for n in NAMES:
+            got = to64(grads[n][0:1, :, h:h + 1])
+            assert rel_l2(got, ref[n]) <= TOL_F32, (h, n, rel_l2(got, ref[n]))
+        assert rel_l2(to64(grads["d_init"][0:1, h:h + 1]), ref["dS0"]) <= TOL_F32
