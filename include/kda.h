@@ -330,8 +330,10 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * batches longer than 8192 tokens run in windows of 8192 tokens: the
  * workspace then holds one window's chunks, the start state of every later
  * window and two state gradients, so it grows by one dk x dv state per 8192
- * tokens instead of two per 32; the forward scan runs twice and the results
- * are identical to an unwindowed run.
+ * tokens instead of two per 32.  The forward scan runs twice (once to
+ * checkpoint the window start states, once per window from its checkpoint);
+ * every per-chunk step is the same arithmetic as in a single pass, with the
+ * fp32 state and state gradient handed across windows unrounded.
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
  */
 KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv,
