@@ -51,6 +51,8 @@ WORKLOADS = {
                    steps=1024, seed=4),
     "backward": dict(name="backward B8 H32 T4096 d128", B=8, T=4096, H=32, dk=128, dv=128,
                      seed=3, varlen=False),
+    "spec_decode": dict(name="speculative verify/replay N256 H32 d128, K=4 draft tokens", N=256,
+                        H=32, dk=128, dv=128, K=4, seed=7),
 }
 
 # bytes per (token, head) of the chunkwise forward, bf16 q/k/v/o, fp32 g/beta:
@@ -640,6 +642,68 @@ def oracle_decode_sample(wl, budget_s=10.0):
     return steps / t_used, nthreads, f"{steps} of {wl['steps']} steps (all {N * H} heads)", t_used
 
 
+def oracle_spec_sample(wl, budget_s=10.0):
+    """The oracle verifying the K draft tokens of every head from its
+    committed state (the recurrence over K tokens, outputs kept, the state
+    left as it was), repeated until the budget is spent."""
+    import oracle
+    N, H, d, K = wl["N"], wl["H"], wl["dk"], wl["K"]
+    nthreads = oracle.default_threads()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_prefill_inputs(N, K, H, d, d, torch.bfloat16, seed=wl["seed"], device=dev)
+    S = W.make_decode_state(N, H, d, d, wl["seed"] + 1, dev).cpu().double().numpy()
+    x = {k: inp[k].detach().to("cpu", torch.float64).numpy() for k in ("q", "k", "v", "z", "beta")}
+    A_log = inp["A_log"].detach().cpu().double().numpy()
+    t_used, launches = 0.0, 0
+    while t_used < budget_s and launches < 1000:
+        t0 = time.perf_counter()
+        g = oracle.gate(x["z"], A_log, -5.0)
+        oracle.forward(x["q"], x["k"], x["v"], g, x["beta"], init_state=S, nthreads=nthreads)
+        t_used += time.perf_counter() - t0
+        launches += 1
+    return (launches * N * K / t_used, nthreads,
+            f"{launches} verify launches (all {N * H} heads, K = {K})", t_used)
+
+
+def bench_spec_line(args, wl, world, rank, peaks):
+    """Speculative decoding on its own line: verify (the step) and replay."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    N, K = wl["N"], wl["K"]
+    reps = max(args.steps, 20)
+    clocks = None if args.no_clocks else ClockSampler(dev.index)
+    barrier(world)
+    res, bv, br, _ = run_spec_decode(dev, N=N, H=wl["H"], d=wl["dk"], K=K, reps=reps,
+                                     seed=wl["seed"])
+    clk = clocks.stop() if clocks else None
+    vms = max_over_ranks(res["verify"], world)
+    rms = max_over_ranks(res["replay"], world)
+    vach, rach = bv / (vms * 1e-3) / 1e9, br / (rms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(N * K * world / (vms * 1e-3) / 1e6, 3),
+        "unit": "M draft tokens/s (verify)", "n_gpus": world, "steps": reps, "warmup": 3,
+        "ms_per_step": round(vms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["name"], "parallelism": f"dp{world} (independent batches)",
+                   "l2": "state (537 MB) larger than L2",
+                   "step": "kda_decode_verify (gate fused)"},
+        "roofline": {"bound": "hbm", "achieved": round(vach, 1), "peak": peaks["hbm"],
+                     "unit": "GB/s", "frac": round(vach / peaks["hbm"], 4), "traffic": None,
+                     "kernel": "decode_multi_kernel (verify)", "kernel_ms": round(vms, 4),
+                     "algorithmic_bytes": bv},
+        "replay": {"ms": round(rms, 4),
+                   "roofline": {"bound": "hbm", "achieved": round(rach, 1), "peak": peaks["hbm"],
+                                "unit": "GB/s", "frac": round(rach / peaks["hbm"], 4),
+                                "algorithmic_bytes": br}},
+        "gpu_launches": 2 * reps, "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, secs = oracle_spec_sample(wl)
+        line["cpu_baseline"] = {"value": round(v / 1e6, 6), "unit": "M draft tokens/s (verify)",
+                                "cores": cores, "kind": "oracle",
+                                "sample": sample + f", {secs:.1f} s"}
+    return line
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -692,6 +756,8 @@ def main():
         line = bench_decode_line(args, wl, world, rank, peaks)
     elif args.workload == "backward":
         line = bench_backward_line(args, wl, world, rank, peaks)
+    elif args.workload == "spec_decode":
+        line = bench_spec_line(args, wl, world, rank, peaks)
     else:
         line = bench_prefill_line(args, wl, world, rank, peaks)
     if rank == 0:
@@ -936,6 +1002,14 @@ def run_reference(args, wl, world):
             t_per.append(1.0 / v)
         value = 1.0 / statistics.mean(t_per)
         unit = "steps/s"
+        cfg = {"workload": wl["name"]}
+    elif args.workload == "spec_decode":
+        vals = []
+        for _ in range(args.steps):
+            v, cores, sample, secs = oracle_spec_sample(wl, budget_s=5.0)
+            vals.append(v / 1e6)
+        value = statistics.mean(vals)
+        unit = "M draft tokens/s (verify)"
         cfg = {"workload": wl["name"]}
     else:
         inp, cu, T, N = make_prefill(wl, dev)
