@@ -12,6 +12,8 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
+# the same sources built with device-side bounds checks (KDA_DEBUG_CHECKS)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libkda_debug.so")
 
 KDA_OK = 0
 KDA_ERR_INVALID_ARG = 1
@@ -21,6 +23,7 @@ KDA_ERR_WORKSPACE = 4
 KDA_ERR_CUDA = 5
 KDA_ERR_TIMEOUT = 6
 KDA_ERR_BAD_SEQLENS = 7
+KDA_ERR_BOUNDS = 8
 
 KDA_F32 = 0
 KDA_BF16 = 1
@@ -63,10 +66,13 @@ _SIGNATURES = {
     "kda_get_device_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "kda_noalloc_get_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _VP]),
     "kda_selftest_bounded_wait": (_I, [_VP, _I64, _VP]),
+    "kda_debug_checks_enabled": (_I, []),
+    "kda_selftest_bounds_check": (_I, [_VP, _VP]),
     "kda_set_wait_limit_ns": (_I, [_I64]),
 }
 
 _lib = None
+_lib_path = LIB_PATH
 
 
 class KdaError(RuntimeError):
@@ -78,21 +84,38 @@ class KdaError(RuntimeError):
         super().__init__(msg)
 
 
+def _load(path):
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{os.path.basename(path)} not found at {path}; build it with "
+            "`python -m gated_delta_rule_158_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
 def lib():
-    """The loaded libkda.so (raises if it is missing: there is no fallback)."""
+    """The selected library, libkda.so unless select_library(debug=True) was
+    called (raises if it is missing: there is no fallback)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"libkda.so not found at {LIB_PATH}; build it with "
-                "`python -m gated_delta_rule_158_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in _SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+def select_library(debug: bool):
+    """Routes every call of this module to libkda_debug.so (debug=True) or
+    libkda.so.  Returns the previously selected library's path."""
+    global _lib, _lib_path
+    prev = _lib_path
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if path != _lib_path or _lib is None:
+        _lib = _load(path)
+        _lib_path = path
+    return prev
 
 
 def _ptr(t):
@@ -329,6 +352,15 @@ def kda_noalloc_get_device_status(stream=None):
 def kda_set_wait_limit_ns(limit_ns):
     """Diagnostic: bound of the chunk kernel's internal waits (default 2e9 ns)."""
     _check(lib().kda_set_wait_limit_ns(int(limit_ns)), "kda_set_wait_limit_ns")
+
+
+def kda_debug_checks_enabled() -> bool:
+    return bool(lib().kda_debug_checks_enabled())
+
+
+def kda_selftest_bounds_check(workspace, stream=None):
+    _check(lib().kda_selftest_bounds_check(_ptr(workspace), _stream(stream)),
+           "kda_selftest_bounds_check")
 
 
 def kda_selftest_bounded_wait(workspace, spin_limit_ns, stream=None):

@@ -99,6 +99,18 @@ cudaError_t launch_varlen_plan(const int32_t* cu_seqlens, int num_seqs, int T, i
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------- bounds-check selftest
+__global__ void selftest_bounds_kernel(StatusBlock* sb) {
+  // index 1 in a buffer of one element: the debug check records the failure;
+  // nothing is read or written either way
+  (void)in_bounds(sb, 1, 1, kSiteSelftest);
+}
+
+cudaError_t launch_selftest_bounds(StatusBlock* sb, cudaStream_t stream) {
+  selftest_bounds_kernel<<<1, 1, 0, stream>>>(sb);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns, cudaStream_t stream) {
   selftest_wait_kernel<<<1, 32, 0, stream>>>(sb, limit_ns);
   return cudaGetLastError();
@@ -120,6 +132,7 @@ const char* kda_status_string(kda_status s) {
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
     case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS";
+    case KDA_ERR_BOUNDS: return "KDA_ERR_BOUNDS";
   }
   return "KDA_ERR_UNKNOWN";
 }
@@ -537,6 +550,24 @@ kda_status kda_set_wait_limit_ns(int64_t limit_ns) {
   if (lim > 5000000000LL) lim = 5000000000LL;
   set_wait_limit_ns(lim);
   return KDA_OK;
+}
+
+int kda_debug_checks_enabled(void) {
+#ifdef KDA_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+kda_status kda_selftest_bounds_check(void* workspace, void* stream) {
+  if (!workspace) return KDA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return KDA_ERR_MISALIGNED;
+  if (!kda_debug_checks_enabled()) return KDA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaError_t em = cudaMemsetAsync(workspace, 0, kStatusBytes, st)) return cuda_failure(em);
+  const cudaError_t e = launch_selftest_bounds(static_cast<StatusBlock*>(workspace), st);
+  return e == cudaSuccess ? KDA_OK : cuda_failure(e);
 }
 
 kda_status kda_selftest_bounded_wait(void* workspace, int64_t spin_limit_ns, void* stream) {

@@ -35,6 +35,7 @@
 #include <algorithm>
 
 #include "kda_bwd.cuh"
+#include "kda_warp_mma.cuh"
 
 namespace kda {
 namespace {
@@ -84,23 +85,6 @@ __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
   for (int i = 0; i < TM; ++i)
 #pragma unroll
     for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-}
-
-// Warp-level tensor-core products in tf32 with fp32 accuracy: each operand
-// x = hi + lo with hi = tf32(x), lo = tf32(x - hi), and a b = a_lo b_hi +
-// a_hi b_lo + a_hi b_hi (the dropped a_lo b_lo is below fp32 rounding).
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
-}
-
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 // m16n8k8 fragments from shared memory (lane = 4 g + t).  A: rows row0 ..
@@ -171,6 +155,8 @@ struct SeqMap {
   int T, H;              // dense: T = tokens processed per sequence (a window of it)
   int64_t row_stride;    // dense: rows from one sequence to the next (0: T)
   int64_t row_off;       // dense: first row of the processed window in each sequence
+  int64_t rows_total;    // rows of the batch (B T)
+  int64_t chunks_total;  // chunk slots of the workspace
 };
 
 struct UnitPos {
@@ -197,6 +183,18 @@ __device__ inline UnitPos unit_pos(const SeqMap& m, int n, int h) {
 }
 
 __device__ inline bool seqs_ok(const SeqMap& m) { return m.cu == nullptr || m.sb->seqlens_ok == 1; }
+
+// KDA_DEBUG_CHECKS builds: a unit's rows lie in the batch and its chunks in
+// the workspace
+__device__ inline bool unit_in_bounds(const SeqMap& m, const UnitPos& up) {
+  StatusBlock* sb = const_cast<StatusBlock*>(m.sb);
+  if (!in_bounds(sb, up.len, m.rows_total + 1, kSiteBwdUnitRows)) return false;
+  if (up.len > 0 && !(in_bounds(sb, up.row0, m.rows_total, kSiteBwdUnitRows) &&
+                      in_bounds(sb, up.row0 + up.len - 1, m.rows_total, kSiteBwdUnitRows)))
+    return false;
+  return up.nc == 0 || (in_bounds(sb, up.chunk0, m.chunks_total, kSiteBwdChunks) &&
+                        in_bounds(sb, up.chunk0 + up.nc - 1, m.chunks_total, kSiteBwdChunks));
+}
 
 // The chunk a block of a per-chunk kernel takes: block = (global chunk cg,
 // head h); dense, chunk cg % nc of sequence cg / nc; packed, the sequence
@@ -354,7 +352,7 @@ __global__ void __launch_bounds__(NTH, 2)
   const int H = map.H;
   int h, c;
   UnitPos up;
-  if (!chunk_of_block(map, N, h, c, up)) return;
+  if (!chunk_of_block(map, N, h, c, up) || !unit_in_bounds(map, up)) return;
   const int t0 = c * C, n = min(C, up.len - t0);
   const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
   const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
@@ -480,6 +478,7 @@ __global__ void __launch_bounds__(NTF, 1)
   const int unit = blockIdx.x;
   const int h = unit % H;
   const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
   const int nc = up.nc;
   const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
   const int tid = threadIdx.x;
@@ -676,6 +675,7 @@ __global__ void __launch_bounds__(NTF, 1)
   const int unit = blockIdx.x;
   const int h = unit % H;
   const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
   const int nc = up.nc;
   const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
   const int tid = threadIdx.x;
@@ -913,7 +913,7 @@ __global__ void __launch_bounds__(NTH, 2)
   const int H = map.H;
   int h, c;
   UnitPos up;
-  if (!chunk_of_block(map, N, h, c, up)) return;
+  if (!chunk_of_block(map, N, h, c, up) || !unit_in_bounds(map, up)) return;
   const int t0 = c * C, n = min(C, up.len - t0);
   const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
   const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
@@ -1371,8 +1371,10 @@ struct Passes {
     if ((e = cudaMemsetAsync(sb, 0, kStatusBytes, st))) return e;
     const int nseq = a.cu_seqlens ? a.num_seqs : a.B;
     const int units = nseq * a.H;
+    const int64_t rows = (int64_t)a.B * a.T;
+    const int64_t chunk_slots = lay.max_chunks * (int64_t)a.H;
     if (!bwd_windowed(a.T, a.cu_seqlens ? a.num_seqs : 0)) {
-      SeqMap map{a.cu_seqlens, a.cu_seqlens ? coff : nullptr, sb, a.T, a.H, 0, 0};
+      SeqMap map{a.cu_seqlens, a.cu_seqlens ? coff : nullptr, sb, a.T, a.H, 0, 0, rows, chunk_slots};
       if (a.cu_seqlens) {
         bwd_varlen_plan<<<1, kPlanThreads, 0, st>>>(a.cu_seqlens, a.num_seqs, a.T, coff, sb);
         if ((e = cudaGetLastError())) return e;
@@ -1392,7 +1394,8 @@ struct Passes {
     const int nw = (a.T + kBwdWindow - 1) / kBwdWindow;
     auto window = [&](int w) {
       const int tw = std::min(kBwdWindow, a.T - w * kBwdWindow);
-      return SeqMap{nullptr, nullptr, sb, tw, a.H, (int64_t)a.T, (int64_t)w * kBwdWindow};
+      return SeqMap{nullptr, nullptr, sb, tw, a.H, (int64_t)a.T, (int64_t)w * kBwdWindow, rows,
+                    chunk_slots};
     };
     auto blocks_of = [&](const SeqMap& m) { return (int64_t)a.B * ((m.T + C - 1) / C) * a.H; };
     auto start_state = [&](int w) -> const float* { return w == 0 ? a.init : ck + (w - 1) * state_floats; };

@@ -79,6 +79,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     L = (int64_t)map.cu_seqlens[n + 1] - row0;
     sidx = (int64_t)n * H + h;
   }
+  {  // KDA_DEBUG_CHECKS builds: the unit's rows and state slot
+    StatusBlock* sb = const_cast<StatusBlock*>(map.status);
+    const int64_t rows = (int64_t)map.B * map.T;
+    if (!in_bounds(sb, L, rows + 1, kSiteSimtUnitRows) ||
+        (L > 0 && !(in_bounds(sb, row0, rows, kSiteSimtUnitRows) &&
+                    in_bounds(sb, row0 + L - 1, rows, kSiteSimtUnitRows))) ||
+        !in_bounds(sb, sidx, gridDim.x / nslices, kSiteSimtStateSlot))
+      return;
+  }
 
   // g is the log-decay, or z when A_log is given (gate fused in)
   const float a_h = A_log ? expf(A_log[h]) : 0.f;

@@ -182,6 +182,14 @@ struct Unit {
   float* final_state;
 };
 
+// KDA_DEBUG_CHECKS builds: the rows [row0, row0 + len) lie in the batch
+__device__ __forceinline__ bool unit_rows_ok(const TcParams& P, int64_t row0, int64_t len) {
+  const int64_t rows = (int64_t)P.B * P.T;
+  return in_bounds(P.sb, len, rows + 1, kSiteTcUnitRows) &&
+         (len == 0 || (in_bounds(P.sb, row0, rows, kSiteTcUnitRows) &&
+                       in_bounds(P.sb, row0 + len - 1, rows, kSiteTcUnitRows)));
+}
+
 __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
   const int H = P.H;
   const size_t DD = (size_t)D * D;
@@ -204,6 +212,10 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
       u.len = (int64_t)P.cu_seqlens[n + 1] - u.row0;
       sidx = (int64_t)n * H + u.h;
     }
+    // one unit per CTA: the state slots are the grid's units
+    if (!unit_rows_ok(P, u.row0, u.len) ||
+        !in_bounds(P.sb, sidx, gridDim.x, kSiteTcStateSlot))
+      return false;
     u.init = P.init_state ? P.init_state + sidx * DD : nullptr;
     u.final_state = P.final_state ? P.final_state + sidx * DD : nullptr;
     return true;
@@ -219,7 +231,11 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
     u.init_identity = kind == 1;
     u.vzero = kind == 1;
     u.out_on = false;
-    u.final_state = P.seg_ws + ((size_t)(un * (P.G - 1) + g) * 2 + kind) * DD;
+    const int64_t slot = (int64_t)(un * (P.G - 1) + g) * 2 + kind;
+    if (!unit_rows_ok(P, u.row0, u.len) ||
+        !in_bounds(P.sb, slot, (int64_t)U * (P.G - 1) * 2, kSiteTcStateSlot))
+      return false;
+    u.final_state = P.seg_ws + (size_t)slot * DD;
     return true;
   }
   // mode 2: outputs of every segment from its true incoming state
@@ -228,10 +244,14 @@ __device__ __forceinline__ bool resolve_unit(const TcParams& P, Unit& u) {
   u.row0 = (int64_t)(un / H) * P.T + (int64_t)g * P.seg_len;
   const int64_t rem = (int64_t)P.T - (int64_t)g * P.seg_len;
   u.len = rem < P.seg_len ? rem : P.seg_len;
-  if (g == 0)
+  if (!unit_rows_ok(P, u.row0, u.len)) return false;
+  if (g == 0) {
     u.init = P.init_state ? P.init_state + (size_t)un * DD : nullptr;
-  else
-    u.init = P.seg_ws + ((size_t)U * (P.G - 1) * 2 + (size_t)un * (P.G - 1) + (g - 1)) * DD;
+  } else {
+    const int64_t slot = (int64_t)U * (P.G - 1) * 2 + (int64_t)un * (P.G - 1) + (g - 1);
+    if (!in_bounds(P.sb, slot, (int64_t)U * (P.G - 1) * 3, kSiteTcStateSlot)) return false;
+    u.init = P.seg_ws + (size_t)slot * DD;
+  }
   u.final_state = (g == P.G - 1 && P.final_state) ? P.final_state + (size_t)un * DD : nullptr;
   return true;
 }
@@ -706,7 +726,9 @@ __global__ void __maxnreg__(128) chunk_tc_kernel(const __grid_constant__ TcParam
       float vo[32];  // O^T (lane j, column r)
       tmem_ld32(tbase + lane_base + o_col(b), vo);
       wait_ld();
-      if (U.out_on) {  // lanes j, j^1 swap values so each writes a bf16 pair
+      if (U.out_on && in_bounds(P.sb, U.row0 + (int64_t)c * C + chunk_rows(c) - 1,
+                                (int64_t)P.B * P.T, kSiteTcOutRows)) {
+        // lanes j, j^1 swap values so each writes a bf16 pair
         const int n = chunk_rows(c);
         const bool odd = lane & 1;
         const int jp = j & ~1;

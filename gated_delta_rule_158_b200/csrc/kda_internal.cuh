@@ -28,6 +28,33 @@ __device__ __forceinline__ void record_status(StatusBlock* sb, int32_t code,
   if (atomicCAS(&sb->status, 0, code) == 0) atomicExch(&sb->detail, detail);
 }
 
+// Device bounds checks of the KDA_DEBUG_CHECKS build: an index outside
+// [0, limit) records KDA_ERR_BOUNDS with the check site as detail and the
+// caller skips the access.  Release builds compile the check away (true).
+__device__ __forceinline__ bool in_bounds(StatusBlock* sb, int64_t idx, int64_t limit,
+                                          int32_t site) {
+#ifdef KDA_DEBUG_CHECKS
+  if (idx >= 0 && idx < limit) return true;
+  record_status(sb, KDA_ERR_BOUNDS, site);
+  return false;
+#else
+  (void)sb; (void)idx; (void)limit; (void)site;
+  return true;
+#endif
+}
+
+// check sites (the detail recorded with KDA_ERR_BOUNDS)
+enum BoundsSite : int32_t {
+  kSiteSelftest = 0x5E1F,
+  kSiteTcUnitRows = 0xB101,    // chunk_tc_kernel: a unit's rows within the batch
+  kSiteTcStateSlot = 0xB102,   // chunk_tc_kernel: init / final / segment state slot
+  kSiteTcOutRows = 0xB103,     // chunk_tc_kernel: rows of o a chunk stores
+  kSiteSimtUnitRows = 0xB201,  // chunk_simt_kernel: a unit's rows
+  kSiteSimtStateSlot = 0xB202, // chunk_simt_kernel: state slot
+  kSiteBwdUnitRows = 0xB401,   // backward: a unit's rows within the batch
+  kSiteBwdChunks = 0xB402,     // backward: a unit's chunk slice of the workspace
+};
+
 // --------------------------------------------------------------- element io
 template <typename T> struct Elem;
 template <> struct Elem<float> {
@@ -131,6 +158,7 @@ cudaError_t launch_state_prefix(const float* pairs, int count, int index, const 
 // Bound of every mbarrier wait in the tensor-core chunk kernel (diagnostics).
 void set_wait_limit_ns(long long ns);
 
+cudaError_t launch_selftest_bounds(StatusBlock* sb, cudaStream_t stream);
 cudaError_t launch_selftest_wait(StatusBlock* sb, long long limit_ns,
                                  cudaStream_t stream);
 

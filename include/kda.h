@@ -32,6 +32,15 @@
  *    returns KDA_ERR_CUDA.  Problems found on the device (a bounded wait that
  *    ran out, malformed cu_seqlens) are never trapped: they are written to a
  *    status word in the workspace, read back with kda_get_device_status().
+ *  - Debug builds (the same sources compiled with -DKDA_DEBUG_CHECKS, shipped
+ *    as libkda_debug.so beside libkda.so) add device-side bounds checks where
+ *    a kernel derives an index from data or from a split plan: the unit and
+ *    segment a CTA resolves (rows from cu_seqlens or the segment plan, state
+ *    slots), the rows of o a chunk stores, the backward's per-chunk workspace
+ *    slices and gradient rows.  A failed check records KDA_ERR_BOUNDS (detail:
+ *    the check site) in the workspace status word and the access is skipped;
+ *    nothing traps.  The decode kernels (no workspace, no status word) are not
+ *    instrumented.  Release builds compile the checks away.
  */
 #ifndef LIBKDA_KDA_H_
 #define LIBKDA_KDA_H_
@@ -57,7 +66,8 @@ typedef enum kda_status {
   KDA_ERR_WORKSPACE = 4,    /* workspace missing or too small */
   KDA_ERR_CUDA = 5,         /* a CUDA launch or runtime call failed */
   KDA_ERR_TIMEOUT = 6,      /* device: a bounded wait gave up */
-  KDA_ERR_BAD_SEQLENS = 7   /* device: cu_seqlens not monotone / not ending at T */
+  KDA_ERR_BAD_SEQLENS = 7,  /* device: cu_seqlens not monotone / not ending at T */
+  KDA_ERR_BOUNDS = 8        /* device, KDA_DEBUG_CHECKS builds: an index left its buffer */
 } kda_status;
 
 typedef enum kda_dtype { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
@@ -371,6 +381,20 @@ KDA_API kda_status kda_get_device_status(const void *workspace, void *stream,
  * KDA_ERR_TIMEOUT in the status word exactly as the chunk kernels do when
  * one of their waits runs out.  Needs 256 bytes of workspace.
  */
+/*
+ * 1 in a KDA_DEBUG_CHECKS build, 0 otherwise (host only, no CUDA call).
+ */
+KDA_API int kda_debug_checks_enabled(void);
+
+/*
+ * Diagnostic for the debug build's bounds checks: launches one thread that
+ * asks the device-side check whether index 1 lies in a buffer of 1 element.
+ * The check records KDA_ERR_BOUNDS (detail 0x5E1F) in the status word of
+ * `workspace` (256 bytes needed) and no memory is accessed.  Returns
+ * KDA_ERR_UNSUPPORTED without launching in a release build.
+ */
+KDA_API kda_status kda_selftest_bounds_check(void *workspace, void *stream);
+
 KDA_API kda_status kda_selftest_bounded_wait(void *workspace, int64_t spin_limit_ns,
                                      void *stream);
 

@@ -40,10 +40,27 @@ def test_library_exports_every_declared_symbol(L):
     assert set(_lib._SIGNATURES) == declared
 
 
+def test_debug_library_exports_the_same_symbols_and_reports_its_checks(L):
+    """libkda_debug.so (KDA_DEBUG_CHECKS) has the release ABI; only its
+    kda_debug_checks_enabled answers 1, and its bounds selftest rejects bad
+    arguments on the host like every other entry point."""
+    D = _lib._load(_lib.DEBUG_LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(D, name), name
+    assert D.kda_debug_checks_enabled() == 1
+    assert L.kda_debug_checks_enabled() == 0
+    assert D.kda_selftest_bounds_check(None, None) == kda.KDA_ERR_INVALID_ARG
+    assert D.kda_selftest_bounds_check(FAKE + 4, None) == kda.KDA_ERR_MISALIGNED
+    # the release build has no checks to exercise: refused before any launch
+    assert L.kda_selftest_bounds_check(FAKE, None) == kda.KDA_ERR_UNSUPPORTED
+    assert D.kda_status_string(8) == b"KDA_ERR_BOUNDS"
+
+
 def test_status_strings(L):
     for code, name in [(0, "KDA_OK"), (1, "KDA_ERR_INVALID_ARG"), (2, "KDA_ERR_UNSUPPORTED"),
                        (3, "KDA_ERR_MISALIGNED"), (4, "KDA_ERR_WORKSPACE"), (5, "KDA_ERR_CUDA"),
-                       (6, "KDA_ERR_TIMEOUT"), (7, "KDA_ERR_BAD_SEQLENS")]:
+                       (6, "KDA_ERR_TIMEOUT"), (7, "KDA_ERR_BAD_SEQLENS"),
+                       (8, "KDA_ERR_BOUNDS")]:
         assert kda.kda_status_string(code) == name
     assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
 
