@@ -418,6 +418,37 @@ def test_decode_replay_accepted_prefix(oracle_mod, dtype):
         assert rel_l2(to64(state[n]), S_ref[0]) <= tol
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_verify_replay_strong_decay(oracle_mod, dtype):
+    """Raw log-decays down to -12 per token over 12 draft tokens (cumulative
+    decays far below fp32's normal range) beside heads with mild decays in
+    the same launch: outputs and replayed states against the oracle."""
+    N, K, H, d = 3, 12, 4, 64
+    inp, S0 = _draft_inputs(N, K, H, d, d, dtype, seed=140)
+    gen = torch.Generator(device=DEV).manual_seed(141)
+    g = -6.0 - 6.0 * torch.rand((N, K, H, d), generator=gen, device=DEV)
+    g[:, :, 2:] *= 0.02  # heads 2, 3: cumulative decay stays well inside the range
+    out = torch.full((N, K, H, d), float("nan"), dtype=dtype, device=DEV)
+    kda.kda_decode_verify(inp["q"], inp["k"], inp["v"], g, inp["beta"], S0, out, scale=0.9)
+    state = S0.clone()
+    acc = torch.tensor([K, 5, 1], dtype=torch.int32, device=DEV)
+    kda.kda_decode_replay(inp["k"], inp["v"], g, inp["beta"], state, acc)
+    torch.cuda.synchronize()
+    o_ref, _ = oracle_mod.forward(to64(inp["q"]), to64(inp["k"]), to64(inp["v"]), to64(g),
+                                  to64(inp["beta"]), init_state=to64(S0), scale=0.9)
+    tol_o = TOL_F32 if dtype == torch.float32 else TOL_BF16_O
+    tol_s = TOL_F32 if dtype == torch.float32 else TOL_BF16_S
+    for h in range(H):
+        assert rel_l2(to64(out[:, :, h]), o_ref[:, :, h]) <= tol_o, h
+    for n, m in enumerate(acc.tolist()):
+        sl = lambda t: t[n:n + 1, :m]
+        _, S_ref = oracle_mod.forward(to64(sl(inp["q"])), to64(sl(inp["k"])), to64(sl(inp["v"])),
+                                      to64(sl(g)), to64(sl(inp["beta"])),
+                                      init_state=to64(S0[n:n + 1]))
+        for h in range(H):
+            assert rel_l2(to64(state[n, h]), S_ref[0, h]) <= tol_s, (n, h)
+
+
 def test_verify_then_replay_equals_step_by_step():
     """verify(K) outputs and replay(K) state equal K single decode steps."""
     N, K, H, d = 4, 6, 2, 128
