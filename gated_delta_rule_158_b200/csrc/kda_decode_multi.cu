@@ -130,10 +130,14 @@ __global__ void __launch_bounds__(threads_per_cta<DV>())
   constexpr int NW = NT / 32;
   constexpr int RPL = DK / kRowLanes;      // key rows per lane
   constexpr int EPL = DK / 32;             // key elements per lane when staging a token
-  static_assert(DVC % kWarpCols == 0 && RPL % 4 == 0, "tile shape");
+  // token rows in shared memory: each row lane's RPL keys padded by 4 floats,
+  // so the 8 row lanes' float4 reads fall in distinct bank groups
+  constexpr int RPS = RPL + 4, KS = kRowLanes * RPS;
+  static_assert(DVC % kWarpCols == 0 && RPL % 4 == 0 && RPL % EPL == 0, "tile shape");
+  auto kpos = [](int i) { return (i / RPL) * RPS + i % RPL; };
 
   // read as float4
-  __shared__ __align__(16) float sk[kMaxK][DK], sq[VERIFY ? kMaxK : 1][DK], sa[kMaxK][DK];
+  __shared__ __align__(16) float sk[kMaxK][KS], sq[VERIFY ? kMaxK : 1][KS], sa[kMaxK][KS];
   __shared__ __align__(16) float sv[kMaxK][DVC];
   __shared__ float sb[kMaxK], skq[kMaxK];
 
@@ -178,10 +182,10 @@ __global__ void __launch_bounds__(threads_per_cta<DV>())
       av[e] = expf(A_log ? gate_value(gv[e], a_h, g_min) : gv[e]);
       if (VERIFY) kq = fmaf(kv[e], qv[e], kq);
     }
-    store_vec<EPL>(&sk[t][lane * EPL], kv);
-    store_vec<EPL>(&sa[t][lane * EPL], av);
+    store_vec<EPL>(&sk[t][kpos(lane * EPL)], kv);
+    store_vec<EPL>(&sa[t][kpos(lane * EPL)], av);
     if (VERIFY) {
-      store_vec<EPL>(&sq[t][lane * EPL], qv);
+      store_vec<EPL>(&sq[t][kpos(lane * EPL)], qv);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
       if (lane == 0) skq[t] = kq;
@@ -199,9 +203,9 @@ __global__ void __launch_bounds__(threads_per_cta<DV>())
   for (int t = 0; t < steps; ++t) {
     // decay, then p = S^T k and (verify) r = S^T q over this lane's rows
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f), rq = p;
-    const float4* k4 = reinterpret_cast<const float4*>(&sk[t][rl * RPL]);
-    const float4* q4 = reinterpret_cast<const float4*>(&sq[VERIFY ? t : 0][rl * RPL]);
-    const float4* a4 = reinterpret_cast<const float4*>(&sa[t][rl * RPL]);
+    const float4* k4 = reinterpret_cast<const float4*>(&sk[t][rl * RPS]);
+    const float4* q4 = reinterpret_cast<const float4*>(&sq[VERIFY ? t : 0][rl * RPS]);
+    const float4* a4 = reinterpret_cast<const float4*>(&sa[t][rl * RPS]);
 #pragma unroll
     for (int r4 = 0; r4 < RPL / 4; ++r4) {
       const float4 kk = k4[r4], aa = a4[r4];
