@@ -69,7 +69,7 @@ def prefill_flops_per_token_head(C=32, dk=128, dv=128):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # chunk_tc_kernel launch, from the ncu capture summarised in
 # profiles/chunk_tc_kernel_prefill_B4_H32_T4096.md (128 (sequence, head) units
-# of 4096 tokens): 673.5 MB read + 122.5 MB written.  Traffic grows with the
+# of 4096 tokens): 673.5 MB read + 123.2 MB written.  Traffic grows with the
 # units a launch processes, so a launch over U such units moves U times the
 # per-unit figure.  The figure belongs to the kernel it was taken on: the
 # text of kda_chunk_tc.cu up to the end of chunk_tc_kernel (its constants,
@@ -81,8 +81,8 @@ CHUNK_TRAFFIC = {
     "headers": ["gated_delta_rule_158_b200/csrc/kda_sync.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
-    "sha256": "9845a17161ba29d48b43ab01805a000c1ba00f5fa867c7b1cc322202029cf9d5",
-    "bytes_per_unit_T4096": (673.471488e6 + 122.477568e6) / 128,
+    "sha256": "8a05c507432424c7366a5b0fd3a8c1621893ebaf761e27b0fb20e9d7f844415f",
+    "bytes_per_unit_T4096": (673.474560e6 + 123.213312e6) / 128,
 }
 
 
