@@ -445,11 +445,16 @@ __global__ void __launch_bounds__(NTH, 2)
 // R = V - Ka S, U = T R (T = X Diag(beta) from pass K) and the state update.
 template <int DK, int DV>
 struct FSmem {
-  static constexpr int LDK = DK + 1, LDV = DV + 1;
-  static constexpr int floats = 3 * C * LDK       // k (then Kc), Gamma, Ka
+  // Tile strides (floats) chosen for the m16n8k8 fragment loads: a row-major
+  // A operand (lane g, t reads row g, column t) is conflict-free at a stride
+  // of 4 (mod 32), a transposed A or a [K][N] B operand (row t, column g) at
+  // 8 (mod 32).  Ka and T are row-major A operands; Kc is a transposed one;
+  // the state, V / R and U are B operands.
+  static constexpr int LDK = DK + 4, LKC = DK + 8, LDV = DV + 8, LDT = C + 4;
+  static constexpr int floats = C * LKC + 2 * C * LDK  // k (then Kc); Gamma, Ka
                                 + DK * LDV        // state
                                 + 2 * C * LDV     // V (then R), U
-                                + C * LDC         // T
+                                + C * LDT         // T
                                 + C + 2 * DK;     // beta, Gamma_C, e^{Gamma_C}
   static constexpr size_t bytes = sizeof(float) * floats;
 };
@@ -460,16 +465,17 @@ __global__ void __launch_bounds__(NTF, 1)
                  const float* __restrict__ g, const float* __restrict__ beta,
                  const float* __restrict__ init, SeqMap map, float* __restrict__ ws,
                  float* __restrict__ fin) {
-  constexpr int LDK = DK + 1, LDV = DV + 1;
+  constexpr int LDK = FSmem<DK, DV>::LDK, LKC = FSmem<DK, DV>::LKC;
+  constexpr int LDV = FSmem<DK, DV>::LDV, LDT = FSmem<DK, DV>::LDT;
   extern __shared__ float sm[];
-  float* kS = sm;                 // [C][LDK]  k, then Kc
-  float* GS = kS + C * LDK;       // [C][LDK]  Gamma
+  float* kS = sm;                 // [C][LKC]  k, then Kc
+  float* GS = kS + C * LKC;       // [C][LDK]  Gamma
   float* KaS = GS + C * LDK;      // [C][LDK]  Ka
   float* SS = KaS + C * LDK;      // [DK][LDV] state
   float* VS = SS + DK * LDV;      // [C][LDV]  V, then R = V - Ka S
   float* US = VS + C * LDV;       // [C][LDV]
-  float* TS = US + C * LDV;       // [C][LDC]
-  float* bS = TS + C * LDC;       // [C]
+  float* TS = US + C * LDV;       // [C][LDT]
+  float* bS = TS + C * LDT;       // [C]
   float* gC = bS + C;             // [DK] Gamma_C
   float* eC = gC + DK;            // [DK] e^{Gamma_C}
 
@@ -499,7 +505,7 @@ __global__ void __launch_bounds__(NTF, 1)
         kv = Elem<Tin>::load(k + off);
         gv = g[off];
       }
-      kS[r * LDK + i] = kv;
+      kS[r * LKC + i] = kv;
       GS[r * LDK + i] = gv;
     }
     for (int idx = tid; idx < C * DV; idx += NTF) {
@@ -523,14 +529,14 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     for (int idx = tid; idx < C * C; idx += NTF) {  // T = X Diag(beta)
       const int r = idx / C, s2 = idx % C;
-      TS[r * LDC + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
+      TS[r * LDT + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka, Kc (into kS)
       const int r = idx / DK, i = idx % DK;
-      const float G = GS[r * LDK + i], kv = kS[r * LDK + i];
+      const float G = GS[r * LDK + i], kv = kS[r * LKC + i];
       KaS[r * LDK + i] = kv * expf(G);
-      kS[r * LDK + i] = kv * expf(gC[i] - G);
+      kS[r * LKC + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
     if constexpr (DK == 128 && DV == 128) {
@@ -559,7 +565,7 @@ __global__ void __launch_bounds__(NTF, 1)
         zero(acc);
         for (int k0 = 0; k0 < C; k0 += 8) {
           Frag3 a;
-          load_a(a, TS, LDC, 16 * mt, k0);
+          load_a(a, TS, LDT, 16 * mt, k0);
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, VS, LDV, 8 * (nt0 + q2), k0);
         }
@@ -580,7 +586,7 @@ __global__ void __launch_bounds__(NTF, 1)
         zero(acc);
         for (int k0 = 0; k0 < C; k0 += 8) {
           Frag3 a;
-          load_a<true>(a, kS, LDK, 16 * mt8, k0);
+          load_a<true>(a, kS, LKC, 16 * mt8, k0);
 #pragma unroll
           for (int q2 = 0; q2 < 8; ++q2) mma3<true>(acc[q2], a, US, LDV, 8 * (nt8 + q2), k0);
         }
@@ -604,7 +610,7 @@ __global__ void __launch_bounds__(NTF, 1)
       {  // U = T R
         float acc[1][DV / 16];
         zero(acc);
-        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDC + kk]; },
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDT + kk]; },
                                  [&](int kk, int nn) { return VS[kk * LDV + nn]; });
         for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
       }
@@ -617,7 +623,7 @@ __global__ void __launch_bounds__(NTF, 1)
       {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
         float acc[DK / 32][DV / 16];
         zero(acc);
-        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LDK + m]; },
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LKC + m]; },
                                         [&](int kk, int nn) { return US[kk * LDV + nn]; });
         for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
           SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
@@ -639,11 +645,15 @@ __global__ void __launch_bounds__(NTF, 1)
 // decays once per chunk).
 template <int DK, int DV>
 struct ASmem {
-  static constexpr int LDK = DK + 1, LDV = DV + 1;
-  static constexpr int floats = 3 * C * LDK       // q (then Qg), k (then Kc), Gamma (then Ka)
+  // Tile strides (floats) for conflict-free m16n8k8 fragment loads (row-major
+  // A operand: 4 (mod 32); transposed A or [K][N] B operand: 8 (mod 32)).
+  // Kc is a row-major A operand; Qg, Ka, A_qk and T are transposed ones; the
+  // state gradient, dO', dU and W are B operands.
+  static constexpr int LDK = DK + 4, LQT = DK + 8, LDV = DV + 8, LDQ = C + 8;
+  static constexpr int floats = C * LDK + 2 * C * LQT  // k (then Kc); q (then Qg), Gamma (then Ka)
                                 + DK * LDV        // state gradient
                                 + 3 * C * LDV     // dO', dU, W
-                                + 2 * C * LDC     // A_qk, T
+                                + 2 * C * LDQ     // A_qk, T
                                 + C + 2 * DK;     // beta, Gamma_C, e^{Gamma_C}
   static constexpr size_t bytes = sizeof(float) * floats;
 };
@@ -655,18 +665,19 @@ __global__ void __launch_bounds__(NTF, 1)
                         const Tin* __restrict__ dout, const float* __restrict__ dfinal,
                         SeqMap map, float scale, float* __restrict__ dv,
                         float* __restrict__ dinit, float* __restrict__ ws) {
-  constexpr int LDK = DK + 1, LDV = DV + 1;
+  constexpr int LDK = ASmem<DK, DV>::LDK, LQT = ASmem<DK, DV>::LQT;
+  constexpr int LDV = ASmem<DK, DV>::LDV, LDQ = ASmem<DK, DV>::LDQ;
   extern __shared__ float sm[];
-  float* qS = sm;                 // [C][LDK]  q, later Qg
-  float* kS = qS + C * LDK;       // [C][LDK]  k, later Kc
-  float* GS = kS + C * LDK;       // [C][LDK]  Gamma, later Ka
-  float* dSS = GS + C * LDK;      // [DK][LDV] state gradient
+  float* qS = sm;                 // [C][LQT]  q, later Qg
+  float* kS = qS + C * LQT;       // [C][LDK]  k, later Kc
+  float* GS = kS + C * LDK;       // [C][LQT]  Gamma, later Ka
+  float* dSS = GS + C * LQT;      // [DK][LDV] state gradient
   float* dOS = dSS + DK * LDV;    // [C][LDV]  scale dO
   float* dUS = dOS + C * LDV;     // [C][LDV]
   float* WS = dUS + C * LDV;      // [C][LDV]
-  float* AqS = WS + C * LDV;      // [C][LDC]
-  float* TS = AqS + C * LDC;      // [C][LDC]
-  float* bS = TS + C * LDC;       // [C]
+  float* AqS = WS + C * LDV;      // [C][LDQ]
+  float* TS = AqS + C * LDQ;      // [C][LDQ]
+  float* bS = TS + C * LDQ;       // [C]
   float* gC = bS + C;             // [DK]
   float* eC = gC + DK;            // [DK]
 
@@ -697,9 +708,9 @@ __global__ void __launch_bounds__(NTF, 1)
         kv = Elem<Tin>::load(k + off);
         gv = g[off];
       }
-      qS[r * LDK + i] = qv;
+      qS[r * LQT + i] = qv;
       kS[r * LDK + i] = kv;
-      GS[r * LDK + i] = gv;
+      GS[r * LQT + i] = gv;
     }
     for (int idx = tid; idx < C * DV; idx += NTF) {
       const int r = idx / DV, j = idx % DV;
@@ -715,8 +726,8 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
       float acc = 0.f;
       for (int r = 0; r < C; ++r) {
-        acc += GS[r * LDK + i];
-        GS[r * LDK + i] = acc;
+        acc += GS[r * LQT + i];
+        GS[r * LQT + i] = acc;
       }
       gC[i] = acc;
       eC[i] = expf(acc);
@@ -724,15 +735,15 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int idx = tid; idx < C * C; idx += NTF) {
       const int r = idx / C, s2 = idx % C;
       const size_t o = ((size_t)c * C + r) * C + s2;
-      AqS[r * LDC + s2] = w.Aqk[o];
-      TS[r * LDC + s2] = w.X[o] * bS[s2];
+      AqS[r * LDQ + s2] = w.Aqk[o];
+      TS[r * LDQ + s2] = w.X[o] * bS[s2];
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {  // Qg, Ka, Kc
       const int r = idx / DK, i = idx % DK;
-      const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LDK + i];
-      qS[r * LDK + i] *= e;
-      GS[r * LDK + i] = kv * e;
+      const float G = GS[r * LQT + i], e = expf(G), kv = kS[r * LDK + i];
+      qS[r * LQT + i] *= e;
+      GS[r * LQT + i] = kv * e;
       kS[r * LDK + i] = kv * expf(gC[i] - G);
     }
     __syncthreads();
@@ -745,7 +756,7 @@ __global__ void __launch_bounds__(NTF, 1)
         zero(acc);
         for (int k0 = 0; k0 < C; k0 += 8) {
           Frag3 a;
-          load_a<true>(a, AqS, LDC, 16 * mt, k0);
+          load_a<true>(a, AqS, LDQ, 16 * mt, k0);
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, dOS, LDV, 8 * (nt0 + q2), k0);
         }
@@ -767,7 +778,7 @@ __global__ void __launch_bounds__(NTF, 1)
         zero(acc);
         for (int k0 = 0; k0 < C; k0 += 8) {
           Frag3 a;
-          load_a<true>(a, TS, LDC, 16 * mt, k0);
+          load_a<true>(a, TS, LDQ, 16 * mt, k0);
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, dUS, LDV, 8 * (nt0 + q2), k0);
         }
@@ -791,8 +802,8 @@ __global__ void __launch_bounds__(NTF, 1)
         zero(acc);
         for (int k0 = 0; k0 < C; k0 += 8) {
           Frag3 a, b;
-          load_a<true>(a, qS, LDK, 16 * mt8, k0);
-          load_a<true>(b, GS, LDK, 16 * mt8, k0, -1.f);
+          load_a<true>(a, qS, LQT, 16 * mt8, k0);
+          load_a<true>(b, GS, LQT, 16 * mt8, k0, -1.f);
 #pragma unroll
           for (int q2 = 0; q2 < 8; ++q2) {
             mma3<true>(acc[q2], a, dOS, LDV, 8 * (nt8 + q2), k0);
@@ -811,7 +822,7 @@ __global__ void __launch_bounds__(NTF, 1)
       {  // dU = A_qk^T dO' + Kc dS
         float acc[1][DV / 16];
         zero(acc);
-        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[kk * LDC + m]; },
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[kk * LDQ + m]; },
                                  [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
         mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return kS[m * LDK + kk]; },
                                   [&](int kk, int nn) { return dSS[kk * LDV + nn]; });
@@ -821,7 +832,7 @@ __global__ void __launch_bounds__(NTF, 1)
       {  // W = T^T dU  (= dv)
         float acc[1][DV / 16];
         zero(acc);
-        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[kk * LDC + m]; },
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[kk * LDQ + m]; },
                                  [&](int kk, int nn) { return dUS[kk * LDV + nn]; });
         for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) {
           WS[m * LDV + nn] = acc[i][j];
@@ -837,9 +848,9 @@ __global__ void __launch_bounds__(NTF, 1)
       {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
         float acc[DK / 32][DV / 16];
         zero(acc);
-        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return qS[kk * LDK + m]; },
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return qS[kk * LQT + m]; },
                                         [&](int kk, int nn) { return dOS[kk * LDV + nn]; });
-        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return -GS[kk * LDK + m]; },
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return -GS[kk * LQT + m]; },
                                         [&](int kk, int nn) { return WS[kk * LDV + nn]; });
         for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
           dSS[m * LDV + nn] = fmaf(eC[m], dSS[m * LDV + nn], acc[i][j]);
