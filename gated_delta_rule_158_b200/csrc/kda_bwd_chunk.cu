@@ -235,12 +235,12 @@ __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int 
   return w;
 }
 
-// chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to C
-template <typename Tin, int DK>
+// chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to
+// C, into [C][LDK] tiles
+template <typename Tin, int DK, int LDK>
 __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const float* beta,
                           size_t rowbase, int H, int n, float* qS, float* kS, float* GS,
                           float* bS) {
-  constexpr int LDK = DK + 1;
   for (int idx = threadIdx.x; idx < C * DK; idx += NTH) {
     const int r = idx / DK, i = idx % DK;
     float qv = 0.f, kv = 0.f, gv = 0.f;
@@ -324,7 +324,9 @@ __global__ void __launch_bounds__(kPlanThreads)
 // (tf32 with the hi/lo split, fp32 accuracy).
 template <int DK>
 struct KSmem {
-  static constexpr int LDK = DK + 1;
+  // 4 (mod 32): the Gram's row-major A operand and its [N][K] B operand are
+  // read by the m16n8k8 fragment loads without bank conflicts
+  static constexpr int LDK = DK + 4;
   static constexpr int floats = 5 * C * LDK       // q (then q factor), k, Gamma, two factors
                                 + 3 * C * LDC     // L, A_qk, X
                                 + C;              // beta
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(NTH, 2)
     bwd_keyside(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 const float* __restrict__ g, const float* __restrict__ beta, SeqMap map, int N,
                 float* __restrict__ ws) {
-  constexpr int LDK = DK + 1;
+  constexpr int LDK = KSmem<DK>::LDK;
   extern __shared__ float sm[];
   float* qS = sm;                 // [C][LDK]  q, then q e^{Gamma - Gamma_15}
   float* kS = qS + C * LDK;       // [C][LDK]
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(NTH, 2)
   const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
   const int tid = threadIdx.x;
 
-  load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  load_keys<Tin, DK, LDK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
   bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
   for (int i = tid; i < DK; i += NTH) {
     const float g15 = GS[MREB * LDK + i];
@@ -875,11 +877,14 @@ constexpr int LDBB = VBB + 4;
 
 template <int DK>
 struct BSmem {
-  static constexpr int LDK = DK + 1;
+  // 8 (mod 32): after the dv-block loop, q, k and the k e^{Gamma_15 - Gamma}
+  // factor are [K][N] operands of the backward through the Gram matrices
+  static constexpr int LDK = DK + 8;
   // the dv-block loop's tiles (S and dS blocks; dO', R, U, dU, W blocks) are
   // dead once the loop ends; the dGamma accumulator and a C x C scratch tile
   // take their place (dq and dk accumulate in their outputs)
-  static constexpr int loop = 2 * DK * LDBB + 5 * C * LDBB;
+  static constexpr int loop = 2 * DK * LDBB + 5 * C * LDBB > 2 * C * LDK
+                                  ? 2 * DK * LDBB + 5 * C * LDBB : 2 * C * LDK;
   static constexpr int after = C * LDK + C * LDC;
   static_assert(after <= loop, "post-loop tiles fit the loop tiles");
   static_assert(2 * C * LDK <= loop, "dGamma and the k e^{Gamma_15 - Gamma} factor fit the loop tiles");
@@ -897,7 +902,7 @@ __global__ void __launch_bounds__(NTH, 2)
                     const Tin* __restrict__ dout, SeqMap map, int N, int DV, float scale,
                     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dg,
                     float* __restrict__ dbeta, float* __restrict__ ws) {
-  constexpr int LDK = DK + 1;
+  constexpr int LDK = BSmem<DK>::LDK;
   extern __shared__ float sm[];
   float* qS = sm;
   float* kS = qS + C * LDK;
@@ -911,7 +916,7 @@ __global__ void __launch_bounds__(NTH, 2)
   float* WS = dUS + C * LDBB;
   float* aG = SS;                 // after the loop: dGamma accumulator [C][LDK]
   float* YS = aG + C * LDK;       //                 scratch [C][LDC]
-  float* XS = WS + C * LDBB;      // [C][LDC]
+  float* XS = SS + BSmem<DK>::loop;  // [C][LDC]
   float* LS = XS + C * LDC;
   float* dAqS = LS + C * LDC;
   float* dTS = dAqS + C * LDC;    // dT, then dM
@@ -931,7 +936,7 @@ __global__ void __launch_bounds__(NTH, 2)
   const int tid = threadIdx.x;
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
-  load_keys<Tin, DK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  load_keys<Tin, DK, LDK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
   // the factorised backward through the Gram matrices scales sums of up to C
   // terms of size e^{|Gamma_r - Gamma_15|} |dL| by the opposite factor, so it
   // takes the chunk only while every |Gamma_r - Gamma_15| stays below 60
