@@ -241,20 +241,31 @@ template <typename Tin, int DK, int LDK>
 __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const float* beta,
                           size_t rowbase, int H, int n, float* qS, float* kS, float* GS,
                           float* bS) {
-  for (int idx = threadIdx.x; idx < C * DK; idx += NTH) {
-    const int r = idx / DK, i = idx % DK;
-    float qv = 0.f, kv = 0.f, gv = 0.f;
+  // every load of the thread in flight before its first store
+  constexpr int IT = C * DK / NTH;
+  static_assert(C * DK % NTH == 0 && C <= NTH, "whole passes");
+  float qv[IT], kv[IT], gv[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int idx = threadIdx.x + it * NTH, r = idx / DK, i = idx % DK;
+    qv[it] = kv[it] = gv[it] = 0.f;
     if (r < n) {
       const size_t off = (rowbase + (size_t)r * H) * DK + i;
-      qv = Elem<Tin>::load(q + off);
-      kv = Elem<Tin>::load(k + off);
-      gv = g[off];
+      qv[it] = Elem<Tin>::load(q + off);
+      kv[it] = Elem<Tin>::load(k + off);
+      gv[it] = g[off];
     }
-    qS[r * LDK + i] = qv;
-    kS[r * LDK + i] = kv;
-    GS[r * LDK + i] = gv;
   }
-  for (int r = threadIdx.x; r < C; r += NTH) bS[r] = r < n ? beta[rowbase + (size_t)r * H] : 0.f;
+  const int rb = threadIdx.x;
+  const float bv = rb < C && rb < n ? beta[rowbase + (size_t)rb * H] : 0.f;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int idx = threadIdx.x + it * NTH, r = idx / DK, i = idx % DK;
+    qS[r * LDK + i] = qv[it];
+    kS[r * LDK + i] = kv[it];
+    GS[r * LDK + i] = gv[it];
+  }
+  if (rb < C) bS[rb] = bv;
   __syncthreads();
   for (int i = threadIdx.x; i < DK; i += NTH) {  // Gamma = inclusive cumsum over the chunk
     float acc = 0.f;
@@ -499,22 +510,39 @@ __global__ void __launch_bounds__(NTF, 1)
     const int t0 = c * C, n = min(C, up.len - t0);
     const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
-    for (int idx = tid; idx < C * DK; idx += NTF) {
-      const int r = idx / DK, i = idx % DK;
-      float kv = 0.f, gv = 0.f;
-      if (r < n) {
-        const size_t off = (rowbase + (size_t)r * H) * DK + i;
-        kv = Elem<Tin>::load(k + off);
-        gv = g[off];
+    {  // the chunk's rows: every load of the thread in flight before its first store
+      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
+      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
+      float kv[IK], gv[IK], vv[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        kv[it] = gv[it] = 0.f;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          kv[it] = Elem<Tin>::load(k + off);
+          gv[it] = g[off];
+        }
       }
-      kS[r * LKC + i] = kv;
-      GS[r * LDK + i] = gv;
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        vv[it] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        kS[r * LKC + i] = kv[it];
+        GS[r * LDK + i] = gv[it];
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        VS[r * LDV + j] = vv[it];
+      }
+      if (tid < C) bS[tid] = bv;
     }
-    for (int idx = tid; idx < C * DV; idx += NTF) {
-      const int r = idx / DV, j = idx % DV;
-      VS[r * LDV + j] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
-    }
-    if (tid < C) bS[tid] = tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
     for (int idx = tid; idx < DK * DV; idx += NTF) {  // chunk-start state
       const int i = idx / DV, j = idx % DV;
       w.S[(size_t)c * DK * DV + idx] = SS[i * LDV + j];
@@ -701,25 +729,41 @@ __global__ void __launch_bounds__(NTF, 1)
     const int t0 = c * C, n = min(C, up.len - t0);
     const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
-    for (int idx = tid; idx < C * DK; idx += NTF) {
-      const int r = idx / DK, i = idx % DK;
-      float qv = 0.f, kv = 0.f, gv = 0.f;
-      if (r < n) {
-        const size_t off = (rowbase + (size_t)r * H) * DK + i;
-        qv = Elem<Tin>::load(q + off);
-        kv = Elem<Tin>::load(k + off);
-        gv = g[off];
+    {  // the chunk's rows: every load of the thread in flight before its first store
+      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
+      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
+      float qv[IK], kv[IK], gv[IK], ov[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        qv[it] = kv[it] = gv[it] = 0.f;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          qv[it] = Elem<Tin>::load(q + off);
+          kv[it] = Elem<Tin>::load(k + off);
+          gv[it] = g[off];
+        }
       }
-      qS[r * LQT + i] = qv;
-      kS[r * LDK + i] = kv;
-      GS[r * LQT + i] = gv;
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        ov[it] = r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        qS[r * LQT + i] = qv[it];
+        kS[r * LDK + i] = kv[it];
+        GS[r * LQT + i] = gv[it];
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        dOS[r * LDV + j] = ov[it];
+      }
+      if (tid < C) bS[tid] = bv;
     }
-    for (int idx = tid; idx < C * DV; idx += NTF) {
-      const int r = idx / DV, j = idx % DV;
-      dOS[r * LDV + j] =
-          r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j) : 0.f;
-    }
-    if (tid < C) bS[tid] = tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
     for (int idx = tid; idx < DK * DV; idx += NTF) {  // dL/dS_next of this chunk
       const int i = idx / DV, j = idx % DV;
       w.dS[(size_t)c * DK * DV + idx] = dSS[i * LDV + j];
