@@ -5,8 +5,9 @@ shortcut), plus properties checked over every output.
 
 Workloads: dense prefill B=8 H=32 T=4096; varlen 64 log-uniform sequences,
 H=16, nonzero initial states; decode 256 x 32 heads for 1024 steps; long
-prefill B=1 H=32 T=1048576 (segment split).  All dk = dv = 128, bf16
-q/k/v, fp32 g/beta/state.
+prefill B=1 H=32 T=1048576 (segment split); speculative verify / replay
+256 x 32 heads with 4 draft tokens.  All dk = dv = 128, bf16 q/k/v, fp32
+g/beta/state.
 """
 import numpy as np
 import pytest
@@ -204,3 +205,43 @@ def test_long_prefill_full_size(oracle_mod):
     for u, h in enumerate(heads):
         assert np.sqrt(num[u] / den[u]) <= TOL_BF16_O, (h, np.sqrt(num[u] / den[u]))
         assert rel_l2(to64(S[0, h]), state[u, 0]) <= TOL_BF16_S, h
+
+
+def test_spec_decode_full_size(oracle_mod):
+    """Speculative verify / replay at the benchmark's size (N256 H32 d128,
+    K = 4 draft tokens, bf16): verify leaves the committed state bit for bit;
+    replay with accepted lengths 0 ... K across the batch leaves the
+    zero-accept sequences untouched; sampled units' outputs and replayed
+    states against the oracle."""
+    N, H, d, K = 256, 32, 128, 4
+    inp = W.make_prefill_inputs(N, K, H, d, d, torch.bfloat16, seed=7, device=DEV)
+    S0 = W.make_decode_state(N, H, d, d, 8, DEV)
+    state = S0.clone()
+    out = torch.full((N, K, H, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    kda.kda_decode_verify(inp["q"], inp["k"], inp["v"], inp["z"], inp["beta"], state, out,
+                          A_log=inp["A_log"])
+    torch.cuda.synchronize()
+    assert torch.equal(state, S0)
+    assert torch.isfinite(out.float()).all()
+    acc = torch.arange(N, device=DEV, dtype=torch.int32) % (K + 1)
+    kda.kda_decode_replay(inp["k"], inp["v"], inp["z"], inp["beta"], state, acc,
+                          A_log=inp["A_log"])
+    torch.cuda.synchronize()
+    zero = (acc == 0).nonzero().flatten()
+    assert torch.equal(state[zero], S0[zero])
+    units = [(0, 0), (1, 7), (2, 31), (3, 12), (4, 20), (129, 5), (254, 30), (255, 31)]
+    A = to64(inp["A_log"])
+    for n, h in units:
+        sl = lambda t: to64(t[n:n + 1, :, h:h + 1])
+        g = oracle_mod.gate(sl(inp["z"]), A[h:h + 1], -5.0)
+        o_ref, _ = oracle_mod.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), g, sl(inp["beta"]),
+                                      init_state=to64(S0[n:n + 1, h:h + 1]))
+        assert rel_l2(to64(out[n, :, h]), o_ref[0, :, 0]) <= TOL_BF16_O, (n, h)
+        m = int(acc[n])
+        if m == 0:
+            continue
+        cut = lambda t: np.ascontiguousarray(t[:, :m])
+        _, S_ref = oracle_mod.forward(cut(sl(inp["q"])), cut(sl(inp["k"])), cut(sl(inp["v"])),
+                                      cut(g), cut(sl(inp["beta"])),
+                                      init_state=to64(S0[n:n + 1, h:h + 1]))
+        assert rel_l2(to64(state[n, h]), S_ref[0, 0]) <= TOL_BF16_S, (n, h)
