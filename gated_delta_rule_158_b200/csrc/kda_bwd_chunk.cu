@@ -918,6 +918,7 @@ __global__ void __launch_bounds__(NTF, 1)
 // rows of 20 floats keep the tensor-core fragment loads free of bank conflicts
 constexpr int VBB = 16;
 constexpr int LDBB = VBB + 4;
+static_assert(LDBB % 4 == 0, "16-byte aligned rows of the dv-block tiles");
 
 template <int DK>
 struct BSmem {
@@ -1033,12 +1034,9 @@ __global__ void __launch_bounds__(NTH, 2)
     for (int j0 = 0; j0 < DV; j0 += VBB) {
       __syncthreads();
       // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
-      auto put4 = [](float* dst, float4 x) {
-        dst[0] = x.x;
-        dst[1] = x.y;
-        dst[2] = x.z;
-        dst[3] = x.w;
-      };
+      // one 16-byte store (every tile of the block loop starts on a multiple
+      // of 4 floats, and rows are LDBB = 20 floats)
+      auto put4 = [](float* dst, float4 x) { *reinterpret_cast<float4*>(dst) = x; };
       for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
         const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
         const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
@@ -1119,12 +1117,9 @@ __global__ void __launch_bounds__(NTH, 2)
     for (int j0 = 0; j0 < DV; j0 += VBB) {
       __syncthreads();
       // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
-      auto put4 = [](float* dst, float4 x) {
-        dst[0] = x.x;
-        dst[1] = x.y;
-        dst[2] = x.z;
-        dst[3] = x.w;
-      };
+      // one 16-byte store (every tile of the block loop starts on a multiple
+      // of 4 floats, and rows are LDBB = 20 floats)
+      auto put4 = [](float* dst, float4 x) { *reinterpret_cast<float4*>(dst) = x; };
       for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
         const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
         const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
