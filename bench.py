@@ -53,11 +53,26 @@ WORKLOADS = {
                      seed=3, varlen=False),
     "spec_decode": dict(name="speculative verify/replay N256 H32 d128, K=4 draft tokens", N=256,
                         H=32, dk=128, dv=128, K=4, seed=7),
+    # fp32 inputs take the CUDA-core chunk kernel (the tensor-core one is bf16)
+    "prefill_fp32": dict(name="prefill fp32 B8 H32 T4096 d128", B=8, T=4096, H=32, dk=128,
+                         dv=128, seed=1, init=False, varlen=False, dtype="f32"),
 }
 
 # bytes per (token, head) of the chunkwise forward, bf16 q/k/v/o, fp32 g/beta:
 # q, k, v 3*256 + g 512 + beta 4 + o 256
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 4 + 256
+
+
+def prefill_bytes_per_token_head(wl):
+    """Algorithmic bytes per (token, head) at d = 128: q, k, v, o in the
+    input type (2 or 4 bytes), z fp32, beta fp32."""
+    if wl.get("dtype", "bf16") == "f32":
+        return 4 * 512 + 512 + 4
+    return PREFILL_BYTES_PER_TOKEN_HEAD
+
+
+def wl_torch_dtype(wl):
+    return torch.float32 if wl.get("dtype", "bf16") == "f32" else torch.bfloat16
 # FLOPs per (token, head) of the chunk form counted once:
 # C(3dk + 2dv) + C^2/3 + 6 dk dv.  The tensor-core kernel runs C = 32
 # (118,869 at d = 128); the reference count of the measurement plan is taken
@@ -108,8 +123,11 @@ def chunk_traffic(B, H, T):
 def kernels_per_step(wl, B, T):
     """libkda kernels one prefill step launches: one chunk kernel; the varlen
     plan kernel in front for varlen; three (transitions, combine, outputs)
-    when the long-sequence split applies (B*H*2 < SMs and T >= 4096)."""
+    when the long-sequence split applies (B*H*2 < SMs and T >= 4096); two
+    (key-side pass, scan) for fp32 inputs."""
     if wl.get("varlen"):
+        return 2
+    if wl.get("dtype", "bf16") == "f32":  # key-side pass, then the scan
         return 2
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     if 2 * B * wl["H"] < sms and T >= 4096:
@@ -231,7 +249,7 @@ def make_prefill(wl, device):
                                     num_states=wl["num_seqs"])
         cu = torch.tensor(cu_list, dtype=torch.int32, device=device)
         return inp, cu, T, wl["num_seqs"]
-    inp = W.make_prefill_inputs(wl["B"], wl["T"], wl["H"], wl["dk"], wl["dv"], torch.bfloat16,
+    inp = W.make_prefill_inputs(wl["B"], wl["T"], wl["H"], wl["dk"], wl["dv"], wl_torch_dtype(wl),
                                 seed=wl["seed"], device=device, init_state=wl["init"])
     return inp, None, wl["T"], wl["B"]
 
@@ -247,8 +265,9 @@ class PrefillStep:
         dv = inp["v"].shape[-1]
         self.out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
         self.final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-        nbytes = kda.kda_chunk_fwd_workspace_size(B, T, H, dk, dv,
-                                                  0 if cu is None else N, 0, kda.KDA_BF16)
+        nbytes = kda.kda_chunk_fwd_workspace_size(
+            B, T, H, dk, dv, 0 if cu is None else N, 0,
+            kda.KDA_BF16 if q.dtype == torch.bfloat16 else kda.KDA_F32)
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device)
 
     def __call__(self, ev=None):
@@ -784,7 +803,7 @@ def measure_prefill(wl, dev, steps, warmup, world, with_clocks):
     ms_per_step = total_ms / steps
     tokens = B * T  # per rank
     tok_heads = tokens * H
-    alg_bytes = tok_heads * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * dk * dv * 4 * (
+    alg_bytes = tok_heads * prefill_bytes_per_token_head(wl) + N * H * dk * dv * 4 * (
         2 if inp["init_state"] is not None else 1)
     achieved = alg_bytes / (chunk_ms * 1e-3) / 1e9
     return dict(inp=inp, cu=cu, T=T, N=N, B=B, H=H, dk=dk, dv=dv, step=step, clk=clk,
@@ -800,8 +819,11 @@ def prefill_roofline(m, peaks, wl):
     secs = m["chunk_ms"] * 1e-3
     return {"bound": "hbm", "achieved": round(m["achieved"], 1), "peak": peaks["hbm"],
             "unit": "GB/s", "frac": round(m["achieved"] / peaks["hbm"], 4),
-            "traffic": chunk_traffic(m["B"], m["H"], m["T"]) if not wl.get("varlen") else None,
-            "kernel": "chunk_tc_kernel (kda_chunk_fwd_gated)",
+            "traffic": (chunk_traffic(m["B"], m["H"], m["T"])
+                        if not wl.get("varlen") and wl.get("dtype", "bf16") == "bf16" else None),
+            "kernel": ("chunk_tc_kernel (kda_chunk_fwd_gated)" if wl.get("dtype", "bf16") == "bf16"
+                       else "bwd_keyside (key-side matrices of every chunk) + fwd_f32_scan "
+                            "(kda_chunk_fwd_gated, fp32 inputs)"),
             "kernel_ms": round(m["chunk_ms"], 4), "algorithmic_bytes": m["alg_bytes"],
             "peak_source": peaks["src"],
             "tensor_frac": round(f32 / secs / (peaks["tc"] * 1e12), 4),
@@ -841,8 +863,8 @@ def bench_prefill_line(args, wl, world, rank, peaks):
     line = {
         "metric": METRIC, "value": round(m["value"], 3), "unit": "Mtokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(m["ms_per_step"], 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.get("dtype", "bf16"), "data": "synthetic",
         "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": T,
                    "heads": H, "dk": dk, "dv": dv, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (no flush needed)",
@@ -853,7 +875,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
         "input_sensitivity": "checked: one value of v changed changes the output; restored gives "
                              "it back bit for bit" if sensitivity else None,
     }
-    if not args.no_e2e:
+    if not args.no_e2e and wl.get("dtype", "bf16") == "bf16":  # the host-buffer entry is bf16
         e2e_ms, h2d, d2h = e2e_prefill(wl, inp, cu, N, max(2, min(args.steps, 5)))
         line["e2e"] = {"value": round(tokens * world / (e2e_ms * 1e-3) / 1e6, 3),
                        "unit": "Mtokens/s", "h2d_bytes_per_step": h2d,

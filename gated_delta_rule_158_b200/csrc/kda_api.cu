@@ -91,6 +91,11 @@ bool use_tc_path(kda_dtype dt, int dk, int dv, int chunk) {
   return dt == KDA_BF16 && dk == 128 && dv == 128 && (chunk == 0 || chunk == 32);
 }
 
+// Everything else with the default chunk takes the fp32-accurate chunk form
+// on warp-level tensor-core products; an explicit chunk of 16 or 64 takes
+// the CUDA-core kernel (the only one built for those chunk sizes).
+bool use_f32_path(int chunk) { return chunk == 0 || chunk == 32; }
+
 }  // namespace
 
 cudaError_t launch_varlen_plan(const int32_t* cu_seqlens, int num_seqs, int T, int32_t* order,
@@ -184,8 +189,12 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
                                     int chunk_size, kda_dtype in_dtype) {
   size_t bytes = kStatusBytes;
   if (num_seqs > 0) bytes += round_up(sizeof(int32_t) * (size_t)num_seqs, 256);
-  if (use_tc_path(in_dtype, dk, dv, chunk_size) && B > 0 && T > 0 && H > 0)
-    bytes += tc_workspace_bytes(B, T, H, num_seqs, device_sm_count());
+  if (B > 0 && T > 0 && H > 0) {
+    if (use_tc_path(in_dtype, dk, dv, chunk_size))
+      bytes += tc_workspace_bytes(B, T, H, num_seqs, device_sm_count());
+    else if (use_f32_path(chunk_size))
+      bytes += chunk_f32_tail_bytes(B, T, H, num_seqs);
+  }
   return bytes;
 }
 
@@ -273,8 +282,10 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
     a.chunk = 32;
     const size_t tail_bytes = workspace_bytes - (size_t)(tail - static_cast<char*>(workspace));
     e = launch_chunk_tc(a, tail, tail_bytes, st);
+  } else if (use_f32_path(chunk_size)) {
+    a.chunk = 32;
+    e = launch_chunk_f32(a, tail, st);
   } else {
-    if (a.chunk == 0) a.chunk = 32;
     e = launch_chunk_simt(a, st);
   }
   return e == cudaSuccess ? KDA_OK : cuda_failure(e);

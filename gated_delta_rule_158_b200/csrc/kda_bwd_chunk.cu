@@ -220,6 +220,17 @@ __device__ inline bool chunk_of_block(const SeqMap& m, int N, int& h, int& c, Un
   return true;
 }
 
+// The fp32 forward's workspace holds only the key-side matrices of each
+// chunk: X, A_qk and L, C x C each, in the same order per unit.
+constexpr int kFwdChunkFloats = 3 * C * C;
+__device__ inline UnitWs unit_ws_fwd(float* ws, int64_t chunk0, int nc) {
+  UnitWs w{};
+  w.X = ws + (size_t)chunk0 * kFwdChunkFloats;
+  w.Aqk = w.X + (size_t)nc * C * C;
+  w.L = w.Aqk + (size_t)nc * C * C;
+  return w;
+}
+
 __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int DV) {
   UnitWs w;
   float* base = ws + (size_t)chunk0 * unit_ws_floats(1, DK, DV);
@@ -237,10 +248,13 @@ __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int 
 
 // chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to
 // C, into [C][LDK] tiles
+// g is the log-decay, or z when A_log is not null (the gate
+// g = g_min sigmoid(e^{A_log[h]} z) formed on load).
 template <typename Tin, int DK, int LDK>
-__device__ void load_keys(const Tin* q, const Tin* k, const float* g, const float* beta,
-                          size_t rowbase, int H, int n, float* qS, float* kS, float* GS,
-                          float* bS) {
+__device__ void load_keys(const Tin* q, const Tin* k, const float* g, const float* A_log,
+                          float g_min, int h, const float* beta, size_t rowbase, int H, int n,
+                          float* qS, float* kS, float* GS, float* bS) {
+  const float a_h = A_log ? expf(A_log[h]) : 0.f;
   // every load of the thread in flight before its first store
   constexpr int IT = C * DK / NTH;
   static_assert(C * DK % NTH == 0 && C <= NTH, "whole passes");
@@ -253,7 +267,7 @@ __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const floa
       const size_t off = (rowbase + (size_t)r * H) * DK + i;
       qv[it] = Elem<Tin>::load(q + off);
       kv[it] = Elem<Tin>::load(k + off);
-      gv[it] = g[off];
+      gv[it] = A_log ? gate_value(g[off], a_h, g_min) : g[off];
     }
   }
   const int rb = threadIdx.x;
@@ -344,11 +358,13 @@ struct KSmem {
   static constexpr size_t bytes = sizeof(float) * floats;
 };
 
-template <typename Tin, int DK, int DV>
+// FWD: the fp32 forward's compact workspace (unit_ws_fwd) instead of the
+// backward's; A_log (nullable): g holds z and the gate is formed on load.
+template <typename Tin, int DK, int DV, bool FWD = false>
 __global__ void __launch_bounds__(NTH, 2)
     bwd_keyside(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                const float* __restrict__ g, const float* __restrict__ beta, SeqMap map, int N,
-                float* __restrict__ ws) {
+                const float* __restrict__ g, const float* __restrict__ A_log, float g_min,
+                const float* __restrict__ beta, SeqMap map, int N, float* __restrict__ ws) {
   constexpr int LDK = KSmem<DK>::LDK;
   extern __shared__ float sm[];
   float* qS = sm;                 // [C][LDK]  q, then q e^{Gamma - Gamma_15}
@@ -368,10 +384,11 @@ __global__ void __launch_bounds__(NTH, 2)
   if (!chunk_of_block(map, N, h, c, up) || !unit_in_bounds(map, up)) return;
   const int t0 = c * C, n = min(C, up.len - t0);
   const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
-  const UnitWs w = unit_ws(ws, up.chunk0, up.nc, DK, DV);
+  const UnitWs w = FWD ? unit_ws_fwd(ws, up.chunk0, up.nc)
+                       : unit_ws(ws, up.chunk0, up.nc, DK, DV);
   const int tid = threadIdx.x;
 
-  load_keys<Tin, DK, LDK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  load_keys<Tin, DK, LDK>(q, k, g, A_log, g_min, h, beta, rowbase, H, n, qS, kS, GS, bS);
   bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
   for (int i = tid; i < DK; i += NTH) {
     const float g15 = GS[MREB * LDK + i];
@@ -981,7 +998,7 @@ __global__ void __launch_bounds__(NTH, 2)
   const int tid = threadIdx.x;
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
-  load_keys<Tin, DK, LDK>(q, k, g, beta, rowbase, H, n, qS, kS, GS, bS);
+  load_keys<Tin, DK, LDK>(q, k, g, nullptr, 0.f, h, beta, rowbase, H, n, qS, kS, GS, bS);
   // the factorised backward through the Gram matrices scales sums of up to C
   // terms of size e^{|Gamma_r - Gamma_15|} |dL| by the opposite factor, so it
   // takes the chunk only while every |Gamma_r - Gamma_15| stays below 60
@@ -1386,7 +1403,8 @@ struct Passes {
   static cudaError_t K(const BwdArgs& a, const SeqMap& m, int nseq, int64_t blocks, float* ws,
                        cudaStream_t st) {
     bwd_keyside<Tin, DK, DV><<<(unsigned)blocks, NTH, KSmem<DK>::bytes, st>>>(
-        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta, m, nseq, ws);
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, nullptr, 0.f, a.beta, m,
+        nseq, ws);
     return cudaGetLastError();
   }
   // F: chunk-start states, R and U, one CTA per unit; fin (nullable) gets the end state
@@ -1482,6 +1500,322 @@ cudaError_t launch_dk(const BwdArgs& a, cudaStream_t st) {
   }
 }
 
+// ============================================================ fp32 forward
+// The chunkwise forward at fp32 accuracy, for the inputs the tensor-core
+// kernel does not take (fp32, dk or dv other than 128): the key-side pass K
+// above (every chunk's X, A_qk, L at once, into the compact unit_ws_fwd
+// layout), then a scan with the state products of F and the outputs
+//   O = Q_gamma S + A_qk U,   U = T (V - Ka S),   S <- Diag(e^{Gamma_C}) S + Kc^T U,
+// O formed from the chunk-start S before its update.  One CTA of 512 threads
+// per (sequence, head), all dv columns; the tile strides are those of F.
+template <int DK, int DV>
+struct OSmem {
+  static constexpr int LDK = FSmem<DK, DV>::LDK, LKC = FSmem<DK, DV>::LKC;
+  static constexpr int LDV = FSmem<DK, DV>::LDV, LDT = FSmem<DK, DV>::LDT;
+  static constexpr int floats = FSmem<DK, DV>::floats
+                                + C * LDK       // q, then Q_gamma (row-major A operand)
+                                + C * LDT;      // A_qk (row-major A operand)
+  static constexpr size_t bytes = sizeof(float) * floats;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(NTF, 1)
+    fwd_f32_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                 const Tin* __restrict__ v, const float* __restrict__ g,
+                 const float* __restrict__ A_log, float g_min, const float* __restrict__ beta,
+                 const float* __restrict__ init, float* __restrict__ fin,
+                 Tin* __restrict__ out, float scale, SeqMap map, float* __restrict__ ws) {
+  constexpr int LDK = OSmem<DK, DV>::LDK, LKC = OSmem<DK, DV>::LKC;
+  constexpr int LDV = OSmem<DK, DV>::LDV, LDT = OSmem<DK, DV>::LDT;
+  extern __shared__ float sm[];
+  float* kS = sm;                 // [C][LKC]  k, then Kc
+  float* GS = kS + C * LKC;       // [C][LDK]  Gamma
+  float* KaS = GS + C * LDK;      // [C][LDK]  Ka
+  float* SS = KaS + C * LDK;      // [DK][LDV] state
+  float* VS = SS + DK * LDV;      // [C][LDV]  V, then R = V - Ka S
+  float* US = VS + C * LDV;       // [C][LDV]
+  float* TS = US + C * LDV;       // [C][LDT]
+  float* bS = TS + C * LDT;       // [C]
+  float* gC = bS + C;             // [DK] Gamma_C
+  float* eC = gC + DK;            // [DK] e^{Gamma_C}
+  float* qS = eC + DK;            // [C][LDK]  q, then Q_gamma
+  float* AqS = qS + C * LDK;      // [C][LDT]
+
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  const int unit = blockIdx.x;
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
+  const int nc = up.nc;
+  const UnitWs w = unit_ws_fwd(ws, up.chunk0, nc);
+  const int tid = threadIdx.x;
+  const float a_h = A_log ? expf(A_log[h]) : 0.f;
+
+  for (int idx = tid; idx < DK * DV; idx += NTF) {
+    const int i = idx / DV, j = idx % DV;
+    SS[i * LDV + j] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
+  }
+  for (int c = 0; c < nc; ++c) {
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+    __syncthreads();
+    {  // the chunk's rows: every load of the thread in flight before its first store
+      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
+      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
+      float qv[IK], kv[IK], gv[IK], vv[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        qv[it] = kv[it] = gv[it] = 0.f;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          qv[it] = Elem<Tin>::load(q + off);
+          kv[it] = Elem<Tin>::load(k + off);
+          gv[it] = A_log ? gate_value(g[off], a_h, g_min) : g[off];
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        vv[it] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
+        qS[r * LDK + i] = qv[it];
+        kS[r * LKC + i] = kv[it];
+        GS[r * LDK + i] = gv[it];
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
+        VS[r * LDV + j] = vv[it];
+      }
+      if (tid < C) bS[tid] = bv;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LDK + i];
+        GS[r * LDK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+    }
+    for (int idx = tid; idx < C * C; idx += NTF) {  // T = X Diag(beta); A_qk
+      const int r = idx / C, s2 = idx % C;
+      TS[r * LDT + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
+      AqS[r * LDT + s2] = w.Aqk[((size_t)c * C + r) * C + s2];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka, Kc (into kS), Q_gamma (into qS)
+      const int r = idx / DK, i = idx % DK;
+      const float G = GS[r * LDK + i], e = expf(G), kv = kS[r * LKC + i];
+      KaS[r * LDK + i] = kv * e;
+      kS[r * LKC + i] = kv * expf(gC[i] - G);
+      qS[r * LDK + i] *= e;
+    }
+    __syncthreads();
+    if constexpr (DK == 128 && DV == 128) {
+      // tensor cores: warp w owns C x DV tiles (w >> 3, 2 (w & 7) + {0, 1}) and
+      // DK x DV tiles (w >> 1, 8 (w & 1) + 0..7)
+      const int wp = tid >> 5, mt = wp >> 3, nt0 = 2 * (wp & 7);
+      const int mt8 = wp >> 1, nt8 = 8 * (wp & 1);
+      {  // R = V - Ka S
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < DK; k0 += 8) {
+          Frag3 a;
+          load_a(a, KaS, LDK, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, SS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            VS[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] -= acc[q2][e];
+      }
+      __syncthreads();
+      {  // U = T R
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a(a, TS, LDT, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, VS, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            US[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] = acc[q2][e];
+      }
+      __syncthreads();
+      {  // O = Q_gamma S + A_qk U, from the chunk-start S
+        float acc[2][4];
+        zero(acc);
+        for (int k0 = 0; k0 < DK; k0 += 8) {
+          Frag3 a;
+          load_a(a, qS, LDK, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, SS, LDV, 8 * (nt0 + q2), k0);
+        }
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a(a, AqS, LDT, 16 * mt, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) mma3<true>(acc[q2], a, US, LDV, 8 * (nt0 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = frag_row(16 * mt, e), j = frag_col(8 * (nt0 + q2), e);
+            if (r < n) Elem<Tin>::store(out + (rowbase + (size_t)r * H) * DV + j, scale * acc[q2][e]);
+          }
+      }
+      __syncthreads();  // S is read by the O product above and rewritten below
+      {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
+        float acc[8][4];
+        zero(acc);
+        for (int k0 = 0; k0 < C; k0 += 8) {
+          Frag3 a;
+          load_a<true>(a, kS, LKC, 16 * mt8, k0);
+#pragma unroll
+          for (int q2 = 0; q2 < 8; ++q2) mma3<true>(acc[q2], a, US, LDV, 8 * (nt8 + q2), k0);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 8; ++q2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = frag_row(16 * mt8, e), j = frag_col(8 * (nt8 + q2), e);
+            SS[i * LDV + j] = fmaf(eC[i], SS[i * LDV + j], acc[q2][e]);
+          }
+      }
+    } else {
+      {  // R = V - Ka S
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return KaS[m * LDK + kk]; },
+                                  [&](int kk, int nn) { return SS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { VS[m * LDV + nn] -= acc[i][j]; });
+      }
+      __syncthreads();
+      {  // U = T R
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return TS[m * LDT + kk]; },
+                                 [&](int kk, int nn) { return VS[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
+      }
+      __syncthreads();
+      {  // O = Q_gamma S + A_qk U, from the chunk-start S
+        float acc[1][DV / 16];
+        zero(acc);
+        mm<C, DV, 1, DV / 16, DK>(acc, [&](int m, int kk) { return qS[m * LDK + kk]; },
+                                  [&](int kk, int nn) { return SS[kk * LDV + nn]; });
+        mm<C, DV, 1, DV / 16, C>(acc, [&](int m, int kk) { return AqS[m * LDT + kk]; },
+                                 [&](int kk, int nn) { return US[kk * LDV + nn]; });
+        for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) {
+          if (m < n) Elem<Tin>::store(out + (rowbase + (size_t)m * H) * DV + nn, scale * acc[i][j]);
+        });
+      }
+      __syncthreads();  // S is read by the O product above and rewritten below
+      {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
+        float acc[DK / 32][DV / 16];
+        zero(acc);
+        mm<DK, DV, DK / 32, DV / 16, C>(acc, [&](int m, int kk) { return kS[kk * LKC + m]; },
+                                        [&](int kk, int nn) { return US[kk * LDV + nn]; });
+        for_tile<DK, DV, DK / 32, DV / 16>([&](int m, int nn, int i, int j) {
+          SS[m * LDV + nn] = fmaf(eC[m], SS[m * LDV + nn], acc[i][j]);
+        });
+      }
+    }
+  }
+  if (fin) {  // the state after the last chunk
+    __syncthreads();
+    for (int idx = tid; idx < DK * DV; idx += NTF) {
+      const int i = idx / DV, j = idx % DV;
+      fin[(size_t)unit * DK * DV + idx] = SS[i * LDV + j];
+    }
+  }
+}
+
+// Tail of the fp32 forward's workspace (after the status word and the
+// varlen order): the packed batch's chunk offsets, then X, A_qk, L per chunk.
+struct FwdLayout {
+  size_t coff_off, data_off, total;
+  int64_t max_chunks;  // per head
+};
+
+FwdLayout fwd_layout(int B, int T, int H, int num_seqs) {
+  FwdLayout L;
+  const int64_t nc = ((int64_t)T + C - 1) / C;
+  L.max_chunks = num_seqs > 0 ? nc + num_seqs : (int64_t)B * nc;
+  L.coff_off = 0;
+  L.data_off = num_seqs > 0 ? (sizeof(int32_t) * ((size_t)num_seqs + 1) + 255) / 256 * 256 : 0;
+  L.total = L.data_off + (size_t)H * L.max_chunks * kFwdChunkFloats * sizeof(float);
+  return L;
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t fwd_f32_launch(const ChunkArgs& a, void* tail, cudaStream_t st) {
+  const int nseq = a.map.cu_seqlens ? a.num_units / a.map.H : a.map.B;
+  const FwdLayout lay = fwd_layout(a.map.B, a.map.T, a.map.H, a.map.cu_seqlens ? nseq : 0);
+  char* base = static_cast<char*>(tail);
+  int32_t* coff = reinterpret_cast<int32_t*>(base + lay.coff_off);
+  float* ws = reinterpret_cast<float*>(base + lay.data_off);
+  cudaError_t e = cudaFuncSetAttribute(bwd_keyside<Tin, DK, DV, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)KSmem<DK>::bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fwd_f32_scan<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)OSmem<DK, DV>::bytes);
+  if (e != cudaSuccess) return e;
+  const SeqMap map{a.map.cu_seqlens, a.map.cu_seqlens ? coff : nullptr, a.sb, a.map.T, a.map.H,
+                   0, 0, (int64_t)a.map.B * a.map.T, lay.max_chunks * (int64_t)a.map.H};
+  if (a.map.cu_seqlens) {
+    bwd_varlen_plan<<<1, kPlanThreads, 0, st>>>(a.map.cu_seqlens, nseq, a.map.T, coff, a.sb);
+    if ((e = cudaGetLastError())) return e;
+  }
+  const float* A_log = a.gated ? a.A_log : nullptr;
+  bwd_keyside<Tin, DK, DV, true><<<(unsigned)(lay.max_chunks * a.map.H), NTH, KSmem<DK>::bytes,
+                                   st>>>(static_cast<const Tin*>(a.q),
+                                         static_cast<const Tin*>(a.k), a.g, A_log, a.g_min,
+                                         a.beta, map, nseq, ws);
+  if ((e = cudaGetLastError())) return e;
+  fwd_f32_scan<Tin, DK, DV><<<(unsigned)a.num_units, NTF, OSmem<DK, DV>::bytes, st>>>(
+      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+      a.g, A_log, a.g_min, a.beta, a.init_state, a.final_state, static_cast<Tin*>(a.out),
+      a.scale, map, ws);
+  return cudaGetLastError();
+}
+
+template <typename Tin, int DK>
+cudaError_t fwd_f32_dv(const ChunkArgs& a, void* tail, cudaStream_t st) {
+  switch (a.dv) {
+    case 32: return fwd_f32_launch<Tin, DK, 32>(a, tail, st);
+    case 64: return fwd_f32_launch<Tin, DK, 64>(a, tail, st);
+    case 128: return fwd_f32_launch<Tin, DK, 128>(a, tail, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename Tin>
+cudaError_t fwd_f32_dk(const ChunkArgs& a, void* tail, cudaStream_t st) {
+  switch (a.dk) {
+    case 32: return fwd_f32_dv<Tin, 32>(a, tail, st);
+    case 64: return fwd_f32_dv<Tin, 64>(a, tail, st);
+    case 128: return fwd_f32_dv<Tin, 128>(a, tail, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <typename Tin>
 cudaError_t by_dk(const BwdArgs& a, cudaStream_t st) {
   switch (a.dk_dim) {
@@ -1496,6 +1830,16 @@ cudaError_t by_dk(const BwdArgs& a, cudaStream_t st) {
 
 size_t bwd_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int num_seqs) {
   return ws_layout(B, T, H, dk, dv, num_seqs).total;
+}
+
+size_t chunk_f32_tail_bytes(int B, int T, int H, int num_seqs) {
+  return fwd_layout(B, T, H, num_seqs).total;
+}
+
+cudaError_t launch_chunk_f32(const ChunkArgs& a, void* tail, cudaStream_t stream) {
+  if (a.num_units == 0) return cudaSuccess;
+  return a.dt == KDA_BF16 ? fwd_f32_dk<__nv_bfloat16>(a, tail, stream)
+                          : fwd_f32_dk<float>(a, tail, stream);
 }
 
 cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t stream) {

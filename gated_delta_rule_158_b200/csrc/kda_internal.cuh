@@ -143,6 +143,14 @@ struct ChunkArgs {
 
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t stream);
 
+// fp32-accurate chunkwise forward on warp-level tensor-core products with
+// split tf32 operands (fp32 inputs, or dk / dv other than 128; chunk 32):
+// the workspace tail it needs after the status word and the varlen order,
+// and its launcher (two kernels: every chunk's key-side matrices, then the
+// state scan with the outputs).
+size_t chunk_f32_tail_bytes(int B, int T, int H, int num_seqs);
+cudaError_t launch_chunk_f32(const ChunkArgs& a, void* ws_tail, cudaStream_t stream);
+
 // tcgen05 tensor-core path (bf16, dk = dv = 128, chunk 32).
 size_t tc_workspace_bytes(int B, int T, int H, int num_seqs, int num_sms);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, void* ws_tail,

@@ -87,7 +87,9 @@ KDA_API kda_status kda_gate_fwd(const float *z, const float *A_log, float g_min,
 /*
  * Bytes of workspace kda_chunk_fwd needs for these arguments (always > 0:
  * it holds at least the device status word).  num_seqs is the number of
- * varlen sequences, or 0 for a dense batch.
+ * varlen sequences, or 0 for a dense batch.  The tensor-core path adds the
+ * segment states of its long-sequence split; the fp32-accuracy path adds
+ * three 32 x 32 matrices per (sequence, head) and 32-token chunk (12 KB).
  */
 KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
                                     int num_seqs, int chunk_size,
@@ -136,8 +138,12 @@ KDA_API kda_status kda_gate_bwd(const float *z, const float *A_log, float g_min,
  *  scale        : finite factor on o (1.0 for o = S^T q).
  *  chunk_size   : 0 = library choice, or 16, 32, 64.  The result does not
  *                 depend on it beyond rounding.  bf16 with dk = dv = 128 and
- *                 chunk 0 or 32 runs the tcgen05 tensor-core kernel; every
- *                 other supported combination runs an fp32 CUDA-core kernel.
+ *                 chunk 0 or 32 runs the tcgen05 tensor-core kernel; other
+ *                 inputs with chunk 0 or 32 (fp32, or dk / dv below 128) run
+ *                 the chunk form at fp32 accuracy on warp-level tensor-core
+ *                 products with split tf32 operands (two kernels: the
+ *                 key-side matrices of every chunk, then the state scan with
+ *                 the outputs); chunk 16 or 64 runs an fp32 CUDA-core kernel.
  *  out          : in_dtype [B, T, H, dv]; must not alias any input.
  *  final_state  : fp32 [N, H, dk, dv] or NULL.
  *  workspace    : device buffer of >= kda_chunk_fwd_workspace_size() bytes;

@@ -139,6 +139,29 @@ def test_chunk_size_invariance():
         assert rel_l2(to64(S), to64(res[0][1])) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype,dk,dv", [(torch.float32, 128, 128), (torch.float32, 64, 32),
+                                         (torch.bfloat16, 64, 64)])
+def test_prefill_f32_path_packed_gated(oracle_mod, dtype, dk, dv):
+    """The fp32-accurate chunk path (key-side pass, then the scan with the
+    outputs) on a packed batch with empty, one-token, ragged and whole-chunk
+    sequences, the gate fused into both of its kernels, initial states and
+    scale, against the oracle: the fp32 state at the fp32 bar for both input
+    types (bf16 inputs are widened exactly and every product keeps fp32
+    accuracy), o at the bar of its type (bf16 o is rounded on store); an
+    empty sequence keeps its initial state."""
+    lengths = [0, 1, 31, 32, 33, 100, 5, 64]
+    cu_list = W.cu_seqlens_from_lengths(lengths)
+    N, H = len(lengths), 3
+    inp = W.make_prefill_inputs(1, cu_list[-1], H, dk, dv, dtype, seed=150, device=DEV,
+                                init_state=True, num_states=N)
+    cu = torch.tensor(cu_list, dtype=torch.int32, device=DEV)
+    o, S = _gated_prefill(inp, cu=cu, scale=0.6)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, cu=cu, scale=0.6)
+    assert rel_l2(to64(o), o_ref) <= (TOL_F32 if dtype == torch.float32 else TOL_BF16_O)
+    assert rel_l2(to64(S), S_ref) <= TOL_F32
+    assert torch.equal(S[0], inp["init_state"][0])
+
+
 def test_state_handoff_equals_full_run():
     """Running T1 then T2 with final_state -> init_state equals one run over T."""
     inp = W.make_prefill_inputs(1, 160, 2, 128, 128, torch.bfloat16, seed=9, device=DEV,
