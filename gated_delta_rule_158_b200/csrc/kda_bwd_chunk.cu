@@ -999,13 +999,17 @@ __global__ void __launch_bounds__(NTH, 2)
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
   load_keys<Tin, DK, LDK>(q, k, g, nullptr, 0.f, h, beta, rowbase, H, n, qS, kS, GS, bS);
-  // the factorised backward through the Gram matrices scales sums of up to C
-  // terms of size e^{|Gamma_r - Gamma_15|} |dL| by the opposite factor, so it
-  // takes the chunk only while every |Gamma_r - Gamma_15| stays below 60
+  // The factorised backward through the Gram matrices works on 16-row
+  // blocks with a reference row per block pair: rows 7 and 23 inside the
+  // diagonal blocks, row 15 between them (where both factors are <= 1).  It
+  // scales sums of up to 16 terms of size e^{|Gamma_r - Gamma_ref|} |dL| by
+  // the opposite factor, so it takes the chunk only while every
+  // |Gamma_r - Gamma_ref| inside a diagonal block stays below 60 (at most 8
+  // steps of the gate's g >= -5, i.e. 40, for every gated input).
   bool wide = false;
   for (int i = tid; i < DK; i += NTH) {
-    const float g15 = GS[MREB * LDK + i];
-    for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - g15) > 60.f;
+    const float g7 = GS[7 * LDK + i], g23 = GS[23 * LDK + i];
+    for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - (r < 16 ? g7 : g23)) > 60.f;
   }
   wide = __syncthreads_or(wide);
   for (int idx = tid; idx < C * C; idx += NTH) {
@@ -1244,15 +1248,18 @@ __global__ void __launch_bounds__(NTH, 2)
   // q a_q); column side: c_k = sum_{r>=s} (dL_rs k_ri + dA_qk,rs q_ri) E_rsi
   // (dk += c_k, dGamma -= k c_k).
   if (!wide) {
-    // E_rsi = a_ri b_si with a = e^{Gamma - Gamma_15}, b = 1 / a, so with
-    // Ka' = k a, Qa' = q a, Kb' = k b:  a_k = a (dL Kb'), a_q = a (dA_qk Kb'),
-    // c_k = b (dL^T Ka' + dA_qk^T Qa'), three C x DK products on the tensor
-    // cores; warp w owns rows 16 (w >> 2) and DK / 32 column tiles of all three,
-    // so each element has one writer.
-    float* KbS = aG + C * LDK;  // the scratch tile is dead: k e^{Gamma_15 - Gamma}
+    // E_rsi = e^{Gamma_ri - Gamma_si} = a_ri b_si with a = e^{Gamma - Gamma_ref},
+    // b = 1 / a for the block pair (R, S) of rows r in R, s in S (S <= R), so
+    // with Ka' = k a, Qa' = q a, Kb' = k b over the blocks' rows:
+    //   a_k = a (dL Kb'), a_q = a (dA_qk Kb'), c_k = b (dL^T Ka' + dA_qk^T Qa'),
+    // C x DK products on the tensor cores over the 16 rows of the other block.
+    // Phase 0 takes the diagonal pairs (ref 7, 23), phase 1 the pair (1, 0)
+    // (ref 15).  Warp w owns rows 16 (w >> 2) and DK / 32 column tiles, so
+    // each element has one writer per phase.
+    float* KbS = aG + C * LDK;  // the scratch tile is dead: k e^{Gamma_ref - Gamma}
     for (int idx = tid; idx < C * DK; idx += NTH) {
       const int r = idx / DK, i = idx % DK;
-      const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+      const float d = GS[r * LDK + i] - GS[(r < 16 ? 7 : 23) * LDK + i];
       const float ea = expf(d), eb = expf(-d), kv = kS[r * LDK + i];
       KbS[r * LDK + i] = kv * eb;
       kS[r * LDK + i] = kv * ea;   // Ka'
@@ -1262,10 +1269,11 @@ __global__ void __launch_bounds__(NTH, 2)
     constexpr int NTW = DK / 32;  // column tiles per warp
     const int wp = tid >> 5, mt = wp >> 2, nt0 = NTW * (wp & 3);
     float p1[NTW][4], p2[NTW][4], p3[NTW][4];
+    // phase 0: within block mt (row side and column side over the same rows)
     zero(p1);
     zero(p2);
     zero(p3);
-    for (int k0 = 0; k0 < C; k0 += 8) {
+    for (int k0 = 16 * mt; k0 < 16 * mt + 16; k0 += 8) {
       Frag3 al, aa, alt, aat;
       load_a(al, dTS, LDC, 16 * mt, k0);
       load_a(aa, dAqS, LDC, 16 * mt, k0);
@@ -1285,7 +1293,7 @@ __global__ void __launch_bounds__(NTH, 2)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = frag_row(16 * mt, e), i = frag_col(8 * (nt0 + q2), e);
-        const float d = GS[r * LDK + i] - GS[MREB * LDK + i];
+        const float d = GS[r * LDK + i] - GS[(mt ? 23 : 7) * LDK + i];
         const float ea = expf(d), eb = expf(-d);
         if (r < n) {
           const size_t o = (rowbase + (size_t)r * H) * DK + i;
@@ -1295,6 +1303,66 @@ __global__ void __launch_bounds__(NTH, 2)
         // k a_k + q a_q - k c_k = Ka' P1 + Qa' P2 - Kb' P3
         aG[r * LDK + i] += fmaf(kS[r * LDK + i], p1[q2][e],
                                 fmaf(qS[r * LDK + i], p2[q2][e], -KbS[r * LDK + i] * p3[q2][e]));
+      }
+    __syncthreads();
+    // phase 1: the pair (1, 0) around row 15 -- Kb' of rows 0..15 from ref 7
+    // to 15, Ka' and Qa' of rows 16..31 from ref 23 to 15 (factors <= 1)
+    for (int idx = tid; idx < 16 * DK; idx += NTH) {
+      const int r = idx / DK, i = idx % DK;
+      const float g15 = GS[15 * LDK + i];
+      KbS[r * LDK + i] *= expf(g15 - GS[7 * LDK + i]);
+      const float fa = expf(GS[23 * LDK + i] - g15);
+      kS[(16 + r) * LDK + i] *= fa;
+      qS[(16 + r) * LDK + i] *= fa;
+    }
+    __syncthreads();
+    zero(p1);
+    zero(p2);
+    zero(p3);
+    // warps of block 1: row side over s in 0..15; warps of block 0: column
+    // side over r in 16..31
+    for (int k0 = 16 * (1 - mt); k0 < 16 * (1 - mt) + 16; k0 += 8) {
+      if (mt == 1) {
+        Frag3 al, aa;
+        load_a(al, dTS, LDC, 16, k0);
+        load_a(aa, dAqS, LDC, 16, k0);
+#pragma unroll
+        for (int q2 = 0; q2 < NTW; ++q2) {
+          const int col0 = 8 * (nt0 + q2);
+          mma3<true>(p1[q2], al, KbS, LDK, col0, k0);
+          mma3<true>(p2[q2], aa, KbS, LDK, col0, k0);
+        }
+      } else {
+        Frag3 alt, aat;
+        load_a<true>(alt, dTS, LDC, 0, k0);
+        load_a<true>(aat, dAqS, LDC, 0, k0);
+#pragma unroll
+        for (int q2 = 0; q2 < NTW; ++q2) {
+          const int col0 = 8 * (nt0 + q2);
+          mma3<true>(p3[q2], alt, kS, LDK, col0, k0);
+          mma3<true>(p3[q2], aat, qS, LDK, col0, k0);
+        }
+      }
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frag_row(16 * mt, e), i = frag_col(8 * (nt0 + q2), e);
+        const float d = GS[r * LDK + i] - GS[15 * LDK + i];
+        const size_t o = (rowbase + (size_t)r * H) * DK + i;
+        if (mt == 1) {  // rows 16..31: a = e^{Gamma_r - Gamma_15} <= 1
+          const float ea = expf(d);
+          if (r < n) {
+            dk[o] += ea * p1[q2][e];
+            dq[o] += ea * p2[q2][e];
+          }
+          aG[r * LDK + i] += fmaf(kS[r * LDK + i], p1[q2][e], qS[r * LDK + i] * p2[q2][e]);
+        } else {  // rows 0..15: b = e^{Gamma_15 - Gamma_r} <= 1
+          const float eb = expf(-d);
+          if (r < n) dk[o] += eb * p3[q2][e];
+          aG[r * LDK + i] -= KbS[r * LDK + i] * p3[q2][e];
+        }
       }
   } else {
     // exponentials of differences, by element owner: thread of channel i owns
