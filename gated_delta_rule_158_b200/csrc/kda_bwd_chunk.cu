@@ -1288,6 +1288,34 @@ __global__ void __launch_bounds__(NTH, 2)
         mma3<true>(p3[q2], aat, qS, LDK, col0, k0);
       }
     }
+    // dk, dq contributions into p1, p2; then the global read-modify-write with
+    // every old value loaded before the first store (the loads overlap)
+    auto add_out = [&](int m0, auto&& has_q) {
+      float od[NTW][4], oq[NTW][4];
+#pragma unroll
+      for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = frag_row(m0, e), i = frag_col(8 * (nt0 + q2), e);
+          od[q2][e] = oq[q2][e] = 0.f;
+          if (r < n) {
+            const size_t o = (rowbase + (size_t)r * H) * DK + i;
+            od[q2][e] = dk[o];
+            if (has_q()) oq[q2][e] = dq[o];
+          }
+        }
+#pragma unroll
+      for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = frag_row(m0, e), i = frag_col(8 * (nt0 + q2), e);
+          if (r < n) {
+            const size_t o = (rowbase + (size_t)r * H) * DK + i;
+            dk[o] = od[q2][e] + p1[q2][e];
+            if (has_q()) dq[o] = oq[q2][e] + p2[q2][e];
+          }
+        }
+    };
 #pragma unroll
     for (int q2 = 0; q2 < NTW; ++q2)
 #pragma unroll
@@ -1295,15 +1323,13 @@ __global__ void __launch_bounds__(NTH, 2)
         const int r = frag_row(16 * mt, e), i = frag_col(8 * (nt0 + q2), e);
         const float d = GS[r * LDK + i] - GS[(mt ? 23 : 7) * LDK + i];
         const float ea = expf(d), eb = expf(-d);
-        if (r < n) {
-          const size_t o = (rowbase + (size_t)r * H) * DK + i;
-          dk[o] += fmaf(ea, p1[q2][e], eb * p3[q2][e]);
-          dq[o] += ea * p2[q2][e];
-        }
         // k a_k + q a_q - k c_k = Ka' P1 + Qa' P2 - Kb' P3
         aG[r * LDK + i] += fmaf(kS[r * LDK + i], p1[q2][e],
                                 fmaf(qS[r * LDK + i], p2[q2][e], -KbS[r * LDK + i] * p3[q2][e]));
+        p1[q2][e] = fmaf(ea, p1[q2][e], eb * p3[q2][e]);  // dk
+        p2[q2][e] *= ea;                                   // dq
       }
+    add_out(16 * mt, [] { return true; });
     __syncthreads();
     // phase 1: the pair (1, 0) around row 15 -- Kb' of rows 0..15 from ref 7
     // to 15, Ka' and Qa' of rows 16..31 from ref 23 to 15 (factors <= 1)
@@ -1350,20 +1376,18 @@ __global__ void __launch_bounds__(NTH, 2)
       for (int e = 0; e < 4; ++e) {
         const int r = frag_row(16 * mt, e), i = frag_col(8 * (nt0 + q2), e);
         const float d = GS[r * LDK + i] - GS[15 * LDK + i];
-        const size_t o = (rowbase + (size_t)r * H) * DK + i;
         if (mt == 1) {  // rows 16..31: a = e^{Gamma_r - Gamma_15} <= 1
           const float ea = expf(d);
-          if (r < n) {
-            dk[o] += ea * p1[q2][e];
-            dq[o] += ea * p2[q2][e];
-          }
           aG[r * LDK + i] += fmaf(kS[r * LDK + i], p1[q2][e], qS[r * LDK + i] * p2[q2][e]);
+          p1[q2][e] *= ea;  // dk
+          p2[q2][e] *= ea;  // dq
         } else {  // rows 0..15: b = e^{Gamma_15 - Gamma_r} <= 1
           const float eb = expf(-d);
-          if (r < n) dk[o] += eb * p3[q2][e];
           aG[r * LDK + i] -= KbS[r * LDK + i] * p3[q2][e];
+          p1[q2][e] = eb * p3[q2][e];  // dk (no dq term)
         }
       }
+    add_out(16 * mt, [&] { return mt == 1; });
   } else {
     // exponentials of differences, by element owner: thread of channel i owns
     // rows r = part, part + P, ... (row side), then columns (column side)
