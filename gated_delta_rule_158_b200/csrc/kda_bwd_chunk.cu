@@ -527,6 +527,15 @@ __global__ void __launch_bounds__(NTF, 1)
     const int t0 = c * C, n = min(C, up.len - t0);
     const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
+    // this chunk's X from the key-side pass, loaded with the rows
+    constexpr int IX = C * C / NTF;
+    static_assert(C * C % NTF == 0, "whole passes");
+    float xv[IX];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {
+      const size_t o = (size_t)c * C * C + tid + it * NTF;
+      xv[it] = w.X[o];
+    }
     {  // the chunk's rows: every load of the thread in flight before its first store
       constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
       static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
@@ -574,9 +583,10 @@ __global__ void __launch_bounds__(NTF, 1)
       gC[i] = acc;
       eC[i] = expf(acc);
     }
-    for (int idx = tid; idx < C * C; idx += NTF) {  // T = X Diag(beta)
-      const int r = idx / C, s2 = idx % C;
-      TS[r * LDT + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {  // T = X Diag(beta)
+      const int idx = tid + it * NTF, r = idx / C, s2 = idx % C;
+      TS[r * LDT + s2] = xv[it] * bS[s2];
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka, Kc (into kS)
@@ -746,6 +756,16 @@ __global__ void __launch_bounds__(NTF, 1)
     const int t0 = c * C, n = min(C, up.len - t0);
     const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
+    // this chunk's X and A_qk from the key-side pass, loaded with the rows
+    constexpr int IX = C * C / NTF;
+    static_assert(C * C % NTF == 0, "whole passes");
+    float xv[IX], aqv[IX];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {
+      const size_t o = (size_t)c * C * C + tid + it * NTF;
+      xv[it] = w.X[o];
+      aqv[it] = w.Aqk[o];
+    }
     {  // the chunk's rows: every load of the thread in flight before its first store
       constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
       static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
@@ -795,11 +815,11 @@ __global__ void __launch_bounds__(NTF, 1)
       gC[i] = acc;
       eC[i] = expf(acc);
     }
-    for (int idx = tid; idx < C * C; idx += NTF) {
-      const int r = idx / C, s2 = idx % C;
-      const size_t o = ((size_t)c * C + r) * C + s2;
-      AqS[r * LDQ + s2] = w.Aqk[o];
-      TS[r * LDQ + s2] = w.X[o] * bS[s2];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {  // A_qk; T = X Diag(beta)
+      const int idx = tid + it * NTF, r = idx / C, s2 = idx % C;
+      AqS[r * LDQ + s2] = aqv[it];
+      TS[r * LDQ + s2] = xv[it] * bS[s2];
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {  // Qg, Ka, Kc
@@ -1652,6 +1672,16 @@ __global__ void __launch_bounds__(NTF, 1)
     const int t0 = c * C, n = min(C, up.len - t0);
     const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
     __syncthreads();
+    // this chunk's X and A_qk from the key-side pass, loaded with the rows
+    constexpr int IX = C * C / NTF;
+    static_assert(C * C % NTF == 0, "whole passes");
+    float xv[IX], aqv[IX];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {
+      const size_t o = (size_t)c * C * C + tid + it * NTF;
+      xv[it] = w.X[o];
+      aqv[it] = w.Aqk[o];
+    }
     {  // the chunk's rows: every load of the thread in flight before its first store
       constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
       static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
@@ -1697,10 +1727,11 @@ __global__ void __launch_bounds__(NTF, 1)
       gC[i] = acc;
       eC[i] = expf(acc);
     }
-    for (int idx = tid; idx < C * C; idx += NTF) {  // T = X Diag(beta); A_qk
-      const int r = idx / C, s2 = idx % C;
-      TS[r * LDT + s2] = w.X[((size_t)c * C + r) * C + s2] * bS[s2];
-      AqS[r * LDT + s2] = w.Aqk[((size_t)c * C + r) * C + s2];
+#pragma unroll
+    for (int it = 0; it < IX; ++it) {  // T = X Diag(beta); A_qk
+      const int idx = tid + it * NTF, r = idx / C, s2 = idx % C;
+      TS[r * LDT + s2] = xv[it] * bS[s2];
+      AqS[r * LDT + s2] = aqv[it];
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTF) {  // Ka, Kc (into kS), Q_gamma (into qS)
