@@ -246,6 +246,20 @@ __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int 
   return w;
 }
 
+// Copies a [rows][W] tile from shared memory (row stride ld) to a dense
+// global [rows][W] array with 16-byte accesses (every tile row and the
+// destination start on a multiple of 4 floats), NT threads.
+template <int NT, int W>
+__device__ __forceinline__ void copy_tile_out(float* __restrict__ dst, const float* src, int ld,
+                                              int rows) {
+  static_assert(W % 4 == 0, "16-byte rows");
+  for (int idx = threadIdx.x; idx < rows * (W / 4); idx += NT) {
+    const int r = idx / (W / 4), j = 4 * (idx % (W / 4));
+    *reinterpret_cast<float4*>(dst + (size_t)r * W + j) =
+        *reinterpret_cast<const float4*>(src + r * ld + j);
+  }
+}
+
 // chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to
 // C, into [C][LDK] tiles
 // g is the log-decay, or z when A_log is not null (the gate
@@ -569,10 +583,7 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       if (tid < C) bS[tid] = bv;
     }
-    for (int idx = tid; idx < DK * DV; idx += NTF) {  // chunk-start state
-      const int i = idx / DV, j = idx % DV;
-      w.S[(size_t)c * DK * DV + idx] = SS[i * LDV + j];
-    }
+    copy_tile_out<NTF, DV>(w.S + (size_t)c * DK * DV, SS, LDV, DK);  // chunk-start state
     __syncthreads();
     for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
       float acc = 0.f;
@@ -633,11 +644,8 @@ __global__ void __launch_bounds__(NTF, 1)
             US[frag_row(16 * mt, e) * LDV + frag_col(8 * (nt0 + q2), e)] = acc[q2][e];
       }
       __syncthreads();
-      for (int idx = tid; idx < C * DV; idx += NTF) {
-        const int r = idx / DV, j = idx % DV;
-        w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
-        w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
-      }
+      copy_tile_out<NTF, DV>(w.R + (size_t)c * C * DV, VS, LDV, C);
+      copy_tile_out<NTF, DV>(w.U + (size_t)c * C * DV, US, LDV, C);
       {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
         float acc[8][4];
         zero(acc);
@@ -672,11 +680,8 @@ __global__ void __launch_bounds__(NTF, 1)
         for_tile<C, DV, 1, DV / 16>([&](int m, int nn, int i, int j) { US[m * LDV + nn] = acc[i][j]; });
       }
       __syncthreads();
-      for (int idx = tid; idx < C * DV; idx += NTF) {
-        const int r = idx / DV, j = idx % DV;
-        w.R[((size_t)c * C + r) * DV + j] = VS[r * LDV + j];
-        w.U[((size_t)c * C + r) * DV + j] = US[r * LDV + j];
-      }
+      copy_tile_out<NTF, DV>(w.R + (size_t)c * C * DV, VS, LDV, C);
+      copy_tile_out<NTF, DV>(w.U + (size_t)c * C * DV, US, LDV, C);
       {  // S <- Diag(e^{Gamma_C}) S + Kc^T U
         float acc[DK / 32][DV / 16];
         zero(acc);
@@ -801,10 +806,7 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       if (tid < C) bS[tid] = bv;
     }
-    for (int idx = tid; idx < DK * DV; idx += NTF) {  // dL/dS_next of this chunk
-      const int i = idx / DV, j = idx % DV;
-      w.dS[(size_t)c * DK * DV + idx] = dSS[i * LDV + j];
-    }
+    copy_tile_out<NTF, DV>(w.dS + (size_t)c * DK * DV, dSS, LDV, DK);  // dL/dS_next of this chunk
     __syncthreads();
     for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
       float acc = 0.f;
@@ -875,11 +877,8 @@ __global__ void __launch_bounds__(NTF, 1)
           }
       }
       __syncthreads();
-      for (int idx = tid; idx < C * DV; idx += NTF) {
-        const int r = idx / DV, j = idx % DV;
-        w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
-        w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
-      }
+      copy_tile_out<NTF, DV>(w.dU + (size_t)c * C * DV, dUS, LDV, C);
+      copy_tile_out<NTF, DV>(w.W + (size_t)c * C * DV, WS, LDV, C);
       {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
         float acc[8][4];
         zero(acc);
@@ -923,11 +922,8 @@ __global__ void __launch_bounds__(NTF, 1)
         });
       }
       __syncthreads();
-      for (int idx = tid; idx < C * DV; idx += NTF) {
-        const int r = idx / DV, j = idx % DV;
-        w.dU[((size_t)c * C + r) * DV + j] = dUS[r * LDV + j];
-        w.W[((size_t)c * C + r) * DV + j] = WS[r * LDV + j];
-      }
+      copy_tile_out<NTF, DV>(w.dU + (size_t)c * C * DV, dUS, LDV, C);
+      copy_tile_out<NTF, DV>(w.W + (size_t)c * C * DV, WS, LDV, C);
       {  // dS <- Diag(e^{Gamma_C}) dS + Qg^T dO' - Ka^T W
         float acc[DK / 32][DV / 16];
         zero(acc);
