@@ -139,6 +139,20 @@ def test_chunk_size_invariance():
         assert rel_l2(to64(S), to64(res[0][1])) <= 1e-5
 
 
+@pytest.mark.parametrize("dk,dv", [(32, 128), (128, 64), (64, 128), (128, 32)])
+@pytest.mark.parametrize("T", [45, 301])
+def test_prefill_bf16_other_head_sizes(oracle_mod, dk, dv, T):
+    """bf16 inputs with dk or dv below 128 take the fp32-accuracy chunk path:
+    ragged lengths, initial states and scale against the oracle (o at the
+    bf16 bar, the fp32 state at the fp32 bar)."""
+    inp = W.make_prefill_inputs(2, T, 3, dk, dv, torch.bfloat16, seed=160 + T, device=DEV,
+                                init_state=True)
+    o, S, _, _ = gpu_prefill(inp, scale=0.8)
+    o_ref, S_ref = oracle_prefill(oracle_mod, inp, scale=0.8)
+    assert rel_l2(to64(o), o_ref) <= TOL_BF16_O
+    assert rel_l2(to64(S), S_ref) <= TOL_F32
+
+
 @pytest.mark.parametrize("dtype,dk,dv", [(torch.float32, 128, 128), (torch.float32, 64, 32),
                                          (torch.bfloat16, 64, 64)])
 def test_prefill_f32_path_packed_gated(oracle_mod, dtype, dk, dv):
