@@ -1,4 +1,7 @@
-// kda_bwd_chunk.cu -- gradients through the KDA recurrence in chunk form.
+// kda_bwd_chunk.cu -- the KDA recurrence in chunk form at fp32 accuracy:
+// its gradients, and the forward for the inputs the tcgen05 kernel does not
+// take (fp32, dk or dv below 128; see "fp32 forward" below: pass K, then a
+// scan like F that also forms O).
 //
 // The recurrence ("NLP--技术报告解读-Kimi-K3", joezjh.github.io, Model
 // Architecture > Kimi Delta Attention (KDA)) evaluated chunk by chunk as in
@@ -31,7 +34,9 @@
 // tf32 parts); the others are register-tiled CUDA-core loops.  Every output
 // element has one writer and every sum a fixed order: results are
 // deterministic.
-// Tail chunks are padded with g = 0, beta = 0, k = q = v = dO = 0.
+// Tail chunks are padded with g = 0, beta = 0, k = q = v = dO = 0.  Dense
+// batches longer than kBwdWindow tokens run in windows from checkpointed
+// start states (bounded workspace).
 #include <algorithm>
 
 #include "kda_bwd.cuh"
