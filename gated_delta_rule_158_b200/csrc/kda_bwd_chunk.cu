@@ -251,6 +251,25 @@ __device__ inline UnitWs unit_ws(float* ws, int64_t chunk0, int nc, int DK, int 
   return w;
 }
 
+// Four consecutive elements as a float4 (the address is 16-byte aligned for
+// fp32, 8-byte for bf16: every row starts on a multiple of 4 elements and
+// the tensors are 16-byte aligned), and a 16-byte shared store.
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float4 gate4(float4 z, float a_h, float g_min) {
+  return make_float4(gate_value(z.x, a_h, g_min), gate_value(z.y, a_h, g_min),
+                     gate_value(z.z, a_h, g_min), gate_value(z.w, a_h, g_min));
+}
+__device__ __forceinline__ float4 scale4(float4 v, float s) {
+  return make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
+}
+
 // Copies a [rows][W] tile from shared memory (row stride ld) to a dense
 // global [rows][W] array with 16-byte accesses (every tile row and the
 // destination start on a multiple of 4 floats), NT threads.
@@ -274,29 +293,31 @@ __device__ void load_keys(const Tin* q, const Tin* k, const float* g, const floa
                           float g_min, int h, const float* beta, size_t rowbase, int H, int n,
                           float* qS, float* kS, float* GS, float* bS) {
   const float a_h = A_log ? expf(A_log[h]) : 0.f;
-  // every load of the thread in flight before its first store
-  constexpr int IT = C * DK / NTH;
-  static_assert(C * DK % NTH == 0 && C <= NTH, "whole passes");
-  float qv[IT], kv[IT], gv[IT];
+  // four channels per load, every load of the thread in flight before its
+  // first store
+  constexpr int V4 = DK / 4, IT = C * V4 / NTH;
+  static_assert(C * V4 % NTH == 0 && C <= NTH, "whole passes");
+  float4 qv[IT], kv[IT], gv[IT];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int idx = threadIdx.x + it * NTH, r = idx / DK, i = idx % DK;
-    qv[it] = kv[it] = gv[it] = 0.f;
+    const int idx = threadIdx.x + it * NTH, r = idx / V4, i = 4 * (idx % V4);
+    qv[it] = kv[it] = gv[it] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < n) {
       const size_t off = (rowbase + (size_t)r * H) * DK + i;
-      qv[it] = Elem<Tin>::load(q + off);
-      kv[it] = Elem<Tin>::load(k + off);
-      gv[it] = A_log ? gate_value(g[off], a_h, g_min) : g[off];
+      qv[it] = ld4(q + off);
+      kv[it] = ld4(k + off);
+      gv[it] = ld4(g + off);
+      if (A_log) gv[it] = gate4(gv[it], a_h, g_min);
     }
   }
   const int rb = threadIdx.x;
   const float bv = rb < C && rb < n ? beta[rowbase + (size_t)rb * H] : 0.f;
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
-    const int idx = threadIdx.x + it * NTH, r = idx / DK, i = idx % DK;
-    qS[r * LDK + i] = qv[it];
-    kS[r * LDK + i] = kv[it];
-    GS[r * LDK + i] = gv[it];
+    const int idx = threadIdx.x + it * NTH, r = idx / V4, i = 4 * (idx % V4);
+    st4(qS + r * LDK + i, qv[it]);
+    st4(kS + r * LDK + i, kv[it]);
+    st4(GS + r * LDK + i, gv[it]);
   }
   if (rb < C) bS[rb] = bv;
   __syncthreads();
@@ -555,36 +576,40 @@ __global__ void __launch_bounds__(NTF, 1)
       const size_t o = (size_t)c * C * C + tid + it * NTF;
       xv[it] = w.X[o];
     }
-    {  // the chunk's rows: every load of the thread in flight before its first store
-      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
-      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
-      float kv[IK], gv[IK], vv[IV];
+    {  // the chunk's rows, four elements per load, every load of the thread in
+       // flight before its first store
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = (C * K4 + NTF - 1) / NTF, IV = (C * V4 + NTF - 1) / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 kv[IK], gv[IK], vv[IV];
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        kv[it] = gv[it] = 0.f;
-        if (r < n) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        kv[it] = gv[it] = z4;
+        if (idx < C * K4 && r < n) {
           const size_t off = (rowbase + (size_t)r * H) * DK + i;
-          kv[it] = Elem<Tin>::load(k + off);
-          gv[it] = g[off];
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
         }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        vv[it] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        vv[it] = idx < C * V4 && r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + j) : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        kS[r * LKC + i] = kv[it];
-        GS[r * LDK + i] = gv[it];
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        if (idx < C * K4) {
+          st4(kS + r * LKC + i, kv[it]);
+          st4(GS + r * LDK + i, gv[it]);
+        }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        VS[r * LDV + j] = vv[it];
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        if (idx < C * V4) st4(VS + r * LDV + j, vv[it]);
       }
       if (tid < C) bS[tid] = bv;
     }
@@ -776,38 +801,44 @@ __global__ void __launch_bounds__(NTF, 1)
       xv[it] = w.X[o];
       aqv[it] = w.Aqk[o];
     }
-    {  // the chunk's rows: every load of the thread in flight before its first store
-      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
-      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
-      float qv[IK], kv[IK], gv[IK], ov[IV];
+    {  // the chunk's rows, four elements per load, every load of the thread in
+       // flight before its first store
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = (C * K4 + NTF - 1) / NTF, IV = (C * V4 + NTF - 1) / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 qv[IK], kv[IK], gv[IK], ov[IV];
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        qv[it] = kv[it] = gv[it] = 0.f;
-        if (r < n) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        qv[it] = kv[it] = gv[it] = z4;
+        if (idx < C * K4 && r < n) {
           const size_t off = (rowbase + (size_t)r * H) * DK + i;
-          qv[it] = Elem<Tin>::load(q + off);
-          kv[it] = Elem<Tin>::load(k + off);
-          gv[it] = g[off];
+          qv[it] = ld4(q + off);
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
         }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        ov[it] = r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        ov[it] = idx < C * V4 && r < n
+                     ? scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + j), scale)
+                     : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        qS[r * LQT + i] = qv[it];
-        kS[r * LDK + i] = kv[it];
-        GS[r * LQT + i] = gv[it];
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        if (idx < C * K4) {
+          st4(qS + r * LQT + i, qv[it]);
+          st4(kS + r * LDK + i, kv[it]);
+          st4(GS + r * LQT + i, gv[it]);
+        }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        dOS[r * LDV + j] = ov[it];
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        if (idx < C * V4) st4(dOS + r * LDV + j, ov[it]);
       }
       if (tid < C) bS[tid] = bv;
     }
@@ -1683,38 +1714,43 @@ __global__ void __launch_bounds__(NTF, 1)
       xv[it] = w.X[o];
       aqv[it] = w.Aqk[o];
     }
-    {  // the chunk's rows: every load of the thread in flight before its first store
-      constexpr int IK = C * DK / NTF, IV = C * DV / NTF;
-      static_assert(C * DK % NTF == 0 && C * DV % NTF == 0, "whole passes");
-      float qv[IK], kv[IK], gv[IK], vv[IV];
+    {  // the chunk's rows, four elements per load, every load of the thread in
+       // flight before its first store
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = (C * K4 + NTF - 1) / NTF, IV = (C * V4 + NTF - 1) / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 qv[IK], kv[IK], gv[IK], vv[IV];
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        qv[it] = kv[it] = gv[it] = 0.f;
-        if (r < n) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        qv[it] = kv[it] = gv[it] = z4;
+        if (idx < C * K4 && r < n) {
           const size_t off = (rowbase + (size_t)r * H) * DK + i;
-          qv[it] = Elem<Tin>::load(q + off);
-          kv[it] = Elem<Tin>::load(k + off);
-          gv[it] = A_log ? gate_value(g[off], a_h, g_min) : g[off];
+          qv[it] = ld4(q + off);
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
+          if (A_log) gv[it] = gate4(gv[it], a_h, g_min);
         }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        vv[it] = r < n ? Elem<Tin>::load(v + (rowbase + (size_t)r * H) * DV + j) : 0.f;
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        vv[it] = idx < C * V4 && r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + j) : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
-        const int idx = tid + it * NTF, r = idx / DK, i = idx % DK;
-        qS[r * LDK + i] = qv[it];
-        kS[r * LKC + i] = kv[it];
-        GS[r * LDK + i] = gv[it];
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        if (idx < C * K4) {
+          st4(qS + r * LDK + i, qv[it]);
+          st4(kS + r * LKC + i, kv[it]);
+          st4(GS + r * LDK + i, gv[it]);
+        }
       }
 #pragma unroll
       for (int it = 0; it < IV; ++it) {
-        const int idx = tid + it * NTF, r = idx / DV, j = idx % DV;
-        VS[r * LDV + j] = vv[it];
+        const int idx = tid + it * NTF, r = idx / V4, j = 4 * (idx % V4);
+        if (idx < C * V4) st4(VS + r * LDV + j, vv[it]);
       }
       if (tid < C) bS[tid] = bv;
     }
