@@ -262,6 +262,14 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+// Two adjacent outputs of an m16n8 fragment (columns 2t, 2t + 1): one 8-byte
+// fp32 or 4-byte bf16 store.
+__device__ __forceinline__ void st2(float* p, float a, float b) {
+  *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+__device__ __forceinline__ void st2(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
 __device__ __forceinline__ float4 gate4(float4 z, float a_h, float g_min) {
   return make_float4(gate_value(z.x, a_h, g_min), gate_value(z.y, a_h, g_min),
                      gate_value(z.z, a_h, g_min), gate_value(z.w, a_h, g_min));
@@ -906,10 +914,11 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {  // elements e, e + 1: adjacent columns
             const int m = frag_row(16 * mt, e), nn = frag_col(8 * (nt0 + q2), e);
             WS[m * LDV + nn] = acc[q2][e];
-            if (m < n) dv[(rowbase + (size_t)m * H) * DV + nn] = acc[q2][e];
+            WS[m * LDV + nn + 1] = acc[q2][e + 1];
+            if (m < n) st2(dv + (rowbase + (size_t)m * H) * DV + nn, acc[q2][e], acc[q2][e + 1]);
           }
       }
       __syncthreads();
@@ -1124,10 +1133,11 @@ __global__ void __launch_bounds__(NTH, 2)
         put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
         put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
       }
-      for (int idx = tid; idx < C * VBB; idx += NTH) {
-        const int r = idx / VBB, j = idx % VBB;
-        dOS[r * LDBB + j] =
-            r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {  // four columns per load
+        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        st4(dOS + r * LDBB + j,
+            r < n ? scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + j0 + j), scale)
+                  : make_float4(0.f, 0.f, 0.f, 0.f));
       }
       __syncthreads();
       for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
@@ -1207,10 +1217,11 @@ __global__ void __launch_bounds__(NTH, 2)
         put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
         put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
       }
-      for (int idx = tid; idx < C * VBB; idx += NTH) {
-        const int r = idx / VBB, j = idx % VBB;
-        dOS[r * LDBB + j] =
-            r < n ? scale * Elem<Tin>::load(dout + (rowbase + (size_t)r * H) * DV + j0 + j) : 0.f;
+      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {  // four columns per load
+        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
+        st4(dOS + r * LDBB + j,
+            r < n ? scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + j0 + j), scale)
+                  : make_float4(0.f, 0.f, 0.f, 0.f));
       }
       __syncthreads();
       for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
@@ -1834,9 +1845,11 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {  // elements e, e + 1: adjacent columns
             const int r = frag_row(16 * mt, e), j = frag_col(8 * (nt0 + q2), e);
-            if (r < n) Elem<Tin>::store(out + (rowbase + (size_t)r * H) * DV + j, scale * acc[q2][e]);
+            if (r < n)
+              st2(out + (rowbase + (size_t)r * H) * DV + j, scale * acc[q2][e],
+                  scale * acc[q2][e + 1]);
           }
       }
       __syncthreads();  // S is read by the O product above and rewritten below
