@@ -1059,6 +1059,16 @@ __global__ void __launch_bounds__(NTH, 2)
   const int tid = threadIdx.x;
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
+  // the chunk's X and L from the key-side pass: loads in flight with the keys'
+  constexpr int IX = C * C / NTH;
+  static_assert(C * C % NTH == 0, "whole passes");
+  float xv[IX], lv[IX];
+#pragma unroll
+  for (int it = 0; it < IX; ++it) {
+    const size_t o = (size_t)c * C * C + tid + it * NTH;
+    xv[it] = w.X[o];
+    lv[it] = w.L[o];
+  }
   load_keys<Tin, DK, LDK>(q, k, g, nullptr, 0.f, h, beta, rowbase, H, n, qS, kS, GS, bS);
   // The factorised backward through the Gram matrices works on 16-row
   // blocks with a reference row per block pair: rows 7 and 23 inside the
@@ -1073,11 +1083,11 @@ __global__ void __launch_bounds__(NTH, 2)
     for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - (r < 16 ? g7 : g23)) > 60.f;
   }
   wide = __syncthreads_or(wide);
-  for (int idx = tid; idx < C * C; idx += NTH) {
-    const int r = idx / C, s = idx % C;
-    const size_t o = ((size_t)c * C + r) * C + s;
-    XS[r * LDC + s] = w.X[o];
-    LS[r * LDC + s] = w.L[o];
+#pragma unroll
+  for (int it = 0; it < IX; ++it) {
+    const int idx = tid + it * NTH, r = idx / C, s = idx % C;
+    XS[r * LDC + s] = xv[it];
+    LS[r * LDC + s] = lv[it];
   }
   for (int i = tid; i < DK; i += NTH) {
     gC[i] = GS[(C - 1) * LDK + i];
