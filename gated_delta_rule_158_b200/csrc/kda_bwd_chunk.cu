@@ -40,6 +40,8 @@
 #include <algorithm>
 
 #include "kda_bwd.cuh"
+#include "kda_sync.cuh"
+#include "kda_tc_ptx.cuh"
 #include "kda_warp_mma.cuh"
 
 namespace kda {
@@ -998,23 +1000,77 @@ constexpr int VBB = 16;
 constexpr int LDBB = VBB + 4;
 static_assert(LDBB % 4 == 0, "16-byte aligned rows of the dv-block tiles");
 
+// At DK = 128 the dv-block products run on tcgen05 (kind::tf32, fp32
+// accumulators in TMEM): each operand is split into a high and a low tf32
+// part when it is staged, and D += a_lo b_hi + a_hi b_lo + a_hi b_hi.  A
+// stage holds one dv block of 16 columns, K-major without swizzle (core
+// matrices of 8 rows x 16 bytes; the four along K adjacent, LBO = 128 B;
+// 8-row groups 512 B apart): the S and dS blocks (128 rows, the A operands
+// of dQg^T, dKa^T, dKc^T) and the C-row tiles in the order dU, dO', W, U, R,
+// so that rows 32..95 ([dO'; W]) and 96..127 (U) are the B operands of
+//   D1 = S [dO'; W]^T  (dQg^T | -dKa^T),   D2 = dS U^T  (dKc^T)
+// and rows 0..127 times rows 96..159 give D3 = [dU; dO'; W; U] [U; R]^T,
+// whose blocks dU R^T (rows 0..31, columns 32..63) and dO' U^T (rows
+// 32..63, columns 0..31) are dT and dA_qk.
+constexpr int TC_VB = 16;
+constexpr int TC_CROWS = 5 * C;
+constexpr int TC_SH = 0, TC_SL = 128 * TC_VB, TC_DH = 2 * 128 * TC_VB, TC_DL = 3 * 128 * TC_VB;
+constexpr int TC_CH = 4 * 128 * TC_VB, TC_CL = TC_CH + TC_CROWS * TC_VB;
+constexpr int TC_STAGE = TC_CL + TC_CROWS * TC_VB;  // floats per stage
+constexpr uint32_t TC_LBO = 128, TC_SBO = 512;
+constexpr uint32_t TC_COLS = 256;                    // TMEM: D1 0..63, D2 64..95, D3 128..191
+constexpr uint32_t TC_D1 = 0, TC_D2 = 64, TC_D3 = 128;
+constexpr int32_t kDetailBwdMma = 0xB410;            // timeout detail: B's MMA barriers
+// float offset of element (row, 4 q) of a stage tile
+__device__ __forceinline__ int tc_off(int row, int q) {
+  return (row >> 3) * 128 + q * 32 + (row & 7) * 4;
+}
+// 16 / 32 consecutive fp32 TMEM columns of this warp's 32 lanes, with the wait
+// in the same asm statement so that no use of v is scheduled before the data
+// has arrived
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float* v) {
+  tmem_ld16_wait(taddr, v);
+  tmem_ld16_wait(taddr + 16, v + 16);
+}
+
 template <int DK>
 struct BSmem {
   // 8 (mod 32): after the dv-block loop, q, k and the k e^{Gamma_15 - Gamma}
   // factor are [K][N] operands of the backward through the Gram matrices
   static constexpr int LDK = DK + 8;
-  // the dv-block loop's tiles (S and dS blocks; dO', R, U, dU, W blocks) are
-  // dead once the loop ends; the dGamma accumulator and a C x C scratch tile
-  // take their place (dq and dk accumulate in their outputs)
-  static constexpr int loop = 2 * DK * LDBB + 5 * C * LDBB > 2 * C * LDK
-                                  ? 2 * DK * LDBB + 5 * C * LDBB : 2 * C * LDK;
+  // CUDA-core loop (DK < 128): its tiles (S and dS blocks; dO', R, U, dU, W
+  // blocks) are dead once the loop ends and the dGamma accumulator and a C x C
+  // scratch tile take their place.  At DK = 128 the tcgen05 stages take the
+  // whole shared memory during the loop and every other tile is filled after it.
+  static constexpr bool tc = DK == 128;
+  static constexpr int loop = tc ? 2 * C * LDK
+                                 : (2 * DK * LDBB + 5 * C * LDBB > 2 * C * LDK
+                                        ? 2 * DK * LDBB + 5 * C * LDBB : 2 * C * LDK);
   static constexpr int after = C * LDK + C * LDC;
   static_assert(after <= loop, "post-loop tiles fit the loop tiles");
   static_assert(2 * C * LDK <= loop, "dGamma and the k e^{Gamma_15 - Gamma} factor fit the loop tiles");
-  static constexpr int floats = 3 * C * LDK      // q, k, Gamma
-                                + loop
-                                + 4 * C * LDC    // X, L, dA_qk, dT (then dM)
-                                + C + 3 * DK;    // beta, Gamma_C, two dGamma_C terms
+  static constexpr int post = 3 * C * LDK      // q, k, Gamma
+                              + loop
+                              + 4 * C * LDC    // X, L, dA_qk, dT (then dM)
+                              + C + 3 * DK;    // beta, Gamma_C, two dGamma_C terms
+  static constexpr int stages = tc ? 2 * TC_STAGE : 0;
+  // then three mbarriers, the TMEM address and an abort flag
+  static constexpr int bar_off = ((post > stages ? post : stages) + 3) / 4 * 4;
+  static constexpr int floats = bar_off + 16;
   static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -1059,40 +1115,42 @@ __global__ void __launch_bounds__(NTH, 2)
   const int tid = threadIdx.x;
   constexpr int TMK = DK / 32;  // rows per thread of the DK x C products
 
-  // the chunk's X and L from the key-side pass: loads in flight with the keys'
-  constexpr int IX = C * C / NTH;
-  static_assert(C * C % NTH == 0, "whole passes");
-  float xv[IX], lv[IX];
+  // The chunk's keys (q, k, Gamma, beta), X and L into shared memory, Gamma_C,
+  // and whether the blocked backward through the Gram matrices takes it.
+  auto prologue = [&]() -> bool {
+    // X and L from the key-side pass: loads in flight with the keys'
+    constexpr int IX = C * C / NTH;
+    static_assert(C * C % NTH == 0, "whole passes");
+    float xv[IX], lv[IX];
 #pragma unroll
-  for (int it = 0; it < IX; ++it) {
-    const size_t o = (size_t)c * C * C + tid + it * NTH;
-    xv[it] = w.X[o];
-    lv[it] = w.L[o];
-  }
-  load_keys<Tin, DK, LDK>(q, k, g, nullptr, 0.f, h, beta, rowbase, H, n, qS, kS, GS, bS);
-  // The factorised backward through the Gram matrices works on 16-row
-  // blocks with a reference row per block pair: rows 7 and 23 inside the
-  // diagonal blocks, row 15 between them (where both factors are <= 1).  It
-  // scales sums of up to 16 terms of size e^{|Gamma_r - Gamma_ref|} |dL| by
-  // the opposite factor, so it takes the chunk only while every
-  // |Gamma_r - Gamma_ref| inside a diagonal block stays below 60 (at most 8
-  // steps of the gate's g >= -5, i.e. 40, for every gated input).
-  bool wide = false;
-  for (int i = tid; i < DK; i += NTH) {
-    const float g7 = GS[7 * LDK + i], g23 = GS[23 * LDK + i];
-    for (int r = 0; r < C; ++r) wide |= fabsf(GS[r * LDK + i] - (r < 16 ? g7 : g23)) > 60.f;
-  }
-  wide = __syncthreads_or(wide);
+    for (int it = 0; it < IX; ++it) {
+      const size_t o = (size_t)c * C * C + tid + it * NTH;
+      xv[it] = w.X[o];
+      lv[it] = w.L[o];
+    }
+    load_keys<Tin, DK, LDK>(q, k, g, nullptr, 0.f, h, beta, rowbase, H, n, qS, kS, GS, bS);
+    // The factorised backward through the Gram matrices works on 16-row
+    // blocks with a reference row per block pair: rows 7 and 23 inside the
+    // diagonal blocks, row 15 between them (where both factors are <= 1).  It
+    // scales sums of up to 16 terms of size e^{|Gamma_r - Gamma_ref|} |dL| by
+    // the opposite factor, so it takes the chunk only while every
+    // |Gamma_r - Gamma_ref| inside a diagonal block stays below 60 (at most 8
+    // steps of the gate's g >= -5, i.e. 40, for every gated input).
+    bool wd = false;
+    for (int i = tid; i < DK; i += NTH) {
+      const float g7 = GS[7 * LDK + i], g23 = GS[23 * LDK + i];
+      for (int r = 0; r < C; ++r) wd |= fabsf(GS[r * LDK + i] - (r < 16 ? g7 : g23)) > 60.f;
+    }
+    wd = __syncthreads_or(wd);
 #pragma unroll
-  for (int it = 0; it < IX; ++it) {
-    const int idx = tid + it * NTH, r = idx / C, s = idx % C;
-    XS[r * LDC + s] = xv[it];
-    LS[r * LDC + s] = lv[it];
-  }
-  for (int i = tid; i < DK; i += NTH) {
-    gC[i] = GS[(C - 1) * LDK + i];
-    rsum[i] = 0.f;
-  }
+    for (int it = 0; it < IX; ++it) {
+      const int idx = tid + it * NTH, r = idx / C, s = idx % C;
+      XS[r * LDC + s] = xv[it];
+      LS[r * LDC + s] = lv[it];
+    }
+    for (int i = tid; i < DK; i += NTH) gC[i] = GS[(C - 1) * LDK + i];
+    return wd;
+  };
 
   // products summed over the dv columns, accumulated block by block from
   // the saved R, U, dU, W:
@@ -1112,95 +1170,163 @@ __global__ void __launch_bounds__(NTH, 2)
     aG[r * LDK + i] = fmaf(fmaf(dQg, qv, dKa * kv), e, -dKc * kv * ec);
     return dKc * kv * ec;  // dKc Kc, summed over r into dGamma_C
   };
+  bool wide;
   if constexpr (DK == 128) {
-    // tensor cores: warp w owns rows 16w .. 16w+15 of dQg^T, -dKa^T, dKc^T
-    // (4 n-tiles of 8 chunk rows each) and one 16 x 16 corner of dA_qk
-    // (warps 0-3) or dT (warps 4-7)
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int mc = (warp & 3) >> 1, nc0 = (warp & 1) * 2;
-    float aQ[4][4], aKa[4][4], aKc[4][4], aC[2][4];
-    zero(aQ);
-    zero(aKa);
-    zero(aKc);
-    zero(aC);
-    for (int j0 = 0; j0 < DV; j0 += VBB) {
-      __syncthreads();
-      // 16-byte loads of the saved blocks (rows of 16 floats, 16-byte aligned)
-      // one 16-byte store (every tile of the block loop starts on a multiple
-      // of 4 floats, and rows are LDBB = 20 floats)
-      auto put4 = [](float* dst, float4 x) { *reinterpret_cast<float4*>(dst) = x; };
-      for (int idx = tid; idx < DK * VBB / 4; idx += NTH) {
-        const int i = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
-        const size_t o = ((size_t)c * DK + i) * DV + j0 + j;
-        put4(SS + i * LDBB + j, *reinterpret_cast<const float4*>(w.S + o));
-        put4(dSS + i * LDBB + j, *reinterpret_cast<const float4*>(w.dS + o));
-      }
-      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {
-        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
-        const size_t o = ((size_t)c * C + r) * DV + j0 + j;
-        put4(RS + r * LDBB + j, *reinterpret_cast<const float4*>(w.R + o));
-        put4(US + r * LDBB + j, *reinterpret_cast<const float4*>(w.U + o));
-        put4(dUS + r * LDBB + j, *reinterpret_cast<const float4*>(w.dU + o));
-        put4(WS + r * LDBB + j, *reinterpret_cast<const float4*>(w.W + o));
-      }
-      for (int idx = tid; idx < C * VBB / 4; idx += NTH) {  // four columns per load
-        const int r = idx / (VBB / 4), j = 4 * (idx % (VBB / 4));
-        st4(dOS + r * LDBB + j,
-            r < n ? scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + j0 + j), scale)
-                  : make_float4(0.f, 0.f, 0.f, 0.f));
-      }
-      __syncthreads();
-      for (int i = tid; i < DK; i += NTH) {  // sum_j dS_ij S_ij of this block (row i: thread i)
-        float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < VBB; ++j) acc = fmaf(dSS[i * LDBB + j], SS[i * LDBB + j], acc);
-        rsum[i] += acc;
-      }
-      for (int k0 = 0; k0 < VBB; k0 += 8) {
-        Frag3 fs, fd, fc;
-        load_a(fs, SS, LDBB, 16 * warp, k0);
-        load_a(fd, dSS, LDBB, 16 * warp, k0);
+    // tcgen05: the block loop fills the stages (every warp loads, splits
+    // and stores; the loads of block j are in flight while the MMAs of block
+    // j - 1 run), thread 0 issues the block's 18 MMAs and commits them to the
+    // stage's barrier, which frees the stage for block j + 2.
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BSmem<DK>::bar_off);  // 2 stages, drain
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 3);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    StatusBlock* sbw = const_cast<StatusBlock*>(map.sb);
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+      for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+      *abort_flag = 0;
+      tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+      tc::tmem_alloc(tslot, TC_COLS);
+      tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tslot;
+    static_assert(128 * TC_VB / 4 == 2 * NTH, "two S and two dS loads per thread");
+    static_assert(TC_CROWS * TC_VB / 4 <= 3 * NTH, "three C-row loads per thread");
+    float racc[2] = {0.f, 0.f};  // sum_j dS_ij S_ij of this thread's S rows
+    bool bad = false;
+    const int nb = DV / TC_VB;
+    for (int jb = 0; jb < nb; ++jb) {
+      const int j0 = jb * TC_VB, b = jb & 1;
+      float* st = sm + b * TC_STAGE;
+      float4 sv[2], dsv[2], cv[3];
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          mma3(aQ[nt], fs, dOS, LDBB, 8 * nt, k0);
-          mma3(aKa[nt], fs, WS, LDBB, 8 * nt, k0);
-          mma3(aKc[nt], fd, US, LDBB, 8 * nt, k0);
+      for (int it = 0; it < 2; ++it) {
+        const int idx = tid + it * NTH, i = idx >> 2, qd = idx & 3;
+        const size_t o = ((size_t)c * DK + i) * DV + j0 + 4 * qd;
+        sv[it] = *reinterpret_cast<const float4*>(w.S + o);
+        dsv[it] = *reinterpret_cast<const float4*>(w.dS + o);
+      }
+#pragma unroll
+      for (int it = 0; it < 3; ++it) {
+        const int idx = tid + it * NTH, row = idx >> 2, qd = idx & 3, r = row & 31;
+        const size_t o = ((size_t)c * C + r) * DV + j0 + 4 * qd;
+        cv[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < TC_CROWS * TC_VB / 4) {
+          switch (row >> 5) {  // warp-uniform: a warp stages 8 rows of one tile
+            case 0: cv[it] = *reinterpret_cast<const float4*>(w.dU + o); break;
+            case 1:
+              if (r < n) cv[it] = scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + j0 + 4 * qd), scale);
+              break;
+            case 2: cv[it] = *reinterpret_cast<const float4*>(w.W + o); break;
+            case 3: cv[it] = *reinterpret_cast<const float4*>(w.U + o); break;
+            default: cv[it] = *reinterpret_cast<const float4*>(w.R + o); break;
+          }
         }
-        load_a(fc, warp < 4 ? dOS : dUS, LDBB, 16 * mc, k0);
+      }
+      // the stage is free once the MMAs of block jb - 2 have completed
+      if (jb >= 2) bad |= !mbar_wait_bounded(&bars[b], ((jb - 2) >> 1) & 1, abort_flag, sbw, kDetailBwdMma);
+      auto put_hl = [&](int hoff, int loff, float4 v) {
+        uint4 hi, lo;
+        split_tf32(v.x, hi.x, lo.x);
+        split_tf32(v.y, hi.y, lo.y);
+        split_tf32(v.z, hi.z, lo.z);
+        split_tf32(v.w, hi.w, lo.w);
+        *reinterpret_cast<uint4*>(st + hoff) = hi;
+        *reinterpret_cast<uint4*>(st + loff) = lo;
+      };
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2)
-          mma3(aC[q2], fc, warp < 4 ? US : RS, LDBB, 8 * (nc0 + q2), k0);
+      for (int it = 0; it < 2; ++it) {
+        const int idx = tid + it * NTH, o = tc_off(idx >> 2, idx & 3);
+        put_hl(TC_SH + o, TC_SL + o, sv[it]);
+        put_hl(TC_DH + o, TC_DL + o, dsv[it]);
+        racc[it] = fmaf(dsv[it].x, sv[it].x, racc[it]);
+        racc[it] = fmaf(dsv[it].y, sv[it].y, racc[it]);
+        racc[it] = fmaf(dsv[it].z, sv[it].z, racc[it]);
+        racc[it] = fmaf(dsv[it].w, sv[it].w, racc[it]);
+      }
+#pragma unroll
+      for (int it = 0; it < 3; ++it) {
+        const int idx = tid + it * NTH, o = tc_off(idx >> 2, idx & 3);
+        if (idx < TC_CROWS * TC_VB / 4) put_hl(TC_CH + o, TC_CL + o, cv[it]);
+      }
+      tc::fence_proxy_async();  // the stores, visible to the tensor cores
+      if (__syncthreads_or(bad)) {
+        bad = true;
+        break;
+      }
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t s0 = smem_u32(st);
+        const uint32_t id64 = tc::idesc(tc::kFmtTF32, 128, 64, false, false, false);
+        const uint32_t id32 = tc::idesc(tc::kFmtTF32, 128, 32, false, false, false);
+        auto dsc = [&](int tile, int row0, int kk) {
+          return tc::plain_desc(s0 + 4u * (uint32_t)tile + (uint32_t)(row0 / 8) * TC_SBO + 2u * TC_LBO * kk,
+                                TC_LBO, TC_SBO);
+        };
+#pragma unroll
+        for (int kk = 0; kk < TC_VB / 8; ++kk)
+#pragma unroll
+          for (int term = 0; term < 3; ++term) {  // a_lo b_hi, a_hi b_lo, a_hi b_hi
+            const int sa = term == 0 ? TC_SL : TC_SH, da = term == 0 ? TC_DL : TC_DH;
+            const int ca = term == 0 ? TC_CL : TC_CH, cb = term == 1 ? TC_CL : TC_CH;
+            const uint32_t acc = (jb > 0 || kk > 0 || term > 0) ? 1u : 0u;
+            tc::mma_ss(tbase + TC_D1, dsc(sa, 0, kk), dsc(cb, 32, kk), id64, 1, acc);
+            tc::mma_ss(tbase + TC_D2, dsc(da, 0, kk), dsc(cb, 96, kk), id32, 1, acc);
+            tc::mma_ss(tbase + TC_D3, dsc(ca, 0, kk), dsc(cb, 96, kk), id64, 1, acc);
+          }
+        tc::mma_commit(&bars[b]);
       }
     }
-    __syncthreads();  // the loop tiles become the dGamma accumulator
-    float kc0 = 0.f, kc1 = 0.f;  // sum_r dKc Kc of rows 16w + g and 16w + g + 8
+    // every MMA issued: wait for them before the stages are reused and TMEM read
+    if (tid == 0) tc::mma_commit(&bars[2]);
+    if (!mbar_wait_bounded(&bars[2], 0, abort_flag, sbw, kDetailBwdMma)) mbar_wait_drain(&bars[2], 0);
+    tc::fence_after_sync();
+    wide = prologue();
+    {  // sum_j dS_ij S_ij: the four threads of each row
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 16 * warp + g + 8 * (e >> 1), r = 8 * nt + 2 * t + (e & 1);
-        const float kk = elem(i, r, aQ[nt][e], -aKa[nt][e], aKc[nt][e]);
-        if (e < 2) kc0 += kk; else kc1 += kk;
+      for (int it = 0; it < 2; ++it) {
+        float v = racc[it];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        if ((tid & 3) == 0) rsum[(tid + it * NTH) >> 2] = v;
       }
-    kc0 += __shfl_xor_sync(0xffffffffu, kc0, 1);
-    kc1 += __shfl_xor_sync(0xffffffffu, kc1, 1);
-    kc0 += __shfl_xor_sync(0xffffffffu, kc0, 2);
-    kc1 += __shfl_xor_sync(0xffffffffu, kc1, 2);
-    if (t == 0) {
-      kcsum[16 * warp + g] = kc0;
-      kcsum[16 * warp + g + 8] = kc1;
+      for (int i = tid; i < DK; i += NTH) kcsum[i] = 0.f;
     }
+    __syncthreads();
+    {  // D1, D2: row i of dQg^T, -dKa^T, dKc^T in TMEM lane i; warps w and w + 4
+       // take chunk rows 0..15 and 16..31
+      const uint32_t lrow = (uint32_t)(32 * (warp & 3)) << 16;
+      const int i = 32 * (warp & 3) + lane, r0 = 16 * (warp >> 2);
+      float vq[16], vw[16], vc[16];
+      tmem_ld16_wait(tbase + lrow + TC_D1 + r0, vq);
+      tmem_ld16_wait(tbase + lrow + TC_D1 + 32 + r0, vw);
+      tmem_ld16_wait(tbase + lrow + TC_D2 + r0, vc);
+      float kc = 0.f;
 #pragma unroll
-    for (int q2 = 0; q2 < 2; ++q2)
+      for (int rr = 0; rr < 16; ++rr) kc += elem(i, r0 + rr, vq[rr], -vw[rr], vc[rr]);
+      atomicAdd(&kcsum[i], kc);  // two addends onto 0: the same sum in either order
+    }
+    if (warp < 2) {  // D3: dT (lanes 0..31, columns 32..63), dA_qk (lanes 32..63, columns 0..31)
+      float v[32];
+      tmem_ld32_wait(tbase + ((uint32_t)(32 * warp) << 16) + TC_D3 + (warp == 0 ? 32 : 0), v);
+      if (warp == 0) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 16 * mc + g + 8 * (e >> 1), s2 = 8 * (nc0 + q2) + 2 * t + (e & 1);
-        if (warp < 4)
-          dAqS[r * LDC + s2] = s2 <= r ? aC[q2][e] : 0.f;
-        else
-          dTS[r * LDC + s2] = aC[q2][e];
+        for (int s2 = 0; s2 < C; ++s2) dTS[lane * LDC + s2] = v[s2];
+      } else {
+#pragma unroll
+        for (int s2 = 0; s2 < C; ++s2) dAqS[lane * LDC + s2] = s2 <= lane ? v[s2] : 0.f;
       }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, TC_COLS);
   } else {
+    wide = prologue();
+    for (int i = tid; i < DK; i += NTH) rsum[i] = 0.f;
     float aQ[TMK][4], aKa[TMK][4], aKc[TMK][4], aA[2][2], aT[2][2];
     zero(aQ);
     zero(aKa);
