@@ -1025,6 +1025,12 @@ constexpr int32_t kDetailBwdMma = 0xB410;            // timeout detail: B's MMA 
 __device__ __forceinline__ int tc_off(int row, int q) {
   return (row >> 3) * 128 + q * 32 + (row & 7) * 4;
 }
+// The (row, q) that staging slot idx takes: 32 consecutive slots cover an
+// 8-row group, the 8 lanes of each quarter-warp one core matrix (8 rows of
+// one q: 128 contiguous bytes, so the 16-byte stores are free of bank
+// conflicts); the four threads of a row are lanes l, l + 8, l + 16, l + 24.
+__device__ __forceinline__ int tc_row(int idx) { return ((idx >> 5) << 3) | (idx & 7); }
+__device__ __forceinline__ int tc_q(int idx) { return (idx >> 3) & 3; }
 // 16 / 32 consecutive fp32 TMEM columns of this warp's 32 lanes, with the wait
 // in the same asm statement so that no use of v is scheduled before the data
 // has arrived
@@ -1205,14 +1211,14 @@ __global__ void __launch_bounds__(NTH, 2)
       float4 sv[2], dsv[2], cv[3];
 #pragma unroll
       for (int it = 0; it < 2; ++it) {
-        const int idx = tid + it * NTH, i = idx >> 2, qd = idx & 3;
+        const int idx = tid + it * NTH, i = tc_row(idx), qd = tc_q(idx);
         const size_t o = ((size_t)c * DK + i) * DV + j0 + 4 * qd;
         sv[it] = *reinterpret_cast<const float4*>(w.S + o);
         dsv[it] = *reinterpret_cast<const float4*>(w.dS + o);
       }
 #pragma unroll
       for (int it = 0; it < 3; ++it) {
-        const int idx = tid + it * NTH, row = idx >> 2, qd = idx & 3, r = row & 31;
+        const int idx = tid + it * NTH, row = tc_row(idx), qd = tc_q(idx), r = row & 31;
         const size_t o = ((size_t)c * C + r) * DV + j0 + 4 * qd;
         cv[it] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (idx < TC_CROWS * TC_VB / 4) {
@@ -1240,7 +1246,7 @@ __global__ void __launch_bounds__(NTH, 2)
       };
 #pragma unroll
       for (int it = 0; it < 2; ++it) {
-        const int idx = tid + it * NTH, o = tc_off(idx >> 2, idx & 3);
+        const int idx = tid + it * NTH, o = tc_off(tc_row(idx), tc_q(idx));
         put_hl(TC_SH + o, TC_SL + o, sv[it]);
         put_hl(TC_DH + o, TC_DL + o, dsv[it]);
         racc[it] = fmaf(dsv[it].x, sv[it].x, racc[it]);
@@ -1250,7 +1256,7 @@ __global__ void __launch_bounds__(NTH, 2)
       }
 #pragma unroll
       for (int it = 0; it < 3; ++it) {
-        const int idx = tid + it * NTH, o = tc_off(idx >> 2, idx & 3);
+        const int idx = tid + it * NTH, o = tc_off(tc_row(idx), tc_q(idx));
         if (idx < TC_CROWS * TC_VB / 4) put_hl(TC_CH + o, TC_CL + o, cv[it]);
       }
       tc::fence_proxy_async();  // the stores, visible to the tensor cores
@@ -1290,9 +1296,9 @@ __global__ void __launch_bounds__(NTH, 2)
 #pragma unroll
       for (int it = 0; it < 2; ++it) {
         float v = racc[it];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if ((tid & 3) == 0) rsum[(tid + it * NTH) >> 2] = v;
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if ((tid & 24) == 0) rsum[tc_row(tid + it * NTH)] = v;
       }
       for (int i = tid; i < DK; i += NTH) kcsum[i] = 0.f;
     }
