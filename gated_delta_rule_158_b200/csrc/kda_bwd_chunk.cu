@@ -540,11 +540,11 @@ struct FSmem {
 };
 
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(NTF, 1)
+__device__ __forceinline__ void
     bwd_fwd_scan(const Tin* __restrict__ k, const Tin* __restrict__ v,
                  const float* __restrict__ g, const float* __restrict__ beta,
                  const float* __restrict__ init, SeqMap map, float* __restrict__ ws,
-                 float* __restrict__ fin) {
+                 float* __restrict__ fin, int unit) {
   constexpr int LDK = FSmem<DK, DV>::LDK, LKC = FSmem<DK, DV>::LKC;
   constexpr int LDV = FSmem<DK, DV>::LDV, LDT = FSmem<DK, DV>::LDT;
   extern __shared__ float sm[];
@@ -561,7 +561,6 @@ __global__ void __launch_bounds__(NTF, 1)
 
   if (!seqs_ok(map)) return;
   const int H = map.H;
-  const int unit = blockIdx.x;
   const int h = unit % H;
   const UnitPos up = unit_pos(map, unit / H, h);
   if (!unit_in_bounds(map, up)) return;
@@ -761,12 +760,12 @@ struct ASmem {
 };
 
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(NTF, 1)
+__device__ __forceinline__ void
     bwd_state_grad_scan(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         const float* __restrict__ g, const float* __restrict__ beta,
                         const Tin* __restrict__ dout, const float* __restrict__ dfinal,
                         SeqMap map, float scale, float* __restrict__ dv,
-                        float* __restrict__ dinit, float* __restrict__ ws) {
+                        float* __restrict__ dinit, float* __restrict__ ws, int unit) {
   constexpr int LDK = ASmem<DK, DV>::LDK, LQT = ASmem<DK, DV>::LQT;
   constexpr int LDV = ASmem<DK, DV>::LDV, LDQ = ASmem<DK, DV>::LDQ;
   extern __shared__ float sm[];
@@ -785,7 +784,6 @@ __global__ void __launch_bounds__(NTF, 1)
 
   if (!seqs_ok(map)) return;
   const int H = map.H;
-  const int unit = blockIdx.x;
   const int h = unit % H;
   const UnitPos up = unit_pos(map, unit / H, h);
   if (!unit_in_bounds(map, up)) return;
@@ -994,6 +992,25 @@ __global__ void __launch_bounds__(NTF, 1)
 }
 
 // ===================================================================== pass B
+// F and A need only the key-side pass, not each other: one launch runs A's
+// units (blocks [0, na): the longer scan first) and then F's (blocks
+// [na, na + nf)), so F's CTAs fill the SMs that A's last, partial wave of
+// units leaves idle.
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(NTF, 1)
+    bwd_scans(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+              const float* __restrict__ g, const float* __restrict__ beta,
+              const Tin* __restrict__ dout, const float* __restrict__ init,
+              const float* __restrict__ dfinal, SeqMap map, float scale, int na,
+              float* __restrict__ dv, float* __restrict__ dinit, float* __restrict__ ws,
+              float* __restrict__ fin) {
+  const int b = (int)blockIdx.x;
+  if (b < na)
+    bwd_state_grad_scan<Tin, DK, DV>(q, k, g, beta, dout, dfinal, map, scale, dv, dinit, ws, b);
+  else
+    bwd_fwd_scan<Tin, DK, DV>(k, v, g, beta, init, map, ws, fin, b - na);
+}
+
 // B takes the dv columns 16 at a time, which keeps it at two CTAs per SM;
 // rows of 20 floats keep the tensor-core fragment loads free of bank conflicts
 constexpr int VBB = 16;
@@ -1684,13 +1701,8 @@ struct Passes {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)KSmem<DK>::bytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_fwd_scan<Tin, DK, DV>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)FSmem<DK, DV>::bytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_state_grad_scan<Tin, DK, DV>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)ASmem<DK, DV>::bytes);
+      e = cudaFuncSetAttribute(bwd_scans<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)std::max(FSmem<DK, DV>::bytes, ASmem<DK, DV>::bytes));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BSmem<DK>::bytes);
@@ -1704,20 +1716,20 @@ struct Passes {
         nseq, ws);
     return cudaGetLastError();
   }
-  // F: chunk-start states, R and U, one CTA per unit; fin (nullable) gets the end state
-  static cudaError_t F(const BwdArgs& a, const SeqMap& m, int units, const float* init,
-                       float* ws, float* fin, cudaStream_t st) {
-    bwd_fwd_scan<Tin, DK, DV><<<units, NTF, FSmem<DK, DV>::bytes, st>>>(
-        static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.g, a.beta, init, m, ws,
-        fin);
-    return cudaGetLastError();
-  }
-  // A: the state gradient in reverse chunk order from dfinal, writing dv and dinit
-  static cudaError_t A(const BwdArgs& a, const SeqMap& m, int units, const float* dfinal,
-                       float* dinit, float* ws, cudaStream_t st) {
-    bwd_state_grad_scan<Tin, DK, DV><<<units, NTF, ASmem<DK, DV>::bytes, st>>>(
-        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
-        static_cast<const Tin*>(a.dout), dfinal, m, a.scale, a.dv, dinit, ws);
+  // F (chunk-start states, R and U from init; fin, nullable, gets the end
+  // state) and / or A (the state gradient in reverse chunk order from dfinal,
+  // writing dv and dinit) in one launch, one CTA per unit each
+  static cudaError_t FA(const BwdArgs& a, const SeqMap& m, int units, bool run_f,
+                        const float* init, float* fin, bool run_a, const float* dfinal,
+                        float* dinit, float* ws, cudaStream_t st) {
+    const int na = run_a ? units : 0, nf = run_f ? units : 0;
+    if (na + nf == 0) return cudaSuccess;
+    const size_t smem = std::max(run_a ? ASmem<DK, DV>::bytes : (size_t)0,
+                                 run_f ? FSmem<DK, DV>::bytes : (size_t)0);
+    bwd_scans<Tin, DK, DV><<<na + nf, NTF, smem, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+        a.g, a.beta, static_cast<const Tin*>(a.dout), init, dfinal, m, a.scale, na, a.dv, dinit,
+        ws, fin);
     return cudaGetLastError();
   }
   // B: every chunk's token gradients, one CTA per (chunk, head)
@@ -1750,11 +1762,9 @@ struct Passes {
         if ((e = cudaGetLastError())) return e;
       }
       const int64_t blocks = lay.max_chunks * a.H;
-      if (a.T > 0) {
-        if ((e = K(a, map, nseq, blocks, ws, st))) return e;
-        if ((e = F(a, map, units, a.init, ws, nullptr, st))) return e;
-      }
-      if ((e = A(a, map, units, a.dfinal, a.dinit, ws, st))) return e;
+      if (a.T > 0 && (e = K(a, map, nseq, blocks, ws, st))) return e;
+      if ((e = FA(a, map, units, a.T > 0, a.init, nullptr, true, a.dfinal, a.dinit, ws, st)))
+        return e;
       if (lay.max_chunks == 0) return cudaSuccess;
       return Bp(a, map, nseq, blocks, ws, st);
     }
@@ -1772,15 +1782,16 @@ struct Passes {
     for (int w = 0; w + 1 < nw; ++w) {  // checkpoints: the start state of every later window
       const SeqMap m = window(w);
       if ((e = K(a, m, nseq, blocks_of(m), ws, st))) return e;
-      if ((e = F(a, m, units, start_state(w), ws, ck + w * state_floats, st))) return e;
+      if ((e = FA(a, m, units, true, start_state(w), ck + w * state_floats, false, nullptr, nullptr,
+                  ws, st)))
+        return e;
     }
     for (int w = nw - 1; w >= 0; --w) {
       const SeqMap m = window(w);
       if ((e = K(a, m, nseq, blocks_of(m), ws, st))) return e;
-      if ((e = F(a, m, units, start_state(w), ws, nullptr, st))) return e;
       const float* dfin = w == nw - 1 ? a.dfinal : ds + ((w + 1) & 1) * state_floats;
       float* dst = w == 0 ? a.dinit : ds + (w & 1) * state_floats;
-      if ((e = A(a, m, units, dfin, dst, ws, st))) return e;
+      if ((e = FA(a, m, units, true, start_state(w), nullptr, true, dfin, dst, ws, st))) return e;
       if ((e = Bp(a, m, nseq, blocks_of(m), ws, st))) return e;
     }
     return cudaSuccess;
