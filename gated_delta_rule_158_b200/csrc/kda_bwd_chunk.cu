@@ -1199,6 +1199,21 @@ __global__ void __launch_bounds__(NTH, 2)
     // and stores; the loads of block j are in flight while the MMAs of block
     // j - 1 run), thread 0 issues the block's 18 MMAs and commits them to the
     // stage's barrier, which frees the stage for block j + 2.
+    {  // the keys, X and L are read after the block loop: into L2 meanwhile
+      auto pf = [](const void* ptr) { asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr)); };
+      constexpr int QL = DK * (int)sizeof(Tin) / 128, GL = DK * 4 / 128;  // 128-byte lines per row
+      constexpr int RL = 2 * QL + GL;
+      for (int idx = tid; idx < C * RL; idx += NTH) {
+        const int r = idx / RL, l = idx % RL;
+        if (r < n) {
+          const size_t row = (rowbase + (size_t)r * H) * DK;
+          if (l < QL) pf(q + row + l * (128 / (int)sizeof(Tin)));
+          else if (l < 2 * QL) pf(k + row + (l - QL) * (128 / (int)sizeof(Tin)));
+          else pf(g + row + (l - 2 * QL) * 32);
+        }
+      }
+      if (tid < 2 * C) pf((tid < C ? w.X : w.L) + (size_t)c * C * C + (tid % C) * 32);
+    }
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BSmem<DK>::bar_off);  // 2 stages, drain
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 3);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -1551,7 +1566,16 @@ __global__ void __launch_bounds__(NTH, 2)
         p1[q2][e] = fmaf(ea, p1[q2][e], eb * p3[q2][e]);  // dk
         p2[q2][e] *= ea;                                   // dq
       }
-    add_out(16 * mt, [] { return true; });
+    // phase 1 adds to the same fragment elements: its dk, dq contributions
+    // join these in registers and one read-modify-write stores both
+    float d0k[NTW][4], d0q[NTW][4];
+#pragma unroll
+    for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        d0k[q2][e] = p1[q2][e];
+        d0q[q2][e] = p2[q2][e];
+      }
     __syncthreads();
     // phase 1: the pair (1, 0) around row 15 -- Kb' of rows 0..15 from ref 7
     // to 15, Ka' and Qa' of rows 16..31 from ref 23 to 15 (factors <= 1)
@@ -1607,9 +1631,12 @@ __global__ void __launch_bounds__(NTH, 2)
           const float eb = expf(-d);
           aG[r * LDK + i] -= KbS[r * LDK + i] * p3[q2][e];
           p1[q2][e] = eb * p3[q2][e];  // dk (no dq term)
+          p2[q2][e] = 0.f;
         }
+        p1[q2][e] += d0k[q2][e];
+        p2[q2][e] += d0q[q2][e];
       }
-    add_out(16 * mt, [&] { return mt == 1; });
+    add_out(16 * mt, [] { return true; });
   } else {
     // exponentials of differences, by element owner: thread of channel i owns
     // rows r = part, part + P, ... (row side), then columns (column side)
