@@ -1213,6 +1213,19 @@ __global__ void __launch_bounds__(NTH, 2)
         }
       }
       if (tid < 2 * C) pf((tid < C ? w.X : w.L) + (size_t)c * C * C + (tid % C) * 32);
+      // and the chunk's saved states and C x dv tiles, read block by block
+      const int sl = DK * DV / 32, cl = C * DV / 32;  // 128-byte lines
+      for (int idx = tid; idx < 2 * sl + 4 * cl; idx += NTH) {
+        const float* p = idx < sl       ? w.S + (size_t)c * DK * DV + (size_t)idx * 32
+                         : idx < 2 * sl ? w.dS + (size_t)c * DK * DV + (size_t)(idx - sl) * 32
+                                        : nullptr;
+        if (p == nullptr) {
+          const int j = idx - 2 * sl, t = j / cl, o = j % cl;
+          const float* base = t == 0 ? w.R : t == 1 ? w.U : t == 2 ? w.dU : w.W;
+          p = base + (size_t)c * C * DV + (size_t)o * 32;
+        }
+        pf(p);
+      }
     }
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BSmem<DK>::bar_off);  // 2 stages, drain
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 3);
