@@ -294,6 +294,17 @@ __device__ __forceinline__ void copy_tile_out(float* __restrict__ dst, const flo
   }
 }
 
+// L2 prefetch (a hint: no registers, nothing waits on it) of rows 0 .. nr-1
+// of a row slice, row r at base + r stride, W elements each, NT threads.
+template <int NT, typename T>
+__device__ __forceinline__ void prefetch_rows(const T* base, size_t stride, int nr, int W) {
+  const int lines = (W * (int)sizeof(T) + 127) / 128, per = 128 / (int)sizeof(T);
+  for (int idx = threadIdx.x; idx < nr * lines; idx += NT) {
+    const int r = idx / lines, l = idx % lines;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (size_t)r * stride + (size_t)l * per));
+  }
+}
+
 // chunk inputs of one (sequence, head): rows t0 .. t0 + n - 1, zero-padded to
 // C, into [C][LDK] tiles
 // g is the log-decay, or z when A_log is not null (the gate
@@ -607,6 +618,14 @@ __device__ __forceinline__ void
         vv[it] = idx < C * V4 && r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + j) : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c + 1 < nc) {  // the next chunk's inputs into L2 while this one runs
+        const int n1 = min(C, up.len - t0 - C);
+        const size_t rb1 = rowbase + (size_t)C * H;
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(v + rb1 * DV, (size_t)H * DV, n1, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c + 1) * C * C, 0, 1, C * C);
+      }
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
         const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
@@ -834,6 +853,15 @@ __device__ __forceinline__ void
                      : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c > 0) {  // the previous chunk's (next in this order) inputs into L2
+        const size_t rb1 = rowbase - (size_t)C * H;
+        prefetch_rows<NTF>(q + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(dout + rb1 * DV, (size_t)H * DV, C, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c - 1) * C * C, 0, 1, C * C);
+        prefetch_rows<NTF>(w.Aqk + (size_t)(c - 1) * C * C, 0, 1, C * C);
+      }
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
         const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
@@ -1942,6 +1970,16 @@ __global__ void __launch_bounds__(NTF, 1)
         vv[it] = idx < C * V4 && r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + j) : z4;
       }
       const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c + 1 < nc) {  // the next chunk's inputs into L2 while this one runs
+        const int n1 = min(C, up.len - t0 - C);
+        const size_t rb1 = rowbase + (size_t)C * H;
+        prefetch_rows<NTF>(q + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(v + rb1 * DV, (size_t)H * DV, n1, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c + 1) * C * C, 0, 1, C * C);
+        prefetch_rows<NTF>(w.Aqk + (size_t)(c + 1) * C * C, 0, 1, C * C);
+      }
 #pragma unroll
       for (int it = 0; it < IK; ++it) {
         const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
