@@ -414,7 +414,7 @@ struct KSmem {
   // read by the m16n8k8 fragment loads without bank conflicts
   static constexpr int LDK = DK + 4;
   static constexpr int floats = 5 * C * LDK       // q (then q factor), k, Gamma, two factors
-                                + 3 * C * LDC     // L, A_qk, X
+                                + 2 * C * LDC     // L, A_qk (X stays in registers)
                                 + C;              // beta
   static constexpr size_t bytes = sizeof(float) * floats;
 };
@@ -435,8 +435,7 @@ __global__ void __launch_bounds__(NTH, 2)
   float* FbS = FaS + C * LDK;     // [C][LDK]  k e^{Gamma_15 - Gamma}
   float* LS = FbS + C * LDK;      // [C][LDC]
   float* AqS = LS + C * LDC;      // [C][LDC]
-  float* XS = AqS + C * LDC;      // [C][LDC]
-  float* bS = XS + C * LDC;       // [C]
+  float* bS = AqS + C * LDC;      // [C]
 
   if (!seqs_ok(map)) return;
   const int H = map.H;
@@ -505,29 +504,34 @@ __global__ void __launch_bounds__(NTH, 2)
     }
   }
   __syncthreads();
-  // X = (I + Diag(beta) L)^-1 by forward substitution; the columns are
-  // independent, so warp w takes columns 4w .. 4w+3 with 8 lanes per column
-  {
-    const int lane = tid & 31, cc = 4 * (tid >> 5) + (lane >> 3), sub = lane & 7;
-    for (int r = sub; r < C; r += 8) XS[r * LDC + cc] = r == cc ? 1.f : 0.f;
-    __syncwarp();
+  // X = (I + Diag(beta) L)^-1 by forward substitution: lane cc of warp 0
+  // holds column cc in registers (x_s = 0 above the diagonal, x_cc = 1) and
+  // forms x_r = -beta_r sum_{s<r} L_rs x_s (L_rs read as broadcasts) while
+  // the other warps store A_qk and L
+  if (tid < 32) {
+    const int cc = tid;
+    float x[C];
+#pragma unroll
+    for (int s2 = 0; s2 < C; ++s2) x[s2] = s2 == cc ? 1.f : 0.f;
+#pragma unroll
     for (int r = 1; r < C; ++r) {
-      float acc = 0.f;
-      for (int s2 = cc + sub; s2 < r; s2 += 8) acc = fmaf(LS[r * LDC + s2], XS[s2 * LDC + cc], acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      if (sub == 0 && r > cc) XS[r * LDC + cc] = -bS[r] * acc;
-      __syncwarp();
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < r; ++s2) {
+        if (s2 & 1) a1 = fmaf(LS[r * LDC + s2], x[s2], a1);
+        else a0 = fmaf(LS[r * LDC + s2], x[s2], a0);
+      }
+      if (r > cc) x[r] = -bS[r] * (a0 + a1);
     }
-  }
-  __syncthreads();
-  for (int idx = tid; idx < C * C; idx += NTH) {
-    const int r = idx / C, s2 = idx % C;
-    const size_t o = ((size_t)c * C + r) * C + s2;
-    w.X[o] = XS[r * LDC + s2];
-    w.Aqk[o] = AqS[r * LDC + s2];
-    w.L[o] = LS[r * LDC + s2];
+#pragma unroll
+    for (int r = 0; r < C; ++r) w.X[((size_t)c * C + r) * C + cc] = x[r];
+  } else {
+    for (int idx = tid - 32; idx < C * C; idx += NTH - 32) {
+      const int r = idx / C, s2 = idx % C;
+      const size_t o = ((size_t)c * C + r) * C + s2;
+      w.Aqk[o] = AqS[r * LDC + s2];
+      w.L[o] = LS[r * LDC + s2];
+    }
   }
 }
 
