@@ -96,8 +96,8 @@ CHUNK_TRAFFIC = {
     "headers": ["gated_delta_rule_158_b200/csrc/kda_sync.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_tc_ptx.cuh",
                 "gated_delta_rule_158_b200/csrc/kda_internal.cuh"],
-    "sha256": "8a05c507432424c7366a5b0fd3a8c1621893ebaf761e27b0fb20e9d7f844415f",
-    "bytes_per_unit_T4096": (673.474560e6 + 123.213312e6) / 128,
+    "sha256": "efbf25df15e88cb84589ea19899855a0296fe8561a4a80db777c9b6b8b91a649",
+    "bytes_per_unit_T4096": (673.389824e6 + 122.219776e6) / 128,
 }
 
 
