@@ -75,6 +75,7 @@ CASES = [
     (2, 97, 2, 64, 32, torch.bfloat16, True, True, 0.5),
     (1, 200, 2, 32, 128, torch.float32, False, True, 1.0),
     (1, 130, 2, 128, 64, torch.bfloat16, True, False, 0.125),
+    (1, 70, 2, 128, 32, torch.float32, True, True, 1.0),    # dk 128, two 16-column dv blocks
     (3, 1, 2, 32, 32, torch.float32, True, True, 1.0),       # one token
     (1, 129, 1, 64, 64, torch.float32, True, True, 1.0),     # one token past two blocks
 ]
@@ -223,14 +224,16 @@ def test_gated_training_backward_chain(oracle_mod):
     assert rel_l2(to64(dA), rA) <= TOL_F32
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_backward_varlen_parity(oracle_mod, dtype):
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 64),
+                                     (torch.bfloat16, 128)])
+def test_backward_varlen_parity(oracle_mod, dtype, d):
     """A packed batch (cu_seqlens) with empty, one-token, ragged and
     whole-chunk sequences: each sequence's gradients and dS0 against the
     oracle run on that sequence alone; an empty sequence passes d_final
-    through to d_init."""
+    through to d_init.  d = 128 takes the tensor-core products (tcgen05 in
+    the token-gradient pass)."""
     lengths = [0, 1, 31, 32, 33, 100, 64, 7, 0, 45]
-    N, H, dk, dv = len(lengths), 2, 64, 64
+    N, H, dk, dv = len(lengths), 2, d, d
     cu_list = W.cu_seqlens_from_lengths(lengths)
     T = cu_list[-1]
     cu = torch.tensor(cu_list, dtype=torch.int32, device=DEV)
@@ -290,12 +293,14 @@ def test_backward_varlen_bad_offsets_are_reported():
 
 # ------------------------------------------------- long sequences (windowed)
 
-def test_backward_windowed_matches_oracle(oracle_mod):
+@pytest.mark.parametrize("d,H", [(64, 2), (128, 1)])
+def test_backward_windowed_matches_oracle(oracle_mod, d, H):
     """T = 20000 > 8192: the bounded-workspace schedule (windows of 8192
     tokens, the last ragged, start states checkpointed, the state gradient
     handed from window to window) against the oracle, with an initial state, a
-    final-state gradient and a scale; every gradient element at the fp32 bar."""
-    B, T, H, d = 1, 20000, 2, 64
+    final-state gradient and a scale; every gradient element at the fp32 bar.
+    d = 128 takes the tensor-core products."""
+    B, T = 1, 20000
     assert kda.kda_recurrent_bwd_workspace_size(B, T, H, d, d) < \
         kda.kda_recurrent_bwd_workspace_size(B, 8192, H, d, d) * 1.1
     inp = W.make_prefill_inputs(B, T, H, d, d, torch.bfloat16, seed=301, device=DEV,
