@@ -1738,6 +1738,339 @@ __global__ void __launch_bounds__(NTH, 2)
   }
 }
 
+// ======================================================= pass F on tcgen05
+// dk = dv = 128.  The transposed state S^T (TMEM lane j = dv column, column
+// i = dk channel) is the fp32 accumulator of the update, and its high and
+// low tf32 parts sit beside it as the A operand of R (tcgen05.mma reads A
+// from TMEM); per chunk, three MMA groups, each operand split in two
+// (D += a_lo b_hi + a_hi b_lo + a_hi b_hi: fp32 accuracy):
+//   D_R = S^T Ka^T           (M 128 = j, N 32 = r, K 128 = i), R^T = V^T - D_R
+//   D_U = R^T T^T            (N 32 = r, K 32 = r'),            U^T = D_U
+//   S^T += U^T Kc            (N 128 = i, K 32 = r), S^T decayed by e^{Gamma_C} first
+// Between the groups the threads read the results out lane = j (the stores
+// of S, R and U to the workspace are coalesced rows) and write the high and
+// low parts back.  Ka, Kc^T and T are K-major shared tiles without swizzle.
+// TMEM columns: S^T 0..127, its parts 128..383, D_R / R_hi 384..415, R_lo
+// 416..447, D_U / U_hi 448..479, U_lo 480..511 (the whole TMEM: one CTA per SM).
+constexpr uint32_t FT_S = 0, FT_SH = 128, FT_SL = 256, FT_RD = 384, FT_RL = 416, FT_UD = 448,
+                   FT_UL = 480, FT_COLS = 512;
+constexpr int32_t kDetailFwdTc = 0xB420;  // timeout detail: F's MMA barriers
+// float offset of element (row, k) of a K-major tile without swizzle whose
+// rows hold K elements: core matrices of 8 rows x 4 elements (128 bytes)
+// consecutive along K (LBO 128 bytes), 8-row groups K * 32 bytes apart (SBO)
+template <int K>
+__device__ __forceinline__ int kmaj(int row, int k) {
+  return (row >> 3) * (K * 8) + (k >> 2) * 32 + (row & 7) * 4 + (k & 3);
+}
+__device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+  tc::tmem_st16(taddr, v);
+  tc::tmem_st16(taddr + 16, v + 16);
+}
+
+struct FtcSmem {
+  static constexpr int LK = 128 + 4;  // k, Gamma rows (4 mod 32)
+  static constexpr int kS = 0, GS = kS + C * LK, VS = GS + C * LK;
+  static constexpr int KaH = VS + C * 128, KaL = KaH + C * 128;
+  static constexpr int KcH = KaL + C * 128, KcL = KcH + 128 * C;
+  static constexpr int TH = KcL + 128 * C, TL = TH + C * C;
+  static constexpr int bS = TL + C * C, gC = bS + C, eC = gC + 128;
+  static constexpr int bar_off = eC + 128;  // 4 mbarriers, TMEM address, abort flag
+  static constexpr int floats = bar_off + 16;
+  static constexpr size_t bytes = sizeof(float) * floats;
+  static_assert(KaH % 32 == 0 && KcH % 32 == 0 && TH % 32 == 0, "128-byte aligned operand tiles");
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(NTF, 1)
+    bwd_fwd_scan_tc(const Tin* __restrict__ k, const Tin* __restrict__ v,
+                    const float* __restrict__ g, const float* __restrict__ beta,
+                    const float* __restrict__ init, SeqMap map, float* __restrict__ ws,
+                    float* __restrict__ fin) {
+  constexpr int DK = 128, DV = 128, LK = FtcSmem::LK;
+  extern __shared__ __align__(1024) float sm[];
+  float* kS = sm + FtcSmem::kS;  // [C][LK] k
+  float* GS = sm + FtcSmem::GS;  // [C][LK] Gamma
+  float* VS = sm + FtcSmem::VS;  // [C][DV] v
+  float* bS = sm + FtcSmem::bS;
+  float* gC = sm + FtcSmem::gC;
+  float* eC = sm + FtcSmem::eC;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + FtcSmem::bar_off);  // R, U, S, drain
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  const int unit = blockIdx.x;
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
+  const int nc = up.nc;
+  const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  StatusBlock* sbw = const_cast<StatusBlock*>(map.sb);
+  // this thread's TMEM lane (a dv column j) and its block of columns
+  const int j = 32 * (warp & 3) + lane, blk = warp >> 2;
+  const uint32_t lrow = (uint32_t)(32 * (warp & 3)) << 16;
+  if (nc == 0) {  // no chunks: the end state is the initial one
+    if (fin)
+      for (int idx = tid; idx < DK * DV; idx += NTF)
+        fin[(size_t)unit * DK * DV + idx] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
+    return;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, FT_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+  const uint32_t sbase = smem_u32(sm);
+  const uint64_t dKaH = tc::plain_desc(sbase + 4u * FtcSmem::KaH, 128, 128 * 8 * 4);
+  const uint64_t dKaL = tc::plain_desc(sbase + 4u * FtcSmem::KaL, 128, 128 * 8 * 4);
+  const uint64_t dTH = tc::plain_desc(sbase + 4u * FtcSmem::TH, 128, C * 8 * 4);
+  const uint64_t dTL = tc::plain_desc(sbase + 4u * FtcSmem::TL, 128, C * 8 * 4);
+  const uint64_t dKcH = tc::plain_desc(sbase + 4u * FtcSmem::KcH, 128, C * 8 * 4);
+  const uint64_t dKcL = tc::plain_desc(sbase + 4u * FtcSmem::KcL, 128, C * 8 * 4);
+  auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
+    uint32_t hi, lo;
+    split_tf32(x, hi, lo);
+    reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
+    reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
+  };
+  bool bad = false;
+  for (int c = 0; c < nc; ++c) {
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+    // ---- the chunk's rows (k, Gamma's increments, v), four elements per load
+    {
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = C * K4 / NTF, IV = C * V4 / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 kv[IK], gv[IK], vv[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        kv[it] = gv[it] = z4;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        vv[it] = r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + jj) : z4;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c + 1 < nc) {  // the next chunk's inputs into L2 while this one runs
+        const int n1 = min(C, up.len - t0 - C);
+        const size_t rb1 = rowbase + (size_t)C * H;
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(v + rb1 * DV, (size_t)H * DV, n1, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c + 1) * C * C, 0, 1, C * C);
+      }
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        st4(kS + r * LK + i, kv[it]);
+        st4(GS + r * LK + i, gv[it]);
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        st4(VS + r * DV + jj, vv[it]);
+      }
+      if (tid < C) bS[tid] = bv;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LK + i];
+        GS[r * LK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+    }
+    __syncthreads();
+    // ---- Ka = k e^Gamma ([r][i], K-major) and T = X Diag(beta) ([r][r']):
+    // their last readers (this unit's previous R and U groups) have completed
+    // (one core matrix of 8 rows x 4 elements per warp instruction)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {  // Ka: 4 row groups x 32 k groups
+      const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
+      const int r = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3);
+      put_hl(FtcSmem::KaH, FtcSmem::KaL, kmaj<DK>(r, i), kS[r * LK + i] * expf(GS[r * LK + i]));
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // T: 4 row groups x 8 k groups
+      const int cm = warp + 16 * t, rg = cm >> 3, kg = cm & 7;
+      const int r = 8 * rg + (lane >> 2), s2 = 4 * kg + (lane & 3);
+      put_hl(FtcSmem::TH, FtcSmem::TL, kmaj<C>(r, s2),
+             w.X[((size_t)c * C + r) * C + s2] * bS[s2]);
+    }
+    // ---- the previous chunk's state update has landed: Kc^T, then S
+    if (c > 0) bad |= !mbar_wait_bounded(&bars[2], (c - 1) & 1, abort_flag, sbw, kDetailFwdTc);
+    tc::fence_after_sync();
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {  // Kc^T ([i][r], K-major): 16 row groups x 8 k groups
+      const int cm = warp + 16 * t, ig = cm >> 3, rg2 = cm & 7;
+      const int i = 8 * ig + (lane >> 2), r = 4 * rg2 + (lane & 3);
+      put_hl(FtcSmem::KcH, FtcSmem::KcL, kmaj<C>(i, r),
+             kS[r * LK + i] * expf(gC[i] - GS[r * LK + i]));
+    }
+    {  // S^T columns 32 blk .. 32 blk + 31 of lane j: the chunk-start state to the
+       // workspace, its tf32 parts to TMEM, then decayed by e^{Gamma_C}
+      float sv[32];
+      const int i0 = 32 * blk;
+      if (c == 0) {
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii)
+          sv[ii] = init ? init[((size_t)unit * DK + i0 + ii) * DV + j] : 0.f;
+      } else {
+        tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+      }
+      uint32_t hv[32], lv[32];
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) {
+        w.S[((size_t)c * DK + i0 + ii) * DV + j] = sv[ii];
+        split_tf32(sv[ii], hv[ii], lv[ii]);
+      }
+      tmem_st32u(tbase + lrow + FT_SH + i0, hv);
+      tmem_st32u(tbase + lrow + FT_SL + i0, lv);
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) sv[ii] *= eC[i0 + ii];
+      tc::tmem_st32(tbase + lrow + FT_S + i0, sv);
+      tc::wait_st();
+    }
+    tc::fence_proxy_async();  // Ka, T, Kc^T visible to the tensor cores
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    constexpr uint32_t id32 = tc::idesc(tc::kFmtTF32, 128, 32, false, false, false);
+    constexpr uint32_t id128 = tc::idesc(tc::kFmtTF32, 128, 128, false, false, false);
+    if (tid == 0) {  // D_R = S^T Ka^T
+      tc::fence_after_sync();
+#pragma unroll 1
+      for (int ks = 0; ks < DK / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + FT_RD, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
+                          (term == 1 ? dKaL : dKaH) + (uint64_t)(16 * ks), id32,
+                          (ks > 0 || term > 0) ? 1u : 0u);
+      tc::mma_commit(&bars[0]);
+    }
+    bad |= !mbar_wait_bounded(&bars[0], c & 1, abort_flag, sbw, kDetailFwdTc);
+    tc::fence_after_sync();
+    {  // R = V - D_R^T, rows 8 blk .. 8 blk + 7 of column j: to the workspace, and
+       // its tf32 parts back (the high part over D_R)
+      const int r0 = 8 * blk;
+      float dr[8];
+      tmem_ld8_wait(tbase + lrow + FT_RD + r0, dr);
+      uint32_t hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const float x = VS[(r0 + rr) * DV + j] - dr[rr];
+        w.R[((size_t)c * C + r0 + rr) * DV + j] = x;
+        split_tf32(x, hv[rr], lv[rr]);
+      }
+      tmem_st8(tbase + lrow + FT_RD + r0, hv);
+      tmem_st8(tbase + lrow + FT_RL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // D_U = R^T T^T
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + FT_UD, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
+                          (term == 1 ? dTL : dTH) + (uint64_t)(16 * ks), id32,
+                          (ks > 0 || term > 0) ? 1u : 0u);
+      tc::mma_commit(&bars[1]);
+    }
+    bad |= !mbar_wait_bounded(&bars[1], c & 1, abort_flag, sbw, kDetailFwdTc);
+    tc::fence_after_sync();
+    {  // U rows 8 blk .. 8 blk + 7 of column j: to the workspace and split
+      const int r0 = 8 * blk;
+      float du[8];
+      tmem_ld8_wait(tbase + lrow + FT_UD + r0, du);
+      uint32_t hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        w.U[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
+        split_tf32(du[rr], hv[rr], lv[rr]);
+      }
+      tmem_st8(tbase + lrow + FT_UD + r0, hv);
+      tmem_st8(tbase + lrow + FT_UL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // S^T += U^T Kc
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + FT_S, tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
+                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id128, 1u);
+      tc::mma_commit(&bars[2]);
+    }
+  }
+  // every MMA issued has landed before TMEM is read or released
+  if (tid == 0) tc::mma_commit(&bars[3]);
+  if (!mbar_wait_bounded(&bars[3], 0, abort_flag, sbw, kDetailFwdTc)) mbar_wait_drain(&bars[3], 0);
+  tc::fence_after_sync();
+  if (fin && !bad) {  // the state after the last chunk (a window's end state)
+    float sv[32];
+    const int i0 = 32 * blk;
+    tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+#pragma unroll
+    for (int ii = 0; ii < 32; ++ii) fin[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii];
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, FT_COLS);
+}
+
 // Dense batches longer than this run in windows of this many tokens (whole
 // chunks) so that the workspace holds one window's chunks, not the sequence's:
 // a first pass of K and F over the windows in order keeps only each window's
@@ -1779,6 +2112,9 @@ struct Passes {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_scans<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)std::max(FSmem<DK, DV>::bytes, ASmem<DK, DV>::bytes));
+    if (e == cudaSuccess && kTcF)
+      e = cudaFuncSetAttribute(bwd_fwd_scan_tc<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)FtcSmem::bytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BSmem<DK>::bytes);
@@ -1795,9 +2131,20 @@ struct Passes {
   // F (chunk-start states, R and U from init; fin, nullable, gets the end
   // state) and / or A (the state gradient in reverse chunk order from dfinal,
   // writing dv and dinit) in one launch, one CTA per unit each
+  // at dk = dv = 128 F runs on tcgen05, in a launch of its own (it takes the
+  // whole TMEM of an SM)
+  static constexpr bool kTcF = DK == 128 && DV == 128;
   static cudaError_t FA(const BwdArgs& a, const SeqMap& m, int units, bool run_f,
                         const float* init, float* fin, bool run_a, const float* dfinal,
                         float* dinit, float* ws, cudaStream_t st) {
+    if (kTcF && run_f && units > 0) {
+      bwd_fwd_scan_tc<Tin><<<units, NTF, FtcSmem::bytes, st>>>(
+          static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.g, a.beta, init, m, ws,
+          fin);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      run_f = false;
+    }
     const int na = run_a ? units : 0, nf = run_f ? units : 0;
     if (na + nf == 0) return cudaSuccess;
     const size_t smem = std::max(run_a ? ASmem<DK, DV>::bytes : (size_t)0,
