@@ -1754,7 +1754,8 @@ __global__ void __launch_bounds__(NTH, 2)
 // 416..447, D_U / U_hi 448..479, U_lo 480..511 (the whole TMEM: one CTA per SM).
 constexpr uint32_t FT_S = 0, FT_SH = 128, FT_SL = 256, FT_RD = 384, FT_RL = 416, FT_UD = 448,
                    FT_UL = 480, FT_COLS = 512;
-constexpr int32_t kDetailFwdTc = 0xB420;  // timeout detail: F's MMA barriers
+constexpr int32_t kDetailFwdTc = 0xB420;   // timeout detail: F's MMA barriers
+constexpr int32_t kDetailGradTc = 0xB421;  // timeout detail: A's MMA barriers
 // float offset of element (row, k) of a K-major tile without swizzle whose
 // rows hold K elements: core matrices of 8 rows x 4 elements (128 bytes)
 // consecutive along K (LBO 128 bytes), 8-row groups K * 32 bytes apart (SBO)
@@ -2071,6 +2072,326 @@ __global__ void __launch_bounds__(NTF, 1)
   if (warp == 0) tc::tmem_dealloc(tbase, FT_COLS);
 }
 
+// ======================================================= pass A on tcgen05
+// dk = dv = 128, reverse chunk order.  The transposed state gradient dS^T
+// (TMEM lane j, column i) is the fp32 accumulator, its tf32 parts beside it;
+// per chunk, with every operand split in two:
+//   D_dU = dO'^T A_qk + dS^T Kc^T       (N 32 = r; K 32 = s, then 128 = i)
+//   D_W  = dU^T T                       (N 32 = r, K 32 = r')
+//   dS^T = e^{Gamma_C} dS^T + dO'^T Qg - W^T Ka   (N 128 = i, K 32 = r)
+// dO'^T is a shared K-major tile (the A operand of two groups), dS^T, dU^T
+// and W^T come from TMEM.  TMEM columns as in F's kernel: dS^T 0..127, its
+// parts 128..383, D_dU / dU_hi 384..415, dU_lo 416..447, D_W / W_hi
+// 448..479, W_lo 480..511.
+struct AtcSmem {
+  static constexpr int LK = 128 + 4, LO = 128 + 8;  // q, k, Gamma rows; dO' rows (8 mod 32)
+  static constexpr int qS = 0, kS = qS + C * LK, GS = kS + C * LK, dOS = GS + C * LK;
+  static constexpr int AqH = dOS + C * LO, AqL = AqH + C * C;        // [r][s]: A_qk^T
+  static constexpr int KcH = AqL + C * C, KcL = KcH + C * 128;       // [r][i]: Kc
+  static constexpr int TtH = KcL + C * 128, TtL = TtH + C * C;       // [r][r']: T^T
+  static constexpr int QgH = TtL + C * C, QgL = QgH + 128 * C;       // [i][r]: Qg^T
+  static constexpr int KaH = QgL + 128 * C, KaL = KaH + 128 * C;     // [i][r]: -Ka^T
+  static constexpr int OtH = KaL + 128 * C, OtL = OtH + 128 * C;     // [j][s]: dO'^T
+  static constexpr int bS = OtL + 128 * C, gC = bS + C, eC = gC + 128;
+  static constexpr int bar_off = eC + 128;  // 4 mbarriers, TMEM address, abort flag
+  static constexpr int floats = bar_off + 16;
+  static constexpr size_t bytes = sizeof(float) * floats;
+  static_assert(AqH % 32 == 0 && KcH % 32 == 0 && TtH % 32 == 0 && QgH % 32 == 0 &&
+                    KaH % 32 == 0 && OtH % 32 == 0, "128-byte aligned operand tiles");
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(NTF, 1)
+    bwd_state_grad_scan_tc(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                           const float* __restrict__ g, const float* __restrict__ beta,
+                           const Tin* __restrict__ dout, const float* __restrict__ dfinal,
+                           SeqMap map, float scale, float* __restrict__ dv,
+                           float* __restrict__ dinit, float* __restrict__ ws) {
+  constexpr int DK = 128, DV = 128, LK = AtcSmem::LK, LO = AtcSmem::LO;
+  extern __shared__ __align__(1024) float sm[];
+  float* qS = sm + AtcSmem::qS;    // [C][LK] q
+  float* kS = sm + AtcSmem::kS;    // [C][LK] k
+  float* GS = sm + AtcSmem::GS;    // [C][LK] Gamma
+  float* dOS = sm + AtcSmem::dOS;  // [C][LO] scale dO
+  float* bS = sm + AtcSmem::bS;
+  float* gC = sm + AtcSmem::gC;
+  float* eC = sm + AtcSmem::eC;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + AtcSmem::bar_off);  // dU, W, dS, drain
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  const int unit = blockIdx.x;
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
+  const int nc = up.nc;
+  const UnitWs w = unit_ws(ws, up.chunk0, nc, DK, DV);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  StatusBlock* sbw = const_cast<StatusBlock*>(map.sb);
+  const int j = 32 * (warp & 3) + lane, blk = warp >> 2;
+  const uint32_t lrow = (uint32_t)(32 * (warp & 3)) << 16;
+  if (nc == 0) {  // no chunks: the gradient of the initial state is d_final
+    if (dinit)
+      for (int idx = tid; idx < DK * DV; idx += NTF)
+        dinit[(size_t)unit * DK * DV + idx] = dfinal ? dfinal[(size_t)unit * DK * DV + idx] : 0.f;
+    return;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, FT_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+  const uint32_t sbase = smem_u32(sm);
+  auto desc = [&](int tile, int K) { return tc::plain_desc(sbase + 4u * tile, 128, K * 8 * 4); };
+  const uint64_t dAqH = desc(AtcSmem::AqH, C), dAqL = desc(AtcSmem::AqL, C);
+  const uint64_t dKcH = desc(AtcSmem::KcH, DK), dKcL = desc(AtcSmem::KcL, DK);
+  const uint64_t dTtH = desc(AtcSmem::TtH, C), dTtL = desc(AtcSmem::TtL, C);
+  const uint64_t dQgH = desc(AtcSmem::QgH, C), dQgL = desc(AtcSmem::QgL, C);
+  const uint64_t dKaH = desc(AtcSmem::KaH, C), dKaL = desc(AtcSmem::KaL, C);
+  const uint64_t dOtH = desc(AtcSmem::OtH, C), dOtL = desc(AtcSmem::OtL, C);
+  auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
+    uint32_t hi, lo;
+    split_tf32(x, hi, lo);
+    reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
+    reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
+  };
+  constexpr uint32_t id32 = tc::idesc(tc::kFmtTF32, 128, 32, false, false, false);
+  constexpr uint32_t id128 = tc::idesc(tc::kFmtTF32, 128, 128, false, false, false);
+  bool bad = false;
+  int it_c = 0;  // chunks processed (barrier phases)
+  for (int c = nc - 1; c >= 0; --c, ++it_c) {
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+    // ---- the chunk's rows (q, k, Gamma's increments, scale dO)
+    {
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = C * K4 / NTF, IV = C * V4 / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 qv[IK], kv[IK], gv[IK], ov[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        qv[it] = kv[it] = gv[it] = z4;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          qv[it] = ld4(q + off);
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        ov[it] = r < n ? scale4(ld4(dout + (rowbase + (size_t)r * H) * DV + jj), scale) : z4;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c > 0) {  // the previous chunk's (next in this order) inputs into L2
+        const size_t rb1 = rowbase - (size_t)C * H;
+        prefetch_rows<NTF>(q + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, C, DK);
+        prefetch_rows<NTF>(dout + rb1 * DV, (size_t)H * DV, C, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c - 1) * C * C, 0, 1, C * C);
+        prefetch_rows<NTF>(w.Aqk + (size_t)(c - 1) * C * C, 0, 1, C * C);
+      }
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        st4(qS + r * LK + i, qv[it]);
+        st4(kS + r * LK + i, kv[it]);
+        st4(GS + r * LK + i, gv[it]);
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        st4(dOS + r * LO + jj, ov[it]);
+      }
+      if (tid < C) bS[tid] = bv;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LK + i];
+        GS[r * LK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+    }
+    __syncthreads();
+    // ---- operands of the dU and W groups (their last readers, the previous
+    // chunk's dU and W groups, have completed): A_qk^T, Kc, T^T
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // A_qk^T [r][s] and T^T [r][r']: 4 x 8 core matrices
+      const int cm = warp + 16 * t, rg = cm >> 3, kg = cm & 7;
+      const int r = 8 * rg + (lane >> 2), s2 = 4 * kg + (lane & 3);
+      const size_t o = ((size_t)c * C + s2) * C + r;
+      put_hl(AtcSmem::AqH, AtcSmem::AqL, kmaj<C>(r, s2), w.Aqk[o]);
+      put_hl(AtcSmem::TtH, AtcSmem::TtL, kmaj<C>(r, s2), w.X[o] * bS[r]);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {  // Kc [r][i]: 4 x 32 core matrices
+      const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
+      const int r = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3);
+      put_hl(AtcSmem::KcH, AtcSmem::KcL, kmaj<DK>(r, i),
+             kS[r * LK + i] * expf(gC[i] - GS[r * LK + i]));
+    }
+    // ---- the later chunk's state-gradient update has landed: Qg^T, -Ka^T,
+    // dO'^T, then dS
+    if (it_c > 0) bad |= !mbar_wait_bounded(&bars[2], (it_c - 1) & 1, abort_flag, sbw, kDetailGradTc);
+    tc::fence_after_sync();
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {  // Qg^T, -Ka^T [i][r] and dO'^T [j][s]: 16 x 8 core matrices
+      const int cm = warp + 16 * t, ig = cm >> 3, rg2 = cm & 7;
+      const int i = 8 * ig + (lane >> 2), r = 4 * rg2 + (lane & 3);
+      const float e = expf(GS[r * LK + i]);
+      const int o = kmaj<C>(i, r);
+      put_hl(AtcSmem::QgH, AtcSmem::QgL, o, qS[r * LK + i] * e);
+      put_hl(AtcSmem::KaH, AtcSmem::KaL, o, -(kS[r * LK + i] * e));
+      put_hl(AtcSmem::OtH, AtcSmem::OtL, o, dOS[r * LO + i]);  // row i is column j = i of dO'
+    }
+    {  // dS^T columns 32 blk .. 32 blk + 31 of lane j: to the workspace, its tf32
+       // parts to TMEM, then decayed by e^{Gamma_C}
+      float sv[32];
+      const int i0 = 32 * blk;
+      if (it_c == 0) {
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii)
+          sv[ii] = dfinal ? dfinal[((size_t)unit * DK + i0 + ii) * DV + j] : 0.f;
+      } else {
+        tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+      }
+      uint32_t hv[32], lv[32];
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) {
+        w.dS[((size_t)c * DK + i0 + ii) * DV + j] = sv[ii];
+        split_tf32(sv[ii], hv[ii], lv[ii]);
+      }
+      tmem_st32u(tbase + lrow + FT_SH + i0, hv);
+      tmem_st32u(tbase + lrow + FT_SL + i0, lv);
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) sv[ii] *= eC[i0 + ii];
+      tc::tmem_st32(tbase + lrow + FT_S + i0, sv);
+      tc::wait_st();
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // D_dU = dO'^T A_qk + dS^T Kc^T
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ss(tbase + FT_RD, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * ks),
+                     (term == 1 ? dAqL : dAqH) + (uint64_t)(16 * ks), id32, 1,
+                     (ks > 0 || term > 0) ? 1u : 0u);
+#pragma unroll 1
+      for (int ks = 0; ks < DK / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + FT_RD, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
+                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id32, 1u);
+      tc::mma_commit(&bars[0]);
+    }
+    bad |= !mbar_wait_bounded(&bars[0], it_c & 1, abort_flag, sbw, kDetailGradTc);
+    tc::fence_after_sync();
+    {  // dU rows 8 blk .. 8 blk + 7 of column j: to the workspace and split
+      const int r0 = 8 * blk;
+      float du[8];
+      tmem_ld8_wait(tbase + lrow + FT_RD + r0, du);
+      uint32_t hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        w.dU[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
+        split_tf32(du[rr], hv[rr], lv[rr]);
+      }
+      tmem_st8(tbase + lrow + FT_RD + r0, hv);
+      tmem_st8(tbase + lrow + FT_RL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // D_W = dU^T T
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + FT_UD, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
+                          (term == 1 ? dTtL : dTtH) + (uint64_t)(16 * ks), id32,
+                          (ks > 0 || term > 0) ? 1u : 0u);
+      tc::mma_commit(&bars[1]);
+    }
+    bad |= !mbar_wait_bounded(&bars[1], it_c & 1, abort_flag, sbw, kDetailGradTc);
+    tc::fence_after_sync();
+    {  // W (= dv) rows 8 blk .. 8 blk + 7 of column j: workspace, dv, split
+      const int r0 = 8 * blk;
+      float wv[8];
+      tmem_ld8_wait(tbase + lrow + FT_UD + r0, wv);
+      uint32_t hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = r0 + rr;
+        w.W[((size_t)c * C + r) * DV + j] = wv[rr];
+        if (r < n) dv[(rowbase + (size_t)r * H) * DV + j] = wv[rr];
+        split_tf32(wv[rr], hv[rr], lv[rr]);
+      }
+      tmem_st8(tbase + lrow + FT_UD + r0, hv);
+      tmem_st8(tbase + lrow + FT_UL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // dS^T += dO'^T Qg - W^T Ka
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+          tc::mma_ss(tbase + FT_S, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * ks),
+                     (term == 1 ? dQgL : dQgH) + (uint64_t)(16 * ks), id128, 1, 1u);
+          tc::mma_ts_tf32(tbase + FT_S, tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
+                          (term == 1 ? dKaL : dKaH) + (uint64_t)(16 * ks), id128, 1u);
+        }
+      tc::mma_commit(&bars[2]);
+    }
+  }
+  if (tid == 0) tc::mma_commit(&bars[3]);
+  if (!mbar_wait_bounded(&bars[3], 0, abort_flag, sbw, kDetailGradTc)) mbar_wait_drain(&bars[3], 0);
+  tc::fence_after_sync();
+  if (dinit && !bad) {
+    float sv[32];
+    const int i0 = 32 * blk;
+    tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+#pragma unroll
+    for (int ii = 0; ii < 32; ++ii) dinit[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii];
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, FT_COLS);
+}
+
 // Dense batches longer than this run in windows of this many tokens (whole
 // chunks) so that the workspace holds one window's chunks, not the sequence's:
 // a first pass of K and F over the windows in order keeps only each window's
@@ -2115,6 +2436,9 @@ struct Passes {
     if (e == cudaSuccess && kTcF)
       e = cudaFuncSetAttribute(bwd_fwd_scan_tc<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)FtcSmem::bytes);
+    if (e == cudaSuccess && kTcF)
+      e = cudaFuncSetAttribute(bwd_state_grad_scan_tc<Tin>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AtcSmem::bytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_chunk_grads<Tin, DK>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BSmem<DK>::bytes);
@@ -2131,8 +2455,8 @@ struct Passes {
   // F (chunk-start states, R and U from init; fin, nullable, gets the end
   // state) and / or A (the state gradient in reverse chunk order from dfinal,
   // writing dv and dinit) in one launch, one CTA per unit each
-  // at dk = dv = 128 F runs on tcgen05, in a launch of its own (it takes the
-  // whole TMEM of an SM)
+  // at dk = dv = 128 F and A run on tcgen05, each in a launch of its own (a
+  // CTA takes the whole TMEM of an SM)
   static constexpr bool kTcF = DK == 128 && DV == 128;
   static cudaError_t FA(const BwdArgs& a, const SeqMap& m, int units, bool run_f,
                         const float* init, float* fin, bool run_a, const float* dfinal,
@@ -2144,6 +2468,14 @@ struct Passes {
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       run_f = false;
+    }
+    if (kTcF && run_a && units > 0) {
+      bwd_state_grad_scan_tc<Tin><<<units, NTF, AtcSmem::bytes, st>>>(
+          static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), a.g, a.beta,
+          static_cast<const Tin*>(a.dout), dfinal, m, a.scale, a.dv, dinit, ws);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      run_a = false;
     }
     const int na = run_a ? units : 0, nf = run_f ? units : 0;
     if (na + nf == 0) return cudaSuccess;
