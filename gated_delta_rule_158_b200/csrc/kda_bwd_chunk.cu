@@ -1836,8 +1836,8 @@ __global__ void __launch_bounds__(NTF, 1)
         fin[(size_t)unit * DK * DV + idx] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
     return;
   }
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+  if (tid == 0) {  // arrivals: the issuing warps of each group (4, 2, 2) and of the drain (4)
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], (i == 0 || i == 3) ? 4 : 2);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -1955,8 +1955,12 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii)
           sv[ii] = init ? init[((size_t)unit * DK + i0 + ii) * DV + j] : 0.f;
-      } else {
+      } else {  // the update's two accumulators
+        float s2v[32];
         tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+        tmem_ld32_wait(tbase + lrow + FT_SH + i0, s2v);
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) sv[ii] += s2v[ii];
       }
       uint32_t hv[32], lv[32];
 #pragma unroll
@@ -1979,15 +1983,17 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     constexpr uint32_t id32 = tc::idesc(tc::kFmtTF32, 128, 32, false, false, false);
     constexpr uint32_t id128 = tc::idesc(tc::kFmtTF32, 128, 128, false, false, false);
-    if (tid == 0) {  // D_R = S^T Ka^T
+    if (lane == 0 && warp < 4) {  // D_R = S^T Ka^T: k-steps w, w + 4, ... issued by
+      // warp w into its own accumulator (the R and U columns, all free now)
       tc::fence_after_sync();
+      const uint32_t dst = tbase + (warp == 0 ? FT_RD : warp == 1 ? FT_RL : warp == 2 ? FT_UD : FT_UL);
 #pragma unroll 1
-      for (int ks = 0; ks < DK / 8; ++ks)
+      for (int ks = warp; ks < DK / 8; ks += 4)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
-          tc::mma_ts_tf32(tbase + FT_RD, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
+          tc::mma_ts_tf32(dst, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
                           (term == 1 ? dKaL : dKaH) + (uint64_t)(16 * ks), id32,
-                          (ks > 0 || term > 0) ? 1u : 0u);
+                          (ks > 3 || term > 0) ? 1u : 0u);
       tc::mma_commit(&bars[0]);
     }
     bad |= !mbar_wait_bounded(&bars[0], c & 1, abort_flag, sbw, kDetailFwdTc);
@@ -1995,12 +2001,15 @@ __global__ void __launch_bounds__(NTF, 1)
     {  // R = V - D_R^T, rows 8 blk .. 8 blk + 7 of column j: to the workspace, and
        // its tf32 parts back (the high part over D_R)
       const int r0 = 8 * blk;
-      float dr[8];
+      float dr[8], dr2[8], dr3[8], dr4[8];
       tmem_ld8_wait(tbase + lrow + FT_RD + r0, dr);
+      tmem_ld8_wait(tbase + lrow + FT_RL + r0, dr2);
+      tmem_ld8_wait(tbase + lrow + FT_UD + r0, dr3);
+      tmem_ld8_wait(tbase + lrow + FT_UL + r0, dr4);
       uint32_t hv[8], lv[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
-        const float x = VS[(r0 + rr) * DV + j] - dr[rr];
+        const float x = VS[(r0 + rr) * DV + j] - ((dr[rr] + dr2[rr]) + (dr3[rr] + dr4[rr]));
         w.R[((size_t)c * C + r0 + rr) * DV + j] = x;
         split_tf32(x, hv[rr], lv[rr]);
       }
@@ -2013,26 +2022,30 @@ __global__ void __launch_bounds__(NTF, 1)
       bad = true;
       break;
     }
-    if (tid == 0) {  // D_U = R^T T^T
+    if (lane == 0 && warp < 2) {  // D_U = R^T T^T: k-steps w, w + 2 by warp w into
+      // the U_hi (w = 0) or U_lo (w = 1) columns
       tc::fence_after_sync();
+      const uint32_t dst = tbase + (warp ? FT_UL : FT_UD);
 #pragma unroll
-      for (int ks = 0; ks < C / 8; ++ks)
+      for (int ks = warp; ks < C / 8; ks += 2)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
-          tc::mma_ts_tf32(tbase + FT_UD, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
+          tc::mma_ts_tf32(dst, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
                           (term == 1 ? dTL : dTH) + (uint64_t)(16 * ks), id32,
-                          (ks > 0 || term > 0) ? 1u : 0u);
+                          (ks > 1 || term > 0) ? 1u : 0u);
       tc::mma_commit(&bars[1]);
     }
     bad |= !mbar_wait_bounded(&bars[1], c & 1, abort_flag, sbw, kDetailFwdTc);
     tc::fence_after_sync();
     {  // U rows 8 blk .. 8 blk + 7 of column j: to the workspace and split
       const int r0 = 8 * blk;
-      float du[8];
+      float du[8], du2[8];
       tmem_ld8_wait(tbase + lrow + FT_UD + r0, du);
+      tmem_ld8_wait(tbase + lrow + FT_UL + r0, du2);
       uint32_t hv[8], lv[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
+        du[rr] += du2[rr];
         w.U[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
         split_tf32(du[rr], hv[rr], lv[rr]);
       }
@@ -2045,27 +2058,31 @@ __global__ void __launch_bounds__(NTF, 1)
       bad = true;
       break;
     }
-    if (tid == 0) {  // S^T += U^T Kc
+    if (lane == 0 && warp < 2) {  // S^T += U^T Kc: k-steps w, w + 2 by warp w, warp 0
+      // onto the decayed state, warp 1 into the S_hi columns (free now; the next
+      // read adds them)
       tc::fence_after_sync();
 #pragma unroll
-      for (int ks = 0; ks < C / 8; ++ks)
+      for (int ks = warp; ks < C / 8; ks += 2)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
-          tc::mma_ts_tf32(tbase + FT_S, tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
-                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id128, 1u);
+          tc::mma_ts_tf32(tbase + (warp ? FT_SH : FT_S), tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
+                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id128,
+                          (warp == 0 || ks > 1 || term > 0) ? 1u : 0u);
       tc::mma_commit(&bars[2]);
     }
   }
-  // every MMA issued has landed before TMEM is read or released
-  if (tid == 0) tc::mma_commit(&bars[3]);
+  // every MMA issued (by lane 0 of warps 0-3) has landed before TMEM is read or released
+  if (lane == 0 && warp < 4) tc::mma_commit(&bars[3]);
   if (!mbar_wait_bounded(&bars[3], 0, abort_flag, sbw, kDetailFwdTc)) mbar_wait_drain(&bars[3], 0);
   tc::fence_after_sync();
   if (fin && !bad) {  // the state after the last chunk (a window's end state)
-    float sv[32];
+    float sv[32], s2v[32];
     const int i0 = 32 * blk;
     tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+    tmem_ld32_wait(tbase + lrow + FT_SH + i0, s2v);
 #pragma unroll
-    for (int ii = 0; ii < 32; ++ii) fin[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii];
+    for (int ii = 0; ii < 32; ++ii) fin[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii] + s2v[ii];
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -2138,8 +2155,8 @@ __global__ void __launch_bounds__(NTF, 1)
         dinit[(size_t)unit * DK * DV + idx] = dfinal ? dfinal[(size_t)unit * DK * DV + idx] : 0.f;
     return;
   }
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+  if (tid == 0) {  // arrivals: the issuing warps of each group (4, 2, 2) and of the drain (4)
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], (i == 0 || i == 3) ? 4 : 2);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -2269,8 +2286,12 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii)
           sv[ii] = dfinal ? dfinal[((size_t)unit * DK + i0 + ii) * DV + j] : 0.f;
-      } else {
+      } else {  // the update's two accumulators
+        float s2v[32];
         tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+        tmem_ld32_wait(tbase + lrow + FT_SH + i0, s2v);
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) sv[ii] += s2v[ii];
       }
       uint32_t hv[32], lv[32];
 #pragma unroll
@@ -2291,20 +2312,20 @@ __global__ void __launch_bounds__(NTF, 1)
       bad = true;
       break;
     }
-    if (tid == 0) {  // D_dU = dO'^T A_qk + dS^T Kc^T
+    if (lane == 0 && warp < 4) {  // D_dU = dO'^T A_qk + dS^T Kc^T: warp w takes k-step
+      // w of the first part and w, w + 4, ... of the second, into its own
+      // accumulator (the dU and W columns, all free now)
       tc::fence_after_sync();
+      const uint32_t dst = tbase + (warp == 0 ? FT_RD : warp == 1 ? FT_RL : warp == 2 ? FT_UD : FT_UL);
 #pragma unroll
-      for (int ks = 0; ks < C / 8; ++ks)
-#pragma unroll
-        for (int term = 0; term < 3; ++term)
-          tc::mma_ss(tbase + FT_RD, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * ks),
-                     (term == 1 ? dAqL : dAqH) + (uint64_t)(16 * ks), id32, 1,
-                     (ks > 0 || term > 0) ? 1u : 0u);
+      for (int term = 0; term < 3; ++term)
+        tc::mma_ss(dst, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * warp),
+                   (term == 1 ? dAqL : dAqH) + (uint64_t)(16 * warp), id32, 1, term > 0 ? 1u : 0u);
 #pragma unroll 1
-      for (int ks = 0; ks < DK / 8; ++ks)
+      for (int ks = warp; ks < DK / 8; ks += 4)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
-          tc::mma_ts_tf32(tbase + FT_RD, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
+          tc::mma_ts_tf32(dst, tbase + (term == 0 ? FT_SL : FT_SH) + 8 * ks,
                           (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id32, 1u);
       tc::mma_commit(&bars[0]);
     }
@@ -2312,11 +2333,15 @@ __global__ void __launch_bounds__(NTF, 1)
     tc::fence_after_sync();
     {  // dU rows 8 blk .. 8 blk + 7 of column j: to the workspace and split
       const int r0 = 8 * blk;
-      float du[8];
+      float du[8], d2[8], d3[8], d4[8];
       tmem_ld8_wait(tbase + lrow + FT_RD + r0, du);
+      tmem_ld8_wait(tbase + lrow + FT_RL + r0, d2);
+      tmem_ld8_wait(tbase + lrow + FT_UD + r0, d3);
+      tmem_ld8_wait(tbase + lrow + FT_UL + r0, d4);
       uint32_t hv[8], lv[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
+        du[rr] = (du[rr] + d2[rr]) + (d3[rr] + d4[rr]);
         w.dU[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
         split_tf32(du[rr], hv[rr], lv[rr]);
       }
@@ -2329,27 +2354,31 @@ __global__ void __launch_bounds__(NTF, 1)
       bad = true;
       break;
     }
-    if (tid == 0) {  // D_W = dU^T T
+    if (lane == 0 && warp < 2) {  // D_W = dU^T T: k-steps w, w + 2 by warp w into the
+      // W_hi (w = 0) or W_lo (w = 1) columns
       tc::fence_after_sync();
+      const uint32_t dst = tbase + (warp ? FT_UL : FT_UD);
 #pragma unroll
-      for (int ks = 0; ks < C / 8; ++ks)
+      for (int ks = warp; ks < C / 8; ks += 2)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
-          tc::mma_ts_tf32(tbase + FT_UD, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
+          tc::mma_ts_tf32(dst, tbase + (term == 0 ? FT_RL : FT_RD) + 8 * ks,
                           (term == 1 ? dTtL : dTtH) + (uint64_t)(16 * ks), id32,
-                          (ks > 0 || term > 0) ? 1u : 0u);
+                          (ks > 1 || term > 0) ? 1u : 0u);
       tc::mma_commit(&bars[1]);
     }
     bad |= !mbar_wait_bounded(&bars[1], it_c & 1, abort_flag, sbw, kDetailGradTc);
     tc::fence_after_sync();
     {  // W (= dv) rows 8 blk .. 8 blk + 7 of column j: workspace, dv, split
       const int r0 = 8 * blk;
-      float wv[8];
+      float wv[8], w2[8];
       tmem_ld8_wait(tbase + lrow + FT_UD + r0, wv);
+      tmem_ld8_wait(tbase + lrow + FT_UL + r0, w2);
       uint32_t hv[8], lv[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
         const int r = r0 + rr;
+        wv[rr] += w2[rr];
         w.W[((size_t)c * C + r) * DV + j] = wv[rr];
         if (r < n) dv[(rowbase + (size_t)r * H) * DV + j] = wv[rr];
         split_tf32(wv[rr], hv[rr], lv[rr]);
@@ -2363,29 +2392,34 @@ __global__ void __launch_bounds__(NTF, 1)
       bad = true;
       break;
     }
-    if (tid == 0) {  // dS^T += dO'^T Qg - W^T Ka
+    if (lane == 0 && warp < 2) {  // dS^T += dO'^T Qg (warp 0, onto the decayed state)
+      // - W^T Ka (warp 1, into the dS_hi columns, free now; the next read adds them)
       tc::fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < C / 8; ++ks)
 #pragma unroll
         for (int term = 0; term < 3; ++term) {
-          tc::mma_ss(tbase + FT_S, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * ks),
-                     (term == 1 ? dQgL : dQgH) + (uint64_t)(16 * ks), id128, 1, 1u);
-          tc::mma_ts_tf32(tbase + FT_S, tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
-                          (term == 1 ? dKaL : dKaH) + (uint64_t)(16 * ks), id128, 1u);
+          if (warp == 0)
+            tc::mma_ss(tbase + FT_S, (term == 0 ? dOtL : dOtH) + (uint64_t)(16 * ks),
+                       (term == 1 ? dQgL : dQgH) + (uint64_t)(16 * ks), id128, 1, 1u);
+          else
+            tc::mma_ts_tf32(tbase + FT_SH, tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
+                            (term == 1 ? dKaL : dKaH) + (uint64_t)(16 * ks), id128,
+                            (ks > 0 || term > 0) ? 1u : 0u);
         }
       tc::mma_commit(&bars[2]);
     }
   }
-  if (tid == 0) tc::mma_commit(&bars[3]);
+  if (lane == 0 && warp < 4) tc::mma_commit(&bars[3]);  // every issuer's MMAs
   if (!mbar_wait_bounded(&bars[3], 0, abort_flag, sbw, kDetailGradTc)) mbar_wait_drain(&bars[3], 0);
   tc::fence_after_sync();
   if (dinit && !bad) {
-    float sv[32];
+    float sv[32], s2v[32];
     const int i0 = 32 * blk;
     tmem_ld32_wait(tbase + lrow + FT_S + i0, sv);
+    tmem_ld32_wait(tbase + lrow + FT_SH + i0, s2v);
 #pragma unroll
-    for (int ii = 0; ii < 32; ++ii) dinit[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii];
+    for (int ii = 0; ii < 32; ++ii) dinit[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii] + s2v[ii];
   }
   tc::fence_before_sync();
   __syncthreads();
