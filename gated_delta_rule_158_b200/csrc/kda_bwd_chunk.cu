@@ -13,8 +13,8 @@
 //   X = (I + Diag(beta) L)^-1,  T = X Diag(beta)
 //   Qg = q e^Gamma,  Ka = k e^Gamma,  Kc = k e^{Gamma_C - Gamma}
 //   U = T (V - Ka S),  S_next = Diag(e^{Gamma_C}) S + Kc^T U,  O = scale (Qg S + A_qk U)
-// Four passes in three launches (F and A share one; plus a plan kernel for
-// packed batches), fp32 accuracy:
+// Four passes (plus a plan kernel for packed batches), fp32 accuracy; F and
+// A share one launch except at dk = dv = 128, where each runs on tcgen05:
 //   K  every chunk at once, one CTA per (chunk, head): the key-side matrices
 //      X, A_qk, L.
 //   F  chunk order, one 512-thread CTA per unit: the chunk-start states and
@@ -31,11 +31,12 @@
 //      then through T, X, L and A_qk (their entries' gradients back onto q, k
 //      and Gamma through E) and the decays, and a reverse cumulative sum of
 //      dGamma gives dg.
-// K's Gram products, at dk = dv = 128 the products of F and A, and B's
-// backward through the Gram matrices run on the tensor cores as mma.sync
-// m16n8k8 (tf32 with each operand split into two tf32 parts); B's dv-block
-// products at dk = 128 as tcgen05 kind::tf32 with the same split; the others
-// are register-tiled CUDA-core loops.  Every output
+// K's Gram products, the products of F and A at head sizes other than
+// dk = dv = 128, and B's backward through the Gram matrices run on the
+// tensor cores as mma.sync m16n8k8 (tf32 with each operand split into two
+// tf32 parts); at dk = dv = 128 F and A, and at dk = 128 B's dv-block
+// products, run as tcgen05 kind::tf32 with the same split ("pass F / A on
+// tcgen05" below, BSmem); the others are register-tiled CUDA-core loops.  Every output
 // element has one writer and every sum a fixed order: results are
 // deterministic.
 // Tail chunks are padded with g = 0, beta = 0, k = q = v = dO = 0.  Dense
