@@ -350,6 +350,13 @@ KDA_API kda_status kda_decode_replay(const void *k, const void *v, const float *
  * checkpoint the window start states, once per window from its checkpoint);
  * every per-chunk step is the same arithmetic as in a single pass, with the
  * fp32 state and state gradient handed across windows unrounded.
+ * Tensor cores: at dk = dv = 128 the two state scans, and at dk = 128 the
+ * token-gradient pass, run their products as tcgen05 MMAs (tf32 operands
+ * split into high and low parts, fp32 accumulators in TMEM: fp32 accuracy);
+ * each scan CTA holds all 512 TMEM columns of its SM, so a kernel of another
+ * stream that holds TMEM delays it.  Their waits on the MMAs are bounded: one
+ * that runs out records KDA_ERR_TIMEOUT (detail 0xB410 the token-gradient
+ * pass, 0xB420 the forward scan, 0xB421 the state-gradient scan).
  * Supported: dk, dv in {32, 64, 128}, B * T * H < 2^31.
  */
 KDA_API size_t kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv,
