@@ -2872,6 +2872,326 @@ __global__ void __launch_bounds__(NTF, 1)
   }
 }
 
+// The fp32-accuracy forward scan at dk = dv = 128 on tcgen05: pass F's TMEM
+// scheme with the output folded into its groups (a tcgen05.mma costs the
+// same whatever N):
+//   [D_O | D_R] = S^T [Q_gamma; Ka]^T          (N 64, K 128 = i)
+//   D_U = R^T T^T                              (N 32, K 32 = r')
+//   [S^T | D_O] += U^T [Kc^T; A_qk]^T          (N 160, K 32 = r), S^T decayed first
+// so D_O = (Q_gamma S + A_qk U)^T of the chunk, read (and stored as o, scaled)
+// once the update has landed, at the start of the next chunk.  TMEM columns:
+// S^T 0..127, D_O 128..159, D_R / R_hi 160..191, R_lo then U_lo 192..223,
+// D_U / U_hi 224..255, S^T's parts 256..511.  The R group is issued by two
+// warps, the second into columns 192..255 (free then), added when R is read.
+constexpr uint32_t OT_S = 0, OT_O = 128, OT_RD = 160, OT_RL = 192, OT_UD = 224, OT_SH = 256,
+                   OT_SL = 384;
+constexpr int32_t kDetailFwdF32Tc = 0xB422;  // timeout detail: the fp32 forward's MMA barriers
+
+struct OtcSmem {
+  static constexpr int LK = 128 + 4;
+  static constexpr int kS = 0, GS = kS + C * LK, qS = GS + C * LK, VS = qS + C * LK;
+  static constexpr int RQH = VS + C * 128, RQL = RQH + 2 * C * 128;    // [Q_gamma; Ka] [r][i]
+  static constexpr int TH = RQL + 2 * C * 128, TL = TH + C * C;        // T [r][r']
+  static constexpr int SBH = TL + C * C, SBL = SBH + (128 + C) * C;    // [Kc^T; A_qk] [n][r]
+  static constexpr int bS = SBL + (128 + C) * C, gC = bS + C, eC = gC + 128;
+  static constexpr int bar_off = eC + 128;  // 4 mbarriers, TMEM address, abort flag
+  static constexpr int floats = bar_off + 16;
+  static constexpr size_t bytes = sizeof(float) * floats;
+  static_assert(RQH % 32 == 0 && TH % 32 == 0 && SBH % 32 == 0, "128-byte aligned operand tiles");
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(NTF, 1)
+    fwd_f32_scan_tc(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                    const Tin* __restrict__ v, const float* __restrict__ g,
+                    const float* __restrict__ A_log, float g_min, const float* __restrict__ beta,
+                    const float* __restrict__ init, float* __restrict__ fin,
+                    Tin* __restrict__ out, float scale, SeqMap map, float* __restrict__ ws) {
+  constexpr int DK = 128, DV = 128, LK = OtcSmem::LK;
+  extern __shared__ __align__(1024) float sm[];
+  float* kS = sm + OtcSmem::kS;
+  float* GS = sm + OtcSmem::GS;
+  float* qS = sm + OtcSmem::qS;
+  float* VS = sm + OtcSmem::VS;
+  float* bS = sm + OtcSmem::bS;
+  float* gC = sm + OtcSmem::gC;
+  float* eC = sm + OtcSmem::eC;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OtcSmem::bar_off);  // R, U, S, drain
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  if (!seqs_ok(map)) return;
+  const int H = map.H;
+  const int unit = blockIdx.x;
+  const int h = unit % H;
+  const UnitPos up = unit_pos(map, unit / H, h);
+  if (!unit_in_bounds(map, up)) return;
+  const int nc = up.nc;
+  const UnitWs w = unit_ws_fwd(ws, up.chunk0, nc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  StatusBlock* sbw = const_cast<StatusBlock*>(map.sb);
+  const int j = 32 * (warp & 3) + lane, blk = warp >> 2;
+  const uint32_t lrow = (uint32_t)(32 * (warp & 3)) << 16;
+  const float a_h = A_log ? expf(A_log[h]) : 0.f;
+  if (nc == 0) {
+    if (fin)
+      for (int idx = tid; idx < DK * DV; idx += NTF)
+        fin[(size_t)unit * DK * DV + idx] = init ? init[(size_t)unit * DK * DV + idx] : 0.f;
+    return;
+  }
+  if (tid == 0) {  // arrivals: the issuing warps of each group (2, 1, 1) and of the drain (2)
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], (i == 0 || i == 3) ? 2 : 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, FT_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+  const uint32_t sbase = smem_u32(sm);
+  auto desc = [&](int tile, int K) { return tc::plain_desc(sbase + 4u * tile, 128, K * 8 * 4); };
+  const uint64_t dRQH = desc(OtcSmem::RQH, DK), dRQL = desc(OtcSmem::RQL, DK);
+  const uint64_t dTH = desc(OtcSmem::TH, C), dTL = desc(OtcSmem::TL, C);
+  const uint64_t dSBH = desc(OtcSmem::SBH, C), dSBL = desc(OtcSmem::SBL, C);
+  auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
+    uint32_t hi, lo;
+    split_tf32(x, hi, lo);
+    reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
+    reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
+  };
+  // o of chunk cc (rows 8 blk .. 8 blk + 7, column j) from D_O, once its
+  // update group has landed
+  auto store_o = [&](int cc) {
+    const int r0 = 8 * blk, n0 = min(C, up.len - cc * C);
+    const size_t rb0 = (size_t)(up.row0 + cc * C) * H + h;
+    float ov[8];
+    tmem_ld8_wait(tbase + lrow + OT_O + r0, ov);
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr)
+      if (r0 + rr < n0) Elem<Tin>::store(out + (rb0 + (size_t)(r0 + rr) * H) * DV + j, scale * ov[rr]);
+  };
+  constexpr uint32_t id64 = tc::idesc(tc::kFmtTF32, 128, 64, false, false, false);
+  constexpr uint32_t id32 = tc::idesc(tc::kFmtTF32, 128, 32, false, false, false);
+  constexpr uint32_t id160 = tc::idesc(tc::kFmtTF32, 128, 160, false, false, false);
+  bool bad = false;
+  for (int c = 0; c < nc; ++c) {
+    const int t0 = c * C, n = min(C, up.len - t0);
+    const size_t rowbase = (size_t)(up.row0 + t0) * H + h;
+    {  // the chunk's rows, four elements per load, the gate formed on load
+      constexpr int K4 = DK / 4, V4 = DV / 4;
+      constexpr int IK = C * K4 / NTF, IV = C * V4 / NTF;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 qv[IK], kv[IK], gv[IK], vv[IV];
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        qv[it] = kv[it] = gv[it] = z4;
+        if (r < n) {
+          const size_t off = (rowbase + (size_t)r * H) * DK + i;
+          qv[it] = ld4(q + off);
+          kv[it] = ld4(k + off);
+          gv[it] = ld4(g + off);
+          if (A_log) gv[it] = gate4(gv[it], a_h, g_min);
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        vv[it] = r < n ? ld4(v + (rowbase + (size_t)r * H) * DV + jj) : z4;
+      }
+      const float bv = tid < C && tid < n ? beta[rowbase + (size_t)tid * H] : 0.f;
+      if (c + 1 < nc) {  // the next chunk's inputs into L2 while this one runs
+        const int n1 = min(C, up.len - t0 - C);
+        const size_t rb1 = rowbase + (size_t)C * H;
+        prefetch_rows<NTF>(q + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(k + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(g + rb1 * DK, (size_t)H * DK, n1, DK);
+        prefetch_rows<NTF>(v + rb1 * DV, (size_t)H * DV, n1, DV);
+        prefetch_rows<NTF>(w.X + (size_t)(c + 1) * C * C, 0, 1, C * C);
+        prefetch_rows<NTF>(w.Aqk + (size_t)(c + 1) * C * C, 0, 1, C * C);
+      }
+#pragma unroll
+      for (int it = 0; it < IK; ++it) {
+        const int idx = tid + it * NTF, r = idx / K4, i = 4 * (idx % K4);
+        st4(qS + r * LK + i, qv[it]);
+        st4(kS + r * LK + i, kv[it]);
+        st4(GS + r * LK + i, gv[it]);
+      }
+#pragma unroll
+      for (int it = 0; it < IV; ++it) {
+        const int idx = tid + it * NTF, r = idx / V4, jj = 4 * (idx % V4);
+        st4(VS + r * DV + jj, vv[it]);
+      }
+      if (tid < C) bS[tid] = bv;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += NTF) {  // Gamma = inclusive cumsum over the chunk
+      float acc = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < C; ++r) {
+        acc += GS[r * LK + i];
+        GS[r * LK + i] = acc;
+      }
+      gC[i] = acc;
+      eC[i] = expf(acc);
+    }
+    __syncthreads();
+    // [Q_gamma; Ka] and T (their last readers, the previous chunk's R and U
+    // groups, have completed)
+#pragma unroll 4
+    for (int t = 0; t < 16; ++t) {  // [Q_gamma; Ka]: 8 row groups x 32 k groups
+      const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
+      const int row = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3), r = row & 31;
+      const float e = expf(GS[r * LK + i]);
+      put_hl(OtcSmem::RQH, OtcSmem::RQL, kmaj<DK>(row, i), (row < C ? qS : kS)[r * LK + i] * e);
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // T [r][r']: 4 x 8 core matrices
+      const int cm = warp + 16 * t, rg = cm >> 3, kg = cm & 7;
+      const int r = 8 * rg + (lane >> 2), s2 = 4 * kg + (lane & 3);
+      put_hl(OtcSmem::TH, OtcSmem::TL, kmaj<C>(r, s2), w.X[((size_t)c * C + r) * C + s2] * bS[s2]);
+    }
+    // ---- the previous chunk's update has landed: its o, then [Kc^T; A_qk], S
+    if (c > 0) {
+      bad |= !mbar_wait_bounded(&bars[2], (c - 1) & 1, abort_flag, sbw, kDetailFwdF32Tc);
+      tc::fence_after_sync();
+      store_o(c - 1);
+    }
+#pragma unroll
+    for (int t = 0; t < 10; ++t) {  // [Kc^T; A_qk] [n][r]: 20 x 8 core matrices
+      const int cm = warp + 16 * t, ng = cm >> 3, rg2 = cm & 7;
+      const int nn = 8 * ng + (lane >> 2), r = 4 * rg2 + (lane & 3);
+      const float x = nn < DK ? kS[r * LK + nn] * expf(gC[nn] - GS[r * LK + nn])
+                              : w.Aqk[((size_t)c * C + (nn - DK)) * C + r];
+      put_hl(OtcSmem::SBH, OtcSmem::SBL, kmaj<C>(nn, r), x);
+    }
+    {  // S^T columns 32 blk .. of lane j: tf32 parts to TMEM, then decayed
+      float sv[32];
+      const int i0 = 32 * blk;
+      if (c == 0) {
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii)
+          sv[ii] = init ? init[((size_t)unit * DK + i0 + ii) * DV + j] : 0.f;
+      } else {
+        tmem_ld32_wait(tbase + lrow + OT_S + i0, sv);
+      }
+      uint32_t hv[32], lv[32];
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) split_tf32(sv[ii], hv[ii], lv[ii]);
+      tmem_st32u(tbase + lrow + OT_SH + i0, hv);
+      tmem_st32u(tbase + lrow + OT_SL + i0, lv);
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) sv[ii] *= eC[i0 + ii];
+      tc::tmem_st32(tbase + lrow + OT_S + i0, sv);
+      tc::wait_st();
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (lane == 0 && warp < 2) {  // [D_O | D_R]: even k-steps by warp 0 (columns 128..191),
+      // odd ones by warp 1 (192..255)
+      tc::fence_after_sync();
+      const uint32_t dst = tbase + (warp ? OT_RL : OT_O);
+#pragma unroll 1
+      for (int ks = warp; ks < DK / 8; ks += 2)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(dst, tbase + (term == 0 ? OT_SL : OT_SH) + 8 * ks,
+                          (term == 1 ? dRQL : dRQH) + (uint64_t)(16 * ks), id64,
+                          (ks > 1 || term > 0) ? 1u : 0u);
+      tc::mma_commit(&bars[0]);
+    }
+    bad |= !mbar_wait_bounded(&bars[0], c & 1, abort_flag, sbw, kDetailFwdF32Tc);
+    tc::fence_after_sync();
+    {  // the two halves summed: D_O back to 128.., R = V - D_R to the R columns
+      const int r0 = 8 * blk;
+      float o1[8], r1[8], o2[8], r2[8];
+      tmem_ld8_wait(tbase + lrow + OT_O + r0, o1);
+      tmem_ld8_wait(tbase + lrow + OT_RD + r0, r1);
+      tmem_ld8_wait(tbase + lrow + OT_RL + r0, o2);
+      tmem_ld8_wait(tbase + lrow + OT_UD + r0, r2);
+      uint32_t ov[8], hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        ov[rr] = __float_as_uint(o1[rr] + o2[rr]);
+        const float x = VS[(r0 + rr) * DV + j] - (r1[rr] + r2[rr]);
+        split_tf32(x, hv[rr], lv[rr]);
+      }
+      tmem_st8(tbase + lrow + OT_O + r0, ov);
+      tmem_st8(tbase + lrow + OT_RD + r0, hv);
+      tmem_st8(tbase + lrow + OT_RL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // D_U = R^T T^T
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + OT_UD, tbase + (term == 0 ? OT_RL : OT_RD) + 8 * ks,
+                          (term == 1 ? dTL : dTH) + (uint64_t)(16 * ks), id32,
+                          (ks > 0 || term > 0) ? 1u : 0u);
+      tc::mma_commit(&bars[1]);
+    }
+    bad |= !mbar_wait_bounded(&bars[1], c & 1, abort_flag, sbw, kDetailFwdF32Tc);
+    tc::fence_after_sync();
+    {  // U split: the high part over D_U, the low one over R_lo (read by the U group, done)
+      const int r0 = 8 * blk;
+      float du[8];
+      tmem_ld8_wait(tbase + lrow + OT_UD + r0, du);
+      uint32_t hv[8], lv[8];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) split_tf32(du[rr], hv[rr], lv[rr]);
+      tmem_st8(tbase + lrow + OT_UD + r0, hv);
+      tmem_st8(tbase + lrow + OT_RL + r0, lv);
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    if (tid == 0) {  // [S^T | D_O] += U^T [Kc^T; A_qk]^T
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+          tc::mma_ts_tf32(tbase + OT_S, tbase + (term == 0 ? OT_RL : OT_UD) + 8 * ks,
+                          (term == 1 ? dSBL : dSBH) + (uint64_t)(16 * ks), id160, 1u);
+      tc::mma_commit(&bars[2]);
+    }
+  }
+  if (lane == 0 && warp < 2) tc::mma_commit(&bars[3]);  // every issuer's MMAs
+  if (!mbar_wait_bounded(&bars[3], 0, abort_flag, sbw, kDetailFwdF32Tc)) mbar_wait_drain(&bars[3], 0);
+  tc::fence_after_sync();
+  if (!bad) {
+    store_o(nc - 1);
+    if (fin) {  // the state after the last chunk
+      float sv[32];
+      const int i0 = 32 * blk;
+      tmem_ld32_wait(tbase + lrow + OT_S + i0, sv);
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) fin[((size_t)unit * DK + i0 + ii) * DV + j] = sv[ii];
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, FT_COLS);
+}
+
 // Tail of the fp32 forward's workspace (after the status word and the
 // varlen order): the packed batch's chunk offsets, then X, A_qk, L per chunk.
 struct FwdLayout {
@@ -2899,9 +3219,13 @@ cudaError_t fwd_f32_launch(const ChunkArgs& a, void* tail, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(bwd_keyside<Tin, DK, DV, true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)KSmem<DK>::bytes);
+  constexpr bool kTc = DK == 128 && DV == 128;  // the scan on tcgen05
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fwd_f32_scan<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)OSmem<DK, DV>::bytes);
+    e = kTc ? cudaFuncSetAttribute(fwd_f32_scan_tc<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)OtcSmem::bytes)
+            : cudaFuncSetAttribute(fwd_f32_scan<Tin, DK, DV>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)OSmem<DK, DV>::bytes);
   if (e != cudaSuccess) return e;
   const SeqMap map{a.map.cu_seqlens, a.map.cu_seqlens ? coff : nullptr, a.sb, a.map.T, a.map.H,
                    0, 0, (int64_t)a.map.B * a.map.T, lay.max_chunks * (int64_t)a.map.H};
@@ -2915,6 +3239,13 @@ cudaError_t fwd_f32_launch(const ChunkArgs& a, void* tail, cudaStream_t st) {
                                          static_cast<const Tin*>(a.k), a.g, A_log, a.g_min,
                                          a.beta, map, nseq, ws);
   if ((e = cudaGetLastError())) return e;
+  if (kTc) {
+    fwd_f32_scan_tc<Tin><<<(unsigned)a.num_units, NTF, OtcSmem::bytes, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+        a.g, A_log, a.g_min, a.beta, a.init_state, a.final_state, static_cast<Tin*>(a.out),
+        a.scale, map, ws);
+    return cudaGetLastError();
+  }
   fwd_f32_scan<Tin, DK, DV><<<(unsigned)a.num_units, NTF, OSmem<DK, DV>::bytes, st>>>(
       static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
       a.g, A_log, a.g_min, a.beta, a.init_state, a.final_state, static_cast<Tin*>(a.out),
