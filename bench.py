@@ -822,8 +822,8 @@ def prefill_roofline(m, peaks, wl):
             "traffic": (chunk_traffic(m["B"], m["H"], m["T"])
                         if not wl.get("varlen") and wl.get("dtype", "bf16") == "bf16" else None),
             "kernel": ("chunk_tc_kernel (kda_chunk_fwd_gated)" if wl.get("dtype", "bf16") == "bf16"
-                       else "bwd_keyside (key-side matrices of every chunk) + fwd_f32_scan "
-                            "(kda_chunk_fwd_gated, fp32 inputs)"),
+                       else "bwd_keyside (key-side matrices of every chunk) + fwd_f32_scan_tc "
+                            "(tcgen05 scan; kda_chunk_fwd_gated, fp32 inputs)"),
             "kernel_ms": round(m["chunk_ms"], 4), "algorithmic_bytes": m["alg_bytes"],
             "peak_source": peaks["src"],
             "tensor_frac": round(f32 / secs / (peaks["tc"] * 1e12), 4),
