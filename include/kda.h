@@ -140,10 +140,14 @@ KDA_API kda_status kda_gate_bwd(const float *z, const float *A_log, float g_min,
  *                 depend on it beyond rounding.  bf16 with dk = dv = 128 and
  *                 chunk 0 or 32 runs the tcgen05 tensor-core kernel; other
  *                 inputs with chunk 0 or 32 (fp32, or dk / dv below 128) run
- *                 the chunk form at fp32 accuracy on warp-level tensor-core
- *                 products with split tf32 operands (two kernels: the
- *                 key-side matrices of every chunk, then the state scan with
- *                 the outputs); chunk 16 or 64 runs an fp32 CUDA-core kernel.
+ *                 the chunk form at fp32 accuracy on tensor-core products
+ *                 with split tf32 operands (two kernels: the key-side
+ *                 matrices of every chunk, then the state scan with the
+ *                 outputs -- at dk = dv = 128 a tcgen05 scan whose CTA holds
+ *                 all 512 TMEM columns of its SM and whose bounded waits
+ *                 record KDA_ERR_TIMEOUT, detail 0xB422, if they run out;
+ *                 warp-level MMAs otherwise); chunk 16 or 64 runs an fp32
+ *                 CUDA-core kernel.
  *  out          : in_dtype [B, T, H, dv]; must not alias any input.
  *  final_state  : fp32 [N, H, dk, dv] or NULL.
  *  workspace    : device buffer of >= kda_chunk_fwd_workspace_size() bytes;
