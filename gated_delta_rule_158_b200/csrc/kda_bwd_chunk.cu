@@ -509,27 +509,31 @@ __global__ void __launch_bounds__(NTH, 2)
     }
   }
   __syncthreads();
-  // X = (I + Diag(beta) L)^-1 by forward substitution: lane cc of warp 0
-  // holds column cc in registers (x_s = 0 above the diagonal, x_cc = 1) and
-  // forms x_r = -beta_r sum_{s<r} L_rs x_s (L_rs read as broadcasts) while
-  // the other warps store A_qk and L
+  // X = (I + Diag(beta) L)^-1 in 16-row blocks (L strictly lower):
+  //   X11 = (I + D1 L11)^-1, X22 = (I + D2 L22)^-1, X21 = -X22 (D2 L21) X11.
+  // Lanes 0-15 / 16-31 of warp 0 each hold one column of X11 / X22 in
+  // registers (x_r = -beta_r sum_{s<r} L_rs x_s, 15 steps) while the other
+  // warps store A_qk and L; then every thread takes one element of the two
+  // 16 x 16 x 16 products.  The key-side tiles are dead: X and the product
+  // live where the factors were.
+  float* XS = FaS;             // [C][LDC]
+  float* YS = XS + C * LDC;    // [16][LDC]: D2 L21 X11
   if (tid < 32) {
-    const int cc = tid;
-    float x[C];
+    const int o = 16 * (tid >> 4), cc = tid & 15;
+    float x[16];
 #pragma unroll
-    for (int s2 = 0; s2 < C; ++s2) x[s2] = s2 == cc ? 1.f : 0.f;
-#pragma unroll
-    for (int r = 1; r < C; ++r) {
+    for (int r = 0; r < 16; ++r) {
       float a0 = 0.f, a1 = 0.f;
 #pragma unroll
       for (int s2 = 0; s2 < r; ++s2) {
-        if (s2 & 1) a1 = fmaf(LS[r * LDC + s2], x[s2], a1);
-        else a0 = fmaf(LS[r * LDC + s2], x[s2], a0);
+        const float l = LS[(o + r) * LDC + o + s2];
+        if (s2 & 1) a1 = fmaf(l, x[s2], a1);
+        else a0 = fmaf(l, x[s2], a0);
       }
-      if (r > cc) x[r] = -bS[r] * (a0 + a1);
+      x[r] = r < cc ? 0.f : r == cc ? 1.f : -bS[o + r] * (a0 + a1);
     }
 #pragma unroll
-    for (int r = 0; r < C; ++r) w.X[((size_t)c * C + r) * C + cc] = x[r];
+    for (int r = 0; r < 16; ++r) XS[(o + r) * LDC + o + cc] = x[r];
   } else {
     for (int idx = tid - 32; idx < C * C; idx += NTH - 32) {
       const int r = idx / C, s2 = idx % C;
@@ -537,6 +541,28 @@ __global__ void __launch_bounds__(NTH, 2)
       w.Aqk[o] = AqS[r * LDC + s2];
       w.L[o] = LS[r * LDC + s2];
     }
+  }
+  static_assert(NTH == 256, "one thread per element of a 16 x 16 block");
+  __syncthreads();
+  const int br = tid >> 4, bc = tid & 15;
+  {  // Y = D2 L21 X11
+    float y = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) y = fmaf(LS[(16 + br) * LDC + s2], XS[s2 * LDC + bc], y);
+    YS[br * LDC + bc] = bS[16 + br] * y;
+  }
+  __syncthreads();
+  {  // X21 = -X22 Y (X22 lower triangular), X12 = 0
+    float x21 = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) x21 = fmaf(XS[(16 + br) * LDC + 16 + s2], YS[s2 * LDC + bc], x21);
+    XS[(16 + br) * LDC + bc] = -x21;
+    XS[br * LDC + 16 + bc] = 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += NTH) {
+    const int r = idx / C, s2 = idx % C;
+    w.X[((size_t)c * C + r) * C + s2] = XS[r * LDC + s2];
   }
 }
 
