@@ -1817,8 +1817,10 @@ struct FtcSmem {
   static constexpr int LK = 128 + 4;  // k, Gamma rows (4 mod 32)
   static constexpr int kS = 0, GS = kS + C * LK, VS = GS + C * LK;
   static constexpr int KaH = VS + C * 128, KaL = KaH + C * 128;
-  static constexpr int KcH = KaL + C * 128, KcL = KcH + 128 * C;
-  static constexpr int TH = KcL + 128 * C, TL = TH + C * C;
+  // Kc^T twice (chunk parity): a chunk writes its own before the previous
+  // chunk's update group, which reads the other, has landed
+  static constexpr int KcH = KaL + C * 128, KcL = KcH + 128 * C, KC_BUF = 2 * 128 * C;
+  static constexpr int TH = KcL + 128 * C + KC_BUF, TL = TH + C * C;
   static constexpr int bS = TL + C * C, gC = bS + C, eC = gC + 128;
   static constexpr int bar_off = eC + 128;  // 4 mbarriers, TMEM address, abort flag
   static constexpr int floats = bar_off + 16;
@@ -1964,16 +1966,18 @@ __global__ void __launch_bounds__(NTF, 1)
       put_hl(FtcSmem::TH, FtcSmem::TL, kmaj<C>(r, s2),
              w.X[((size_t)c * C + r) * C + s2] * bS[s2]);
     }
-    // ---- the previous chunk's state update has landed: Kc^T, then S
-    if (c > 0) bad |= !mbar_wait_bounded(&bars[2], (c - 1) & 1, abort_flag, sbw, kDetailFwdTc);
-    tc::fence_after_sync();
+    // Kc^T ([i][r], K-major) into this chunk's buffer: 16 row groups x 8 k groups
+    const int kcb = (c & 1) * FtcSmem::KC_BUF;
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {  // Kc^T ([i][r], K-major): 16 row groups x 8 k groups
+    for (int t = 0; t < 8; ++t) {
       const int cm = warp + 16 * t, ig = cm >> 3, rg2 = cm & 7;
       const int i = 8 * ig + (lane >> 2), r = 4 * rg2 + (lane & 3);
-      put_hl(FtcSmem::KcH, FtcSmem::KcL, kmaj<C>(i, r),
+      put_hl(FtcSmem::KcH + kcb, FtcSmem::KcL + kcb, kmaj<C>(i, r),
              kS[r * LK + i] * expf(gC[i] - GS[r * LK + i]));
     }
+    // ---- the previous chunk's state update has landed: S
+    if (c > 0) bad |= !mbar_wait_bounded(&bars[2], (c - 1) & 1, abort_flag, sbw, kDetailFwdTc);
+    tc::fence_after_sync();
     {  // S^T columns 32 blk .. 32 blk + 31 of lane j: the chunk-start state to the
        // workspace, its tf32 parts to TMEM, then decayed by e^{Gamma_C}
       float sv[32];
@@ -2094,7 +2098,8 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
         for (int term = 0; term < 3; ++term)
           tc::mma_ts_tf32(tbase + (warp ? FT_SH : FT_S), tbase + (term == 0 ? FT_UL : FT_UD) + 8 * ks,
-                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks), id128,
+                          (term == 1 ? dKcL : dKcH) + (uint64_t)(16 * ks + (c & 1) * FtcSmem::KC_BUF / 4),
+                          id128,
                           (warp == 0 || ks > 1 || term > 0) ? 1u : 0u);
       tc::mma_commit(&bars[2]);
     }
