@@ -1101,15 +1101,6 @@ constexpr uint32_t TC_LBO = 128, TC_SBO = 512;
 constexpr uint32_t TC_COLS = 256;                    // TMEM: D1 0..63, D2 64..95, D3 128..191
 constexpr uint32_t TC_D1 = 0, TC_D2 = 64, TC_D3 = 128;
 constexpr int32_t kDetailBwdMma = 0xB410;            // timeout detail: B's MMA barriers
-// x = hi + lo for the tcgen05 operands: hi is x with the 13 low mantissa bits
-// cleared (a tf32 value), lo = x - hi exactly; lo keeps up to 13 significant
-// bits of which a tf32 MMA uses 10, so each product's error stays below 2^-21
-// of |a b| (two instructions instead of three for rounded parts)
-__device__ __forceinline__ void split_tf32_fast(float x, uint32_t& hi, uint32_t& lo) {
-  hi = __float_as_uint(x) & 0xFFFFE000u;
-  lo = __float_as_uint(x - __uint_as_float(hi));
-}
-
 // float offset of element (row, 4 q) of a stage tile
 __device__ __forceinline__ int tc_off(int row, int q) {
   return (row >> 3) * 128 + q * 32 + (row & 7) * 4;
@@ -1354,10 +1345,10 @@ __global__ void __launch_bounds__(NTH, 2)
       if (jb >= 2) bad |= !mbar_wait_bounded(&bars[b], ((jb - 2) >> 1) & 1, abort_flag, sbw, kDetailBwdMma);
       auto put_hl = [&](int hoff, int loff, float4 v) {
         uint4 hi, lo;
-        split_tf32_fast(v.x, hi.x, lo.x);
-        split_tf32_fast(v.y, hi.y, lo.y);
-        split_tf32_fast(v.z, hi.z, lo.z);
-        split_tf32_fast(v.w, hi.w, lo.w);
+        split_tf32(v.x, hi.x, lo.x);
+        split_tf32(v.y, hi.y, lo.y);
+        split_tf32(v.z, hi.z, lo.z);
+        split_tf32(v.w, hi.w, lo.w);
         *reinterpret_cast<uint4*>(st + hoff) = hi;
         *reinterpret_cast<uint4*>(st + loff) = lo;
       };
@@ -1896,7 +1887,7 @@ __global__ void __launch_bounds__(NTF, 1)
   const uint64_t dKcL = tc::plain_desc(sbase + 4u * FtcSmem::KcL, 128, C * 8 * 4);
   auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
     uint32_t hi, lo;
-    split_tf32_fast(x, hi, lo);
+    split_tf32(x, hi, lo);
     reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
     reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
   };
@@ -2006,7 +1997,7 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
       for (int ii = 0; ii < 32; ++ii) {
         w.S[((size_t)c * DK + i0 + ii) * DV + j] = sv[ii];
-        split_tf32_fast(sv[ii], hv[ii], lv[ii]);
+        split_tf32(sv[ii], hv[ii], lv[ii]);
       }
       tmem_st32u(tbase + lrow + FT_SH + i0, hv);
       tmem_st32u(tbase + lrow + FT_SL + i0, lv);
@@ -2051,7 +2042,7 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int rr = 0; rr < 8; ++rr) {
         const float x = VS[(r0 + rr) * DV + j] - ((dr[rr] + dr2[rr]) + (dr3[rr] + dr4[rr]));
         w.R[((size_t)c * C + r0 + rr) * DV + j] = x;
-        split_tf32_fast(x, hv[rr], lv[rr]);
+        split_tf32(x, hv[rr], lv[rr]);
       }
       tmem_st8(tbase + lrow + FT_RD + r0, hv);
       tmem_st8(tbase + lrow + FT_RL + r0, lv);
@@ -2087,7 +2078,7 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int rr = 0; rr < 8; ++rr) {
         du[rr] += du2[rr];
         w.U[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
-        split_tf32_fast(du[rr], hv[rr], lv[rr]);
+        split_tf32(du[rr], hv[rr], lv[rr]);
       }
       tmem_st8(tbase + lrow + FT_UD + r0, hv);
       tmem_st8(tbase + lrow + FT_UL + r0, lv);
@@ -2219,7 +2210,7 @@ __global__ void __launch_bounds__(NTF, 1)
   const uint64_t dOtH = desc(AtcSmem::OtH, C), dOtL = desc(AtcSmem::OtL, C);
   auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
     uint32_t hi, lo;
-    split_tf32_fast(x, hi, lo);
+    split_tf32(x, hi, lo);
     reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
     reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
   };
@@ -2338,7 +2329,7 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
       for (int ii = 0; ii < 32; ++ii) {
         w.dS[((size_t)c * DK + i0 + ii) * DV + j] = sv[ii];
-        split_tf32_fast(sv[ii], hv[ii], lv[ii]);
+        split_tf32(sv[ii], hv[ii], lv[ii]);
       }
       tmem_st32u(tbase + lrow + FT_SH + i0, hv);
       tmem_st32u(tbase + lrow + FT_SL + i0, lv);
@@ -2384,7 +2375,7 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int rr = 0; rr < 8; ++rr) {
         du[rr] = (du[rr] + d2[rr]) + (d3[rr] + d4[rr]);
         w.dU[((size_t)c * C + r0 + rr) * DV + j] = du[rr];
-        split_tf32_fast(du[rr], hv[rr], lv[rr]);
+        split_tf32(du[rr], hv[rr], lv[rr]);
       }
       tmem_st8(tbase + lrow + FT_RD + r0, hv);
       tmem_st8(tbase + lrow + FT_RL + r0, lv);
@@ -2422,7 +2413,7 @@ __global__ void __launch_bounds__(NTF, 1)
         wv[rr] += w2[rr];
         w.W[((size_t)c * C + r) * DV + j] = wv[rr];
         if (r < n) dv[(rowbase + (size_t)r * H) * DV + j] = wv[rr];
-        split_tf32_fast(wv[rr], hv[rr], lv[rr]);
+        split_tf32(wv[rr], hv[rr], lv[rr]);
       }
       tmem_st8(tbase + lrow + FT_UD + r0, hv);
       tmem_st8(tbase + lrow + FT_UL + r0, lv);
@@ -2999,7 +2990,7 @@ __global__ void __launch_bounds__(NTF, 1)
   const uint64_t dSBH = desc(OtcSmem::SBH, C), dSBL = desc(OtcSmem::SBL, C);
   auto put_hl = [&](int tile_h, int tile_l, int off, float x) {
     uint32_t hi, lo;
-    split_tf32_fast(x, hi, lo);
+    split_tf32(x, hi, lo);
     reinterpret_cast<uint32_t*>(sm + tile_h)[off] = hi;
     reinterpret_cast<uint32_t*>(sm + tile_l)[off] = lo;
   };
@@ -3121,7 +3112,7 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       uint32_t hv[32], lv[32];
 #pragma unroll
-      for (int ii = 0; ii < 32; ++ii) split_tf32_fast(sv[ii], hv[ii], lv[ii]);
+      for (int ii = 0; ii < 32; ++ii) split_tf32(sv[ii], hv[ii], lv[ii]);
       tmem_st32u(tbase + lrow + OT_SH + i0, hv);
       tmem_st32u(tbase + lrow + OT_SL + i0, lv);
 #pragma unroll
@@ -3162,7 +3153,7 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int rr = 0; rr < 8; ++rr) {
         ov[rr] = __float_as_uint(o1[rr] + o2[rr]);
         const float x = VS[(r0 + rr) * DV + j] - (r1[rr] + r2[rr]);
-        split_tf32_fast(x, hv[rr], lv[rr]);
+        split_tf32(x, hv[rr], lv[rr]);
       }
       tmem_st8(tbase + lrow + OT_O + r0, ov);
       tmem_st8(tbase + lrow + OT_RD + r0, hv);
@@ -3193,7 +3184,7 @@ __global__ void __launch_bounds__(NTF, 1)
       tmem_ld8_wait(tbase + lrow + OT_UD + r0, du);
       uint32_t hv[8], lv[8];
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) split_tf32_fast(du[rr], hv[rr], lv[rr]);
+      for (int rr = 0; rr < 8; ++rr) split_tf32(du[rr], hv[rr], lv[rr]);
       tmem_st8(tbase + lrow + OT_UD + r0, hv);
       tmem_st8(tbase + lrow + OT_RL + r0, lv);
       tc::wait_st();

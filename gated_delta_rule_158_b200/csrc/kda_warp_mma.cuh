@@ -12,12 +12,15 @@
 
 namespace kda {
 
-// tf32 with fp32 accuracy: x = hi + lo with hi = tf32(x), lo = tf32(x - hi),
-// and a b = a_lo b_hi + a_hi b_lo + a_hi b_hi (the dropped a_lo b_lo is
-// below fp32 rounding).
+// tf32 with fp32 accuracy: x = hi + lo with hi = x with its 13 low mantissa
+// bits cleared (a tf32 value) and lo = x - hi exactly, and
+// a b = a_lo b_hi + a_hi b_lo + a_hi b_hi.  A tf32 MMA uses 10 of lo's up to
+// 13 significant bits, and the dropped a_lo b_lo is as small, so each
+// product's error stays below ~2^-20 of |a b| (two instructions; the tf32
+// MMAs of tcgen05 and mma.sync take the same parts).
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
