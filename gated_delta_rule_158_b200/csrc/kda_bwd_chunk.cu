@@ -1779,6 +1779,10 @@ __global__ void __launch_bounds__(NTH, 2)
 // low parts back.  Ka, Kc^T and T are K-major shared tiles without swizzle.
 // TMEM columns: S^T 0..127, its parts 128..383, D_R / R_hi 384..415, R_lo
 // 416..447, D_U / U_hi 448..479, U_lo 480..511 (the whole TMEM: one CTA per SM).
+// A tcgen05.mma costs a fixed ~135-190 cycles on its issuing thread whatever
+// N, so each group is issued by several warps into accumulators of its own
+// in columns free at that point, summed when read: R by four (the R and U
+// columns), U by two (U_hi, U_lo), the update by two (S^T and S_hi).
 constexpr uint32_t FT_S = 0, FT_SH = 128, FT_SL = 256, FT_RD = 384, FT_RL = 416, FT_UD = 448,
                    FT_UL = 480, FT_COLS = 512;
 constexpr int32_t kDetailFwdTc = 0xB420;   // timeout detail: F's MMA barriers
