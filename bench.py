@@ -941,7 +941,7 @@ def bench_prefill_line(args, wl, world, rank, peaks):
             "ms_per_call": round(ms, 3),
             "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
                          "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
-                         "kernel": "bwd_keyside + bwd_scans (F and A) + bwd_chunk_grads "
+                         "kernel": "bwd_keyside + bwd_fwd_scan_tc + bwd_state_grad_scan_tc + bwd_chunk_grads "
                                    "(one kda_recurrent_bwd call)", "algorithmic_bytes": alg}}
     return line
 
@@ -994,10 +994,10 @@ def bench_backward_line(args, wl, world, rank, peaks):
                    "step": "kda_recurrent_bwd (bf16 q/k/v/dout, fp32 gradients)"},
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"],
                      "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4), "traffic": None,
-                     "kernel": "bwd_keyside + bwd_scans (F and A) + bwd_chunk_grads "
+                     "kernel": "bwd_keyside + bwd_fwd_scan_tc + bwd_state_grad_scan_tc + bwd_chunk_grads "
                                "(one kda_recurrent_bwd call)", "kernel_ms": round(ms, 3),
                      "algorithmic_bytes": alg},
-        "gpu_launches": 3 * args.steps, "clocks": clk,
+        "gpu_launches": 4 * args.steps, "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, secs = oracle_backward_sample(T=T, d=d)
