@@ -453,6 +453,23 @@ __global__ void __launch_bounds__(NTH, 2)
                        : unit_ws(ws, up.chunk0, up.nc, DK, DV);
   const int tid = threadIdx.x;
 
+  if (map.cu == nullptr) {  // dense batch: the rows of the CTA that likely takes this
+    // slot next (two CTAs per SM) into L2 while this one runs -- a hint only
+    uint32_t nsm;
+    asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+    const int64_t nb = (int64_t)blockIdx.x + 2 * (int64_t)nsm;
+    if (nb < (int64_t)gridDim.x) {
+      const int64_t cg = nb / H;
+      const int hh = (int)(nb % H), nc0 = (map.T + C - 1) / C;
+      const int64_t sq = cg / nc0;
+      const int cc = (int)(cg % nc0), n1 = min(C, map.T - cc * C);
+      const int64_t row0 = sq * (map.row_stride ? map.row_stride : (int64_t)map.T) + map.row_off;
+      const size_t rb = (size_t)(row0 + (int64_t)cc * C) * H + hh;
+      prefetch_rows<NTH>(q + rb * DK, (size_t)H * DK, n1, DK);
+      prefetch_rows<NTH>(k + rb * DK, (size_t)H * DK, n1, DK);
+      prefetch_rows<NTH>(g + rb * DK, (size_t)H * DK, n1, DK);
+    }
+  }
   load_keys<Tin, DK, LDK>(q, k, g, A_log, g_min, h, beta, rowbase, H, n, qS, kS, GS, bS);
   bool wide = false;  // some factor e^{+-(Gamma_r - Gamma_15)} would exceed e^80
   for (int i = tid; i < DK; i += NTH) {
