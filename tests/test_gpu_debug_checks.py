@@ -3,9 +3,10 @@
 Its device-side bounds checks record KDA_ERR_BOUNDS in the workspace status
 word instead of trapping; the selftest makes one check fail (without any
 memory access) and the context must stay usable.  On valid inputs the checks
-never fire: every path (dense, packed, segment split, fp32 CUDA-core kernel,
-backward including its windowed schedule) must report KDA_OK and give
-results bit-identical to the release library's.
+never fire: every path (dense, packed, segment split, the fp32-accuracy
+scans at d 64 and 128, backward at d 64 and 128 including its windowed
+schedule) must report KDA_OK and give results bit-identical to the release
+library's.
 """
 import pytest
 import torch
@@ -66,7 +67,7 @@ def _prefill(inp, cu=None, num_states=None):
     return out, fin, kda.kda_get_device_status(ws)
 
 
-@pytest.mark.parametrize("case", ["dense", "varlen", "split", "fp32"])
+@pytest.mark.parametrize("case", ["dense", "varlen", "split", "fp32", "fp32_128"])
 def test_debug_build_prefill_matches_release(case):
     cu = None
     if case == "dense":
@@ -81,8 +82,11 @@ def test_debug_build_prefill_matches_release(case):
     elif case == "split":  # B*H*2 < SMs and T >= 4096: the segment split
         inp = W.make_prefill_inputs(1, 9000, 2, 128, 128, torch.bfloat16, seed=63, device=DEV,
                                     init_state=True)
-    else:  # fp32 inputs: the CUDA-core kernel
+    elif case == "fp32":  # fp32 inputs, d 64: the warp-MMA scan
         inp = W.make_prefill_inputs(2, 130, 3, 64, 64, torch.float32, seed=64, device=DEV,
+                                    init_state=True)
+    else:  # fp32 inputs, d 128: the tcgen05 scan
+        inp = W.make_prefill_inputs(2, 130, 3, 128, 128, torch.float32, seed=65, device=DEV,
                                     init_state=True)
     o_r, f_r, st_r = _with(False, lambda: _prefill(inp, cu))
     o_d, f_d, st_d = _with(True, lambda: _prefill(inp, cu))
@@ -107,11 +111,13 @@ def _backward(inp, cot, g, cu=None, N=None):
     return grads, kda.kda_get_device_status(ws)
 
 
-@pytest.mark.parametrize("case", ["dense", "varlen", "windowed"])
+@pytest.mark.parametrize("case", ["dense", "dense128", "varlen", "windowed"])
 def test_debug_build_backward_matches_release(case):
     cu, N = None, None
     if case == "dense":
         B, T, H, d = 2, 150, 3, 64
+    elif case == "dense128":  # the tcgen05 scans and token-gradient products
+        B, T, H, d = 2, 150, 3, 128
     elif case == "windowed":  # longer than one 8192-token window
         B, T, H, d = 1, 9000, 1, 32
     else:
