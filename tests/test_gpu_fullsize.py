@@ -3,7 +3,8 @@ configuration bench.py times, on sampled (sequence, head) units that the
 fp64 oracle recomputes one by one (whole sequences: the recurrence has no
 shortcut), plus properties checked over every output.
 
-Workloads: dense prefill B=8 H=32 T=4096; varlen 64 log-uniform sequences,
+Workloads: dense prefill B=8 H=32 T=4096 (bf16, and fp32 inputs on the
+fp32-accuracy path); varlen 64 log-uniform sequences,
 H=16, nonzero initial states; decode 256 x 32 heads for 1024 steps; long
 prefill B=1 H=32 T=1048576 (segment split); speculative verify / replay
 256 x 32 heads with 4 draft tokens.  All dk = dv = 128, bf16 q/k/v, fp32
@@ -16,7 +17,8 @@ import torch
 import gated_delta_rule_158_b200 as kda
 from gated_delta_rule_158_b200 import workloads as W
 
-from kda_testutil import (TOL_BF16_O, TOL_BF16_S, gpu_gate, gpu_prefill, rel_l2, to64)
+from kda_testutil import (TOL_BF16_O, TOL_BF16_S, TOL_F32, gpu_gate, gpu_prefill, rel_l2,
+                          to64)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -90,6 +92,21 @@ def test_dense_prefill_full_size(oracle_mod):
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
     units = [(0, 0), (3, 17), (7, 31), (5, 9)]
     _check_units(o, S, _oracle_units(oracle_mod, inp, units), units)
+
+
+def test_prefill_fp32_full_size(oracle_mod):
+    """The fp32-accuracy path (key-side pass, then the tcgen05 scan) at the
+    prefill_fp32 workload's size, B=8 H=32 T=4096 with fp32 inputs and
+    initial states: sampled units against the oracle at the fp32 bar."""
+    inp = W.make_prefill_inputs(8, 4096, 32, 128, 128, torch.float32, seed=1, device=DEV,
+                                init_state=True)
+    o, S, _, ws = gpu_prefill(inp)
+    assert kda.kda_get_device_status(ws)[0] == kda.KDA_OK
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    units = [(0, 0), (2, 13), (7, 31)]
+    for (n, h), (o_ref, S_ref) in zip(units, _oracle_units(oracle_mod, inp, units)):
+        assert rel_l2(to64(o[n, :, h]), o_ref) <= TOL_F32, (n, h, rel_l2(to64(o[n, :, h]), o_ref))
+        assert rel_l2(to64(S[n, h]), S_ref) <= TOL_F32, (n, h)
 
 
 def test_varlen_prefill_full_size(oracle_mod):
