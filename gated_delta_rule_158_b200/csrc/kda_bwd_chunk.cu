@@ -1807,6 +1807,13 @@ constexpr int32_t kDetailGradTc = 0xB421;  // timeout detail: A's MMA barriers
 // float offset of element (row, k) of a K-major tile without swizzle whose
 // rows hold K elements: core matrices of 8 rows x 4 elements (128 bytes)
 // consecutive along K (LBO 128 bytes), 8-row groups K * 32 bytes apart (SBO)
+// e^x (x <= 0) for the scans' operand tiles: 2^(x log2 e) on the special-
+// function unit; the relative error stays near 1e-6 for the exponents that
+// matter (|x| up to ~20; beyond, the factor is below 1e-9 and underflows
+// towards 0 as the exact one does)
+__device__ __forceinline__ float exp_tile(float x) {
+  return tc::ex2_approx(x * 1.4426950408889634f);
+}
 template <int K>
 __device__ __forceinline__ int kmaj(int row, int k) {
   return (row >> 3) * (K * 8) + (k >> 2) * 32 + (row & 7) * 4 + (k & 3);
@@ -1978,7 +1985,7 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int t = 0; t < 8; ++t) {  // Ka: 4 row groups x 32 k groups
       const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
       const int r = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3);
-      put_hl(FtcSmem::KaH, FtcSmem::KaL, kmaj<DK>(r, i), kS[r * LK + i] * expf(GS[r * LK + i]));
+      put_hl(FtcSmem::KaH, FtcSmem::KaL, kmaj<DK>(r, i), kS[r * LK + i] * exp_tile(GS[r * LK + i]));
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {  // T: 4 row groups x 8 k groups
@@ -1994,7 +2001,7 @@ __global__ void __launch_bounds__(NTF, 1)
       const int cm = warp + 16 * t, ig = cm >> 3, rg2 = cm & 7;
       const int i = 8 * ig + (lane >> 2), r = 4 * rg2 + (lane & 3);
       put_hl(FtcSmem::KcH + kcb, FtcSmem::KcL + kcb, kmaj<C>(i, r),
-             kS[r * LK + i] * expf(gC[i] - GS[r * LK + i]));
+             kS[r * LK + i] * exp_tile(gC[i] - GS[r * LK + i]));
     }
     // ---- the previous chunk's state update has landed: S
     if (c > 0) bad |= !mbar_wait_bounded(&bars[2], (c - 1) & 1, abort_flag, sbw, kDetailFwdTc);
@@ -2315,7 +2322,7 @@ __global__ void __launch_bounds__(NTF, 1)
       const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
       const int r = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3);
       put_hl(AtcSmem::KcH, AtcSmem::KcL, kmaj<DK>(r, i),
-             kS[r * LK + i] * expf(gC[i] - GS[r * LK + i]));
+             kS[r * LK + i] * exp_tile(gC[i] - GS[r * LK + i]));
     }
     // ---- the later chunk's state-gradient update has landed: Qg^T, -Ka^T,
     // dO'^T, then dS
@@ -2325,7 +2332,7 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int t = 0; t < 8; ++t) {  // Qg^T, -Ka^T [i][r] and dO'^T [j][s]: 16 x 8 core matrices
       const int cm = warp + 16 * t, ig = cm >> 3, rg2 = cm & 7;
       const int i = 8 * ig + (lane >> 2), r = 4 * rg2 + (lane & 3);
-      const float e = expf(GS[r * LK + i]);
+      const float e = exp_tile(GS[r * LK + i]);
       const int o = kmaj<C>(i, r);
       put_hl(AtcSmem::QgH, AtcSmem::QgL, o, qS[r * LK + i] * e);
       put_hl(AtcSmem::KaH, AtcSmem::KaL, o, -(kS[r * LK + i] * e));
@@ -3098,7 +3105,7 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int t = 0; t < 16; ++t) {  // [Q_gamma; Ka]: 8 row groups x 32 k groups
       const int cm = warp + 16 * t, rg = cm >> 5, kg = cm & 31;
       const int row = 8 * rg + (lane >> 2), i = 4 * kg + (lane & 3), r = row & 31;
-      const float e = expf(GS[r * LK + i]);
+      const float e = exp_tile(GS[r * LK + i]);
       put_hl(OtcSmem::RQH, OtcSmem::RQL, kmaj<DK>(row, i), (row < C ? qS : kS)[r * LK + i] * e);
     }
 #pragma unroll
@@ -3117,7 +3124,7 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int t = 0; t < 10; ++t) {  // [Kc^T; A_qk] [n][r]: 20 x 8 core matrices
       const int cm = warp + 16 * t, ng = cm >> 3, rg2 = cm & 7;
       const int nn = 8 * ng + (lane >> 2), r = 4 * rg2 + (lane & 3);
-      const float x = nn < DK ? kS[r * LK + nn] * expf(gC[nn] - GS[r * LK + nn])
+      const float x = nn < DK ? kS[r * LK + nn] * exp_tile(gC[nn] - GS[r * LK + nn])
                               : w.Aqk[((size_t)c * C + (nn - DK)) * C + r];
       put_hl(OtcSmem::SBH, OtcSmem::SBL, kmaj<C>(nn, r), x);
     }
