@@ -1,6 +1,7 @@
 // kda_warp_mma.cuh -- warp-level tensor-core products in tf32
-// (mma.sync.m16n8k8), shared by the backward and the speculative-decoding
-// kernels.
+// (mma.sync.m16n8k8) and the tf32 high/low split that the backward's and
+// the fp32-accuracy forward's tensor-core products (warp-level and tcgen05)
+// take.
 //
 // Fragment layout (lane = 4 g + t, PTX ISA m16n8k8 .tf32): A (16 x 8, row
 // major) a0 = (g, t), a1 = (g + 8, t), a2 = (g, t + 4), a3 = (g + 8, t + 4);
@@ -21,12 +22,6 @@ namespace kda {
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
   hi = __float_as_uint(x) & 0xFFFFE000u;
   lo = __float_as_uint(x - __uint_as_float(hi));
-}
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
 }
 
 // d += a b
